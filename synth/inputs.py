@@ -1,0 +1,222 @@
+"""Seeded synthetic inputs shared by the oracle and the CUDA path.
+
+This module holds shapes, seeds and random draws only: it performs none of
+the model's arithmetic.  Every tensor is drawn from its own counter-seeded
+PCG64 stream, so any single layer can be generated on its own (the CPU
+oracle never has to materialise a full 28-layer model to check one layer).
+
+Shapes follow the DM0-base configuration on the DM0 architecture notes page
+(dregs-remover.com/news/27019, section 1): 28+28 Qwen3 layers, VLM hidden
+2048, action-expert hidden 1024, 16 query heads, 8 KV heads, head_dim 128,
+action dim 32, chunk 50.  Intermediate sizes (6144 / 3072), RoPE theta 1e6
+and the N(0, 0.02) weight / N(0, 1) embedding and noise distributions are the
+workload definitions this library is measured on.
+
+Matrices are returned as float32 arrays whose values are exactly
+representable in bfloat16 (round-to-nearest-even of an fp32 draw): the GPU
+stores them as bf16 and the oracle upcasts the same values, so both sides see
+identical parameters.  Norm gains and biases stay float32.
+"""
+from __future__ import annotations
+
+import dataclasses
+from dataclasses import dataclass
+
+import numpy as np
+
+# tensor order inside one decoder layer (also the blob order)
+LAYER_TENSORS = ("attn_norm", "Wq", "Wk", "Wv", "q_norm", "k_norm",
+                 "Wo", "mlp_norm", "Wg", "Wu", "Wd")
+HEAD_TENSORS = ("W_in", "b_in", "final_norm", "W_out", "b_out")
+BRANCH_VLM, BRANCH_ACTION = 0, 1
+
+
+@dataclass(frozen=True)
+class Dims:
+    layers: int
+    hidden_v: int
+    inter_v: int
+    hidden_a: int
+    inter_a: int
+    n_q: int
+    n_kv: int
+    head_dim: int
+    chunk: int = 50
+    action_dim: int = 32
+    rope_theta: float = 1.0e6
+    rms_eps: float = 1.0e-6
+
+    def hidden(self, branch: int) -> int:
+        return self.hidden_v if branch == BRANCH_VLM else self.hidden_a
+
+    def inter(self, branch: int) -> int:
+        return self.inter_v if branch == BRANCH_VLM else self.inter_a
+
+    def replace(self, **kw) -> "Dims":
+        return dataclasses.replace(self, **kw)
+
+
+# DM0-base shapes (28-layer Qwen3 VLM hidden 2048 + 28-layer Qwen3 action expert hidden 1024)
+DM0_BASE = Dims(layers=28, hidden_v=2048, inter_v=6144, hidden_a=1024, inter_a=3072,
+                n_q=16, n_kv=8, head_dim=128)
+# tiny merged-attention model: 2 layers, hidden 256/128, 4 q / 2 kv heads of 32
+TINY = Dims(layers=2, hidden_v=256, inter_v=512, hidden_a=128, inter_a=256,
+            n_q=4, n_kv=2, head_dim=32)
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    dims: Dims
+    batch: int
+    prefix: int          # P prefix tokens per sample
+    steps: int           # Euler steps K
+    random_kv: bool = False  # denoise over an injected random bf16 KV cache
+
+
+WORKLOADS = {
+    # 2 layers, P=64, S=50, 4 Euler steps, fp32-sized toy
+    "tiny": Workload("tiny", TINY, batch=1, prefix=64, steps=4),
+    # one full-width merged layer, P=816 (3 views x 256 image tokens + 48 text tokens)
+    "merged_layer": Workload("merged_layer", DM0_BASE.replace(layers=1), batch=1, prefix=816, steps=0),
+    # 28-layer action expert over a random bf16 prefix KV cache, 10 steps, batch 1
+    "denoise_b1": Workload("denoise_b1", DM0_BASE, batch=1, prefix=816, steps=10, random_kv=True),
+    # prefill (P=816) + 10-step denoise at batch 1
+    "e2e_b1": Workload("e2e_b1", DM0_BASE, batch=1, prefix=816, steps=10),
+    # batch 16, P=2048 each, 10 steps
+    "e2e_b16": Workload("e2e_b16", DM0_BASE, batch=16, prefix=2048, steps=10),
+}
+
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """fp32 -> nearest bf16 value (ties to even), returned as fp32."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    r = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) & np.uint32(0xFFFF0000)
+    return r.view(np.float32)
+
+
+def bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Upper 16 bits of fp32 values that are already bf16-representable."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    return (u >> np.uint32(16)).astype(np.uint16)
+
+
+def _normal(entropy: tuple, shape, scale: float = 1.0) -> np.ndarray:
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence(list(entropy))))
+    out = rng.standard_normal(size=shape, dtype=np.float32)
+    if scale != 1.0:
+        out *= np.float32(scale)
+    return out
+
+
+def layer_shapes(d: Dims, branch: int) -> dict:
+    H, I, D = d.hidden(branch), d.inter(branch), d.head_dim
+    return {
+        "attn_norm": (H,), "Wq": (d.n_q * D, H), "Wk": (d.n_kv * D, H), "Wv": (d.n_kv * D, H),
+        "q_norm": (D,), "k_norm": (D,), "Wo": (H, d.n_q * D), "mlp_norm": (H,),
+        "Wg": (I, H), "Wu": (I, H), "Wd": (H, I),
+    }
+
+
+def head_shapes(d: Dims) -> dict:
+    return {"W_in": (d.hidden_a, d.action_dim), "b_in": (d.hidden_a,),
+            "final_norm": (d.hidden_a,), "W_out": (d.action_dim, d.hidden_a),
+            "b_out": (d.action_dim,)}
+
+
+def _gain(entropy, shape, jitter):
+    if jitter == 0.0:
+        return np.ones(shape, dtype=np.float32)
+    return (1.0 + _normal(entropy, shape, jitter)).astype(np.float32)
+
+
+def layer_weights(d: Dims, branch: int, layer: int, seed: int = 0,
+                  std: float = 0.02, gain_jitter: float = 0.0) -> dict:
+    """Parameters of one decoder layer of one branch (VLM=0, action expert=1).
+
+    Matrices are [out][in] and bf16-representable; norm gains are 1, or
+    1 + gain_jitter * N(0,1) when gain_jitter > 0.
+    """
+    out = {}
+    for tid, (name, shape) in enumerate(layer_shapes(d, branch).items()):
+        ent = (seed, branch, layer, tid)
+        if name.endswith("norm"):
+            out[name] = _gain(ent, shape, gain_jitter)
+        else:
+            out[name] = round_bf16(_normal(ent, shape, std))
+    return out
+
+
+def head_weights(d: Dims, seed: int = 0, std: float = 0.02, gain_jitter: float = 0.0) -> dict:
+    """action_in_proj (W_in, b_in), final RMSNorm gain, action_out_proj (W_out, b_out)."""
+    out = {}
+    for tid, (name, shape) in enumerate(head_shapes(d).items()):
+        ent = (seed, 2, 0, tid)
+        if name == "final_norm":
+            out[name] = _gain(ent, shape, gain_jitter)
+        elif name.startswith("W"):
+            out[name] = round_bf16(_normal(ent, shape, std))
+        else:
+            out[name] = _normal(ent, shape, std)
+    return out
+
+
+class Weights:
+    """Lazily generated model parameters (per-layer access, cached on request)."""
+
+    def __init__(self, d: Dims, seed: int = 0, std: float = 0.02, gain_jitter: float = 0.0,
+                 cache: bool = True):
+        self.d, self.seed, self.std, self.gain_jitter = d, seed, std, gain_jitter
+        self._cache = {} if cache else None
+        self._head = None
+        self.overrides = {}   # (branch, layer, name) or ("head", name) -> array
+
+    def layer(self, branch: int, layer: int) -> dict:
+        key = (branch, layer)
+        if self._cache is not None and key in self._cache:
+            w = self._cache[key]
+        else:
+            w = layer_weights(self.d, branch, layer, self.seed, self.std, self.gain_jitter)
+            if self._cache is not None:
+                self._cache[key] = w
+        if any(k[:2] == key for k in self.overrides if len(k) == 3):
+            w = dict(w)
+            for k, v in self.overrides.items():
+                if len(k) == 3 and k[:2] == key:
+                    w[k[2]] = v
+        return w
+
+    def head(self) -> dict:
+        if self._head is None:
+            self._head = head_weights(self.d, self.seed, self.std, self.gain_jitter)
+        w = self._head
+        if any(k[0] == "head" for k in self.overrides):
+            w = dict(w)
+            for k, v in self.overrides.items():
+                if k[0] == "head":
+                    w[k[1]] = v
+        return w
+
+
+def prefix_embeddings(d: Dims, batch: int, prefix: int, seed: int = 1000) -> np.ndarray:
+    """[B][P][hidden_v] N(0,1) prefix embeddings, bf16-representable (sample b uses seed+b)."""
+    return np.stack([round_bf16(_normal((seed + b,), (prefix, d.hidden_v))) for b in range(batch)])
+
+
+def noise(d: Dims, batch: int, seed: int = 2000) -> np.ndarray:
+    """[B][chunk][action_dim] N(0,1) fp32 initial x_1 (sample b uses seed+b)."""
+    return np.stack([_normal((seed + b,), (d.chunk, d.action_dim)) for b in range(batch)])
+
+
+def random_kv_layer(d: Dims, batch: int, prefix: int, layer: int, seed: int = 3000):
+    """bf16-representable N(0,1) K and V of one layer: each [B][n_kv][P][head_dim]."""
+    k = np.stack([round_bf16(_normal((seed + b, layer, 0), (d.n_kv, prefix, d.head_dim)))
+                  for b in range(batch)])
+    v = np.stack([round_bf16(_normal((seed + b, layer, 1), (d.n_kv, prefix, d.head_dim)))
+                  for b in range(batch)])
+    return k, v
+
+
+def hidden_states(batch_tokens: int, hidden: int, seed: int, scale: float = 1.0) -> np.ndarray:
+    """fp32 N(0, scale^2) residual-stream inputs for single-layer checks."""
+    return _normal((seed, 7), (batch_tokens, hidden), scale)
