@@ -1,0 +1,202 @@
+/*
+ * dm0.h - C ABI of the DM0 dual-expert merged-attention inference path on
+ * NVIDIA B200 (sm_100a).
+ *
+ * What it computes (page title and section of the sources):
+ *   - DM0 architecture notes (dregs-remover.com/news/27019), section 1: in each
+ *     of L Qwen3-style layers a VLM branch (hidden Hv) and an action-expert
+ *     branch (hidden Ha) make their own Q/K/V with the same head count and
+ *     head_dim; the two sets are concatenated along the sequence axis, run
+ *     through one attention, split back, and each branch applies its own
+ *     O-projection, residual and SwiGLU MLP.  DM0-base: L = 28, Hv = 2048,
+ *     Ha = 1024, 16 query heads, 8 KV heads, head_dim 128, action dim 32,
+ *     chunk 50.
+ *   - "DM0.5: High-Performance Embodied VLA and OpenDM Open Source
+ *     Introduction", section 5.1 (the prefix runs once and its per-layer KV
+ *     cache is kept), 5.2 (action_in_proj -> action expert -> action_out_proj
+ *     gives the velocity v(x_t, t | c)), 5.3 (Euler integration from noise
+ *     x_1 with diffusion_steps = 10 returns the whole chunk), 6.5 (fixed
+ *     shapes and a graph captured once and replayed).
+ *
+ * Conventions shared by every entry point:
+ *   - Every call returns a dm0_status; no call throws or aborts.  After a
+ *     failure dm0_last_error() describes it.
+ *   - "device pointer" arguments are CUDA device addresses of the current
+ *     device, owned by the caller, and must stay valid until the work queued on
+ *     `stream` has finished.  `stream` is a cudaStream_t (NULL = legacy default
+ *     stream).  Device-pointer calls are asynchronous on `stream`.
+ *   - Layouts are dense row-major with the innermost index last.  bf16 is the
+ *     IEEE-754 bfloat16 bit pattern in a uint16_t.
+ *   - Kernels never trap.  A kernel that meets an internal timeout or a bad
+ *     index sets a device error word and returns early; the next call on the
+ *     context (or dm0_sync) reports DM0_EDEVICE and the context stays in
+ *     that state until dm0_clear_error().
+ *   - A context is bound to the CUDA device that was current at dm0_create and
+ *     is not thread-safe: calls on one context must be serialised by the caller.
+ */
+#ifndef DM0_H_
+#define DM0_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct dm0_ctx dm0_ctx;
+
+/* Model shapes and capacity.  Constraints checked by dm0_create:
+ *   head_dim in {32, 64, 128}; n_q % n_kv == 0;
+ *   hidden_v, hidden_a, n_q*head_dim, n_kv*head_dim multiples of 32 and
+ *   hidden_v, hidden_a, inter_v, inter_a, n_q*head_dim multiples of 128
+ *   (tensor-core tile rows), 2*inter multiples of 128;
+ *   action_dim <= 64; chunk >= 1; max_batch >= 1; max_prefix >= 1;
+ *   max_prefix + chunk <= 65536. */
+typedef struct {
+  int layers;       /* decoder layers per branch (28 for DM0-base) */
+  int hidden_v;     /* VLM hidden size (2048) */
+  int inter_v;      /* VLM SwiGLU intermediate size (6144) */
+  int hidden_a;     /* action-expert hidden size (1024) */
+  int inter_a;      /* action-expert SwiGLU intermediate size (3072) */
+  int n_q;          /* query heads (16) */
+  int n_kv;         /* key/value heads (8) */
+  int head_dim;     /* 128 */
+  int chunk;        /* action tokens per sample S (50) */
+  int action_dim;   /* A (32) */
+  int max_batch;    /* largest B any call will use */
+  int max_prefix;   /* largest P any call will use */
+  float rope_theta; /* 1e6 */
+  float rms_eps;    /* 1e-6 */
+} dm0_config;
+
+typedef enum {
+  DM0_OK = 0,
+  DM0_EINVAL = -1,   /* null pointer or malformed argument */
+  DM0_ESHAPE = -2,   /* B, P, steps or a size outside the context's capacity */
+  DM0_ENOMEM = -3,   /* device or host allocation failed */
+  DM0_ECUDA = -4,    /* a CUDA runtime/driver call failed */
+  DM0_EDEVICE = -5,  /* a kernel reported an internal timeout or bad index */
+  DM0_ESTATE = -6    /* call out of order (no weights, or no KV cache yet) */
+} dm0_status;
+
+/* Allocate a context on the current CUDA device: weight storage, the
+ * per-layer KV cache for max_batch x max_prefix, activation buffers and the
+ * RoPE table (built on the device).  *out receives the context.  Nothing is
+ * allocated afterwards except CUDA-graph instantiations (one per distinct
+ * (B, P, steps) of dm0_denoise). */
+dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out);
+
+/* Weight blob size in bytes for `cfg`. */
+size_t dm0_weights_bytes(const dm0_config* cfg);
+
+/* Copy weights from a HOST blob (caller keeps ownership) into the context,
+ * repacking for the kernels (Q/K/V rows fused, gate/up rows interleaved in
+ * 64-row blocks).  Synchronous.  Blob layout, all little-endian, no padding:
+ *   for branch in (VLM, action expert): for l in 0..layers-1:
+ *     attn_norm f32[H] | Wq bf16[n_q*D][H] | Wk bf16[n_kv*D][H] |
+ *     Wv bf16[n_kv*D][H] | q_norm f32[D] | k_norm f32[D] |
+ *     Wo bf16[H][n_q*D] | mlp_norm f32[H] | Wg bf16[I][H] | Wu bf16[I][H] |
+ *     Wd bf16[H][I]
+ *   then W_in bf16[Ha][A] | b_in f32[Ha] | final_norm f32[Ha] |
+ *        W_out bf16[A][Ha] | b_out f32[A]
+ * Matrices are [out][in].  `bytes` must equal dm0_weights_bytes(). */
+dm0_status dm0_load_weights(dm0_ctx* ctx, const void* blob, size_t bytes);
+
+/* Prefix pass (DM0.5 page, section 5.1): runs the VLM branch alone over the
+ * prefix and fills the context-owned KV cache.
+ *   prefix_emb: device bf16 [B][P][hidden_v] prefix embeddings.
+ * The cache holds, per layer, K after QK-norm and RoPE (positions 0..P-1) and
+ * V, as two planes of bf16 [layers][B][n_kv][P][head_dim] (see dm0_kv_view).
+ * Returns DM0_ESHAPE unless 1 <= B <= max_batch and 1 <= P <= max_prefix. */
+dm0_status dm0_prefill(dm0_ctx* ctx, const void* prefix_emb, int B, int P, void* stream);
+
+/* Device pointers of the KV-cache planes (context-owned, valid until
+ * dm0_destroy).  With the (B, P) of the last prefill or dm0_kv_commit, plane
+ * element [l][b][h][p][d] sits at index (((l*B + b)*n_kv + h)*P + p)*head_dim + d.
+ * Capacity: layers*max_batch*n_kv*max_prefix*head_dim elements per plane. */
+dm0_status dm0_kv_view(dm0_ctx* ctx, void** k_plane, void** v_plane);
+
+/* Declare that the caller wrote a KV cache of shape (B, P) through
+ * dm0_kv_view (for a denoise over an externally provided prefix cache). */
+dm0_status dm0_kv_commit(dm0_ctx* ctx, int B, int P);
+
+/* Flow-matching Euler sampler (DM0.5 page, sections 5.2-5.3) over the cached
+ * prefix of the last prefill / kv_commit: x = noise;
+ * for k in 0..steps-1: t = 1 - k/steps, x <- x - v(x, t)/steps.
+ *   noise:      device f32 [B][chunk][action_dim] (x_1), read once.
+ *   actions:    device f32 [B][chunk][action_dim] output x_0 (may alias noise).
+ *   velocities: device f32 [steps][B][chunk][action_dim] per-step v, or NULL.
+ * The step loop is captured once per (B, P, steps, velocities != NULL) as a
+ * CUDA graph and replayed; no host work happens inside the loop.
+ * Returns DM0_ESTATE without a cache, DM0_ESHAPE unless 1 <= steps <= 1000. */
+dm0_status dm0_denoise(dm0_ctx* ctx, const float* noise, int steps, float* actions, float* velocities,
+                       void* stream);
+
+/* Observation -> action chunk from HOST memory: copies prefix_emb (host bf16
+ * [B][P][hidden_v]) and noise (host f32 [B][chunk][action_dim]) to the device,
+ * runs dm0_prefill and dm0_denoise, copies the chunk back to `actions` (host
+ * f32) and waits for `stream`.  Host buffers should be pinned for full copy
+ * bandwidth; pageable memory works but is slower. */
+dm0_status dm0_infer_host(dm0_ctx* ctx, const void* prefix_emb, const float* noise, int B, int P, int steps,
+                          float* actions, void* stream);
+
+/* One dual-expert layer `layer` with both branches over the concatenated
+ * [prefix; suffix] sequence (DM0 architecture notes, section 1), for tests:
+ *   h_prefix  device f32 [B][P][hidden_v]   VLM residual stream in
+ *   h_suffix  device f32 [B][chunk][hidden_a] action residual stream in
+ *   out_prefix/out_suffix: device f32, same shapes, residual streams out
+ *   k_out/v_out: device bf16 [B][n_kv][P][head_dim], the prefix K (after
+ *   QK-norm + RoPE) and V of this layer.
+ * Prefix rows attend to prefix keys only; suffix rows to all P + chunk keys.
+ * Uses the context's buffers; overwrites the KV cache slot of `layer`. */
+dm0_status dm0_merged_layer(dm0_ctx* ctx, int layer, const float* h_prefix, const float* h_suffix, int B, int P,
+                            float* out_prefix, float* out_suffix, void* k_out, void* v_out, void* stream);
+
+/* Kernel-level entry points used by the unit tests. -------------------- */
+
+/* Tensor-core GEMM in fp32 accumulation:
+ *   swap == 0: C[M][N]  = A[M][K] * B[N][K]^T, C written.
+ *   swap == 1: C[N][M] += A[M][K] * B[N][K]^T transposed (A plays the weight
+ *              operand, B the token operand, N <= 128); C must be zeroed by
+ *              the caller; `splits` K-splits accumulate atomically.
+ * A, B device bf16 K-contiguous; C device f32.  M % 128 == 0 when swap == 1;
+ * K % 64 == 0 and K >= 64; splits >= 1 (only 1 when swap == 0). */
+dm0_status dm0_op_gemm(dm0_ctx* ctx, const void* A, const void* B, float* C, int M, int N, int K, int swap,
+                       int splits, void* stream);
+
+/* Merged GQA attention of one segment pair, for tests:
+ *   q:  device bf16 [B][Tq][n_q][head_dim]
+ *   ka/va: device bf16 [B][n_kv][Ta][head_dim]; kb/vb: [B][n_kv][Tb][head_dim]
+ *   (kb/vb may be NULL with Tb = 0)
+ *   o:  device bf16 [B][Tq][n_q][head_dim]
+ * Every query row sees all Ta + Tb keys; scale 1/sqrt(head_dim); query head h
+ * reads KV head h / (n_q / n_kv).  splits >= 1 splits the keys (64-key
+ * blocks) across CTAs and combines partial softmax states. */
+dm0_status dm0_op_attention(dm0_ctx* ctx, const void* q, const void* ka, const void* va, int Ta, const void* kb,
+                            const void* vb, int Tb, void* o, int B, int Tq, int splits, void* stream);
+
+/* Errors and lifetime. -------------------------------------------------- */
+
+/* Wait for `stream`, then report DM0_EDEVICE if a kernel raised the device
+ * error word, else DM0_OK (DM0_ECUDA if the wait itself failed). */
+dm0_status dm0_sync(dm0_ctx* ctx, void* stream);
+
+/* Device error word (0 when clean; bit 0..4: producer / MMA / epilogue
+ * timeout, bad index, drain timeout). */
+int dm0_device_error(const dm0_ctx* ctx);
+
+/* Clear the device error word and re-zero the split-K accumulators and
+ * counters so the context can be used again.  Synchronous. */
+dm0_status dm0_clear_error(dm0_ctx* ctx);
+
+/* Human-readable description of the last failure on `ctx` (never NULL). */
+const char* dm0_last_error(const dm0_ctx* ctx);
+
+/* Free everything the context owns.  NULL is ignored. */
+void dm0_destroy(dm0_ctx* ctx);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DM0_H_ */

@@ -101,12 +101,42 @@ def bf16_bits(x: np.ndarray) -> np.ndarray:
     return (u >> np.uint32(16)).astype(np.uint16)
 
 
-def _normal(entropy: tuple, shape, scale: float = 1.0) -> np.ndarray:
-    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence(list(entropy))))
-    out = rng.standard_normal(size=shape, dtype=np.float32)
+_CHUNK = 1 << 20
+_POOL = None
+
+
+def _pool():
+    global _POOL
+    if _POOL is None:
+        import concurrent.futures
+        import os
+        _POOL = concurrent.futures.ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1))
+    return _POOL
+
+
+def _fill(out: np.ndarray, entropy: tuple, c: int, scale: float, bf16: bool):
+    lo = c * _CHUNK
+    part = out[lo:lo + _CHUNK]
+    rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence(list(entropy) + [c])))
+    rng.standard_normal(size=part.shape, dtype=np.float32, out=part)
     if scale != 1.0:
-        out *= np.float32(scale)
-    return out
+        part *= np.float32(scale)
+    if bf16:
+        part[...] = round_bf16(part)
+
+
+def _normal(entropy: tuple, shape, scale: float = 1.0, bf16: bool = False) -> np.ndarray:
+    """N(0, scale^2) fp32 draw; element chunk c (2^20 elements) comes from its own
+    PCG64 stream seeded by (entropy..., c), so the result does not depend on
+    how many threads fill it.  bf16=True rounds every value to bf16 (RNE)."""
+    n = int(np.prod(shape))
+    out = np.empty(n, dtype=np.float32)
+    chunks = (n + _CHUNK - 1) // _CHUNK
+    if chunks <= 1:
+        _fill(out, entropy, 0, scale, bf16)
+    else:
+        list(_pool().map(lambda c: _fill(out, entropy, c, scale, bf16), range(chunks)))
+    return out.reshape(shape)
 
 
 def layer_shapes(d: Dims, branch: int) -> dict:
@@ -143,7 +173,7 @@ def layer_weights(d: Dims, branch: int, layer: int, seed: int = 0,
         if name.endswith("norm"):
             out[name] = _gain(ent, shape, gain_jitter)
         else:
-            out[name] = round_bf16(_normal(ent, shape, std))
+            out[name] = _normal(ent, shape, std, bf16=True)
     return out
 
 
@@ -155,7 +185,7 @@ def head_weights(d: Dims, seed: int = 0, std: float = 0.02, gain_jitter: float =
         if name == "final_norm":
             out[name] = _gain(ent, shape, gain_jitter)
         elif name.startswith("W"):
-            out[name] = round_bf16(_normal(ent, shape, std))
+            out[name] = _normal(ent, shape, std, bf16=True)
         else:
             out[name] = _normal(ent, shape, std)
     return out
@@ -200,7 +230,7 @@ class Weights:
 
 def prefix_embeddings(d: Dims, batch: int, prefix: int, seed: int = 1000) -> np.ndarray:
     """[B][P][hidden_v] N(0,1) prefix embeddings, bf16-representable (sample b uses seed+b)."""
-    return np.stack([round_bf16(_normal((seed + b,), (prefix, d.hidden_v))) for b in range(batch)])
+    return np.stack([_normal((seed + b,), (prefix, d.hidden_v), bf16=True) for b in range(batch)])
 
 
 def noise(d: Dims, batch: int, seed: int = 2000) -> np.ndarray:
@@ -210,9 +240,9 @@ def noise(d: Dims, batch: int, seed: int = 2000) -> np.ndarray:
 
 def random_kv_layer(d: Dims, batch: int, prefix: int, layer: int, seed: int = 3000):
     """bf16-representable N(0,1) K and V of one layer: each [B][n_kv][P][head_dim]."""
-    k = np.stack([round_bf16(_normal((seed + b, layer, 0), (d.n_kv, prefix, d.head_dim)))
+    k = np.stack([_normal((seed + b, layer, 0), (d.n_kv, prefix, d.head_dim), bf16=True)
                   for b in range(batch)])
-    v = np.stack([round_bf16(_normal((seed + b, layer, 1), (d.n_kv, prefix, d.head_dim)))
+    v = np.stack([_normal((seed + b, layer, 1), (d.n_kv, prefix, d.head_dim), bf16=True)
                   for b in range(batch)])
     return k, v
 

@@ -1,0 +1,85 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every symbol include/dm0.h declares, sizes its weight blob like the binding
+packs it, and rejects malformed configurations before touching a device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from synth import inputs as I
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _lib():
+    from vla_dual_expert_b200 import build
+    build.build()
+    from vla_dual_expert_b200 import _abi
+    return _abi, _abi.load_library()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "dm0.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(dm0_[a-z_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    abi, lib = _lib()
+    declared = _declared()
+    assert len(declared) >= 16
+    assert sorted(abi.EXPORTS) == declared
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_blob_size_matches_packer():
+    abi, lib = _lib()
+    d = I.TINY
+    cfg = abi.make_config(d, 1, 64)
+    w = I.Weights(d, seed=0)
+    blob = abi.pack_weights(w, d.layers)
+    assert blob.nbytes == lib.dm0_weights_bytes(ctypes.byref(cfg))
+
+
+def test_blob_layout_first_tensors():
+    abi, _ = _lib()
+    d = I.TINY
+    w = I.Weights(d, seed=3, gain_jitter=0.1)
+    blob = abi.pack_weights(w, d.layers)
+    l0 = w.layer(0, 0)
+    H = d.hidden_v
+    np.testing.assert_array_equal(blob[:4 * H].view(np.float32), l0["attn_norm"])
+    wq_bits = blob[4 * H:4 * H + 2 * l0["Wq"].size].view(np.uint16)
+    back = (wq_bits.astype(np.uint32) << 16).view(np.float32).reshape(l0["Wq"].shape)
+    np.testing.assert_array_equal(back, l0["Wq"])
+
+
+@pytest.mark.parametrize("field,value", [("head_dim", 96), ("n_kv", 3), ("hidden_v", 200), ("action_dim", 0),
+                                         ("max_batch", 0), ("inter_a", 100)])
+def test_create_rejects_bad_config_on_host(field, value):
+    abi, lib = _lib()
+    d = I.TINY
+    cfg = abi.make_config(d, 1, 64)
+    setattr(cfg, field, value)
+    h = ctypes.c_void_p()
+    st = lib.dm0_create(ctypes.byref(cfg), ctypes.byref(h))
+    assert st == -2 and not h.value
+
+
+def test_null_arguments_rejected():
+    _, lib = _lib()
+    assert lib.dm0_create(None, None) == -1
+    assert lib.dm0_sync(None, None) == -1
+    assert lib.dm0_last_error(None) == b"null context"
+    lib.dm0_destroy(None)
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    from vla_dual_expert_b200 import _abi
+    monkeypatch.setattr(_abi, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(_abi, "_lib", None)
+    with pytest.raises(ImportError):
+        _abi.load_library()

@@ -1,0 +1,136 @@
+"""DM0 dual-expert merged-attention inference on B200 (sm_100a).
+
+Python face of the C ABI in include/dm0.h.  `Engine` owns one dm0_ctx and
+takes torch CUDA tensors (or host numpy arrays for `infer_host`); it only
+passes their pointers, sizes and the current CUDA stream to the library.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+
+from ._abi import (EXPORTS, LIB_PATH, Dm0Config, Dm0Error, load_library, make_config,  # noqa: F401
+                   pack_weights)
+
+__all__ = ["Engine", "Dm0Error", "pack_weights", "load_library", "EXPORTS", "LIB_PATH"]
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else t.data_ptr()
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check_cuda(t, dtype, shape, name):
+    import torch
+    if not (isinstance(t, torch.Tensor) and t.is_cuda and t.dtype == dtype and t.is_contiguous()):
+        raise TypeError(f"{name} must be a contiguous CUDA {dtype} tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+class Engine:
+    """One dm0_ctx on the current CUDA device."""
+
+    def __init__(self, dims, max_batch: int, max_prefix: int):
+        self.lib = load_library()
+        self.dims = dims
+        self.cfg = make_config(dims, max_batch, max_prefix)
+        h = ctypes.c_void_p()
+        st = self.lib.dm0_create(ctypes.byref(self.cfg), ctypes.byref(h))
+        if st != 0 or not h.value:
+            raise Dm0Error(st, "dm0_create failed (configuration or device allocation)")
+        self.h = h
+
+    # ------------------------------------------------------------------ helpers
+    def _chk(self, st: int):
+        if st != 0:
+            raise Dm0Error(st, self.lib.dm0_last_error(self.h).decode())
+
+    def close(self):
+        if getattr(self, "h", None) is not None and self.h.value:
+            self.lib.dm0_destroy(self.h)
+            self.h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # ------------------------------------------------------------------ API
+    def weights_bytes(self) -> int:
+        return int(self.lib.dm0_weights_bytes(ctypes.byref(self.cfg)))
+
+    def load_weights(self, blob: np.ndarray):
+        blob = np.ascontiguousarray(blob, dtype=np.uint8)
+        self._chk(self.lib.dm0_load_weights(self.h, blob.ctypes.data_as(ctypes.c_void_p), blob.nbytes))
+
+    def load_from(self, provider):
+        self.load_weights(pack_weights(provider, self.dims.layers))
+
+    def prefill(self, prefix_emb, stream=None):
+        import torch
+        B, P = prefix_emb.shape[:2]
+        _check_cuda(prefix_emb, torch.bfloat16, (B, P, self.dims.hidden_v), "prefix_emb")
+        self._chk(self.lib.dm0_prefill(self.h, _ptr(prefix_emb), B, P, _stream(stream)))
+
+    def kv_view(self):
+        k, v = ctypes.c_void_p(), ctypes.c_void_p()
+        self._chk(self.lib.dm0_kv_view(self.h, ctypes.byref(k), ctypes.byref(v)))
+        return k.value, v.value
+
+    def kv_commit(self, B: int, P: int):
+        self._chk(self.lib.dm0_kv_commit(self.h, B, P))
+
+    def denoise(self, noise, steps: int, actions=None, velocities=None, stream=None):
+        import torch
+        _check_cuda(noise, torch.float32, noise.shape, "noise")
+        if actions is None:
+            actions = torch.empty_like(noise)
+        self._chk(self.lib.dm0_denoise(self.h, _ptr(noise), steps, _ptr(actions), _ptr(velocities),
+                                       _stream(stream)))
+        return actions
+
+    def infer_host(self, prefix_bits: np.ndarray, noise: np.ndarray, steps: int, actions: np.ndarray = None,
+                   stream=None) -> np.ndarray:
+        """prefix_bits: host uint16 bf16 bit patterns [B][P][Hv]; noise: host f32 [B][S][A]."""
+        B, P = prefix_bits.shape[:2]
+        if actions is None:
+            actions = np.empty_like(noise, dtype=np.float32)
+        self._chk(self.lib.dm0_infer_host(self.h, prefix_bits.ctypes.data_as(ctypes.c_void_p),
+                                          noise.ctypes.data_as(ctypes.c_void_p), B, P, steps,
+                                          actions.ctypes.data_as(ctypes.c_void_p), _stream(stream)))
+        return actions
+
+    def merged_layer(self, layer, h_prefix, h_suffix, out_prefix, out_suffix, k_out, v_out, stream=None):
+        B, P = h_prefix.shape[:2]
+        self._chk(self.lib.dm0_merged_layer(self.h, layer, _ptr(h_prefix), _ptr(h_suffix), B, P, _ptr(out_prefix),
+                                            _ptr(out_suffix), _ptr(k_out), _ptr(v_out), _stream(stream)))
+
+    def op_gemm(self, A, B, C, swap=0, splits=1, stream=None):
+        M, K = A.shape
+        N = B.shape[0]
+        self._chk(self.lib.dm0_op_gemm(self.h, _ptr(A), _ptr(B), _ptr(C), M, N, K, swap, splits, _stream(stream)))
+
+    def op_attention(self, q, ka, va, kb, vb, o, splits=1, stream=None):
+        B, Tq = q.shape[:2]
+        Ta = ka.shape[2]
+        Tb = 0 if kb is None else kb.shape[2]
+        self._chk(self.lib.dm0_op_attention(self.h, _ptr(q), _ptr(ka), _ptr(va), Ta, _ptr(kb), _ptr(vb), Tb,
+                                            _ptr(o), B, Tq, splits, _stream(stream)))
+
+    def sync(self, stream=None):
+        self._chk(self.lib.dm0_sync(self.h, _stream(stream)))
+
+    def device_error(self) -> int:
+        return int(self.lib.dm0_device_error(self.h))
+
+    def clear_error(self):
+        self._chk(self.lib.dm0_clear_error(self.h))

@@ -1,0 +1,124 @@
+"""ctypes binding of libdm0.so (include/dm0.h): argument marshalling only.
+
+Every function here forwards device pointers, sizes and a CUDA stream to the
+C ABI; all arithmetic of the path runs in the library's CUDA kernels.  If
+libdm0.so is missing or fails to load, importing the binding raises: there is
+no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libdm0.so")
+
+c_int, c_float, c_size_t, c_void_p = ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_void_p
+
+STATUS = {0: "DM0_OK", -1: "DM0_EINVAL", -2: "DM0_ESHAPE", -3: "DM0_ENOMEM", -4: "DM0_ECUDA",
+          -5: "DM0_EDEVICE", -6: "DM0_ESTATE"}
+
+# every symbol include/dm0.h declares
+EXPORTS = ("dm0_create", "dm0_weights_bytes", "dm0_load_weights", "dm0_prefill", "dm0_kv_view",
+           "dm0_kv_commit", "dm0_denoise", "dm0_infer_host", "dm0_merged_layer", "dm0_op_gemm",
+           "dm0_op_attention", "dm0_sync", "dm0_device_error", "dm0_clear_error", "dm0_last_error",
+           "dm0_destroy")
+
+
+class Dm0Config(ctypes.Structure):
+    _fields_ = [("layers", c_int), ("hidden_v", c_int), ("inter_v", c_int), ("hidden_a", c_int),
+                ("inter_a", c_int), ("n_q", c_int), ("n_kv", c_int), ("head_dim", c_int),
+                ("chunk", c_int), ("action_dim", c_int), ("max_batch", c_int), ("max_prefix", c_int),
+                ("rope_theta", c_float), ("rms_eps", c_float)]
+
+
+class Dm0Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{STATUS.get(status, status)}: {what}")
+        self.status = status
+
+
+_lib = None
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libdm0.so from the package directory (raises if it is absent)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run `python -m vla_dual_expert_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = c_void_p
+    sig = {
+        "dm0_create": (c_int, [ctypes.POINTER(Dm0Config), ctypes.POINTER(P)]),
+        "dm0_weights_bytes": (c_size_t, [ctypes.POINTER(Dm0Config)]),
+        "dm0_load_weights": (c_int, [P, P, c_size_t]),
+        "dm0_prefill": (c_int, [P, P, c_int, c_int, P]),
+        "dm0_kv_view": (c_int, [P, ctypes.POINTER(P), ctypes.POINTER(P)]),
+        "dm0_kv_commit": (c_int, [P, c_int, c_int]),
+        "dm0_denoise": (c_int, [P, P, c_int, P, P, P]),
+        "dm0_infer_host": (c_int, [P, P, P, c_int, c_int, c_int, P, P]),
+        "dm0_merged_layer": (c_int, [P, c_int, P, P, c_int, c_int, P, P, P, P, P]),
+        "dm0_op_gemm": (c_int, [P, P, P, P, c_int, c_int, c_int, c_int, c_int, P]),
+        "dm0_op_attention": (c_int, [P, P, P, P, c_int, P, P, c_int, P, c_int, c_int, c_int, P]),
+        "dm0_sync": (c_int, [P, P]),
+        "dm0_device_error": (c_int, [P]),
+        "dm0_clear_error": (c_int, [P]),
+        "dm0_last_error": (ctypes.c_char_p, [P]),
+        "dm0_destroy": (None, [P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def make_config(dims, max_batch: int, max_prefix: int) -> Dm0Config:
+    """dims: any object with the model-shape attributes (layers, hidden_v, ...)."""
+    return Dm0Config(dims.layers, dims.hidden_v, dims.inter_v, dims.hidden_a, dims.inter_a, dims.n_q,
+                     dims.n_kv, dims.head_dim, dims.chunk, dims.action_dim, max_batch, max_prefix,
+                     float(dims.rope_theta), float(dims.rms_eps))
+
+
+def _bf16_bits(a: np.ndarray) -> np.ndarray:
+    """fp32 -> bf16 bit patterns, round to nearest even."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
+    return ((u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)).astype(np.uint16)
+
+
+LAYER_ORDER = (("attn_norm", "f32"), ("Wq", "bf16"), ("Wk", "bf16"), ("Wv", "bf16"), ("q_norm", "f32"),
+               ("k_norm", "f32"), ("Wo", "bf16"), ("mlp_norm", "f32"), ("Wg", "bf16"), ("Wu", "bf16"),
+               ("Wd", "bf16"))
+HEAD_ORDER = (("W_in", "bf16"), ("b_in", "f32"), ("final_norm", "f32"), ("W_out", "bf16"), ("b_out", "f32"))
+
+
+def pack_weights(provider, layers: int) -> np.ndarray:
+    """Serialise parameters into the blob layout dm0_load_weights reads.
+
+    provider.layer(branch, l) -> dict and provider.head() -> dict of fp32 arrays
+    (matrices [out][in]); branch 0 = VLM, 1 = action expert.
+    """
+    def nbytes(arr, kind):
+        return arr.size * (2 if kind == "bf16" else 4)
+
+    tensors = []
+    for br in (0, 1):
+        for l in range(layers):
+            w = provider.layer(br, l)
+            tensors += [(w[n], k) for n, k in LAYER_ORDER]
+    h = provider.head()
+    tensors += [(h[n], k) for n, k in HEAD_ORDER]
+    total = sum(nbytes(a, k) for a, k in tensors)
+    out = np.empty(total, dtype=np.uint8)
+    off = 0
+    for a, k in tensors:
+        n = nbytes(a, k)
+        src = _bf16_bits(a) if k == "bf16" else np.ascontiguousarray(a, dtype=np.float32)
+        out[off:off + n] = src.reshape(-1).view(np.uint8)
+        off += n
+    return out

@@ -1,0 +1,838 @@
+// C ABI of the DM0 dual-expert merged-attention path (declared in dm0.h):
+// context and buffer ownership, weight repacking, TMA descriptors, and the
+// launch schedules of the prefix pass, the merged layer and the Euler loop.
+//
+// Schedule (DM0.5 page, sections 5.1-5.3 and 6.5):
+//   prefill  : rows_prep, then per VLM layer
+//              QKV GEMM (+QK-norm, RoPE, KV-cache write) -> attention
+//              -> O GEMM (+residual, next-norm operand) -> gate/up GEMM (+SwiGLU)
+//              -> down GEMM (+residual, next-norm operand)
+//   denoise  : step_kernel(input of step 0), then per step 28 action layers of
+//              the same five kernels (attention over [prefix cache; suffix])
+//              and step_kernel(velocity, Euler update, input of the next step).
+//              The whole loop is captured once per (B, P, steps) into a CUDA
+//              graph and replayed.
+// Every kernel is launched with programmatic stream serialization, so each
+// kernel's prologue (TMEM allocation, barrier set-up, weight-tile requests)
+// overlaps the previous kernel's tail.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <map>
+#include <string>
+#include <tuple>
+#include <vector>
+
+#include "dm0.h"
+#include "attention.cuh"
+#include "elementwise.cuh"
+#include "gemm.cuh"
+#include "ptx.cuh"
+
+using dm0::AttnArgs;
+using dm0::GemmArgs;
+using dm0::StepArgs;
+typedef __nv_bfloat16 bf16;
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+struct LayerW {
+  bf16 *wqkv, *wo, *wgu, *wd;
+  float *attn_norm, *q_norm, *k_norm, *mlp_norm;
+};
+
+struct TmapKey {
+  const void* p;
+  uint64_t rows, cols;
+  uint32_t box;
+  bool operator<(const TmapKey& o) const {
+    return std::tie(p, rows, cols, box) < std::tie(o.p, o.rows, o.cols, o.box);
+  }
+};
+
+constexpr int kGemmStages = 4;
+constexpr int kPartSlots = 1024;   // split-KV partial-state slots (x 128 rows)
+
+}  // namespace
+
+struct dm0_ctx {
+  dm0_config cfg{};
+  int device = 0;
+  int num_sms = 148;
+  bool use_pdl = true, use_graph = true;
+  std::string err;
+
+  void* wbuf = nullptr;
+  LayerW* lw[2] = {nullptr, nullptr};
+  std::vector<LayerW> lw_store[2];
+  bf16 *W_in = nullptr, *W_out = nullptr;
+  float *b_in = nullptr, *final_norm = nullptr, *b_out = nullptr;
+  bool weights_loaded = false;
+
+  bf16 *kplane = nullptr, *vplane = nullptr;
+  int kv_B = 0, kv_P = 0;
+
+  // VLM side, Mp = max_batch * max_prefix rows
+  float* h_v = nullptr;
+  bf16 *xn_v = nullptr, *q_v = nullptr, *o_v = nullptr, *act_v = nullptr;
+  float* ssq_v = nullptr;
+  // action side, Ms = max_batch * chunk rows
+  float* h_a = nullptr;
+  bf16 *xn_a = nullptr, *q_a = nullptr, *o_a = nullptr, *act_a = nullptr, *k_s = nullptr, *v_s = nullptr;
+  float *ssq_a = nullptr, *x = nullptr;
+  // split-K / split-KV scratch
+  float* acc = nullptr;
+  size_t acc_elems = 0;
+  int* gcount = nullptr;
+  int* acount = nullptr;
+  int acount_n = 0;
+  float* part_o = nullptr;
+  float2* part_ml = nullptr;
+  float2* rope = nullptr;
+  int* d_err = nullptr;
+  // dm0_infer_host staging
+  bf16* stage_prefix = nullptr;
+
+  cudaStream_t cap_stream = nullptr;
+  std::map<std::tuple<int, int, int>, cudaGraphExec_t> graphs;
+  std::map<TmapKey, CUtensorMap> tmaps;
+  std::vector<void*> allocs;
+};
+
+namespace {
+
+dm0_status fail(dm0_ctx* c, dm0_status st, const std::string& msg) {
+  if (c) c->err = msg;
+  return st;
+}
+
+#define CK(call)                                                                              \
+  do {                                                                                        \
+    cudaError_t e_ = (call);                                                                  \
+    if (e_ != cudaSuccess) return fail(c, DM0_ECUDA, std::string(#call) + ": " + cudaGetErrorString(e_)); \
+  } while (0)
+
+#define TRY(expr)                  \
+  do {                             \
+    dm0_status s_ = (expr);        \
+    if (s_ != DM0_OK) return s_;   \
+  } while (0)
+
+template <typename T>
+dm0_status dalloc(dm0_ctx* c, T** p, size_t elems) {
+  void* v = nullptr;
+  const size_t bytes = elems * sizeof(T) > 0 ? elems * sizeof(T) : 16;
+  cudaError_t e = cudaMalloc(&v, bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(c, DM0_ENOMEM, "cudaMalloc of " + std::to_string(bytes) + " bytes failed: " + cudaGetErrorString(e));
+  }
+  c->allocs.push_back(v);
+  *p = static_cast<T*>(v);
+  return DM0_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int qkv_rows(const dm0_config& g) { return (g.n_q + 2 * g.n_kv) * g.head_dim; }
+int hidden_of(const dm0_config& g, int br) { return br == 0 ? g.hidden_v : g.hidden_a; }
+int inter_of(const dm0_config& g, int br) { return br == 0 ? g.inter_v : g.inter_a; }
+
+dm0_status get_tmap(dm0_ctx* c, CUtensorMap* out, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box) {
+  const TmapKey key{ptr, rows, cols, box};
+  auto it = c->tmaps.find(key);
+  if (it != c->tmaps.end()) {
+    *out = it->second;
+    return DM0_OK;
+  }
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(c, DM0_ECUDA, "cuTensorMapEncodeTiled is unavailable");
+  if (reinterpret_cast<uintptr_t>(ptr) % 16 != 0 || cols % 64 != 0)
+    return fail(c, DM0_EINVAL, "TMA operand must be 16-byte aligned with a multiple of 64 columns");
+  CUtensorMap m;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t boxd[2] = {64, box};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, boxd, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(c, DM0_ECUDA, "cuTensorMapEncodeTiled failed (" + std::to_string(r) + ")");
+  c->tmaps[key] = m;
+  *out = m;
+  return DM0_OK;
+}
+
+template <typename... KArgs, typename... Args>
+dm0_status launch(dm0_ctx* c, cudaStream_t s, void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                  Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = c->use_pdl ? 1 : 0;
+  CK(cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...));
+  return DM0_OK;
+}
+
+// ---------------------------------------------------------------- GEMM dispatch
+dm0_status run_gemm(dm0_ctx* c, cudaStream_t s, const bf16* act, int tokens, int K, const bf16* W, int wrows,
+                    GemmArgs g, int force_swap = -1, int force_splits = 0) {
+  if (tokens <= 0) return DM0_OK;
+  if (K % 64 != 0 || wrows % 128 != 0)
+    return fail(c, DM0_ESHAPE, "GEMM needs K % 64 == 0 and weight rows % 128 == 0");
+  const bool swap = force_swap >= 0 ? force_swap != 0 : tokens <= 128;
+  const int KB = K / 64;
+  g.K = K;
+  g.tokens = tokens;
+  g.err = c->d_err;
+  g.counters = c->gcount;
+  CUtensorMap ta, tb;
+  if (swap) {
+    if (tokens > 128) return fail(c, DM0_ESHAPE, "swapped GEMM takes at most 128 tokens");
+    const int BN = tokens <= 64 ? 64 : 128;
+    const int tiles = wrows / 128;
+    if (tiles > 1024) return fail(c, DM0_ESHAPE, "too many feature tiles");
+    int splits = force_splits > 0 ? force_splits : (c->num_sms + tiles / 2) / tiles;
+    splits = splits < 1 ? 1 : (splits > KB ? KB : splits);
+    const int kbps = (KB + splits - 1) / splits;
+    splits = (KB + kbps - 1) / kbps;
+    g.M = wrows;
+    g.N = tokens;
+    g.swap = 1;
+    g.kb_per_split = kbps;
+    if (g.mode != dm0::kModeResid && g.mode != dm0::kModeStoreF32) {
+      if (static_cast<size_t>(tokens) * wrows > c->acc_elems) return fail(c, DM0_ESHAPE, "split-K scratch too small");
+      g.acc = c->acc;
+      g.ld_acc = wrows;
+    }
+    TRY(get_tmap(c, &ta, W, wrows, K, 128));
+    TRY(get_tmap(c, &tb, act, tokens, K, BN));
+    const dim3 grid(tiles, 1, splits);
+    if (BN == 64)
+      return launch(c, s, dm0::gemm_tc_kernel<64, kGemmStages>, grid, dim3(dm0::kGemmThreads),
+                    dm0::GemmSmem<64, kGemmStages>::kBytes, ta, tb, g);
+    return launch(c, s, dm0::gemm_tc_kernel<128, kGemmStages>, grid, dim3(dm0::kGemmThreads),
+                  dm0::GemmSmem<128, kGemmStages>::kBytes, ta, tb, g);
+  }
+  const int BN = (wrows % 256 == 0) ? 256 : 128;
+  g.M = tokens;
+  g.N = wrows;
+  g.swap = 0;
+  g.kb_per_split = KB;
+  TRY(get_tmap(c, &ta, act, tokens, K, 128));
+  TRY(get_tmap(c, &tb, W, wrows, K, BN));
+  const dim3 grid((tokens + 127) / 128, wrows / BN, 1);
+  if (BN == 256)
+    return launch(c, s, dm0::gemm_tc_kernel<256, kGemmStages>, grid, dim3(dm0::kGemmThreads),
+                  dm0::GemmSmem<256, kGemmStages>::kBytes, ta, tb, g);
+  return launch(c, s, dm0::gemm_tc_kernel<128, kGemmStages>, grid, dim3(dm0::kGemmThreads),
+                dm0::GemmSmem<128, kGemmStages>::kBytes, ta, tb, g);
+}
+
+// ---------------------------------------------------------------- attention dispatch
+dm0_status run_attn(dm0_ctx* c, cudaStream_t s, const bf16* q, int seq_q, const bf16* ka, const bf16* va, int len_a,
+                    const bf16* kb, const bf16* vb, int len_b, bf16* o, int B, int splits_req, int a_stable) {
+  const dm0_config& g = c->cfg;
+  const int G = g.n_q / g.n_kv;
+  const int tiles = (G * seq_q + 127) / 128;
+  const int groups = B * g.n_kv;
+  const int nblk = (len_a + len_b + 63) / 64;
+  if (nblk == 0 || seq_q == 0) return DM0_OK;
+  int splits = splits_req;
+  if (splits <= 0) {
+    const int ctas = groups * tiles;
+    splits = ctas >= c->num_sms ? 1 : (2 * c->num_sms + ctas - 1) / ctas;
+  }
+  if (splits > nblk) splits = nblk;
+  while (splits > 1 && groups * tiles * splits > kPartSlots) --splits;
+  const int bps = (nblk + splits - 1) / splits;
+  splits = (nblk + bps - 1) / bps;
+  if (splits > 1 && groups * tiles > c->acount_n) return fail(c, DM0_ESHAPE, "attention split counters too small");
+  AttnArgs a{};
+  a.q = q;
+  a.seq_q = seq_q;
+  a.ka = ka;
+  a.va = va;
+  a.len_a = len_a;
+  a.kb = kb;
+  a.vb = vb;
+  a.len_b = len_b;
+  a.o = o;
+  a.n_q = g.n_q;
+  a.n_kv = g.n_kv;
+  a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(g.head_dim)));
+  a.blocks_per_split = bps;
+  a.a_stable = a_stable;
+  a.part_o = c->part_o;
+  a.part_ml = c->part_ml;
+  a.counters = c->acount;
+  a.err = c->d_err;
+  const dim3 grid(tiles, groups, splits);
+  switch (g.head_dim) {
+    case 128:
+      return launch(c, s, dm0::attn_kernel<128>, grid, dim3(dm0::kAttnThreads), dm0::AttnSmem<128>::kBytes, a);
+    case 64:
+      return launch(c, s, dm0::attn_kernel<64>, grid, dim3(dm0::kAttnThreads), dm0::AttnSmem<64>::kBytes, a);
+    default:
+      return launch(c, s, dm0::attn_kernel<32>, grid, dim3(dm0::kAttnThreads), dm0::AttnSmem<32>::kBytes, a);
+  }
+}
+
+dm0_status rows_prep(dm0_ctx* c, cudaStream_t s, const void* in, int in_bf16, float* h, bf16* xn, const float* gain,
+                     float* ssq, int n_slots, int M, int H) {
+  return launch(c, s, dm0::rows_prep_kernel, dim3((M + 7) / 8), dim3(256), 0, in, in_bf16, h, xn, gain, ssq,
+                n_slots, M, M, H);
+}
+
+GemmArgs base_args(dm0_ctx* c) {
+  GemmArgs g{};
+  const dm0_config& cf = c->cfg;
+  g.eps = cf.rms_eps;
+  g.n_q = cf.n_q;
+  g.n_kv = cf.n_kv;
+  g.head_dim = cf.head_dim;
+  g.rope = c->rope;
+  return g;
+}
+
+// QKV projection of one branch with QK-norm + RoPE; K/V to [B][n_kv][kv_seq][D]
+dm0_status layer_qkv(dm0_ctx* c, cudaStream_t s, int br, int l, const bf16* xn, const float* ssq_in, int tokens,
+                     int seq, int pos_offset, bf16* q_out, bf16* k_out, bf16* v_out) {
+  const LayerW& w = c->lw[br][l];
+  const int H = hidden_of(c->cfg, br);
+  GemmArgs g = base_args(c);
+  g.mode = dm0::kModeQKV;
+  g.ssq_in = ssq_in;
+  g.inv_hidden = 1.0f / H;
+  g.q_out = q_out;
+  g.k_out = k_out;
+  g.v_out = v_out;
+  g.q_gain = w.q_norm;
+  g.k_gain = w.k_norm;
+  g.seq_len = seq;
+  g.pos_offset = pos_offset;
+  g.kv_seq = seq;
+  return run_gemm(c, s, xn, tokens, H, w.wqkv, qkv_rows(c->cfg), g);
+}
+
+// O-proj (+residual) -> gate/up (+SwiGLU) -> down (+residual) of one branch
+dm0_status layer_rest(dm0_ctx* c, cudaStream_t s, int br, int l, int tokens, float* h, bf16* xn, const bf16* o,
+                      bf16* act, float* ssq_mlp, const float* next_gain, float* next_ssq) {
+  const dm0_config& cf = c->cfg;
+  const LayerW& w = c->lw[br][l];
+  const int H = hidden_of(cf, br), I = inter_of(cf, br);
+  GemmArgs g = base_args(c);
+  g.mode = dm0::kModeResid;
+  g.h = h;
+  g.H = H;
+  g.xn = xn;
+  g.gain_next = w.mlp_norm;
+  g.ssq_out = ssq_mlp;
+  TRY(run_gemm(c, s, o, tokens, cf.n_q * cf.head_dim, w.wo, H, g));
+  GemmArgs u = base_args(c);
+  u.mode = dm0::kModeSwiGLU;
+  u.ssq_in = ssq_mlp;
+  u.inv_hidden = 1.0f / H;
+  u.act = act;
+  u.inter = I;
+  TRY(run_gemm(c, s, xn, tokens, H, w.wgu, 2 * I, u));
+  GemmArgs d = base_args(c);
+  d.mode = dm0::kModeResid;
+  d.h = h;
+  d.H = H;
+  d.xn = next_gain ? xn : nullptr;
+  d.gain_next = next_gain;
+  d.ssq_out = next_gain ? next_ssq : nullptr;
+  return run_gemm(c, s, act, tokens, I, w.wd, H, d);
+}
+
+dm0_status enqueue_prefill(dm0_ctx* c, cudaStream_t s, const void* prefix_emb, int B, int P) {
+  const dm0_config& cf = c->cfg;
+  const int M = B * P, L = cf.layers, D = cf.head_dim;
+  const size_t lstride = static_cast<size_t>(B) * cf.n_kv * P * D;
+  TRY(rows_prep(c, s, prefix_emb, 1, c->h_v, c->xn_v, c->lw[0][0].attn_norm, c->ssq_v, 2 * L, M, cf.hidden_v));
+  for (int l = 0; l < L; ++l) {
+    bf16* kl = c->kplane + l * lstride;
+    bf16* vl = c->vplane + l * lstride;
+    float* ssq_attn = c->ssq_v + static_cast<size_t>(2 * l) * M;
+    float* ssq_mlp = ssq_attn + M;
+    TRY(layer_qkv(c, s, 0, l, c->xn_v, ssq_attn, M, P, 0, c->q_v, kl, vl));
+    TRY(run_attn(c, s, c->q_v, P, kl, vl, P, nullptr, nullptr, 0, c->o_v, B, 1, 0));
+    const bool more = l + 1 < L;
+    TRY(layer_rest(c, s, 0, l, M, c->h_v, c->xn_v, c->o_v, c->act_v, ssq_mlp,
+                   more ? c->lw[0][l + 1].attn_norm : nullptr, more ? ssq_mlp + M : nullptr));
+  }
+  return DM0_OK;
+}
+
+dm0_status step(dm0_ctx* c, cudaStream_t s, int B, int k_out, int k_in, int steps, float* vel) {
+  const dm0_config& cf = c->cfg;
+  StepArgs a{};
+  a.x = c->x;
+  a.h = c->h_a;
+  a.xn = c->xn_a;
+  a.ssq = c->ssq_a;
+  a.n_slots = 2 * cf.layers;
+  a.tokens = B * cf.chunk;
+  a.W_in = c->W_in;
+  a.b_in = c->b_in;
+  a.attn_norm0 = c->lw[1][0].attn_norm;
+  a.final_norm = c->final_norm;
+  a.W_out = c->W_out;
+  a.b_out = c->b_out;
+  a.Ha = cf.hidden_a;
+  a.A = cf.action_dim;
+  a.eps = cf.rms_eps;
+  a.k_out = k_out;
+  a.k_in = k_in;
+  a.steps = steps;
+  a.vel = vel;
+  return launch(c, s, dm0::step_kernel, dim3(B * cf.chunk), dim3(256), 0, a);
+}
+
+// Euler loop over the KV cache; x already holds x_1
+dm0_status enqueue_denoise(dm0_ctx* c, cudaStream_t s, int steps, float* vel) {
+  const dm0_config& cf = c->cfg;
+  const int B = c->kv_B, P = c->kv_P, S = cf.chunk, L = cf.layers, D = cf.head_dim;
+  const int Ms = B * S;
+  const size_t lstride = static_cast<size_t>(B) * cf.n_kv * P * D;
+  TRY(step(c, s, B, -1, 0, steps, vel));
+  for (int k = 0; k < steps; ++k) {
+    for (int l = 0; l < L; ++l) {
+      const bf16* kl = c->kplane + l * lstride;
+      const bf16* vl = c->vplane + l * lstride;
+      float* ssq_attn = c->ssq_a + static_cast<size_t>(2 * l) * Ms;
+      float* ssq_mlp = ssq_attn + Ms;
+      TRY(layer_qkv(c, s, 1, l, c->xn_a, ssq_attn, Ms, S, P, c->q_a, c->k_s, c->v_s));
+      TRY(run_attn(c, s, c->q_a, S, kl, vl, P, c->k_s, c->v_s, S, c->o_a, B, 0, 1));
+      const bool more = l + 1 < L;
+      TRY(layer_rest(c, s, 1, l, Ms, c->h_a, c->xn_a, c->o_a, c->act_a, ssq_mlp,
+                     more ? c->lw[1][l + 1].attn_norm : nullptr, more ? ssq_mlp + Ms : nullptr));
+    }
+    TRY(step(c, s, B, k, k + 1 < steps ? k + 1 : -1, steps, vel));
+  }
+  return DM0_OK;
+}
+
+dm0_status denoise_from_x(dm0_ctx* c, cudaStream_t s, int steps, float* vel) {
+  if (vel || !c->use_graph) return enqueue_denoise(c, s, steps, vel);
+  const auto key = std::make_tuple(c->kv_B, c->kv_P, steps);
+  auto it = c->graphs.find(key);
+  if (it == c->graphs.end()) {
+    CK(cudaStreamBeginCapture(c->cap_stream, cudaStreamCaptureModeThreadLocal));
+    dm0_status st = enqueue_denoise(c, c->cap_stream, steps, nullptr);
+    cudaGraph_t graph = nullptr;
+    cudaError_t e = cudaStreamEndCapture(c->cap_stream, &graph);
+    if (st != DM0_OK) {
+      if (graph) cudaGraphDestroy(graph);
+      return st;
+    }
+    if (e != cudaSuccess) return fail(c, DM0_ECUDA, std::string("graph capture: ") + cudaGetErrorString(e));
+    cudaGraphExec_t exec = nullptr;
+    e = cudaGraphInstantiate(&exec, graph, 0);
+    cudaGraphDestroy(graph);
+    if (e != cudaSuccess) return fail(c, DM0_ECUDA, std::string("graph instantiate: ") + cudaGetErrorString(e));
+    it = c->graphs.emplace(key, exec).first;
+  }
+  CK(cudaGraphLaunch(it->second, s));
+  return DM0_OK;
+}
+
+bool cfg_ok(const dm0_config& g, std::string* why) {
+  auto bad = [&](const char* m) {
+    *why = m;
+    return false;
+  };
+  if (g.layers < 1) return bad("layers must be >= 1");
+  if (g.head_dim != 32 && g.head_dim != 64 && g.head_dim != 128) return bad("head_dim must be 32, 64 or 128");
+  if (g.n_q < 1 || g.n_kv < 1 || g.n_q % g.n_kv != 0) return bad("n_q must be a positive multiple of n_kv");
+  if (g.hidden_v % 128 || g.hidden_a % 128) return bad("hidden sizes must be multiples of 128");
+  if (g.inter_v % 128 || g.inter_a % 128) return bad("intermediate sizes must be multiples of 128");
+  if ((g.n_q * g.head_dim) % 128 || (g.n_kv * g.head_dim) % 32) return bad("head layout must tile by 128 columns");
+  if (qkv_rows(g) % 128) return bad("(n_q + 2 n_kv) * head_dim must be a multiple of 128");
+  if (g.action_dim < 1 || g.action_dim > 64) return bad("action_dim must be in [1, 64]");
+  if (g.chunk < 1 || g.max_batch < 1 || g.max_prefix < 1) return bad("chunk, max_batch, max_prefix must be >= 1");
+  if (g.max_prefix + g.chunk > 65536) return bad("max_prefix + chunk must be <= 65536");
+  if (static_cast<long long>(g.max_batch) * g.chunk > 1 << 20) return bad("max_batch * chunk too large");
+  if (!(g.rms_eps > 0.f) || !(g.rope_theta > 1.f)) return bad("rms_eps must be > 0 and rope_theta > 1");
+  return true;
+}
+
+size_t layer_bytes(const dm0_config& g, int br) {
+  const size_t H = hidden_of(g, br), I = inter_of(g, br), D = g.head_dim;
+  const size_t qd = g.n_q * D, kvd = g.n_kv * D;
+  return 4 * (H + D + D + H) + 2 * (qd * H + 2 * kvd * H + H * qd + 2 * I * H + H * I);
+}
+
+size_t blob_bytes(const dm0_config& g) {
+  const size_t Ha = g.hidden_a, A = g.action_dim;
+  return g.layers * (layer_bytes(g, 0) + layer_bytes(g, 1)) + 2 * Ha * A + 4 * Ha + 4 * Ha + 2 * A * Ha + 4 * A;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+
+extern "C" {
+
+size_t dm0_weights_bytes(const dm0_config* cfg) { return cfg ? blob_bytes(*cfg) : 0; }
+
+dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
+  if (!cfg || !out) return DM0_EINVAL;
+  *out = nullptr;
+  std::string why;
+  if (!cfg_ok(*cfg, &why)) return DM0_ESHAPE;
+  dm0_ctx* c = new dm0_ctx();
+  c->cfg = *cfg;
+  const dm0_config& g = c->cfg;
+  auto bail = [&](dm0_status st) {
+    dm0_destroy(c);
+    return st;
+  };
+  if (cudaGetDevice(&c->device) != cudaSuccess) return bail(DM0_ECUDA);
+  cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device);
+  if (const char* e = std::getenv("DM0_NO_PDL")) c->use_pdl = e[0] == '0';
+  if (const char* e = std::getenv("DM0_NO_GRAPH")) c->use_graph = e[0] == '0';
+
+  // weights: one allocation, 256-byte aligned sub-buffers
+  size_t total = 0;
+  std::vector<size_t> offs;
+  auto take = [&](size_t bytes) {
+    offs.push_back(total);
+    total += align256(bytes);
+  };
+  for (int br = 0; br < 2; ++br) {
+    const size_t H = hidden_of(g, br), I = inter_of(g, br);
+    for (int l = 0; l < g.layers; ++l) {
+      take(2 * qkv_rows(g) * H);
+      take(2 * H * g.n_q * g.head_dim);
+      take(2 * 2 * I * H);
+      take(2 * H * I);
+      take(4 * H);
+      take(4 * g.head_dim);
+      take(4 * g.head_dim);
+      take(4 * H);
+    }
+  }
+  take(2 * g.hidden_a * g.action_dim);
+  take(4 * g.hidden_a);
+  take(4 * g.hidden_a);
+  take(2 * g.action_dim * g.hidden_a);
+  take(4 * g.action_dim);
+  uint8_t* wb = nullptr;
+  if (dalloc(c, &wb, total) != DM0_OK) return bail(DM0_ENOMEM);
+  c->wbuf = wb;
+  size_t k = 0;
+  for (int br = 0; br < 2; ++br) {
+    c->lw_store[br].resize(g.layers);
+    for (int l = 0; l < g.layers; ++l) {
+      LayerW& w = c->lw_store[br][l];
+      w.wqkv = reinterpret_cast<bf16*>(wb + offs[k++]);
+      w.wo = reinterpret_cast<bf16*>(wb + offs[k++]);
+      w.wgu = reinterpret_cast<bf16*>(wb + offs[k++]);
+      w.wd = reinterpret_cast<bf16*>(wb + offs[k++]);
+      w.attn_norm = reinterpret_cast<float*>(wb + offs[k++]);
+      w.q_norm = reinterpret_cast<float*>(wb + offs[k++]);
+      w.k_norm = reinterpret_cast<float*>(wb + offs[k++]);
+      w.mlp_norm = reinterpret_cast<float*>(wb + offs[k++]);
+    }
+    c->lw[br] = c->lw_store[br].data();
+  }
+  c->W_in = reinterpret_cast<bf16*>(wb + offs[k++]);
+  c->b_in = reinterpret_cast<float*>(wb + offs[k++]);
+  c->final_norm = reinterpret_cast<float*>(wb + offs[k++]);
+  c->W_out = reinterpret_cast<bf16*>(wb + offs[k++]);
+  c->b_out = reinterpret_cast<float*>(wb + offs[k++]);
+
+  const size_t D = g.head_dim, qd = g.n_q * D;
+  const size_t Mp = static_cast<size_t>(g.max_batch) * g.max_prefix;
+  const size_t Ms = static_cast<size_t>(g.max_batch) * g.chunk;
+  const size_t plane = static_cast<size_t>(g.layers) * g.max_batch * g.n_kv * g.max_prefix * D;
+  dm0_status st = DM0_OK;
+  auto A = [&](dm0_status s2) {
+    if (st == DM0_OK) st = s2;
+  };
+  A(dalloc(c, &c->kplane, plane));
+  A(dalloc(c, &c->vplane, plane));
+  A(dalloc(c, &c->h_v, Mp * g.hidden_v));
+  A(dalloc(c, &c->xn_v, Mp * g.hidden_v));
+  A(dalloc(c, &c->q_v, Mp * qd));
+  A(dalloc(c, &c->o_v, Mp * qd));
+  A(dalloc(c, &c->act_v, Mp * g.inter_v));
+  A(dalloc(c, &c->ssq_v, Mp * 2 * g.layers));
+  A(dalloc(c, &c->h_a, Ms * g.hidden_a));
+  A(dalloc(c, &c->xn_a, Ms * g.hidden_a));
+  A(dalloc(c, &c->q_a, Ms * qd));
+  A(dalloc(c, &c->o_a, Ms * qd));
+  A(dalloc(c, &c->act_a, Ms * g.inter_a));
+  A(dalloc(c, &c->ssq_a, Ms * 2 * g.layers));
+  A(dalloc(c, &c->x, Ms * g.action_dim));
+  A(dalloc(c, &c->k_s, Ms * g.n_kv * D));
+  A(dalloc(c, &c->v_s, Ms * g.n_kv * D));
+  size_t widest = qkv_rows(g);
+  for (int br = 0; br < 2; ++br) widest = std::max(widest, static_cast<size_t>(2 * inter_of(g, br)));
+  c->acc_elems = 128 * widest;
+  A(dalloc(c, &c->acc, c->acc_elems));
+  A(dalloc(c, &c->gcount, 1024));
+  const int G = g.n_q / g.n_kv;
+  c->acount_n = g.max_batch * g.n_kv * ((G * std::max(g.max_prefix, g.chunk) + 127) / 128) + 64;
+  A(dalloc(c, &c->acount, c->acount_n));
+  A(dalloc(c, &c->part_o, static_cast<size_t>(kPartSlots) * 128 * D));
+  A(dalloc(c, &c->part_ml, static_cast<size_t>(kPartSlots) * 128));
+  const int max_pos = g.max_prefix + g.chunk;
+  A(dalloc(c, &c->rope, static_cast<size_t>(max_pos) * D / 2));
+  A(dalloc(c, &c->d_err, 1));
+  A(dalloc(c, &c->stage_prefix, Mp * g.hidden_v));
+  if (st != DM0_OK) return bail(st);
+  if (cudaMemset(c->acc, 0, c->acc_elems * 4) != cudaSuccess || cudaMemset(c->gcount, 0, 1024 * 4) != cudaSuccess ||
+      cudaMemset(c->acount, 0, c->acount_n * 4) != cudaSuccess || cudaMemset(c->d_err, 0, 4) != cudaSuccess)
+    return bail(DM0_ECUDA);
+  const int nrope = max_pos * static_cast<int>(D / 2);
+  dm0::rope_table_kernel<<<(nrope + 255) / 256, 256>>>(c->rope, max_pos, static_cast<int>(D / 2),
+                                                       std::log(static_cast<double>(g.rope_theta)));
+  if (cudaGetLastError() != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) return bail(DM0_ECUDA);
+  if (cudaStreamCreateWithFlags(&c->cap_stream, cudaStreamNonBlocking) != cudaSuccess) return bail(DM0_ECUDA);
+
+  auto smem_attr = [&](auto kernel, int bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+  };
+  bool ok = smem_attr(dm0::gemm_tc_kernel<64, kGemmStages>, dm0::GemmSmem<64, kGemmStages>::kBytes) &&
+            smem_attr(dm0::gemm_tc_kernel<128, kGemmStages>, dm0::GemmSmem<128, kGemmStages>::kBytes) &&
+            smem_attr(dm0::gemm_tc_kernel<256, kGemmStages>, dm0::GemmSmem<256, kGemmStages>::kBytes) &&
+            smem_attr(dm0::attn_kernel<128>, dm0::AttnSmem<128>::kBytes) &&
+            smem_attr(dm0::attn_kernel<64>, dm0::AttnSmem<64>::kBytes) &&
+            smem_attr(dm0::attn_kernel<32>, dm0::AttnSmem<32>::kBytes);
+  if (!ok) return bail(DM0_ECUDA);
+  *out = c;
+  return DM0_OK;
+}
+
+dm0_status dm0_load_weights(dm0_ctx* c, const void* blob, size_t bytes) {
+  if (!c || !blob) return fail(c, DM0_EINVAL, "null context or blob");
+  const dm0_config& g = c->cfg;
+  if (bytes != blob_bytes(g))
+    return fail(c, DM0_ESHAPE, "blob is " + std::to_string(bytes) + " bytes, expected " + std::to_string(blob_bytes(g)));
+  const uint8_t* p = static_cast<const uint8_t*>(blob);
+  auto put = [&](void* dst, size_t n) -> dm0_status {
+    CK(cudaMemcpy(dst, p, n, cudaMemcpyHostToDevice));
+    p += n;
+    return DM0_OK;
+  };
+  const size_t D = g.head_dim;
+  for (int br = 0; br < 2; ++br) {
+    const size_t H = hidden_of(g, br), I = inter_of(g, br);
+    const size_t qd = g.n_q * D, kvd = g.n_kv * D;
+    for (int l = 0; l < g.layers; ++l) {
+      const LayerW& w = c->lw[br][l];
+      TRY(put(w.attn_norm, 4 * H));
+      TRY(put(w.wqkv, 2 * qd * H));
+      TRY(put(w.wqkv + qd * H, 2 * kvd * H));
+      TRY(put(w.wqkv + (qd + kvd) * H, 2 * kvd * H));
+      TRY(put(w.q_norm, 4 * D));
+      TRY(put(w.k_norm, 4 * D));
+      TRY(put(w.wo, 2 * H * qd));
+      TRY(put(w.mlp_norm, 4 * H));
+      // gate/up interleaved in 64-row blocks: rows [128j, 128j+64) gate block j, [128j+64, 128j+128) up block j
+      for (int part = 0; part < 2; ++part) {
+        CK(cudaMemcpy2D(w.wgu + part * 64 * H, 128 * H * 2, p, 64 * H * 2, 64 * H * 2, I / 64,
+                        cudaMemcpyHostToDevice));
+        p += 2 * I * H;
+      }
+      TRY(put(w.wd, 2 * H * I));
+    }
+  }
+  const size_t Ha = g.hidden_a, Ad = g.action_dim;
+  TRY(put(c->W_in, 2 * Ha * Ad));
+  TRY(put(c->b_in, 4 * Ha));
+  TRY(put(c->final_norm, 4 * Ha));
+  TRY(put(c->W_out, 2 * Ad * Ha));
+  TRY(put(c->b_out, 4 * Ad));
+  c->weights_loaded = true;
+  return DM0_OK;
+}
+
+dm0_status dm0_prefill(dm0_ctx* c, const void* prefix_emb, int B, int P, void* stream) {
+  if (!c || !prefix_emb) return fail(c, DM0_EINVAL, "null context or prefix");
+  if (!c->weights_loaded) return fail(c, DM0_ESTATE, "weights not loaded");
+  if (B < 1 || B > c->cfg.max_batch || P < 1 || P > c->cfg.max_prefix)
+    return fail(c, DM0_ESHAPE, "B or P outside the context capacity");
+  c->kv_B = 0;
+  TRY(enqueue_prefill(c, static_cast<cudaStream_t>(stream), prefix_emb, B, P));
+  c->kv_B = B;
+  c->kv_P = P;
+  return DM0_OK;
+}
+
+dm0_status dm0_kv_view(dm0_ctx* c, void** k, void** v) {
+  if (!c || !k || !v) return fail(c, DM0_EINVAL, "null argument");
+  *k = c->kplane;
+  *v = c->vplane;
+  return DM0_OK;
+}
+
+dm0_status dm0_kv_commit(dm0_ctx* c, int B, int P) {
+  if (!c) return DM0_EINVAL;
+  if (B < 1 || B > c->cfg.max_batch || P < 1 || P > c->cfg.max_prefix)
+    return fail(c, DM0_ESHAPE, "B or P outside the context capacity");
+  c->kv_B = B;
+  c->kv_P = P;
+  return DM0_OK;
+}
+
+dm0_status dm0_denoise(dm0_ctx* c, const float* noise, int steps, float* actions, float* vel, void* stream) {
+  if (!c || !noise || !actions) return fail(c, DM0_EINVAL, "null argument");
+  if (!c->weights_loaded) return fail(c, DM0_ESTATE, "weights not loaded");
+  if (c->kv_B == 0) return fail(c, DM0_ESTATE, "no KV cache: call dm0_prefill or dm0_kv_commit first");
+  if (steps < 1 || steps > 1000) return fail(c, DM0_ESHAPE, "steps must be in [1, 1000]");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t bytes = static_cast<size_t>(c->kv_B) * c->cfg.chunk * c->cfg.action_dim * sizeof(float);
+  CK(cudaMemcpyAsync(c->x, noise, bytes, cudaMemcpyDeviceToDevice, s));
+  TRY(denoise_from_x(c, s, steps, vel));
+  CK(cudaMemcpyAsync(actions, c->x, bytes, cudaMemcpyDeviceToDevice, s));
+  return DM0_OK;
+}
+
+dm0_status dm0_infer_host(dm0_ctx* c, const void* prefix_emb, const float* noise, int B, int P, int steps,
+                          float* actions, void* stream) {
+  if (!c || !prefix_emb || !noise || !actions) return fail(c, DM0_EINVAL, "null argument");
+  if (!c->weights_loaded) return fail(c, DM0_ESTATE, "weights not loaded");
+  if (B < 1 || B > c->cfg.max_batch || P < 1 || P > c->cfg.max_prefix || steps < 1 || steps > 1000)
+    return fail(c, DM0_ESHAPE, "B, P or steps outside the context capacity");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t pbytes = static_cast<size_t>(B) * P * c->cfg.hidden_v * 2;
+  const size_t xbytes = static_cast<size_t>(B) * c->cfg.chunk * c->cfg.action_dim * sizeof(float);
+  CK(cudaMemcpyAsync(c->stage_prefix, prefix_emb, pbytes, cudaMemcpyHostToDevice, s));
+  CK(cudaMemcpyAsync(c->x, noise, xbytes, cudaMemcpyHostToDevice, s));
+  c->kv_B = 0;
+  TRY(enqueue_prefill(c, s, c->stage_prefix, B, P));
+  c->kv_B = B;
+  c->kv_P = P;
+  TRY(denoise_from_x(c, s, steps, nullptr));
+  CK(cudaMemcpyAsync(actions, c->x, xbytes, cudaMemcpyDeviceToHost, s));
+  CK(cudaStreamSynchronize(s));
+  return DM0_OK;
+}
+
+dm0_status dm0_merged_layer(dm0_ctx* c, int layer, const float* h_prefix, const float* h_suffix, int B, int P,
+                            float* out_prefix, float* out_suffix, void* k_out, void* v_out, void* stream) {
+  if (!c || !h_prefix || !h_suffix || !out_prefix || !out_suffix || !k_out || !v_out)
+    return fail(c, DM0_EINVAL, "null argument");
+  if (!c->weights_loaded) return fail(c, DM0_ESTATE, "weights not loaded");
+  const dm0_config& g = c->cfg;
+  if (layer < 0 || layer >= g.layers || B < 1 || B > g.max_batch || P < 1 || P > g.max_prefix)
+    return fail(c, DM0_ESHAPE, "layer, B or P outside the context capacity");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int Mp = B * P, S = g.chunk, Ms = B * S;
+  bf16* kp = static_cast<bf16*>(k_out);
+  bf16* vp = static_cast<bf16*>(v_out);
+  TRY(rows_prep(c, s, h_prefix, 0, c->h_v, c->xn_v, c->lw[0][layer].attn_norm, c->ssq_v, 2, Mp, g.hidden_v));
+  TRY(rows_prep(c, s, h_suffix, 0, c->h_a, c->xn_a, c->lw[1][layer].attn_norm, c->ssq_a, 2, Ms, g.hidden_a));
+  TRY(layer_qkv(c, s, 0, layer, c->xn_v, c->ssq_v, Mp, P, 0, c->q_v, kp, vp));
+  TRY(layer_qkv(c, s, 1, layer, c->xn_a, c->ssq_a, Ms, S, P, c->q_a, c->k_s, c->v_s));
+  // the block mask: prefix rows see the prefix; suffix rows see prefix and suffix
+  TRY(run_attn(c, s, c->q_v, P, kp, vp, P, nullptr, nullptr, 0, c->o_v, B, 1, 0));
+  TRY(run_attn(c, s, c->q_a, S, kp, vp, P, c->k_s, c->v_s, S, c->o_a, B, 0, 0));
+  TRY(layer_rest(c, s, 0, layer, Mp, c->h_v, c->xn_v, c->o_v, c->act_v, c->ssq_v + Mp, nullptr, nullptr));
+  TRY(layer_rest(c, s, 1, layer, Ms, c->h_a, c->xn_a, c->o_a, c->act_a, c->ssq_a + Ms, nullptr, nullptr));
+  CK(cudaMemcpyAsync(out_prefix, c->h_v, static_cast<size_t>(Mp) * g.hidden_v * 4, cudaMemcpyDeviceToDevice, s));
+  CK(cudaMemcpyAsync(out_suffix, c->h_a, static_cast<size_t>(Ms) * g.hidden_a * 4, cudaMemcpyDeviceToDevice, s));
+  return DM0_OK;
+}
+
+dm0_status dm0_op_gemm(dm0_ctx* c, const void* A, const void* B, float* C, int M, int N, int K, int swap,
+                       int splits, void* stream) {
+  if (!c || !A || !B || !C) return fail(c, DM0_EINVAL, "null argument");
+  if (M < 1 || N < 1 || K < 64 || K % 64 != 0 || splits < 1) return fail(c, DM0_ESHAPE, "bad GEMM shape");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  GemmArgs g = base_args(c);
+  g.mode = dm0::kModeStoreF32;
+  if (swap) {
+    if (M % 128 != 0 || N > 128) return fail(c, DM0_ESHAPE, "swap GEMM needs M % 128 == 0 and N <= 128");
+    g.acc = C;
+    g.ld_acc = M;
+    return run_gemm(c, s, static_cast<const bf16*>(B), N, K, static_cast<const bf16*>(A), M, g, 1, splits);
+  }
+  if (N % 128 != 0 || splits != 1) return fail(c, DM0_ESHAPE, "GEMM needs N % 128 == 0 and splits == 1");
+  g.out_f32 = C;
+  return run_gemm(c, s, static_cast<const bf16*>(A), M, K, static_cast<const bf16*>(B), N, g, 0, 1);
+}
+
+dm0_status dm0_op_attention(dm0_ctx* c, const void* q, const void* ka, const void* va, int Ta, const void* kb,
+                            const void* vb, int Tb, void* o, int B, int Tq, int splits, void* stream) {
+  if (!c || !q || !ka || !va || !o || (Tb > 0 && (!kb || !vb))) return fail(c, DM0_EINVAL, "null argument");
+  if (B < 1 || Tq < 1 || Ta < 1 || Tb < 0 || splits < 1) return fail(c, DM0_ESHAPE, "bad attention shape");
+  const int G = c->cfg.n_q / c->cfg.n_kv;
+  if (splits > 1 && B * c->cfg.n_kv * ((G * Tq + 127) / 128) > c->acount_n)
+    return fail(c, DM0_ESHAPE, "too many row tiles for a split launch");
+  return run_attn(c, static_cast<cudaStream_t>(stream), static_cast<const bf16*>(q), Tq, static_cast<const bf16*>(ka),
+                  static_cast<const bf16*>(va), Ta, static_cast<const bf16*>(kb), static_cast<const bf16*>(vb), Tb,
+                  static_cast<bf16*>(o), B, splits, 0);
+}
+
+dm0_status dm0_sync(dm0_ctx* c, void* stream) {
+  if (!c) return DM0_EINVAL;
+  CK(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  int e = 0;
+  CK(cudaMemcpy(&e, c->d_err, 4, cudaMemcpyDeviceToHost));
+  if (e) return fail(c, DM0_EDEVICE, "device error word " + std::to_string(e));
+  return DM0_OK;
+}
+
+int dm0_device_error(const dm0_ctx* c) {
+  if (!c) return -1;
+  int e = 0;
+  if (cudaMemcpy(&e, c->d_err, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return -1;
+  return e;
+}
+
+dm0_status dm0_clear_error(dm0_ctx* c) {
+  if (!c) return DM0_EINVAL;
+  CK(cudaDeviceSynchronize());
+  CK(cudaMemset(c->d_err, 0, 4));
+  CK(cudaMemset(c->acc, 0, c->acc_elems * 4));
+  CK(cudaMemset(c->gcount, 0, 1024 * 4));
+  CK(cudaMemset(c->acount, 0, c->acount_n * 4));
+  CK(cudaDeviceSynchronize());
+  return DM0_OK;
+}
+
+const char* dm0_last_error(const dm0_ctx* c) {
+  if (!c) return "null context";
+  return c->err.c_str();
+}
+
+void dm0_destroy(dm0_ctx* c) {
+  if (!c) return;
+  for (auto& kv : c->graphs) cudaGraphExecDestroy(kv.second);
+  if (c->cap_stream) cudaStreamDestroy(c->cap_stream);
+  for (void* p : c->allocs) cudaFree(p);
+  delete c;
+}
+
+}  // extern "C"
