@@ -1,0 +1,373 @@
+#!/usr/bin/env python
+"""Throughput of the DM0 merged-attention inference path on B200.
+
+One step = the whole hot path over one batch: dm0_prefill of B prefixes of P
+tokens (28 VLM layers, KV cache) + a 10-step Euler dm0_denoise of the
+28-layer action expert, producing B action chunks of 50 x 32.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload e2e_b16|e2e_b1]
+                    [--impl native|reference]
+
+Default workload e2e_b16: B = 16, P = 2048 (the batched throughput regime);
+the same line also carries the batch-1 figure (B = 1, P = 816) under
+"batch1".  Inputs are seeded synthetic data of the DM0-base shapes with
+random N(0, 0.02) weights.  Multi-GPU: one process per GPU, each rank runs
+its own batch (samples are independent: no collective on the data path).
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded
+sample of the same workload (the reference arm of this library).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "action chunks/sec (prefill+10-step denoise) at batch 1 and 16; HBM GB/s, TC util"
+EULER_STEPS = 10
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained", j["bf16_tflops"]), "src": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "src": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self._t = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, smax, reasons = [], 0.0, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax = max(smax, float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        sm.sort()
+        med = sm[len(sm) // 2] if sm else None
+        return {"sm_mhz": med, "sm_max_mhz": smax or None, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ algorithmic work per unit
+
+def layer_params(d, branch):
+    H, I, D = d.hidden(branch), d.inter(branch), d.head_dim
+    return H * (d.n_q + 2 * d.n_kv) * D + d.n_q * D * H + 3 * H * I
+
+
+def prefill_gateup_flops(d, B, P):
+    """One VLM gate/up GEMM launch: [B*P x H] x [H -> 2I]."""
+    return 2.0 * B * P * d.hidden_v * 2 * d.inter_v
+
+
+def denoise_bytes_per_step(d, B, P):
+    """Algorithmic HBM bytes of one Euler step: action-expert bf16 weights + prefix KV cache read once."""
+    w = d.layers * layer_params(d, 1) * 2
+    kv = d.layers * B * d.n_kv * P * d.head_dim * 2 * 2
+    return w + kv
+
+
+# ------------------------------------------------------------------ native arm
+
+def run_native(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    from synth import inputs as I
+    from vla_dual_expert_b200 import Engine
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    d = I.DM0_BASE
+    wl_main = I.WORKLOADS[args.workload]
+    weights = I.Weights(d, seed=0)
+    peaks = _peaks()
+    eng = Engine(d, max(wl_main.batch, 1), max(wl_main.prefix, 816))
+    eng.load_from(weights)
+    stream = torch.cuda.current_stream()
+
+    def measure(wl, steps, warmup, probe):
+        B, P = wl.batch, wl.prefix
+        emb = torch.from_numpy(I.prefix_embeddings(d, B, P, seed=1000 + 97 * rank)).cuda().to(torch.bfloat16)
+        noise = torch.from_numpy(I.noise(d, B, seed=2000 + 97 * rank)).cuda()
+        out = torch.empty_like(noise)
+        for _ in range(warmup):
+            eng.prefill(emb)
+            eng.denoise(noise, EULER_STEPS, actions=out)
+        eng.sync()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+               torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        barrier()
+        torch.cuda.synchronize()
+        eng.probe(probe)
+        launches0 = eng.launch_count()
+        with ClockSampler(local_rank) as clk:
+            t0 = torch.cuda.Event(enable_timing=True)
+            t1 = torch.cuda.Event(enable_timing=True)
+            t0.record(stream)
+            for i in range(steps):
+                ev[i][0].record(stream)
+                eng.prefill(emb)
+                ev[i][1].record(stream)
+                eng.denoise(noise, EULER_STEPS, actions=out)
+                ev[i][2].record(stream)
+            t1.record(stream)
+            torch.cuda.synchronize()
+        barrier()
+        launches = eng.launch_count() - launches0
+        probe_n, probe_ms = eng.probe_read()
+        eng.probe(0)
+        eng.sync()
+        ms = max_over_ranks(t0.elapsed_time(t1) / steps)
+        pre = sorted(e[0].elapsed_time(e[1]) for e in ev)
+        den = sorted(e[1].elapsed_time(e[2]) for e in ev)
+        assert bool(torch.isfinite(out).all())
+        return {"ms": ms, "prefill_ms_p50": pre[len(pre) // 2], "denoise_ms_p50": den[len(den) // 2],
+                "prefill_ms_p90": pre[min(len(pre) - 1, int(0.9 * len(pre)))],
+                "denoise_ms_p90": den[min(len(den) - 1, int(0.9 * len(den)))],
+                "launches": launches, "probe_n": probe_n, "probe_ms": probe_ms, "clocks": clk.summary()}
+
+    def measure_e2e(wl, steps, warmup):
+        """Through dm0_infer_host: pinned host inputs copied in and the chunk copied out every step."""
+        B, P = wl.batch, wl.prefix
+        emb_bits = torch.from_numpy(I.bf16_bits(I.prefix_embeddings(d, B, P, seed=1000 + 97 * rank)))
+        emb_h = torch.empty(emb_bits.shape, dtype=torch.int16, pin_memory=True)
+        emb_h.copy_(emb_bits.view(torch.int16))
+        noise_h = torch.empty((B, d.chunk, d.action_dim), dtype=torch.float32, pin_memory=True)
+        noise_h.copy_(torch.from_numpy(I.noise(d, B, seed=2000 + 97 * rank)))
+        out_h = torch.empty_like(noise_h).pin_memory()
+        a_emb, a_noise, a_out = emb_h.numpy(), noise_h.numpy(), out_h.numpy()
+        for _ in range(warmup):
+            eng.infer_host(a_emb, a_noise, EULER_STEPS, actions=a_out)
+        barrier()
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(steps):
+            eng.infer_host(a_emb, a_noise, EULER_STEPS, actions=a_out)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms = max_over_ranks(t0.elapsed_time(t1) / steps)
+        return {"ms": ms, "h2d": emb_h.numel() * 2 + noise_h.numel() * 4, "d2h": out_h.numel() * 4}
+
+    # probe kind 1 = the VLM gate/up GEMM of the prefix pass (the largest launch of the step)
+    main = measure(wl_main, args.steps, args.warmup, probe=1)
+    e2e = measure_e2e(wl_main, max(2, args.steps // 2), 1)
+    B, P = wl_main.batch, wl_main.prefix
+    value = world * B * 1000.0 / main["ms"]
+    gu_ms = main["probe_ms"] / max(main["probe_n"], 1)
+    gu_tf = prefill_gateup_flops(d, B, P) / (gu_ms * 1e-3) / 1e12
+    tc_peak = peaks["bf16_tflops_sustained"]
+    result = {
+        "metric": METRIC, "value": round(value, 3), "unit": "chunks/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(main["ms"], 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) prefix embeddings and noise; "
+                                                      "random N(0,0.02) DM0-base weights)",
+        "config": {"workload": f"{wl_main.name}: prefill B={B} x P={P} + {EULER_STEPS}-step denoise, chunk 50x32, "
+                               "DM0-base 28+28 layers", "batch_per_gpu": B, "prefix_len": P,
+                   "euler_steps": EULER_STEPS, "parallelism": f"replicas x{world} (data-parallel by sample)",
+                   "l2": "inputs larger than L2 (3.7 GB of weights streamed per step)"},
+        "prefill_ms_p50": round(main["prefill_ms_p50"], 3), "denoise_ms_p50": round(main["denoise_ms_p50"], 3),
+        "prefill_ms_p90": round(main["prefill_ms_p90"], 3), "denoise_ms_p90": round(main["denoise_ms_p90"], 3),
+        "roofline": {"bound": "tensor", "kernel": "gemm_tc_kernel<256> (prefill gate/up, M=B*P, N=2*6144, K=2048)",
+                     "achieved": round(gu_tf, 1), "peak": tc_peak, "unit": "TFLOP/s",
+                     "frac": round(gu_tf / tc_peak, 4), "traffic": None,
+                     "peak_src": f"{peaks['src']} bf16_tflops_sustained", "launches": main["probe_n"],
+                     "avg_launch_ms": round(gu_ms, 4)},
+        "e2e": {"value": round(world * B * 1000.0 / e2e["ms"], 3), "unit": "chunks/s",
+                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
+        "gpu_launches": main["launches"],
+        "clocks": main["clocks"],
+    }
+    if args.workload == "e2e_b16" and not args.skip_batch1:
+        wl1 = I.WORKLOADS["e2e_b1"]
+        b1 = measure(wl1, max(args.steps, 5), args.warmup, probe=0)
+        den_gbs = denoise_bytes_per_step(d, 1, wl1.prefix) * EULER_STEPS / (b1["denoise_ms_p50"] * 1e-3) / 1e9
+        result["batch1"] = {
+            "workload": "e2e_b1: prefill B=1 x P=816 + 10-step denoise", "value": round(world * 1000.0 / b1["ms"], 3),
+            "unit": "chunks/s", "ms_per_step": round(b1["ms"], 3), "prefill_ms_p50": round(b1["prefill_ms_p50"], 3),
+            "denoise_ms_p50": round(b1["denoise_ms_p50"], 3), "denoise_ms_p90": round(b1["denoise_ms_p90"], 3),
+            "gpu_launches": b1["launches"],
+            "denoise_roofline": {"bound": "hbm", "achieved": round(den_gbs, 1), "peak": peaks["hbm_gbs"],
+                                 "unit": "GB/s", "frac": round(den_gbs / peaks["hbm_gbs"], 4),
+                                 "algorithmic_bytes_per_euler_step": denoise_bytes_per_step(d, 1, wl1.prefix)},
+        }
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        result["cpu_baseline"] = cpu_baseline(wl_main, budget_s=args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    eng.close()
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ the oracle on the host cores
+
+def cpu_baseline(wl, budget_s=20.0):
+    """Time the fp64 oracle as it stands on a bounded sample of the workload and scale to chunks/s.
+
+    Sample: VLM layers 0..nv-1 of the prefix pass of sample 0 and na action-expert layer evaluations
+    (one Euler step's layers over a prefix cache of length P); the per-chunk time is
+    28 * t(VLM layer) + 28 * 10 * t(action layer).
+    """
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    from oracle import dm0_oracle as O
+    from synth import inputs as I
+
+    d = wl.dims
+    P = wl.prefix
+    w = I.Weights(d.replace(layers=2), seed=0)
+    emb = I.prefix_embeddings(d, 1, P)[0]
+    x = I.noise(d, 1)[0]
+    h = np.asarray(emb, np.float64)
+    vis = np.ones((P, P), dtype=bool)
+    t0 = time.perf_counter()
+    nv = 0
+    k_last = v_last = None
+    while True:
+        wv = w.layer(0, nv % 2)
+        q, k, v = O.project_qkv(wv, h, np.arange(P), d)
+        h = O.finish_layer(wv, h, O.attention(q, k, v, vis), d)
+        k_last, v_last = k, v
+        nv += 1
+        if time.perf_counter() - t0 > budget_s * 0.7 or nv >= 28:
+            break
+    t_v = (time.perf_counter() - t0) / nv
+    head = w.head()
+    ha = O.action_input(head, x, 1.0, d)
+    t1 = time.perf_counter()
+    na = 0
+    while True:
+        ha = O.suffix_layer(w.layer(1, na % 2), ha, k_last, v_last, d)
+        na += 1
+        if time.perf_counter() - t1 > budget_s * 0.3 or na >= 280:
+            break
+    t_a = (time.perf_counter() - t1) / na
+    t_chunk = d.layers * t_v + d.layers * EULER_STEPS * t_a
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return {"value": round(1.0 / t_chunk, 6), "unit": "chunks/s", "cores": threads, "kind": "oracle",
+            "sample": f"{nv} VLM layers (P={P}) + {na} action layer evaluations of sample 0, fp64 numpy; "
+                      f"per-chunk time = 28*{t_v:.3f}s + 280*{t_a:.4f}s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    from synth import inputs as I
+    wl = I.WORKLOADS[args.workload]
+    steps, warmup = max(args.steps, 1), max(args.warmup, 0)
+    budget = max(5.0, min(30.0, 150.0 / (steps + warmup)))
+    for _ in range(warmup):
+        cpu_baseline(wl, budget_s=budget / 3)
+    vals = [cpu_baseline(wl, budget_s=budget) for _ in range(steps)]
+    v = sum(x["value"] for x in vals) / len(vals)
+    cb = dict(vals[-1])
+    cb["value"] = round(v, 6)
+    res = {"impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": "chunks/s", "n_gpus": world,
+           "steps": steps, "warmup": warmup, "ms_per_step": round(1000.0 / v, 1), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": f"{wl.name}: prefill B={wl.batch} x P={wl.prefix} + {EULER_STEPS}-step denoise "
+                                  "(bounded per-layer sample, scaled per chunk)"},
+           "cpu_baseline": cb, "e2e": {"value": round(v, 6), "unit": "chunks/s", "h2d_bytes_per_step": 0,
+                                       "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=("native", "reference"))
+    ap.add_argument("--workload", default="e2e_b16", choices=("e2e_b16", "e2e_b1"))
+    ap.add_argument("--skip-batch1", action="store_true")
+    ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "native":
+        args.warmup = 3
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    run_native(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -176,6 +176,35 @@ dm0_status dm0_op_gemm(dm0_ctx* ctx, const void* A, const void* B, float* C, int
 dm0_status dm0_op_attention(dm0_ctx* ctx, const void* q, const void* ka, const void* va, int Ta, const void* kb,
                             const void* vb, int Tb, void* o, int B, int Tq, int splits, void* stream);
 
+/* Device pointer of an internal activation buffer, for tests that check
+ * intermediate results.  `name` is one of: h_v, xn_v, q_v, o_v, act_v, ssq_v
+ * (VLM side, rows = B*P tokens) and h_a, xn_a, q_a, o_a, act_a, ssq_a, x,
+ * k_s, v_s (action side, rows = B*chunk tokens).  Layouts: h_* f32 [rows][H];
+ * xn_* bf16 [rows][H] (gain * h of the pending RMSNorm); q_*, o_* bf16
+ * [rows][n_q*head_dim]; act_* bf16 [rows][inter]; ssq_* f32 [2*layers][rows]
+ * (sum of squares of h for each pending norm); x f32 [rows][action_dim];
+ * k_s/v_s bf16 [B][n_kv][chunk][head_dim].  Context-owned; contents are only
+ * meaningful after the call that fills them has completed. */
+dm0_status dm0_debug_view(dm0_ctx* ctx, const char* name, void** ptr);
+
+/* Instrumentation. ------------------------------------------------------- */
+
+/* Number of kernels this context has enqueued so far (a replayed graph counts
+ * every kernel it contains).  Host-side counter; never synchronises. */
+uint64_t dm0_launch_count(const dm0_ctx* ctx);
+
+/* Time one kernel site with CUDA events recorded on the launching stream
+ * around each of its launches.  kind 0: off; kind 1: the gate/up GEMM of
+ * every VLM layer of dm0_prefill.  Enabling resets the record.  Each timed
+ * launch is preceded by an event record, so it is launched in plain stream
+ * order instead of overlapping the previous kernel.  Events are created on
+ * demand (256 at a time, at most 8192); the graphed denoise is never timed. */
+dm0_status dm0_probe(dm0_ctx* ctx, int kind);
+
+/* Wait for the recorded events and return the number of timed launches and
+ * their summed duration in milliseconds; then clear the record. */
+dm0_status dm0_probe_read(dm0_ctx* ctx, int* launches, double* total_ms);
+
 /* Errors and lifetime. -------------------------------------------------- */
 
 /* Wait for `stream`, then report DM0_EDEVICE if a kernel raised the device

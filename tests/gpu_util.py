@@ -40,3 +40,25 @@ def rel_err(got, ref) -> float:
     e = float(np.max(np.abs(got - ref)) / max(rms(ref), 1e-30))
     print(f"  parity max|d|/rms = {e:.3e}  shape={ref.shape}")
     return e
+
+
+def check_fp(got, ref, tol: float, what: str = ""):
+    """fp32 outputs: max |got - ref| <= tol * RMS(ref)."""
+    e = rel_err(got, ref)
+    assert e <= tol, f"{what}: max|d|/rms {e:.3e} > {tol:.1e}"
+
+
+def check_bf16(got, ref, atol_rms: float, what: str = "", rms_tol: float = 5e-3):
+    """Tensors stored in bf16: |d_i| <= atol_rms * RMS(ref) + 2^-8 |ref_i| for every element
+    (the second term is one bf16 rounding step of the stored value, 2^-9, doubled), and the
+    RMS of the error <= rms_tol * RMS(ref)."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values in GPU output"
+    r = max(rms(ref), 1e-30)
+    d = np.abs(got - ref)
+    ratio = float(np.max(d / (atol_rms * r + 2.0 ** -8 * np.abs(ref))))
+    rms_e = rms(d) / r
+    print(f"  bf16 parity {what}: max ratio {ratio:.3f}, rms err {rms_e:.3e}, max|d|/rms {np.max(d) / r:.3e}")
+    assert ratio <= 1.0 and rms_e <= rms_tol, f"{what}: ratio {ratio:.3f}, rms err {rms_e:.3e}"

@@ -1,10 +1,15 @@
 """Parity of the CUDA path (through the C ABI) with the fp64 oracle.
 
-Tolerances (max |gpu - oracle| / RMS(oracle)):
-  raw GEMM            1e-4   bf16 operands are exact; only fp32 accumulation order differs
-  attention           1e-2   P is rounded to bf16 before PV and O is stored as bf16 (2^-9 each)
-  one merged layer    1e-2   per output tensor (residual streams, prefix K and V)
-  action chunk        2e-2   final x_0; per-step velocities are held to the same 2e-2 of RMS(v)
+Tolerances, as max |gpu - oracle| / RMS(oracle) unless stated:
+  raw GEMM               1e-4  bf16 operands are exact; only the fp32 summation order differs
+  one merged layer       1e-2  fp32 residual-stream outputs of both branches
+  action chunk           2e-2  final x_0; per-step velocities held to 2e-2 of RMS(v)
+  bf16-stored tensors    |d_i| <= a * RMS + 2^-8 |ref_i| and RMS(d) <= r * RMS: the 2^-8 term is
+                         the rounding of the stored bf16 value itself (2^-9, doubled).
+                           K/V cache of one layer        a = 1e-2, r = 5e-3
+                           K/V after several layers      a = 2e-2, r = 1e-2
+                           attention output              a = 2e-2, r = 5e-3 (P is also rounded
+                                                         to bf16 before PV)
 """
 import numpy as np
 import pytest
@@ -12,11 +17,11 @@ import torch
 
 from oracle import dm0_oracle as O
 from synth import inputs as I
-from tests.gpu_util import device_view_bf16, host, rel_err, to_dev_bf16, to_dev_f32
+from tests.gpu_util import check_bf16, check_fp, device_view_bf16, host, rel_err, to_dev_bf16, to_dev_f32
 
 pytestmark = pytest.mark.gpu
 
-TOL_GEMM, TOL_ATTN, TOL_LAYER, TOL_CHUNK = 1e-4, 1e-2, 1e-2, 2e-2
+TOL_GEMM, TOL_LAYER, TOL_CHUNK = 1e-4, 1e-2, 2e-2
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -52,7 +57,7 @@ def test_gemm_normal(layer_engine, M, N, K):
     rng = np.random.default_rng(M + N + K)
     A = I.round_bf16(rng.standard_normal((M, K)).astype(np.float32))
     B = I.round_bf16(rng.standard_normal((N, K)).astype(np.float32))
-    C = torch.full((M, N), float("nan"), device="cuda")
+    C = torch.full((M, N), float("nan"), device="cuda", dtype=torch.float32)
     eng.op_gemm(to_dev_bf16(A), to_dev_bf16(B), C, swap=0)
     eng.sync()
     ref = A.astype(np.float64) @ B.astype(np.float64).T
@@ -66,7 +71,7 @@ def test_gemm_swap_split_k(layer_engine, M, N, K, splits):
     rng = np.random.default_rng(7 * M + N + K + splits)
     W = I.round_bf16(rng.standard_normal((M, K)).astype(np.float32))
     X = I.round_bf16(rng.standard_normal((N, K)).astype(np.float32))
-    C = torch.zeros((N, M), device="cuda")
+    C = torch.zeros((N, M), device="cuda", dtype=torch.float32)
     eng.op_gemm(to_dev_bf16(W), to_dev_bf16(X), C, swap=1, splits=splits)
     eng.sync()
     ref = X.astype(np.float64) @ W.astype(np.float64).T
@@ -94,7 +99,7 @@ def test_attention(layer_engine, B, Tq, Ta, Tb, splits):
         v = va[b] if not Tb else np.concatenate([va[b], vb[b]], axis=1)
         ref = O.attention(q[b].transpose(1, 0, 2).astype(np.float64), k.astype(np.float64), v.astype(np.float64),
                           np.ones((Tq, Ta + Tb), dtype=bool)).transpose(1, 0, 2)
-        assert rel_err(host(o[b]), ref) <= TOL_ATTN
+        check_bf16(host(o[b]), ref, 2e-2, f"attention b={b}")
 
 
 # ------------------------------------------------------------------ one dual-expert layer
@@ -103,18 +108,19 @@ def _check_merged_layer(d, w, eng, layer, B, P, seed):
     S = d.chunk
     hp = np.stack([I.hidden_states(P, d.hidden_v, seed=seed + b) for b in range(B)])
     hs = np.stack([I.hidden_states(S, d.hidden_a, seed=seed + 100 + b) for b in range(B)])
-    outp = torch.empty((B, P, d.hidden_v), device="cuda")
-    outs = torch.empty((B, S, d.hidden_a), device="cuda")
+    outp = torch.empty((B, P, d.hidden_v), device="cuda", dtype=torch.float32)
+    outs = torch.empty((B, S, d.hidden_a), device="cuda", dtype=torch.float32)
     k = torch.empty((B, d.n_kv, P, d.head_dim), device="cuda", dtype=torch.bfloat16)
     v = torch.empty_like(k)
     eng.merged_layer(layer, to_dev_f32(hp), to_dev_f32(hs), outp, outs, k, v)
     eng.sync()
+    assert eng.device_error() == 0
     for b in range(B):
         rp, rs, rk, rv = O.merged_layer(w.layer(0, layer), w.layer(1, layer), hp[b], hs[b], d)
-        assert rel_err(host(outp[b]), rp) <= TOL_LAYER
-        assert rel_err(host(outs[b]), rs) <= TOL_LAYER
-        assert rel_err(host(k[b]), rk) <= TOL_LAYER
-        assert rel_err(host(v[b]), rv) <= TOL_LAYER
+        check_fp(host(outp[b]), rp, TOL_LAYER, "prefix out")
+        check_fp(host(outs[b]), rs, TOL_LAYER, "suffix out")
+        check_bf16(host(k[b]), rk, 1e-2, "prefix K")
+        check_bf16(host(v[b]), rv, 1e-2, "prefix V")
         # the layer's own contribution, not only the residual-dominated sum
         assert rel_err(host(outp[b]) - hp[b], rp - hp[b]) <= 3 * TOL_LAYER
         assert rel_err(host(outs[b]) - hs[b], rs - hs[b]) <= 3 * TOL_LAYER
@@ -161,18 +167,19 @@ def test_tiny_prefill_and_denoise(tiny, B, P, steps):
     emb = I.prefix_embeddings(d, B, P)
     noise = I.noise(d, B)
     eng.prefill(to_dev_bf16(emb))
-    vel = torch.empty((steps, B, d.chunk, d.action_dim), device="cuda")
+    vel = torch.empty((steps, B, d.chunk, d.action_dim), device="cuda", dtype=torch.float32)
     chunk = eng.denoise(to_dev_f32(noise), steps, velocities=vel)
     eng.sync()
     kc, vc = _kv_planes(eng, d, B, P)
     ref_chunks, caches, ref_vels = O.infer(w, emb, noise, steps)
     for b in range(B):
         for l in range(d.layers):
-            assert rel_err(host(kc[l, b]), caches[b][0][l]) <= TOL_LAYER
-            assert rel_err(host(vc[l, b]), caches[b][1][l]) <= TOL_LAYER
+            a, r = (1e-2, 5e-3) if l == 0 else (2e-2, 1e-2)
+            check_bf16(host(kc[l, b]), caches[b][0][l], a, f"K layer {l}", r)
+            check_bf16(host(vc[l, b]), caches[b][1][l], a, f"V layer {l}", r)
         for k in range(steps):
-            assert rel_err(host(vel[k, b]), ref_vels[b][k]) <= TOL_CHUNK
-    assert rel_err(host(chunk), ref_chunks) <= TOL_CHUNK
+            check_fp(host(vel[k, b]), ref_vels[b][k], TOL_CHUNK, f"velocity step {k}")
+    check_fp(host(chunk), ref_chunks, TOL_CHUNK, "chunk")
 
 
 def test_tiny_graph_replay_matches_direct(tiny):
@@ -180,7 +187,7 @@ def test_tiny_graph_replay_matches_direct(tiny):
     d, w, eng = tiny
     emb, noise = I.prefix_embeddings(d, 1, 64), I.noise(d, 1)
     eng.prefill(to_dev_bf16(emb))
-    vel = torch.empty((4, 1, d.chunk, d.action_dim), device="cuda")
+    vel = torch.empty((4, 1, d.chunk, d.action_dim), device="cuda", dtype=torch.float32)
     direct = eng.denoise(to_dev_f32(noise), 4, velocities=vel).clone()
     g1 = eng.denoise(to_dev_f32(noise), 4).clone()
     g2 = eng.denoise(to_dev_f32(noise), 4).clone()
@@ -268,7 +275,7 @@ def test_denoise_b1_over_random_prefix_cache(dm0):
         vs.append(v[0].astype(np.float64))
     eng.kv_commit(B, P)
     noise = I.noise(d, B)
-    vel = torch.empty((steps, B, d.chunk, d.action_dim), device="cuda")
+    vel = torch.empty((steps, B, d.chunk, d.action_dim), device="cuda", dtype=torch.float32)
     chunk = eng.denoise(to_dev_f32(noise), steps, velocities=vel)
     graphed = eng.denoise(to_dev_f32(noise), steps)
     eng.sync()
@@ -289,8 +296,9 @@ def test_e2e_b1(dm0):
     ks, vs, _ = O.prefill(w, emb[0])
     kc, vc = _kv_planes(eng, d, 1, 816)
     for l in (0, 13, 27):
-        assert rel_err(host(kc[l, 0]), ks[l]) <= TOL_LAYER
-        assert rel_err(host(vc[l, 0]), vs[l]) <= TOL_LAYER
+        a, r = (1e-2, 5e-3) if l == 0 else (2e-2, 1e-2)
+        check_bf16(host(kc[l, 0]), ks[l], a, f"K layer {l}", r)
+        check_bf16(host(vc[l, 0]), vs[l], a, f"V layer {l}", r)
     ref, _ = O.denoise(w, ks, vs, noise[0], 10)
     assert rel_err(host(chunk[0]), ref) <= TOL_CHUNK
 

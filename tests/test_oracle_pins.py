@@ -15,7 +15,14 @@ import torch.nn.functional as Fnn
 from oracle import dm0_oracle as O
 from synth import inputs as I
 
-torch.set_default_dtype(torch.float64)
+@pytest.fixture(autouse=True)
+def _fp64_default():
+    """Library references in this module run in fp64; restore the default afterwards so that
+    tests collected in the same session keep torch's fp32 default."""
+    old = torch.get_default_dtype()
+    torch.set_default_dtype(torch.float64)
+    yield
+    torch.set_default_dtype(old)
 
 
 def _rms(x):

@@ -16,6 +16,9 @@ from ._abi import (EXPORTS, LIB_PATH, Dm0Config, Dm0Error, load_library, make_co
 __all__ = ["Engine", "Dm0Error", "pack_weights", "load_library", "EXPORTS", "LIB_PATH"]
 
 
+c_int_t = ctypes.c_int
+
+
 def _ptr(t) -> int:
     return 0 if t is None else t.data_ptr()
 
@@ -94,6 +97,9 @@ class Engine:
         _check_cuda(noise, torch.float32, noise.shape, "noise")
         if actions is None:
             actions = torch.empty_like(noise)
+        _check_cuda(actions, torch.float32, noise.shape, "actions")
+        if velocities is not None:
+            _check_cuda(velocities, torch.float32, (steps,) + tuple(noise.shape), "velocities")
         self._chk(self.lib.dm0_denoise(self.h, _ptr(noise), steps, _ptr(actions), _ptr(velocities),
                                        _stream(stream)))
         return actions
@@ -110,21 +116,54 @@ class Engine:
         return actions
 
     def merged_layer(self, layer, h_prefix, h_suffix, out_prefix, out_suffix, k_out, v_out, stream=None):
+        import torch
+        d = self.dims
         B, P = h_prefix.shape[:2]
+        _check_cuda(h_prefix, torch.float32, (B, P, d.hidden_v), "h_prefix")
+        _check_cuda(h_suffix, torch.float32, (B, d.chunk, d.hidden_a), "h_suffix")
+        _check_cuda(out_prefix, torch.float32, (B, P, d.hidden_v), "out_prefix")
+        _check_cuda(out_suffix, torch.float32, (B, d.chunk, d.hidden_a), "out_suffix")
+        _check_cuda(k_out, torch.bfloat16, (B, d.n_kv, P, d.head_dim), "k_out")
+        _check_cuda(v_out, torch.bfloat16, (B, d.n_kv, P, d.head_dim), "v_out")
         self._chk(self.lib.dm0_merged_layer(self.h, layer, _ptr(h_prefix), _ptr(h_suffix), B, P, _ptr(out_prefix),
                                             _ptr(out_suffix), _ptr(k_out), _ptr(v_out), _stream(stream)))
 
     def op_gemm(self, A, B, C, swap=0, splits=1, stream=None):
+        import torch
         M, K = A.shape
         N = B.shape[0]
+        _check_cuda(A, torch.bfloat16, (M, K), "A")
+        _check_cuda(B, torch.bfloat16, (N, K), "B")
+        _check_cuda(C, torch.float32, (N, M) if swap else (M, N), "C")
         self._chk(self.lib.dm0_op_gemm(self.h, _ptr(A), _ptr(B), _ptr(C), M, N, K, swap, splits, _stream(stream)))
 
     def op_attention(self, q, ka, va, kb, vb, o, splits=1, stream=None):
+        import torch
+        for t, nm in ((q, "q"), (ka, "ka"), (va, "va"), (kb, "kb"), (vb, "vb"), (o, "o")):
+            if t is not None:
+                _check_cuda(t, torch.bfloat16, t.shape, nm)
         B, Tq = q.shape[:2]
         Ta = ka.shape[2]
         Tb = 0 if kb is None else kb.shape[2]
         self._chk(self.lib.dm0_op_attention(self.h, _ptr(q), _ptr(ka), _ptr(va), Ta, _ptr(kb), _ptr(vb), Tb,
                                             _ptr(o), B, Tq, splits, _stream(stream)))
+
+    def debug_view(self, name: str) -> int:
+        """Device address of an internal activation buffer (see dm0_debug_view)."""
+        p = ctypes.c_void_p()
+        self._chk(self.lib.dm0_debug_view(self.h, name.encode(), ctypes.byref(p)))
+        return p.value
+
+    def launch_count(self) -> int:
+        return int(self.lib.dm0_launch_count(self.h))
+
+    def probe(self, kind: int):
+        self._chk(self.lib.dm0_probe(self.h, kind))
+
+    def probe_read(self):
+        n, ms = c_int_t(), ctypes.c_double()
+        self._chk(self.lib.dm0_probe_read(self.h, ctypes.byref(n), ctypes.byref(ms)))
+        return n.value, ms.value
 
     def sync(self, stream=None):
         self._chk(self.lib.dm0_sync(self.h, _stream(stream)))

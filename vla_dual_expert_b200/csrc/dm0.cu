@@ -80,6 +80,11 @@ struct dm0_ctx {
   int device = 0;
   int num_sms = 148;
   bool use_pdl = true, use_graph = true;
+  // true when the previous operation this context queued on the stream was one of its own
+  // kernels: only then may the next kernel overlap it (programmatic dependent launch).  The first
+  // kernel of every API call follows foreign work (caller kernels, copies) and waits for it in
+  // plain stream order.
+  bool pdl_ok = false;
   std::string err;
 
   void* wbuf = nullptr;
@@ -114,7 +119,16 @@ struct dm0_ctx {
   bf16* stage_prefix = nullptr;
 
   cudaStream_t cap_stream = nullptr;
-  std::map<std::tuple<int, int, int>, cudaGraphExec_t> graphs;
+  struct Graph {
+    cudaGraphExec_t exec;
+    uint64_t kernels;
+  };
+  std::map<std::tuple<int, int, int>, Graph> graphs;
+  uint64_t launches = 0;   // kernels this context has put on a stream (graph replays count their kernels)
+  // event probe around the launches of one kernel site (dm0_probe)
+  int probe = 0;
+  std::vector<cudaEvent_t> probe_ev;
+  size_t probe_used = 0;
   std::map<TmapKey, CUtensorMap> tmaps;
   std::vector<void*> allocs;
 };
@@ -195,8 +209,25 @@ dm0_status launch(dm0_ctx* c, cudaStream_t s, void (*kernel)(KArgs...), dim3 gri
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = c->use_pdl ? 1 : 0;
+  cfg.numAttrs = (c->use_pdl && c->pdl_ok) ? 1 : 0;
   CK(cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...));
+  c->pdl_ok = true;
+  ++c->launches;
+  return DM0_OK;
+}
+
+// CUDA-event pair around one launch of the probed kernel site
+dm0_status probe_mark(dm0_ctx* c, cudaStream_t s) {
+  if (c->probe_used >= c->probe_ev.size()) {
+    if (c->probe_ev.size() >= 8192) return DM0_OK;   // full: later launches are not timed
+    for (int i = 0; i < 256; ++i) {
+      cudaEvent_t e;
+      CK(cudaEventCreate(&e));
+      c->probe_ev.push_back(e);
+    }
+  }
+  CK(cudaEventRecord(c->probe_ev[c->probe_used++], s));
+  c->pdl_ok = false;   // the next kernel follows an event record, not one of our kernels
   return DM0_OK;
 }
 
@@ -327,6 +358,7 @@ dm0_status layer_qkv(dm0_ctx* c, cudaStream_t s, int br, int l, const bf16* xn, 
   const LayerW& w = c->lw[br][l];
   const int H = hidden_of(c->cfg, br);
   GemmArgs g = base_args(c);
+  g.w_stable = 1;
   g.mode = dm0::kModeQKV;
   g.ssq_in = ssq_in;
   g.inv_hidden = 1.0f / H;
@@ -348,6 +380,7 @@ dm0_status layer_rest(dm0_ctx* c, cudaStream_t s, int br, int l, int tokens, flo
   const LayerW& w = c->lw[br][l];
   const int H = hidden_of(cf, br), I = inter_of(cf, br);
   GemmArgs g = base_args(c);
+  g.w_stable = 1;
   g.mode = dm0::kModeResid;
   g.h = h;
   g.H = H;
@@ -356,13 +389,18 @@ dm0_status layer_rest(dm0_ctx* c, cudaStream_t s, int br, int l, int tokens, flo
   g.ssq_out = ssq_mlp;
   TRY(run_gemm(c, s, o, tokens, cf.n_q * cf.head_dim, w.wo, H, g));
   GemmArgs u = base_args(c);
+  u.w_stable = 1;
   u.mode = dm0::kModeSwiGLU;
   u.ssq_in = ssq_mlp;
   u.inv_hidden = 1.0f / H;
   u.act = act;
   u.inter = I;
+  const bool probed = c->probe == 1 && br == 0;
+  if (probed) TRY(probe_mark(c, s));
   TRY(run_gemm(c, s, xn, tokens, H, w.wgu, 2 * I, u));
+  if (probed) TRY(probe_mark(c, s));
   GemmArgs d = base_args(c);
+  d.w_stable = 1;
   d.mode = dm0::kModeResid;
   d.h = h;
   d.H = H;
@@ -374,6 +412,7 @@ dm0_status layer_rest(dm0_ctx* c, cudaStream_t s, int br, int l, int tokens, flo
 
 dm0_status enqueue_prefill(dm0_ctx* c, cudaStream_t s, const void* prefix_emb, int B, int P) {
   const dm0_config& cf = c->cfg;
+  c->pdl_ok = false;
   const int M = B * P, L = cf.layers, D = cf.head_dim;
   const size_t lstride = static_cast<size_t>(B) * cf.n_kv * P * D;
   TRY(rows_prep(c, s, prefix_emb, 1, c->h_v, c->xn_v, c->lw[0][0].attn_norm, c->ssq_v, 2 * L, M, cf.hidden_v));
@@ -419,6 +458,7 @@ dm0_status step(dm0_ctx* c, cudaStream_t s, int B, int k_out, int k_in, int step
 // Euler loop over the KV cache; x already holds x_1
 dm0_status enqueue_denoise(dm0_ctx* c, cudaStream_t s, int steps, float* vel) {
   const dm0_config& cf = c->cfg;
+  c->pdl_ok = false;
   const int B = c->kv_B, P = c->kv_P, S = cf.chunk, L = cf.layers, D = cf.head_dim;
   const int Ms = B * S;
   const size_t lstride = static_cast<size_t>(B) * cf.n_kv * P * D;
@@ -446,7 +486,10 @@ dm0_status denoise_from_x(dm0_ctx* c, cudaStream_t s, int steps, float* vel) {
   auto it = c->graphs.find(key);
   if (it == c->graphs.end()) {
     CK(cudaStreamBeginCapture(c->cap_stream, cudaStreamCaptureModeThreadLocal));
+    const uint64_t l0 = c->launches;
     dm0_status st = enqueue_denoise(c, c->cap_stream, steps, nullptr);
+    const uint64_t nk = c->launches - l0;
+    c->launches = l0;
     cudaGraph_t graph = nullptr;
     cudaError_t e = cudaStreamEndCapture(c->cap_stream, &graph);
     if (st != DM0_OK) {
@@ -458,9 +501,10 @@ dm0_status denoise_from_x(dm0_ctx* c, cudaStream_t s, int steps, float* vel) {
     e = cudaGraphInstantiate(&exec, graph, 0);
     cudaGraphDestroy(graph);
     if (e != cudaSuccess) return fail(c, DM0_ECUDA, std::string("graph instantiate: ") + cudaGetErrorString(e));
-    it = c->graphs.emplace(key, exec).first;
+    it = c->graphs.emplace(key, dm0_ctx::Graph{exec, nk}).first;
   }
-  CK(cudaGraphLaunch(it->second, s));
+  CK(cudaGraphLaunch(it->second.exec, s));
+  c->launches += it->second.kernels;
   return DM0_OK;
 }
 
@@ -751,6 +795,7 @@ dm0_status dm0_merged_layer(dm0_ctx* c, int layer, const float* h_prefix, const 
   const int Mp = B * P, S = g.chunk, Ms = B * S;
   bf16* kp = static_cast<bf16*>(k_out);
   bf16* vp = static_cast<bf16*>(v_out);
+  c->pdl_ok = false;
   TRY(rows_prep(c, s, h_prefix, 0, c->h_v, c->xn_v, c->lw[0][layer].attn_norm, c->ssq_v, 2, Mp, g.hidden_v));
   TRY(rows_prep(c, s, h_suffix, 0, c->h_a, c->xn_a, c->lw[1][layer].attn_norm, c->ssq_a, 2, Ms, g.hidden_a));
   TRY(layer_qkv(c, s, 0, layer, c->xn_v, c->ssq_v, Mp, P, 0, c->q_v, kp, vp));
@@ -770,6 +815,7 @@ dm0_status dm0_op_gemm(dm0_ctx* c, const void* A, const void* B, float* C, int M
   if (!c || !A || !B || !C) return fail(c, DM0_EINVAL, "null argument");
   if (M < 1 || N < 1 || K < 64 || K % 64 != 0 || splits < 1) return fail(c, DM0_ESHAPE, "bad GEMM shape");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  c->pdl_ok = false;
   GemmArgs g = base_args(c);
   g.mode = dm0::kModeStoreF32;
   if (swap) {
@@ -790,9 +836,48 @@ dm0_status dm0_op_attention(dm0_ctx* c, const void* q, const void* ka, const voi
   const int G = c->cfg.n_q / c->cfg.n_kv;
   if (splits > 1 && B * c->cfg.n_kv * ((G * Tq + 127) / 128) > c->acount_n)
     return fail(c, DM0_ESHAPE, "too many row tiles for a split launch");
+  c->pdl_ok = false;
   return run_attn(c, static_cast<cudaStream_t>(stream), static_cast<const bf16*>(q), Tq, static_cast<const bf16*>(ka),
                   static_cast<const bf16*>(va), Ta, static_cast<const bf16*>(kb), static_cast<const bf16*>(vb), Tb,
                   static_cast<bf16*>(o), B, splits, 0);
+}
+
+dm0_status dm0_debug_view(dm0_ctx* c, const char* name, void** ptr) {
+  if (!c || !name || !ptr) return fail(c, DM0_EINVAL, "null argument");
+  const std::map<std::string, void*> bufs = {
+      {"h_v", c->h_v},     {"xn_v", c->xn_v},   {"q_v", c->q_v},     {"o_v", c->o_v},     {"act_v", c->act_v},
+      {"ssq_v", c->ssq_v}, {"h_a", c->h_a},     {"xn_a", c->xn_a},   {"q_a", c->q_a},     {"o_a", c->o_a},
+      {"act_a", c->act_a}, {"ssq_a", c->ssq_a}, {"x", c->x},         {"k_s", c->k_s},     {"v_s", c->v_s}};
+  auto it = bufs.find(name);
+  if (it == bufs.end()) return fail(c, DM0_EINVAL, std::string("unknown buffer ") + name);
+  *ptr = it->second;
+  return DM0_OK;
+}
+
+uint64_t dm0_launch_count(const dm0_ctx* c) { return c ? c->launches : 0; }
+
+dm0_status dm0_probe(dm0_ctx* c, int kind) {
+  if (!c) return DM0_EINVAL;
+  if (kind < 0 || kind > 1) return fail(c, DM0_EINVAL, "unknown probe kind");
+  c->probe = kind;
+  c->probe_used = 0;
+  return DM0_OK;
+}
+
+dm0_status dm0_probe_read(dm0_ctx* c, int* launches, double* total_ms) {
+  if (!c || !launches || !total_ms) return fail(c, DM0_EINVAL, "null argument");
+  double tot = 0.0;
+  const size_t pairs = c->probe_used / 2;
+  for (size_t i = 0; i < pairs; ++i) {
+    CK(cudaEventSynchronize(c->probe_ev[2 * i + 1]));
+    float ms = 0.f;
+    CK(cudaEventElapsedTime(&ms, c->probe_ev[2 * i], c->probe_ev[2 * i + 1]));
+    tot += ms;
+  }
+  *launches = static_cast<int>(pairs);
+  *total_ms = tot;
+  c->probe_used = 0;
+  return DM0_OK;
 }
 
 dm0_status dm0_sync(dm0_ctx* c, void* stream) {
@@ -829,7 +914,8 @@ const char* dm0_last_error(const dm0_ctx* c) {
 
 void dm0_destroy(dm0_ctx* c) {
   if (!c) return;
-  for (auto& kv : c->graphs) cudaGraphExecDestroy(kv.second);
+  for (auto& kv : c->graphs) cudaGraphExecDestroy(kv.second.exec);
+  for (cudaEvent_t e : c->probe_ev) cudaEventDestroy(e);
   if (c->cap_stream) cudaStreamDestroy(c->cap_stream);
   for (void* p : c->allocs) cudaFree(p);
   delete c;

@@ -36,6 +36,7 @@ struct GemmArgs {
   int swap;
   int mode;
   int tokens;         // valid activation rows
+  int w_stable;       // weight operand was written before the previous kernel: fetch it before the PDL wait
   int* err;           // device error word
   // input row scale: inv_rms(token) = rsqrt(ssq_in[token] * inv_hidden + eps); null -> 1
   const float* ssq_in;
@@ -259,12 +260,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       auto wdst = [&](int s) { return smem + s * L::kStage + (a.swap ? 0 : L::kA); };
       auto xdst = [&](int s) { return smem + s * L::kStage + (a.swap ? L::kA : 0); };
       const int pre = nkb < STAGES ? nkb : STAGES;
-      // weights do not depend on the previous kernel: request them first
+      // model weights do not depend on the previous kernel: request them before the dependency wait
+      if (!a.w_stable) pdl_wait();
       for (int i = 0; i < pre; ++i) {
         mbar_arrive_expect_tx(&full[i], L::kStage);
         tma_load_2d(wdst(i), wmap, &full[i], (kb0 + i) * 64, wrow, pol_w);
       }
-      pdl_wait();
+      if (a.w_stable) pdl_wait();
       for (int i = 0; i < pre; ++i) tma_load_2d(xdst(i), xmap, &full[i], (kb0 + i) * 64, xrow, pol_x);
       int last_issued = pre - 1;
       for (int i = pre; i < nkb; ++i) {
