@@ -224,7 +224,8 @@ def run_native(args, rank, world, local_rank):
 
     # probe kind 1 = the VLM gate/up GEMM of the prefix pass (the largest launch of the step)
     main = measure(wl_main, args.steps, args.warmup, probe=1)
-    e2e = measure_e2e(wl_main, max(2, args.steps // 2), 1)
+    e2e = measure_e2e(wl_main, max(2, args.steps // 2), 1) if not args.skip_e2e else {"ms": float("nan"), "h2d": 0,
+                                                                                        "d2h": 0}
     B, P = wl_main.batch, wl_main.prefix
     value = world * B * 1000.0 / main["ms"]
     gu_ms = main["probe_ms"] / max(main["probe_n"], 1)
@@ -356,6 +357,7 @@ def main():
     ap.add_argument("--workload", default="e2e_b16", choices=("e2e_b16", "e2e_b1"))
     ap.add_argument("--skip-batch1", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "native":

@@ -7,7 +7,9 @@ Tolerances, as max |gpu - oracle| / RMS(oracle) unless stated:
   bf16-stored tensors    |d_i| <= a * RMS + 2^-8 |ref_i| and RMS(d) <= r * RMS: the 2^-8 term is
                          the rounding of the stored bf16 value itself (2^-9, doubled).
                            K/V cache of one layer        a = 1e-2, r = 5e-3
-                           K/V after several layers      a = 2e-2, r = 1e-2
+                           K/V of layer l of a prefill   a = 1.2e-2 sqrt(l+1), r = 2.5e-3 sqrt(l+1):
+                                                         independent bf16 roundings of each layer's
+                                                         GEMM inputs add up as a random walk
                            attention output              a = 2e-2, r = 5e-3 (P is also rounded
                                                          to bf16 before PV)
 """
@@ -154,6 +156,12 @@ def test_tiny_merged_layer(tiny, B, P):
     _check_merged_layer(d, w, eng, 1, B, P, seed=30)
 
 
+def _depth_tol(layer):
+    """(atol, rms) tolerance of the bf16 K/V of prefill layer `layer` (see the module docstring)."""
+    f = float(np.sqrt(layer + 1))
+    return 1.2e-2 * f, 2.5e-3 * f
+
+
 def _kv_planes(eng, d, B, P):
     kp, vp = eng.kv_view()
     n = d.layers * B * d.n_kv * P * d.head_dim
@@ -174,7 +182,7 @@ def test_tiny_prefill_and_denoise(tiny, B, P, steps):
     ref_chunks, caches, ref_vels = O.infer(w, emb, noise, steps)
     for b in range(B):
         for l in range(d.layers):
-            a, r = (1e-2, 5e-3) if l == 0 else (2e-2, 1e-2)
+            a, r = _depth_tol(l)
             check_bf16(host(kc[l, b]), caches[b][0][l], a, f"K layer {l}", r)
             check_bf16(host(vc[l, b]), caches[b][1][l], a, f"V layer {l}", r)
         for k in range(steps):
@@ -296,7 +304,7 @@ def test_e2e_b1(dm0):
     ks, vs, _ = O.prefill(w, emb[0])
     kc, vc = _kv_planes(eng, d, 1, 816)
     for l in (0, 13, 27):
-        a, r = (1e-2, 5e-3) if l == 0 else (2e-2, 1e-2)
+        a, r = _depth_tol(l)
         check_bf16(host(kc[l, 0]), ks[l], a, f"K layer {l}", r)
         check_bf16(host(vc[l, 0]), vs[l], a, f"V layer {l}", r)
     ref, _ = O.denoise(w, ks, vs, noise[0], 10)
