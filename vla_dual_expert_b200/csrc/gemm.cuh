@@ -70,7 +70,6 @@ struct GemmArgs {
 };
 
 constexpr int kGemmThreads = 192;
-constexpr int kTileLd = 129;   // padded row stride (floats) of the smem staging tile
 
 template <int BN, int STAGES>
 struct GemmSmem {
@@ -78,136 +77,187 @@ struct GemmSmem {
   static constexpr uint32_t kB = BN * 128;
   static constexpr uint32_t kStage = kA + kB;
   static constexpr uint32_t kPipe = STAGES * kStage;
-  static constexpr uint32_t kTile = 128 * kTileLd * 4;
-  static_assert(kPipe >= kTile, "staging tile must fit in the pipeline buffers");
   static constexpr uint32_t kBytes = kPipe + 256 + 1024;   // + barriers + alignment slack
   static constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
 };
 
-// ---------------------------------------------------------------- epilogue on one 128-column group
+// ---------------------------------------------------------------- epilogue of one accumulator row
 //
-// Rows are tokens, the 128 columns are output features [col0, col0 + 128).
-// Warp `wid` (0..3) handles rows wid, wid + 4, ...; lane L holds columns
-// L + 32 i, i = 0..3.  `src` is either the smem staging tile (normal) or the
-// global split-K target (swap, read through L2).
-template <bool kGlobal>
-__device__ __forceinline__ void finalize_group(const GemmArgs& a, float* src, int ld, int tok0, int nrows, int col0,
-                                               int wid, int lane) {
+// One thread owns one output row (a token) and walks one 128-column group of
+// output features [col0, col0 + 128) in four 32-column chunks.  `load(c, v)`
+// delivers the raw accumulator of chunk c: straight from TMEM (normal
+// orientation: TMEM lane = token) or from the split-K scratch in L2 (swapped
+// orientation, last CTA of a feature tile).  Every reduction the fused
+// operations need (the head's RMSNorm, the sum of squares of the residual) is
+// local to the thread, RoPE partners (d, d + D/2) sit in the same thread, and
+// all loads and stores of a tile are in flight together.
+//
+// The TMEM loader is warp-collective: it is called for every row, valid or
+// not; stores are predicated on `valid`.
+
+__device__ __forceinline__ void st_f32x32(float* dst, const float (&v)[32]) {
+  float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+}
+__device__ __forceinline__ void ld_f32x32(const float* src, float (&v)[32]) {
+  const float4* s4 = reinterpret_cast<const float4*>(src);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 t = __ldcg(s4 + i);
+    v[4 * i] = t.x;
+    v[4 * i + 1] = t.y;
+    v[4 * i + 2] = t.z;
+    v[4 * i + 3] = t.w;
+  }
+}
+__device__ __forceinline__ uint32_t bf2(float lo, float hi) {
+  __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&b);
+}
+// 32 consecutive bf16 (64 bytes, 16-byte aligned)
+__device__ __forceinline__ void st_bf16x32(__nv_bfloat16* dst, const float (&v)[32]) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    d4[i] = make_uint4(bf2(v[8 * i], v[8 * i + 1]), bf2(v[8 * i + 2], v[8 * i + 3]), bf2(v[8 * i + 4], v[8 * i + 5]),
+                       bf2(v[8 * i + 6], v[8 * i + 7]));
+}
+
+template <bool kFromScratch, class Load>
+__device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool valid, int col0, float& ssq_acc,
+                                             Load&& load) {
   const int D = a.head_dim;
-  for (int r = wid; r < nrows; r += 4) {
-    const int tok = tok0 + r;
-    float x[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float* p = src + static_cast<size_t>(r) * ld + lane + 32 * i;
-      x[i] = kGlobal ? __ldcg(p) : *p;
+  if (a.mode == kModeStoreF32) {
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      float v[32];
+      load(c, v);
+      if (valid) st_f32x32(a.out_f32 + static_cast<size_t>(tok) * a.N + col0 + 32 * c, v);
     }
-    if (a.mode == kModeResid) {
-      float sq = 0.f;
+    return;
+  }
+  if (a.mode == kModeResid) {
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      float v[32];
+      load(c, v);
+      if (!valid) continue;
+      float* hp = a.h + static_cast<size_t>(tok) * a.H + col0 + 32 * c;
+      if (!kFromScratch) {   // normal orientation: add into the residual stream here
+        float hv[32];
+        ld_f32x32(hp, hv);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int col = col0 + lane + 32 * i;
-        float* hp = a.h + static_cast<size_t>(tok) * a.H + col;
-        float hv = x[i];
-        if (!kGlobal) {
-          hv += *hp;
-          *hp = hv;
+        for (int j = 0; j < 32; ++j) v[j] += hv[j];
+        st_f32x32(hp, v);
+      }
+      if (a.xn) {
+        float g[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          g[j] = a.gain_next[col0 + 32 * c + j] * v[j];
+          ssq_acc += v[j] * v[j];
         }
-        sq += hv * hv;
-        if (a.xn) a.xn[static_cast<size_t>(tok) * a.H + col] = __float2bfloat16_rn(a.gain_next[col] * hv);
+        st_bf16x32(a.xn + static_cast<size_t>(tok) * a.H + col0 + 32 * c, g);
       }
-      if (a.ssq_out) {
-        sq = warp_sum(sq);
-        if (lane == 0) atomicAdd(a.ssq_out + tok, sq);
+    }
+    return;
+  }
+  // QKV and SwiGLU consume the pending RMSNorm's 1/rms of this token
+  const float s = (a.ssq_in && valid) ? rsqrtf(__ldcg(a.ssq_in + tok) * a.inv_hidden + a.eps) : 1.f;
+  if (a.mode == kModeSwiGLU) {
+    // group = [64 gate rows | 64 up rows] of outputs [col0/2, col0/2 + 64)
+#pragma unroll 1
+    for (int c = 0; c < 2; ++c) {
+      float g[32], u[32];
+      load(c, g);
+      load(c + 2, u);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) g[j] = silu_f(g[j] * s) * (u[j] * s);
+      if (valid) st_bf16x32(a.act + static_cast<size_t>(tok) * a.inter + col0 / 2 + 32 * c, g);
+    }
+    return;
+  }
+  // kModeQKV: a 32-column chunk never straddles a head or a q/k/v section (D >= 32)
+  const int qdim = a.n_q * D, kvdim = a.n_kv * D;
+  const int b = tok / a.seq_len, p = tok - b * a.seq_len;
+  const int pos = a.pos_offset + p;
+  const int half = D >> 1;
+  const float2* cs_row = a.rope + static_cast<size_t>(pos) * half;
+  auto dst_of = [&](int col) -> __nv_bfloat16* {
+    if (col < qdim) return a.q_out + static_cast<size_t>(tok) * qdim + col;
+    const int sec = col < qdim + kvdim ? 1 : 2;
+    const int c2 = col - qdim - (sec == 2 ? kvdim : 0);
+    const int kvh = c2 / D, d = c2 - kvh * D;
+    __nv_bfloat16* base = sec == 1 ? a.k_out : a.v_out;
+    return base + ((static_cast<size_t>(b) * a.n_kv + kvh) * a.kv_seq + p) * D + d;
+  };
+  const int cph = D >> 5;   // 32-column chunks per head
+#pragma unroll 1
+  for (int h0 = 0; h0 < 4; h0 += cph) {
+    const int colh = col0 + 32 * h0;
+    const bool is_v = colh >= qdim + kvdim;
+    if (is_v) {
+#pragma unroll 1
+      for (int c = h0; c < h0 + cph; ++c) {
+        float v[32];
+        load(c, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] *= s;
+        if (valid) st_bf16x32(dst_of(col0 + 32 * c), v);
       }
       continue;
     }
-    if (a.mode == kModeStoreF32) {
-      if (!kGlobal) {
+    const float* gain = colh < qdim ? a.q_gain : a.k_gain;
+    // pass 1: RMS of the head
+    float ss = 0.f;
+#pragma unroll 1
+    for (int c = h0; c < h0 + cph; ++c) {
+      float v[32];
+      load(c, v);
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          a.out_f32[static_cast<size_t>(tok) * a.N + col0 + lane + 32 * i] = x[i];
+      for (int j = 0; j < 32; ++j) ss += v[j] * v[j];
+    }
+    const float rn = s * rsqrtf(ss * s * s / D + a.eps);
+    if (D == 32) {
+      // one chunk, pairs (j, j + 16)
+      float v[32];
+      load(h0, v);
+      float o[32];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float x0 = v[j] * rn * gain[j], x1 = v[j + 16] * rn * gain[j + 16];
+        const float2 cs = cs_row[j];
+        o[j] = x0 * cs.x - x1 * cs.y;
+        o[j + 16] = x1 * cs.x + x0 * cs.y;
       }
-      continue;
-    }
-    // QKV and SwiGLU consume the pending RMSNorm's 1/rms of this token
-    float s = 1.f;
-    if (a.ssq_in) s = rsqrtf(__ldcg(a.ssq_in + tok) * a.inv_hidden + a.eps);
+      if (valid) st_bf16x32(dst_of(colh), o);
+    } else {
+      // chunk c (head dims 32c'..) pairs with chunk c + cph/2
+#pragma unroll 1
+      for (int c = 0; c < cph / 2; ++c) {
+        float lo[32], hi[32];
+        load(h0 + c, lo);
+        load(h0 + c + cph / 2, hi);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) x[i] *= s;
-    if (kGlobal) {   // leave the split-K target zeroed for the next launch
-#pragma unroll
-      for (int i = 0; i < 4; ++i) src[static_cast<size_t>(r) * ld + lane + 32 * i] = 0.f;
-    }
-    if (a.mode == kModeSwiGLU) {
-      // group = [64 gate rows | 64 up rows] of outputs [col0/2, col0/2 + 64)
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int j = col0 / 2 + lane + 32 * i;
-        a.act[static_cast<size_t>(tok) * a.inter + j] = __float2bfloat16_rn(silu_f(x[i]) * x[i + 2]);
-      }
-      continue;
-    }
-    // kModeQKV: 32-column chunks never straddle a head or a q/k/v section (D >= 32)
-    const int qdim = a.n_q * D, kvdim = a.n_kv * D;
-    float sq[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) sq[i] = warp_sum(x[i] * x[i]);
-    const int b = tok / a.seq_len, p = tok - b * a.seq_len;
-    const int pos = a.pos_offset + p;
-    const int half = D >> 1;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int col = col0 + 32 * i + lane;
-      const int sec = col < qdim ? 0 : (col < qdim + kvdim ? 1 : 2);
-      const int d = col % D;
-      float y = x[i];
-      if (sec < 2) {
-        // RMSNorm over this head's D columns: chunks i' with the same head as chunk i
-        float ss = 0.f;
-        const int chunks = D >> 5;             // 32-col chunks per head
-        const int first = (i / chunks) * chunks;
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (j >= first && j < first + chunks) ss += sq[j];
-        const float* g = sec == 0 ? a.q_gain : a.k_gain;
-        y = y * rsqrtf(ss / D + a.eps) * g[d];
-      }
-      x[i] = y;   // normalised, before rotation
-    }
-    // RoPE (rotate-half): partner of column d is d +- D/2
-    float part[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if (D == 128) part[i] = x[i ^ 2];
-      else if (D == 64) part[i] = x[i ^ 1];
-      else part[i] = __shfl_xor_sync(0xffffffffu, x[i], 16);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int col = col0 + 32 * i + lane;
-      const int sec = col < qdim ? 0 : (col < qdim + kvdim ? 1 : 2);
-      const int d = col % D;
-      float y = x[i];
-      if (sec < 2) {
-        const float2 cs = a.rope[static_cast<size_t>(pos) * half + (d % half)];
-        y = d < half ? (y * cs.x - part[i] * cs.y) : (y * cs.x + part[i] * cs.y);
-      }
-      const __nv_bfloat16 o = __float2bfloat16_rn(y);
-      if (sec == 0) {
-        a.q_out[static_cast<size_t>(tok) * qdim + col] = o;
-      } else {
-        const int c2 = col - qdim - (sec == 2 ? kvdim : 0);
-        const int kvh = c2 / D;
-        __nv_bfloat16* dst = sec == 1 ? a.k_out : a.v_out;
-        dst[((static_cast<size_t>(b) * a.n_kv + kvh) * a.kv_seq + p) * D + d] = o;
+        for (int j = 0; j < 32; ++j) {
+          const int d = 32 * c + j;
+          const float x0 = lo[j] * rn * gain[d], x1 = hi[j] * rn * gain[d + half];
+          const float2 cs = cs_row[d];
+          lo[j] = x0 * cs.x - x1 * cs.y;
+          hi[j] = x1 * cs.x + x0 * cs.y;
+        }
+        if (valid) {
+          st_bf16x32(dst_of(colh + 32 * c), lo);
+          st_bf16x32(dst_of(colh + 32 * c + half), hi);
+        }
       }
     }
   }
 }
 
 template <int BN, int STAGES>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kGemmThreads, 2)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmArgs a) {
   using L = GemmSmem<BN, STAGES>;
@@ -330,24 +380,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const bool go = *abort_flag == 0;
     if (go) {
       tc_fence_after();
+      const uint32_t tl = tmem + (static_cast<uint32_t>(lane_base) << 16);
       if (!a.swap) {
-        float* tile = reinterpret_cast<float*>(smem);
-        const int nrows = min(128, a.M - m_tile * 128);
+        // TMEM lane = token row of this tile
+        const int tok = m_tile * 128 + lane_base + lane;
+        const bool valid = tok < a.M;
+        float ssq_acc = 0.f;
         for (int g = 0; g < BN / 128; ++g) {
-          const int row = lane_base + lane;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            float v[32];
-            tmem_ld32(tmem + (static_cast<uint32_t>(lane_base) << 16) + g * 128 + c * 32, v);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) tile[row * kTileLd + c * 32 + j] = v[j];
-          }
-          named_bar_sync(1, 128);
-          finalize_group<false>(a, tile, kTileLd, m_tile * 128, nrows, n_tile * BN + g * 128, wid, lane);
-          named_bar_sync(1, 128);
+          const uint32_t tg = tl + g * 128;
+          row_epilogue<false>(a, tok, valid, n_tile * BN + g * 128, ssq_acc,
+                              [&](int c, float (&v)[32]) { tmem_ld32(tg + c * 32, v); });
         }
+        if (a.mode == kModeResid && a.ssq_out && valid) atomicAdd(a.ssq_out + tok, ssq_acc);
       } else {
-        // lanes = output features, columns = tokens
+        // lanes = output features, columns = tokens: add this split's partial sums
         const int feat = m_tile * 128 + lane_base + lane;
         float* dst = a.mode == kModeResid ? a.h : a.acc;
         const int ld = a.mode == kModeResid ? a.H : a.ld_acc;
@@ -355,7 +401,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
         for (int c = 0; c < BN / 32; ++c) {
           float v[32];
-          tmem_ld32(tmem + (static_cast<uint32_t>(lane_base) << 16) + c * 32, v);
+          tmem_ld32(tl + c * 32, v);
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int tok = tokbase + c * 32 + j;
@@ -373,7 +419,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         named_bar_sync(1, 128);
         if (*last_flag && a.mode != kModeStoreF32) {
           __threadfence();
-          finalize_group<true>(a, dst + m_tile * 128, ld, 0, a.tokens, m_tile * 128, wid, lane);
+          // the last CTA of this feature tile: one thread per token
+          const int tok = wid * 32 + lane;
+          const bool valid = tok < a.tokens;
+          float* row = dst + static_cast<size_t>(valid ? tok : 0) * ld + m_tile * 128;
+          const bool zero_after = a.mode != kModeResid;
+          float ssq_acc = 0.f;
+          row_epilogue<true>(a, tok, valid, m_tile * 128, ssq_acc, [&](int c, float (&v)[32]) {
+            if (valid) {
+              ld_f32x32(row + 32 * c, v);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] = 0.f;
+            }
+          });
+          if (a.mode == kModeResid && a.ssq_out && valid) atomicAdd(a.ssq_out + tok, ssq_acc);
+          if (zero_after && valid) {   // leave the split-K scratch zeroed for the next launch
+            float4* r4 = reinterpret_cast<float4*>(row);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
         }
       }
     }
