@@ -187,6 +187,31 @@ dm0_status dm0_op_attention(dm0_ctx* ctx, const void* q, const void* ka, const v
  * meaningful after the call that fills them has completed. */
 dm0_status dm0_debug_view(dm0_ctx* ctx, const char* name, void** ptr);
 
+/* Merged GQA attention that allocates nothing, for callers that cannot call
+ * cudaMalloc: a real-time control loop that must not allocate once it runs,
+ * code that runs inside stream capture, or a host whose device memory is
+ * owned by another allocator.  It needs no dm0_ctx (creating one allocates).
+ * The pages have no counterpart: this is a deployment variant of
+ * dm0_op_attention.
+ *
+ * Same arguments, layouts and result as dm0_op_attention, with the head
+ * layout given explicitly (n_q, n_kv, head_dim in {32, 64, 128}).  When the
+ * keys are split (splits > 1, after clamping to the number of 64-key blocks),
+ * the partial softmax states go to a fixed device-side scratch area inside
+ * the library (about 2 MB, held by every GPU that loads the library until the
+ * process exits) of 32 slots: B * n_kv * ceil((n_q/n_kv) * Tq / 128) * splits
+ * must be <= 32, otherwise DM0_ESHAPE.  The caller passes inputs and outputs only.
+ *
+ * The first call on a device looks up the scratch's device address and sets
+ * the kernels' shared-memory limit; make that first call before any stream
+ * capture.  Every call shares the one scratch area and resets its counters
+ * on `stream`: calls that overlap on the GPU (different streams without
+ * ordering) race and give wrong results.  Asynchronous on `stream`; returns
+ * DM0_EINVAL / DM0_ESHAPE / DM0_ECUDA on bad arguments or launch failure. */
+dm0_status dm0_attention_noalloc(const void* q, const void* ka, const void* va, int Ta, const void* kb,
+                                 const void* vb, int Tb, void* o, int B, int Tq, int n_q, int n_kv, int head_dim,
+                                 int splits, void* stream);
+
 /* Instrumentation. ------------------------------------------------------- */
 
 /* Number of kernels this context has enqueued so far (a replayed graph counts

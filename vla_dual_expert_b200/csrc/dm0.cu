@@ -23,6 +23,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <map>
+#include <mutex>
 #include <string>
 #include <tuple>
 #include <vector>
@@ -541,6 +542,45 @@ size_t blob_bytes(const dm0_config& g) {
 
 }  // namespace
 
+// ====================================================================== allocation-free attention
+//
+// Scratch for dm0_attention_noalloc: the split-KV partial states and arrival
+// counters live in this file-scope device array instead of memory from
+// cudaMalloc.  Every GPU that loads the library holds it (about 2 MB) until the
+// process exits.  In host code the name is only a host-side stand-in; the
+// device address is fetched per device with cudaGetSymbolAddress.
+constexpr int kNoAllocSlots = 32;                               // (group x row tile x split) partial states
+constexpr int kNoAllocOFloats = kNoAllocSlots * 128 * 128;      // partial O, head_dim up to 128
+constexpr int kNoAllocMlFloats = kNoAllocSlots * 128 * 2;       // (m, l) per partial row
+constexpr int kNoAllocCounters = kNoAllocSlots;                 // one arrival counter per (group, row tile)
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocOFloats + kNoAllocMlFloats + kNoAllocCounters];
+
+namespace {
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+float* g_noalloc_base[kNoAllocMaxDevices] = {};
+
+// Once per device, with that device current: the array's device address and the
+// attention kernels' shared-memory limit.
+dm0_status noalloc_setup(int dev, float** base) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_base[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return DM0_ECUDA;
+    if (cudaFuncSetAttribute(dm0::attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             dm0::AttnSmem<128>::kBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(dm0::attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             dm0::AttnSmem<64>::kBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(dm0::attn_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             dm0::AttnSmem<32>::kBytes) != cudaSuccess)
+      return DM0_ECUDA;
+    g_noalloc_base[dev] = static_cast<float*>(p);
+  }
+  *base = g_noalloc_base[dev];
+  return DM0_OK;
+}
+}  // namespace
+
 // ====================================================================== C ABI
 
 extern "C" {
@@ -878,6 +918,64 @@ dm0_status dm0_probe_read(dm0_ctx* c, int* launches, double* total_ms) {
   *total_ms = tot;
   c->probe_used = 0;
   return DM0_OK;
+}
+
+dm0_status dm0_attention_noalloc(const void* q, const void* ka, const void* va, int Ta, const void* kb, const void* vb,
+                                 int Tb, void* o, int B, int Tq, int n_q, int n_kv, int head_dim, int splits,
+                                 void* stream) {
+  if (!q || !ka || !va || !o || (Tb > 0 && (!kb || !vb))) return DM0_EINVAL;
+  if (B < 1 || Tq < 1 || Ta < 1 || Tb < 0 || splits < 1 || n_q < 1 || n_kv < 1 || n_q % n_kv != 0)
+    return DM0_ESHAPE;
+  if (head_dim != 32 && head_dim != 64 && head_dim != 128) return DM0_ESHAPE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DM0_ECUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return DM0_ECUDA;
+  float* base = nullptr;
+  TRY(noalloc_setup(dev, &base));
+  const int G = n_q / n_kv;
+  const long long tiles = (static_cast<long long>(G) * Tq + 127) / 128;
+  const long long groups = static_cast<long long>(B) * n_kv;
+  const int nblk = (Ta + Tb + 63) / 64;
+  if (tiles > 65535 || groups > 65535) return DM0_ESHAPE;
+  if (splits > nblk) splits = nblk;
+  const int bps = (nblk + splits - 1) / splits;
+  splits = (nblk + bps - 1) / bps;
+  if (splits > 1 && groups * tiles * splits > kNoAllocSlots) return DM0_ESHAPE;   // beyond the static scratch
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* counters = reinterpret_cast<int*>(base + kNoAllocOFloats + kNoAllocMlFloats);
+  if (splits > 1 && cudaMemsetAsync(counters, 0, kNoAllocCounters * sizeof(int), s) != cudaSuccess)
+    return DM0_ECUDA;
+  AttnArgs a{};
+  a.q = static_cast<const bf16*>(q);
+  a.seq_q = Tq;
+  a.ka = static_cast<const bf16*>(ka);
+  a.va = static_cast<const bf16*>(va);
+  a.len_a = Ta;
+  a.kb = static_cast<const bf16*>(kb);
+  a.vb = static_cast<const bf16*>(vb);
+  a.len_b = Tb;
+  a.o = static_cast<bf16*>(o);
+  a.n_q = n_q;
+  a.n_kv = n_kv;
+  a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(head_dim)));
+  a.blocks_per_split = bps;
+  a.a_stable = 0;
+  a.part_o = base;
+  a.part_ml = reinterpret_cast<float2*>(base + kNoAllocOFloats);
+  a.counters = counters;
+  a.err = nullptr;
+  const dim3 grid(static_cast<unsigned>(tiles), static_cast<unsigned>(groups), splits);
+  switch (head_dim) {
+    case 128:
+      dm0::attn_kernel<128><<<grid, dm0::kAttnThreads, dm0::AttnSmem<128>::kBytes, s>>>(a);
+      break;
+    case 64:
+      dm0::attn_kernel<64><<<grid, dm0::kAttnThreads, dm0::AttnSmem<64>::kBytes, s>>>(a);
+      break;
+    default:
+      dm0::attn_kernel<32><<<grid, dm0::kAttnThreads, dm0::AttnSmem<32>::kBytes, s>>>(a);
+  }
+  return cudaGetLastError() == cudaSuccess ? DM0_OK : DM0_ECUDA;
 }
 
 dm0_status dm0_sync(dm0_ctx* c, void* stream) {
