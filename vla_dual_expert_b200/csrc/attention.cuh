@@ -72,9 +72,11 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+constexpr int kAttnStages = 3;   // K/V tiles in flight per CTA
+
 template <int D>
 struct AttnSmem {
-  static constexpr int kBytes = (128 + 4 * 64) * D * 2;   // Q tile + double-buffered K and V tiles
+  static constexpr int kBytes = (128 + 2 * kAttnStages * 64) * D * 2;   // Q tile + K/V ring
 };
 
 template <int D>
@@ -85,7 +87,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnArgs a) {
   extern __shared__ __align__(128) uint8_t attn_smem[];
   __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(attn_smem);
   __nv_bfloat16* sK = sQ + 128 * D;
-  __nv_bfloat16* sV = sK + 2 * 64 * D;
+  __nv_bfloat16* sV = sK + kAttnStages * 64 * D;
   __shared__ int s_last;
 
   const int tile = blockIdx.x, grp = blockIdx.y, split = blockIdx.z;
@@ -120,8 +122,12 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnArgs a) {
   };
 
   pdl_launch_dependents();
-  const bool pre = a.a_stable && (blk0 + 1) * 64 <= a.len_a && blk0 < blk1;
-  if (pre) load_kv(blk0, 0);
+  // prologue: blocks blk0 .. blk0 + kAttnStages - 2 and the Q tile.  Commit groups are kept uniform:
+  // group 0 = {block blk0 (+ any pre-issued blocks), Q}, then one group per further block.
+  constexpr int NPRE = kAttnStages - 1;
+  const bool pre = a.a_stable && (blk0 + NPRE) * 64 <= a.len_a && blk0 + NPRE <= blk1;
+  if (pre)
+    for (int i = 0; i < NPRE; ++i) load_kv(blk0 + i, i);   // the prefix cache predates the previous kernel
   pdl_wait();
   if (!pre && blk0 < blk1) load_kv(blk0, 0);
   for (int idx = tid; idx < 128 * CH; idx += kAttnThreads) {
@@ -136,6 +142,10 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnArgs a) {
     cp_async16(sQ + off(r, c), src, valid);
   }
   cp_async_commit();
+  for (int i = 1; i < NPRE; ++i) {
+    if (!pre && blk0 + i < blk1) load_kv(blk0 + i, i);
+    cp_async_commit();
+  }
 
   float m_r[2] = {kNegInf, kNegInf}, l_r[2] = {0.f, 0.f};
   float acc[D / 8][4];
@@ -145,17 +155,19 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnArgs a) {
   const int g = lane >> 2, t4 = lane & 3;
 
   for (int blk = blk0; blk < blk1; ++blk) {
-    const int buf = (blk - blk0) & 1;
-    cp_async_wait_all();
+    const int it = blk - blk0;
+    const int buf = it % kAttnStages;
+    asm volatile("cp.async.wait_group %0;" ::"n"(kAttnStages - 2) : "memory");
     __syncthreads();
-    if (blk == blk0) {
+    if (it == 0) {
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const int row = warp * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
         ldsm_x4(qf[kk], smem_u32(sQ + off(row, kk * 2 + (lane >> 4))));
       }
     }
-    if (blk + 1 < blk1) load_kv(blk + 1, buf ^ 1);
+    // refill the slot computed on in the previous iteration (every thread passed the barrier above)
+    if (blk + NPRE < blk1) load_kv(blk + NPRE, (it + NPRE) % kAttnStages);
     cp_async_commit();
 
     const __nv_bfloat16* Kb = sK + buf * 64 * D;
@@ -273,29 +285,50 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnArgs a) {
   __syncthreads();
   if (!s_last) return;
   __threadfence();
+  // combine: (m, l) of every (split, row) into shared memory in one coalesced pass, per-row
+  // weights w_s = 2^(m_s - M) / L once, then every output element reduced over the splits with
+  // independent loads spread over all threads
   const int nsplit = gridDim.z;
-  for (int row = warp; row < 128; row += kAttnThreads / 32) {
-    const int pr = tile * 128 + row;
-    if (pr >= rows_total) break;
+  float* sm_m = reinterpret_cast<float*>(attn_smem);   // [nsplit][128], reuses the Q/K/V area
+  float* sm_l = sm_m + nsplit * 128;
+  for (int i = tid; i < nsplit * 128; i += kAttnThreads) {
+    const float2 ml = __ldcg(&a.part_ml[slot0 * 128 + i]);
+    sm_m[i] = ml.x;
+    sm_l[i] = ml.y;
+  }
+  __syncthreads();
+  if (tid < 128) {
     float mmax = kNegInf;
-    for (int sp = 0; sp < nsplit; ++sp) mmax = fmaxf(mmax, __ldcg(&a.part_ml[(slot0 + sp) * 128 + row].x));
+    for (int sp = 0; sp < nsplit; ++sp) mmax = fmaxf(mmax, sm_m[sp * 128 + tid]);
     float lsum = 0.f;
-    float o[D / 32];
-#pragma unroll
-    for (int i = 0; i < D / 32; ++i) o[i] = 0.f;
     for (int sp = 0; sp < nsplit; ++sp) {
-      const float2 ml = __ldcg(&a.part_ml[(slot0 + sp) * 128 + row]);
-      const float w = exp2f(ml.x - mmax);
-      lsum += w * ml.y;
-      const float* po = a.part_o + ((slot0 + sp) * 128 + row) * D;
-#pragma unroll
-      for (int i = 0; i < D / 32; ++i) o[i] += w * __ldcg(po + lane + 32 * i);
+      const float w = exp2f(sm_m[sp * 128 + tid] - mmax);
+      sm_m[sp * 128 + tid] = w;
+      lsum += w * sm_l[sp * 128 + tid];
     }
-    const int head = kvh * G + pr / a.seq_q, pos = pr % a.seq_q;
-    __nv_bfloat16* dst = a.o + ((static_cast<size_t>(b) * a.seq_q + pos) * a.n_q + head) * D;
     const float inv = 1.f / lsum;
-#pragma unroll
-    for (int i = 0; i < D / 32; ++i) dst[lane + 32 * i] = __float2bfloat16_rn(o[i] * inv);
+    for (int sp = 0; sp < nsplit; ++sp) sm_m[sp * 128 + tid] *= inv;
+  }
+  __syncthreads();
+  const int rows_here = min(128, rows_total - tile * 128);
+  constexpr int Q4 = D / 4;
+  for (int item = tid; item < rows_here * Q4; item += kAttnThreads) {
+    const int row = item / Q4, d4 = item - row * Q4;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4* po = reinterpret_cast<const float4*>(a.part_o + (slot0 * 128 + row) * D) + d4;
+#pragma unroll 4
+    for (int sp = 0; sp < nsplit; ++sp) {
+      const float w = sm_m[sp * 128 + row];
+      const float4 t = __ldcg(po + static_cast<size_t>(sp) * 128 * Q4);
+      o.x += w * t.x;
+      o.y += w * t.y;
+      o.z += w * t.z;
+      o.w += w * t.w;
+    }
+    const int pr = tile * 128 + row;
+    const int head = kvh * G + pr / a.seq_q, pos = pr % a.seq_q;
+    __nv_bfloat16* dst = a.o + ((static_cast<size_t>(b) * a.seq_q + pos) * a.n_q + head) * D + 4 * d4;
+    *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16(o.x, o.y), pack_bf16(o.z, o.w));
   }
 }
 

@@ -1,0 +1,356 @@
+// Flash attention on tcgen05 for both attention shapes of the dual-expert layer
+// (DM0 architecture notes, section 1): prefix rows over the prefix keys, and
+// suffix rows over [prefix cache; suffix keys] (DM0.5 page, sections 5.1, 6.2).
+// Keys come from up to two segments (A, B), each a [B][n_kv][len][128] array;
+// every query row of a launch sees all keys of both.
+//
+// One CTA owns 128 query rows of one (sample, KV head) group; the G query heads
+// sharing the KV head are packed along the rows as in attn_kernel, so every K/V
+// tile serves all of them.  Per 128-key block j:
+//   S_j = Q K_j^T        tcgen05.mma (M 128, N 128 keys, K 128), fp32 in TMEM,
+//                        double-buffered so S_{j+1} overlaps the softmax of S_j
+//   P_j = 2^(s - m)      softmax warps, one thread per row, read S from TMEM and
+//                        write P (bf16) to shared memory as a K-major operand
+//   O  += P_j V_j        tcgen05.mma (M 128, N 128 dims, K 128 keys); V is read
+//                        in its stored [key][dim] order as an MN-major operand
+// The running max is only moved (and O, l rescaled in TMEM) when a row's max
+// grows by more than 2^8: p stays <= 256 in between and the final O / l uses a
+// consistent reference, so the result is exact up to rounding.
+//
+// Warp roles (192 threads): warp 0 TMA producer for K/V, warp 1 TMEM owner and
+// MMA issuer, warps 2..5 Q staging, softmax, O correction and output.
+#pragma once
+#include "attention.cuh"
+#include "ptx.cuh"
+
+namespace dm0 {
+
+constexpr int kFaThreads = 192;
+
+struct FaSmem {
+  static constexpr uint32_t kTile = 32768;                  // 128 rows x 128 bf16, two 64-column SW128 halves
+  static constexpr int kStages = 2;                         // K/V blocks in flight
+  static constexpr uint32_t kOffQ = 0;
+  static constexpr uint32_t kOffK = kOffQ + kTile;
+  static constexpr uint32_t kOffV = kOffK + kStages * kTile;
+  static constexpr uint32_t kOffP = kOffV + kStages * kTile;
+  static constexpr uint32_t kOffBar = kOffP + 2 * kTile;    // 229376
+  static constexpr uint32_t kBytes = kOffBar + 256 + 1024;
+};
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// MN-major operand, SWIZZLE_128B: 64 contiguous elements per 128-byte row, the
+// next 64 along MN `mn_stride` bytes further, 8-row groups along K 1024 bytes apart.
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_addr, uint32_t mn_stride) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((mn_stride >> 4) & 0x3FFFu) << 16;   // leading byte offset: next 64 along MN
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;                   // stride byte offset: next 8 rows along K
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
+// byte offset of element (row, col) of a 128 x 128 bf16 tile stored as two 64-column SW128 halves
+__device__ __forceinline__ uint32_t sw128_off(int row, int col) {
+  const int half = col >> 6, c16 = (col & 63) >> 3;
+  return half * 16384 + row * 128 + ((c16 ^ (row & 7)) << 4) + ((col & 7) << 1);
+}
+
+__global__ void __launch_bounds__(kFaThreads, 1)
+    fa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                 const __grid_constant__ CUtensorMap tmKb, const __grid_constant__ CUtensorMap tmVb, const AttnArgs a) {
+  constexpr int D = 128;
+  extern __shared__ uint8_t fa_smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fa_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + FaSmem::kOffBar);
+  uint64_t* kv_full = bars;        // [2] TMA landed K_j, V_j
+  uint64_t* kv_empty = bars + 2;   // [2] PV_j done: K/V slot free
+  uint64_t* s_full = bars + 4;     // [2] S_j in TMEM
+  uint64_t* s_free = bars + 6;     // [2] softmax finished reading S_j
+  uint64_t* p_full = bars + 8;     // P_j in smem and O corrected (one phase per block)
+  uint64_t* pv_done = bars + 9;    // PV_j finished (one phase per block)
+  uint64_t* q_ready = bars + 10;
+  uint64_t* drain = bars + 11;     // every issued MMA complete (before TMEM is released)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x, grp = blockIdx.y;
+  const int b = grp / a.n_kv, kvh = grp - b * a.n_kv;
+  const int G = a.n_q / a.n_kv;
+  const int rows_total = G * a.seq_q;
+  // 128-key blocks: segment A first, then segment B (a block never mixes segments)
+  const int nA = (a.len_a + 127) >> 7, nB = (a.len_b + 127) >> 7;
+  const int nblk = nA + nB;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 4);
+    }
+    mbar_init(p_full, 4);
+    mbar_init(pv_done, 1);
+    mbar_init(q_ready, 4);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;   // S_0 at column 0, S_1 at 128, O at 256
+  pdl_launch_dependents();
+
+  if (warp == 0) {
+    // ------------------------------------------------ K/V producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      if (nB) {
+        tma_prefetch_desc(&tmKb);
+        tma_prefetch_desc(&tmVb);
+      }
+      const uint64_t pol = policy_evict_last();
+      auto issue = [&](int j) {
+        const int s = j & 1;
+        const bool segA = j < nA;
+        const CUtensorMap* mk = segA ? &tmK : &tmKb;
+        const CUtensorMap* mv = segA ? &tmV : &tmVb;
+        const int row = segA ? grp * a.len_a + j * 128 : grp * a.len_b + (j - nA) * 128;
+        mbar_arrive_expect_tx(&kv_full[s], 2 * FaSmem::kTile);
+        uint8_t* kd = smem + FaSmem::kOffK + s * FaSmem::kTile;
+        uint8_t* vd = smem + FaSmem::kOffV + s * FaSmem::kTile;
+        tma_load_2d(kd, mk, &kv_full[s], 0, row, pol);
+        tma_load_2d(kd + 16384, mk, &kv_full[s], 64, row, pol);
+        tma_load_2d(vd, mv, &kv_full[s], 0, row, pol);
+        tma_load_2d(vd + 16384, mv, &kv_full[s], 64, row, pol);
+      };
+      // segment A written before the previous kernel (the prefix cache during the Euler loop) may be
+      // requested before the dependency wait
+      int issued = 0;
+      if (a.a_stable)
+        for (; issued < 2 && issued < nA; ++issued) issue(issued);
+      pdl_wait();
+      for (int j = issued; j < nblk; ++j) {
+        const int s = j & 1;
+        if (j >= 2 && !mbar_wait(&kv_empty[s], ((j >> 1) - 1) & 1, abort_flag)) {
+          *abort_flag = 1;
+          raise_error(a.err, kErrTimeoutProducer);
+          break;
+        }
+        issue(j);
+        issued = j + 1;
+      }
+      for (int j = issued - 2; j < issued; ++j) {   // copies in flight land before the CTA exits
+        if (j < 0) continue;
+        if (!mbar_wait(&kv_full[j & 1], (j >> 1) & 1, nullptr, kDrainTimeoutNs)) raise_error(a.err, kErrDrain);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16_f32(128, 128);
+      const uint32_t idesc_pv = idesc_bf16_f32(128, 128) | (1u << 16);   // B (V) is MN-major
+      const uint32_t qa = smem_u32(smem + FaSmem::kOffQ);
+      bool ok = mbar_wait(q_ready, 0, abort_flag);
+      auto pv = [&](int i) -> bool {
+        if (!mbar_wait(p_full, i & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t pa = smem_u32(smem + FaSmem::kOffP + (i & 1) * FaSmem::kTile);
+        const uint32_t vb = smem_u32(smem + FaSmem::kOffV + (i & 1) * FaSmem::kTile);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          umma_bf16(tmem + 256, sw128_kmajor_desc(pa + (ks >> 2) * 16384 + (ks & 3) * 32),
+                    sw128_mnmajor_desc(vb + ks * 2048, 16384), idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
+        umma_commit(pv_done);
+        umma_commit(&kv_empty[i & 1]);
+        return true;
+      };
+      for (int j = 0; ok && j < nblk; ++j) {
+        const int s = j & 1;
+        if (!mbar_wait(&kv_full[s], (j >> 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (j >= 2 && !mbar_wait(&s_free[s], ((j >> 1) - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t kb = smem_u32(smem + FaSmem::kOffK + s * FaSmem::kTile);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          umma_bf16(tmem + s * 128, sw128_kmajor_desc(qa + (ks >> 2) * 16384 + (ks & 3) * 32),
+                    sw128_kmajor_desc(kb + (ks >> 2) * 16384 + (ks & 3) * 32), idesc_s, ks > 0 ? 1u : 0u);
+        umma_commit(&s_full[s]);
+        if (j >= 1 && !pv(j - 1)) {
+          ok = false;
+          break;
+        }
+      }
+      if (ok && nblk > 0) ok = pv(nblk - 1);
+      if (!ok) {
+        *abort_flag = 1;
+        raise_error(a.err, kErrTimeoutMma);
+      }
+      // every issued MMA completes before TMEM is released
+      umma_commit(drain);
+      if (!mbar_wait(drain, 0, nullptr, kWaitTimeoutNs + kDrainTimeoutNs)) raise_error(a.err, kErrDrain);
+    }
+  } else {
+    // ------------------------------------------------ softmax / correction / output warps
+    const int lane_base = (warp & 3) * 32;
+    const int r = lane_base + lane;                 // TMEM lane = query row of this tile
+    const uint32_t tl = tmem + (static_cast<uint32_t>(lane_base) << 16);
+    const int pr = tile * 128 + r;
+    const bool valid = pr < rows_total;
+    const int head = valid ? kvh * G + pr / a.seq_q : 0;
+    const int pos = valid ? pr % a.seq_q : 0;
+    pdl_wait();
+    {   // Q row -> shared memory in the SW128 K-major layout
+      const uint4* src = reinterpret_cast<const uint4*>(a.q + ((static_cast<size_t>(b) * a.seq_q + pos) * a.n_q + head) * D);
+      uint8_t* qs = smem + FaSmem::kOffQ;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const uint4 v = valid ? src[c] : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(qs + sw128_off(r, c * 8)) = v;
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_ready);
+    }
+    float m_ref = -__int_as_float(0x7f800000), l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nblk; ++j) {
+      const int s = j & 1;
+      if (!mbar_wait(&s_full[s], (j >> 1) & 1, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int nvalid = j < nA ? min(128, a.len_a - j * 128) : min(128, a.len_b - (j - nA) * 128);
+      // pass 1: block max
+      float mx = -__int_as_float(0x7f800000);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32(tl + s * 128 + c * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (c * 32 + i < nvalid) mx = fmaxf(mx, v[i]);
+      }
+      const float m_blk = mx * a.scale_log2;
+      const bool move = m_blk > m_ref + 8.f;        // also true on the first block
+      const float m_new = move ? m_blk : m_ref;
+      const float alpha = move ? exp2f(m_ref - m_new) : 1.f;   // 0 on the first block
+      // pass 2: P = 2^(s*scale - m), row sum, packed to bf16
+      uint32_t pk[64];
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32(tl + s * 128 + c * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const float p0 = (c * 32 + i < nvalid) ? exp2f(v[i] * a.scale_log2 - m_new) : 0.f;
+          const float p1 = (c * 32 + i + 1 < nvalid) ? exp2f(v[i + 1] * a.scale_log2 - m_new) : 0.f;
+          sum += p0 + p1;
+          pk[c * 16 + i / 2] = pack_bf16(p0, p1);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[s]);
+      l_run = l_run * alpha + sum;
+      m_ref = m_new;
+      // O and the P slot of block j-2 are in use until PV_{j-1} completes
+      if (j >= 1) {
+        if (!mbar_wait(pv_done, (j - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, move)) {
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            float o[32];
+            tmem_ld32(tl + 256 + c * 32, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st32(tl + 256 + c * 32, o);
+          }
+          tmem_wait_st();
+        }
+      }
+      uint8_t* ps = smem + FaSmem::kOffP + s * FaSmem::kTile;
+#pragma unroll
+      for (int c = 0; c < 16; ++c)
+        *reinterpret_cast<uint4*>(ps + sw128_off(r, c * 8)) =
+            make_uint4(pk[c * 4], pk[c * 4 + 1], pk[c * 4 + 2], pk[c * 4 + 3]);
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      raise_error(a.err, kErrTimeoutEpilogue);
+    } else if (nblk > 0) {
+      if (mbar_wait(pv_done, (nblk - 1) & 1, abort_flag)) {
+        tc_fence_after();
+        const float inv = 1.f / l_run;
+        __nv_bfloat16* dst = a.o + ((static_cast<size_t>(b) * a.seq_q + pos) * a.n_q + head) * D;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float o[32];
+          tmem_ld32(tl + 256 + c * 32, o);
+          if (valid) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              d4[i] = make_uint4(pack_bf16(o[8 * i] * inv, o[8 * i + 1] * inv), pack_bf16(o[8 * i + 2] * inv, o[8 * i + 3] * inv),
+                                 pack_bf16(o[8 * i + 4] * inv, o[8 * i + 5] * inv), pack_bf16(o[8 * i + 6] * inv, o[8 * i + 7] * inv));
+          }
+        }
+      } else {
+        *abort_flag = 1;
+        raise_error(a.err, kErrTimeoutEpilogue);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace dm0

@@ -30,6 +30,7 @@
 
 #include "dm0.h"
 #include "attention.cuh"
+#include "attention_tc.cuh"
 #include "elementwise.cuh"
 #include "gemm.cuh"
 #include "ptx.cuh"
@@ -272,7 +273,11 @@ dm0_status run_gemm(dm0_ctx* c, cudaStream_t s, const bf16* act, int tokens, int
     return launch(c, s, dm0::gemm_tc_kernel<128, kGemmStages>, grid, dim3(dm0::kGemmThreads),
                   dm0::GemmSmem<128, kGemmStages>::kBytes, ta, tb, g);
   }
-  const int BN = (wrows % 256 == 0) ? 256 : 128;
+  const int mt = (tokens + 127) / 128;
+  int BN = (wrows % 256 == 0) ? 256 : 128;
+  // narrower tiles when the grid would leave SMs idle; a 64-wide tile only for column-independent epilogues
+  const int min_bn = (g.mode == dm0::kModeResid || g.mode == dm0::kModeStoreF32) ? 64 : 128;
+  while (BN > min_bn && mt * (wrows / BN) < c->num_sms) BN /= 2;
   g.M = tokens;
   g.N = wrows;
   g.swap = 0;
@@ -283,8 +288,11 @@ dm0_status run_gemm(dm0_ctx* c, cudaStream_t s, const bf16* act, int tokens, int
   if (BN == 256)
     return launch(c, s, dm0::gemm_tc_kernel<256, kGemmStages>, grid, dim3(dm0::kGemmThreads),
                   dm0::GemmSmem<256, kGemmStages>::kBytes, ta, tb, g);
-  return launch(c, s, dm0::gemm_tc_kernel<128, kGemmStages>, grid, dim3(dm0::kGemmThreads),
-                dm0::GemmSmem<128, kGemmStages>::kBytes, ta, tb, g);
+  if (BN == 128)
+    return launch(c, s, dm0::gemm_tc_kernel<128, kGemmStages>, grid, dim3(dm0::kGemmThreads),
+                  dm0::GemmSmem<128, kGemmStages>::kBytes, ta, tb, g);
+  return launch(c, s, dm0::gemm_tc_kernel<64, kGemmStages>, grid, dim3(dm0::kGemmThreads),
+                dm0::GemmSmem<64, kGemmStages>::kBytes, ta, tb, g);
 }
 
 // ---------------------------------------------------------------- attention dispatch
@@ -303,6 +311,10 @@ dm0_status run_attn(dm0_ctx* c, cudaStream_t s, const bf16* q, int seq_q, const 
   }
   if (splits > nblk) splits = nblk;
   while (splits > 1 && groups * tiles * splits > kPartSlots) --splits;
+  // the combine keeps (m, l) of every split and row in the kernel's shared memory
+  const int smem_bytes = g.head_dim == 128 ? dm0::AttnSmem<128>::kBytes
+                                           : (g.head_dim == 64 ? dm0::AttnSmem<64>::kBytes : dm0::AttnSmem<32>::kBytes);
+  while (splits > 1 && splits * 128 * 8 > smem_bytes) --splits;
   const int bps = (nblk + splits - 1) / splits;
   splits = (nblk + bps - 1) / bps;
   if (splits > 1 && groups * tiles > c->acount_n) return fail(c, DM0_ESHAPE, "attention split counters too small");
@@ -325,6 +337,21 @@ dm0_status run_attn(dm0_ctx* c, cudaStream_t s, const bf16* q, int seq_q, const 
   a.part_ml = c->part_ml;
   a.counters = c->acount;
   a.err = c->d_err;
+  if (g.head_dim == 128 && splits_req <= 1) {
+    // tcgen05 flash attention, K/V tiles of both segments by TMA, no key split
+    CUtensorMap tk, tv, tkb, tvb;
+    TRY(get_tmap(c, &tk, ka, static_cast<uint64_t>(groups) * len_a, 128, 128));
+    TRY(get_tmap(c, &tv, va, static_cast<uint64_t>(groups) * len_a, 128, 128));
+    if (len_b > 0) {
+      TRY(get_tmap(c, &tkb, kb, static_cast<uint64_t>(groups) * len_b, 128, 128));
+      TRY(get_tmap(c, &tvb, vb, static_cast<uint64_t>(groups) * len_b, 128, 128));
+    } else {
+      tkb = tk;
+      tvb = tv;
+    }
+    return launch(c, s, dm0::fa_tc_kernel, dim3(tiles, groups, 1), dim3(dm0::kFaThreads), dm0::FaSmem::kBytes, tk,
+                  tv, tkb, tvb, a);
+  }
   const dim3 grid(tiles, groups, splits);
   switch (g.head_dim) {
     case 128:
@@ -471,7 +498,7 @@ dm0_status enqueue_denoise(dm0_ctx* c, cudaStream_t s, int steps, float* vel) {
       float* ssq_attn = c->ssq_a + static_cast<size_t>(2 * l) * Ms;
       float* ssq_mlp = ssq_attn + Ms;
       TRY(layer_qkv(c, s, 1, l, c->xn_a, ssq_attn, Ms, S, P, c->q_a, c->k_s, c->v_s));
-      TRY(run_attn(c, s, c->q_a, S, kl, vl, P, c->k_s, c->v_s, S, c->o_a, B, 0, 1));
+      TRY(run_attn(c, s, c->q_a, S, kl, vl, P, c->k_s, c->v_s, S, c->o_a, B, 1, 1));
       const bool more = l + 1 < L;
       TRY(layer_rest(c, s, 1, l, Ms, c->h_a, c->xn_a, c->o_a, c->act_a, ssq_mlp,
                      more ? c->lw[1][l + 1].attn_norm : nullptr, more ? ssq_mlp + Ms : nullptr));
@@ -711,7 +738,8 @@ dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
             smem_attr(dm0::gemm_tc_kernel<256, kGemmStages>, dm0::GemmSmem<256, kGemmStages>::kBytes) &&
             smem_attr(dm0::attn_kernel<128>, dm0::AttnSmem<128>::kBytes) &&
             smem_attr(dm0::attn_kernel<64>, dm0::AttnSmem<64>::kBytes) &&
-            smem_attr(dm0::attn_kernel<32>, dm0::AttnSmem<32>::kBytes);
+            smem_attr(dm0::attn_kernel<32>, dm0::AttnSmem<32>::kBytes) &&
+            smem_attr(dm0::fa_tc_kernel, dm0::FaSmem::kBytes);
   if (!ok) return bail(DM0_ECUDA);
   *out = c;
   return DM0_OK;
@@ -842,7 +870,7 @@ dm0_status dm0_merged_layer(dm0_ctx* c, int layer, const float* h_prefix, const 
   TRY(layer_qkv(c, s, 1, layer, c->xn_a, c->ssq_a, Ms, S, P, c->q_a, c->k_s, c->v_s));
   // the block mask: prefix rows see the prefix; suffix rows see prefix and suffix
   TRY(run_attn(c, s, c->q_v, P, kp, vp, P, nullptr, nullptr, 0, c->o_v, B, 1, 0));
-  TRY(run_attn(c, s, c->q_a, S, kp, vp, P, c->k_s, c->v_s, S, c->o_a, B, 0, 0));
+  TRY(run_attn(c, s, c->q_a, S, kp, vp, P, c->k_s, c->v_s, S, c->o_a, B, 1, 0));
   TRY(layer_rest(c, s, 0, layer, Mp, c->h_v, c->xn_v, c->o_v, c->act_v, c->ssq_v + Mp, nullptr, nullptr));
   TRY(layer_rest(c, s, 1, layer, Ms, c->h_a, c->xn_a, c->o_a, c->act_a, c->ssq_a + Ms, nullptr, nullptr));
   CK(cudaMemcpyAsync(out_prefix, c->h_v, static_cast<size_t>(Mp) * g.hidden_v * 4, cudaMemcpyDeviceToDevice, s));

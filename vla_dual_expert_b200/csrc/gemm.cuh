@@ -124,13 +124,15 @@ __device__ __forceinline__ void st_bf16x32(__nv_bfloat16* dst, const float (&v)[
                        bf2(v[8 * i + 6], v[8 * i + 7]));
 }
 
+// `nchunks` (4, or 2 for a 64-column tile) applies to the column-independent modes (residual, store);
+// QKV and SwiGLU always take a full 128-column group.
 template <bool kFromScratch, class Load>
 __device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool valid, int col0, float& ssq_acc,
-                                             Load&& load) {
+                                             Load&& load, int nchunks = 4) {
   const int D = a.head_dim;
   if (a.mode == kModeStoreF32) {
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < nchunks; ++c) {
       float v[32];
       load(c, v);
       if (valid) st_f32x32(a.out_f32 + static_cast<size_t>(tok) * a.N + col0 + 32 * c, v);
@@ -139,7 +141,7 @@ __device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool va
   }
   if (a.mode == kModeResid) {
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < nchunks; ++c) {
       float v[32];
       load(c, v);
       if (!valid) continue;
@@ -386,10 +388,15 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
         const int tok = m_tile * 128 + lane_base + lane;
         const bool valid = tok < a.M;
         float ssq_acc = 0.f;
-        for (int g = 0; g < BN / 128; ++g) {
-          const uint32_t tg = tl + g * 128;
-          row_epilogue<false>(a, tok, valid, n_tile * BN + g * 128, ssq_acc,
-                              [&](int c, float (&v)[32]) { tmem_ld32(tg + c * 32, v); });
+        if (BN >= 128) {
+          for (int g = 0; g < BN / 128; ++g) {
+            const uint32_t tg = tl + g * 128;
+            row_epilogue<false>(a, tok, valid, n_tile * BN + g * 128, ssq_acc,
+                                [&](int c, float (&v)[32]) { tmem_ld32(tg + c * 32, v); });
+          }
+        } else {   // 64-column tile: residual / store modes only
+          row_epilogue<false>(a, tok, valid, n_tile * BN, ssq_acc,
+                              [&](int c, float (&v)[32]) { tmem_ld32(tl + c * 32, v); }, BN / 32);
         }
         if (a.mode == kModeResid && a.ssq_out && valid) atomicAdd(a.ssq_out + tok, ssq_acc);
       } else {
