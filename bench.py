@@ -169,7 +169,7 @@ def run_native(args, rank, world, local_rank):
                torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
         barrier()
         torch.cuda.synchronize()
-        eng.probe(probe)
+        eng.probe(0 if probe is None else 1 << probe)
         launches0 = eng.launch_count()
         with ClockSampler(local_rank) as clk:
             t0 = torch.cuda.Event(enable_timing=True)
@@ -185,7 +185,7 @@ def run_native(args, rank, world, local_rank):
             torch.cuda.synchronize()
         barrier()
         launches = eng.launch_count() - launches0
-        probe_n, probe_ms = eng.probe_read()
+        probe_n, probe_ms = eng.probe_read(probe) if probe is not None else (0, 0.0)
         eng.probe(0)
         eng.sync()
         ms = max_over_ranks(t0.elapsed_time(t1) / steps)
@@ -196,6 +196,25 @@ def run_native(args, rank, world, local_rank):
                 "prefill_ms_p90": pre[min(len(pre) - 1, int(0.9 * len(pre)))],
                 "denoise_ms_p90": den[min(len(den) - 1, int(0.9 * len(den)))],
                 "launches": launches, "probe_n": probe_n, "probe_ms": probe_ms, "clocks": clk.summary()}
+
+    def breakdown(eng, wl):
+        """One extra (untimed) step with every kernel site probed by CUDA-event pairs: per-site
+        milliseconds per step.  Probed launches lose their overlap with the previous kernel and
+        the denoise runs without its graph, so the sum exceeds the timed step."""
+        from vla_dual_expert_b200 import SITES
+        B, P = wl.batch, wl.prefix
+        emb = torch.from_numpy(I.prefix_embeddings(d, B, P, seed=1000 + 97 * rank)).cuda().to(torch.bfloat16)
+        noise = torch.from_numpy(I.noise(d, B, seed=2000 + 97 * rank)).cuda()
+        eng.probe((1 << len(SITES)) - 1)
+        eng.prefill(emb)
+        eng.denoise(noise, EULER_STEPS)
+        eng.sync()
+        out = {}
+        for i, name in enumerate(SITES):
+            n, ms = eng.probe_read(i)
+            out[name] = {"launches": n, "ms": round(ms, 3), "avg_us": round(1000.0 * ms / max(n, 1), 2)}
+        eng.probe(0)
+        return out
 
     def measure_e2e(wl, steps, warmup):
         """Through dm0_infer_host: pinned host inputs copied in and the chunk copied out every step."""
@@ -222,8 +241,8 @@ def run_native(args, rank, world, local_rank):
         ms = max_over_ranks(t0.elapsed_time(t1) / steps)
         return {"ms": ms, "h2d": emb_h.numel() * 2 + noise_h.numel() * 4, "d2h": out_h.numel() * 4}
 
-    # probe kind 1 = the VLM gate/up GEMM of the prefix pass (the largest launch of the step)
-    main = measure(wl_main, args.steps, args.warmup, probe=1)
+    # probe site 3 = the VLM gate/up GEMM of the prefix pass (the largest launch of the step)
+    main = measure(wl_main, args.steps, args.warmup, probe=3)
     e2e = measure_e2e(wl_main, max(2, args.steps // 2), 1) if not args.skip_e2e else {"ms": float("nan"), "h2d": 0,
                                                                                         "d2h": 0}
     B, P = wl_main.batch, wl_main.prefix
@@ -254,7 +273,7 @@ def run_native(args, rank, world, local_rank):
     }
     if args.workload == "e2e_b16" and not args.skip_batch1:
         wl1 = I.WORKLOADS["e2e_b1"]
-        b1 = measure(wl1, max(args.steps, 5), args.warmup, probe=0)
+        b1 = measure(wl1, max(args.steps, 5), args.warmup, probe=None)
         den_gbs = denoise_bytes_per_step(d, 1, wl1.prefix) * EULER_STEPS / (b1["denoise_ms_p50"] * 1e-3) / 1e9
         result["batch1"] = {
             "workload": "e2e_b1: prefill B=1 x P=816 + 10-step denoise", "value": round(world * 1000.0 / b1["ms"], 3),
@@ -265,6 +284,10 @@ def run_native(args, rank, world, local_rank):
                                  "unit": "GB/s", "frac": round(den_gbs / peaks["hbm_gbs"], 4),
                                  "algorithmic_bytes_per_euler_step": denoise_bytes_per_step(d, 1, wl1.prefix)},
         }
+    if not args.skip_breakdown:
+        result["breakdown_ms_per_step"] = breakdown(eng, wl_main)
+        if "batch1" in result:
+            result["batch1"]["breakdown_ms_per_step"] = breakdown(eng, I.WORKLOADS["e2e_b1"])
     if rank == 0 and world == 1 and not args.skip_cpu:
         result["cpu_baseline"] = cpu_baseline(wl_main, budget_s=args.cpu_budget)
     if rank == 0:
@@ -358,6 +381,7 @@ def main():
     ap.add_argument("--skip-batch1", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--skip-breakdown", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "native":

@@ -218,17 +218,34 @@ dm0_status dm0_attention_noalloc(const void* q, const void* ka, const void* va, 
  * every kernel it contains).  Host-side counter; never synchronises. */
 uint64_t dm0_launch_count(const dm0_ctx* ctx);
 
-/* Time one kernel site with CUDA events recorded on the launching stream
- * around each of its launches.  kind 0: off; kind 1: the gate/up GEMM of
- * every VLM layer of dm0_prefill.  Enabling resets the record.  Each timed
- * launch is preceded by an event record, so it is launched in plain stream
- * order instead of overlapping the previous kernel.  Events are created on
- * demand (256 at a time, at most 8192); the graphed denoise is never timed. */
-dm0_status dm0_probe(dm0_ctx* ctx, int kind);
+/* Kernel sites dm0_probe can time. */
+enum {
+  DM0_SITE_VLM_QKV = 0,     /* prefix pass: Q/K/V GEMM (+QK-norm, RoPE, cache write) */
+  DM0_SITE_VLM_ATTN = 1,    /* prefix pass: attention */
+  DM0_SITE_VLM_O = 2,       /* prefix pass: O GEMM (+residual) */
+  DM0_SITE_VLM_GATEUP = 3,  /* prefix pass: gate/up GEMM (+SwiGLU) */
+  DM0_SITE_VLM_DOWN = 4,    /* prefix pass: down GEMM (+residual) */
+  DM0_SITE_ACT_QKV = 5,     /* Euler loop: the same five action-expert kernels */
+  DM0_SITE_ACT_ATTN = 6,
+  DM0_SITE_ACT_O = 7,
+  DM0_SITE_ACT_GATEUP = 8,
+  DM0_SITE_ACT_DOWN = 9,
+  DM0_SITE_STEP = 10,       /* Euler step boundary (velocity, update, next input) */
+  DM0_SITE_COUNT = 11
+};
 
-/* Wait for the recorded events and return the number of timed launches and
- * their summed duration in milliseconds; then clear the record. */
-dm0_status dm0_probe_read(dm0_ctx* ctx, int* launches, double* total_ms);
+/* Time the launches of the sites in `site_mask` (bit i = site i) with CUDA
+ * events recorded on the launching stream around each launch; 0 turns the
+ * probe off.  Enabling resets the record.  A timed launch follows an event
+ * record, so it runs in plain stream order instead of overlapping the
+ * previous kernel, and while any site is probed dm0_denoise launches its
+ * kernels directly instead of replaying its graph.  Events are created on
+ * demand (256 at a time, at most 16384). */
+dm0_status dm0_probe(dm0_ctx* ctx, int site_mask);
+
+/* Wait for the recorded events of `site` and return its number of timed
+ * launches and their summed duration in milliseconds. */
+dm0_status dm0_probe_read(dm0_ctx* ctx, int site, int* launches, double* total_ms);
 
 /* Errors and lifetime. -------------------------------------------------- */
 

@@ -10,7 +10,7 @@ import ctypes
 
 import numpy as np
 
-from ._abi import (EXPORTS, LIB_PATH, Dm0Config, Dm0Error, load_library, make_config,  # noqa: F401
+from ._abi import (EXPORTS, LIB_PATH, SITES, Dm0Config, Dm0Error, load_library, make_config,  # noqa: F401
                    pack_weights)
 
 __all__ = ["Engine", "Dm0Error", "pack_weights", "load_library", "EXPORTS", "LIB_PATH"]
@@ -157,12 +157,12 @@ class Engine:
     def launch_count(self) -> int:
         return int(self.lib.dm0_launch_count(self.h))
 
-    def probe(self, kind: int):
-        self._chk(self.lib.dm0_probe(self.h, kind))
+    def probe(self, site_mask: int):
+        self._chk(self.lib.dm0_probe(self.h, site_mask))
 
-    def probe_read(self):
+    def probe_read(self, site: int):
         n, ms = c_int_t(), ctypes.c_double()
-        self._chk(self.lib.dm0_probe_read(self.h, ctypes.byref(n), ctypes.byref(ms)))
+        self._chk(self.lib.dm0_probe_read(self.h, site, ctypes.byref(n), ctypes.byref(ms)))
         return n.value, ms.value
 
     def sync(self, stream=None):

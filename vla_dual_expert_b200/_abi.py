@@ -70,7 +70,7 @@ def load_library() -> ctypes.CDLL:
         "dm0_debug_view": (c_int, [P, ctypes.c_char_p, ctypes.POINTER(P)]),
         "dm0_launch_count": (ctypes.c_uint64, [P]),
         "dm0_probe": (c_int, [P, c_int]),
-        "dm0_probe_read": (c_int, [P, ctypes.POINTER(c_int), ctypes.POINTER(ctypes.c_double)]),
+        "dm0_probe_read": (c_int, [P, c_int, ctypes.POINTER(c_int), ctypes.POINTER(ctypes.c_double)]),
         "dm0_sync": (c_int, [P, P]),
         "dm0_device_error": (c_int, [P]),
         "dm0_clear_error": (c_int, [P]),
@@ -97,6 +97,10 @@ def _bf16_bits(a: np.ndarray) -> np.ndarray:
     u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
     return ((u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)).astype(np.uint16)
 
+
+# kernel sites of dm0_probe (include/dm0.h)
+SITES = ("vlm_qkv", "vlm_attn", "vlm_o", "vlm_gateup", "vlm_down", "act_qkv", "act_attn", "act_o", "act_gateup",
+         "act_down", "step")
 
 LAYER_ORDER = (("attn_norm", "f32"), ("Wq", "bf16"), ("Wk", "bf16"), ("Wv", "bf16"), ("q_norm", "f32"),
                ("k_norm", "f32"), ("Wo", "bf16"), ("mlp_norm", "f32"), ("Wg", "bf16"), ("Wu", "bf16"),

@@ -74,6 +74,82 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 
 constexpr int kAttnStages = 3;   // K/V tiles in flight per CTA
 
+// Last CTA of a (group, row tile): merge the split-KV partial states (O unnormalised,
+// m and l in the base-2 domain against any common reference).  (m, l) of every
+// (split, row) go to shared memory in one coalesced pass, per-row weights
+// w_s = 2^(m_s - M) / L are computed once, then every output element is reduced
+// over the splits with independent loads spread over all threads.
+template <int D>
+__device__ __forceinline__ void combine_splits(const AttnArgs& a, size_t slot0, int tile, int b, int kvh,
+                                               float* scratch, int tid, int nthreads) {
+  const float kNegInf = __int_as_float(0xff800000);
+  const int G = a.n_q / a.n_kv;
+  const int rows_total = G * a.seq_q;
+  const int nsplit = gridDim.z;
+  float* sm_m = scratch;   // [nsplit][128]
+  float* sm_l = sm_m + nsplit * 128;
+  for (int i = tid; i < nsplit * 128; i += nthreads) {
+    const float2 ml = __ldcg(&a.part_ml[slot0 * 128 + i]);
+    sm_m[i] = ml.x;
+    sm_l[i] = ml.y;
+  }
+  __syncthreads();
+  if (tid < 128) {
+    float mmax = kNegInf;
+    for (int sp = 0; sp < nsplit; ++sp) mmax = fmaxf(mmax, sm_m[sp * 128 + tid]);
+    float lsum = 0.f;
+    for (int sp = 0; sp < nsplit; ++sp) {
+      const float w = exp2f(sm_m[sp * 128 + tid] - mmax);
+      sm_m[sp * 128 + tid] = w;
+      lsum += w * sm_l[sp * 128 + tid];
+    }
+    const float inv = 1.f / lsum;
+    for (int sp = 0; sp < nsplit; ++sp) sm_m[sp * 128 + tid] *= inv;
+  }
+  __syncthreads();
+  const int rows_here = min(128, rows_total - tile * 128);
+  constexpr int Q4 = D / 4;
+  constexpr int U = 8;   // output items per thread in flight
+  const int total = rows_here * Q4;
+  for (int base = tid; base < total; base += nthreads * U) {
+    float4 o[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) o[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int sp = 0; sp < nsplit; ++sp) {
+      float4 t[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int item = base + u * nthreads;
+        if (item < total) {
+          const int row = item / Q4, d4 = item - row * Q4;
+          t[u] = __ldcg(reinterpret_cast<const float4*>(a.part_o + ((slot0 + sp) * 128 + row) * D) + d4);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int item = base + u * nthreads;
+        if (item < total) {
+          const float w = sm_m[sp * 128 + item / Q4];
+          o[u].x += w * t[u].x;
+          o[u].y += w * t[u].y;
+          o[u].z += w * t[u].z;
+          o[u].w += w * t[u].w;
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int item = base + u * nthreads;
+      if (item >= total) continue;
+      const int row = item / Q4, d4 = item - row * Q4;
+      const int pr = tile * 128 + row;
+      const int head = kvh * G + pr / a.seq_q, pos = pr % a.seq_q;
+      __nv_bfloat16* dst = a.o + ((static_cast<size_t>(b) * a.seq_q + pos) * a.n_q + head) * D + 4 * d4;
+      *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16(o[u].x, o[u].y), pack_bf16(o[u].z, o[u].w));
+    }
+  }
+}
+
 template <int D>
 struct AttnSmem {
   static constexpr int kBytes = (128 + 2 * kAttnStages * 64) * D * 2;   // Q tile + K/V ring
@@ -285,51 +361,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnArgs a) {
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  // combine: (m, l) of every (split, row) into shared memory in one coalesced pass, per-row
-  // weights w_s = 2^(m_s - M) / L once, then every output element reduced over the splits with
-  // independent loads spread over all threads
-  const int nsplit = gridDim.z;
-  float* sm_m = reinterpret_cast<float*>(attn_smem);   // [nsplit][128], reuses the Q/K/V area
-  float* sm_l = sm_m + nsplit * 128;
-  for (int i = tid; i < nsplit * 128; i += kAttnThreads) {
-    const float2 ml = __ldcg(&a.part_ml[slot0 * 128 + i]);
-    sm_m[i] = ml.x;
-    sm_l[i] = ml.y;
-  }
-  __syncthreads();
-  if (tid < 128) {
-    float mmax = kNegInf;
-    for (int sp = 0; sp < nsplit; ++sp) mmax = fmaxf(mmax, sm_m[sp * 128 + tid]);
-    float lsum = 0.f;
-    for (int sp = 0; sp < nsplit; ++sp) {
-      const float w = exp2f(sm_m[sp * 128 + tid] - mmax);
-      sm_m[sp * 128 + tid] = w;
-      lsum += w * sm_l[sp * 128 + tid];
-    }
-    const float inv = 1.f / lsum;
-    for (int sp = 0; sp < nsplit; ++sp) sm_m[sp * 128 + tid] *= inv;
-  }
-  __syncthreads();
-  const int rows_here = min(128, rows_total - tile * 128);
-  constexpr int Q4 = D / 4;
-  for (int item = tid; item < rows_here * Q4; item += kAttnThreads) {
-    const int row = item / Q4, d4 = item - row * Q4;
-    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-    const float4* po = reinterpret_cast<const float4*>(a.part_o + (slot0 * 128 + row) * D) + d4;
-#pragma unroll 4
-    for (int sp = 0; sp < nsplit; ++sp) {
-      const float w = sm_m[sp * 128 + row];
-      const float4 t = __ldcg(po + static_cast<size_t>(sp) * 128 * Q4);
-      o.x += w * t.x;
-      o.y += w * t.y;
-      o.z += w * t.z;
-      o.w += w * t.w;
-    }
-    const int pr = tile * 128 + row;
-    const int head = kvh * G + pr / a.seq_q, pos = pr % a.seq_q;
-    __nv_bfloat16* dst = a.o + ((static_cast<size_t>(b) * a.seq_q + pos) * a.n_q + head) * D + 4 * d4;
-    *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16(o.x, o.y), pack_bf16(o.z, o.w));
-  }
+  combine_splits<D>(a, slot0, tile, b, kvh, reinterpret_cast<float*>(attn_smem), tid, kAttnThreads);
 }
 
 }  // namespace dm0

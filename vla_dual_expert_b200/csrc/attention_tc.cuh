@@ -7,18 +7,20 @@
 // One CTA owns 128 query rows of one (sample, KV head) group; the G query heads
 // sharing the KV head are packed along the rows as in attn_kernel, so every K/V
 // tile serves all of them.  Per 128-key block j:
-//   S_j = Q K_j^T        tcgen05.mma (M 128, N 128 keys, K 128), fp32 in TMEM,
+//   S_j = Q K_j^T        tcgen05.mma (M 128, N 64 keys, K 128), fp32 in TMEM,
 //                        double-buffered so S_{j+1} overlaps the softmax of S_j
 //   P_j = 2^(s - m)      softmax warps, one thread per row, read S from TMEM and
 //                        write P (bf16) to shared memory as a K-major operand
-//   O  += P_j V_j        tcgen05.mma (M 128, N 128 dims, K 128 keys); V is read
+//   O  += P_j V_j        tcgen05.mma (M 128, N 128 dims, K 64 keys); V is read
 //                        in its stored [key][dim] order as an MN-major operand
 // The running max is only moved (and O, l rescaled in TMEM) when a row's max
 // grows by more than 2^8: p stays <= 256 in between and the final O / l uses a
 // consistent reference, so the result is exact up to rounding.
 //
 // Warp roles (192 threads): warp 0 TMA producer for K/V, warp 1 TMEM owner and
-// MMA issuer, warps 2..5 Q staging, softmax, O correction and output.
+// MMA issuer, warps 2..5 Q staging, softmax, O correction and output.  112 KB of
+// shared memory, 256 TMEM columns and <= 168 registers per thread let two CTAs
+// share an SM, so one CTA's softmax overlaps the other's tensor-core work.
 #pragma once
 #include "attention.cuh"
 #include "ptx.cuh"
@@ -28,14 +30,19 @@ namespace dm0 {
 constexpr int kFaThreads = 192;
 
 struct FaSmem {
-  static constexpr uint32_t kTile = 32768;                  // 128 rows x 128 bf16, two 64-column SW128 halves
+  static constexpr int kKeys = 64;                          // keys per block
+  static constexpr uint32_t kQ = 32768;                     // 128 rows x 128 dims: two 64-column SW128 halves
+  static constexpr uint32_t kKV = 16384;                    // 64 keys x 128 dims: two 8 KB SW128 halves
+  static constexpr uint32_t kHalfKV = 8192;
+  static constexpr uint32_t kP = 16384;                     // 128 rows x 64 keys, one SW128 block
   static constexpr int kStages = 2;                         // K/V blocks in flight
   static constexpr uint32_t kOffQ = 0;
-  static constexpr uint32_t kOffK = kOffQ + kTile;
-  static constexpr uint32_t kOffV = kOffK + kStages * kTile;
-  static constexpr uint32_t kOffP = kOffV + kStages * kTile;
-  static constexpr uint32_t kOffBar = kOffP + 2 * kTile;    // 229376
-  static constexpr uint32_t kBytes = kOffBar + 256 + 1024;
+  static constexpr uint32_t kOffK = kOffQ + kQ;
+  static constexpr uint32_t kOffV = kOffK + kStages * kKV;
+  static constexpr uint32_t kOffP = kOffV + kStages * kKV;
+  static constexpr uint32_t kOffBar = kOffP + kP;           // 114688
+  static constexpr uint32_t kSlack = 256;                   // the dynamic base is 1024-aligned (no static smem)
+  static constexpr uint32_t kBytes = kOffBar + 256 + kSlack;
 };
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
@@ -71,18 +78,22 @@ __device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_addr, uint3
   return d;
 }
 
-// byte offset of element (row, col) of a 128 x 128 bf16 tile stored as two 64-column SW128 halves
+// byte offset of element (row, col) of a 128-row bf16 tile stored as 64-column SW128 halves
 __device__ __forceinline__ uint32_t sw128_off(int row, int col) {
   const int half = col >> 6, c16 = (col & 63) >> 3;
   return half * 16384 + row * 128 + ((c16 ^ (row & 7)) << 4) + ((col & 7) << 1);
 }
 
-__global__ void __launch_bounds__(kFaThreads, 1)
+__global__ void __launch_bounds__(kFaThreads, 2)
     fa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const __grid_constant__ CUtensorMap tmKb, const __grid_constant__ CUtensorMap tmVb, const AttnArgs a) {
   constexpr int D = 128;
   extern __shared__ uint8_t fa_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fa_smem_raw) + 1023) & ~uintptr_t(1023));
+  if (smem - fa_smem_raw > static_cast<ptrdiff_t>(FaSmem::kSlack)) {   // never expected: refuse rather than overrun
+    if (threadIdx.x == 0) raise_error(a.err, kErrBounds);
+    return;
+  }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + FaSmem::kOffBar);
   uint64_t* kv_full = bars;        // [2] TMA landed K_j, V_j
   uint64_t* kv_empty = bars + 2;   // [2] PV_j done: K/V slot free
@@ -100,9 +111,12 @@ __global__ void __launch_bounds__(kFaThreads, 1)
   const int b = grp / a.n_kv, kvh = grp - b * a.n_kv;
   const int G = a.n_q / a.n_kv;
   const int rows_total = G * a.seq_q;
-  // 128-key blocks: segment A first, then segment B (a block never mixes segments)
-  const int nA = (a.len_a + 127) >> 7, nB = (a.len_b + 127) >> 7;
-  const int nblk = nA + nB;
+  // 64-key blocks: segment A first, then segment B (a block never mixes segments); split z of
+  // gridDim.z takes blocks [jb0, jb1)
+  const int nA = (a.len_a + 63) >> 6, nB = (a.len_b + 63) >> 6;
+  const int jb0 = blockIdx.z * a.blocks_per_split;
+  const int jb1 = min(nA + nB, jb0 + a.blocks_per_split);
+  const int nblk = jb1 - jb0;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -119,13 +133,13 @@ __global__ void __launch_bounds__(kFaThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 512);
+    tmem_alloc(tmem_slot, 256);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;   // S_0 at column 0, S_1 at 128, O at 256
+  const uint32_t tmem = *tmem_slot;   // S_0 at column 0, S_1 at 64, O at 128
   pdl_launch_dependents();
 
   if (warp == 0) {
@@ -140,23 +154,24 @@ __global__ void __launch_bounds__(kFaThreads, 1)
       const uint64_t pol = policy_evict_last();
       auto issue = [&](int j) {
         const int s = j & 1;
-        const bool segA = j < nA;
+        const int jj = jb0 + j;   // global block index
+        const bool segA = jj < nA;
         const CUtensorMap* mk = segA ? &tmK : &tmKb;
         const CUtensorMap* mv = segA ? &tmV : &tmVb;
-        const int row = segA ? grp * a.len_a + j * 128 : grp * a.len_b + (j - nA) * 128;
-        mbar_arrive_expect_tx(&kv_full[s], 2 * FaSmem::kTile);
-        uint8_t* kd = smem + FaSmem::kOffK + s * FaSmem::kTile;
-        uint8_t* vd = smem + FaSmem::kOffV + s * FaSmem::kTile;
+        const int row = segA ? grp * a.len_a + jj * 64 : grp * a.len_b + (jj - nA) * 64;
+        mbar_arrive_expect_tx(&kv_full[s], 2 * FaSmem::kKV);
+        uint8_t* kd = smem + FaSmem::kOffK + s * FaSmem::kKV;
+        uint8_t* vd = smem + FaSmem::kOffV + s * FaSmem::kKV;
         tma_load_2d(kd, mk, &kv_full[s], 0, row, pol);
-        tma_load_2d(kd + 16384, mk, &kv_full[s], 64, row, pol);
+        tma_load_2d(kd + FaSmem::kHalfKV, mk, &kv_full[s], 64, row, pol);
         tma_load_2d(vd, mv, &kv_full[s], 0, row, pol);
-        tma_load_2d(vd + 16384, mv, &kv_full[s], 64, row, pol);
+        tma_load_2d(vd + FaSmem::kHalfKV, mv, &kv_full[s], 64, row, pol);
       };
       // segment A written before the previous kernel (the prefix cache during the Euler loop) may be
       // requested before the dependency wait
       int issued = 0;
       if (a.a_stable)
-        for (; issued < 2 && issued < nA; ++issued) issue(issued);
+        for (; issued < 2 && issued < nblk && jb0 + issued < nA; ++issued) issue(issued);
       pdl_wait();
       for (int j = issued; j < nblk; ++j) {
         const int s = j & 1;
@@ -176,19 +191,19 @@ __global__ void __launch_bounds__(kFaThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(128, 128);
+      const uint32_t idesc_s = idesc_bf16_f32(128, 64);
       const uint32_t idesc_pv = idesc_bf16_f32(128, 128) | (1u << 16);   // B (V) is MN-major
       const uint32_t qa = smem_u32(smem + FaSmem::kOffQ);
       bool ok = mbar_wait(q_ready, 0, abort_flag);
       auto pv = [&](int i) -> bool {
         if (!mbar_wait(p_full, i & 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t pa = smem_u32(smem + FaSmem::kOffP + (i & 1) * FaSmem::kTile);
-        const uint32_t vb = smem_u32(smem + FaSmem::kOffV + (i & 1) * FaSmem::kTile);
+        const uint32_t pa = smem_u32(smem + FaSmem::kOffP);
+        const uint32_t vb = smem_u32(smem + FaSmem::kOffV + (i & 1) * FaSmem::kKV);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-          umma_bf16(tmem + 256, sw128_kmajor_desc(pa + (ks >> 2) * 16384 + (ks & 3) * 32),
-                    sw128_mnmajor_desc(vb + ks * 2048, 16384), idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
+        for (int ks = 0; ks < 4; ++ks)
+          umma_bf16(tmem + 128, sw128_kmajor_desc(pa + ks * 32), sw128_mnmajor_desc(vb + ks * 2048, FaSmem::kHalfKV),
+                    idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
         umma_commit(pv_done);
         umma_commit(&kv_empty[i & 1]);
         return true;
@@ -204,11 +219,11 @@ __global__ void __launch_bounds__(kFaThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t kb = smem_u32(smem + FaSmem::kOffK + s * FaSmem::kTile);
+        const uint32_t kb = smem_u32(smem + FaSmem::kOffK + s * FaSmem::kKV);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          umma_bf16(tmem + s * 128, sw128_kmajor_desc(qa + (ks >> 2) * 16384 + (ks & 3) * 32),
-                    sw128_kmajor_desc(kb + (ks >> 2) * 16384 + (ks & 3) * 32), idesc_s, ks > 0 ? 1u : 0u);
+          umma_bf16(tmem + s * 64, sw128_kmajor_desc(qa + (ks >> 2) * 16384 + (ks & 3) * 32),
+                    sw128_kmajor_desc(kb + (ks >> 2) * FaSmem::kHalfKV + (ks & 3) * 32), idesc_s, ks > 0 ? 1u : 0u);
         umma_commit(&s_full[s]);
         if (j >= 1 && !pv(j - 1)) {
           ok = false;
@@ -255,39 +270,60 @@ __global__ void __launch_bounds__(kFaThreads, 1)
         break;
       }
       tc_fence_after();
-      const int nvalid = j < nA ? min(128, a.len_a - j * 128) : min(128, a.len_b - (j - nA) * 128);
-      // pass 1: block max
-      float mx = -__int_as_float(0x7f800000);
+      const int jj = jb0 + j;
+      const int nvalid = jj < nA ? min(64, a.len_a - jj * 64) : min(64, a.len_b - (jj - nA) * 64);
+      // the whole S row in registers: two TMEM loads, one wait
+      float sv[64];
+      {
+        uint32_t* u = reinterpret_cast<uint32_t*>(sv);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32(tl + s * 128 + c * 32, v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (c * 32 + i < nvalid) mx = fmaxf(mx, v[i]);
+        for (int c = 0; c < 2; ++c)
+          asm volatile(
+              "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+              "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+              "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+              : "=r"(u[c * 32 + 0]), "=r"(u[c * 32 + 1]), "=r"(u[c * 32 + 2]), "=r"(u[c * 32 + 3]),
+                "=r"(u[c * 32 + 4]), "=r"(u[c * 32 + 5]), "=r"(u[c * 32 + 6]), "=r"(u[c * 32 + 7]),
+                "=r"(u[c * 32 + 8]), "=r"(u[c * 32 + 9]), "=r"(u[c * 32 + 10]), "=r"(u[c * 32 + 11]),
+                "=r"(u[c * 32 + 12]), "=r"(u[c * 32 + 13]), "=r"(u[c * 32 + 14]), "=r"(u[c * 32 + 15]),
+                "=r"(u[c * 32 + 16]), "=r"(u[c * 32 + 17]), "=r"(u[c * 32 + 18]), "=r"(u[c * 32 + 19]),
+                "=r"(u[c * 32 + 20]), "=r"(u[c * 32 + 21]), "=r"(u[c * 32 + 22]), "=r"(u[c * 32 + 23]),
+                "=r"(u[c * 32 + 24]), "=r"(u[c * 32 + 25]), "=r"(u[c * 32 + 26]), "=r"(u[c * 32 + 27]),
+                "=r"(u[c * 32 + 28]), "=r"(u[c * 32 + 29]), "=r"(u[c * 32 + 30]), "=r"(u[c * 32 + 31])
+              : "r"(tl + s * 64 + c * 32));
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
       }
+      // S buffer consumed: the MMA warp may overwrite it with S_{j+2}
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[s]);
+      // block max over the valid keys, eight independent chains
+      const float ninf = -__int_as_float(0x7f800000);
+      float mx8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx8[k] = ninf;
+#pragma unroll
+      for (int i = 0; i < 64; ++i)
+        if (i < nvalid) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_blk = mx * a.scale_log2;
       const bool move = m_blk > m_ref + 8.f;        // also true on the first block
       const float m_new = move ? m_blk : m_ref;
       const float alpha = move ? exp2f(m_ref - m_new) : 1.f;   // 0 on the first block
-      // pass 2: P = 2^(s*scale - m), row sum, packed to bf16
-      uint32_t pk[64];
-      float sum = 0.f;
+      // P = 2^(s*scale - m), row sum in eight partial sums, packed to bf16
+      uint32_t pk[32];
+      float sum8[8];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float v[32];
-        tmem_ld32(tl + s * 128 + c * 32, v);
+      for (int k = 0; k < 8; ++k) sum8[k] = 0.f;
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          const float p0 = (c * 32 + i < nvalid) ? exp2f(v[i] * a.scale_log2 - m_new) : 0.f;
-          const float p1 = (c * 32 + i + 1 < nvalid) ? exp2f(v[i + 1] * a.scale_log2 - m_new) : 0.f;
-          sum += p0 + p1;
-          pk[c * 16 + i / 2] = pack_bf16(p0, p1);
-        }
+      for (int i = 0; i < 64; i += 2) {
+        const float p0 = (i < nvalid) ? exp2f(fmaf(sv[i], a.scale_log2, -m_new)) : 0.f;
+        const float p1 = (i + 1 < nvalid) ? exp2f(fmaf(sv[i + 1], a.scale_log2, -m_new)) : 0.f;
+        sum8[(i >> 1) & 7] += p0 + p1;
+        pk[i >> 1] = pack_bf16(p0, p1);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[s]);
+      const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
       l_run = l_run * alpha + sum;
       m_ref = m_new;
       // O and the P slot of block j-2 are in use until PV_{j-1} completes
@@ -301,17 +337,17 @@ __global__ void __launch_bounds__(kFaThreads, 1)
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {
             float o[32];
-            tmem_ld32(tl + 256 + c * 32, o);
+            tmem_ld32(tl + 128 + c * 32, o);
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] *= alpha;
-            tmem_st32(tl + 256 + c * 32, o);
+            tmem_st32(tl + 128 + c * 32, o);
           }
           tmem_wait_st();
         }
       }
-      uint8_t* ps = smem + FaSmem::kOffP + s * FaSmem::kTile;
+      uint8_t* ps = smem + FaSmem::kOffP;   // one buffer: PV_{j-1} has completed
 #pragma unroll
-      for (int c = 0; c < 16; ++c)
+      for (int c = 0; c < 8; ++c)
         *reinterpret_cast<uint4*>(ps + sw128_off(r, c * 8)) =
             make_uint4(pk[c * 4], pk[c * 4 + 1], pk[c * 4 + 2], pk[c * 4 + 3]);
       fence_async_smem();
@@ -325,19 +361,37 @@ __global__ void __launch_bounds__(kFaThreads, 1)
     } else if (nblk > 0) {
       if (mbar_wait(pv_done, (nblk - 1) & 1, abort_flag)) {
         tc_fence_after();
-        const float inv = 1.f / l_run;
-        __nv_bfloat16* dst = a.o + ((static_cast<size_t>(b) * a.seq_q + pos) * a.n_q + head) * D;
+        if (gridDim.z == 1) {
+          const float inv = 1.f / l_run;
+          __nv_bfloat16* dst = a.o + ((static_cast<size_t>(b) * a.seq_q + pos) * a.n_q + head) * D;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          float o[32];
-          tmem_ld32(tl + 256 + c * 32, o);
-          if (valid) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+          for (int c = 0; c < 4; ++c) {
+            float o[32];
+            tmem_ld32(tl + 128 + c * 32, o);
+            if (valid) {
+              uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              d4[i] = make_uint4(pack_bf16(o[8 * i] * inv, o[8 * i + 1] * inv), pack_bf16(o[8 * i + 2] * inv, o[8 * i + 3] * inv),
-                                 pack_bf16(o[8 * i + 4] * inv, o[8 * i + 5] * inv), pack_bf16(o[8 * i + 6] * inv, o[8 * i + 7] * inv));
+              for (int i = 0; i < 4; ++i)
+                d4[i] = make_uint4(pack_bf16(o[8 * i] * inv, o[8 * i + 1] * inv),
+                                   pack_bf16(o[8 * i + 2] * inv, o[8 * i + 3] * inv),
+                                   pack_bf16(o[8 * i + 4] * inv, o[8 * i + 5] * inv),
+                                   pack_bf16(o[8 * i + 6] * inv, o[8 * i + 7] * inv));
+            }
           }
+        } else {
+          // split keys: this split's unnormalised O and (m, l) against its reference max
+          const size_t mine = ((static_cast<size_t>(grp) * gridDim.x + tile) * gridDim.z + blockIdx.z) * 128 + r;
+          float* po = a.part_o + mine * D;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            float o[32];
+            tmem_ld32(tl + 128 + c * 32, o);
+            float4* p4 = reinterpret_cast<float4*>(po + c * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) p4[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+          }
+          a.part_ml[mine] = make_float2(m_ref, l_run);
+          __threadfence();
         }
       } else {
         *abort_flag = 1;
@@ -349,7 +403,23 @@ __global__ void __launch_bounds__(kFaThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, 256);
+  }
+  if (gridDim.z > 1) {
+    // the last split of this (group, row tile) merges the partial states
+    int* s_last = reinterpret_cast<int*>(tmem_slot + 2);
+    if (threadIdx.x == 0) {
+      int* ctr = a.counters + static_cast<size_t>(grp) * gridDim.x + tile;
+      const int prev = atomicAdd(ctr, 1);
+      *s_last = prev == static_cast<int>(gridDim.z) - 1;
+      if (*s_last) *ctr = 0;
+    }
+    __syncthreads();
+    if (*s_last && !*abort_flag) {
+      __threadfence();
+      const size_t slot0 = (static_cast<size_t>(grp) * gridDim.x + tile) * gridDim.z;
+      combine_splits<128>(a, slot0, tile, b, kvh, reinterpret_cast<float*>(smem), threadIdx.x, kFaThreads);
+    }
   }
 }
 

@@ -127,10 +127,14 @@ struct dm0_ctx {
   };
   std::map<std::tuple<int, int, int>, Graph> graphs;
   uint64_t launches = 0;   // kernels this context has put on a stream (graph replays count their kernels)
-  // event probe around the launches of one kernel site (dm0_probe)
-  int probe = 0;
+  // event probe around the launches of selected kernel sites (dm0_probe)
+  int probe_mask = 0;
   std::vector<cudaEvent_t> probe_ev;
   size_t probe_used = 0;
+  struct ProbeRec {
+    int site, e0, e1;
+  };
+  std::vector<ProbeRec> probe_recs;
   std::map<TmapKey, CUtensorMap> tmaps;
   std::vector<void*> allocs;
 };
@@ -218,19 +222,28 @@ dm0_status launch(dm0_ctx* c, cudaStream_t s, void (*kernel)(KArgs...), dim3 gri
   return DM0_OK;
 }
 
-// CUDA-event pair around one launch of the probed kernel site
-dm0_status probe_mark(dm0_ctx* c, cudaStream_t s) {
+// CUDA-event pair around the launches of a probed kernel site: begin returns the first
+// event's index (or -1 when the site is not probed or the pool is full)
+int probe_event(dm0_ctx* c, cudaStream_t s) {
   if (c->probe_used >= c->probe_ev.size()) {
-    if (c->probe_ev.size() >= 8192) return DM0_OK;   // full: later launches are not timed
+    if (c->probe_ev.size() >= 16384) return -1;
     for (int i = 0; i < 256; ++i) {
       cudaEvent_t e;
-      CK(cudaEventCreate(&e));
+      if (cudaEventCreate(&e) != cudaSuccess) return -1;
       c->probe_ev.push_back(e);
     }
   }
-  CK(cudaEventRecord(c->probe_ev[c->probe_used++], s));
+  if (cudaEventRecord(c->probe_ev[c->probe_used], s) != cudaSuccess) return -1;
   c->pdl_ok = false;   // the next kernel follows an event record, not one of our kernels
-  return DM0_OK;
+  return static_cast<int>(c->probe_used++);
+}
+int probe_begin(dm0_ctx* c, cudaStream_t s, int site) {
+  return (c->probe_mask >> site) & 1 ? probe_event(c, s) : -1;
+}
+void probe_end(dm0_ctx* c, cudaStream_t s, int site, int e0) {
+  if (e0 < 0) return;
+  const int e1 = probe_event(c, s);
+  if (e1 >= 0) c->probe_recs.push_back({site, e0, e1});
 }
 
 // ---------------------------------------------------------------- GEMM dispatch
@@ -284,15 +297,17 @@ dm0_status run_gemm(dm0_ctx* c, cudaStream_t s, const bf16* act, int tokens, int
   g.kb_per_split = KB;
   TRY(get_tmap(c, &ta, act, tokens, K, 128));
   TRY(get_tmap(c, &tb, W, wrows, K, BN));
-  const dim3 grid((tokens + 127) / 128, wrows / BN, 1);
+  // persistent: at most one CTA per SM walking the tiles
+  const int ntiles = mt * (wrows / BN);
+  const dim3 grid(std::min(ntiles, c->num_sms));
   if (BN == 256)
-    return launch(c, s, dm0::gemm_tc_kernel<256, kGemmStages>, grid, dim3(dm0::kGemmThreads),
-                  dm0::GemmSmem<256, kGemmStages>::kBytes, ta, tb, g);
+    return launch(c, s, dm0::gemm_tc_persistent<256, kGemmStages>, grid, dim3(dm0::kGemmThreads),
+                  dm0::PGemmSmem<256, kGemmStages>::kBytes, ta, tb, g);
   if (BN == 128)
-    return launch(c, s, dm0::gemm_tc_kernel<128, kGemmStages>, grid, dim3(dm0::kGemmThreads),
-                  dm0::GemmSmem<128, kGemmStages>::kBytes, ta, tb, g);
-  return launch(c, s, dm0::gemm_tc_kernel<64, kGemmStages>, grid, dim3(dm0::kGemmThreads),
-                dm0::GemmSmem<64, kGemmStages>::kBytes, ta, tb, g);
+    return launch(c, s, dm0::gemm_tc_persistent<128, kGemmStages>, grid, dim3(dm0::kGemmThreads),
+                  dm0::PGemmSmem<128, kGemmStages>::kBytes, ta, tb, g);
+  return launch(c, s, dm0::gemm_tc_persistent<64, kGemmStages>, grid, dim3(dm0::kGemmThreads),
+                dm0::PGemmSmem<64, kGemmStages>::kBytes, ta, tb, g);
 }
 
 // ---------------------------------------------------------------- attention dispatch
@@ -337,19 +352,32 @@ dm0_status run_attn(dm0_ctx* c, cudaStream_t s, const bf16* q, int seq_q, const 
   a.part_ml = c->part_ml;
   a.counters = c->acount;
   a.err = c->d_err;
-  if (g.head_dim == 128 && splits_req <= 1) {
-    // tcgen05 flash attention, K/V tiles of both segments by TMA, no key split
+  if (g.head_dim == 128) {
+    // tcgen05 flash attention, K/V tiles of both segments by TMA; keys split in 64-key blocks
+    const int fblk = (len_a + 63) / 64 + (len_b + 63) / 64;
+    int fs = splits_req;
+    if (fs <= 0) {   // about two CTAs per SM, at most 4 splits (the combine reads every split's partial O)
+      const int ctas = groups * tiles;
+      fs = std::max(1, std::min(4, (2 * c->num_sms + ctas / 2) / ctas));
+    }
+    fs = std::min(fs, fblk);
+    while (fs > 1 && groups * tiles * fs > kPartSlots) --fs;
+    while (fs > 1 && fs * 128 * 8 > static_cast<int>(dm0::FaSmem::kOffBar)) --fs;   // combine keeps (m, l) in smem
+    int fbps = (fblk + fs - 1) / fs;
+    fs = (fblk + fbps - 1) / fbps;
+    if (fs > 1 && groups * tiles > c->acount_n) return fail(c, DM0_ESHAPE, "attention split counters too small");
+    a.blocks_per_split = fbps;
     CUtensorMap tk, tv, tkb, tvb;
-    TRY(get_tmap(c, &tk, ka, static_cast<uint64_t>(groups) * len_a, 128, 128));
-    TRY(get_tmap(c, &tv, va, static_cast<uint64_t>(groups) * len_a, 128, 128));
+    TRY(get_tmap(c, &tk, ka, static_cast<uint64_t>(groups) * len_a, 128, dm0::FaSmem::kKeys));
+    TRY(get_tmap(c, &tv, va, static_cast<uint64_t>(groups) * len_a, 128, dm0::FaSmem::kKeys));
     if (len_b > 0) {
-      TRY(get_tmap(c, &tkb, kb, static_cast<uint64_t>(groups) * len_b, 128, 128));
-      TRY(get_tmap(c, &tvb, vb, static_cast<uint64_t>(groups) * len_b, 128, 128));
+      TRY(get_tmap(c, &tkb, kb, static_cast<uint64_t>(groups) * len_b, 128, dm0::FaSmem::kKeys));
+      TRY(get_tmap(c, &tvb, vb, static_cast<uint64_t>(groups) * len_b, 128, dm0::FaSmem::kKeys));
     } else {
       tkb = tk;
       tvb = tv;
     }
-    return launch(c, s, dm0::fa_tc_kernel, dim3(tiles, groups, 1), dim3(dm0::kFaThreads), dm0::FaSmem::kBytes, tk,
+    return launch(c, s, dm0::fa_tc_kernel, dim3(tiles, groups, fs), dim3(dm0::kFaThreads), dm0::FaSmem::kBytes, tk,
                   tv, tkb, tvb, a);
   }
   const dim3 grid(tiles, groups, splits);
@@ -398,7 +426,11 @@ dm0_status layer_qkv(dm0_ctx* c, cudaStream_t s, int br, int l, const bf16* xn, 
   g.seq_len = seq;
   g.pos_offset = pos_offset;
   g.kv_seq = seq;
-  return run_gemm(c, s, xn, tokens, H, w.wqkv, qkv_rows(c->cfg), g);
+  const int site = br == 0 ? DM0_SITE_VLM_QKV : DM0_SITE_ACT_QKV;
+  const int e0 = probe_begin(c, s, site);
+  TRY(run_gemm(c, s, xn, tokens, H, w.wqkv, qkv_rows(c->cfg), g));
+  probe_end(c, s, site, e0);
+  return DM0_OK;
 }
 
 // O-proj (+residual) -> gate/up (+SwiGLU) -> down (+residual) of one branch
@@ -415,7 +447,10 @@ dm0_status layer_rest(dm0_ctx* c, cudaStream_t s, int br, int l, int tokens, flo
   g.xn = xn;
   g.gain_next = w.mlp_norm;
   g.ssq_out = ssq_mlp;
+  const int so = br == 0 ? DM0_SITE_VLM_O : DM0_SITE_ACT_O;
+  int e0 = probe_begin(c, s, so);
   TRY(run_gemm(c, s, o, tokens, cf.n_q * cf.head_dim, w.wo, H, g));
+  probe_end(c, s, so, e0);
   GemmArgs u = base_args(c);
   u.w_stable = 1;
   u.mode = dm0::kModeSwiGLU;
@@ -423,10 +458,10 @@ dm0_status layer_rest(dm0_ctx* c, cudaStream_t s, int br, int l, int tokens, flo
   u.inv_hidden = 1.0f / H;
   u.act = act;
   u.inter = I;
-  const bool probed = c->probe == 1 && br == 0;
-  if (probed) TRY(probe_mark(c, s));
+  const int su = br == 0 ? DM0_SITE_VLM_GATEUP : DM0_SITE_ACT_GATEUP;
+  e0 = probe_begin(c, s, su);
   TRY(run_gemm(c, s, xn, tokens, H, w.wgu, 2 * I, u));
-  if (probed) TRY(probe_mark(c, s));
+  probe_end(c, s, su, e0);
   GemmArgs d = base_args(c);
   d.w_stable = 1;
   d.mode = dm0::kModeResid;
@@ -435,7 +470,11 @@ dm0_status layer_rest(dm0_ctx* c, cudaStream_t s, int br, int l, int tokens, flo
   d.xn = next_gain ? xn : nullptr;
   d.gain_next = next_gain;
   d.ssq_out = next_gain ? next_ssq : nullptr;
-  return run_gemm(c, s, act, tokens, I, w.wd, H, d);
+  const int sd = br == 0 ? DM0_SITE_VLM_DOWN : DM0_SITE_ACT_DOWN;
+  e0 = probe_begin(c, s, sd);
+  TRY(run_gemm(c, s, act, tokens, I, w.wd, H, d));
+  probe_end(c, s, sd, e0);
+  return DM0_OK;
 }
 
 dm0_status enqueue_prefill(dm0_ctx* c, cudaStream_t s, const void* prefix_emb, int B, int P) {
@@ -450,7 +489,9 @@ dm0_status enqueue_prefill(dm0_ctx* c, cudaStream_t s, const void* prefix_emb, i
     float* ssq_attn = c->ssq_v + static_cast<size_t>(2 * l) * M;
     float* ssq_mlp = ssq_attn + M;
     TRY(layer_qkv(c, s, 0, l, c->xn_v, ssq_attn, M, P, 0, c->q_v, kl, vl));
+    const int e0 = probe_begin(c, s, DM0_SITE_VLM_ATTN);
     TRY(run_attn(c, s, c->q_v, P, kl, vl, P, nullptr, nullptr, 0, c->o_v, B, 1, 0));
+    probe_end(c, s, DM0_SITE_VLM_ATTN, e0);
     const bool more = l + 1 < L;
     TRY(layer_rest(c, s, 0, l, M, c->h_v, c->xn_v, c->o_v, c->act_v, ssq_mlp,
                    more ? c->lw[0][l + 1].attn_norm : nullptr, more ? ssq_mlp + M : nullptr));
@@ -480,7 +521,10 @@ dm0_status step(dm0_ctx* c, cudaStream_t s, int B, int k_out, int k_in, int step
   a.k_in = k_in;
   a.steps = steps;
   a.vel = vel;
-  return launch(c, s, dm0::step_kernel, dim3(B * cf.chunk), dim3(256), 0, a);
+  const int e0 = probe_begin(c, s, DM0_SITE_STEP);
+  TRY(launch(c, s, dm0::step_kernel, dim3(B * cf.chunk), dim3(256), 0, a));
+  probe_end(c, s, DM0_SITE_STEP, e0);
+  return DM0_OK;
 }
 
 // Euler loop over the KV cache; x already holds x_1
@@ -498,7 +542,9 @@ dm0_status enqueue_denoise(dm0_ctx* c, cudaStream_t s, int steps, float* vel) {
       float* ssq_attn = c->ssq_a + static_cast<size_t>(2 * l) * Ms;
       float* ssq_mlp = ssq_attn + Ms;
       TRY(layer_qkv(c, s, 1, l, c->xn_a, ssq_attn, Ms, S, P, c->q_a, c->k_s, c->v_s));
-      TRY(run_attn(c, s, c->q_a, S, kl, vl, P, c->k_s, c->v_s, S, c->o_a, B, 1, 1));
+      const int e0 = probe_begin(c, s, DM0_SITE_ACT_ATTN);
+      TRY(run_attn(c, s, c->q_a, S, kl, vl, P, c->k_s, c->v_s, S, c->o_a, B, 0, 1));
+      probe_end(c, s, DM0_SITE_ACT_ATTN, e0);
       const bool more = l + 1 < L;
       TRY(layer_rest(c, s, 1, l, Ms, c->h_a, c->xn_a, c->o_a, c->act_a, ssq_mlp,
                      more ? c->lw[1][l + 1].attn_norm : nullptr, more ? ssq_mlp + Ms : nullptr));
@@ -509,7 +555,7 @@ dm0_status enqueue_denoise(dm0_ctx* c, cudaStream_t s, int steps, float* vel) {
 }
 
 dm0_status denoise_from_x(dm0_ctx* c, cudaStream_t s, int steps, float* vel) {
-  if (vel || !c->use_graph) return enqueue_denoise(c, s, steps, vel);
+  if (vel || !c->use_graph || c->probe_mask) return enqueue_denoise(c, s, steps, vel);
   const auto key = std::make_tuple(c->kv_B, c->kv_P, steps);
   auto it = c->graphs.find(key);
   if (it == c->graphs.end()) {
@@ -736,6 +782,9 @@ dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
   bool ok = smem_attr(dm0::gemm_tc_kernel<64, kGemmStages>, dm0::GemmSmem<64, kGemmStages>::kBytes) &&
             smem_attr(dm0::gemm_tc_kernel<128, kGemmStages>, dm0::GemmSmem<128, kGemmStages>::kBytes) &&
             smem_attr(dm0::gemm_tc_kernel<256, kGemmStages>, dm0::GemmSmem<256, kGemmStages>::kBytes) &&
+            smem_attr(dm0::gemm_tc_persistent<64, kGemmStages>, dm0::PGemmSmem<64, kGemmStages>::kBytes) &&
+            smem_attr(dm0::gemm_tc_persistent<128, kGemmStages>, dm0::PGemmSmem<128, kGemmStages>::kBytes) &&
+            smem_attr(dm0::gemm_tc_persistent<256, kGemmStages>, dm0::PGemmSmem<256, kGemmStages>::kBytes) &&
             smem_attr(dm0::attn_kernel<128>, dm0::AttnSmem<128>::kBytes) &&
             smem_attr(dm0::attn_kernel<64>, dm0::AttnSmem<64>::kBytes) &&
             smem_attr(dm0::attn_kernel<32>, dm0::AttnSmem<32>::kBytes) &&
@@ -870,7 +919,7 @@ dm0_status dm0_merged_layer(dm0_ctx* c, int layer, const float* h_prefix, const 
   TRY(layer_qkv(c, s, 1, layer, c->xn_a, c->ssq_a, Ms, S, P, c->q_a, c->k_s, c->v_s));
   // the block mask: prefix rows see the prefix; suffix rows see prefix and suffix
   TRY(run_attn(c, s, c->q_v, P, kp, vp, P, nullptr, nullptr, 0, c->o_v, B, 1, 0));
-  TRY(run_attn(c, s, c->q_a, S, kp, vp, P, c->k_s, c->v_s, S, c->o_a, B, 1, 0));
+  TRY(run_attn(c, s, c->q_a, S, kp, vp, P, c->k_s, c->v_s, S, c->o_a, B, 0, 0));
   TRY(layer_rest(c, s, 0, layer, Mp, c->h_v, c->xn_v, c->o_v, c->act_v, c->ssq_v + Mp, nullptr, nullptr));
   TRY(layer_rest(c, s, 1, layer, Ms, c->h_a, c->xn_a, c->o_a, c->act_a, c->ssq_a + Ms, nullptr, nullptr));
   CK(cudaMemcpyAsync(out_prefix, c->h_v, static_cast<size_t>(Mp) * g.hidden_v * 4, cudaMemcpyDeviceToDevice, s));
@@ -924,27 +973,29 @@ dm0_status dm0_debug_view(dm0_ctx* c, const char* name, void** ptr) {
 
 uint64_t dm0_launch_count(const dm0_ctx* c) { return c ? c->launches : 0; }
 
-dm0_status dm0_probe(dm0_ctx* c, int kind) {
+dm0_status dm0_probe(dm0_ctx* c, int site_mask) {
   if (!c) return DM0_EINVAL;
-  if (kind < 0 || kind > 1) return fail(c, DM0_EINVAL, "unknown probe kind");
-  c->probe = kind;
+  if (site_mask < 0 || site_mask >= (1 << DM0_SITE_COUNT)) return fail(c, DM0_EINVAL, "unknown probe site");
+  c->probe_mask = site_mask;
   c->probe_used = 0;
+  c->probe_recs.clear();
   return DM0_OK;
 }
 
-dm0_status dm0_probe_read(dm0_ctx* c, int* launches, double* total_ms) {
+dm0_status dm0_probe_read(dm0_ctx* c, int site, int* launches, double* total_ms) {
   if (!c || !launches || !total_ms) return fail(c, DM0_EINVAL, "null argument");
   double tot = 0.0;
-  const size_t pairs = c->probe_used / 2;
-  for (size_t i = 0; i < pairs; ++i) {
-    CK(cudaEventSynchronize(c->probe_ev[2 * i + 1]));
+  int n = 0;
+  for (const auto& r : c->probe_recs) {
+    if (r.site != site) continue;
+    CK(cudaEventSynchronize(c->probe_ev[r.e1]));
     float ms = 0.f;
-    CK(cudaEventElapsedTime(&ms, c->probe_ev[2 * i], c->probe_ev[2 * i + 1]));
+    CK(cudaEventElapsedTime(&ms, c->probe_ev[r.e0], c->probe_ev[r.e1]));
     tot += ms;
+    ++n;
   }
-  *launches = static_cast<int>(pairs);
+  *launches = n;
   *total_ms = tot;
-  c->probe_used = 0;
   return DM0_OK;
 }
 

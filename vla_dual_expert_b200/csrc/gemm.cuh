@@ -459,3 +459,192 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
 }
 
 }  // namespace dm0
+
+namespace dm0 {
+
+// ---------------------------------------------------------------- persistent normal-orientation GEMM
+//
+// One CTA per SM walks output tiles t = blockIdx.x,
+// blockIdx.x + gridDim.x, ...; tile t is (m = t % m_tiles, n = t / m_tiles), so
+// CTAs running together share a weight tile in L2.  The producer streams
+// k-blocks of consecutive tiles through one ring without pausing between tiles,
+// and the accumulator is double-buffered in TMEM (2 x BN columns): while the
+// epilogue warps finish tile i from one buffer, the MMA warp already
+// accumulates tile i+1 into the other.
+template <int BN, int STAGES>
+struct PGemmSmem {
+  static constexpr uint32_t kA = 128 * 128;
+  static constexpr uint32_t kB = BN * 128;
+  static constexpr uint32_t kStage = kA + kB;
+  static constexpr uint32_t kPipe = STAGES * kStage;
+  static constexpr uint32_t kBytes = kPipe + 256 + 1024;
+  static constexpr uint32_t kTmemCols = 2 * BN;
+};
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                       const GemmArgs a) {
+  using L = PGemmSmem<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kPipe);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;   // [2] accumulator buffer complete
+  uint64_t* tempty = tfull + 2;       // [2] epilogue finished with the buffer
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int KB = (a.K + 63) >> 6;
+  const int mt = (a.M + 127) >> 7;
+  const int ntiles = mt * (a.N / BN);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_launch_dependents();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+      const uint64_t pol_w = policy_evict_last();   // a weight tile is shared by the CTAs running together
+      const uint64_t pol_x = policy_evict_first();
+      int it = 0;
+      bool waited = false;
+      // the first tile's weight k-blocks may be requested before the dependency wait
+      const int first = blockIdx.x;
+      int pre = 0;
+      if (a.w_stable && first < ntiles) {
+        pre = KB < STAGES ? KB : STAGES;
+        const int n0 = first / mt;
+        for (int k = 0; k < pre; ++k) {
+          mbar_arrive_expect_tx(&full[k], L::kStage);
+          tma_load_2d(smem + k * L::kStage + L::kA, &tmB, &full[k], k * 64, n0 * BN, pol_w);
+        }
+      }
+      pdl_wait();
+      waited = true;
+      (void)waited;
+      for (int t = first; t < ntiles && !*abort_flag; t += gridDim.x) {
+        const int m0 = (t % mt) * 128, n0 = (t / mt) * BN;
+        for (int k = 0; k < KB; ++k, ++it) {
+          const int s = it % STAGES;
+          if (it < pre) {   // weight half already requested
+            tma_load_2d(smem + s * L::kStage, &tmA, &full[s], k * 64, m0, pol_x);
+            continue;
+          }
+          if (it >= STAGES && !mbar_wait(&empty[s], ((it / STAGES) - 1) & 1, abort_flag)) {
+            *abort_flag = 1;
+            raise_error(a.err, kErrTimeoutProducer);
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], L::kStage);
+          tma_load_2d(smem + s * L::kStage, &tmA, &full[s], k * 64, m0, pol_x);
+          tma_load_2d(smem + s * L::kStage + L::kA, &tmB, &full[s], k * 64, n0, pol_w);
+        }
+      }
+      for (int i = it - STAGES; i < it; ++i) {   // copies in flight land before the CTA exits
+        if (i < 0) continue;
+        if (!mbar_wait(&full[i % STAGES], (i / STAGES) & 1, nullptr, kDrainTimeoutNs)) raise_error(a.err, kErrDrain);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, BN);
+      int it = 0, local = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x, ++local) {
+        const int buf = local & 1;
+        if (local >= 2 && !mbar_wait(&tempty[buf], ((local >> 1) - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int k = 0; k < KB; ++k, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(&full[s], (it / STAGES) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * L::kStage);
+          const uint32_t b_addr = a_addr + L::kA;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(tmem + buf * BN, sw128_kmajor_desc(a_addr + 32 * kk), sw128_kmajor_desc(b_addr + 32 * kk),
+                      idesc, (k | kk) != 0 ? 1u : 0u);
+          umma_commit(&empty[s]);
+        }
+        if (ok) umma_commit(&tfull[buf]);
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        raise_error(a.err, kErrTimeoutMma);
+      }
+      umma_commit(drain);
+      if (!mbar_wait(drain, 0, nullptr, kWaitTimeoutNs + kDrainTimeoutNs)) raise_error(a.err, kErrDrain);
+    }
+  } else {
+    const int lane_base = (warp & 3) * 32;
+    pdl_wait();
+    int local = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++local) {
+      const int buf = local & 1;
+      if (!mbar_wait(&tfull[buf], (local >> 1) & 1, abort_flag)) {
+        *abort_flag = 1;
+        raise_error(a.err, kErrTimeoutEpilogue);
+        break;
+      }
+      tc_fence_after();
+      const int m_tile = t % mt, n_tile = t / mt;
+      const uint32_t tl = tmem + (static_cast<uint32_t>(lane_base) << 16) + buf * BN;
+      const int tok = m_tile * 128 + lane_base + lane;
+      const bool valid = tok < a.M;
+      float ssq_acc = 0.f;
+      if (BN >= 128) {
+        for (int g = 0; g < BN / 128; ++g) {
+          const uint32_t tg = tl + g * 128;
+          row_epilogue<false>(a, tok, valid, n_tile * BN + g * 128, ssq_acc,
+                              [&](int c, float (&v)[32]) { tmem_ld32(tg + c * 32, v); });
+        }
+      } else {
+        row_epilogue<false>(a, tok, valid, n_tile * BN, ssq_acc,
+                            [&](int c, float (&v)[32]) { tmem_ld32(tl + c * 32, v); }, BN / 32);
+      }
+      if (a.mode == kModeResid && a.ssq_out && valid) atomicAdd(a.ssq_out + tok, ssq_acc);
+      // the accumulator buffer is free for tile local + 2
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[buf]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+}  // namespace dm0
