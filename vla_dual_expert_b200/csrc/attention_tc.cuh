@@ -29,21 +29,27 @@ namespace dm0 {
 
 constexpr int kFaThreads = 192;
 
-struct FaSmem {
+template <int ST>
+struct FaSmemT {
   static constexpr int kKeys = 64;                          // keys per block
   static constexpr uint32_t kQ = 32768;                     // 128 rows x 128 dims: two 64-column SW128 halves
   static constexpr uint32_t kKV = 16384;                    // 64 keys x 128 dims: two 8 KB SW128 halves
   static constexpr uint32_t kHalfKV = 8192;
   static constexpr uint32_t kP = 16384;                     // 128 rows x 64 keys, one SW128 block
-  static constexpr int kStages = 2;                         // K/V blocks in flight
+  static constexpr int kStages = ST;                        // K/V blocks in flight
   static constexpr uint32_t kOffQ = 0;
   static constexpr uint32_t kOffK = kOffQ + kQ;
   static constexpr uint32_t kOffV = kOffK + kStages * kKV;
   static constexpr uint32_t kOffP = kOffV + kStages * kKV;
-  static constexpr uint32_t kOffBar = kOffP + kP;           // 114688
+  static constexpr uint32_t kOffBar = kOffP + kP;
   static constexpr uint32_t kSlack = 256;                   // the dynamic base is 1024-aligned (no static smem)
   static constexpr uint32_t kBytes = kOffBar + 256 + kSlack;
 };
+// two stages (112 KB): two CTAs per SM, for the prefix pass whose K/V blocks are shared by many
+// CTAs through L2; five stages (208 KB): one CTA per SM with deeper prefetch, for the suffix
+// attention whose cached prefix K/V is read from DRAM once
+using FaSmem = FaSmemT<2>;
+constexpr int kFaDeepStages = 5;
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
   asm volatile(
@@ -84,26 +90,28 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int col) {
   return half * 16384 + row * 128 + ((c16 ^ (row & 7)) << 4) + ((col & 7) << 1);
 }
 
-__global__ void __launch_bounds__(kFaThreads, 2)
+template <int ST>
+__global__ void __launch_bounds__(kFaThreads, ST <= 2 ? 2 : 1)
     fa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const __grid_constant__ CUtensorMap tmKb, const __grid_constant__ CUtensorMap tmVb, const AttnArgs a) {
   constexpr int D = 128;
+  using FS = FaSmemT<ST>;
   extern __shared__ uint8_t fa_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fa_smem_raw) + 1023) & ~uintptr_t(1023));
-  if (smem - fa_smem_raw > static_cast<ptrdiff_t>(FaSmem::kSlack)) {   // never expected: refuse rather than overrun
+  if (smem - fa_smem_raw > static_cast<ptrdiff_t>(FS::kSlack)) {   // never expected: refuse rather than overrun
     if (threadIdx.x == 0) raise_error(a.err, kErrBounds);
     return;
   }
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + FaSmem::kOffBar);
-  uint64_t* kv_full = bars;        // [2] TMA landed K_j, V_j
-  uint64_t* kv_empty = bars + 2;   // [2] PV_j done: K/V slot free
-  uint64_t* s_full = bars + 4;     // [2] S_j in TMEM
-  uint64_t* s_free = bars + 6;     // [2] softmax finished reading S_j
-  uint64_t* p_full = bars + 8;     // P_j in smem and O corrected (one phase per block)
-  uint64_t* pv_done = bars + 9;    // PV_j finished (one phase per block)
-  uint64_t* q_ready = bars + 10;
-  uint64_t* drain = bars + 11;     // every issued MMA complete (before TMEM is released)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + FS::kOffBar);
+  uint64_t* kv_full = bars;             // [ST] TMA landed K_j, V_j
+  uint64_t* kv_empty = bars + ST;       // [ST] PV_j done: K/V slot free
+  uint64_t* s_full = bars + 2 * ST;     // [2] S_j in TMEM
+  uint64_t* s_free = s_full + 2;        // [2] softmax finished reading S_j
+  uint64_t* p_full = s_free + 2;        // P_j in smem and O corrected (one phase per block)
+  uint64_t* pv_done = p_full + 1;       // PV_j finished (one phase per block)
+  uint64_t* q_ready = pv_done + 1;
+  uint64_t* drain = q_ready + 1;        // every issued MMA complete (before TMEM is released)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -119,9 +127,11 @@ __global__ void __launch_bounds__(kFaThreads, 2)
   const int nblk = jb1 - jb0;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < ST; ++i) {
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 4);
     }
@@ -153,29 +163,29 @@ __global__ void __launch_bounds__(kFaThreads, 2)
       }
       const uint64_t pol = policy_evict_last();
       auto issue = [&](int j) {
-        const int s = j & 1;
+        const int s = j % ST;
         const int jj = jb0 + j;   // global block index
         const bool segA = jj < nA;
         const CUtensorMap* mk = segA ? &tmK : &tmKb;
         const CUtensorMap* mv = segA ? &tmV : &tmVb;
         const int row = segA ? grp * a.len_a + jj * 64 : grp * a.len_b + (jj - nA) * 64;
-        mbar_arrive_expect_tx(&kv_full[s], 2 * FaSmem::kKV);
-        uint8_t* kd = smem + FaSmem::kOffK + s * FaSmem::kKV;
-        uint8_t* vd = smem + FaSmem::kOffV + s * FaSmem::kKV;
+        mbar_arrive_expect_tx(&kv_full[s], 2 * FS::kKV);
+        uint8_t* kd = smem + FS::kOffK + s * FS::kKV;
+        uint8_t* vd = smem + FS::kOffV + s * FS::kKV;
         tma_load_2d(kd, mk, &kv_full[s], 0, row, pol);
-        tma_load_2d(kd + FaSmem::kHalfKV, mk, &kv_full[s], 64, row, pol);
+        tma_load_2d(kd + FS::kHalfKV, mk, &kv_full[s], 64, row, pol);
         tma_load_2d(vd, mv, &kv_full[s], 0, row, pol);
-        tma_load_2d(vd + FaSmem::kHalfKV, mv, &kv_full[s], 64, row, pol);
+        tma_load_2d(vd + FS::kHalfKV, mv, &kv_full[s], 64, row, pol);
       };
       // segment A written before the previous kernel (the prefix cache during the Euler loop) may be
       // requested before the dependency wait
       int issued = 0;
       if (a.a_stable)
-        for (; issued < 2 && issued < nblk && jb0 + issued < nA; ++issued) issue(issued);
+        for (; issued < ST && issued < nblk && jb0 + issued < nA; ++issued) issue(issued);
       pdl_wait();
       for (int j = issued; j < nblk; ++j) {
-        const int s = j & 1;
-        if (j >= 2 && !mbar_wait(&kv_empty[s], ((j >> 1) - 1) & 1, abort_flag)) {
+        const int s = j % ST;
+        if (j >= ST && !mbar_wait(&kv_empty[s], ((j / ST) - 1) & 1, abort_flag)) {
           *abort_flag = 1;
           raise_error(a.err, kErrTimeoutProducer);
           break;
@@ -183,9 +193,9 @@ __global__ void __launch_bounds__(kFaThreads, 2)
         issue(j);
         issued = j + 1;
       }
-      for (int j = issued - 2; j < issued; ++j) {   // copies in flight land before the CTA exits
+      for (int j = issued - ST; j < issued; ++j) {   // copies in flight land before the CTA exits
         if (j < 0) continue;
-        if (!mbar_wait(&kv_full[j & 1], (j >> 1) & 1, nullptr, kDrainTimeoutNs)) raise_error(a.err, kErrDrain);
+        if (!mbar_wait(&kv_full[j % ST], (j / ST) & 1, nullptr, kDrainTimeoutNs)) raise_error(a.err, kErrDrain);
       }
     }
   } else if (warp == 1) {
@@ -193,24 +203,25 @@ __global__ void __launch_bounds__(kFaThreads, 2)
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(128, 64);
       const uint32_t idesc_pv = idesc_bf16_f32(128, 128) | (1u << 16);   // B (V) is MN-major
-      const uint32_t qa = smem_u32(smem + FaSmem::kOffQ);
+      const uint32_t qa = smem_u32(smem + FS::kOffQ);
       bool ok = mbar_wait(q_ready, 0, abort_flag);
       auto pv = [&](int i) -> bool {
         if (!mbar_wait(p_full, i & 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t pa = smem_u32(smem + FaSmem::kOffP);
-        const uint32_t vb = smem_u32(smem + FaSmem::kOffV + (i & 1) * FaSmem::kKV);
+        const uint32_t pa = smem_u32(smem + FS::kOffP);
+        const uint32_t vb = smem_u32(smem + FS::kOffV + (i % ST) * FS::kKV);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          umma_bf16(tmem + 128, sw128_kmajor_desc(pa + ks * 32), sw128_mnmajor_desc(vb + ks * 2048, FaSmem::kHalfKV),
+          umma_bf16(tmem + 128, sw128_kmajor_desc(pa + ks * 32), sw128_mnmajor_desc(vb + ks * 2048, FS::kHalfKV),
                     idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
         umma_commit(pv_done);
-        umma_commit(&kv_empty[i & 1]);
+        umma_commit(&kv_empty[i % ST]);
         return true;
       };
       for (int j = 0; ok && j < nblk; ++j) {
-        const int s = j & 1;
-        if (!mbar_wait(&kv_full[s], (j >> 1) & 1, abort_flag)) {
+        const int s = j & 1;          // S buffer
+        const int kvs = j % ST;       // K/V slot
+        if (!mbar_wait(&kv_full[kvs], (j / ST) & 1, abort_flag)) {
           ok = false;
           break;
         }
@@ -219,11 +230,11 @@ __global__ void __launch_bounds__(kFaThreads, 2)
           break;
         }
         tc_fence_after();
-        const uint32_t kb = smem_u32(smem + FaSmem::kOffK + s * FaSmem::kKV);
+        const uint32_t kb = smem_u32(smem + FS::kOffK + kvs * FS::kKV);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
           umma_bf16(tmem + s * 64, sw128_kmajor_desc(qa + (ks >> 2) * 16384 + (ks & 3) * 32),
-                    sw128_kmajor_desc(kb + (ks >> 2) * FaSmem::kHalfKV + (ks & 3) * 32), idesc_s, ks > 0 ? 1u : 0u);
+                    sw128_kmajor_desc(kb + (ks >> 2) * FS::kHalfKV + (ks & 3) * 32), idesc_s, ks > 0 ? 1u : 0u);
         umma_commit(&s_full[s]);
         if (j >= 1 && !pv(j - 1)) {
           ok = false;
@@ -251,7 +262,7 @@ __global__ void __launch_bounds__(kFaThreads, 2)
     pdl_wait();
     {   // Q row -> shared memory in the SW128 K-major layout
       const uint4* src = reinterpret_cast<const uint4*>(a.q + ((static_cast<size_t>(b) * a.seq_q + pos) * a.n_q + head) * D);
-      uint8_t* qs = smem + FaSmem::kOffQ;
+      uint8_t* qs = smem + FS::kOffQ;
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
         const uint4 v = valid ? src[c] : make_uint4(0, 0, 0, 0);
@@ -345,7 +356,7 @@ __global__ void __launch_bounds__(kFaThreads, 2)
           tmem_wait_st();
         }
       }
-      uint8_t* ps = smem + FaSmem::kOffP;   // one buffer: PV_{j-1} has completed
+      uint8_t* ps = smem + FS::kOffP;   // one buffer: PV_{j-1} has completed
 #pragma unroll
       for (int c = 0; c < 8; ++c)
         *reinterpret_cast<uint4*>(ps + sw128_off(r, c * 8)) =

@@ -356,9 +356,11 @@ dm0_status run_attn(dm0_ctx* c, cudaStream_t s, const bf16* q, int seq_q, const 
     // tcgen05 flash attention, K/V tiles of both segments by TMA; keys split in 64-key blocks
     const int fblk = (len_a + 63) / 64 + (len_b + 63) / 64;
     int fs = splits_req;
-    if (fs <= 0) {   // about two CTAs per SM, at most 4 splits (the combine reads every split's partial O)
+    if (fs <= 0) {   // fill the SMs once (two CTAs per SM for the prefix kernel, one for the deep suffix
+                     // kernel), at most 4 splits: the combine reads every split's partial O
       const int ctas = groups * tiles;
-      fs = std::max(1, std::min(4, (2 * c->num_sms + ctas / 2) / ctas));
+      const int slots = (len_b == 0 ? 2 : 1) * c->num_sms;
+      fs = std::max(1, std::min(4, (slots + ctas / 2) / ctas));
     }
     fs = std::min(fs, fblk);
     while (fs > 1 && groups * tiles * fs > kPartSlots) --fs;
@@ -377,8 +379,13 @@ dm0_status run_attn(dm0_ctx* c, cudaStream_t s, const bf16* q, int seq_q, const 
       tkb = tk;
       tvb = tv;
     }
-    return launch(c, s, dm0::fa_tc_kernel, dim3(tiles, groups, fs), dim3(dm0::kFaThreads), dm0::FaSmem::kBytes, tk,
-                  tv, tkb, tvb, a);
+    const dim3 grid(tiles, groups, fs);
+    if (len_b == 0)   // prefix pass: K/V blocks shared by many CTAs through L2, two CTAs per SM
+      return launch(c, s, dm0::fa_tc_kernel<2>, grid, dim3(dm0::kFaThreads), dm0::FaSmemT<2>::kBytes, tk, tv, tkb,
+                    tvb, a);
+    // merged suffix attention: the cached prefix is read from DRAM once, deeper K/V prefetch
+    return launch(c, s, dm0::fa_tc_kernel<dm0::kFaDeepStages>, grid, dim3(dm0::kFaThreads),
+                  dm0::FaSmemT<dm0::kFaDeepStages>::kBytes, tk, tv, tkb, tvb, a);
   }
   const dim3 grid(tiles, groups, splits);
   switch (g.head_dim) {
@@ -788,7 +795,8 @@ dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
             smem_attr(dm0::attn_kernel<128>, dm0::AttnSmem<128>::kBytes) &&
             smem_attr(dm0::attn_kernel<64>, dm0::AttnSmem<64>::kBytes) &&
             smem_attr(dm0::attn_kernel<32>, dm0::AttnSmem<32>::kBytes) &&
-            smem_attr(dm0::fa_tc_kernel, dm0::FaSmem::kBytes);
+            smem_attr(dm0::fa_tc_kernel<2>, dm0::FaSmemT<2>::kBytes) &&
+            smem_attr(dm0::fa_tc_kernel<dm0::kFaDeepStages>, dm0::FaSmemT<dm0::kFaDeepStages>::kBytes);
   if (!ok) return bail(DM0_ECUDA);
   *out = c;
   return DM0_OK;

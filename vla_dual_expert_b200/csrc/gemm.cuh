@@ -464,13 +464,27 @@ namespace dm0 {
 
 // ---------------------------------------------------------------- persistent normal-orientation GEMM
 //
-// One CTA per SM walks output tiles t = blockIdx.x,
-// blockIdx.x + gridDim.x, ...; tile t is (m = t % m_tiles, n = t / m_tiles), so
-// CTAs running together share a weight tile in L2.  The producer streams
+// One CTA per SM walks output tiles t = blockIdx.x, blockIdx.x + gridDim.x, ...
+// in a banded raster: bands of kBandM m-tiles, m fastest inside a band, so the
+// CTAs running together cover a few weight tiles and at most kBandM activation
+// tiles; both stay in L2 while the band is worked (activation tiles are read
+// from DRAM once, weights once per band).  The producer streams
 // k-blocks of consecutive tiles through one ring without pausing between tiles,
 // and the accumulator is double-buffered in TMEM (2 x BN columns): while the
 // epilogue warps finish tile i from one buffer, the MMA warp already
 // accumulates tile i+1 into the other.
+constexpr int kBandM = 64;   // m-tiles per raster band (64 x 128 rows x K bf16 stays L2-resident)
+
+// output tile index t -> (m_tile, n_tile) in the banded raster
+__device__ __forceinline__ void band_tile(int t, int mt, int nt, int& m_tile, int& n_tile) {
+  const int band = t / (kBandM * nt);
+  const int m0 = band * kBandM;
+  const int bm = min(kBandM, mt - m0);   // m-tiles in this band
+  const int r = t - band * kBandM * nt;
+  m_tile = m0 + r % bm;
+  n_tile = r / bm;
+}
+
 template <int BN, int STAGES>
 struct PGemmSmem {
   static constexpr uint32_t kA = 128 * 128;
@@ -537,7 +551,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int pre = 0;
       if (a.w_stable && first < ntiles) {
         pre = KB < STAGES ? KB : STAGES;
-        const int n0 = first / mt;
+        int m_first, n0;
+        band_tile(first, mt, a.N / BN, m_first, n0);
         for (int k = 0; k < pre; ++k) {
           mbar_arrive_expect_tx(&full[k], L::kStage);
           tma_load_2d(smem + k * L::kStage + L::kA, &tmB, &full[k], k * 64, n0 * BN, pol_w);
@@ -547,7 +562,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       waited = true;
       (void)waited;
       for (int t = first; t < ntiles && !*abort_flag; t += gridDim.x) {
-        const int m0 = (t % mt) * 128, n0 = (t / mt) * BN;
+        int mtile, ntile;
+        band_tile(t, mt, a.N / BN, mtile, ntile);
+        const int m0 = mtile * 128, n0 = ntile * BN;
         for (int k = 0; k < KB; ++k, ++it) {
           const int s = it % STAGES;
           if (it < pre) {   // weight half already requested
@@ -617,7 +634,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after();
-      const int m_tile = t % mt, n_tile = t / mt;
+      int m_tile, n_tile;
+      band_tile(t, mt, a.N / BN, m_tile, n_tile);
       const uint32_t tl = tmem + (static_cast<uint32_t>(lane_base) << 16) + buf * BN;
       const int tok = m_tile * 128 + lane_base + lane;
       const bool valid = tok < a.M;
