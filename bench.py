@@ -32,6 +32,10 @@ sys.path.insert(0, ROOT)
 
 METRIC = "action chunks/sec (prefill+10-step denoise) at batch 1 and 16; HBM GB/s, TC util"
 EULER_STEPS = 10
+# DRAM bytes (read + write) of one prefix-pass gate/up GEMM launch at B=16, P=2048 (M=32768,
+# N=12288, K=2048), from the ncu capture of the same kernel and launch shape summarised in
+# profiles/gemm_tc_persistent_gateup_M32768.md (3.167 GB read + 0.352 GB written)
+GATEUP_TRAFFIC_BYTES = 3.519e9
 
 
 def _peaks():
@@ -263,7 +267,9 @@ def run_native(args, rank, world, local_rank):
         "prefill_ms_p90": round(main["prefill_ms_p90"], 3), "denoise_ms_p90": round(main["denoise_ms_p90"], 3),
         "roofline": {"bound": "tensor", "kernel": "gemm_tc_kernel<256> (prefill gate/up, M=B*P, N=2*6144, K=2048)",
                      "achieved": round(gu_tf, 1), "peak": tc_peak, "unit": "TFLOP/s",
-                     "frac": round(gu_tf / tc_peak, 4), "traffic": None,
+                     "frac": round(gu_tf / tc_peak, 4),
+                     "traffic": GATEUP_TRAFFIC_BYTES if (B, P) == (16, 2048) else None,
+                     "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
                      "peak_src": f"{peaks['src']} bf16_tflops_sustained", "launches": main["probe_n"],
                      "avg_launch_ms": round(gu_ms, 4)},
         "e2e": {"value": round(world * B * 1000.0 / e2e["ms"], 3), "unit": "chunks/s",
@@ -371,6 +377,29 @@ def run_reference(args, rank, world):
     print(json.dumps(res), flush=True)
 
 
+def run_one_layer(args):
+    """Profiling workload: one DM0-base layer (both experts) at B=16, P=2048 — two iterations of
+    dm0_prefill + a 1-step dm0_denoise with per-step velocities (direct launches).  Holds about 2 GB
+    on the device, small enough for full ncu captures of every kernel of the step."""
+    import torch
+
+    from synth import inputs as I
+    from vla_dual_expert_b200 import Engine
+    d = I.DM0_BASE.replace(layers=1)
+    B, P = 16, 2048
+    eng = Engine(d, B, P)
+    eng.load_from(I.Weights(d, seed=0))
+    emb = torch.from_numpy(I.prefix_embeddings(d, B, P)).cuda().to(torch.bfloat16)
+    noise = torch.from_numpy(I.noise(d, B)).cuda()
+    vel = torch.empty((1, B, d.chunk, d.action_dim), device="cuda", dtype=torch.float32)
+    for _ in range(2):
+        eng.prefill(emb)
+        eng.denoise(noise, 1, velocities=vel)
+    eng.sync()
+    print(json.dumps({"one_layer": "ok", "mean_abs_velocity": float(vel.abs().mean())}))
+    eng.close()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -382,6 +411,7 @@ def main():
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-breakdown", action="store_true")
+    ap.add_argument("--one-layer", action="store_true", help="profiling workload: one layer, B=16, P=2048")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "native":
@@ -391,6 +421,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.one_layer:
+        run_one_layer(args)
         return
     run_native(args, rank, world, local_rank)
 
