@@ -123,6 +123,23 @@ def denoise_bytes_per_step(d, B, P):
     return w + kv
 
 
+# ------------------------------------------------------------------ rank plumbing
+
+def max_over_ranks(x: float, dist=None, device=None) -> float:
+    """The slowest rank's time (every rank calls this in the same order)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_chunks_per_s(world: int, batch_per_rank: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank runs its own batch (weak scaling, no cross-rank data)."""
+    return world * batch_per_rank * 1000.0 / ms_per_step
+
+
 # ------------------------------------------------------------------ native arm
 
 def run_native(args, rank, world, local_rank):
@@ -145,12 +162,8 @@ def run_native(args, rank, world, local_rank):
         if dist is not None:
             dist.barrier()
 
-    def max_over_ranks(x):
-        if dist is None:
-            return x
-        t = torch.tensor([x], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def rank_max(x):
+        return max_over_ranks(x, dist, "cuda")
 
     d = I.DM0_BASE
     wl_main = I.WORKLOADS[args.workload]
@@ -192,7 +205,7 @@ def run_native(args, rank, world, local_rank):
         probe_n, probe_ms = eng.probe_read(probe) if probe is not None else (0, 0.0)
         eng.probe(0)
         eng.sync()
-        ms = max_over_ranks(t0.elapsed_time(t1) / steps)
+        ms = rank_max(t0.elapsed_time(t1) / steps)
         pre = sorted(e[0].elapsed_time(e[1]) for e in ev)
         den = sorted(e[1].elapsed_time(e[2]) for e in ev)
         assert bool(torch.isfinite(out).all())
@@ -242,7 +255,7 @@ def run_native(args, rank, world, local_rank):
         t1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        ms = max_over_ranks(t0.elapsed_time(t1) / steps)
+        ms = rank_max(t0.elapsed_time(t1) / steps)
         return {"ms": ms, "h2d": emb_h.numel() * 2 + noise_h.numel() * 4, "d2h": out_h.numel() * 4}
 
     # probe site 3 = the VLM gate/up GEMM of the prefix pass (the largest launch of the step)
@@ -250,7 +263,7 @@ def run_native(args, rank, world, local_rank):
     e2e = measure_e2e(wl_main, max(2, args.steps // 2), 1) if not args.skip_e2e else {"ms": float("nan"), "h2d": 0,
                                                                                         "d2h": 0}
     B, P = wl_main.batch, wl_main.prefix
-    value = world * B * 1000.0 / main["ms"]
+    value = job_chunks_per_s(world, B, main["ms"])
     gu_ms = main["probe_ms"] / max(main["probe_n"], 1)
     gu_tf = prefill_gateup_flops(d, B, P) / (gu_ms * 1e-3) / 1e12
     tc_peak = peaks["bf16_tflops_sustained"]
@@ -272,7 +285,7 @@ def run_native(args, rank, world, local_rank):
                      "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
                      "peak_src": f"{peaks['src']} bf16_tflops_sustained", "launches": main["probe_n"],
                      "avg_launch_ms": round(gu_ms, 4)},
-        "e2e": {"value": round(world * B * 1000.0 / e2e["ms"], 3), "unit": "chunks/s",
+        "e2e": {"value": round(job_chunks_per_s(world, B, e2e["ms"]), 3), "unit": "chunks/s",
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
         "gpu_launches": main["launches"],
         "clocks": main["clocks"],
@@ -282,7 +295,8 @@ def run_native(args, rank, world, local_rank):
         b1 = measure(wl1, max(args.steps, 5), args.warmup, probe=None)
         den_gbs = denoise_bytes_per_step(d, 1, wl1.prefix) * EULER_STEPS / (b1["denoise_ms_p50"] * 1e-3) / 1e9
         result["batch1"] = {
-            "workload": "e2e_b1: prefill B=1 x P=816 + 10-step denoise", "value": round(world * 1000.0 / b1["ms"], 3),
+            "workload": "e2e_b1: prefill B=1 x P=816 + 10-step denoise",
+            "value": round(job_chunks_per_s(world, 1, b1["ms"]), 3),
             "unit": "chunks/s", "ms_per_step": round(b1["ms"], 3), "prefill_ms_p50": round(b1["prefill_ms_p50"], 3),
             "denoise_ms_p50": round(b1["denoise_ms_p50"], 3), "denoise_ms_p90": round(b1["denoise_ms_p90"], 3),
             "gpu_launches": b1["launches"],

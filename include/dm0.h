@@ -247,6 +247,14 @@ dm0_status dm0_probe(dm0_ctx* ctx, int site_mask);
  * launches and their summed duration in milliseconds. */
 dm0_status dm0_probe_read(dm0_ctx* ctx, int site, int* launches, double* total_ms);
 
+/* Failure-path self-test (no counterpart on the pages): launches a kernel
+ * whose bounded mbarrier wait — the same wait every pipeline of the library
+ * uses — is given an mbarrier nothing ever arrives on.  The wait gives up
+ * after `limit_us` microseconds (1..1e6), the kernel sets the device error
+ * word and returns; dm0_sync then reports DM0_EDEVICE and dm0_clear_error
+ * makes the context usable again.  Asynchronous on `stream`. */
+dm0_status dm0_selftest_timeout(dm0_ctx* ctx, int limit_us, void* stream);
+
 /* Errors and lifetime. -------------------------------------------------- */
 
 /* Wait for `stream`, then report DM0_EDEVICE if a kernel raised the device

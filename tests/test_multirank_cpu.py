@@ -1,0 +1,71 @@
+"""The multi-GPU path of bench.py on CPU: two gloo ranks.
+
+The method shards by sample (independent chunks, per-sample KV cache), so
+`bench.py --gpus N` runs one replica per GPU on its own batch and the only
+cross-rank steps are the barrier and the max-over-ranks timing reduction.
+These tests run exactly that reduction with the gloo backend and check the
+job throughput every rank reports, plus the reference arm's rank handling.
+"""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(rank, world, port, times, out):
+    import datetime
+
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        dist.barrier()
+        ms = bench.max_over_ranks(times[rank], dist, "cpu")
+        out.put((rank, ms, bench.job_chunks_per_s(world, 16, ms)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_weak_scaling_value_with_gloo():
+    world, port = 2, _free_port()
+    times = [180.0, 195.5]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_rank, args=(r, world, port, times, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, ms, value in res:
+        assert ms == max(times)                       # every rank sees the slowest rank's time
+        assert value == pytest.approx(world * 16 * 1000.0 / max(times))
+
+
+def test_reference_arm_only_rank0_reports():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "0"], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_single_rank_passthrough():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(12.5) == 12.5
+    assert bench.job_chunks_per_s(1, 16, 200.0) == pytest.approx(80.0)

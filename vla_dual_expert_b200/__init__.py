@@ -165,6 +165,9 @@ class Engine:
         self._chk(self.lib.dm0_probe_read(self.h, site, ctypes.byref(n), ctypes.byref(ms)))
         return n.value, ms.value
 
+    def selftest_timeout(self, limit_us: int = 20000, stream=None):
+        self._chk(self.lib.dm0_selftest_timeout(self.h, limit_us, _stream(stream)))
+
     def sync(self, stream=None):
         self._chk(self.lib.dm0_sync(self.h, _stream(stream)))
 

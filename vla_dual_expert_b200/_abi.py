@@ -24,7 +24,7 @@ STATUS = {0: "DM0_OK", -1: "DM0_EINVAL", -2: "DM0_ESHAPE", -3: "DM0_ENOMEM", -4:
 EXPORTS = ("dm0_create", "dm0_weights_bytes", "dm0_load_weights", "dm0_prefill", "dm0_kv_view",
            "dm0_kv_commit", "dm0_denoise", "dm0_infer_host", "dm0_merged_layer", "dm0_op_gemm",
            "dm0_op_attention", "dm0_attention_noalloc", "dm0_debug_view", "dm0_launch_count", "dm0_probe",
-           "dm0_probe_read", "dm0_sync", "dm0_device_error", "dm0_clear_error", "dm0_last_error",
+           "dm0_probe_read", "dm0_selftest_timeout", "dm0_sync", "dm0_device_error", "dm0_clear_error", "dm0_last_error",
            "dm0_destroy")
 
 
@@ -71,6 +71,7 @@ def load_library() -> ctypes.CDLL:
         "dm0_launch_count": (ctypes.c_uint64, [P]),
         "dm0_probe": (c_int, [P, c_int]),
         "dm0_probe_read": (c_int, [P, c_int, ctypes.POINTER(c_int), ctypes.POINTER(ctypes.c_double)]),
+        "dm0_selftest_timeout": (c_int, [P, c_int, P]),
         "dm0_sync": (c_int, [P, P]),
         "dm0_device_error": (c_int, [P]),
         "dm0_clear_error": (c_int, [P]),

@@ -1065,6 +1065,16 @@ dm0_status dm0_attention_noalloc(const void* q, const void* ka, const void* va, 
   return cudaGetLastError() == cudaSuccess ? DM0_OK : DM0_ECUDA;
 }
 
+dm0_status dm0_selftest_timeout(dm0_ctx* c, int limit_us, void* stream) {
+  if (!c) return DM0_EINVAL;
+  if (limit_us < 1 || limit_us > 1000000) return fail(c, DM0_ESHAPE, "limit_us must be in [1, 1e6]");
+  c->pdl_ok = false;
+  dm0::wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      c->d_err, static_cast<unsigned long long>(limit_us) * 1000ull);
+  CK(cudaGetLastError());
+  return DM0_OK;
+}
+
 dm0_status dm0_sync(dm0_ctx* c, void* stream) {
   if (!c) return DM0_EINVAL;
   CK(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));

@@ -121,6 +121,18 @@ __global__ void __launch_bounds__(256) step_kernel(const StepArgs a) {
   }
 }
 
+// Failure-path self-test: one thread waits, with the library's bounded wait, on an mbarrier
+// that nothing ever arrives on.  The wait gives up after `limit_ns`, the kernel records the
+// timeout in the device error word and returns normally.
+__global__ void wait_timeout_selftest_kernel(int* err, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    if (!mbar_wait(&bar, 0, nullptr, limit_ns)) raise_error(err, kErrTimeoutProducer);
+  }
+}
+
 __global__ void rope_table_kernel(float2* tab, int max_pos, int half, double log_theta) {
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= max_pos * half) return;
