@@ -278,7 +278,7 @@ def run_native(args, rank, world, local_rank):
                    "l2": "inputs larger than L2 (3.7 GB of weights streamed per step)"},
         "prefill_ms_p50": round(main["prefill_ms_p50"], 3), "denoise_ms_p50": round(main["denoise_ms_p50"], 3),
         "prefill_ms_p90": round(main["prefill_ms_p90"], 3), "denoise_ms_p90": round(main["denoise_ms_p90"], 3),
-        "roofline": {"bound": "tensor", "kernel": "gemm_tc_kernel<256> (prefill gate/up, M=B*P, N=2*6144, K=2048)",
+        "roofline": {"bound": "tensor", "kernel": "gemm_tc_persistent<256,4> (prefix-pass gate/up + SwiGLU, M=B*P, N=2*6144, K=2048)",
                      "achieved": round(gu_tf, 1), "peak": tc_peak, "unit": "TFLOP/s",
                      "frac": round(gu_tf / tc_peak, 4),
                      "traffic": GATEUP_TRAFFIC_BYTES if (B, P) == (16, 2048) else None,

@@ -29,7 +29,7 @@ namespace dm0 {
 
 constexpr int kFaThreads = 192;
 
-template <int ST>
+template <int ST, int NP>
 struct FaSmemT {
   static constexpr int kKeys = 64;                          // keys per block
   static constexpr uint32_t kQ = 32768;                     // 128 rows x 128 dims: two 64-column SW128 halves
@@ -37,19 +37,20 @@ struct FaSmemT {
   static constexpr uint32_t kHalfKV = 8192;
   static constexpr uint32_t kP = 16384;                     // 128 rows x 64 keys, one SW128 block
   static constexpr int kStages = ST;                        // K/V blocks in flight
+  static constexpr int kPBufs = NP;                         // P buffers
   static constexpr uint32_t kOffQ = 0;
   static constexpr uint32_t kOffK = kOffQ + kQ;
   static constexpr uint32_t kOffV = kOffK + kStages * kKV;
   static constexpr uint32_t kOffP = kOffV + kStages * kKV;
-  static constexpr uint32_t kOffBar = kOffP + kP;
+  static constexpr uint32_t kOffBar = kOffP + NP * kP;
   static constexpr uint32_t kSlack = 256;                   // the dynamic base is 1024-aligned (no static smem)
   static constexpr uint32_t kBytes = kOffBar + 256 + kSlack;
 };
-// two stages (112 KB): two CTAs per SM, for the prefix pass whose K/V blocks are shared by many
-// CTAs through L2; five stages (208 KB): one CTA per SM with deeper prefetch, for the suffix
-// attention whose cached prefix K/V is read from DRAM once
-using FaSmem = FaSmemT<2>;
-constexpr int kFaDeepStages = 5;
+// Prefix pass: 2 K/V stages, one P buffer (112 KB): two CTAs per SM, K/V blocks shared by many CTAs
+// through L2.  Suffix attention: 4 K/V stages and two P buffers (192 KB, one CTA per SM): deeper
+// prefetch for the once-read prefix cache, and the softmax of block j+1 never waits for PV_j.
+using FaSmem = FaSmemT<2, 1>;
+constexpr int kFaDeepStages = 4;
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
   asm volatile(
@@ -90,12 +91,12 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int col) {
   return half * 16384 + row * 128 + ((c16 ^ (row & 7)) << 4) + ((col & 7) << 1);
 }
 
-template <int ST>
-__global__ void __launch_bounds__(kFaThreads, ST <= 2 ? 2 : 1)
+template <int ST, int NP>
+__global__ void __launch_bounds__(kFaThreads, NP == 1 ? 2 : 1)
     fa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const __grid_constant__ CUtensorMap tmKb, const __grid_constant__ CUtensorMap tmVb, const AttnArgs a) {
   constexpr int D = 128;
-  using FS = FaSmemT<ST>;
+  using FS = FaSmemT<ST, NP>;
   extern __shared__ uint8_t fa_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fa_smem_raw) + 1023) & ~uintptr_t(1023));
   if (smem - fa_smem_raw > static_cast<ptrdiff_t>(FS::kSlack)) {   // never expected: refuse rather than overrun
@@ -107,9 +108,9 @@ __global__ void __launch_bounds__(kFaThreads, ST <= 2 ? 2 : 1)
   uint64_t* kv_empty = bars + ST;       // [ST] PV_j done: K/V slot free
   uint64_t* s_full = bars + 2 * ST;     // [2] S_j in TMEM
   uint64_t* s_free = s_full + 2;        // [2] softmax finished reading S_j
-  uint64_t* p_full = s_free + 2;        // P_j in smem and O corrected (one phase per block)
-  uint64_t* pv_done = p_full + 1;       // PV_j finished (one phase per block)
-  uint64_t* q_ready = pv_done + 1;
+  uint64_t* p_full = s_free + 2;        // [NP] P_j in buffer j % NP and O corrected
+  uint64_t* pv_done = p_full + NP;      // [NP] PV_j (which read buffer j % NP) finished
+  uint64_t* q_ready = pv_done + NP;
   uint64_t* drain = q_ready + 1;        // every issued MMA complete (before TMEM is released)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -135,8 +136,10 @@ __global__ void __launch_bounds__(kFaThreads, ST <= 2 ? 2 : 1)
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 4);
     }
-    mbar_init(p_full, 4);
-    mbar_init(pv_done, 1);
+    for (int i = 0; i < NP; ++i) {
+      mbar_init(&p_full[i], 4);
+      mbar_init(&pv_done[i], 1);
+    }
     mbar_init(q_ready, 4);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -206,15 +209,15 @@ __global__ void __launch_bounds__(kFaThreads, ST <= 2 ? 2 : 1)
       const uint32_t qa = smem_u32(smem + FS::kOffQ);
       bool ok = mbar_wait(q_ready, 0, abort_flag);
       auto pv = [&](int i) -> bool {
-        if (!mbar_wait(p_full, i & 1, abort_flag)) return false;
+        if (!mbar_wait(&p_full[i % NP], (i / NP) & 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t pa = smem_u32(smem + FS::kOffP);
+        const uint32_t pa = smem_u32(smem + FS::kOffP + (i % NP) * FS::kP);
         const uint32_t vb = smem_u32(smem + FS::kOffV + (i % ST) * FS::kKV);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
           umma_bf16(tmem + 128, sw128_kmajor_desc(pa + ks * 32), sw128_mnmajor_desc(vb + ks * 2048, FS::kHalfKV),
                     idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
-        umma_commit(pv_done);
+        umma_commit(&pv_done[i % NP]);
         umma_commit(&kv_empty[i % ST]);
         return true;
       };
@@ -337,14 +340,24 @@ __global__ void __launch_bounds__(kFaThreads, ST <= 2 ? 2 : 1)
       const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
       l_run = l_run * alpha + sum;
       m_ref = m_new;
-      // O and the P slot of block j-2 are in use until PV_{j-1} completes
-      if (j >= 1) {
-        if (!mbar_wait(pv_done, (j - 1) & 1, abort_flag)) {
+      // P buffer j % NP is free once PV_{j-NP} completed; O may only be rescaled after PV_{j-1}
+      const bool any_move = __any_sync(0xffffffffu, move);
+      if (j >= NP) {
+        if (!mbar_wait(&pv_done[j % NP], ((j / NP) - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+      }
+      if (j >= 1 && (NP == 1 || any_move)) {
+        const int i = j - 1;
+        if (NP > 1 && !mbar_wait(&pv_done[i % NP], (i / NP) & 1, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, move)) {
+      }
+      if (j >= 1 && any_move) {
+        {
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {
             float o[32];
@@ -356,7 +369,7 @@ __global__ void __launch_bounds__(kFaThreads, ST <= 2 ? 2 : 1)
           tmem_wait_st();
         }
       }
-      uint8_t* ps = smem + FS::kOffP;   // one buffer: PV_{j-1} has completed
+      uint8_t* ps = smem + FS::kOffP + (j % NP) * FS::kP;
 #pragma unroll
       for (int c = 0; c < 8; ++c)
         *reinterpret_cast<uint4*>(ps + sw128_off(r, c * 8)) =
@@ -364,13 +377,13 @@ __global__ void __launch_bounds__(kFaThreads, ST <= 2 ? 2 : 1)
       fence_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[j % NP]);
     }
     if (!ok) {
       *abort_flag = 1;
       raise_error(a.err, kErrTimeoutEpilogue);
     } else if (nblk > 0) {
-      if (mbar_wait(pv_done, (nblk - 1) & 1, abort_flag)) {
+      if (mbar_wait(&pv_done[(nblk - 1) % NP], ((nblk - 1) / NP) & 1, abort_flag)) {
         tc_fence_after();
         if (gridDim.z == 1) {
           const float inv = 1.f / l_run;

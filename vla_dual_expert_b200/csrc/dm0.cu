@@ -300,14 +300,15 @@ dm0_status run_gemm(dm0_ctx* c, cudaStream_t s, const bf16* act, int tokens, int
   // persistent: at most one CTA per SM walking the tiles
   const int ntiles = mt * (wrows / BN);
   const dim3 grid(std::min(ntiles, c->num_sms));
+  // as many stages as fit in ~192 KB: more bytes in flight per SM for the narrower tiles
   if (BN == 256)
-    return launch(c, s, dm0::gemm_tc_persistent<256, kGemmStages>, grid, dim3(dm0::kGemmThreads),
-                  dm0::PGemmSmem<256, kGemmStages>::kBytes, ta, tb, g);
+    return launch(c, s, dm0::gemm_tc_persistent<256, 4>, grid, dim3(dm0::kGemmThreads),
+                  dm0::PGemmSmem<256, 4>::kBytes, ta, tb, g);
   if (BN == 128)
-    return launch(c, s, dm0::gemm_tc_persistent<128, kGemmStages>, grid, dim3(dm0::kGemmThreads),
-                  dm0::PGemmSmem<128, kGemmStages>::kBytes, ta, tb, g);
-  return launch(c, s, dm0::gemm_tc_persistent<64, kGemmStages>, grid, dim3(dm0::kGemmThreads),
-                dm0::PGemmSmem<64, kGemmStages>::kBytes, ta, tb, g);
+    return launch(c, s, dm0::gemm_tc_persistent<128, 6>, grid, dim3(dm0::kGemmThreads),
+                  dm0::PGemmSmem<128, 6>::kBytes, ta, tb, g);
+  return launch(c, s, dm0::gemm_tc_persistent<64, 8>, grid, dim3(dm0::kGemmThreads), dm0::PGemmSmem<64, 8>::kBytes,
+                ta, tb, g);
 }
 
 // ---------------------------------------------------------------- attention dispatch
@@ -359,7 +360,7 @@ dm0_status run_attn(dm0_ctx* c, cudaStream_t s, const bf16* q, int seq_q, const 
     if (fs <= 0) {   // fill the SMs once (two CTAs per SM for the prefix kernel, one for the deep suffix
                      // kernel), at most 4 splits: the combine reads every split's partial O
       const int ctas = groups * tiles;
-      const int slots = (len_b == 0 ? 2 : 1) * c->num_sms;
+      const int slots = (len_b == 0 || groups * tiles <= c->num_sms / 8 ? 2 : 1) * c->num_sms;
       fs = std::max(1, std::min(4, (slots + ctas / 2) / ctas));
     }
     fs = std::min(fs, fblk);
@@ -380,12 +381,16 @@ dm0_status run_attn(dm0_ctx* c, cudaStream_t s, const bf16* q, int seq_q, const 
       tvb = tv;
     }
     const dim3 grid(tiles, groups, fs);
-    if (len_b == 0)   // prefix pass: K/V blocks shared by many CTAs through L2, two CTAs per SM
-      return launch(c, s, dm0::fa_tc_kernel<2>, grid, dim3(dm0::kFaThreads), dm0::FaSmemT<2>::kBytes, tk, tv, tkb,
-                    tvb, a);
-    // merged suffix attention: the cached prefix is read from DRAM once, deeper K/V prefetch
-    return launch(c, s, dm0::fa_tc_kernel<dm0::kFaDeepStages>, grid, dim3(dm0::kFaThreads),
-                  dm0::FaSmemT<dm0::kFaDeepStages>::kBytes, tk, tv, tkb, tvb, a);
+    // prefix pass (K/V blocks shared by many CTAs through L2), and the suffix attention of small
+    // batches: two CTAs per SM, small enough (113 KB, 24.5K registers) to share an SM with a
+    // swapped GEMM CTA, so neighbouring kernels overlap under programmatic dependent launch
+    if (len_b == 0 || groups * tiles * fs <= c->num_sms / 2)
+      return launch(c, s, dm0::fa_tc_kernel<2, 1>, grid, dim3(dm0::kFaThreads), dm0::FaSmemT<2, 1>::kBytes, tk, tv,
+                    tkb, tvb, a);
+    // merged suffix attention: the cached prefix is read from DRAM once; deeper K/V prefetch and
+    // two P buffers so the softmax runs ahead of the PV MMAs
+    return launch(c, s, dm0::fa_tc_kernel<dm0::kFaDeepStages, 2>, grid, dim3(dm0::kFaThreads),
+                  dm0::FaSmemT<dm0::kFaDeepStages, 2>::kBytes, tk, tv, tkb, tvb, a);
   }
   const dim3 grid(tiles, groups, splits);
   switch (g.head_dim) {
@@ -789,14 +794,14 @@ dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
   bool ok = smem_attr(dm0::gemm_tc_kernel<64, kGemmStages>, dm0::GemmSmem<64, kGemmStages>::kBytes) &&
             smem_attr(dm0::gemm_tc_kernel<128, kGemmStages>, dm0::GemmSmem<128, kGemmStages>::kBytes) &&
             smem_attr(dm0::gemm_tc_kernel<256, kGemmStages>, dm0::GemmSmem<256, kGemmStages>::kBytes) &&
-            smem_attr(dm0::gemm_tc_persistent<64, kGemmStages>, dm0::PGemmSmem<64, kGemmStages>::kBytes) &&
-            smem_attr(dm0::gemm_tc_persistent<128, kGemmStages>, dm0::PGemmSmem<128, kGemmStages>::kBytes) &&
-            smem_attr(dm0::gemm_tc_persistent<256, kGemmStages>, dm0::PGemmSmem<256, kGemmStages>::kBytes) &&
+            smem_attr(dm0::gemm_tc_persistent<64, 8>, dm0::PGemmSmem<64, 8>::kBytes) &&
+            smem_attr(dm0::gemm_tc_persistent<128, 6>, dm0::PGemmSmem<128, 6>::kBytes) &&
+            smem_attr(dm0::gemm_tc_persistent<256, 4>, dm0::PGemmSmem<256, 4>::kBytes) &&
             smem_attr(dm0::attn_kernel<128>, dm0::AttnSmem<128>::kBytes) &&
             smem_attr(dm0::attn_kernel<64>, dm0::AttnSmem<64>::kBytes) &&
             smem_attr(dm0::attn_kernel<32>, dm0::AttnSmem<32>::kBytes) &&
-            smem_attr(dm0::fa_tc_kernel<2>, dm0::FaSmemT<2>::kBytes) &&
-            smem_attr(dm0::fa_tc_kernel<dm0::kFaDeepStages>, dm0::FaSmemT<dm0::kFaDeepStages>::kBytes);
+            smem_attr(dm0::fa_tc_kernel<2, 1>, dm0::FaSmemT<2, 1>::kBytes) &&
+            smem_attr(dm0::fa_tc_kernel<dm0::kFaDeepStages, 2>, dm0::FaSmemT<dm0::kFaDeepStages, 2>::kBytes);
   if (!ok) return bail(DM0_ECUDA);
   *out = c;
   return DM0_OK;
