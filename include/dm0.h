@@ -127,8 +127,12 @@ dm0_status dm0_kv_commit(dm0_ctx* ctx, int B, int P);
  *   noise:      device f32 [B][chunk][action_dim] (x_1), read once.
  *   actions:    device f32 [B][chunk][action_dim] output x_0 (may alias noise).
  *   velocities: device f32 [steps][B][chunk][action_dim] per-step v, or NULL.
- * The step loop is captured once per (B, P, steps, velocities != NULL) as a
- * CUDA graph and replayed; no host work happens inside the loop.
+ * One observation (B = 1) with head_dim 128 runs the whole loop as ONE
+ * persistent kernel (one CTA per SM, grid barriers between the phases of a
+ * layer); otherwise, and when the environment variable DM0_NO_PERSIST=1 was
+ * set at dm0_create, the loop is a chain of per-layer kernels captured once
+ * per (B, P, steps) as a CUDA graph and replayed (launched directly when
+ * velocities are requested).  No host work happens inside the loop.
  * Returns DM0_ESTATE without a cache, DM0_ESHAPE unless 1 <= steps <= 1000. */
 dm0_status dm0_denoise(dm0_ctx* ctx, const float* noise, int steps, float* actions, float* velocities,
                        void* stream);
@@ -184,7 +188,14 @@ dm0_status dm0_op_attention(dm0_ctx* ctx, const void* q, const void* ka, const v
  * [rows][n_q*head_dim]; act_* bf16 [rows][inter]; ssq_* f32 [2*layers][rows]
  * (sum of squares of h for each pending norm); x f32 [rows][action_dim];
  * k_s/v_s bf16 [B][n_kv][chunk][head_dim].  Context-owned; contents are only
- * meaningful after the call that fills them has completed. */
+ * meaningful after the call that fills them has completed.
+ * "loop_trace" (NULL unless DM0_PERSIST_TRACE=1 was set at dm0_create): u64
+ * %globaltimer marks of the persistent Euler loop (runs of <= 16 steps),
+ * [phase][CTA][8] = phase start, operand staged, first accumulator (or S tile)
+ * ready, results issued, release fence done, barrier arrival, MMA warp saw the
+ * operand, MMA warp issued its last MMA;
+ * phase 0 is the input of step 0, then per step 5 phases per layer (QKV,
+ * attention, O, gate/up, down) and the step boundary. */
 dm0_status dm0_debug_view(dm0_ctx* ctx, const char* name, void** ptr);
 
 /* Merged GQA attention that allocates nothing, for callers that cannot call
@@ -231,7 +242,9 @@ enum {
   DM0_SITE_ACT_GATEUP = 8,
   DM0_SITE_ACT_DOWN = 9,
   DM0_SITE_STEP = 10,       /* Euler step boundary (velocity, update, next input) */
-  DM0_SITE_COUNT = 11
+  DM0_SITE_LOOP = 11,       /* the whole Euler loop as one persistent kernel (one observation; the
+                               per-layer sites 5-10 are then not launched) */
+  DM0_SITE_COUNT = 12
 };
 
 /* Time the launches of the sites in `site_mask` (bit i = site i) with CUDA

@@ -101,7 +101,7 @@ def _bf16_bits(a: np.ndarray) -> np.ndarray:
 
 # kernel sites of dm0_probe (include/dm0.h)
 SITES = ("vlm_qkv", "vlm_attn", "vlm_o", "vlm_gateup", "vlm_down", "act_qkv", "act_attn", "act_o", "act_gateup",
-         "act_down", "step")
+         "act_down", "step", "loop")
 
 LAYER_ORDER = (("attn_norm", "f32"), ("Wq", "bf16"), ("Wk", "bf16"), ("Wv", "bf16"), ("q_norm", "f32"),
                ("k_norm", "f32"), ("Wo", "bf16"), ("mlp_norm", "f32"), ("Wg", "bf16"), ("Wu", "bf16"),

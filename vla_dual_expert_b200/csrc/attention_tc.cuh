@@ -332,8 +332,8 @@ __global__ void __launch_bounds__(kFaThreads, NP == 1 ? 2 : 1)
       for (int k = 0; k < 8; ++k) sum8[k] = 0.f;
 #pragma unroll
       for (int i = 0; i < 64; i += 2) {
-        const float p0 = (i < nvalid) ? exp2f(fmaf(sv[i], a.scale_log2, -m_new)) : 0.f;
-        const float p1 = (i + 1 < nvalid) ? exp2f(fmaf(sv[i + 1], a.scale_log2, -m_new)) : 0.f;
+        const float p0 = (i < nvalid) ? ex2_fast(fmaf(sv[i], a.scale_log2, -m_new)) : 0.f;
+        const float p1 = (i + 1 < nvalid) ? ex2_fast(fmaf(sv[i + 1], a.scale_log2, -m_new)) : 0.f;
         sum8[(i >> 1) & 7] += p0 + p1;
         pk[i >> 1] = pack_bf16(p0, p1);
       }

@@ -18,6 +18,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
@@ -31,6 +32,7 @@
 #include "dm0.h"
 #include "attention.cuh"
 #include "attention_tc.cuh"
+#include "denoise_persistent.cuh"
 #include "elementwise.cuh"
 #include "gemm.cuh"
 #include "ptx.cuh"
@@ -82,6 +84,10 @@ struct dm0_ctx {
   int device = 0;
   int num_sms = 148;
   bool use_pdl = true, use_graph = true;
+  // single-observation Euler loop as one persistent kernel (DM0_NO_PERSIST=1 selects the graph of
+  // per-layer kernels instead); DM0_PERSIST_SPLITS overrides its attention key splits per KV head
+  bool use_persist = true;
+  int persist_splits = 7;
   // true when the previous operation this context queued on the stream was one of its own
   // kernels: only then may the next kernel overlap it (programmatic dependent launch).  The first
   // kernel of every API call follows foreign work (caller kernels, copies) and waits for it in
@@ -119,6 +125,12 @@ struct dm0_ctx {
   int* d_err = nullptr;
   // dm0_infer_host staging
   bf16* stage_prefix = nullptr;
+  // persistent Euler loop: split-K sums, sums of squares, grid-barrier words, per-layer norm gains
+  float *pacc_qkv = nullptr, *pacc_gu = nullptr, *pssq = nullptr;
+  unsigned* psync = nullptr;
+  dm0::PdLayer* players = nullptr;
+  unsigned long long* ptrace = nullptr;   // DM0_PERSIST_TRACE=1: phase timestamps of the persistent loop
+  int ptrace_steps = 0;
 
   cudaStream_t cap_stream = nullptr;
   struct Graph {
@@ -534,7 +546,7 @@ dm0_status step(dm0_ctx* c, cudaStream_t s, int B, int k_out, int k_in, int step
   a.steps = steps;
   a.vel = vel;
   const int e0 = probe_begin(c, s, DM0_SITE_STEP);
-  TRY(launch(c, s, dm0::step_kernel, dim3(B * cf.chunk), dim3(256), 0, a));
+  TRY(launch(c, s, dm0::step_kernel, dim3(B * cf.chunk), dim3(256), sizeof(float) * cf.hidden_a, a));
   probe_end(c, s, DM0_SITE_STEP, e0);
   return DM0_OK;
 }
@@ -566,7 +578,121 @@ dm0_status enqueue_denoise(dm0_ctx* c, cudaStream_t s, int steps, float* vel) {
   return DM0_OK;
 }
 
+// The persistent Euler loop covers one observation of the DM0-base shapes: head_dim 128, at most
+// 64 suffix tokens and 128 attention rows per KV head, 128-row weight tiles, and per GEMM phase at
+// most kPdBTiles pairs (and two weight tiles) per CTA.  Fills everything of `a` but the stream-time
+// fields; false (with the reason) sends the loop to the per-layer kernels.
+bool persist_plan(dm0_ctx* c, int steps, float* vel, dm0::PdArgs* a, std::string* why) {
+  const dm0_config& g = c->cfg;
+  auto no = [&](const char* m) {
+    *why = m;
+    return false;
+  };
+  if (!c->use_persist) return no("disabled");
+  if (g.head_dim != 128) return no("head_dim != 128");
+  const int B = c->kv_B, P = c->kv_P, T = B * g.chunk, G = g.n_q / g.n_kv;
+  if (B != 1 || T > 61 || G * T > 128) return no("more than one observation");   // RoPE rows fit a P buffer
+  if (g.hidden_a % 128 || qkv_rows(g) % 128 || g.inter_a % 64) return no("shapes do not tile by 128");
+  const int nsm = c->num_sms;
+  const int nblk = (P + 63) / 64 + 1;
+  int splits = std::min({c->persist_splits, dm0::kPdMaxSplits, nblk, nsm / g.n_kv});
+  if (splits < 1) return no("too few SMs");
+  const int bps = (nblk + splits - 1) / splits;
+  splits = (nblk + bps - 1) / bps;   // every split owns at least one block
+  // per GEMM phase (QKV, O, gate/up, down): tiles, k-blocks, landing bytes per staged pair
+  const long land_per[4] = {256L * T, 136L * splits * T, 256L * T, 512L * T};
+  const int geo[4][2] = {{qkv_rows(g) / 128, g.hidden_a / 64},
+                         {g.hidden_a / 128, g.n_q * 2},
+                         {g.inter_a / 64, g.hidden_a / 64},
+                         {g.hidden_a / 128, g.inter_a / 64}};
+  for (int ph = 0; ph < 4; ++ph) {
+    const int per = (geo[ph][0] * geo[ph][1] + nsm - 1) / nsm;
+    if (per > dm0::kPdBTiles || per > geo[ph][1]) return no("GEMM ranges too long for the staging area");
+    if (per * land_per[ph] > static_cast<long>(dm0::PdSmem::kLandG)) return no("operand copies exceed the landing area");
+  }
+  if (g.n_kv * splits > kPartSlots) return no("partial-state slots");
+  *a = dm0::PdArgs{};
+  a->L = g.layers;
+  a->T = T;
+  a->P = P;
+  a->steps = steps;
+  a->Ha = g.hidden_a;
+  a->Ia = g.inter_a;
+  a->n_q = g.n_q;
+  a->n_kv = g.n_kv;
+  a->QR = qkv_rows(g);
+  a->eps = g.rms_eps;
+  a->scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(g.head_dim)));
+  a->splits = splits;
+  a->bps = bps;
+  a->layers = c->players;
+  a->rope = c->rope;
+  a->h = c->h_a;
+  a->acc_qkv = c->pacc_qkv;
+  a->acc_gu = c->pacc_gu;
+  a->ssq = c->pssq;
+  a->part_o = reinterpret_cast<bf16*>(c->part_o);   // bf16 partials in the fp32 slot area
+  a->part_ml = c->part_ml;
+  a->sync = c->psync;
+  a->err = c->d_err;
+  a->trace = steps <= c->ptrace_steps ? c->ptrace : nullptr;
+  StepArgs& st = a->step;
+  st.x = c->x;
+  st.h = c->h_a;
+  st.xn = nullptr;
+  st.ssq = nullptr;
+  st.n_slots = 0;
+  st.tokens = T;
+  st.W_in = c->W_in;
+  st.b_in = c->b_in;
+  st.attn_norm0 = nullptr;
+  st.final_norm = c->final_norm;
+  st.W_out = c->W_out;
+  st.b_out = c->b_out;
+  st.Ha = g.hidden_a;
+  st.A = g.action_dim;
+  st.eps = g.rms_eps;
+  st.steps = steps;
+  st.vel = vel;
+  return true;
+}
+
+dm0_status enqueue_denoise_persistent(dm0_ctx* c, cudaStream_t s, const dm0::PdArgs& a) {
+  const dm0_config& g = c->cfg;
+  const uint64_t L = g.layers;
+  CUtensorMap tq, to, tgu, td, tk, tv;
+  TRY(get_tmap(c, &tq, c->lw[1][0].wqkv, L * qkv_rows(g), g.hidden_a, 128));
+  TRY(get_tmap(c, &to, c->lw[1][0].wo, L * g.hidden_a, static_cast<uint64_t>(g.n_q) * g.head_dim, 128));
+  TRY(get_tmap(c, &tgu, c->lw[1][0].wgu, L * 2 * g.inter_a, g.hidden_a, 128));
+  TRY(get_tmap(c, &td, c->lw[1][0].wd, L * g.hidden_a, g.inter_a, 128));
+  const uint64_t kv_rows = L * g.n_kv * static_cast<uint64_t>(a.P);
+  TRY(get_tmap(c, &tk, c->kplane, kv_rows, 128, 64));
+  TRY(get_tmap(c, &tv, c->vplane, kv_rows, 128, 64));
+  CK(cudaMemsetAsync(c->psync, 0, 4 * sizeof(unsigned), s));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(c->num_sms);
+  cfg.blockDim = dim3(dm0::kPdThreads);
+  cfg.dynamicSmemBytes = dm0::PdSmem::kBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;   // grid barriers: every CTA must be resident
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const int e0 = probe_begin(c, s, DM0_SITE_LOOP);
+  CK(cudaLaunchKernelEx(&cfg, dm0::denoise_persistent_kernel, tq, to, tgu, td, tk, tv, a));
+  probe_end(c, s, DM0_SITE_LOOP, e0);
+  c->launches += 1;
+  c->pdl_ok = false;
+  return DM0_OK;
+}
+
 dm0_status denoise_from_x(dm0_ctx* c, cudaStream_t s, int steps, float* vel) {
+  {
+    dm0::PdArgs pa;
+    std::string why;
+    if (persist_plan(c, steps, vel, &pa, &why)) return enqueue_denoise_persistent(c, s, pa);
+  }
   if (vel || !c->use_graph || c->probe_mask) return enqueue_denoise(c, s, steps, vel);
   const auto key = std::make_tuple(c->kv_B, c->kv_P, steps);
   auto it = c->graphs.find(key);
@@ -688,6 +814,8 @@ dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
   cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device);
   if (const char* e = std::getenv("DM0_NO_PDL")) c->use_pdl = e[0] == '0';
   if (const char* e = std::getenv("DM0_NO_GRAPH")) c->use_graph = e[0] == '0';
+  if (const char* e = std::getenv("DM0_NO_PERSIST")) c->use_persist = e[0] == '0';
+  if (const char* e = std::getenv("DM0_PERSIST_SPLITS")) c->persist_splits = std::max(1, std::atoi(e));
 
   // weights: one allocation, 256-byte aligned sub-buffers
   size_t total = 0;
@@ -696,13 +824,16 @@ dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
     offs.push_back(total);
     total += align256(bytes);
   };
+  // the four matrices of a branch are each stacked over the layers ([L][rows][cols], no padding), so
+  // one 2-D TMA descriptor per matrix type covers every layer
+  const size_t Lz = static_cast<size_t>(g.layers);
   for (int br = 0; br < 2; ++br) {
     const size_t H = hidden_of(g, br), I = inter_of(g, br);
+    take(Lz * 2 * qkv_rows(g) * H);
+    take(Lz * 2 * H * g.n_q * g.head_dim);
+    take(Lz * 2 * 2 * I * H);
+    take(Lz * 2 * H * I);
     for (int l = 0; l < g.layers; ++l) {
-      take(2 * qkv_rows(g) * H);
-      take(2 * H * g.n_q * g.head_dim);
-      take(2 * 2 * I * H);
-      take(2 * H * I);
       take(4 * H);
       take(4 * g.head_dim);
       take(4 * g.head_dim);
@@ -719,13 +850,18 @@ dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
   c->wbuf = wb;
   size_t k = 0;
   for (int br = 0; br < 2; ++br) {
+    const size_t H = hidden_of(g, br), I = inter_of(g, br);
     c->lw_store[br].resize(g.layers);
+    bf16* wqkv0 = reinterpret_cast<bf16*>(wb + offs[k++]);
+    bf16* wo0 = reinterpret_cast<bf16*>(wb + offs[k++]);
+    bf16* wgu0 = reinterpret_cast<bf16*>(wb + offs[k++]);
+    bf16* wd0 = reinterpret_cast<bf16*>(wb + offs[k++]);
     for (int l = 0; l < g.layers; ++l) {
       LayerW& w = c->lw_store[br][l];
-      w.wqkv = reinterpret_cast<bf16*>(wb + offs[k++]);
-      w.wo = reinterpret_cast<bf16*>(wb + offs[k++]);
-      w.wgu = reinterpret_cast<bf16*>(wb + offs[k++]);
-      w.wd = reinterpret_cast<bf16*>(wb + offs[k++]);
+      w.wqkv = wqkv0 + l * qkv_rows(g) * H;
+      w.wo = wo0 + l * H * g.n_q * g.head_dim;
+      w.wgu = wgu0 + l * 2 * I * H;
+      w.wd = wd0 + l * H * I;
       w.attn_norm = reinterpret_cast<float*>(wb + offs[k++]);
       w.q_norm = reinterpret_cast<float*>(wb + offs[k++]);
       w.k_norm = reinterpret_cast<float*>(wb + offs[k++]);
@@ -778,7 +914,27 @@ dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
   A(dalloc(c, &c->rope, static_cast<size_t>(max_pos) * D / 2));
   A(dalloc(c, &c->d_err, 1));
   A(dalloc(c, &c->stage_prefix, Mp * g.hidden_v));
+  A(dalloc(c, &c->pacc_qkv, static_cast<size_t>(64) * qkv_rows(g)));
+  A(dalloc(c, &c->pacc_gu, static_cast<size_t>(64) * 2 * g.inter_a));
+  A(dalloc(c, &c->pssq, 128));
+  A(dalloc(c, &c->psync, 4));
+  A(dalloc(c, &c->players, g.layers));
+  if (const char* e = std::getenv("DM0_PERSIST_TRACE")) {
+    if (e[0] == '1') {
+      c->ptrace_steps = 16;
+      A(dalloc(c, &c->ptrace, static_cast<size_t>(1 + c->ptrace_steps * (5 * g.layers + 1)) * c->num_sms * dm0::kPdTraceSlots));
+    }
+  }
   if (st != DM0_OK) return bail(st);
+  {
+    std::vector<dm0::PdLayer> pl(g.layers);
+    for (int l = 0; l < g.layers; ++l) {
+      const LayerW& w = c->lw[1][l];
+      pl[l] = dm0::PdLayer{w.attn_norm, w.q_norm, w.k_norm, w.mlp_norm};
+    }
+    if (cudaMemcpy(c->players, pl.data(), pl.size() * sizeof(dm0::PdLayer), cudaMemcpyHostToDevice) != cudaSuccess)
+      return bail(DM0_ECUDA);
+  }
   if (cudaMemset(c->acc, 0, c->acc_elems * 4) != cudaSuccess || cudaMemset(c->gcount, 0, 1024 * 4) != cudaSuccess ||
       cudaMemset(c->acount, 0, c->acount_n * 4) != cudaSuccess || cudaMemset(c->d_err, 0, 4) != cudaSuccess)
     return bail(DM0_ECUDA);
@@ -801,7 +957,8 @@ dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
             smem_attr(dm0::attn_kernel<64>, dm0::AttnSmem<64>::kBytes) &&
             smem_attr(dm0::attn_kernel<32>, dm0::AttnSmem<32>::kBytes) &&
             smem_attr(dm0::fa_tc_kernel<2, 1>, dm0::FaSmemT<2, 1>::kBytes) &&
-            smem_attr(dm0::fa_tc_kernel<dm0::kFaDeepStages, 2>, dm0::FaSmemT<dm0::kFaDeepStages, 2>::kBytes);
+            smem_attr(dm0::fa_tc_kernel<dm0::kFaDeepStages, 2>, dm0::FaSmemT<dm0::kFaDeepStages, 2>::kBytes) &&
+            smem_attr(dm0::denoise_persistent_kernel, dm0::PdSmem::kBytes);
   if (!ok) return bail(DM0_ECUDA);
   *out = c;
   return DM0_OK;
@@ -977,7 +1134,8 @@ dm0_status dm0_debug_view(dm0_ctx* c, const char* name, void** ptr) {
   const std::map<std::string, void*> bufs = {
       {"h_v", c->h_v},     {"xn_v", c->xn_v},   {"q_v", c->q_v},     {"o_v", c->o_v},     {"act_v", c->act_v},
       {"ssq_v", c->ssq_v}, {"h_a", c->h_a},     {"xn_a", c->xn_a},   {"q_a", c->q_a},     {"o_a", c->o_a},
-      {"act_a", c->act_a}, {"ssq_a", c->ssq_a}, {"x", c->x},         {"k_s", c->k_s},     {"v_s", c->v_s}};
+      {"act_a", c->act_a}, {"ssq_a", c->ssq_a}, {"x", c->x},         {"k_s", c->k_s},     {"v_s", c->v_s},
+      {"loop_trace", c->ptrace}};
   auto it = bufs.find(name);
   if (it == bufs.end()) return fail(c, DM0_EINVAL, std::string("unknown buffer ") + name);
   *ptr = it->second;

@@ -57,29 +57,47 @@ struct StepArgs {
   float* vel;                  // [steps][tokens][A] or null
 };
 
-// One CTA (256 threads) per action token.
-__global__ void __launch_bounds__(256) step_kernel(const StepArgs a) {
-  __shared__ float sx[64];
-  __shared__ float sred[8];
-  pdl_launch_dependents();
-  pdl_wait();
-  const int tok = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+// Step boundary for one action token, run by `nthr` threads (a multiple of 32, >= the action
+// dimension, <= 256) that synchronise with `sync()`.  `hs` is shared scratch for Ha floats.  Reads
+// of h go through L2: in the persistent Euler loop other CTAs produced them.  xn / ssq are written
+// only when non-null.  Weight rows are read 16 bytes at a time when the shapes allow it, so the
+// loads of a row are in flight together.
+template <class Sync>
+__device__ __forceinline__ void step_token(const StepArgs& a, int tok, int tid, int nthr, float* sx, float* sred,
+                                           float* hs, Sync&& sync) {
+  const int nw = nthr >> 5, warp = tid >> 5, lane = tid & 31;
   float* hrow = a.h + static_cast<size_t>(tok) * a.Ha;
+  const bool vec_out = (a.Ha % 256) == 0, vec_in = (a.A % 8) == 0;
   if (a.k_out >= 0) {
     float sq = 0.f;
-    for (int j = tid; j < a.Ha; j += 256) sq += hrow[j] * hrow[j];
+    for (int j = tid; j < a.Ha; j += nthr) {
+      const float hv = __ldcg(hrow + j);
+      hs[j] = hv * a.final_norm[j];
+      sq += hv * hv;
+    }
     sq = warp_sum(sq);
     if (lane == 0) sred[warp] = sq;
-    __syncthreads();
+    sync();
     float tot = 0.f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) tot += sred[w];
+    for (int w = 0; w < nw; ++w) tot += sred[w];
     const float inv = rsqrtf(tot / a.Ha + a.eps);
     const float dt = -1.0f / a.steps;
-    for (int o = warp; o < a.A; o += 8) {
+    for (int o = warp; o < a.A; o += nw) {
+      const __nv_bfloat16* wr = a.W_out + static_cast<size_t>(o) * a.Ha;
       float acc = 0.f;
-      for (int j = lane; j < a.Ha; j += 32)
-        acc += __bfloat162float(a.W_out[static_cast<size_t>(o) * a.Ha + j]) * (hrow[j] * a.final_norm[j]);
+      if (vec_out) {   // lane reads 8 consecutive weights per 256-wide slice
+        for (int j0 = lane * 8; j0 < a.Ha; j0 += 256) {
+          const uint4 w8 = __ldg(reinterpret_cast<const uint4*>(wr + j0));
+          const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&w8);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(w2[e]);
+            acc += f.x * hs[j0 + 2 * e] + f.y * hs[j0 + 2 * e + 1];
+          }
+        }
+      } else {
+        for (int j = lane; j < a.Ha; j += 32) acc += __bfloat162float(wr[j]) * hs[j];
+      }
       acc = warp_sum(acc);
       if (lane == 0) {
         const float v = acc * inv + a.b_out[o];
@@ -88,37 +106,61 @@ __global__ void __launch_bounds__(256) step_kernel(const StepArgs a) {
         if (a.vel) a.vel[(static_cast<size_t>(a.k_out) * a.tokens + tok) * a.A + o] = v;
       }
     }
-    __syncthreads();
+    sync();
   }
   if (a.k_in >= 0) {
     if (tid < a.A) sx[tid] = a.x[static_cast<size_t>(tok) * a.A + tid];
-    __syncthreads();
+    sync();
     const float t = 1.0f - static_cast<float>(a.k_in) / static_cast<float>(a.steps);
     const int half = a.Ha >> 1;
     const float kLog2_10000 = 13.287712379549449f;
     float sq = 0.f;
-    for (int j = tid; j < a.Ha; j += 256) {
+    for (int j = tid; j < a.Ha; j += nthr) {
       float e = a.b_in[j];
       const __nv_bfloat16* w = a.W_in + static_cast<size_t>(j) * a.A;
-      for (int i = 0; i < a.A; ++i) e += __bfloat162float(w[i]) * sx[i];
+      if (vec_in) {
+        for (int i0 = 0; i0 < a.A; i0 += 8) {
+          const uint4 w8 = __ldg(reinterpret_cast<const uint4*>(w + i0));
+          const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&w8);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 f = __bfloat1622float2(w2[q]);
+            e += f.x * sx[i0 + 2 * q] + f.y * sx[i0 + 2 * q + 1];
+          }
+        }
+      } else {
+        for (int i = 0; i < a.A; ++i) e += __bfloat162float(w[i]) * sx[i];
+      }
       const int fi = j < half ? j : j - half;
       const float arg = t * exp2f(-static_cast<float>(fi) / half * kLog2_10000);
       e += j < half ? sinf(arg) : cosf(arg);
       hrow[j] = e;
-      a.xn[static_cast<size_t>(tok) * a.Ha + j] = __float2bfloat16_rn(a.attn_norm0[j] * e);
+      if (a.xn) a.xn[static_cast<size_t>(tok) * a.Ha + j] = __float2bfloat16_rn(a.attn_norm0[j] * e);
       sq += e * e;
     }
-    sq = warp_sum(sq);
-    __syncthreads();
-    if (lane == 0) sred[warp] = sq;
-    __syncthreads();
-    if (tid == 0) {
-      float tot = 0.f;
-      for (int w = 0; w < 8; ++w) tot += sred[w];
-      a.ssq[tok] = tot;
+    if (a.ssq) {
+      sq = warp_sum(sq);
+      sync();
+      if (lane == 0) sred[warp] = sq;
+      sync();
+      if (tid == 0) {
+        float tot = 0.f;
+        for (int w = 0; w < nw; ++w) tot += sred[w];
+        a.ssq[tok] = tot;
+      }
+      for (int s = 1 + tid; s < a.n_slots; s += nthr) a.ssq[static_cast<size_t>(s) * a.tokens + tok] = 0.f;
     }
-    for (int s = 1 + tid; s < a.n_slots; s += 256) a.ssq[static_cast<size_t>(s) * a.tokens + tok] = 0.f;
   }
+}
+
+// One CTA (256 threads) per action token; dynamic shared memory: Ha floats.
+__global__ void __launch_bounds__(256) step_kernel(const StepArgs a) {
+  __shared__ float sx[64];
+  __shared__ float sred[8];
+  extern __shared__ float step_hs[];
+  pdl_launch_dependents();
+  pdl_wait();
+  step_token(a, blockIdx.x, threadIdx.x, 256, sx, sred, step_hs, [] { __syncthreads(); });
 }
 
 // Failure-path self-test: one thread waits, with the library's bounded wait, on an mbarrier

@@ -185,5 +185,12 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
+// 2^x by the special-function unit's ex2.approx (flush-to-zero; 2^-inf = 0), for softmax weights
+// that are rounded to bf16 right after
+__device__ __forceinline__ float ex2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 }  // namespace dm0
