@@ -48,12 +48,9 @@
 
 namespace dm0 {
 
-#ifndef DM0_PD_COMPUTE_WARPS
-#define DM0_PD_COMPUTE_WARPS 8
-#endif
-constexpr int kPdCompute = 32 * DM0_PD_COMPUTE_WARPS;   // warps 2.. (4 or 8)
+constexpr int kPdCompute = 256;                 // warps 2-9
 constexpr int kPdThreads = 64 + kPdCompute;
-constexpr int kPdHalves = kPdCompute / 128;              // warps sharing a TMEM lane quarter
+constexpr int kPdHalves = 2;                     // warps sharing a TMEM lane quarter
 constexpr int kPdStages = 4;       // 16 KB ring stages
 constexpr int kPdBTiles = 6;       // staged activation tiles per GEMM phase
 constexpr int kPdMaxSplits = 8;    // attention key splits per KV head
@@ -105,7 +102,8 @@ struct PdArgs {
   float* ssq;               // [2][T]: attention-norm and MLP-norm sums of squares, zero at launch
   __nv_bfloat16* part_o;    // [n_kv * splits][128 rows][128]: O / l of the split
   float2* part_ml;          // [n_kv * splits][128 rows]: (max, sum) of the split
-  unsigned* sync;           // [0] barrier arrivals, [1] abort; zero at launch
+  unsigned* sync;           // [0] barrier arrivals, [1] abort, [2 + g] suffix K/V of KV head g ready; zero at launch
+  __nv_bfloat16* kv_sfx;    // [n_kv][K, V][64 keys][128] bf16, each tile in the shared-memory SW128 layout
   int* err;
   unsigned long long* trace;  // optional [phase][CTA][kPdTraceSlots] %globaltimer marks; null: off
   StepArgs step;            // x, h, W_in, b_in, final_norm, W_out, b_out, Ha, A, eps, steps, tokens, vel
@@ -139,41 +137,74 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
   return v;
 }
 
-// Operand staging, one function per phase type, kept out of line.  Every compute thread first
-// issues 16-byte cp.async copies of its share of the phase's L2 data into a shared-memory landing
-// area (no registers are held while the copies are in flight, so the whole stage costs one L2 round
-// trip), then the operand is built from shared memory.  A unit of the build is one 16-byte bf16
-// chunk (8 values) of a staged row; unit u goes to compute thread u % kPdCompute, so the 8 chunks of
-// a 64-column row segment sit in 8 adjacent lanes and a thread keeps the chunk index c8 = ct % 8.
-__device__ __forceinline__ void pd_cp16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+// TMA bulk reduce-add of a shared-memory fp32 tile into global memory (async proxy), and the fences
+// that order it with the generic-proxy accesses of this and other CTAs
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, const void* src, int x, int y) {
+  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
 }
-// commit this thread's copies and wait for all of them
-__device__ __forceinline__ void pd_cp_wait() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+// this warp's part of the operand of staged pair i is complete: make it visible to the tensor core
+// and arrive on the pair's barrier (one arrival per compute warp)
+__device__ __forceinline__ void pd_pair_ready(uint64_t* btf, int i, int ct) {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  __syncwarp();
+  if ((ct & 31) == 0) mbar_arrive(&btf[i]);
+}
+
+// Operand staging, one function per phase type, kept out of line.  Thread 0 of the compute group
+// requests the phase's L2 data with a few TMA tensor / bulk copies into a shared-memory landing
+// area (after a proxy fence: other CTAs wrote that data through the generic proxy) and every
+// compute thread waits on the stage mbarrier; the operand is then built from shared memory.  A
+// unit of the build is one 16-byte bf16 chunk (8 values) of a staged row; unit u goes to compute
+// thread u % kPdCompute, so the 8 chunks of a 64-column row segment sit in 8 adjacent lanes and a
+// thread keeps the chunk index c8 = ct % 8.  Each function returns the stage barrier's next parity.
+__device__ __forceinline__ void tma_load_2d_plain(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+// contiguous copy; both addresses 16-byte aligned, bytes a multiple of 16
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void pd_stage_wait(uint64_t* sbar, uint32_t par, volatile int* abort_flag) {
+  if (!mbar_wait(sbar, par, abort_flag)) *abort_flag = 1;
+}
 
 // (A, D) bf16(g * h) for pairs [p0, p0 + np); weight tile 0 also adds sum h^2 into ssq
 template <int kT>
-__device__ __noinline__ void pd_stage_norm(const PdArgs& a, uint8_t* smem, int ct, int p0, int np, int nkb,
-                                           const float* gain, float* ssq, unsigned long long* mk) {
+__device__ __noinline__ uint32_t pd_stage_norm(const PdArgs& a, uint8_t* smem, int ct, int p0, int np, int nkb,
+                                               const float* gain, float* ssq, unsigned long long* mk, uint64_t* btf,
+                                               uint64_t* sbar, uint32_t par, const CUtensorMap* map_h,
+                                               volatile int* abort_flag) {
   using SM = PdSmem;
   const int T = kT > 0 ? kT : a.T;   // tokens; a compile-time constant for the common shape
   const int c8 = ct & 7;
   float* land = reinterpret_cast<float*>(smem + SM::kOffLandG);   // [np][T][64]
   float* sg = reinterpret_cast<float*>(smem + SM::kOffAux);       // [np][64]
-  const float* h = a.h;
-  const int Ha = a.Ha;
-  int kb = p0 % nkb;
-  for (int i = 0; i < np; ++i) {
-    for (int q = ct; q < T * 16; q += kPdCompute) {
-      const int t = q >> 4, c = q & 15;
-      pd_cp16(land + (i * T + t) * 64 + c * 4, h + static_cast<size_t>(t) * Ha + kb * 64 + c * 4);
+  if (ct == 0) {
+    fence_proxy_async_global();
+    mbar_arrive_expect_tx(sbar, np * (T * 256 + 256));
+    int kb = p0 % nkb;
+    for (int i = 0; i < np; ++i) {
+      tma_load_2d_plain(land + i * T * 64, map_h, sbar, kb * 64, 0);
+      bulk_load(sg + i * 64, gain + kb * 64, 256, sbar);
+      if (++kb == nkb) kb = 0;
     }
-    if (ct < 16) pd_cp16(sg + i * 64 + ct * 4, gain + kb * 64 + ct * 4);
-    if (++kb == nkb) kb = 0;
+    if (mk) mk[8] = globaltimer();
   }
-  if (mk && ct == 0) mk[8] = globaltimer();
-  pd_cp_wait();
-  named_bar_sync(1, kPdCompute);
+  pd_stage_wait(sbar, par, abort_flag);
   if (mk && ct == 0) mk[9] = globaltimer();
   const int tile0_pairs = p0 < nkb ? min(np, nkb - p0) : 0;   // pairs of weight tile 0 add to ssq
   for (int i = 0; i < np; ++i) {
@@ -198,52 +229,65 @@ __device__ __noinline__ void pd_stage_norm(const PdArgs& a, uint8_t* smem, int c
         if (t < T && c8 == 0) atomicAdd(ssq + t, ss);
       }
     }
+    pd_pair_ready(btf, i, ct);
   }
+  return par ^ 1u;
 }
 
-// (C) attention output o = sum_j w_j o_j / sum_j w_j, w_j = l_j 2^(m_j - max m), over the key splits
+// (C) attention output o = sum_j w_j o_j, w_j = l_j 2^(m_j - max m) / sum_j l_j 2^(m_j - max m), over
+// the key splits j
 template <int kT>
-__device__ __noinline__ void pd_stage_attn_out(const PdArgs& a, uint8_t* smem, int ct, int p0, int np, int nkb, unsigned long long* mk) {
+__device__ __noinline__ uint32_t pd_stage_attn_out(const PdArgs& a, uint8_t* smem, int ct, int p0, int np, int nkb,
+                                                   unsigned long long* mk, uint64_t* btf, uint64_t* sbar,
+                                                   uint32_t par, const CUtensorMap* map_po, volatile int* abort_flag) {
   using SM = PdSmem;
   const int T = kT > 0 ? kT : a.T;   // tokens; a compile-time constant for the common shape
   const int c8 = ct & 7;
   const int G = a.n_q / a.n_kv, S = a.splits;
+  const int nrows = np * S * T;
   __nv_bfloat16* lo = reinterpret_cast<__nv_bfloat16*>(smem + SM::kOffLandG);   // [np][S][T][64]
-  float2* lml = reinterpret_cast<float2*>(lo + static_cast<size_t>(np) * S * T * 64);   // [np][S][T]
-  int kb = p0 % nkb;
-  for (int i = 0; i < np; ++i) {
-    const int hq = kb >> 1, g2 = hq / G, hh = hq - g2 * G;
-    for (int sp = 0; sp < S; ++sp) {
-      const size_t src = (static_cast<size_t>(g2) * S + sp) * 128 + hh * T;   // row of token 0
-      const int dst = (i * S + sp) * T;
-      for (int q = ct; q < T * 8; q += kPdCompute) {
-        const int t = q >> 3, c = q & 7;
-        pd_cp16(lo + (dst + t) * 64 + c * 8, a.part_o + (src + t) * 128 + (kb & 1) * 64 + c * 8);
+  float2* lml = reinterpret_cast<float2*>(lo + static_cast<size_t>(nrows) * 64);   // [np][S][T]
+  float* wts = reinterpret_cast<float*>(lml + nrows);                             // [np][S][T]
+  if (ct == 0) {
+    fence_proxy_async_global();
+    mbar_arrive_expect_tx(sbar, nrows * (128 + 8));
+    int kb = p0 % nkb;
+    for (int i = 0; i < np; ++i) {
+      const int hq = kb >> 1, g2 = hq / G, hh = hq - g2 * G;
+      for (int sp = 0; sp < S; ++sp) {
+        const int src = (g2 * S + sp) * 128 + hh * T;   // partial-state row of token 0
+        const int dst = (i * S + sp) * T;
+        tma_load_2d_plain(lo + static_cast<size_t>(dst) * 64, map_po, sbar, (kb & 1) * 64, src);
+        bulk_load(lml + dst, a.part_ml + src, T * 8, sbar);
       }
-      if ((src & 1) == 0 && (T & 1) == 0) {   // (m, l) of two tokens per 16-byte copy
-        for (int q = ct; q < T / 2; q += kPdCompute) pd_cp16(lml + dst + 2 * q, a.part_ml + src + 2 * q);
-      } else {
-        for (int q = ct; q < T; q += kPdCompute) lml[dst + q] = __ldcg(a.part_ml + src + q);
-      }
+      if (++kb == nkb) kb = 0;
     }
-    if (++kb == nkb) kb = 0;
+    if (mk) mk[8] = globaltimer();
   }
-  if (mk && ct == 0) mk[8] = globaltimer();
-  pd_cp_wait();
-  named_bar_sync(1, kPdCompute);
+  pd_stage_wait(sbar, par, abort_flag);
   if (mk && ct == 0) mk[9] = globaltimer();
+  for (int q = ct; q < np * T; q += kPdCompute) {   // normalised split weights of each (pair, token)
+    const int i = q / T, t = q - i * T;
+    float mx = -__int_as_float(0x7f800000);
+    for (int sp = 0; sp < S; ++sp) mx = fmaxf(mx, lml[(i * S + sp) * T + t].x);
+    float den = 0.f;
+    for (int sp = 0; sp < S; ++sp) {
+      const float2 ml = lml[(i * S + sp) * T + t];
+      const float w = ml.y * ex2_fast(ml.x - mx);
+      wts[(i * S + sp) * T + t] = w;
+      den += w;
+    }
+    const float inv = 1.f / den;
+    for (int sp = 0; sp < S; ++sp) wts[(i * S + sp) * T + t] *= inv;
+  }
+  named_bar_sync(1, kPdCompute);
   for (int i = 0; i < np; ++i) {
     for (int u = ct; u < T * 8; u += kPdCompute) {
       const int t = u >> 3;
-      float mx = -__int_as_float(0x7f800000);
-      for (int sp = 0; sp < S; ++sp) mx = fmaxf(mx, lml[(i * S + sp) * T + t].x);
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      float den = 0.f;
       for (int sp = 0; sp < S; ++sp) {
-        const float2 ml = lml[(i * S + sp) * T + t];
-        const float w = ml.y * exp2f(ml.x - mx);
-        den += w;
-        const uint4 ov = *reinterpret_cast<const uint4*>(lo + ((i * S + sp) * T + t) * 64 + c8 * 8);
+        const float w = wts[(i * S + sp) * T + t];
+        const uint4 ov = *reinterpret_cast<const uint4*>(lo + static_cast<size_t>((i * S + sp) * T + t) * 64 + c8 * 8);
         const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -252,37 +296,36 @@ __device__ __noinline__ void pd_stage_attn_out(const PdArgs& a, uint8_t* smem, i
           acc[2 * e + 1] += w * f.y;
         }
       }
-      const float inv = 1.f / den;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] *= inv;
       *reinterpret_cast<uint4*>(smem + SM::kOffWork + i * SM::kBTile + sw_chunk(t, c8)) = pack8(acc);
     }
+    pd_pair_ready(btf, i, ct);
   }
+  return par ^ 1u;
 }
 
 // (E) SwiGLU of the gate/up sums with 1/rms of the MLP norm
 template <int kT>
-__device__ __noinline__ void pd_stage_swiglu(const PdArgs& a, uint8_t* smem, int ct, int p0, int np, int nkb, unsigned long long* mk) {
+__device__ __noinline__ uint32_t pd_stage_swiglu(const PdArgs& a, uint8_t* smem, int ct, int p0, int np, int nkb,
+                                                 unsigned long long* mk, uint64_t* btf, uint64_t* sbar, uint32_t par,
+                                                 const CUtensorMap* map_gu, volatile int* abort_flag) {
   using SM = PdSmem;
   const int T = kT > 0 ? kT : a.T;   // tokens; a compile-time constant for the common shape
   const int c8 = ct & 7;
   const float inv_Ha = 1.0f / a.Ha;
   float* land = reinterpret_cast<float*>(smem + SM::kOffLandG);   // [np][T][128]: gate 64 | up 64
   float* sq = reinterpret_cast<float*>(smem + SM::kOffAux);       // [2T] both sums of squares
-  const float* gu = a.acc_gu;
-  const int ld = 2 * a.Ia;
-  int kb = p0 % nkb;
-  for (int i = 0; i < np; ++i) {
-    for (int q = ct; q < T * 32; q += kPdCompute) {
-      const int t = q >> 5, c = q & 31;
-      pd_cp16(land + (i * T + t) * 128 + c * 4, gu + static_cast<size_t>(t) * ld + 128 * kb + c * 4);
+  if (ct == 0) {
+    fence_proxy_async_global();
+    mbar_arrive_expect_tx(sbar, np * T * 512 + 8 * T);
+    int kb = p0 % nkb;
+    for (int i = 0; i < np; ++i) {
+      tma_load_2d_plain(land + i * T * 128, map_gu, sbar, 128 * kb, 0);
+      if (++kb == nkb) kb = 0;
     }
-    if (++kb == nkb) kb = 0;
+    bulk_load(sq, a.ssq, 8 * T, sbar);
+    if (mk) mk[8] = globaltimer();
   }
-  for (int q = T / 4 + ct; q < (2 * T + 3) / 4; q += kPdCompute) pd_cp16(sq + 4 * q, a.ssq + 4 * q);
-  if (mk && ct == 0) mk[8] = globaltimer();
-  pd_cp_wait();
-  named_bar_sync(1, kPdCompute);
+  pd_stage_wait(sbar, par, abort_flag);
   if (mk && ct == 0) mk[9] = globaltimer();
   for (int i = 0; i < np; ++i) {
     for (int u = ct; u < T * 8; u += kPdCompute) {
@@ -297,123 +340,126 @@ __device__ __noinline__ void pd_stage_swiglu(const PdArgs& a, uint8_t* smem, int
       for (int e = 0; e < 8; ++e) y[e] = silu_f(gg[e] * s) * (uu[e] * s);
       *reinterpret_cast<uint4*>(smem + SM::kOffWork + i * SM::kBTile + sw_chunk(t, c8)) = pack8(y);
     }
+    pd_pair_ready(btf, i, ct);
   }
+  return par ^ 1u;
 }
 
-// Q rows (then the suffix K and V rows) of one attention item.  Build unit = (row, c8): dims
-// [8 c8, 8 c8 + 8) and their RoPE partners [64 + 8 c8, ...) sit in one thread; a row's 8 units are
-// adjacent lanes, so the head's sum of squares is a 3-step shuffle.
+// Rows of Q (one attention item: G heads x T tokens) or of the suffix K and V (a helper CTA), built
+// from the QKV sums.  Build unit = (row, c8): dims [8 c8, 8 c8 + 8) and their RoPE partners
+// [64 + 8 c8, ...) sit in one thread; a row's 8 units are adjacent lanes, so the head's sum of
+// squares is a 3-step shuffle.  kv = false: Q rows into the Q tile; kv = true: K rows 0..63 and V
+// rows 64..127, written in the SW128 tile layout to `kv_out` (global) instead of shared memory.
 template <int kT>
-__device__ __noinline__ void pd_stage_qkv(const PdArgs& a, uint8_t* smem, int ct, int l, int kvg, bool has_sfx, unsigned long long* mk) {
+__device__ __noinline__ uint32_t pd_stage_qkv(const PdArgs& a, uint8_t* smem, int ct, int l, int kvg, bool kv,
+                                              __nv_bfloat16* kv_out, unsigned long long* mk, uint64_t* sbar,
+                                              uint32_t par, const CUtensorMap* map_qkv, volatile int* abort_flag) {
   using SM = PdSmem;
   const int T = kT > 0 ? kT : a.T;   // tokens; a compile-time constant for the common shape
   const int c8 = ct & 7;
   const int G = a.n_q / a.n_kv, GT = G * T;
   const int qd = a.n_q * 128, kvd = a.n_kv * 128;
   const float inv_Ha = 1.0f / a.Ha;
-  const int QR = a.QR;
-  const float* acc = a.acc_qkv;
   float* land = reinterpret_cast<float*>(smem + SM::kOffLandA);   // [128 rows][128]
   // the P buffers are idle while the operands are built: sums of squares, QK-norm gains, RoPE rows
-  float* sq = reinterpret_cast<float*>(smem + SM::kOffP);             // [T]
+  float* sq = reinterpret_cast<float*>(smem + SM::kOffP);             // [T] (+ padding to 16 bytes)
   float* sgq = reinterpret_cast<float*>(smem + SM::kOffP + 256);      // [128]
   float* sgk = reinterpret_cast<float*>(smem + SM::kOffP + 768);      // [128]
   float2* srope = reinterpret_cast<float2*>(smem + SM::kOffP + 1280); // [T][64] (cos, sin) at P + t
-  for (int set = 0; set < (has_sfx ? 2 : 1); ++set) {
-    const bool kv = set == 1;
-    // rows: Q (set 0) r < GT = (head-in-group r / T, token r % T); K (set 1) r < 64, V r >= 64
+  if (ct == 0) {
+    const PdLayer& ly = a.layers[l];
+    const uint32_t sq_bytes = (4 * T + 15) & ~15u;
+    fence_proxy_async_global();
+    mbar_arrive_expect_tx(sbar, (kv ? 2 : G) * T * 512 + T * 512 + 1024 + sq_bytes);
     if (!kv) {
       for (int r = 0; r < G; ++r)   // head r of the group: rows r T .. r T + T - 1
-        for (int q = ct; q < T * 32; q += kPdCompute) {
-          const int t = q >> 5, c = q & 31;
-          pd_cp16(land + (r * T + t) * 128 + c * 4, acc + static_cast<size_t>(t) * QR + (kvg * G + r) * 128 + c * 4);
-        }
-      const PdLayer& ly = a.layers[l];
-      for (int q = ct; q < (T + 3) / 4; q += kPdCompute) pd_cp16(sq + 4 * q, a.ssq + 4 * q);
-      if (ct < 32) pd_cp16(sgq + 4 * ct, ly.q_norm + 4 * ct);
-      else if (ct < 64) pd_cp16(sgk + 4 * (ct - 32), ly.k_norm + 4 * (ct - 32));
-      for (int q = ct; q < T * 32; q += kPdCompute)
-        pd_cp16(reinterpret_cast<float*>(srope) + 4 * q, reinterpret_cast<const float*>(a.rope + static_cast<size_t>(a.P) * 64) + 4 * q);
+        tma_load_2d_plain(land + r * T * 128, map_qkv, sbar, (kvg * G + r) * 128, 0);
     } else {
-      for (int w = 0; w < 2; ++w)
-        for (int q = ct; q < T * 32; q += kPdCompute) {
-          const int t = q >> 5, c = q & 31;
-          pd_cp16(land + (w * 64 + t) * 128 + c * 4, acc + static_cast<size_t>(t) * QR + qd + w * kvd + kvg * 128 + c * 4);
-        }
+      for (int w = 0; w < 2; ++w)   // K rows at 0.., V rows at 64..
+        tma_load_2d_plain(land + w * 64 * 128, map_qkv, sbar, qd + w * kvd + kvg * 128, 0);
     }
-    if (mk && ct == 0 && set == 0) mk[8] = globaltimer();
-    pd_cp_wait();
-    named_bar_sync(1, kPdCompute);
-    if (mk && ct == 0 && set == 0) mk[9] = globaltimer();
-    for (int u = ct; u < 1024; u += kPdCompute) {   // 128 rows x 8 units; warp-uniform trip count
-      const int r = u >> 3;
-      const bool valid = kv ? (r & 63) < T : r < GT;
-      const int which = kv ? (r >> 6) : 0;
-      const int t = kv ? (r & 63) : (valid ? r % T : 0);
-      float x[16];
-      if (valid) {
-        const float4* s4 = reinterpret_cast<const float4*>(land + r * 128);
-        const float4 v0 = s4[2 * c8], v1 = s4[2 * c8 + 1], v2 = s4[16 + 2 * c8], v3 = s4[16 + 2 * c8 + 1];
-        x[0] = v0.x, x[1] = v0.y, x[2] = v0.z, x[3] = v0.w, x[4] = v1.x, x[5] = v1.y, x[6] = v1.z, x[7] = v1.w;
-        x[8] = v2.x, x[9] = v2.y, x[10] = v2.z, x[11] = v2.w, x[12] = v3.x, x[13] = v3.y, x[14] = v3.z, x[15] = v3.w;
-      } else {
-#pragma unroll
-        for (int e = 0; e < 16; ++e) x[e] = 0.f;
-      }
-      float ss = 0.f;
-#pragma unroll
-      for (int e = 0; e < 16; ++e) ss += x[e] * x[e];
-      ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-      ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-      ss += __shfl_xor_sync(0xffffffffu, ss, 4);
-      uint8_t* dst;
-      uint32_t hstride;
-      int drow;
-      if (!kv) {
-        dst = smem + SM::kOffQ, hstride = 16384, drow = r;
-      } else {
-        dst = smem + (which ? SM::kOffSV : SM::kOffSK), hstride = 8192, drow = r & 63;
-      }
-      if (valid) {
-        const float s = rsqrtf(sq[t] * inv_Ha + a.eps);
-        if (kv && which == 1) {   // V: 1/rms only
-#pragma unroll
-          for (int e = 0; e < 16; ++e) x[e] *= s;
-        } else {                  // Q / K: 1/rms, RMSNorm over the head, RoPE at position P + t
-          const float* gain = kv ? sgk : sgq;
-          const float rn = s * rsqrtf(ss * s * s / 128.f + a.eps);
-          const float2* cs = srope + t * 64 + c8 * 8;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int d = c8 * 8 + e;
-            const float2 c2 = cs[e];
-            const float x0 = x[e] * rn * gain[d], x1 = x[8 + e] * rn * gain[d + 64];
-            x[e] = x0 * c2.x - x1 * c2.y;
-            x[8 + e] = x1 * c2.x + x0 * c2.y;
-          }
-        }
-      }
-      *reinterpret_cast<uint4*>(dst + sw_chunk(drow, c8)) = pack8(x);
-      *reinterpret_cast<uint4*>(dst + hstride + sw_chunk(drow, c8)) = pack8(x + 8);
-    }
-    named_bar_sync(1, kPdCompute);   // the landing area is reused by the next set
+    bulk_load(srope, a.rope + static_cast<size_t>(a.P) * 64, T * 512, sbar);
+    bulk_load(sgq, ly.q_norm, 512, sbar);
+    bulk_load(sgk, ly.k_norm, 512, sbar);
+    bulk_load(sq, a.ssq, sq_bytes, sbar);
+    if (mk) mk[8] = globaltimer();
   }
+  pd_stage_wait(sbar, par, abort_flag);
+  if (mk && ct == 0) mk[9] = globaltimer();
+#pragma unroll 1
+  for (int u = ct; u < 1024; u += kPdCompute) {   // 128 rows x 8 units; warp-uniform trip count
+    const int r = u >> 3;
+    const bool valid = kv ? (r & 63) < T : r < GT;
+    const int which = kv ? (r >> 6) : 0;
+    const int t = kv ? (r & 63) : (valid ? r % T : 0);
+    float x[16];
+    if (valid) {
+      const float4* s4 = reinterpret_cast<const float4*>(land + r * 128);
+      const float4 v0 = s4[2 * c8], v1 = s4[2 * c8 + 1], v2 = s4[16 + 2 * c8], v3 = s4[16 + 2 * c8 + 1];
+      x[0] = v0.x, x[1] = v0.y, x[2] = v0.z, x[3] = v0.w, x[4] = v1.x, x[5] = v1.y, x[6] = v1.z, x[7] = v1.w;
+      x[8] = v2.x, x[9] = v2.y, x[10] = v2.z, x[11] = v2.w, x[12] = v3.x, x[13] = v3.y, x[14] = v3.z, x[15] = v3.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) x[e] = 0.f;
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) ss += x[e] * x[e];
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+    if (valid) {
+      const float s = rsqrtf(sq[t] * inv_Ha + a.eps);
+      if (kv && which == 1) {   // V: 1/rms only
+#pragma unroll
+        for (int e = 0; e < 16; ++e) x[e] *= s;
+      } else {                  // Q / K: 1/rms, RMSNorm over the head, RoPE at position P + t
+        const float* gain = kv ? sgk : sgq;
+        const float rn = s * rsqrtf(ss * s * s / 128.f + a.eps);
+        const float2* cs = srope + t * 64 + c8 * 8;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int d = c8 * 8 + e;
+          const float2 c2 = cs[e];
+          const float x0 = x[e] * rn * gain[d], x1 = x[8 + e] * rn * gain[d + 64];
+          x[e] = x0 * c2.x - x1 * c2.y;
+          x[8 + e] = x1 * c2.x + x0 * c2.y;
+        }
+      }
+    }
+    if (!kv) {
+      uint8_t* dst = smem + SM::kOffQ;
+      *reinterpret_cast<uint4*>(dst + sw_chunk(r, c8)) = pack8(x);
+      *reinterpret_cast<uint4*>(dst + 16384 + sw_chunk(r, c8)) = pack8(x + 8);
+    } else {
+      uint8_t* dst = reinterpret_cast<uint8_t*>(kv_out) + which * 16384;
+      *reinterpret_cast<uint4*>(dst + sw_chunk(r & 63, c8)) = pack8(x);
+      *reinterpret_cast<uint4*>(dst + 8192 + sw_chunk(r & 63, c8)) = pack8(x + 8);
+    }
+  }
+  return par ^ 1u;
 }
 
-// the 50-token chunk of one observation gets staging code with the token count folded in
-#define PD_STAGE(fn, ...)          \
-  do {                             \
-    if (a.T == 50)                 \
-      fn<50>(__VA_ARGS__);         \
-    else                           \
-      fn<0>(__VA_ARGS__);          \
-  } while (0)
+// step boundary of token blockIdx.x (velocity, Euler update, next input), out of line
+__device__ __noinline__ void pd_step(const PdArgs& a, int k_out, int k_in, int ct, float* sx, float* sred, float* hs) {
+  StepArgs s = a.step;
+  s.k_out = k_out;
+  s.k_in = k_in;
+  step_token(s, blockIdx.x, ct, kPdCompute, sx, sred, hs, [] { named_bar_sync(1, kPdCompute); });
+}
+
+// the 50-token chunk of one observation gets staging code with the token count folded in; the value
+// is the stage barrier's next parity
+#define PD_STAGE(fn, ...) (a.T == 50 ? fn<50>(__VA_ARGS__) : fn<0>(__VA_ARGS__))
 
 __global__ void __launch_bounds__(kPdThreads, 1)
     denoise_persistent_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmO,
                               const __grid_constant__ CUtensorMap tmGU, const __grid_constant__ CUtensorMap tmD,
                               const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                              const __grid_constant__ PdArgs a) {
+                              const __grid_constant__ CUtensorMap tmAccQKV, const __grid_constant__ CUtensorMap tmH,
+                              const __grid_constant__ CUtensorMap tmAccGU, const __grid_constant__ CUtensorMap tmHLd,
+                              const __grid_constant__ CUtensorMap tmGULd, const __grid_constant__ CUtensorMap tmQKVLd,
+                              const __grid_constant__ CUtensorMap tmPO, const __grid_constant__ PdArgs a) {
   using SM = PdSmem;
   constexpr int NST = kPdStages;
   extern __shared__ uint8_t pd_smem_raw[];
@@ -428,15 +474,17 @@ __global__ void __launch_bounds__(kPdThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kOffBar);
   uint64_t* ring_full = bars;              // [NST] TMA landed
   uint64_t* ring_empty = bars + NST;       // [NST] the MMAs that read the stage completed
-  uint64_t* btile_full = bars + 2 * NST;   // activation tiles of this GEMM phase staged
-  uint64_t* acc_full = btile_full + 1;     // [2] accumulator segment complete
+  uint64_t* btile_full = bars + 2 * NST;   // [kPdBTiles] activation tile of staged pair i ready
+  uint64_t* acc_full = btile_full + kPdBTiles;   // [2] accumulator segment complete
   uint64_t* q_ready = acc_full + 2;        // Q (and the suffix K/V) staged
   uint64_t* s_full = q_ready + 1;          // [2]
   uint64_t* s_free = s_full + 2;           // [2]
   uint64_t* p_full = s_free + 2;           // [2] P_i in buffer i % 2 (and O corrected)
   uint64_t* pv_done = p_full + 2;          // [2] PV_i (which read buffer i % 2) finished
   uint64_t* drain = pv_done + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* stage_bar = drain + 1;         // TMA copies of a phase's operand data landed
+  uint64_t* kvs_ready = stage_bar + 1;     // suffix K/V tiles copied in from the helper CTA
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(kvs_ready + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* sx = reinterpret_cast<float*>(smem + SM::kOffMisc);   // [64]
   float* sred = sx + 64;                                        // [8]
@@ -454,25 +502,29 @@ __global__ void __launch_bounds__(kPdThreads, 1)
   const int nb = jb1 - jb0;
   const int npre = max(0, min(jb1, nA) - jb0);    // prefix blocks of this item
   const bool has_sfx = has_item && jb1 > nA;
+  // helper CTA of KV head (blockIdx.x - n_items): builds that head's suffix K and V each layer
+  const bool kv_helper = !has_item && static_cast<int>(blockIdx.x) < n_items + a.n_kv;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NST; ++i) {
       mbar_init(&ring_full[i], 1);
       mbar_init(&ring_empty[i], 1);
     }
-    mbar_init(btile_full, 1);
+    for (int i = 0; i < kPdBTiles; ++i) mbar_init(&btile_full[i], kPdCompute / 32);
     mbar_init(&acc_full[0], 1);
     mbar_init(&acc_full[1], 1);
-    mbar_init(q_ready, 1);
+    mbar_init(q_ready, kPdCompute / 32);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);
+      mbar_init(&s_free[i], kPdCompute / 32);   // every compute warp reads its half of S
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&p_full[i], 4);
+      mbar_init(&p_full[i], kPdCompute / 32);
       mbar_init(&pv_done[i], 1);
     }
     mbar_init(drain, 1);
+    mbar_init(stage_bar, 1);
+    mbar_init(kvs_ready, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -523,6 +575,26 @@ __global__ void __launch_bounds__(kPdThreads, 1)
                   ++rs;
                 }
               }
+              if (ok && has_sfx) {
+                // the suffix K/V tiles of this layer, built by this head's helper CTA in the same phase
+                const unsigned want = 2u + static_cast<unsigned>(k * (5 * a.L + 1) + 5 * l + 1);
+                const uint64_t t0 = globaltimer();
+                for (uint32_t it = 0;; ++it) {
+                  if (ld_acquire_u32(a.sync + 2 + kvg) >= want) break;
+                  if ((it & 15u) == 15u && (*abort_flag || globaltimer() - t0 > kWaitTimeoutNs)) {
+                    ok = false;
+                    break;
+                  }
+                  __nanosleep(64);
+                }
+                if (ok) {
+                  fence_proxy_async_global();
+                  mbar_arrive_expect_tx(kvs_ready, 32768);
+                  const __nv_bfloat16* src = a.kv_sfx + static_cast<size_t>(kvg) * 16384;
+                  bulk_load(smem + SM::kOffSK, src, 16384, kvs_ready);
+                  bulk_load(smem + SM::kOffSV, src + 8192, 16384, kvs_ready);
+                }
+              }
               continue;
             }
             int tiles, nkb, rpl, p0, p1;
@@ -557,7 +629,7 @@ __global__ void __launch_bounds__(kPdThreads, 1)
       const uint32_t idesc_g = idesc_bf16_f32(128, 64);
       const uint32_t idesc_s = idesc_bf16_f32(128, 64);
       const uint32_t idesc_pv = idesc_bf16_f32(128, 128) | (1u << 16);   // B (V) is MN-major
-      uint32_t rs = 0, n_gemm = 0, n_att = 0, blk = 0;
+      uint32_t rs = 0, n_att = 0, n_sfx = 0, blk = 0, bt_par = 0;   // bt_par bit i: parity of btile_full[i]
       bool ok = true;
       auto mmark = [&](int k, int l, int ph, int slot) {
         if (a.trace) {
@@ -620,6 +692,11 @@ __global__ void __launch_bounds__(kPdThreads, 1)
                   }
                   kaddr = smem_u32(smem + SM::kOffRing + kst * SM::kStage);
                 } else {
+                  if (!mbar_wait(kvs_ready, n_sfx & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                  }
+                  ++n_sfx;
                   kaddr = smem_u32(smem + SM::kOffSK);
                 }
                 if (i >= 2 && !mbar_wait(&s_free[sb], ((i >> 1) - 1) & 1, abort_flag)) {
@@ -648,22 +725,22 @@ __global__ void __launch_bounds__(kPdThreads, 1)
             pd_geom(a, ph, tiles, nkb, rpl);
             pd_range(tiles * nkb, blockIdx.x, gridDim.x, p0, p1);
             if (p0 >= p1) continue;
-            if (!mbar_wait(btile_full, n_gemm & 1, abort_flag)) {
-              ok = false;
-              break;
-            }
-            ++n_gemm;
-            mmark(k, l, ph, 6);
-            tc_fence_after();
-            int seg = 0, seg_start = p0, cur_tile = p0 / nkb;
+            int seg = 0, seg_start = p0, cur_tile = p0 / nkb, kbc = p0 - cur_tile * nkb;
             for (int p = p0; p < p1; ++p) {
-              const int tile = p / nkb;
-              if (tile != cur_tile) {
+              if (p > p0 && ++kbc == nkb) {   // next weight tile
+                kbc = 0;
                 umma_commit(&acc_full[seg]);
                 ++seg;
-                cur_tile = tile;
+                ++cur_tile;
                 seg_start = p;
               }
+              const int i = p - p0;
+              if (!mbar_wait(&btile_full[i], (bt_par >> i) & 1u, abort_flag)) {
+                ok = false;
+                break;
+              }
+              bt_par ^= 1u << i;
+              if (i == 0) mmark(k, l, ph, 6);
               const int st = full_stage(rs);
               if (st < 0) {
                 ok = false;
@@ -701,7 +778,7 @@ __global__ void __launch_bounds__(kPdThreads, 1)
     const float inv_Ha = 1.0f / a.Ha;
     float* ssq_attn = a.ssq;
     float* ssq_mlp = a.ssq + a.T;
-    uint32_t gen = 0, acc_use[2] = {0u, 0u}, blk = 0;
+    uint32_t gen = 0, acc_use[2] = {0u, 0u}, blk = 0, stage_par = 0;
     bool ok = true;
     auto csync = [] { named_bar_sync(1, kPdCompute); };
     // one lane waits, the whole warp gets the same answer (the warp-collective TMEM loads that follow
@@ -756,144 +833,150 @@ __global__ void __launch_bounds__(kPdThreads, 1)
     };
 
     // (A, D) bf16(g * h) for pairs [p0, p0 + np); weight tile 0 also adds sum h^2 into ssq
-    auto btiles_ready = [&] {
-      fence_async_smem();
-      tc_fence_before();
-      csync();
-      if (ct == 0) mbar_arrive(btile_full);
-      mark(1);
-    };
-    // accumulator segments -> fp32 reductions into dst[t][feature]; this thread: feature row r,
-    // tokens [32 half, 32 half + 32)
-    auto reduce_out = [&](int p0, int p1, int nkb, float* dst, int ld) -> bool {
-      int seg = 0;
-      for (int tt = p0 / nkb; tt <= (p1 - 1) / nkb; ++tt, ++seg) {
-        if (!warp_wait(&acc_full[seg], acc_use[seg] & 1)) return false;
+    // accumulator segments -> fp32 tile [64 tokens][128 features] per segment in shared memory, then
+    // one TMA bulk reduce-add per segment into dst[t][feature]; this thread: feature row r, tokens
+    // [32 half, 32 half + 32)
+    auto reduce_out = [&](int p0, int p1, int nkb, const CUtensorMap* map) -> bool {
+      const int tt0 = p0 / nkb, nseg = (p1 - 1) / nkb - tt0 + 1;
+      bool good = true;
+      for (int seg = 0; seg < nseg && good; ++seg) {
+        if (!warp_wait(&acc_full[seg], acc_use[seg] & 1)) {
+          good = false;
+          break;
+        }
         ++acc_use[seg];
         if (seg == 0) mark(2);
         tc_fence_after();
-        float* col = dst + tt * 128 + r;
+        float* rt = reinterpret_cast<float*>(smem + SM::kOffLandG + seg * 32768);
 #pragma unroll 1
         for (int hc = half; hc < 2; hc += kPdHalves) {
           float v[32];
           tmem_ld32(tl + seg * 64 + hc * 32, v);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int t = hc * 32 + j;
-            if (t < a.T) atomicAdd(col + static_cast<size_t>(t) * ld, v[j]);
-          }
+          for (int j = 0; j < 32; ++j) rt[(hc * 32 + j) * 128 + r] = v[j];
         }
       }
       tc_fence_before();
-      return true;
+      fence_async_smem();
+      csync();
+      // (earlier generic writes to the destination, the zeroing and other CTAs' sums, are ordered before
+      // these async-proxy adds by the proxy fence this thread issued before the phase's operand copies)
+      if (ct == 0 && *abort_flag == 0 && good) {
+        for (int seg = 0; seg < nseg; ++seg)
+          tma_reduce_add_2d(map, smem + SM::kOffLandG + seg * 32768, (tt0 + seg) * 128, 0);
+        bulk_commit();
+        bulk_wait_all();
+        fence_proxy_async_global();   // the sums are in place before this CTA's barrier arrival
+      }
+      return good;
     };
     auto step_phase = [&](int k_out, int k_in) {
-      if (static_cast<int>(blockIdx.x) < a.T) {
-        StepArgs s = a.step;
-        s.k_out = k_out;
-        s.k_in = k_in;
-        step_token(s, blockIdx.x, ct, kPdCompute, sx, sred, reinterpret_cast<float*>(smem + SM::kOffLandG), csync);
-      }
+      if (static_cast<int>(blockIdx.x) < a.T) pd_step(a, k_out, k_in, ct, sx, sred, reinterpret_cast<float*>(smem + SM::kOffLandG));
     };
     // ---- attention of one (KV head, key split) item
     auto attention = [&](int l) -> bool {
       const PdLayer& ly = a.layers[l];
       const int GT = G * a.T;
-      PD_STAGE(pd_stage_qkv, a, smem, ct, l, kvg, has_sfx, mk_row());
+      stage_par = PD_STAGE(pd_stage_qkv, a, smem, ct, l, kvg, false, nullptr, mk_row(), stage_bar, stage_par,
+                           &tmQKVLd, abort_flag);
       fence_async_smem();
       tc_fence_before();
-      csync();
-      if (ct == 0) mbar_arrive(q_ready);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_ready);   // one arrival per compute warp
       mark(1);
 
-      float m_ref = -__int_as_float(0x7f800000), l_run = 0.f;
-      if (half == 0) {   // softmax: warps 2-5, one thread per query row
-        for (int b = 0; b < nb; ++b) {
-          const uint32_t i = blk + b;
-          const int sb = i & 1;
-          if (!warp_wait(&s_full[sb], (i >> 1) & 1)) break;
-          if (b == 0) mark(2);
-          if (b < 2) mark(10 + 2 * b);
-          tc_fence_after();
-          const int jj = jb0 + b;
-          const int nvalid = jj < nA ? min(64, a.P - jj * 64) : a.T;
-          float mx = -__int_as_float(0x7f800000);
-#pragma unroll 1
-          for (int hc = 0; hc < 2; ++hc) {   // pass 1: the block max over the valid keys
-            float sv[32];
-            tmem_ld32(tl + sb * 64 + hc * 32, sv);
+      // softmax: two threads per query row (warp w and w + 4 share a TMEM lane quarter), each on 32 of
+      // the block's 64 keys; the row max is exchanged through shared memory once per block
+      float m_ref = -__int_as_float(0x7f800000), l_run = 0.f;   // l_run: this half's share of the row sum
+      // [2 blocks][2 halves][128 rows], in landing rows 112.. (Q uses rows < G T <= 112; a warp may
+      // start here while others still convert Q from the landing area)
+      float* xm = reinterpret_cast<float*>(smem + SM::kOffLandA + 112 * 512);
+      for (int b = 0; b < nb; ++b) {
+        const uint32_t i = blk + b;
+        const int sb = i & 1;
+        bool good = *abort_flag == 0 && warp_wait(&s_full[sb], (i >> 1) & 1);
+        if (b == 0) mark(2);
+        if (b < 2) mark(10 + 2 * b);
+        tc_fence_after();
+        const int jj = jb0 + b;
+        const int nvalid = jj < nA ? min(64, a.P - jj * 64) : a.T;
+        float sv[32];
+        float mx = -__int_as_float(0x7f800000);
+        if (good) {
+          tmem_ld32(tl + sb * 64 + half * 32, sv);
 #pragma unroll
-            for (int q = 0; q < 32; ++q)
-              if (hc * 32 + q < nvalid) mx = fmaxf(mx, sv[q]);
-          }
-          const float m_blk = mx * a.scale_log2;
-          const bool move = m_blk > m_ref + 8.f;   // also true on the first block
-          const float m_new = move ? m_blk : m_ref;
-          const float alpha = move ? exp2f(m_ref - m_new) : 1.f;
-          const bool any_move = __any_sync(0xffffffffu, move);
-          // P buffer i % 2 is free once PV_{i-2} completed
-          if (i >= 2 && !warp_wait(&pv_done[sb], ((i >> 1) - 1) & 1)) break;
+          for (int q = 0; q < 32; ++q)
+            if (half * 32 + q < nvalid) mx = fmaxf(mx, sv[q]);
+        }
+        xm[((b & 1) * 2 + half) * 128 + r] = mx;
+        csync();
+        mx = fmaxf(mx, xm[((b & 1) * 2 + (half ^ 1)) * 128 + r]);
+        const float m_blk = mx * a.scale_log2;
+        const bool move = m_blk > m_ref + 8.f;   // also true on the first block
+        const float m_new = move ? m_blk : m_ref;
+        const float alpha = move ? exp2f(m_ref - m_new) : 1.f;
+        const bool any_move = __any_sync(0xffffffffu, move);
+        // P buffer i % 2 is free once PV_{i-2} completed
+        if (good && i >= 2) good = warp_wait(&pv_done[sb], ((i >> 1) - 1) & 1);
+        float sum = 0.f;
+        if (good) {
           uint8_t* ps = smem + SM::kOffP + sb * 16384;
-          float sum = 0.f;
-#pragma unroll 1
-          for (int hc = 0; hc < 2; ++hc) {   // pass 2: P = 2^(s scale - m) in bf16, the row sum
-            float sv[32];
-            tmem_ld32(tl + sb * 64 + hc * 32, sv);
-            uint32_t pk[16];
+          uint32_t pk[16];
 #pragma unroll
-            for (int q = 0; q < 32; q += 2) {
-              const int kq = hc * 32 + q;
-              const float e0 = kq < nvalid ? ex2_fast(fmaf(sv[q], a.scale_log2, -m_new)) : 0.f;
-              const float e1 = kq + 1 < nvalid ? ex2_fast(fmaf(sv[q + 1], a.scale_log2, -m_new)) : 0.f;
-              sum += e0 + e1;
-              pk[q >> 1] = bf2(e0, e1);
-            }
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-              *reinterpret_cast<uint4*>(ps + sw_chunk(r, hc * 4 + c)) =
-                  make_uint4(pk[c * 4], pk[c * 4 + 1], pk[c * 4 + 2], pk[c * 4 + 3]);
+          for (int q = 0; q < 32; q += 2) {
+            const int kq = half * 32 + q;
+            const float e0 = kq < nvalid ? ex2_fast(fmaf(sv[q], a.scale_log2, -m_new)) : 0.f;
+            const float e1 = kq + 1 < nvalid ? ex2_fast(fmaf(sv[q + 1], a.scale_log2, -m_new)) : 0.f;
+            sum += e0 + e1;
+            pk[q >> 1] = bf2(e0, e1);
           }
-          // S buffer consumed: the MMA warp may overwrite it with S_{i+2}
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&s_free[sb]);
-          l_run = l_run * alpha + sum;
-          m_ref = m_new;
-          // O is rescaled only after PV_{i-1}
-          if (b >= 1 && any_move) {
-            if (!warp_wait(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1)) break;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<uint4*>(ps + sw_chunk(r, half * 4 + c)) =
+                make_uint4(pk[c * 4], pk[c * 4 + 1], pk[c * 4 + 2], pk[c * 4 + 3]);
+        }
+        // S buffer consumed: the MMA warp may overwrite it with S_{i+2}
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_free[sb]);
+        l_run = l_run * alpha + sum;
+        m_ref = m_new;
+        // O (this half's 64 columns) is rescaled only after PV_{i-1}
+        if (good && b >= 1 && any_move) {
+          good = warp_wait(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1);
+          if (good) {
             tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
               float o[32];
-              tmem_ld32(tl + 128 + c * 32, o);
+              tmem_ld32(tl + 128 + half * 64 + c * 32, o);
 #pragma unroll
               for (int q = 0; q < 32; ++q) o[q] *= alpha;
-              tmem_st32(tl + 128 + c * 32, o);
+              tmem_st32(tl + 128 + half * 64 + c * 32, o);
             }
             tmem_wait_st();
           }
-          fence_async_smem();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&p_full[sb]);
-          if (b < 2) mark(11 + 2 * b);
         }
+        fence_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[sb]);
+        if (b < 2) mark(11 + 2 * b);
       }
       if (nb > 0) {
         // all eight warps read O: (row r, 64 of the 128 columns); (m, l) of the row via shared memory
         // (m, l) of each row pass to the other half through the Q tile: the last S MMA, the last
         // reader of Q, completed before the softmax finished
-        float2* sml = reinterpret_cast<float2*>(smem + SM::kOffQ);
+        float2* sml = reinterpret_cast<float2*>(smem + SM::kOffQ);   // [2 halves][128 rows]
         const uint32_t il = blk + nb - 1;
-        if (half == 0) sml[r] = make_float2(m_ref, l_run);
+        sml[half * 128 + r] = make_float2(m_ref, l_run);
         csync();
         if (ct == 0 && *abort_flag == 0 && !mbar_wait(&pv_done[il & 1], (il >> 1) & 1, abort_flag)) *abort_flag = 1;
         csync();
         if (*abort_flag) return false;
         mark(14);
         tc_fence_after();
-        const float2 ml = sml[r];
+        const float2 ml = make_float2(m_ref, sml[r].y + sml[128 + r].y);
         const float inv = 1.f / ml.y;
         const size_t mine = static_cast<size_t>(item) * 128 + r;
 #pragma unroll 1
@@ -924,6 +1007,16 @@ __global__ void __launch_bounds__(kPdThreads, 1)
           mark(0);
           if (ph == 1) {
             if (has_item && !attention(l)) *abort_flag = 1;
+            if (kv_helper) {
+              const int g = blockIdx.x - n_items;
+              stage_par = PD_STAGE(pd_stage_qkv, a, smem, ct, l, g, true, a.kv_sfx + static_cast<size_t>(g) * 16384,
+                                   mk_row(), stage_bar, stage_par, &tmQKVLd, abort_flag);
+              csync();
+              if (ct == 0) {
+                __threadfence();
+                asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(a.sync + 2 + g), "r"(gen + 1u) : "memory");
+              }
+            }
             mark(3);
             ok = grid_sync();
             continue;
@@ -933,11 +1026,11 @@ __global__ void __launch_bounds__(kPdThreads, 1)
           pd_range(tiles * nkb, blockIdx.x, gridDim.x, p0, p1);
           const int np = p1 - p0;
           if (np > 0) {
-            if (ph == 0) PD_STAGE(pd_stage_norm, a, smem, ct, p0, np, nkb, ly.attn_norm, ssq_attn, mk_row());
-            else if (ph == 2) PD_STAGE(pd_stage_attn_out, a, smem, ct, p0, np, nkb, mk_row());
-            else if (ph == 3) PD_STAGE(pd_stage_norm, a, smem, ct, p0, np, nkb, ly.mlp_norm, ssq_mlp, mk_row());
-            else PD_STAGE(pd_stage_swiglu, a, smem, ct, p0, np, nkb, mk_row());
-            btiles_ready();
+            if (ph == 0) stage_par = PD_STAGE(pd_stage_norm, a, smem, ct, p0, np, nkb, ly.attn_norm, ssq_attn, mk_row(), btile_full, stage_bar, stage_par, &tmHLd, abort_flag);
+            else if (ph == 2) stage_par = PD_STAGE(pd_stage_attn_out, a, smem, ct, p0, np, nkb, mk_row(), btile_full, stage_bar, stage_par, &tmPO, abort_flag);
+            else if (ph == 3) stage_par = PD_STAGE(pd_stage_norm, a, smem, ct, p0, np, nkb, ly.mlp_norm, ssq_mlp, mk_row(), btile_full, stage_bar, stage_par, &tmHLd, abort_flag);
+            else stage_par = PD_STAGE(pd_stage_swiglu, a, smem, ct, p0, np, nkb, mk_row(), btile_full, stage_bar, stage_par, &tmGULd, abort_flag);
+            mark(1);
           }
           // scratch of the other half of the layer, idle in this phase
           if (ph == 0) {
@@ -948,9 +1041,8 @@ __global__ void __launch_bounds__(kPdThreads, 1)
             if (blockIdx.x == 0 && ct < a.T) ssq_attn[ct] = 0.f;
           }
           if (np > 0) {
-            float* dst = ph == 0 ? a.acc_qkv : (ph == 3 ? a.acc_gu : a.h);
-            const int ld = ph == 0 ? a.QR : (ph == 3 ? 2 * a.Ia : a.Ha);
-            if (!reduce_out(p0, p1, nkb, dst, ld)) *abort_flag = 1;
+            const CUtensorMap* map = ph == 0 ? &tmAccQKV : (ph == 3 ? &tmAccGU : &tmH);
+            if (!reduce_out(p0, p1, nkb, map)) *abort_flag = 1;
           }
           mark(3);
           ok = grid_sync();

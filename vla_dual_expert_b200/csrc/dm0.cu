@@ -127,7 +127,8 @@ struct dm0_ctx {
   bf16* stage_prefix = nullptr;
   // persistent Euler loop: split-K sums, sums of squares, grid-barrier words, per-layer norm gains
   float *pacc_qkv = nullptr, *pacc_gu = nullptr, *pssq = nullptr;
-  unsigned* psync = nullptr;
+  unsigned* psync = nullptr;   // [0] barrier, [1] abort, [2 + g] suffix K/V flags
+  bf16* pkv_sfx = nullptr;      // [n_kv][2][64][128] suffix K/V tiles built by the helper CTAs
   dm0::PdLayer* players = nullptr;
   unsigned long long* ptrace = nullptr;   // DM0_PERSIST_TRACE=1: phase timestamps of the persistent loop
   int ptrace_steps = 0;
@@ -212,6 +213,25 @@ dm0_status get_tmap(dm0_ctx* c, CUtensorMap* out, const void* ptr, uint64_t rows
   if (r != CUDA_SUCCESS) return fail(c, DM0_ECUDA, "cuTensorMapEncodeTiled failed (" + std::to_string(r) + ")");
   c->tmaps[key] = m;
   *out = m;
+  return DM0_OK;
+}
+
+// 2-D map without swizzle (row-major boxes of box_cols x box_rows): fp32 (esize 4) or bf16 (esize 2);
+// the persistent Euler loop's operand copies and split-K reduce-adds
+dm0_status get_tmap_plain(dm0_ctx* c, CUtensorMap* out, const void* ptr, int esize, uint64_t rows, uint64_t cols,
+                          uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(c, DM0_ECUDA, "cuTensorMapEncodeTiled is unavailable");
+  if (reinterpret_cast<uintptr_t>(ptr) % 16 != 0 || (cols * esize) % 16 != 0 || (box_cols * esize) % 16 != 0)
+    return fail(c, DM0_EINVAL, "TMA operand must be 16-byte aligned with 16-byte rows");
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * esize};
+  cuuint32_t boxd[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(out, esize == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void*>(ptr), dims, strides, boxd, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(c, DM0_ECUDA, "cuTensorMapEncodeTiled (plain) failed (" + std::to_string(r) + ")");
   return DM0_OK;
 }
 
@@ -591,7 +611,8 @@ bool persist_plan(dm0_ctx* c, int steps, float* vel, dm0::PdArgs* a, std::string
   if (!c->use_persist) return no("disabled");
   if (g.head_dim != 128) return no("head_dim != 128");
   const int B = c->kv_B, P = c->kv_P, T = B * g.chunk, G = g.n_q / g.n_kv;
-  if (B != 1 || T > 61 || G * T > 128) return no("more than one observation");   // RoPE rows fit a P buffer
+  if (B != 1 || T > 61 || G * T > 112) return no("more than one observation");   // RoPE rows fit a P buffer
+  if (T % 2) return no("odd token count");   // bulk copies of T (max, sum) pairs need 16-byte sizes
   if (g.hidden_a % 128 || qkv_rows(g) % 128 || g.inter_a % 64) return no("shapes do not tile by 128");
   const int nsm = c->num_sms;
   const int nblk = (P + 63) / 64 + 1;
@@ -600,7 +621,7 @@ bool persist_plan(dm0_ctx* c, int steps, float* vel, dm0::PdArgs* a, std::string
   const int bps = (nblk + splits - 1) / splits;
   splits = (nblk + bps - 1) / bps;   // every split owns at least one block
   // per GEMM phase (QKV, O, gate/up, down): tiles, k-blocks, landing bytes per staged pair
-  const long land_per[4] = {256L * T, 136L * splits * T, 256L * T, 512L * T};
+  const long land_per[4] = {256L * T, 140L * splits * T, 256L * T, 512L * T};
   const int geo[4][2] = {{qkv_rows(g) / 128, g.hidden_a / 64},
                          {g.hidden_a / 128, g.n_q * 2},
                          {g.inter_a / 64, g.hidden_a / 64},
@@ -611,6 +632,7 @@ bool persist_plan(dm0_ctx* c, int steps, float* vel, dm0::PdArgs* a, std::string
     if (per * land_per[ph] > static_cast<long>(dm0::PdSmem::kLandG)) return no("operand copies exceed the landing area");
   }
   if (g.n_kv * splits > kPartSlots) return no("partial-state slots");
+  if (g.n_kv * (splits + 1) > nsm) return no("too few SMs for the attention items and their helpers");
   *a = dm0::PdArgs{};
   a->L = g.layers;
   a->T = T;
@@ -634,6 +656,7 @@ bool persist_plan(dm0_ctx* c, int steps, float* vel, dm0::PdArgs* a, std::string
   a->part_o = reinterpret_cast<bf16*>(c->part_o);   // bf16 partials in the fp32 slot area
   a->part_ml = c->part_ml;
   a->sync = c->psync;
+  a->kv_sfx = c->pkv_sfx;
   a->err = c->d_err;
   a->trace = steps <= c->ptrace_steps ? c->ptrace : nullptr;
   StepArgs& st = a->step;
@@ -668,7 +691,17 @@ dm0_status enqueue_denoise_persistent(dm0_ctx* c, cudaStream_t s, const dm0::PdA
   const uint64_t kv_rows = L * g.n_kv * static_cast<uint64_t>(a.P);
   TRY(get_tmap(c, &tk, c->kplane, kv_rows, 128, 64));
   TRY(get_tmap(c, &tv, c->vplane, kv_rows, 128, 64));
-  CK(cudaMemsetAsync(c->psync, 0, 4 * sizeof(unsigned), s));
+  const uint64_t T = a.T, QR = qkv_rows(g), GU = 2 * static_cast<uint64_t>(g.inter_a);
+  CUtensorMap tacc_qkv, th, tacc_gu;   // split-K reduce-add destinations, [T][features] fp32
+  TRY(get_tmap_plain(c, &tacc_qkv, c->pacc_qkv, 4, T, QR, 128, 64));
+  TRY(get_tmap_plain(c, &th, c->h_a, 4, T, g.hidden_a, 128, 64));
+  TRY(get_tmap_plain(c, &tacc_gu, c->pacc_gu, 4, T, GU, 128, 64));
+  CUtensorMap th_ld, tgu_ld, tqkv_ld, tpo;   // operand copies: [T] rows of one 64- or 128-column block
+  TRY(get_tmap_plain(c, &th_ld, c->h_a, 4, T, g.hidden_a, 64, a.T));
+  TRY(get_tmap_plain(c, &tgu_ld, c->pacc_gu, 4, T, GU, 128, a.T));
+  TRY(get_tmap_plain(c, &tqkv_ld, c->pacc_qkv, 4, T, QR, 128, a.T));
+  TRY(get_tmap_plain(c, &tpo, c->part_o, 2, static_cast<uint64_t>(g.n_kv) * a.splits * 128, 128, 64, a.T));
+  CK(cudaMemsetAsync(c->psync, 0, (2 + g.n_kv) * sizeof(unsigned), s));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(c->num_sms);
   cfg.blockDim = dim3(dm0::kPdThreads);
@@ -680,7 +713,8 @@ dm0_status enqueue_denoise_persistent(dm0_ctx* c, cudaStream_t s, const dm0::PdA
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const int e0 = probe_begin(c, s, DM0_SITE_LOOP);
-  CK(cudaLaunchKernelEx(&cfg, dm0::denoise_persistent_kernel, tq, to, tgu, td, tk, tv, a));
+  CK(cudaLaunchKernelEx(&cfg, dm0::denoise_persistent_kernel, tq, to, tgu, td, tk, tv, tacc_qkv, th, tacc_gu, th_ld,
+                        tgu_ld, tqkv_ld, tpo, a));
   probe_end(c, s, DM0_SITE_LOOP, e0);
   c->launches += 1;
   c->pdl_ok = false;
@@ -917,7 +951,8 @@ dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
   A(dalloc(c, &c->pacc_qkv, static_cast<size_t>(64) * qkv_rows(g)));
   A(dalloc(c, &c->pacc_gu, static_cast<size_t>(64) * 2 * g.inter_a));
   A(dalloc(c, &c->pssq, 128));
-  A(dalloc(c, &c->psync, 4));
+  A(dalloc(c, &c->psync, 2 + g.n_kv));
+  A(dalloc(c, &c->pkv_sfx, static_cast<size_t>(g.n_kv) * 2 * 64 * 128));
   A(dalloc(c, &c->players, g.layers));
   if (const char* e = std::getenv("DM0_PERSIST_TRACE")) {
     if (e[0] == '1') {

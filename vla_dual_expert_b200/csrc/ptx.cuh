@@ -184,7 +184,7 @@ __device__ __forceinline__ float warp_sum(float v) {
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
-__device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
+__device__ __forceinline__ float silu_f(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 // 2^x by the special-function unit's ex2.approx (flush-to-zero; 2^-inf = 0), for softmax weights
 // that are rounded to bf16 right after
 __device__ __forceinline__ float ex2_fast(float x) {
