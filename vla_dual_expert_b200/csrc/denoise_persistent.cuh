@@ -171,6 +171,14 @@ __device__ __forceinline__ void tma_load_2d_plain(void* dst, const CUtensorMap* 
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
 }
+__device__ __forceinline__ void tma_load_3d_plain(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
+                                                 int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
 // contiguous copy; both addresses 16-byte aligned, bytes a multiple of 16
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -236,30 +244,30 @@ __device__ __noinline__ uint32_t pd_stage_norm(const PdArgs& a, uint8_t* smem, i
 
 // (C) attention output o = sum_j w_j o_j, w_j = l_j 2^(m_j - max m) / sum_j l_j 2^(m_j - max m), over
 // the key splits j
+// map_po: partial O as [slot][128 rows][128 dims] bf16, box {64 dims, T rows, S slots}; map_ml: (max, sum)
+// as [slot][128 rows] 8-byte elements, box {T rows, S slots}: one copy each per staged pair
 template <int kT>
 __device__ __noinline__ uint32_t pd_stage_attn_out(const PdArgs& a, uint8_t* smem, int ct, int p0, int np, int nkb,
                                                    unsigned long long* mk, uint64_t* btf, uint64_t* sbar,
-                                                   uint32_t par, const CUtensorMap* map_po, volatile int* abort_flag) {
+                                                   uint32_t par, const CUtensorMap* map_po, const CUtensorMap* map_ml,
+                                                   volatile int* abort_flag) {
   using SM = PdSmem;
   const int T = kT > 0 ? kT : a.T;   // tokens; a compile-time constant for the common shape
   const int c8 = ct & 7;
   const int G = a.n_q / a.n_kv, S = a.splits;
   const int nrows = np * S * T;
+  const int mls = (S * T + 15) & ~15;   // (max, sum) entries per pair, padded to 128 bytes
   __nv_bfloat16* lo = reinterpret_cast<__nv_bfloat16*>(smem + SM::kOffLandG);   // [np][S][T][64]
-  float2* lml = reinterpret_cast<float2*>(lo + static_cast<size_t>(nrows) * 64);   // [np][S][T]
-  float* wts = reinterpret_cast<float*>(lml + nrows);                             // [np][S][T]
+  float2* lml = reinterpret_cast<float2*>(lo + static_cast<size_t>(nrows) * 64);   // [np][mls]: [S][T] used
+  float* wts = reinterpret_cast<float*>(lml + np * mls);                          // [np][S][T]
   if (ct == 0) {
     fence_proxy_async_global();
     mbar_arrive_expect_tx(sbar, nrows * (128 + 8));
     int kb = p0 % nkb;
     for (int i = 0; i < np; ++i) {
-      const int hq = kb >> 1, g2 = hq / G, hh = hq - g2 * G;
-      for (int sp = 0; sp < S; ++sp) {
-        const int src = (g2 * S + sp) * 128 + hh * T;   // partial-state row of token 0
-        const int dst = (i * S + sp) * T;
-        tma_load_2d_plain(lo + static_cast<size_t>(dst) * 64, map_po, sbar, (kb & 1) * 64, src);
-        bulk_load(lml + dst, a.part_ml + src, T * 8, sbar);
-      }
+      const int hq = kb >> 1, g2 = hq / G, hh = hq - g2 * G;   // slots g2 S .. g2 S + S - 1, rows hh T ..
+      tma_load_3d_plain(lo + static_cast<size_t>(i) * S * T * 64, map_po, sbar, (kb & 1) * 64, hh * T, g2 * S);
+      tma_load_2d_plain(lml + i * mls, map_ml, sbar, hh * T, g2 * S);
       if (++kb == nkb) kb = 0;
     }
     if (mk) mk[8] = globaltimer();
@@ -269,10 +277,10 @@ __device__ __noinline__ uint32_t pd_stage_attn_out(const PdArgs& a, uint8_t* sme
   for (int q = ct; q < np * T; q += kPdCompute) {   // normalised split weights of each (pair, token)
     const int i = q / T, t = q - i * T;
     float mx = -__int_as_float(0x7f800000);
-    for (int sp = 0; sp < S; ++sp) mx = fmaxf(mx, lml[(i * S + sp) * T + t].x);
+    for (int sp = 0; sp < S; ++sp) mx = fmaxf(mx, lml[i * mls + sp * T + t].x);
     float den = 0.f;
     for (int sp = 0; sp < S; ++sp) {
-      const float2 ml = lml[(i * S + sp) * T + t];
+      const float2 ml = lml[i * mls + sp * T + t];
       const float w = ml.y * ex2_fast(ml.x - mx);
       wts[(i * S + sp) * T + t] = w;
       den += w;
@@ -459,7 +467,8 @@ __global__ void __launch_bounds__(kPdThreads, 1)
                               const __grid_constant__ CUtensorMap tmAccQKV, const __grid_constant__ CUtensorMap tmH,
                               const __grid_constant__ CUtensorMap tmAccGU, const __grid_constant__ CUtensorMap tmHLd,
                               const __grid_constant__ CUtensorMap tmGULd, const __grid_constant__ CUtensorMap tmQKVLd,
-                              const __grid_constant__ CUtensorMap tmPO, const __grid_constant__ PdArgs a) {
+                              const __grid_constant__ CUtensorMap tmPO, const __grid_constant__ CUtensorMap tmML,
+                              const __grid_constant__ PdArgs a) {
   using SM = PdSmem;
   constexpr int NST = kPdStages;
   extern __shared__ uint8_t pd_smem_raw[];
@@ -1027,7 +1036,7 @@ __global__ void __launch_bounds__(kPdThreads, 1)
           const int np = p1 - p0;
           if (np > 0) {
             if (ph == 0) stage_par = PD_STAGE(pd_stage_norm, a, smem, ct, p0, np, nkb, ly.attn_norm, ssq_attn, mk_row(), btile_full, stage_bar, stage_par, &tmHLd, abort_flag);
-            else if (ph == 2) stage_par = PD_STAGE(pd_stage_attn_out, a, smem, ct, p0, np, nkb, mk_row(), btile_full, stage_bar, stage_par, &tmPO, abort_flag);
+            else if (ph == 2) stage_par = PD_STAGE(pd_stage_attn_out, a, smem, ct, p0, np, nkb, mk_row(), btile_full, stage_bar, stage_par, &tmPO, &tmML, abort_flag);
             else if (ph == 3) stage_par = PD_STAGE(pd_stage_norm, a, smem, ct, p0, np, nkb, ly.mlp_norm, ssq_mlp, mk_row(), btile_full, stage_bar, stage_par, &tmHLd, abort_flag);
             else stage_par = PD_STAGE(pd_stage_swiglu, a, smem, ct, p0, np, nkb, mk_row(), btile_full, stage_bar, stage_par, &tmGULd, abort_flag);
             mark(1);

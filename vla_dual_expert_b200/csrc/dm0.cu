@@ -621,7 +621,7 @@ bool persist_plan(dm0_ctx* c, int steps, float* vel, dm0::PdArgs* a, std::string
   const int bps = (nblk + splits - 1) / splits;
   splits = (nblk + bps - 1) / bps;   // every split owns at least one block
   // per GEMM phase (QKV, O, gate/up, down): tiles, k-blocks, landing bytes per staged pair
-  const long land_per[4] = {256L * T, 140L * splits * T, 256L * T, 512L * T};
+  const long land_per[4] = {256L * T, 140L * splits * T + 128, 256L * T, 512L * T};
   const int geo[4][2] = {{qkv_rows(g) / 128, g.hidden_a / 64},
                          {g.hidden_a / 128, g.n_q * 2},
                          {g.inter_a / 64, g.hidden_a / 64},
@@ -700,7 +700,26 @@ dm0_status enqueue_denoise_persistent(dm0_ctx* c, cudaStream_t s, const dm0::PdA
   TRY(get_tmap_plain(c, &th_ld, c->h_a, 4, T, g.hidden_a, 64, a.T));
   TRY(get_tmap_plain(c, &tgu_ld, c->pacc_gu, 4, T, GU, 128, a.T));
   TRY(get_tmap_plain(c, &tqkv_ld, c->pacc_qkv, 4, T, QR, 128, a.T));
-  TRY(get_tmap_plain(c, &tpo, c->part_o, 2, static_cast<uint64_t>(g.n_kv) * a.splits * 128, 128, 64, a.T));
+  CUtensorMap tml;
+  {   // split-attention partials: O as [slot][128 rows][128 dims] bf16, (max, sum) as [slot][128 rows] 8-byte
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return fail(c, DM0_ECUDA, "cuTensorMapEncodeTiled is unavailable");
+    const cuuint64_t nslot = static_cast<cuuint64_t>(g.n_kv) * a.splits;
+    cuuint64_t d3[3] = {128, 128, nslot};
+    cuuint64_t s3[2] = {128 * 2, 128 * 128 * 2};
+    cuuint32_t b3[3] = {64, static_cast<cuuint32_t>(a.T), static_cast<cuuint32_t>(a.splits)};
+    cuuint32_t e3[3] = {1, 1, 1};
+    CUresult r = enc(&tpo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, c->part_o, d3, s3, b3, e3, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(c, DM0_ECUDA, "cuTensorMapEncodeTiled (partial O) failed (" + std::to_string(r) + ")");
+    cuuint64_t d2[2] = {128, nslot};
+    cuuint64_t s2[1] = {128 * 8};
+    cuuint32_t b2[2] = {static_cast<cuuint32_t>(a.T), static_cast<cuuint32_t>(a.splits)};
+    cuuint32_t e2[2] = {1, 1};
+    r = enc(&tml, CU_TENSOR_MAP_DATA_TYPE_INT64, 2, c->part_ml, d2, s2, b2, e2, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(c, DM0_ECUDA, "cuTensorMapEncodeTiled (partial max/sum) failed (" + std::to_string(r) + ")");
+  }
   CK(cudaMemsetAsync(c->psync, 0, (2 + g.n_kv) * sizeof(unsigned), s));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(c->num_sms);
@@ -714,7 +733,7 @@ dm0_status enqueue_denoise_persistent(dm0_ctx* c, cudaStream_t s, const dm0::PdA
   cfg.numAttrs = 1;
   const int e0 = probe_begin(c, s, DM0_SITE_LOOP);
   CK(cudaLaunchKernelEx(&cfg, dm0::denoise_persistent_kernel, tq, to, tgu, td, tk, tv, tacc_qkv, th, tacc_gu, th_ld,
-                        tgu_ld, tqkv_ld, tpo, a));
+                        tgu_ld, tqkv_ld, tpo, tml, a));
   probe_end(c, s, DM0_SITE_LOOP, e0);
   c->launches += 1;
   c->pdl_ok = false;
