@@ -33,9 +33,13 @@ sys.path.insert(0, ROOT)
 METRIC = "action chunks/sec (prefill+10-step denoise) at batch 1 and 16; HBM GB/s, TC util"
 EULER_STEPS = 10
 # DRAM bytes (read + write) of one prefix-pass gate/up GEMM launch at B=16, P=2048 (M=32768,
-# N=12288, K=2048), from the ncu capture of the same kernel and launch shape summarised in
-# profiles/gemm_tc_persistent_gateup_M32768.md (3.167 GB read + 0.352 GB written)
+# N=12288, K=2048), from an ncu capture of the same kernel and launch shape in `bench.py --one-layer`
+# (3.167 GB read + 0.352 GB written)
 GATEUP_TRAFFIC_BYTES = 3.519e9
+# DRAM bytes (read + write) of the persistent Euler loop per step of 28 action layers at B=1, P=816:
+# the ncu capture of `bench.py --b1-loop` (3 layers, 1 step: 104.79 MB read + 4.15 MB written)
+# scaled by 28/3
+LOOP_TRAFFIC_BYTES_PER_STEP = 1.0168e9
 
 
 def _peaks():
@@ -300,9 +304,13 @@ def run_native(args, rank, world, local_rank):
             "unit": "chunks/s", "ms_per_step": round(b1["ms"], 3), "prefill_ms_p50": round(b1["prefill_ms_p50"], 3),
             "denoise_ms_p50": round(b1["denoise_ms_p50"], 3), "denoise_ms_p90": round(b1["denoise_ms_p90"], 3),
             "gpu_launches": b1["launches"],
-            "denoise_roofline": {"bound": "hbm", "achieved": round(den_gbs, 1), "peak": peaks["hbm_gbs"],
+            "denoise_roofline": {"bound": "hbm",
+                                 "kernel": "denoise_persistent_kernel (the 10-step Euler loop, one launch)",
+                                 "achieved": round(den_gbs, 1), "peak": peaks["hbm_gbs"],
                                  "unit": "GB/s", "frac": round(den_gbs / peaks["hbm_gbs"], 4),
-                                 "algorithmic_bytes_per_euler_step": denoise_bytes_per_step(d, 1, wl1.prefix)},
+                                 "algorithmic_bytes_per_euler_step": denoise_bytes_per_step(d, 1, wl1.prefix),
+                                 "traffic_per_euler_step": LOOP_TRAFFIC_BYTES_PER_STEP,
+                                 "peak_src": f"{peaks['src']} hbm_gbs"},
         }
     if not args.skip_breakdown:
         result["breakdown_ms_per_step"] = breakdown(eng, wl_main)
@@ -414,6 +422,36 @@ def run_one_layer(args):
     eng.close()
 
 
+def run_b1_loop(args):
+    """Profiling workload for the single-launch Euler loop of one observation: DM0-base widths with
+    3 action layers (the kernel walks every layer the same way), B=1, a random 816-token prefix cache,
+    three 1-step dm0_denoise calls.  Holds about 0.5 GB on the device, small enough for full ncu
+    captures of the persistent kernel."""
+    import torch
+
+    from synth import inputs as I
+    from vla_dual_expert_b200 import Engine
+    d = I.DM0_BASE.replace(layers=3)
+    P = 816
+    eng = Engine(d, 1, P)
+    eng.load_from(I.Weights(d, seed=0))
+    n = d.layers * d.n_kv * P * d.head_dim
+    g = torch.Generator(device="cuda").manual_seed(3000)
+    for ptr in eng.kv_view():   # the context-owned cache planes, filled in place with N(0, 1)
+        view = type("Plane", (), {"__cuda_array_interface__": {"shape": (n,), "typestr": "<u2",
+                                                                "data": (ptr, False), "version": 3}})()
+        torch.as_tensor(view, device="cuda").view(torch.bfloat16).normal_(generator=g)
+    eng.kv_commit(1, P)
+    noise = torch.from_numpy(I.noise(d, 1)).cuda()
+    n0 = eng.launch_count()
+    for _ in range(3):
+        out = eng.denoise(noise, 1)
+    eng.sync()
+    print(json.dumps({"b1_loop": "ok", "launches": eng.launch_count() - n0,
+                      "mean_abs_action": float(out.abs().mean())}))
+    eng.close()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -426,6 +464,7 @@ def main():
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-breakdown", action="store_true")
     ap.add_argument("--one-layer", action="store_true", help="profiling workload: one layer, B=16, P=2048")
+    ap.add_argument("--b1-loop", action="store_true", help="profiling workload: persistent Euler loop, 3 layers, B=1")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "native":
@@ -438,6 +477,9 @@ def main():
         return
     if args.one_layer:
         run_one_layer(args)
+        return
+    if args.b1_loop:
+        run_b1_loop(args)
         return
     run_native(args, rank, world, local_rank)
 

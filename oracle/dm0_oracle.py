@@ -20,7 +20,7 @@ Sources (page title and section):
               u_t = eps - a, Euler integration from x_1 with diffusion_steps=10),
               6.2 (the suffix reads the prefix cache while processing the chunk).
 
-Readings of points the pages leave open (each also listed in the design doc):
+Readings of points the pages leave open:
   R1 RMSNorm: x / sqrt(mean(x^2) + eps) * g, eps 1e-6 (Qwen3 default).
   R2 RoPE: rotate-half pairing (i, i + D/2), inv_freq_i = theta^(-2i/D),
      theta 1e6; prefix positions 0..P-1, suffix positions P..P+S-1.
