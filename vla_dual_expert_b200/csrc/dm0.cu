@@ -320,9 +320,13 @@ dm0_status run_gemm(dm0_ctx* c, cudaStream_t s, const bf16* act, int tokens, int
   }
   const int mt = (tokens + 127) / 128;
   int BN = (wrows % 256 == 0) ? 256 : 128;
-  // narrower tiles when the grid would leave SMs idle; a 64-wide tile only for column-independent epilogues
+  // narrower tiles when the grid would leave SMs idle, but only while the narrower tiling still fits
+  // in one wave: a tile's k-loop is a chain of dependent MMAs whose time hardly depends on the tile
+  // width, so a second, partial wave of narrow tiles costs more than idle SMs (M = 816: the O and
+  // down projections take 128-wide tiles, 112 CTAs, instead of 224 64-wide ones); a 64-wide tile
+  // only for column-independent epilogues
   const int min_bn = (g.mode == dm0::kModeResid || g.mode == dm0::kModeStoreF32) ? 64 : 128;
-  while (BN > min_bn && mt * (wrows / BN) < c->num_sms) BN /= 2;
+  while (BN > min_bn && mt * (wrows / BN) < c->num_sms && mt * (wrows / (BN / 2)) <= c->num_sms) BN /= 2;
   g.M = tokens;
   g.N = wrows;
   g.swap = 0;
