@@ -10,20 +10,21 @@
 // a weight stream.  Here weights do not depend on activations, so the TMA
 // producer warp of every CTA runs ahead across phase and layer boundaries,
 // limited only by its shared-memory ring; the dependent chain per phase is one
-// grid barrier, one L2 round trip to stage the activation operand, the MMAs
-// and the fp32 reductions.
+// grid barrier, one TMA copy of the L2-resident sums, the operand build, the
+// MMAs and one TMA bulk reduce-add of the split-K partial tile.
 //
-// Per layer l, five phases (T = tokens <= 64, the padded MMA N is 64):
+// Per layer l, five phases (T = tokens <= 61, the padded MMA N is 64):
 //   A  qkv_acc[t][f]  += sum_k Wqkv[f][k] * bf16(g_attn[k] h[t][k])   split-K over all CTAs
 //                       (tile-0 CTAs also add sum_k h[t][k]^2 for the pending RMSNorm)
 //   B  attention: one CTA per (KV head, key split).  The CTA finishes q of
-//      its G query heads (1/rms, QK-RMSNorm, RoPE at position P + t) and, if it
-//      owns the suffix block, the suffix K/V, then runs 64-key blocks of the
-//      prefix cache (TMA) and the suffix (shared memory) through tcgen05:
-//      S = Q K^T and O += P V in TMEM; it stores its partial O / l in bf16
-//      with its (max, sum).
+//      its G query heads (1/rms, QK-RMSNorm, RoPE at position P + t), then
+//      runs 64-key blocks of the prefix cache (TMA) and, for the last split,
+//      the suffix block through tcgen05: S = Q K^T and O += P V in TMEM; it
+//      stores its partial O / l in bf16 with its (max, sum).  One helper CTA
+//      per KV head builds that head's suffix K and V (K-RMSNorm, RoPE, 1/rms)
+//      and publishes them with a flag; the suffix owner's producer copies them in.
 //   C  h[t][f] += sum_k Wo[f][k] * o[t][k], the B operand o combined from the
-//      key splits while it is staged (residual add by fp32 reduction into h)
+//      key splits while it is staged (residual add by the reduce-add into h)
 //   D  gu_acc[t][f] += sum_k Wgu[f][k] * bf16(g_mlp[k] h[t][k])  (+ MLP sum of squares)
 //   E  h[t][f] += sum_k Wd[f][k] * bf16(silu(gate / rms) * (up / rms))
 // and after layer L-1 the step boundary (velocity, Euler update, next input;
@@ -32,14 +33,14 @@
 // per CTA; a range covers at most two tiles, each accumulated in its own
 // 64-column TMEM segment.
 //
-// Warp roles (320 threads): warp 0 TMA producer (weights, prefix K/V), warp 1
-// TMEM owner and tcgen05.mma issuer, warps 2-9 everything else: operand
-// staging (every thread issues all of its L2 loads before using any, so a
-// stage costs one round trip), reductions (two warps per TMEM lane quarter,
-// one per 32-column half), grid barriers; warps 2-5 also run the softmax.
-// Every wait is bounded; a CTA that gives up raises the device error word and
-// a global abort word that every other CTA's barrier polls, so the whole grid
-// unwinds.
+// Warp roles (320 threads): warp 0 TMA producer (weights, prefix K/V, the
+// suffix K/V from the helper), warp 1 TMEM owner and tcgen05.mma issuer (it
+// starts on each staged pair as soon as its operand is ready), warps 2-9
+// everything else: operand staging, the split-K epilogue (two warps per TMEM
+// lane quarter, one per 32-column half), the softmax (two threads per query
+// row, one per 32 keys of a block) and the grid barriers.  Every wait is
+// bounded; a CTA that gives up raises the device error word and a global abort
+// word that every other CTA's barrier polls, so the whole grid unwinds.
 #pragma once
 #include "attention_tc.cuh"
 #include "elementwise.cuh"
