@@ -88,6 +88,7 @@ struct dm0_ctx {
   // per-layer kernels instead); DM0_PERSIST_SPLITS overrides its attention key splits per KV head
   bool use_persist = true;
   int persist_splits = 7;
+  int persist_resident = -1;   // -1: not checked yet
   // true when the previous operation this context queued on the stream was one of its own
   // kernels: only then may the next kernel overlap it (programmatic dependent launch).  The first
   // kernel of every API call follows foreign work (caller kernels, copies) and waits for it in
@@ -613,6 +614,16 @@ bool persist_plan(dm0_ctx* c, int steps, float* vel, dm0::PdArgs* a, std::string
     return false;
   };
   if (!c->use_persist) return no("disabled");
+  if (c->persist_resident < 0) {   // once per context: can one CTA of the kernel live on every SM?
+    int per_sm = 0, coop = 0;
+    cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, c->device);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dm0::denoise_persistent_kernel, dm0::kPdThreads,
+                                                      dm0::PdSmem::kBytes) != cudaSuccess)
+      per_sm = 0;
+    cudaGetLastError();
+    c->persist_resident = (coop && per_sm >= 1) ? 1 : 0;
+  }
+  if (!c->persist_resident) return no("the persistent kernel cannot be resident on every SM");
   if (g.head_dim != 128) return no("head_dim != 128");
   const int B = c->kv_B, P = c->kv_P, T = B * g.chunk, G = g.n_q / g.n_kv;
   if (B != 1 || T > 61 || G * T > 112) return no("more than one observation");   // RoPE rows fit a P buffer
@@ -736,8 +747,14 @@ dm0_status enqueue_denoise_persistent(dm0_ctx* c, cudaStream_t s, const dm0::PdA
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const int e0 = probe_begin(c, s, DM0_SITE_LOOP);
-  CK(cudaLaunchKernelEx(&cfg, dm0::denoise_persistent_kernel, tq, to, tgu, td, tk, tv, tacc_qkv, th, tacc_gu, th_ld,
-                        tgu_ld, tqkv_ld, tpo, tml, a));
+  const cudaError_t le = cudaLaunchKernelEx(&cfg, dm0::denoise_persistent_kernel, tq, to, tgu, td, tk, tv, tacc_qkv, th,
+                                            tacc_gu, th_ld, tgu_ld, tqkv_ld, tpo, tml, a);
+  if (le == cudaErrorCooperativeLaunchTooLarge) {   // fewer SMs available than the device has: use the
+    cudaGetLastError();                             // per-layer kernels from now on
+    c->persist_resident = 0;
+    return DM0_ESTATE;
+  }
+  CK(le);
   probe_end(c, s, DM0_SITE_LOOP, e0);
   c->launches += 1;
   c->pdl_ok = false;
@@ -748,7 +765,10 @@ dm0_status denoise_from_x(dm0_ctx* c, cudaStream_t s, int steps, float* vel) {
   {
     dm0::PdArgs pa;
     std::string why;
-    if (persist_plan(c, steps, vel, &pa, &why)) return enqueue_denoise_persistent(c, s, pa);
+    if (persist_plan(c, steps, vel, &pa, &why)) {
+      const dm0_status st = enqueue_denoise_persistent(c, s, pa);
+      if (!(st == DM0_ESTATE && c->persist_resident == 0)) return st;   // else fall through
+    }
   }
   if (vel || !c->use_graph || c->probe_mask) return enqueue_denoise(c, s, steps, vel);
   const auto key = std::make_tuple(c->kv_B, c->kv_P, steps);
