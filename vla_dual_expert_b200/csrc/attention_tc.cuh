@@ -28,6 +28,13 @@
 namespace dm0 {
 
 constexpr int kFaThreads = 192;
+// softmax warps: 4 (one thread per query row) in the two-CTAs-per-SM variant; 8 (two threads per
+// row, 32 keys each) in the one-CTA-per-SM suffix variant, whose softmax is its critical path
+template <int NP>
+struct FaWarps {
+  static constexpr int kSoftmax = NP == 2 ? 8 : 4;
+  static constexpr int kThreads = 64 + 32 * kSoftmax;
+};
 
 template <int ST, int NP>
 struct FaSmemT {
@@ -42,7 +49,9 @@ struct FaSmemT {
   static constexpr uint32_t kOffK = kOffQ + kQ;
   static constexpr uint32_t kOffV = kOffK + kStages * kKV;
   static constexpr uint32_t kOffP = kOffV + kStages * kKV;
-  static constexpr uint32_t kOffBar = kOffP + NP * kP;
+  static constexpr uint32_t kOffX = kOffP + NP * kP;       // two-thread rows: [2][2][128] row maxima, [2][128] sums
+  static constexpr uint32_t kX = NP == 2 ? 3072 : 0;
+  static constexpr uint32_t kOffBar = kOffX + kX;
   static constexpr uint32_t kSlack = 256;                   // the dynamic base is 1024-aligned (no static smem)
   static constexpr uint32_t kBytes = kOffBar + 256 + kSlack;
 };
@@ -92,7 +101,7 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int col) {
 }
 
 template <int ST, int NP>
-__global__ void __launch_bounds__(kFaThreads, NP == 1 ? 2 : 1)
+__global__ void __launch_bounds__(FaWarps<NP>::kThreads, NP == 1 ? 2 : 1)
     fa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const __grid_constant__ CUtensorMap tmKb, const __grid_constant__ CUtensorMap tmVb, const AttnArgs a) {
   constexpr int D = 128;
@@ -134,10 +143,10 @@ __global__ void __launch_bounds__(kFaThreads, NP == 1 ? 2 : 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);
+      mbar_init(&s_free[i], FaWarps<NP>::kSoftmax);
     }
     for (int i = 0; i < NP; ++i) {
-      mbar_init(&p_full[i], 4);
+      mbar_init(&p_full[i], FaWarps<NP>::kSoftmax);
       mbar_init(&pv_done[i], 1);
     }
     mbar_init(q_ready, 4);
@@ -252,6 +261,154 @@ __global__ void __launch_bounds__(kFaThreads, NP == 1 ? 2 : 1)
       // every issued MMA completes before TMEM is released
       umma_commit(drain);
       if (!mbar_wait(drain, 0, nullptr, kWaitTimeoutNs + kDrainTimeoutNs)) raise_error(a.err, kErrDrain);
+    }
+  } else if constexpr (FaWarps<NP>::kSoftmax == 8) {
+    // ------------------------------------------------ softmax / correction / output: two threads per row
+    constexpr int kSM = 256;                        // softmax threads (named barrier 1)
+    const int half = (warp - 2) >> 2;               // keys [32 half, 32 half + 32) of each block
+    const int lane_base = (warp & 3) * 32;
+    const int r = lane_base + lane;                 // TMEM lane = query row of this tile
+    const uint32_t tl = tmem + (static_cast<uint32_t>(lane_base) << 16);
+    const int pr = tile * 128 + r;
+    const bool valid = pr < rows_total;
+    const int head = valid ? kvh * G + pr / a.seq_q : 0;
+    const int pos = valid ? pr % a.seq_q : 0;
+    float* xm = reinterpret_cast<float*>(smem + FS::kOffX);   // [2 blocks][2 halves][128 rows]
+    float* xl = xm + 512;                                     // [2 halves][128 rows]
+    // one lane waits, the warp shares the answer (the TMEM loads after it are warp-collective)
+    auto warp_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      int good = 1;
+      if (lane == 0) good = mbar_wait(bar, parity, abort_flag) ? 1 : 0;
+      good = __shfl_sync(0xffffffffu, good, 0);
+      if (!good) *abort_flag = 1;
+      return good != 0;
+    };
+    pdl_wait();
+    if (half == 0) {   // Q row -> shared memory in the SW128 K-major layout
+      const uint4* src = reinterpret_cast<const uint4*>(a.q + ((static_cast<size_t>(b) * a.seq_q + pos) * a.n_q + head) * D);
+      uint8_t* qs = smem + FS::kOffQ;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const uint4 v = valid ? src[c] : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(qs + sw128_off(r, c * 8)) = v;
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_ready);
+    }
+    float m_ref = -__int_as_float(0x7f800000), l_run = 0.f;   // l_run: this half's share of the row sum
+    for (int j = 0; j < nblk; ++j) {
+      const int s = j & 1;
+      bool good = *abort_flag == 0 && warp_wait(&s_full[s], (j >> 1) & 1);
+      tc_fence_after();
+      const int jj = jb0 + j;
+      const int nvalid = jj < nA ? min(64, a.len_a - jj * 64) : min(64, a.len_b - (jj - nA) * 64);
+      float sv[32];
+      float mx = -__int_as_float(0x7f800000);
+      if (good) {
+        tmem_ld32(tl + s * 64 + half * 32, sv);
+#pragma unroll
+        for (int q = 0; q < 32; ++q)
+          if (half * 32 + q < nvalid) mx = fmaxf(mx, sv[q]);
+      }
+      xm[((j & 1) * 2 + half) * 128 + r] = mx;
+      named_bar_sync(1, kSM);
+      mx = fmaxf(mx, xm[((j & 1) * 2 + (half ^ 1)) * 128 + r]);
+      const float m_blk = mx * a.scale_log2;
+      const bool move = m_blk > m_ref + 8.f;        // also true on the first block
+      const float m_new = move ? m_blk : m_ref;
+      const float alpha = move ? exp2f(m_ref - m_new) : 1.f;   // 0 on the first block
+      const bool any_move = __any_sync(0xffffffffu, move);
+      // P buffer j % NP is free once PV_{j-NP} completed
+      if (good && j >= NP) good = warp_wait(&pv_done[j % NP], ((j / NP) - 1) & 1);
+      float sum = 0.f;
+      if (good) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int q = 0; q < 32; q += 2) {
+          const int kq = half * 32 + q;
+          const float p0 = kq < nvalid ? ex2_fast(fmaf(sv[q], a.scale_log2, -m_new)) : 0.f;
+          const float p1 = kq + 1 < nvalid ? ex2_fast(fmaf(sv[q + 1], a.scale_log2, -m_new)) : 0.f;
+          sum += p0 + p1;
+          pk[q >> 1] = pack_bf16(p0, p1);
+        }
+        uint8_t* ps = smem + FS::kOffP + (j % NP) * FS::kP;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(ps + sw128_off(r, (half * 4 + c) * 8)) =
+              make_uint4(pk[c * 4], pk[c * 4 + 1], pk[c * 4 + 2], pk[c * 4 + 3]);
+      }
+      // S buffer consumed: the MMA warp may overwrite it with S_{j+2}
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[s]);
+      l_run = l_run * alpha + sum;
+      m_ref = m_new;
+      // O (this half's 64 columns) may only be rescaled after PV_{j-1}
+      if (good && j >= 1 && any_move) {
+        const int i = j - 1;
+        good = warp_wait(&pv_done[i % NP], (i / NP) & 1);
+        if (good) {
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < 2; ++c) {
+            float o[32];
+            tmem_ld32(tl + 128 + half * 64 + c * 32, o);
+#pragma unroll
+            for (int q = 0; q < 32; ++q) o[q] *= alpha;
+            tmem_st32(tl + 128 + half * 64 + c * 32, o);
+          }
+          tmem_wait_st();
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[j % NP]);
+    }
+    if (nblk > 0) {
+      xl[half * 128 + r] = l_run;
+      named_bar_sync(1, kSM);
+      const float l_tot = xl[r] + xl[128 + r];
+      const bool good = *abort_flag == 0 && warp_wait(&pv_done[(nblk - 1) % NP], ((nblk - 1) / NP) & 1);
+      if (good) {
+        tc_fence_after();
+        if (gridDim.z == 1) {
+          const float inv = 1.f / l_tot;
+          __nv_bfloat16* dst = a.o + ((static_cast<size_t>(b) * a.seq_q + pos) * a.n_q + head) * D;
+#pragma unroll 1
+          for (int c = half * 2; c < half * 2 + 2; ++c) {
+            float o[32];
+            tmem_ld32(tl + 128 + c * 32, o);
+            if (valid) {
+              uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                d4[i] = make_uint4(pack_bf16(o[8 * i] * inv, o[8 * i + 1] * inv),
+                                   pack_bf16(o[8 * i + 2] * inv, o[8 * i + 3] * inv),
+                                   pack_bf16(o[8 * i + 4] * inv, o[8 * i + 5] * inv),
+                                   pack_bf16(o[8 * i + 6] * inv, o[8 * i + 7] * inv));
+            }
+          }
+        } else {
+          // split keys: this split's unnormalised O and (m, l) against its reference max
+          const size_t mine = ((static_cast<size_t>(grp) * gridDim.x + tile) * gridDim.z + blockIdx.z) * 128 + r;
+          float* po = a.part_o + mine * D;
+#pragma unroll 1
+          for (int c = half * 2; c < half * 2 + 2; ++c) {
+            float o[32];
+            tmem_ld32(tl + 128 + c * 32, o);
+            float4* p4 = reinterpret_cast<float4*>(po + c * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) p4[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+          }
+          if (half == 0) a.part_ml[mine] = make_float2(m_ref, l_tot);
+          __threadfence();
+        }
+      } else {
+        *abort_flag = 1;
+        raise_error(a.err, kErrTimeoutEpilogue);
+      }
     }
   } else {
     // ------------------------------------------------ softmax / correction / output warps
@@ -442,7 +599,7 @@ __global__ void __launch_bounds__(kFaThreads, NP == 1 ? 2 : 1)
     if (*s_last && !*abort_flag) {
       __threadfence();
       const size_t slot0 = (static_cast<size_t>(grp) * gridDim.x + tile) * gridDim.z;
-      combine_splits<128>(a, slot0, tile, b, kvh, reinterpret_cast<float*>(smem), threadIdx.x, kFaThreads);
+      combine_splits<128>(a, slot0, tile, b, kvh, reinterpret_cast<float*>(smem), threadIdx.x, FaWarps<NP>::kThreads);
     }
   }
 }

@@ -426,7 +426,7 @@ dm0_status run_attn(dm0_ctx* c, cudaStream_t s, const bf16* q, int seq_q, const 
                     tkb, tvb, a);
     // merged suffix attention: the cached prefix is read from DRAM once; deeper K/V prefetch and
     // two P buffers so the softmax runs ahead of the PV MMAs
-    return launch(c, s, dm0::fa_tc_kernel<dm0::kFaDeepStages, 2>, grid, dim3(dm0::kFaThreads),
+    return launch(c, s, dm0::fa_tc_kernel<dm0::kFaDeepStages, 2>, grid, dim3(dm0::FaWarps<2>::kThreads),
                   dm0::FaSmemT<dm0::kFaDeepStages, 2>::kBytes, tk, tv, tkb, tvb, a);
   }
   const dim3 grid(tiles, groups, splits);
