@@ -34,8 +34,8 @@ METRIC = "action chunks/sec (prefill+10-step denoise) at batch 1 and 16; HBM GB/
 EULER_STEPS = 10
 # DRAM bytes (read + write) of one prefix-pass gate/up GEMM launch at B=16, P=2048 (M=32768,
 # N=12288, K=2048), from an ncu capture of the same kernel and launch shape in `bench.py --one-layer`
-# (3.167 GB read + 0.352 GB written)
-GATEUP_TRAFFIC_BYTES = 3.519e9
+# (3.079 GB read + 0.353 GB written)
+GATEUP_TRAFFIC_BYTES = 3.432e9
 # DRAM bytes (read + write) of the persistent Euler loop per step of 28 action layers at B=1, P=816:
 # the ncu capture of `bench.py --b1-loop` (3 layers, 1 step: 104.79 MB read + 4.15 MB written)
 # scaled by 28/3
