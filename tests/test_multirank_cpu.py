@@ -69,3 +69,22 @@ def test_single_rank_passthrough():
     import bench
     assert bench.max_over_ranks(12.5) == 12.5
     assert bench.job_chunks_per_s(1, 16, 200.0) == pytest.approx(80.0)
+
+
+def test_reference_arm_json_line_on_rank0():
+    """The reference arm (the fp64 oracle on the host cores, a bounded sample) prints one JSON line with
+    the native arm's metric and unit and its own cpu_baseline / e2e objects."""
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "0"], env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    sys.path.insert(0, ROOT)
+    import bench
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "chunks/s"
+    assert d["value"] > 0 and d["higher_is_better"] is True
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"] == {"value": d["value"], "unit": "chunks/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
