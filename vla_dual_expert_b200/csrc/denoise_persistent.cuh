@@ -849,6 +849,10 @@ __global__ void __launch_bounds__(kPdThreads, 1)
     auto reduce_out = [&](int p0, int p1, int nkb, const CUtensorMap* map) -> bool {
       const int tt0 = p0 / nkb, nseg = (p1 - 1) / nkb - tt0 + 1;
       bool good = true;
+      // the reduce tiles reuse the landing area of the operand copies: every warp must be done
+      // building its operands (pairs are handed to the MMA warp per warp, and the first segment
+      // can complete while another warp still converts a later pair)
+      csync();
       for (int seg = 0; seg < nseg && good; ++seg) {
         if (!warp_wait(&acc_full[seg], acc_use[seg] & 1)) {
           good = false;
