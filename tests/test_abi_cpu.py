@@ -83,3 +83,14 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(_abi, "_lib", None)
     with pytest.raises(ImportError):
         _abi.load_library()
+
+
+def test_probe_site_names_match_the_header():
+    """The binding's SITES tuple names dm0.h's DM0_SITE_* enum in order, one name per site."""
+    from vla_dual_expert_b200 import SITES
+    src = open(os.path.join(ROOT, "include", "dm0.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    sites = dict((m.group(1), int(m.group(2))) for m in re.finditer(r"DM0_SITE_([A-Z_]+)\s*=\s*(\d+)", src))
+    count = sites.pop("COUNT")
+    assert count == len(SITES) == len(sites)
+    assert [n.lower() for n, _ in sorted(sites.items(), key=lambda kv: kv[1])] == list(SITES)
