@@ -36,6 +36,11 @@ Readings of points the pages leave open:
   R8 Euler: t_k = 1 - k/K (k = 0..K-1), x <- x + dt * v(x, t_k), dt = -1/K;
      integration runs from noise (t=1) to data (t=0) because dx/dt = u = eps-a.
   R9 The KV cache holds K after QK-norm and RoPE, and V.
+  R11 (the FP8 prefix MLP, a next step; [DM05] 6.3 names FP8 E4M3 for the gate/up/down GEMMs
+     with scales but gives no scaling scheme): OCP E4M3 values (1-4-3, exponent bias 7, no
+     infinities, largest finite 448), round to nearest with ties to even, saturating at +-448;
+     per-token activation scales and per-output-channel weight scales, s = amax(|row|) / 448;
+     products accumulated wide (fp64 here).
 
 Precision: fp64 throughout.  Weights are the bf16-representable values from
 synth/inputs.py, upcast.  No blocking, fusion or reordering beyond the
@@ -237,3 +242,48 @@ def infer(weights, prefix_emb, noise, steps):
         caches.append((ks, vs))
         vels.append(v)
     return np.stack(chunks), caches, vels
+
+
+# ---------------------------------------------------------------- FP8 E4M3 prefix MLP (reading R11)
+
+E4M3_MAX = 448.0
+
+
+def e4m3(x):
+    """R11: x rounded to the nearest FP8 E4M3 value (ties to even), saturating at +-448.
+
+    Representable magnitudes are m 2^(e-3) for e in [-6, 8] and integer m in [8, 15] (normals), and
+    m 2^-9 for m in [0, 7] (subnormals): the spacing at |x| is 2^(floor(log2|x|) - 3), clamped below
+    to the subnormal spacing 2^-9 and above to that of the top binade, 2^5.
+    """
+    x = np.asarray(x, F)
+    a = np.abs(x)
+    e = np.clip(np.floor(np.log2(np.where(a > 0, a, 1.0))), -6, 8)
+    step = np.exp2(e - 3)
+    q = np.minimum(np.rint(a / step) * step, E4M3_MAX)   # numpy rint: ties to even
+    return np.copysign(q, x)
+
+
+def quantize_rows(x, quant=e4m3):
+    """R11: per-row scale s = amax(|row|) / 448 (1 for an all-zero row) and the codes quant(x / s)."""
+    x = np.asarray(x, F)
+    amax = np.max(np.abs(x), axis=-1, keepdims=True)
+    s = np.where(amax > 0, amax / E4M3_MAX, 1.0)
+    return quant(x / s), s
+
+
+def gemm_e4m3(x, w, quant=e4m3):
+    """x [T, K] @ w[N, K]^T with both operands quantised (per-token / per-output-channel scales, R11)
+    and the products of the codes summed in fp64, then rescaled."""
+    xq, sx = quantize_rows(x, quant)
+    wq, sw = quantize_rows(w, quant)
+    return (xq @ wq.T) * sx * sw.T
+
+
+def mlp_fp8(w, r, quant=e4m3):
+    """[DM05] 6.3 with reading R11: the SwiGLU MLP of a VLM layer with its gate, up and down GEMMs in
+    E4M3.  r [T, Hv] is the MLP's RMSNorm output; returns the MLP output added to the residual."""
+    gate = gemm_e4m3(r, w["Wg"], quant)
+    up = gemm_e4m3(r, w["Wu"], quant)
+    return gemm_e4m3(silu(gate) * up, w["Wd"], quant)
+
