@@ -129,10 +129,14 @@ dm0_status dm0_kv_commit(dm0_ctx* ctx, int B, int P);
  *   velocities: device f32 [steps][B][chunk][action_dim] per-step v, or NULL.
  * One observation (B = 1) with head_dim 128 runs the whole loop as ONE
  * persistent kernel (one CTA per SM, grid barriers between the phases of a
- * layer); otherwise, and when the environment variable DM0_NO_PERSIST=1 was
- * set at dm0_create, the loop is a chain of per-layer kernels captured once
- * per (B, P, steps) as a CUDA graph and replayed (launched directly when
- * velocities are requested).  No host work happens inside the loop.
+ * layer; DM0_PERSIST_SPLITS at dm0_create sets its attention key splits per
+ * KV head, default 7); otherwise, when the kernel cannot be resident on every
+ * SM, and when the environment variable DM0_NO_PERSIST=1 was set at
+ * dm0_create, the loop is a chain of per-layer kernels captured once per
+ * (B, P, steps) as a CUDA graph and replayed (launched directly when
+ * velocities are requested).  No host work happens inside the loop.  The
+ * persistent loop's split-K sums arrive in any order, so repeated calls are
+ * not bitwise identical.
  * Returns DM0_ESTATE without a cache, DM0_ESHAPE unless 1 <= steps <= 1000. */
 dm0_status dm0_denoise(dm0_ctx* ctx, const float* noise, int steps, float* actions, float* velocities,
                        void* stream);
