@@ -227,6 +227,23 @@ dm0_status dm0_attention_noalloc(const void* q, const void* ka, const void* va, 
                                  const void* vb, int Tb, void* o, int B, int Tq, int n_q, int n_kv, int head_dim,
                                  int splits, void* stream);
 
+/* FP8 packing (host). ---------------------------------------------------- */
+
+/* Packs a row-major fp32 matrix into FP8 E4M3 codes with one scale per row,
+ * the weight format of an FP8 GEMM whose rows are output channels (DM0.5 page,
+ * section 6.3: FP8 E4M3 for the prefix MLP's gate/up/down GEMMs, with scales).
+ * Per row r: s_r = max_k |x[r][k]| / 448 (1 for an all-zero row); code[r][k] is
+ * the E4M3 value nearest x[r][k] / s_r (1 sign, 4 exponent bits with bias 7, 3
+ * mantissa bits, no infinities, largest finite 448; ties to even; values beyond
+ * +-448 saturate), so x[r][k] ~= s_r * e4m3(code[r][k]).  Scales and quotients
+ * are computed in double.
+ *   x:      host f32 [rows][cols], read only.
+ *   codes:  host u8 [rows][cols] (OCP E4M3 bit patterns; no NaN is produced).
+ *   scales: host f32 [rows].
+ * Host-only and synchronous; no GPU is needed.  Returns DM0_EINVAL for null
+ * pointers or a non-finite input, DM0_ESHAPE unless rows, cols >= 1. */
+dm0_status dm0_pack_e4m3_rows(const float* x, int64_t rows, int64_t cols, uint8_t* codes, float* scales);
+
 /* Instrumentation. ------------------------------------------------------- */
 
 /* Number of kernels this context has enqueued so far (a replayed graph counts

@@ -23,7 +23,7 @@ def _lib():
 def _declared():
     src = open(os.path.join(ROOT, "include", "dm0.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(dm0_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(dm0_[a-z0-9_]+)\s*\(", src)))
 
 
 def test_library_exports_every_declared_symbol():

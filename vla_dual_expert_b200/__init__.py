@@ -13,7 +13,7 @@ import numpy as np
 from ._abi import (EXPORTS, LIB_PATH, SITES, Dm0Config, Dm0Error, load_library, make_config,  # noqa: F401
                    pack_weights)
 
-__all__ = ["Engine", "Dm0Error", "pack_weights", "load_library", "EXPORTS", "LIB_PATH"]
+__all__ = ["Engine", "Dm0Error", "pack_weights", "pack_e4m3_rows", "load_library", "EXPORTS", "LIB_PATH"]
 
 
 c_int_t = ctypes.c_int
@@ -36,6 +36,21 @@ def _check_cuda(t, dtype, shape, name):
         raise TypeError(f"{name} must be a contiguous CUDA {dtype} tensor")
     if tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def pack_e4m3_rows(x: np.ndarray):
+    """FP8 E4M3 codes (uint8, OCP bit patterns) and one fp32 scale per row of a 2-D array, through
+    dm0_pack_e4m3_rows (host code; no GPU needed)."""
+    lib = load_library()
+    a = np.ascontiguousarray(x, np.float32)
+    if a.ndim != 2:
+        raise ValueError("pack_e4m3_rows expects a 2-D array")
+    codes = np.empty(a.shape, np.uint8)
+    scales = np.empty(a.shape[0], np.float32)
+    st = lib.dm0_pack_e4m3_rows(a.ctypes.data, a.shape[0], a.shape[1], codes.ctypes.data, scales.ctypes.data)
+    if st != 0:
+        raise Dm0Error(st, "dm0_pack_e4m3_rows")
+    return codes, scales
 
 
 class Engine:

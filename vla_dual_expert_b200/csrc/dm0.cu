@@ -1357,4 +1357,42 @@ void dm0_destroy(dm0_ctx* c) {
   delete c;
 }
 
+dm0_status dm0_pack_e4m3_rows(const float* x, int64_t rows, int64_t cols, uint8_t* codes, float* scales) {
+  if (!x || !codes || !scales) return DM0_EINVAL;
+  if (rows < 1 || cols < 1) return DM0_ESHAPE;
+  for (int64_t r = 0; r < rows; ++r) {
+    const float* row = x + r * cols;
+    double amax = 0.0;
+    for (int64_t k = 0; k < cols; ++k) {
+      if (!std::isfinite(row[k])) return DM0_EINVAL;
+      amax = std::max(amax, std::fabs(static_cast<double>(row[k])));
+    }
+    const double s = amax > 0.0 ? amax / 448.0 : 1.0;
+    scales[r] = static_cast<float>(s);
+    for (int64_t k = 0; k < cols; ++k) {
+      const double v = static_cast<double>(row[k]) / s;
+      const double a = std::fabs(v);
+      // spacing 2^(e-3) with e = floor(log2 a) in [-6, 8] (below 2^-6: the subnormal spacing 2^-9)
+      int e = a > 0.0 ? static_cast<int>(std::floor(std::log2(a))) : -6;
+      e = std::min(8, std::max(-6, e));
+      double q = std::nearbyint(std::ldexp(a, 3 - e));   // the default rounding mode: ties to even
+      q = std::ldexp(q, e - 3);
+      if (q > 448.0) q = 448.0;
+      uint8_t bits = 0;
+      if (q > 0.0) {
+        if (q < 0.015625) {   // subnormal: m 2^-9, m in 1..7
+          bits = static_cast<uint8_t>(std::lrint(std::ldexp(q, 9)));
+        } else {              // normal: (1 + m/8) 2^E, biased exponent E + 7 in 1..15
+          const int E = static_cast<int>(std::floor(std::log2(q)));
+          const int m = static_cast<int>(std::lrint(std::ldexp(q, 3 - E))) - 8;
+          bits = static_cast<uint8_t>(((E + 7) << 3) | m);
+        }
+      }
+      if (std::signbit(v) && q > 0.0) bits |= 0x80;
+      codes[r * cols + k] = bits;
+    }
+  }
+  return DM0_OK;
+}
+
 }  // extern "C"
