@@ -98,9 +98,13 @@ def project_qkv(w, h, positions, d):
     h [T, H] -> q [Hq, T, D], k [Hkv, T, D], v [Hkv, T, D].  [DM0-arch]: each
     branch makes its own Q/K/V with the same head count and head_dim.
     """
-    T = h.shape[0]
+    return qkv_from_normed(w, rms_norm(h, w["attn_norm"], d.rms_eps), positions, d)
+
+
+def qkv_from_normed(w, r, positions, d):
+    """The part of project_qkv after the pre-norm: r [T, H] (the normalised residual) -> q, k, v."""
+    T = r.shape[0]
     D = d.head_dim
-    r = rms_norm(h, w["attn_norm"], d.rms_eps)
     q = (r @ np.asarray(w["Wq"], F).T).reshape(T, d.n_q, D).transpose(1, 0, 2)
     k = (r @ np.asarray(w["Wk"], F).T).reshape(T, d.n_kv, D).transpose(1, 0, 2)
     v = (r @ np.asarray(w["Wv"], F).T).reshape(T, d.n_kv, D).transpose(1, 0, 2)

@@ -28,6 +28,10 @@ import numpy as np
 LAYER_TENSORS = ("attn_norm", "Wq", "Wk", "Wv", "q_norm", "k_norm",
                  "Wo", "mlp_norm", "Wg", "Wu", "Wd")
 HEAD_TENSORS = ("W_in", "b_in", "final_norm", "W_out", "b_out")
+# time-modulated action expert (DM0.5): the time MLP and the final norm's modulator ...
+TIME_TENSORS = ("W_ti", "b_ti", "W_to", "b_to", "W_mf", "b_mf")
+# ... and one modulator per action layer for each of its two pre-norms (attention, MLP)
+MOD_TENSORS = ("W_ma", "b_ma", "W_mm", "b_mm")
 BRANCH_VLM, BRANCH_ACTION = 0, 1
 
 
@@ -191,6 +195,34 @@ def head_weights(d: Dims, seed: int = 0, std: float = 0.02, gain_jitter: float =
     return out
 
 
+def time_shapes(d: Dims) -> dict:
+    H = d.hidden_a
+    return {"W_ti": (H, H), "b_ti": (H,), "W_to": (H, H), "b_to": (H,),
+            "W_mf": (2 * H, H), "b_mf": (2 * H,)}
+
+
+def mod_shapes(d: Dims) -> dict:
+    H = d.hidden_a
+    return {"W_ma": (3 * H, H), "b_ma": (3 * H,), "W_mm": (3 * H, H), "b_mm": (3 * H,)}
+
+
+def _draw_group(shapes: dict, ent0: tuple, std: float) -> dict:
+    """Matrices N(0, std^2) rounded to bf16; vectors (biases) N(0, std^2) fp32."""
+    return {name: _normal(ent0 + (tid,), shape, std, bf16=len(shape) == 2)
+            for tid, (name, shape) in enumerate(shapes.items())}
+
+
+def time_weights(d: Dims, seed: int = 0, std: float = 0.02) -> dict:
+    """time_mlp_in (W_ti, b_ti), time_mlp_out (W_to, b_to) and the final norm's modulator (W_mf, b_mf)."""
+    return _draw_group(time_shapes(d), (seed, 4, 0), std)
+
+
+def mod_weights(d: Dims, layer: int, seed: int = 0, std: float = 0.02) -> dict:
+    """The two time modulators of action layer `layer`: attention pre-norm (W_ma, b_ma), MLP pre-norm
+    (W_mm, b_mm); each maps the time condition to three vectors of hidden_a."""
+    return _draw_group(mod_shapes(d), (seed, 3, layer), std)
+
+
 class Weights:
     """Lazily generated model parameters (per-layer access, cached on request)."""
 
@@ -199,7 +231,10 @@ class Weights:
         self.d, self.seed, self.std, self.gain_jitter = d, seed, std, gain_jitter
         self._cache = {} if cache else None
         self._head = None
-        self.overrides = {}   # (branch, layer, name) or ("head", name) -> array
+        self._time = None
+        self._mods = {} if cache else None
+        # (branch, layer, name), ("head", name), ("time", name) or ("mod", layer, name) -> array
+        self.overrides = {}
 
     def layer(self, branch: int, layer: int) -> dict:
         key = (branch, layer)
@@ -209,12 +244,32 @@ class Weights:
             w = layer_weights(self.d, branch, layer, self.seed, self.std, self.gain_jitter)
             if self._cache is not None:
                 self._cache[key] = w
-        if any(k[:2] == key for k in self.overrides if len(k) == 3):
+        if any(k[:2] == key for k in self.overrides if len(k) == 3 and k[0] != "mod"):
             w = dict(w)
             for k, v in self.overrides.items():
                 if len(k) == 3 and k[:2] == key:
                     w[k[2]] = v
         return w
+
+    def _with_overrides(self, w: dict, key: tuple) -> dict:
+        extra = {k[-1]: v for k, v in self.overrides.items() if k[:-1] == key}
+        return dict(w, **extra) if extra else w
+
+    def time(self) -> dict:
+        """Time MLP and final-norm modulator of the time-modulated action expert."""
+        if self._time is None:
+            self._time = time_weights(self.d, self.seed, self.std)
+        return self._with_overrides(self._time, ("time",))
+
+    def mod(self, layer: int) -> dict:
+        """Time modulators of action layer `layer`."""
+        if self._mods is not None and layer in self._mods:
+            w = self._mods[layer]
+        else:
+            w = mod_weights(self.d, layer, self.seed, self.std)
+            if self._mods is not None:
+                self._mods[layer] = w
+        return self._with_overrides(w, ("mod", layer))
 
     def head(self) -> dict:
         if self._head is None:
@@ -250,3 +305,26 @@ def random_kv_layer(d: Dims, batch: int, prefix: int, layer: int, seed: int = 30
 def hidden_states(batch_tokens: int, hidden: int, seed: int, scale: float = 1.0) -> np.ndarray:
     """fp32 N(0, scale^2) residual-stream inputs for single-layer checks."""
     return _normal((seed, 7), (batch_tokens, hidden), scale)
+
+
+def train_batch(d: Dims, batch: int, seed: int = 4000):
+    """Synthetic flow-matching training inputs, sample b from seed + b.
+
+    actions a and noise eps: [B][chunk][action_dim] N(0, 1) fp32; t: [B] uniform in [0, 1) (float64);
+    mask: [B][chunk][action_dim] bool marking the valid entries: the first n_dims action dimensions
+    (a robot whose action vector is shorter than action_dim, zero-padded) of the first n_steps chunk
+    positions (an episode that ends inside the chunk), n_dims uniform in [1, action_dim] and n_steps
+    uniform in [1, chunk].
+    """
+    a, eps, t, mask = [], [], [], []
+    for b in range(batch):
+        a.append(_normal((seed + b, 0), (d.chunk, d.action_dim)))
+        eps.append(_normal((seed + b, 1), (d.chunk, d.action_dim)))
+        rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed + b, 2])))
+        t.append(rng.random())
+        n_dims = int(rng.integers(1, d.action_dim + 1))
+        n_steps = int(rng.integers(1, d.chunk + 1))
+        m = np.zeros((d.chunk, d.action_dim), dtype=bool)
+        m[:n_steps, :n_dims] = True
+        mask.append(m)
+    return np.stack(a), np.stack(eps), np.asarray(t, np.float64), np.stack(mask)
