@@ -173,6 +173,31 @@ dm0_status dm0_merged_layer(dm0_ctx* ctx, int layer, const float* h_prefix, cons
 dm0_status dm0_op_gemm(dm0_ctx* ctx, const void* A, const void* B, float* C, int M, int N, int K, int swap,
                        int splits, void* stream);
 
+/* Per-row FP8 E4M3 quantisation on the GPU (the operand step of the FP8
+ * prefix MLP, DM0.5 page, section 6.3).  Row r of x, y[c] = x[r][c], times
+ * gain[c] when gain is not null, times 1/sqrt(ssq[r] / cols + eps_rms) when ssq
+ * is not null (a pending RMSNorm; eps from the context's config), in fp32:
+ *   scales[r] = max_c |y[c]| / 448 (an fp32 division; 1 for an all-zero row),
+ *   codes[r][c] = E4M3(y[c] / scales[r]), the quotient an IEEE fp32 division
+ *   and the conversion round-to-nearest-even, saturating at +-448.
+ * x device [rows][cols], fp32 when x_f32 != 0 else bf16 (16-byte aligned);
+ * gain device f32 [cols] (16-byte aligned) or null; ssq device f32 [rows] or
+ * null; codes device u8 [rows][cols] (8-byte aligned; OCP E4M3 bit patterns);
+ * scales device f32 [rows].  rows >= 1, cols >= 8 and cols % 8 == 0, else
+ * DM0_ESHAPE; null required pointers or misalignment give DM0_EINVAL.
+ * Asynchronous on `stream`. */
+dm0_status dm0_op_quant_e4m3(dm0_ctx* ctx, const void* x, int x_f32, int rows, int cols, const float* gain,
+                             const float* ssq, void* codes, float* scales, void* stream);
+
+/* FP8 E4M3 tensor-core GEMM with per-row scales on both operands:
+ *   C[m][n] = sa[m] * sb[n] * sum_k e4m3(A[m][k]) e4m3(B[n][k]),
+ * products of codes accumulated in fp32.  A device u8 [M][K] and B device u8
+ * [N][K] codes, K-contiguous (16-byte aligned); sa device f32 [M]; sb device
+ * f32 [N] (16-byte aligned); C device f32 [M][N], written.  M >= 1, N % 128 ==
+ * 0, K % 128 == 0, else DM0_ESHAPE.  Asynchronous on `stream`. */
+dm0_status dm0_op_gemm_e4m3(dm0_ctx* ctx, const void* A, const float* sa, const void* B, const float* sb, float* C,
+                            int M, int N, int K, void* stream);
+
 /* Merged GQA attention of one segment pair, for tests:
  *   q:  device bf16 [B][Tq][n_q][head_dim]
  *   ka/va: device bf16 [B][n_kv][Ta][head_dim]; kb/vb: [B][n_kv][Tb][head_dim]
@@ -226,6 +251,25 @@ dm0_status dm0_debug_view(dm0_ctx* ctx, const char* name, void** ptr);
 dm0_status dm0_attention_noalloc(const void* q, const void* ka, const void* va, int Ta, const void* kb,
                                  const void* vb, int Tb, void* o, int B, int Tq, int n_q, int n_kv, int head_dim,
                                  int splits, void* stream);
+
+/* FP8 E4M3 prefix MLP (DM0.5 page, section 6.3). ---------------------------- */
+
+/* enable != 0: from now on every VLM-branch MLP of this context (dm0_prefill
+ * and the VLM half of dm0_merged_layer) runs its gate/up and down GEMMs in
+ * FP8 E4M3: the weights are quantised once here, per output channel, from the
+ * resident bf16 weights (and again by every later dm0_load_weights); each
+ * GEMM's operand is quantised per token from fp32 just before it (the gate/up
+ * operand is the normalised residual rms(h) * g, the down operand the SwiGLU
+ * output; the rules of dm0_op_quant_e4m3); products accumulate in fp32 and
+ * both scales are applied in the GEMM's epilogue.  The action expert stays bf16.  enable == 0 returns
+ * to the bf16 MLP (the FP8 copies are kept).
+ * Needs loaded weights (DM0_ESTATE) and hidden_v, inter_v multiples of 128
+ * (DM0_ESHAPE).  The first enable allocates the FP8 weights (1 byte per MLP
+ * weight of the VLM) and operands (max_batch * max_prefix * (hidden_v +
+ * 5 inter_v) bytes: codes and the fp32 SwiGLU output); DM0_ENOMEM if that
+ * fails.  The weight quantisation is
+ * queued on `stream`. */
+dm0_status dm0_set_prefix_fp8(dm0_ctx* ctx, int enable, void* stream);
 
 /* FP8 packing (host). ---------------------------------------------------- */
 

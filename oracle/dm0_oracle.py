@@ -113,12 +113,17 @@ def qkv_from_normed(w, r, positions, d):
     return q, k, v
 
 
-def finish_layer(w, h, o, d):
-    """Branch-own O-proj + residual, then pre-norm SwiGLU MLP + residual. o [Hq, T, D]."""
+def finish_layer(w, h, o, d, fp8=None):
+    """Branch-own O-proj + residual, then pre-norm SwiGLU MLP + residual. o [Hq, T, D].
+
+    fp8: None for the plain MLP; True for the E4M3 MLP of R11 (mlp_fp8); a row quantiser (as qrows of
+    gemm_e4m3) for the E4M3 MLP with that quantiser."""
     T = h.shape[0]
     o_flat = o.transpose(1, 0, 2).reshape(T, d.n_q * d.head_dim)
     h = np.asarray(h, F) + o_flat @ np.asarray(w["Wo"], F).T
     r = rms_norm(h, w["mlp_norm"], d.rms_eps)
+    if fp8 is not None:
+        return h + mlp_fp8(w, r, qrows=None if fp8 is True else fp8)
     gate = r @ np.asarray(w["Wg"], F).T
     up = r @ np.asarray(w["Wu"], F).T
     return h + (silu(gate) * up) @ np.asarray(w["Wd"], F).T
@@ -132,11 +137,12 @@ def block_mask(P, S):
     return vis
 
 
-def merged_layer(wv, wa, h_prefix, h_suffix, d):
+def merged_layer(wv, wa, h_prefix, h_suffix, d, vlm_fp8=None):
     """One dual-expert layer over the explicitly concatenated sequence ([DM0-arch]).
 
     h_prefix [P, Hv], h_suffix [S, Ha] (one sample).  Returns
-    (h_prefix', h_suffix', k_prefix [Hkv,P,D], v_prefix [Hkv,P,D]).
+    (h_prefix', h_suffix', k_prefix [Hkv,P,D], v_prefix [Hkv,P,D]).  vlm_fp8 selects the VLM
+    branch's E4M3 MLP as finish_layer's fp8 does (the action branch stays plain).
     """
     P, S = h_prefix.shape[0], h_suffix.shape[0]
     qv, kv, vv = project_qkv(wv, h_prefix, np.arange(P), d)
@@ -145,7 +151,7 @@ def merged_layer(wv, wa, h_prefix, h_suffix, d):
     k = np.concatenate([kv, ka], axis=1)
     v = np.concatenate([vv, va], axis=1)
     o = attention(q, k, v, block_mask(P, S))
-    return (finish_layer(wv, h_prefix, o[:, :P], d),
+    return (finish_layer(wv, h_prefix, o[:, :P], d, vlm_fp8),
             finish_layer(wa, h_suffix, o[:, P:], d), kv, vv)
 
 
@@ -276,18 +282,52 @@ def quantize_rows(x, quant=e4m3):
     return quant(x / s), s
 
 
-def gemm_e4m3(x, w, quant=e4m3):
+def quantize_rows_f32(x):
+    """R11 with the decision taken in fp32, the precision of the GPU quantiser: a code is an integer
+    decided by floating point, so for code-level parity both sides decide it the same way.  The scale
+    is fp32(amax) / 448 and the quotient x / scale an fp32 division (IEEE, correctly rounded in both
+    numpy and the GPU), then rounded to E4M3 as in e4m3()."""
+    x32 = np.asarray(x, np.float32)
+    amax = np.max(np.abs(x32), axis=-1, keepdims=True)
+    s = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    return e4m3((x32 / s).astype(F)), s.astype(F)
+
+
+def gemm_e4m3(x, w, quant=e4m3, qrows=None):
     """x [T, K] @ w[N, K]^T with both operands quantised (per-token / per-output-channel scales, R11)
-    and the products of the codes summed in fp64, then rescaled."""
-    xq, sx = quantize_rows(x, quant)
-    wq, sw = quantize_rows(w, quant)
+    and the products of the codes summed in fp64, then rescaled.  qrows(m) -> (codes, scales) replaces
+    the row quantiser (default: quantize_rows with the element rounding `quant`)."""
+    if qrows is None:
+        def qrows(m):
+            return quantize_rows(m, quant)
+    xq, sx = qrows(x)
+    wq, sw = qrows(w)
     return (xq @ wq.T) * sx * sw.T
 
 
-def mlp_fp8(w, r, quant=e4m3):
+def mlp_fp8(w, r, quant=e4m3, qrows=None):
     """[DM05] 6.3 with reading R11: the SwiGLU MLP of a VLM layer with its gate, up and down GEMMs in
-    E4M3.  r [T, Hv] is the MLP's RMSNorm output; returns the MLP output added to the residual."""
-    gate = gemm_e4m3(r, w["Wg"], quant)
-    up = gemm_e4m3(r, w["Wu"], quant)
-    return gemm_e4m3(silu(gate) * up, w["Wd"], quant)
+    E4M3.  r [T, Hv] is the MLP's RMSNorm output; returns the MLP output (the residual add is the
+    caller's)."""
+    gate = gemm_e4m3(r, w["Wg"], quant, qrows)
+    up = gemm_e4m3(r, w["Wu"], quant, qrows)
+    return gemm_e4m3(silu(gate) * up, w["Wd"], quant, qrows)
+
+
+def prefill_fp8(weights, prefix_emb, qrows=None):
+    """The prefix pass (as prefill) with every VLM MLP in E4M3 (R11): the attention half of each layer
+    is unchanged, the MLP is mlp_fp8 of the MLP's RMSNorm output (qrows as in gemm_e4m3).  Returns
+    ([k_l], [v_l], h_final)."""
+    d = weights.d
+    h = np.asarray(prefix_emb, F)
+    P = h.shape[0]
+    ks, vs = [], []
+    vis = np.ones((P, P), dtype=bool)
+    for l in range(d.layers):
+        w = weights.layer(0, l)
+        q, k, v = project_qkv(w, h, np.arange(P), d)
+        ks.append(k)
+        vs.append(v)
+        h = finish_layer(w, h, attention(q, k, v, vis), d, True if qrows is None else qrows)
+    return ks, vs, h
 

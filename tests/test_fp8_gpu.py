@@ -1,0 +1,234 @@
+"""Parity of the FP8 E4M3 prefix-MLP path (reading R11 of the DM0.5 page, section 6.3) with the oracle.
+
+Code decisions are integers decided by floating point, so the oracle side takes them in the GPU
+quantiser's precision (quantize_rows_f32: fp32 scale and fp32 quotient).  Tolerances:
+  quantiser, same fp32 / bf16 input      bit-exact codes and scales
+  quantiser with the pending RMSNorm     scales within 1e-6; at most 0.5 % of codes differ, each by one
+                                         E4M3 step (the normalised row is rounded differently in fp32
+                                         on the GPU and in fp64 in the oracle)
+  FP8 GEMM                               max |d| <= 2e-5 RMS: the products of E4M3 codes are exact in
+                                         fp32, only the order of the fp32 summation differs
+  one merged layer, FP8 VLM MLP          K / V and the action branch as in the bf16 layer test; the VLM
+                                         output RMS(d) <= 5e-3 RMS, max <= 0.1 RMS and at most 2 % of the
+                                         elements beyond 1e-2 RMS: a code whose fp32 quotient lies within
+                                         a few fp32 ulps of an E4M3 midpoint can round either way, and
+                                         one such flip moves a whole output column by a step of 2^-3
+                                         relative (emulated on the CPU with 3-ulp noise on the operands:
+                                         max 0.024, RMS 8e-4, 0.2 % of the elements beyond 1e-2 RMS)
+The kernels in this file have not yet run on a GPU; DM0_RUN_FP8=1 selects them.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import dm0_oracle as O
+from synth import inputs as I
+from tests.gpu_util import check_bf16, check_fp, host, rel_err, rms, to_dev_bf16, to_dev_f32
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(os.environ.get("DM0_RUN_FP8") != "1",
+                                 reason="FP8 kernels await their first GPU run (DM0_RUN_FP8=1)")]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from vla_dual_expert_b200 import build
+    build.build()
+
+
+def _engine(d, max_batch, max_prefix, w):
+    from vla_dual_expert_b200 import Engine
+    eng = Engine(d, max_batch, max_prefix)
+    eng.load_from(w)
+    return eng
+
+
+@pytest.fixture(scope="module")
+def eng1():
+    d = I.DM0_BASE.replace(layers=1)
+    w = I.Weights(d, seed=0, gain_jitter=0.1)
+    eng = _engine(d, 2, 816, w)
+    yield d, w, eng
+    eng.close()
+
+
+def _decode(codes: torch.Tensor) -> np.ndarray:
+    return codes.cpu().view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def _quant(eng, x, gain=None, ssq=None):
+    rows, cols = x.shape
+    codes = torch.empty((rows, cols), device="cuda", dtype=torch.uint8)
+    scales = torch.empty(rows, device="cuda", dtype=torch.float32)
+    eng.op_quant_e4m3(x, codes, scales, gain, ssq)
+    eng.sync()
+    assert eng.device_error() == 0
+    return codes, scales
+
+
+# ------------------------------------------------------------------ quantiser
+
+@pytest.mark.parametrize("rows,cols", [(3, 8), (37, 2048), (300, 6144)])
+def test_quant_bf16_rows_bit_exact(eng1, rows, cols):
+    _, _, eng = eng1
+    rng = np.random.default_rng(rows)
+    x = I.round_bf16((rng.standard_normal((rows, cols)) * np.exp2(rng.uniform(-20, 20, (rows, 1)))).astype(np.float32))
+    x[rows // 2] = 0.0                                  # all-zero row: scale 1, codes 0
+    x[-1, :] = 0.0
+    x[-1, cols // 3] = -3.5                             # a single nonzero maps to -448
+    codes, scales = _quant(eng, to_dev_bf16(x))
+    q, s = O.quantize_rows_f32(x)
+    assert np.array_equal(_decode(codes), q)
+    assert np.array_equal(host(scales), s[:, 0])
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 128), (129, 2048)])
+def test_quant_f32_rows_bit_exact(eng1, rows, cols):
+    _, _, eng = eng1
+    rng = np.random.default_rng(100 + rows)
+    x = (rng.standard_normal((rows, cols)) * np.exp2(rng.uniform(-8, 8, (rows, 1)))).astype(np.float32)
+    codes, scales = _quant(eng, to_dev_f32(x))
+    q, s = O.quantize_rows_f32(x)
+    assert np.array_equal(_decode(codes), q)
+    assert np.array_equal(host(scales), s[:, 0])
+
+
+def test_quant_with_pending_rmsnorm(eng1):
+    d, _, eng = eng1
+    rng = np.random.default_rng(7)
+    M, H = 200, d.hidden_v
+    h = rng.standard_normal((M, H)).astype(np.float32) * 3.0
+    g = (1.0 + 0.1 * rng.standard_normal(H)).astype(np.float32)
+    ssq = np.sum(h.astype(np.float64) ** 2, axis=1).astype(np.float32)
+    codes, scales = _quant(eng, to_dev_f32(h), to_dev_f32(g), to_dev_f32(ssq))
+    r = O.rms_norm(h, g, d.rms_eps)
+    q, s = O.quantize_rows_f32(r)
+    np.testing.assert_allclose(host(scales), s[:, 0], rtol=1e-6)
+    got = _decode(codes)
+    differ = got != q
+    assert differ.mean() <= 5e-3
+    step = np.exp2(np.clip(np.floor(np.log2(np.maximum(np.abs(q[differ]), 2.0 ** -9))), -6, 8) - 3)
+    assert np.all(np.abs(got[differ] - q[differ]) <= step * 1.0000001)
+
+
+# ------------------------------------------------------------------ FP8 GEMM
+
+@pytest.mark.parametrize("M,N,K", [(1, 128, 128), (300, 384, 256), (129, 256, 6144), (816, 12288, 2048)])
+def test_gemm_e4m3_matches_exact_products(eng1, M, N, K):
+    _, _, eng = eng1
+    rng = np.random.default_rng(M + N + K)
+    a = rng.standard_normal((M, K)).astype(np.float32)
+    b = (0.02 * rng.standard_normal((N, K))).astype(np.float32)
+    A, sa = _quant(eng, to_dev_f32(a))
+    B, sb = _quant(eng, to_dev_f32(b))
+    C = torch.empty((M, N), device="cuda", dtype=torch.float32)
+    eng.op_gemm_e4m3(A, sa, B, sb, C)
+    eng.sync()
+    assert eng.device_error() == 0
+    ref = (_decode(A) @ _decode(B).T) * host(sa)[:, None] * host(sb)[None, :]
+    check_fp(host(C), ref, 2e-5, f"FP8 GEMM {M}x{N}x{K}")
+
+
+# ------------------------------------------------------------------ one merged layer with the FP8 VLM MLP
+
+def _fp8_stats(got, ref, what):
+    d = np.abs(np.asarray(got, np.float64) - ref)
+    r = rms(ref)
+    out = (float(np.sqrt(np.mean(d ** 2)) / r), float(d.max() / r), float(np.mean(d > 1e-2 * r)))
+    print(f"  {what}: RMS(d)/RMS {out[0]:.2e}  max/RMS {out[1]:.2e}  beyond 1e-2 {out[2]:.2e}")
+    return out
+
+
+@pytest.mark.parametrize("B,P", [(1, 816), (2, 333)])
+def test_merged_layer_fp8(eng1, B, P):
+    d, w, eng = eng1
+    S = d.chunk
+    hp = np.stack([I.hidden_states(P, d.hidden_v, seed=40 + b) for b in range(B)])
+    hs = np.stack([I.hidden_states(S, d.hidden_a, seed=140 + b) for b in range(B)])
+    outp = torch.empty((B, P, d.hidden_v), device="cuda", dtype=torch.float32)
+    outs = torch.empty((B, S, d.hidden_a), device="cuda", dtype=torch.float32)
+    k = torch.empty((B, d.n_kv, P, d.head_dim), device="cuda", dtype=torch.bfloat16)
+    v = torch.empty_like(k)
+    eng.set_prefix_fp8(True)
+    try:
+        eng.merged_layer(0, to_dev_f32(hp), to_dev_f32(hs), outp, outs, k, v)
+        eng.sync()
+    finally:
+        eng.set_prefix_fp8(False)
+    assert eng.device_error() == 0
+    for b in range(B):
+        rp, rs_, rk, rv = O.merged_layer(w.layer(0, 0), w.layer(1, 0), hp[b], hs[b], d, vlm_fp8=O.quantize_rows_f32)
+        check_bf16(host(k[b]), rk, 1e-2, "prefix K")
+        check_bf16(host(v[b]), rv, 1e-2, "prefix V")
+        check_fp(host(outs[b]), rs_, 1e-2, "suffix out (bf16 action branch)")
+        r_rms, r_max, r_frac = _fp8_stats(host(outp[b]), rp, "prefix out, FP8 MLP")
+        assert r_rms <= 5e-3 and r_max <= 0.1 and r_frac <= 0.02
+        # and it is the FP8 MLP that was run: far closer to the FP8 oracle than to the plain one
+        plain = O.merged_layer(w.layer(0, 0), w.layer(1, 0), hp[b], hs[b], d)[0]
+        assert rms(host(outp[b]) - rp) < 0.25 * rms(plain - rp)
+
+
+def test_fp8_toggle_leaves_the_bf16_path_unchanged(eng1):
+    d, _, eng = eng1
+    P, S = 200, d.chunk
+    hp, hs = I.hidden_states(P, d.hidden_v, seed=60)[None], I.hidden_states(S, d.hidden_a, seed=61)[None]
+
+    def run():
+        outp = torch.empty((1, P, d.hidden_v), device="cuda", dtype=torch.float32)
+        outs = torch.empty((1, S, d.hidden_a), device="cuda", dtype=torch.float32)
+        k = torch.empty((1, d.n_kv, P, d.head_dim), device="cuda", dtype=torch.bfloat16)
+        eng.merged_layer(0, to_dev_f32(hp), to_dev_f32(hs), outp, outs, k, torch.empty_like(k))
+        eng.sync()
+        return host(outp)
+
+    before = run()
+    eng.set_prefix_fp8(True)
+    fp8 = run()
+    eng.set_prefix_fp8(False)
+    after = run()
+    assert np.array_equal(before, after)
+    assert not np.array_equal(before, fp8)
+
+
+def test_enable_before_weights_is_a_state_error():
+    from vla_dual_expert_b200 import Dm0Error, Engine
+    eng = Engine(I.TINY, 1, 64)
+    try:
+        with pytest.raises(Dm0Error):
+            eng.set_prefix_fp8(True)
+    finally:
+        eng.close()
+
+
+# ------------------------------------------------------------------ a whole prefix pass (tiny model)
+
+def test_tiny_prefill_fp8(eng1):
+    from vla_dual_expert_b200 import Engine
+    d = I.TINY
+    w = I.Weights(d, seed=0, gain_jitter=0.1)
+    P = 64
+    emb = I.prefix_embeddings(d, 1, P)
+    eng = Engine(d, 1, P)
+    try:
+        eng.load_from(w)
+        eng.set_prefix_fp8(True)
+        eng.prefill(to_dev_bf16(emb))
+        eng.sync()
+        assert eng.device_error() == 0
+        kp, vp = eng.kv_view()
+        from tests.gpu_util import device_view_bf16
+        K = host(device_view_bf16(kp, (d.layers, d.n_kv, P, d.head_dim)))
+        V = host(device_view_bf16(vp, (d.layers, d.n_kv, P, d.head_dim)))
+    finally:
+        eng.close()
+    ks, vs, _ = O.prefill_fp8(w, emb[0], qrows=O.quantize_rows_f32)
+    ks0, vs0, _ = O.prefill(w, emb[0])
+    for l in range(d.layers):
+        for got, ref, plain, nm in ((K[l], ks[l], ks0[l], "K"), (V[l], vs[l], vs0[l], "V")):
+            r_rms, _, _ = _fp8_stats(got, ref, f"layer {l} {nm}")
+            assert r_rms <= 1e-2 * np.sqrt(l + 1)
+            if l > 0:   # layer 0's K/V precede any MLP
+                assert rms(got - ref) < 0.5 * rms(plain - ref)

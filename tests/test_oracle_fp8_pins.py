@@ -89,3 +89,49 @@ def test_mlp_plumbing_with_an_exact_quantiser():
     fp8 = O.mlp_fp8(w, r)
     rel = np.sqrt(np.mean((fp8 - exact) ** 2)) / np.sqrt(np.mean(exact ** 2))
     assert 1e-3 < rel < 0.1                                 # E4M3 error, not a wiring error
+
+
+def test_fp32_quantiser_matches_torch_fp32_arithmetic():
+    # the decision in fp32 (the GPU quantiser's precision): torch float32 amax / 448 and float32
+    # division, then torch's E4M3 cast (no value exceeds 448 after the division by amax / 448)
+    rng = np.random.default_rng(17)
+    x = (rng.standard_normal((40, 300)) * np.exp2(rng.uniform(-30, 30, size=(40, 1)))).astype(np.float32)
+    x[5] = 0.0
+    q, s = O.quantize_rows_f32(x)
+    xt = torch.from_numpy(x)
+    amax = xt.abs().amax(dim=1, keepdim=True)
+    st = torch.where(amax > 0, amax / torch.tensor(448.0, dtype=torch.float32), torch.ones_like(amax))
+    ref = (xt / st).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(q, ref) and np.array_equal(s, st.to(torch.float64).numpy())
+    assert np.all(np.max(np.abs(q[np.arange(40) != 5]), axis=1) == O.E4M3_MAX)   # the row's amax maps to 448
+    assert s[5, 0] == 1.0 and not q[5].any()
+
+
+def test_fp32_and_fp64_quantisers_differ_only_at_rounding_boundaries():
+    # the two decisions agree except where x / s lies within fp32 rounding of an E4M3 midpoint
+    rng = np.random.default_rng(18)
+    x = rng.standard_normal((64, 512)).astype(np.float32)
+    q32, s32 = O.quantize_rows_f32(x)
+    q64, s64 = O.quantize_rows(x.astype(np.float64))
+    assert np.max(np.abs(s32 / s64 - 1.0)) < 2.0 ** -23
+    differ = q32 != q64
+    assert differ.mean() < 1e-3
+    # where they differ, they are neighbouring E4M3 values (one step apart)
+    steps = np.exp2(np.clip(np.floor(np.log2(np.maximum(np.abs(q64[differ]), 2.0 ** -9))), -6, 8) - 3)
+    assert np.all(np.abs(q32[differ] - q64[differ]) <= steps * 1.0000001)
+
+
+def test_fp8_prefill_reduces_to_the_bf16_prefill_with_an_exact_quantiser():
+    from synth import inputs as I
+    d = I.TINY
+    w = I.Weights(d, seed=0, gain_jitter=0.1)
+    emb = I.prefix_embeddings(d, 1, 24)[0]
+    ks, vs, h = O.prefill(w, emb)
+    ident = lambda m: (np.asarray(m, np.float64), np.ones((np.shape(m)[0], 1)))   # noqa: E731
+    ks8, vs8, h8 = O.prefill_fp8(w, emb, qrows=ident)
+    assert np.max(np.abs(h8 - h)) <= 1e-12 * np.max(np.abs(h))
+    for a, b in zip(ks8 + vs8, ks + vs):
+        assert np.max(np.abs(a - b)) <= 1e-12 * np.max(np.abs(b))
+    _, _, hq = O.prefill_fp8(w, emb)
+    rel = np.sqrt(np.mean((hq - h) ** 2)) / np.sqrt(np.mean(h ** 2))
+    assert 1e-5 < rel < 0.05     # E4M3 noise on the MLP branch only, not a wiring error

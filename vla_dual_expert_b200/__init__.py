@@ -152,6 +152,36 @@ class Engine:
         _check_cuda(C, torch.float32, (N, M) if swap else (M, N), "C")
         self._chk(self.lib.dm0_op_gemm(self.h, _ptr(A), _ptr(B), _ptr(C), M, N, K, swap, splits, _stream(stream)))
 
+    def set_prefix_fp8(self, enable: bool = True, stream=None):
+        """Run the VLM MLP's gate/up and down GEMMs in FP8 E4M3 (dm0_set_prefix_fp8)."""
+        self._chk(self.lib.dm0_set_prefix_fp8(self.h, 1 if enable else 0, _stream(stream)))
+
+    def op_quant_e4m3(self, x, codes, scales, gain=None, ssq=None, stream=None):
+        import torch
+        rows, cols = x.shape
+        f32 = x.dtype == torch.float32
+        _check_cuda(x, torch.float32 if f32 else torch.bfloat16, (rows, cols), "x")
+        _check_cuda(codes, torch.uint8, (rows, cols), "codes")
+        _check_cuda(scales, torch.float32, (rows,), "scales")
+        if gain is not None:
+            _check_cuda(gain, torch.float32, (cols,), "gain")
+        if ssq is not None:
+            _check_cuda(ssq, torch.float32, (rows,), "ssq")
+        self._chk(self.lib.dm0_op_quant_e4m3(self.h, _ptr(x), int(f32), rows, cols, _ptr(gain), _ptr(ssq),
+                                             _ptr(codes), _ptr(scales), _stream(stream)))
+
+    def op_gemm_e4m3(self, A, sa, B, sb, C, stream=None):
+        import torch
+        M, K = A.shape
+        N = B.shape[0]
+        _check_cuda(A, torch.uint8, (M, K), "A")
+        _check_cuda(B, torch.uint8, (N, K), "B")
+        _check_cuda(sa, torch.float32, (M,), "sa")
+        _check_cuda(sb, torch.float32, (N,), "sb")
+        _check_cuda(C, torch.float32, (M, N), "C")
+        self._chk(self.lib.dm0_op_gemm_e4m3(self.h, _ptr(A), _ptr(sa), _ptr(B), _ptr(sb), _ptr(C), M, N, K,
+                                            _stream(stream)))
+
     def op_attention(self, q, ka, va, kb, vb, o, splits=1, stream=None):
         import torch
         for t, nm in ((q, "q"), (ka, "ka"), (va, "va"), (kb, "kb"), (vb, "vb"), (o, "o")):

@@ -25,7 +25,8 @@ EXPORTS = ("dm0_create", "dm0_weights_bytes", "dm0_load_weights", "dm0_prefill",
            "dm0_kv_commit", "dm0_denoise", "dm0_infer_host", "dm0_merged_layer", "dm0_op_gemm",
            "dm0_op_attention", "dm0_attention_noalloc", "dm0_debug_view", "dm0_launch_count", "dm0_probe",
            "dm0_probe_read", "dm0_selftest_timeout", "dm0_sync", "dm0_device_error", "dm0_clear_error", "dm0_last_error",
-           "dm0_destroy", "dm0_pack_e4m3_rows")
+           "dm0_destroy", "dm0_pack_e4m3_rows", "dm0_set_prefix_fp8", "dm0_op_quant_e4m3",
+           "dm0_op_gemm_e4m3")
 
 
 class Dm0Config(ctypes.Structure):
@@ -78,6 +79,9 @@ def load_library() -> ctypes.CDLL:
         "dm0_last_error": (ctypes.c_char_p, [P]),
         "dm0_destroy": (None, [P]),
         "dm0_pack_e4m3_rows": (c_int, [P, ctypes.c_int64, ctypes.c_int64, P, P]),
+        "dm0_set_prefix_fp8": (c_int, [P, c_int, P]),
+        "dm0_op_quant_e4m3": (c_int, [P, P, c_int, c_int, c_int, P, P, P, P, P]),
+        "dm0_op_gemm_e4m3": (c_int, [P, P, P, P, P, P, c_int, c_int, c_int, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

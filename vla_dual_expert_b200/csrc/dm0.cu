@@ -133,6 +133,17 @@ struct dm0_ctx {
   dm0::PdLayer* players = nullptr;
   unsigned long long* ptrace = nullptr;   // DM0_PERSIST_TRACE=1: phase timestamps of the persistent loop
   int ptrace_steps = 0;
+  // FP8 E4M3 prefix MLP (dm0_set_prefix_fp8): per VLM layer the gate/up (interleaved as the bf16
+  // copy) and down weights as codes with per-output-channel scales, and the per-token operands
+  struct F8Layer {
+    uint8_t *wgu, *wd;
+    float *sgu, *sd;
+  };
+  bool fp8_mlp = false;
+  std::vector<F8Layer> f8;
+  uint8_t *xq_v = nullptr, *aq_v = nullptr;   // [Mp][hidden_v], [Mp][inter_v] codes
+  float *sxq_v = nullptr, *saq_v = nullptr;   // [Mp] scales
+  float* act32_v = nullptr;                   // [Mp][inter_v] SwiGLU output in fp32
 
   cudaStream_t cap_stream = nullptr;
   struct Graph {
@@ -233,6 +244,34 @@ dm0_status get_tmap_plain(dm0_ctx* c, CUtensorMap* out, const void* ptr, int esi
                    const_cast<void*>(ptr), dims, strides, boxd, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(c, DM0_ECUDA, "cuTensorMapEncodeTiled (plain) failed (" + std::to_string(r) + ")");
+  return DM0_OK;
+}
+
+// 2-D map of FP8 codes (one byte each) with 128-byte swizzle: boxes of one 128-byte row (128 codes of K)
+// x box_rows rows, the operand layout of the FP8 GEMM (the same bytes per row as a bf16 k-block)
+dm0_status get_tmap_u8(dm0_ctx* c, CUtensorMap* out, const void* ptr, uint64_t rows, uint64_t cols,
+                       uint32_t box_rows) {
+  const TmapKey key{ptr, rows, cols, box_rows | 0x80000000u};   // kept apart from bf16 maps of the same pointer
+  auto it = c->tmaps.find(key);
+  if (it != c->tmaps.end()) {
+    *out = it->second;
+    return DM0_OK;
+  }
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(c, DM0_ECUDA, "cuTensorMapEncodeTiled is unavailable");
+  if (reinterpret_cast<uintptr_t>(ptr) % 16 != 0 || cols % 128 != 0)
+    return fail(c, DM0_EINVAL, "FP8 TMA operand must be 16-byte aligned with a multiple of 128 columns");
+  CUtensorMap m;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t boxd[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, boxd, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(c, DM0_ECUDA, "cuTensorMapEncodeTiled (u8) failed (" + std::to_string(r) + ")");
+  c->tmaps[key] = m;
+  *out = m;
   return DM0_OK;
 }
 
@@ -346,6 +385,54 @@ dm0_status run_gemm(dm0_ctx* c, cudaStream_t s, const bf16* act, int tokens, int
                   dm0::PGemmSmem<128, 6>::kBytes, ta, tb, g);
   return launch(c, s, dm0::gemm_tc_persistent<64, 8>, grid, dim3(dm0::kGemmThreads), dm0::PGemmSmem<64, 8>::kBytes,
                 ta, tb, g);
+}
+
+// FP8 E4M3 GEMM: act [tokens][K] codes with per-token scales sa, W [wrows][K] codes with per-row scales
+// sw; always the persistent normal-orientation kernel (rows past `tokens` of the last 128-row tile are
+// zero-filled by TMA and their stores predicated off), tile width by the same one-wave rule as bf16
+dm0_status run_gemm_e4m3(dm0_ctx* c, cudaStream_t s, const uint8_t* act, const float* sa, int tokens, int K,
+                         const uint8_t* W, const float* sw, int wrows, GemmArgs g) {
+  if (tokens <= 0) return DM0_OK;
+  if (K % 128 != 0 || wrows % 128 != 0)
+    return fail(c, DM0_ESHAPE, "FP8 GEMM needs K % 128 == 0 and weight rows % 128 == 0");
+  g.K = K;
+  g.tokens = tokens;
+  g.err = c->d_err;
+  g.counters = c->gcount;
+  g.row_scale = sa;
+  g.col_scale = sw;
+  const int mt = (tokens + 127) / 128;
+  int BN = (wrows % 256 == 0) ? 256 : 128;
+  const int min_bn = (g.mode == dm0::kModeResid || g.mode == dm0::kModeStoreF32) ? 64 : 128;
+  while (BN > min_bn && mt * (wrows / BN) < c->num_sms && mt * (wrows / (BN / 2)) <= c->num_sms) BN /= 2;
+  g.M = tokens;
+  g.N = wrows;
+  g.swap = 0;
+  g.kb_per_split = K / 128;
+  CUtensorMap ta, tb;
+  TRY(get_tmap_u8(c, &ta, act, tokens, K, 128));
+  TRY(get_tmap_u8(c, &tb, W, wrows, K, BN));
+  const int ntiles = mt * (wrows / BN);
+  const dim3 grid(std::min(ntiles, c->num_sms));
+  if (BN == 256)
+    return launch(c, s, dm0::gemm_tc_persistent<256, 4, true>, grid, dim3(dm0::kGemmThreads),
+                  dm0::PGemmSmem<256, 4>::kBytes, ta, tb, g);
+  if (BN == 128)
+    return launch(c, s, dm0::gemm_tc_persistent<128, 6, true>, grid, dim3(dm0::kGemmThreads),
+                  dm0::PGemmSmem<128, 6>::kBytes, ta, tb, g);
+  return launch(c, s, dm0::gemm_tc_persistent<64, 8, true>, grid, dim3(dm0::kGemmThreads),
+                dm0::PGemmSmem<64, 8>::kBytes, ta, tb, g);
+}
+
+// per-row E4M3 codes and scales of a matrix [rows][cols] (bf16 or fp32), each row optionally scaled by
+// gain[c] and its pending RMSNorm factor from ssq[row] first
+template <typename T>
+dm0_status quant_rows(dm0_ctx* c, cudaStream_t s, const T* x, int rows, int cols, uint8_t* q, float* scale,
+                      const float* gain = nullptr, const float* ssq = nullptr) {
+  if (rows <= 0) return DM0_OK;
+  if (cols <= 0 || cols % 8 != 0) return fail(c, DM0_ESHAPE, "E4M3 row quantisation needs cols % 8 == 0");
+  return launch(c, s, dm0::quant_rows_e4m3_kernel<T>, dim3(rows), dim3(256), 0, x, rows, cols, gain, ssq,
+                1.0f / cols, c->cfg.rms_eps, q, scale);
 }
 
 // ---------------------------------------------------------------- attention dispatch
@@ -500,6 +587,10 @@ dm0_status layer_rest(dm0_ctx* c, cudaStream_t s, int br, int l, int tokens, flo
   int e0 = probe_begin(c, s, so);
   TRY(run_gemm(c, s, o, tokens, cf.n_q * cf.head_dim, w.wo, H, g));
   probe_end(c, s, so, e0);
+  // FP8 prefix MLP: each GEMM's bf16 operand is quantised per token first (its probe site covers both)
+  const bool f8 = br == 0 && c->fp8_mlp;
+  // FP8: the gate/up operand is the normalised residual rms(h) * g in fp32, quantised per token (the
+  // GEMM's epilogue then has no pending 1/rms to apply), and SwiGLU writes fp32 for the down operand
   GemmArgs u = base_args(c);
   u.w_stable = 1;
   u.mode = dm0::kModeSwiGLU;
@@ -509,7 +600,15 @@ dm0_status layer_rest(dm0_ctx* c, cudaStream_t s, int br, int l, int tokens, flo
   u.inter = I;
   const int su = br == 0 ? DM0_SITE_VLM_GATEUP : DM0_SITE_ACT_GATEUP;
   e0 = probe_begin(c, s, su);
-  TRY(run_gemm(c, s, xn, tokens, H, w.wgu, 2 * I, u));
+  if (f8) {
+    TRY(quant_rows(c, s, static_cast<const float*>(h), tokens, H, c->xq_v, c->sxq_v, w.mlp_norm, ssq_mlp));
+    u.ssq_in = nullptr;
+    u.act = nullptr;
+    u.act_f32 = c->act32_v;
+    TRY(run_gemm_e4m3(c, s, c->xq_v, c->sxq_v, tokens, H, c->f8[l].wgu, c->f8[l].sgu, 2 * I, u));
+  } else {
+    TRY(run_gemm(c, s, xn, tokens, H, w.wgu, 2 * I, u));
+  }
   probe_end(c, s, su, e0);
   GemmArgs d = base_args(c);
   d.w_stable = 1;
@@ -521,7 +620,12 @@ dm0_status layer_rest(dm0_ctx* c, cudaStream_t s, int br, int l, int tokens, flo
   d.ssq_out = next_gain ? next_ssq : nullptr;
   const int sd = br == 0 ? DM0_SITE_VLM_DOWN : DM0_SITE_ACT_DOWN;
   e0 = probe_begin(c, s, sd);
-  TRY(run_gemm(c, s, act, tokens, I, w.wd, H, d));
+  if (f8) {
+    TRY(quant_rows(c, s, static_cast<const float*>(c->act32_v), tokens, I, c->aq_v, c->saq_v));
+    TRY(run_gemm_e4m3(c, s, c->aq_v, c->saq_v, tokens, I, c->f8[l].wd, c->f8[l].sd, H, d));
+  } else {
+    TRY(run_gemm(c, s, act, tokens, I, w.wd, H, d));
+  }
   probe_end(c, s, sd, e0);
   return DM0_OK;
 }
@@ -871,6 +975,44 @@ dm0_status noalloc_setup(int dev, float** base) {
 
 // ====================================================================== C ABI
 
+namespace {
+// FP8 prefix MLP buffers, allocated on first use: per VLM layer the gate/up and down codes and scales,
+// and the per-token operand codes and scales for max_batch * max_prefix tokens
+dm0_status ensure_fp8(dm0_ctx* c) {
+  if (!c->f8.empty()) return DM0_OK;
+  const dm0_config& g = c->cfg;
+  const size_t H = g.hidden_v, I = g.inter_v;
+  const size_t Mp = static_cast<size_t>(g.max_batch) * g.max_prefix;
+  std::vector<dm0_ctx::F8Layer> f8(g.layers);
+  for (auto& w : f8) {
+    TRY(dalloc(c, &w.wgu, 2 * I * H));
+    TRY(dalloc(c, &w.sgu, 2 * I));
+    TRY(dalloc(c, &w.wd, H * I));
+    TRY(dalloc(c, &w.sd, H));
+  }
+  TRY(dalloc(c, &c->xq_v, Mp * H));
+  TRY(dalloc(c, &c->aq_v, Mp * I));
+  TRY(dalloc(c, &c->sxq_v, Mp));
+  TRY(dalloc(c, &c->saq_v, Mp));
+  TRY(dalloc(c, &c->act32_v, Mp * I));
+  c->f8 = std::move(f8);
+  return DM0_OK;
+}
+
+// codes and per-output-channel scales of every VLM layer's gate/up and down weights, from the bf16 copy
+dm0_status pack_fp8_weights(dm0_ctx* c, cudaStream_t s) {
+  const dm0_config& g = c->cfg;
+  const int H = g.hidden_v, I = g.inter_v;
+  c->pdl_ok = false;
+  for (int l = 0; l < g.layers; ++l) {
+    const LayerW& w = c->lw[0][l];
+    TRY(quant_rows(c, s, w.wgu, 2 * I, H, c->f8[l].wgu, c->f8[l].sgu));
+    TRY(quant_rows(c, s, w.wd, H, I, c->f8[l].wd, c->f8[l].sd));
+  }
+  return DM0_OK;
+}
+}  // namespace
+
 extern "C" {
 
 size_t dm0_weights_bytes(const dm0_config* cfg) { return cfg ? blob_bytes(*cfg) : 0; }
@@ -1031,6 +1173,9 @@ dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
             smem_attr(dm0::gemm_tc_persistent<64, 8>, dm0::PGemmSmem<64, 8>::kBytes) &&
             smem_attr(dm0::gemm_tc_persistent<128, 6>, dm0::PGemmSmem<128, 6>::kBytes) &&
             smem_attr(dm0::gemm_tc_persistent<256, 4>, dm0::PGemmSmem<256, 4>::kBytes) &&
+            smem_attr(dm0::gemm_tc_persistent<64, 8, true>, dm0::PGemmSmem<64, 8>::kBytes) &&
+            smem_attr(dm0::gemm_tc_persistent<128, 6, true>, dm0::PGemmSmem<128, 6>::kBytes) &&
+            smem_attr(dm0::gemm_tc_persistent<256, 4, true>, dm0::PGemmSmem<256, 4>::kBytes) &&
             smem_attr(dm0::attn_kernel<128>, dm0::AttnSmem<128>::kBytes) &&
             smem_attr(dm0::attn_kernel<64>, dm0::AttnSmem<64>::kBytes) &&
             smem_attr(dm0::attn_kernel<32>, dm0::AttnSmem<32>::kBytes) &&
@@ -1083,6 +1228,26 @@ dm0_status dm0_load_weights(dm0_ctx* c, const void* blob, size_t bytes) {
   TRY(put(c->W_out, 2 * Ad * Ha));
   TRY(put(c->b_out, 4 * Ad));
   c->weights_loaded = true;
+  if (c->fp8_mlp) {   // keep the FP8 copies in step with the new weights
+    TRY(pack_fp8_weights(c, nullptr));
+    CK(cudaStreamSynchronize(nullptr));
+  }
+  return DM0_OK;
+}
+
+dm0_status dm0_set_prefix_fp8(dm0_ctx* c, int enable, void* stream) {
+  if (!c) return DM0_EINVAL;
+  if (!enable) {
+    c->fp8_mlp = false;
+    return DM0_OK;
+  }
+  if (!c->weights_loaded) return fail(c, DM0_ESTATE, "load the weights before enabling the FP8 prefix MLP");
+  const dm0_config& g = c->cfg;
+  if (g.hidden_v % 128 != 0 || g.inter_v % 128 != 0)
+    return fail(c, DM0_ESHAPE, "the FP8 prefix MLP needs hidden_v and inter_v multiples of 128");
+  TRY(ensure_fp8(c));
+  TRY(pack_fp8_weights(c, static_cast<cudaStream_t>(stream)));
+  c->fp8_mlp = true;
   return DM0_OK;
 }
 
@@ -1192,6 +1357,34 @@ dm0_status dm0_op_gemm(dm0_ctx* c, const void* A, const void* B, float* C, int M
   if (N % 128 != 0 || splits != 1) return fail(c, DM0_ESHAPE, "GEMM needs N % 128 == 0 and splits == 1");
   g.out_f32 = C;
   return run_gemm(c, s, static_cast<const bf16*>(A), M, K, static_cast<const bf16*>(B), N, g, 0, 1);
+}
+
+dm0_status dm0_op_quant_e4m3(dm0_ctx* c, const void* x, int x_f32, int rows, int cols, const float* gain,
+                             const float* ssq, void* codes, float* scales, void* stream) {
+  if (!c || !x || !codes || !scales) return fail(c, DM0_EINVAL, "null argument");
+  if (rows < 1 || cols < 8 || cols % 8 != 0) return fail(c, DM0_ESHAPE, "quantisation needs rows >= 1, cols % 8 == 0");
+  if (reinterpret_cast<uintptr_t>(x) % 16 != 0 || reinterpret_cast<uintptr_t>(codes) % 8 != 0 ||
+      (gain && reinterpret_cast<uintptr_t>(gain) % 16 != 0))
+    return fail(c, DM0_EINVAL, "x and gain must be 16-byte and codes 8-byte aligned");
+  c->pdl_ok = false;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* q = static_cast<uint8_t*>(codes);
+  if (x_f32) return quant_rows(c, s, static_cast<const float*>(x), rows, cols, q, scales, gain, ssq);
+  return quant_rows(c, s, static_cast<const bf16*>(x), rows, cols, q, scales, gain, ssq);
+}
+
+dm0_status dm0_op_gemm_e4m3(dm0_ctx* c, const void* A, const float* sa, const void* B, const float* sb, float* C,
+                            int M, int N, int K, void* stream) {
+  if (!c || !A || !sa || !B || !sb || !C) return fail(c, DM0_EINVAL, "null argument");
+  if (M < 1 || N < 128 || N % 128 != 0 || K < 128 || K % 128 != 0)
+    return fail(c, DM0_ESHAPE, "FP8 GEMM needs M >= 1, N % 128 == 0, K % 128 == 0");
+  if (reinterpret_cast<uintptr_t>(sb) % 16 != 0) return fail(c, DM0_EINVAL, "sb must be 16-byte aligned");
+  c->pdl_ok = false;
+  GemmArgs g = base_args(c);
+  g.mode = dm0::kModeStoreF32;
+  g.out_f32 = C;
+  return run_gemm_e4m3(c, static_cast<cudaStream_t>(stream), static_cast<const uint8_t*>(A), sa, M, K,
+                       static_cast<const uint8_t*>(B), sb, N, g);
 }
 
 dm0_status dm0_op_attention(dm0_ctx* c, const void* q, const void* ka, const void* va, int Ta, const void* kb,

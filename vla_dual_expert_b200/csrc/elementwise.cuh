@@ -8,6 +8,8 @@
 //                  e = x W_in^T + b_in + tau(t) with t = 1 - k/K.
 //   rope_table   : (cos, sin) of position * theta^(-2i/D), in double precision.
 #pragma once
+#include <cuda_fp8.h>
+
 #include "ptx.cuh"
 
 namespace dm0 {
@@ -172,6 +174,88 @@ __global__ void wait_timeout_selftest_kernel(int* err, unsigned long long limit_
     mbar_init(&bar, 1);
     fence_mbar_init();
     if (!mbar_wait(&bar, 0, nullptr, limit_ns)) raise_error(err, kErrTimeoutProducer);
+  }
+}
+
+// FP8 E4M3 row quantisation (the operands of the FP8 prefix-MLP GEMMs; DM0.5 page, section 6.3, with
+// per-row scales).  Row r of x (bf16 or fp32), optionally times gain[c] and the row's pending RMSNorm
+// factor 1/sqrt(ssq[r] / cols + eps), is y[c]; scale[r] = amax(|y|) / 448 in fp32 (1 for an all-zero
+// row) and q[r][c] = E4M3(y[c] / scale[r]), the quotient an IEEE fp32 division and the conversion
+// round to nearest even, saturating.  One CTA of 256 threads per row, 16-byte loads (8 bf16 or 4
+// fp32), cols a multiple of 8; the row is read twice, the second time from L1 / L2.  Used for the
+// weights once (bf16 rows = output channels) and for the activations (fp32 rows = tokens).
+template <typename T>
+__device__ __forceinline__ void quant_load(const T* row, const float* gain, float rn, int v, float (&y)[16 / sizeof(T)]) {
+  constexpr int kV = 16 / sizeof(T);
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(row) + v);
+  if constexpr (sizeof(T) == 2) {
+    const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(b[i]);
+      y[2 * i] = f.x;
+      y[2 * i + 1] = f.y;
+    }
+  } else {
+    y[0] = __uint_as_float(u.x);
+    y[1] = __uint_as_float(u.y);
+    y[2] = __uint_as_float(u.z);
+    y[3] = __uint_as_float(u.w);
+  }
+  if (gain) {
+#pragma unroll
+    for (int i = 0; i < kV; ++i) y[i] = y[i] * rn * __ldg(gain + v * kV + i);
+  } else if (rn != 1.f) {
+#pragma unroll
+    for (int i = 0; i < kV; ++i) y[i] *= rn;
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) quant_rows_e4m3_kernel(const T* x, int rows, int cols, const float* gain,
+                                                              const float* ssq, float inv_cols, float eps,
+                                                              uint8_t* q, float* scale) {
+  constexpr int kV = 16 / sizeof(T);
+  __shared__ float red[8];
+  pdl_launch_dependents();
+  pdl_wait();
+  const int row = blockIdx.x;
+  if (row >= rows) return;
+  const T* src = x + static_cast<size_t>(row) * cols;
+  const float rn = ssq ? rsqrtf(__ldcg(ssq + row) * inv_cols + eps) : 1.f;
+  const int nvec = cols / kV;
+  float amax = 0.f;
+  for (int v = threadIdx.x; v < nvec; v += 256) {
+    float y[kV];
+    quant_load(src, gain, rn, v, y);
+#pragma unroll
+    for (int i = 0; i < kV; ++i) amax = fmaxf(amax, fabsf(y[i]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = red[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) amax = fmaxf(amax, red[w]);
+  const float s = amax > 0.f ? amax / 448.f : 1.f;
+  if (threadIdx.x == 0) scale[row] = s;
+  uint8_t* dst = q + static_cast<size_t>(row) * cols;
+  for (int v = threadIdx.x; v < nvec; v += 256) {
+    float y[kV];
+    quant_load(src, gain, rn, v, y);
+    uint32_t w[kV / 4];
+#pragma unroll
+    for (int i = 0; i < kV / 4; ++i) {
+      w[i] = 0u;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        w[i] |= static_cast<uint32_t>(__nv_cvt_float_to_fp8(y[4 * i + j] / s, __NV_SATFINITE, __NV_E4M3)) << (8 * j);
+    }
+    if constexpr (kV == 8)
+      reinterpret_cast<uint2*>(dst)[v] = make_uint2(w[0], w[1]);
+    else
+      reinterpret_cast<uint32_t*>(dst)[v] = w[0];
   }
 }
 

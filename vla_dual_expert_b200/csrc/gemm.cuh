@@ -65,8 +65,13 @@ struct GemmArgs {
   // kModeSwiGLU
   __nv_bfloat16* act; // [tokens][inter]
   int inter;
+  float* act_f32;     // [tokens][inter] fp32 instead of act when not null (the FP8 MLP's down operand)
   // kModeStoreF32
   float* out_f32;     // normal: [M][N]
+  // FP8 E4M3 operands (persistent normal-orientation GEMM only): the accumulator of (token, feature)
+  // is multiplied by row_scale[token] * col_scale[feature] before the mode's epilogue
+  const float* row_scale;   // [M] per-token activation scale
+  const float* col_scale;   // [N] per-output-channel weight scale
 };
 
 constexpr int kGemmThreads = 192;
@@ -176,7 +181,13 @@ __device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool va
       load(c + 2, u);
 #pragma unroll
       for (int j = 0; j < 32; ++j) g[j] = silu_f(g[j] * s) * (u[j] * s);
-      if (valid) st_bf16x32(a.act + static_cast<size_t>(tok) * a.inter + col0 / 2 + 32 * c, g);
+      if (valid) {
+        const size_t off = static_cast<size_t>(tok) * a.inter + col0 / 2 + 32 * c;
+        if (a.act_f32)
+          st_f32x32(a.act_f32 + off, g);
+        else
+          st_bf16x32(a.act + off, g);
+      }
     }
     return;
   }
@@ -495,11 +506,15 @@ struct PGemmSmem {
   static constexpr uint32_t kTmemCols = 2 * BN;
 };
 
-template <int BN, int STAGES>
+// kF8: both operands FP8 E4M3 (tensor maps of bytes), a k-block is 128 values instead of 64 (the
+// same 128-byte rows, so the ring, the swizzle and the descriptors are unchanged), and the epilogue
+// applies the per-token and per-output-channel scales.
+template <int BN, int STAGES, bool kF8 = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const GemmArgs a) {
   using L = PGemmSmem<BN, STAGES>;
+  constexpr int kKB = kF8 ? 128 : 64;   // operand values per 128-byte k-block row
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kPipe);
@@ -511,7 +526,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int KB = (a.K + 63) >> 6;
+  const int KB = (a.K + kKB - 1) / kKB;
   const int mt = (a.M + 127) >> 7;
   const int ntiles = mt * (a.N / BN);
 
@@ -555,7 +570,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         band_tile(first, mt, a.N / BN, m_first, n0);
         for (int k = 0; k < pre; ++k) {
           mbar_arrive_expect_tx(&full[k], L::kStage);
-          tma_load_2d(smem + k * L::kStage + L::kA, &tmB, &full[k], k * 64, n0 * BN, pol_w);
+          tma_load_2d(smem + k * L::kStage + L::kA, &tmB, &full[k], k * kKB, n0 * BN, pol_w);
         }
       }
       pdl_wait();
@@ -568,7 +583,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int k = 0; k < KB; ++k, ++it) {
           const int s = it % STAGES;
           if (it < pre) {   // weight half already requested
-            tma_load_2d(smem + s * L::kStage, &tmA, &full[s], k * 64, m0, pol_x);
+            tma_load_2d(smem + s * L::kStage, &tmA, &full[s], k * kKB, m0, pol_x);
             continue;
           }
           if (it >= STAGES && !mbar_wait(&empty[s], ((it / STAGES) - 1) & 1, abort_flag)) {
@@ -577,8 +592,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(&full[s], L::kStage);
-          tma_load_2d(smem + s * L::kStage, &tmA, &full[s], k * 64, m0, pol_x);
-          tma_load_2d(smem + s * L::kStage + L::kA, &tmB, &full[s], k * 64, n0, pol_w);
+          tma_load_2d(smem + s * L::kStage, &tmA, &full[s], k * kKB, m0, pol_x);
+          tma_load_2d(smem + s * L::kStage + L::kA, &tmB, &full[s], k * kKB, n0, pol_w);
         }
       }
       for (int i = it - STAGES; i < it; ++i) {   // copies in flight land before the CTA exits
@@ -588,7 +603,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(128, BN);
+      const uint32_t idesc = kF8 ? idesc_e4m3_f32(128, BN) : idesc_bf16_f32(128, BN);
       int it = 0, local = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x, ++local) {
@@ -608,9 +623,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t a_addr = smem_u32(smem + s * L::kStage);
           const uint32_t b_addr = a_addr + L::kA;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_bf16(tmem + buf * BN, sw128_kmajor_desc(a_addr + 32 * kk), sw128_kmajor_desc(b_addr + 32 * kk),
-                      idesc, (k | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {
+            if constexpr (kF8)
+              umma_e4m3(tmem + buf * BN, sw128_kmajor_desc(a_addr + 32 * kk), sw128_kmajor_desc(b_addr + 32 * kk),
+                        idesc, (k | kk) != 0 ? 1u : 0u);
+            else
+              umma_bf16(tmem + buf * BN, sw128_kmajor_desc(a_addr + 32 * kk), sw128_kmajor_desc(b_addr + 32 * kk),
+                        idesc, (k | kk) != 0 ? 1u : 0u);
+          }
           umma_commit(&empty[s]);
         }
         if (ok) umma_commit(&tfull[buf]);
@@ -640,15 +660,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int tok = m_tile * 128 + lane_base + lane;
       const bool valid = tok < a.M;
       float ssq_acc = 0.f;
+      // FP8: the token's activation scale (0 for rows past M, whose stores are predicated off anyway)
+      const float rs = kF8 && valid ? __ldg(a.row_scale + tok) : 0.f;
+      auto scaled = [&](uint32_t taddr, int col, float (&v)[32]) {
+        tmem_ld32(taddr, v);
+        if constexpr (kF8) {
+          const float4* cs4 = reinterpret_cast<const float4*>(a.col_scale + col);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 cs = __ldg(cs4 + i);
+            v[4 * i] *= rs * cs.x;
+            v[4 * i + 1] *= rs * cs.y;
+            v[4 * i + 2] *= rs * cs.z;
+            v[4 * i + 3] *= rs * cs.w;
+          }
+        }
+      };
       if (BN >= 128) {
         for (int g = 0; g < BN / 128; ++g) {
           const uint32_t tg = tl + g * 128;
-          row_epilogue<false>(a, tok, valid, n_tile * BN + g * 128, ssq_acc,
-                              [&](int c, float (&v)[32]) { tmem_ld32(tg + c * 32, v); });
+          const int col0 = n_tile * BN + g * 128;
+          row_epilogue<false>(a, tok, valid, col0, ssq_acc,
+                              [&](int c, float (&v)[32]) { scaled(tg + c * 32, col0 + 32 * c, v); });
         }
       } else {
-        row_epilogue<false>(a, tok, valid, n_tile * BN, ssq_acc,
-                            [&](int c, float (&v)[32]) { tmem_ld32(tl + c * 32, v); }, BN / 32);
+        const int col0 = n_tile * BN;
+        row_epilogue<false>(a, tok, valid, col0, ssq_acc,
+                            [&](int c, float (&v)[32]) { scaled(tl + c * 32, col0 + 32 * c, v); }, BN / 32);
       }
       if (a.mode == kModeResid && a.ssq_out && valid) atomicAdd(a.ssq_out + tok, ssq_acc);
       // the accumulator buffer is free for tile local + 2
