@@ -15,7 +15,8 @@ quantiser's precision (quantize_rows_f32: fp32 scale and fp32 quotient).  Tolera
                                          one such flip moves a whole output column by a step of 2^-3
                                          relative (emulated on the CPU with 3-ulp noise on the operands:
                                          max 0.024, RMS 8e-4, 0.2 % of the elements beyond 1e-2 RMS)
-The kernels in this file have not yet run on a GPU; DM0_RUN_FP8=1 selects them.
+The quantiser and GEMM tests have run on a B200; the layer-level tests (marked `pending`) run only
+with DM0_RUN_FP8=1 until their first GPU run.
 """
 import os
 
@@ -27,9 +28,9 @@ from oracle import dm0_oracle as O
 from synth import inputs as I
 from tests.gpu_util import check_bf16, check_fp, host, rel_err, rms, to_dev_bf16, to_dev_f32
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skipif(os.environ.get("DM0_RUN_FP8") != "1",
-                                 reason="FP8 kernels await their first GPU run (DM0_RUN_FP8=1)")]
+pytestmark = pytest.mark.gpu
+pending = pytest.mark.skipif(os.environ.get("DM0_RUN_FP8") != "1",
+                             reason="awaits its first GPU run (DM0_RUN_FP8=1)")
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -142,6 +143,7 @@ def _fp8_stats(got, ref, what):
     return out
 
 
+@pending
 @pytest.mark.parametrize("B,P", [(1, 816), (2, 333)])
 def test_merged_layer_fp8(eng1, B, P):
     d, w, eng = eng1
@@ -189,8 +191,10 @@ def test_fp8_toggle_leaves_the_bf16_path_unchanged(eng1):
     fp8 = run()
     eng.set_prefix_fp8(False)
     after = run()
-    assert np.array_equal(before, after)
-    assert not np.array_equal(before, fp8)
+    # the bf16 layer is not bitwise repeatable (the residual epilogue's sums of squares are atomic
+    # fp32 adds in any order), so "unchanged" means equal to fp32 rounding of those sums
+    assert rel_err(after, before) <= 1e-5
+    assert rel_err(fp8, before) > 1e-3
 
 
 def test_enable_before_weights_is_a_state_error():
@@ -205,6 +209,7 @@ def test_enable_before_weights_is_a_state_error():
 
 # ------------------------------------------------------------------ a whole prefix pass (tiny model)
 
+@pending
 def test_tiny_prefill_fp8(eng1):
     from vla_dual_expert_b200 import Engine
     d = I.TINY
