@@ -312,6 +312,23 @@ def run_native(args, rank, world, local_rank):
                                  "traffic_per_euler_step": LOOP_TRAFFIC_BYTES_PER_STEP,
                                  "peak_src": f"{peaks['src']} hbm_gbs"},
         }
+    if args.prefix_fp8:
+        # the same step with the VLM MLP's GEMMs in FP8 E4M3 (opt-in; the headline stays bf16): the
+        # probed gate/up site covers the operand quantisation and the FP8 GEMM
+        eng.set_prefix_fp8(True)
+        f8 = measure(wl_main, args.steps, args.warmup, probe=3)
+        eng.set_prefix_fp8(False)
+        f8_ms = f8["probe_ms"] / max(f8["probe_n"], 1)
+        f8_tf = prefill_gateup_flops(d, B, P) / (f8_ms * 1e-3) / 1e12
+        fp8_peak = 2.0 * tc_peak
+        result["prefix_fp8"] = {
+            "value": round(job_chunks_per_s(world, B, f8["ms"]), 3), "unit": "chunks/s",
+            "ms_per_step": round(f8["ms"], 3), "prefill_ms_p50": round(f8["prefill_ms_p50"], 3),
+            "gateup_site": {"kernels": "quant_rows_e4m3_kernel<float> + gemm_tc_persistent<256,4,true>",
+                            "avg_ms": round(f8_ms, 4), "achieved": round(f8_tf, 1), "peak": round(fp8_peak, 1),
+                            "unit": "TFLOP/s", "frac": round(f8_tf / fp8_peak, 4),
+                            "peak_src": f"{peaks['src']} bf16_tflops_sustained x 2 (nominal fp8 / bf16 ratio)"},
+            "gpu_launches": f8["launches"], "clocks": f8["clocks"]}
     if not args.skip_breakdown:
         result["breakdown_ms_per_step"] = breakdown(eng, wl_main)
         if "batch1" in result:
@@ -466,6 +483,8 @@ def main():
     ap.add_argument("--one-layer", action="store_true", help="profiling workload: one layer, B=16, P=2048")
     ap.add_argument("--b1-loop", action="store_true", help="profiling workload: persistent Euler loop, 3 layers, B=1")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--prefix-fp8", action="store_true",
+                    help="also time the step with the VLM MLP in FP8 E4M3 (reported under prefix_fp8)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "native":
         args.warmup = 3
