@@ -52,7 +52,7 @@ typedef struct dm0_ctx dm0_ctx;
  *   hidden_v, hidden_a, inter_v, inter_a, n_q*head_dim multiples of 128
  *   (tensor-core tile rows), 2*inter multiples of 128;
  *   action_dim <= 64; chunk >= 1; max_batch >= 1; max_prefix >= 1;
- *   max_prefix + chunk <= 65536. */
+ *   max_prefix + chunk <= 65536; time_mod in {0, 1}. */
 typedef struct {
   int layers;       /* decoder layers per branch (28 for DM0-base) */
   int hidden_v;     /* VLM hidden size (2048) */
@@ -68,6 +68,15 @@ typedef struct {
   int max_prefix;   /* largest P any call will use */
   float rope_theta; /* 1e6 */
   float rms_eps;    /* 1e-6 */
+  int time_mod;     /* 0: DM0 action expert (time embedding added to the input);
+                       1: DM0.5 time-modulated action expert (DM0.5 page, section 5.2):
+                       a time MLP turns tau(t) into a condition c, and every
+                       action-expert RMSNorm (attention, MLP, final) becomes
+                       x / rms(x) * (1 + scale) + shift with [scale | shift | gate] =
+                       W_m silu(c) + b_m, the gate scaling the sublayer's residual
+                       add; the static gains of those norms are unused.  The blob
+                       gains the time tensors (see dm0_load_weights); the Euler loop
+                       runs as per-layer kernels. */
 } dm0_config;
 
 typedef enum {
@@ -100,6 +109,11 @@ size_t dm0_weights_bytes(const dm0_config* cfg);
  *     Wd bf16[H][I]
  *   then W_in bf16[Ha][A] | b_in f32[Ha] | final_norm f32[Ha] |
  *        W_out bf16[A][Ha] | b_out f32[A]
+ *   and, when time_mod = 1: W_ti bf16[Ha][Ha] | b_ti f32[Ha] | W_to bf16[Ha][Ha] |
+ *        b_to f32[Ha] | W_mf bf16[2Ha][Ha] | b_mf f32[2Ha] (time_mlp_in, time_mlp_out,
+ *        the final norm's [scale | shift] modulator), then for l in 0..layers-1:
+ *        W_ma bf16[3Ha][Ha] | b_ma f32[3Ha] | W_mm bf16[3Ha][Ha] | b_mm f32[3Ha]
+ *        (the attention and MLP pre-norms' [scale | shift | gate] modulators)
  * Matrices are [out][in].  `bytes` must equal dm0_weights_bytes(). */
 dm0_status dm0_load_weights(dm0_ctx* ctx, const void* blob, size_t bytes);
 
@@ -137,6 +151,12 @@ dm0_status dm0_kv_commit(dm0_ctx* ctx, int B, int P);
  * velocities are requested).  No host work happens inside the loop.  The
  * persistent loop's split-K sums arrive in any order, so repeated calls are
  * not bitwise identical.
+ * With time_mod = 1 each call first builds, for its K steps, every norm's
+ * [1 + scale | shift | gate] from the time MLP and the modulators, and the two
+ * shifts of each layer projected through its QKV and gate/up weights (one pass
+ * over those weights per call); the layers then run the per-layer kernels with
+ * the per-step gains, a feature bias after the pending 1/rms and a gate on each
+ * residual add (the persistent loop covers the DM0 expert only).
  * Returns DM0_ESTATE without a cache, DM0_ESHAPE unless 1 <= steps <= 1000. */
 dm0_status dm0_denoise(dm0_ctx* ctx, const float* noise, int steps, float* actions, float* velocities,
                        void* stream);
@@ -157,7 +177,8 @@ dm0_status dm0_infer_host(dm0_ctx* ctx, const void* prefix_emb, const float* noi
  *   k_out/v_out: device bf16 [B][n_kv][P][head_dim], the prefix K (after
  *   QK-norm + RoPE) and V of this layer.
  * Prefix rows attend to prefix keys only; suffix rows to all P + chunk keys.
- * Uses the context's buffers; overwrites the KV cache slot of `layer`. */
+ * Uses the context's buffers; overwrites the KV cache slot of `layer`.  The
+ * layer has no flow time, so a time_mod context returns DM0_EINVAL. */
 dm0_status dm0_merged_layer(dm0_ctx* ctx, int layer, const float* h_prefix, const float* h_suffix, int B, int P,
                             float* out_prefix, float* out_suffix, void* k_out, void* v_out, void* stream);
 

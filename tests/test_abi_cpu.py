@@ -44,6 +44,33 @@ def test_blob_size_matches_packer():
     assert blob.nbytes == lib.dm0_weights_bytes(ctypes.byref(cfg))
 
 
+@pytest.mark.parametrize("dims", [I.TINY, I.DM0_BASE.replace(layers=2)])
+def test_time_modulated_blob_size_matches_packer(dims):
+    abi, lib = _lib()
+    cfg = abi.make_config(dims, 1, 64, time_mod=True)
+    w = I.Weights(dims, seed=0)
+    blob = abi.pack_weights(w, dims.layers, time_mod=True)
+    assert blob.nbytes == lib.dm0_weights_bytes(ctypes.byref(cfg))
+    plain = lib.dm0_weights_bytes(ctypes.byref(abi.make_config(dims, 1, 64)))
+    Ha, L = dims.hidden_a, dims.layers
+    # time MLP 2 x [Ha][Ha] bf16 + 2 biases, final modulator [2Ha][Ha] + bias, 2 x [3Ha][Ha] + biases per layer
+    assert blob.nbytes - plain == 2 * (2 * Ha * Ha + 2 * Ha * Ha) + 4 * (4 * Ha) + L * (2 * 6 * Ha * Ha + 4 * 6 * Ha)
+
+
+def test_time_modulated_blob_tail_layout():
+    abi, _ = _lib()
+    d = I.TINY
+    w = I.Weights(d, seed=5)
+    blob = abi.pack_weights(w, d.layers, time_mod=True)
+    plain = abi.pack_weights(w, d.layers)
+    assert np.array_equal(blob[:plain.nbytes], plain)
+    Ha = d.hidden_a
+    wti = (blob[plain.nbytes:plain.nbytes + 2 * Ha * Ha].view(np.uint16).astype(np.uint32) << 16).view(np.float32)
+    np.testing.assert_array_equal(wti.reshape(Ha, Ha), w.time()["W_ti"])
+    # the last tensor is the last layer's b_mm
+    np.testing.assert_array_equal(blob[-4 * 3 * Ha:].view(np.float32), w.mod(d.layers - 1)["b_mm"])
+
+
 def test_blob_layout_first_tensors():
     abi, _ = _lib()
     d = I.TINY
@@ -58,7 +85,7 @@ def test_blob_layout_first_tensors():
 
 
 @pytest.mark.parametrize("field,value", [("head_dim", 96), ("n_kv", 3), ("hidden_v", 200), ("action_dim", 0),
-                                         ("max_batch", 0), ("inter_a", 100)])
+                                         ("max_batch", 0), ("inter_a", 100), ("time_mod", 2)])
 def test_create_rejects_bad_config_on_host(field, value):
     abi, lib = _lib()
     d = I.TINY

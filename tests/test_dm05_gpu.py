@@ -1,0 +1,119 @@
+"""Parity of the time-modulated action expert (DM0.5 page, section 5.2; reading R12) on the GPU with the
+oracle in oracle/dm05_oracle.py.
+
+The modulation tables (every step's scale, shift and gate, and the shifts projected through the QKV
+and gate/up weights) are built once per Euler loop from bf16 operands, and the layers then run the
+DM0 kernels with a feature bias, a gate and per-step gains, so the DM0 tolerances apply: the final
+chunk within 2e-2 of RMS and each step's velocity within 2e-2 of RMS(v) (max), against the oracle's
+fp64 definition.  These tests await their first GPU run (DM0_RUN_DM05=1 selects them).
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import dm0_oracle as O
+from oracle import dm05_oracle as M
+from synth import inputs as I
+from tests.gpu_util import check_fp, host, to_dev_bf16
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(os.environ.get("DM0_RUN_DM05") != "1",
+                                 reason="awaits its first GPU run (DM0_RUN_DM05=1)")]
+
+TOL_CHUNK = 2e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from vla_dual_expert_b200 import build
+    build.build()
+
+
+def _engine(d, B, P, w):
+    from vla_dual_expert_b200 import Engine
+    eng = Engine(d, B, P, time_mod=True)
+    eng.load_from(w)
+    return eng
+
+
+def _check(got_x, got_v, ref_x, ref_v, what):
+    check_fp(got_x, ref_x, TOL_CHUNK, f"{what}: chunk")
+    for k, (gv, rv) in enumerate(zip(got_v, ref_v)):
+        check_fp(gv, rv, TOL_CHUNK, f"{what}: velocity of step {k}")
+
+
+@pytest.mark.parametrize("B,P,steps", [(1, 64, 4), (2, 37, 3)])
+def test_tiny_time_modulated_prefill_and_denoise(B, P, steps):
+    d = I.TINY
+    w = I.Weights(d, seed=0, gain_jitter=0.1)
+    emb, noise = I.prefix_embeddings(d, B, P), I.noise(d, B)
+    eng = _engine(d, B, P, w)
+    try:
+        eng.prefill(to_dev_bf16(emb))
+        vel = torch.empty((steps, B, d.chunk, d.action_dim), device="cuda", dtype=torch.float32)
+        out = eng.denoise(torch.from_numpy(noise).cuda(), steps, velocities=vel)
+        eng.sync()
+        assert eng.device_error() == 0
+        x, v = host(out), host(vel)
+    finally:
+        eng.close()
+    for b in range(B):
+        ks, vs, _ = O.prefill(w, emb[b])
+        rx, rv = M.denoise(w, ks, vs, noise[b], steps)
+        _check(x[b], [v[k, b] for k in range(steps)], rx, rv, f"tiny b={b}")
+
+
+def test_full_width_two_layers_over_a_random_cache():
+    """DM0-base widths (head_dim 128), 2 layers, a random 100-token prefix cache, B = 2, 3 steps,
+    through the CUDA graph (no velocities requested) and directly (velocities requested)."""
+    d = I.DM0_BASE.replace(layers=2)
+    w = I.Weights(d, seed=0, gain_jitter=0.1)
+    B, P, steps = 2, 100, 3
+    eng = _engine(d, B, P, w)
+    try:
+        kp, vp = eng.kv_view()
+        from tests.gpu_util import device_view_bf16
+        K = device_view_bf16(kp, (d.layers, B, d.n_kv, P, d.head_dim))
+        V = device_view_bf16(vp, (d.layers, B, d.n_kv, P, d.head_dim))
+        caches = [([], []) for _ in range(B)]
+        for l in range(d.layers):
+            k, v = I.random_kv_layer(d, B, P, l)
+            K[l].copy_(to_dev_bf16(k))
+            V[l].copy_(to_dev_bf16(v))
+            for b in range(B):
+                caches[b][0].append(k[b].astype(np.float64))
+                caches[b][1].append(v[b].astype(np.float64))
+        eng.kv_commit(B, P)
+        noise = I.noise(d, B)
+        x_graph = host(eng.denoise(torch.from_numpy(noise).cuda(), steps))
+        vel = torch.empty((steps, B, d.chunk, d.action_dim), device="cuda", dtype=torch.float32)
+        x_direct = host(eng.denoise(torch.from_numpy(noise).cuda(), steps, velocities=vel))
+        eng.sync()
+        assert eng.device_error() == 0
+        v = host(vel)
+    finally:
+        eng.close()
+    for b in range(B):
+        rx, rv = M.denoise(w, caches[b][0], caches[b][1], noise[b], steps)
+        _check(x_direct[b], [v[k, b] for k in range(steps)], rx, rv, f"base b={b}")
+        check_fp(x_graph[b], rx, TOL_CHUNK, f"base b={b}: chunk through the graph")
+
+
+def test_zero_velocity_head_keeps_noise():
+    """W_out = 0 and b_out = 0: every velocity is exactly 0 whatever the modulation, so x_0 = noise."""
+    d = I.TINY
+    w = I.Weights(d, seed=0)
+    w.overrides[("head", "W_out")] = np.zeros((d.action_dim, d.hidden_a), np.float32)
+    w.overrides[("head", "b_out")] = np.zeros(d.action_dim, np.float32)
+    eng = _engine(d, 1, 64, w)
+    try:
+        eng.prefill(to_dev_bf16(I.prefix_embeddings(d, 1, 64)))
+        noise = I.noise(d, 1)
+        x = host(eng.denoise(torch.from_numpy(noise).cuda(), 5))
+        eng.sync()
+    finally:
+        eng.close()
+    assert np.array_equal(x, noise.astype(np.float64))

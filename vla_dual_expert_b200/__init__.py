@@ -56,10 +56,12 @@ def pack_e4m3_rows(x: np.ndarray):
 class Engine:
     """One dm0_ctx on the current CUDA device."""
 
-    def __init__(self, dims, max_batch: int, max_prefix: int):
+    def __init__(self, dims, max_batch: int, max_prefix: int, time_mod: bool = False):
+        """time_mod: the time-modulated action expert (DM0.5 page, section 5.2) instead of the DM0 one."""
         self.lib = load_library()
         self.dims = dims
-        self.cfg = make_config(dims, max_batch, max_prefix)
+        self.time_mod = bool(time_mod)
+        self.cfg = make_config(dims, max_batch, max_prefix, self.time_mod)
         h = ctypes.c_void_p()
         st = self.lib.dm0_create(ctypes.byref(self.cfg), ctypes.byref(h))
         if st != 0 or not h.value:
@@ -91,7 +93,7 @@ class Engine:
         self._chk(self.lib.dm0_load_weights(self.h, blob.ctypes.data_as(ctypes.c_void_p), blob.nbytes))
 
     def load_from(self, provider):
-        self.load_weights(pack_weights(provider, self.dims.layers))
+        self.load_weights(pack_weights(provider, self.dims.layers, self.time_mod))
 
     def prefill(self, prefix_emb, stream=None):
         import torch

@@ -33,7 +33,7 @@ class Dm0Config(ctypes.Structure):
     _fields_ = [("layers", c_int), ("hidden_v", c_int), ("inter_v", c_int), ("hidden_a", c_int),
                 ("inter_a", c_int), ("n_q", c_int), ("n_kv", c_int), ("head_dim", c_int),
                 ("chunk", c_int), ("action_dim", c_int), ("max_batch", c_int), ("max_prefix", c_int),
-                ("rope_theta", c_float), ("rms_eps", c_float)]
+                ("rope_theta", c_float), ("rms_eps", c_float), ("time_mod", c_int)]
 
 
 class Dm0Error(RuntimeError):
@@ -91,11 +91,12 @@ def load_library() -> ctypes.CDLL:
     return lib
 
 
-def make_config(dims, max_batch: int, max_prefix: int) -> Dm0Config:
-    """dims: any object with the model-shape attributes (layers, hidden_v, ...)."""
+def make_config(dims, max_batch: int, max_prefix: int, time_mod: bool = False) -> Dm0Config:
+    """dims: any object with the model-shape attributes (layers, hidden_v, ...); time_mod selects the
+    time-modulated action expert."""
     return Dm0Config(dims.layers, dims.hidden_v, dims.inter_v, dims.hidden_a, dims.inter_a, dims.n_q,
                      dims.n_kv, dims.head_dim, dims.chunk, dims.action_dim, max_batch, max_prefix,
-                     float(dims.rope_theta), float(dims.rms_eps))
+                     float(dims.rope_theta), float(dims.rms_eps), 1 if time_mod else 0)
 
 
 def _bf16_bits(a: np.ndarray) -> np.ndarray:
@@ -112,13 +113,19 @@ LAYER_ORDER = (("attn_norm", "f32"), ("Wq", "bf16"), ("Wk", "bf16"), ("Wv", "bf1
                ("k_norm", "f32"), ("Wo", "bf16"), ("mlp_norm", "f32"), ("Wg", "bf16"), ("Wu", "bf16"),
                ("Wd", "bf16"))
 HEAD_ORDER = (("W_in", "bf16"), ("b_in", "f32"), ("final_norm", "f32"), ("W_out", "bf16"), ("b_out", "f32"))
+# time-modulated action expert: after the head, the time MLP and final modulator, then per layer the two
+# pre-norm modulators
+TIME_ORDER = (("W_ti", "bf16"), ("b_ti", "f32"), ("W_to", "bf16"), ("b_to", "f32"), ("W_mf", "bf16"),
+              ("b_mf", "f32"))
+MOD_ORDER = (("W_ma", "bf16"), ("b_ma", "f32"), ("W_mm", "bf16"), ("b_mm", "f32"))
 
 
-def pack_weights(provider, layers: int) -> np.ndarray:
+def pack_weights(provider, layers: int, time_mod: bool = False) -> np.ndarray:
     """Serialise parameters into the blob layout dm0_load_weights reads.
 
     provider.layer(branch, l) -> dict and provider.head() -> dict of fp32 arrays
-    (matrices [out][in]); branch 0 = VLM, 1 = action expert.
+    (matrices [out][in]); branch 0 = VLM, 1 = action expert.  With time_mod, provider.time() and
+    provider.mod(l) give the time MLP / final modulator and layer l's modulators.
     """
     def nbytes(arr, kind):
         return arr.size * (2 if kind == "bf16" else 4)
@@ -130,6 +137,12 @@ def pack_weights(provider, layers: int) -> np.ndarray:
             tensors += [(w[n], k) for n, k in LAYER_ORDER]
     h = provider.head()
     tensors += [(h[n], k) for n, k in HEAD_ORDER]
+    if time_mod:
+        t = provider.time()
+        tensors += [(t[n], k) for n, k in TIME_ORDER]
+        for l in range(layers):
+            m = provider.mod(l)
+            tensors += [(m[n], k) for n, k in MOD_ORDER]
     total = sum(nbytes(a, k) for a, k in tensors)
     out = np.empty(total, dtype=np.uint8)
     off = 0

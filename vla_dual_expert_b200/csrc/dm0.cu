@@ -139,6 +139,14 @@ struct dm0_ctx {
     uint8_t *wgu, *wd;
     float *sgu, *sd;
   };
+  // time-modulated action expert (cfg.time_mod): time MLP and modulator weights, and the tables of
+  // every Euler step's scales, shifts and gates and of the shifts projected through the weights
+  bf16 *tm_W_ti = nullptr, *tm_W_to = nullptr, *tm_Wmod = nullptr;   // [Ha][Ha] x 2, [(6L + 2) Ha][Ha]
+  float *tm_b_ti = nullptr, *tm_b_to = nullptr, *tm_bmod = nullptr;
+  int tm_cap = 0;                                                    // steps the tables hold
+  bf16 *tm_tau = nullptr, *tm_act = nullptr, *tm_beta = nullptr;     // [cap][Ha] x 2, [L][2][cap][Ha]
+  float *tm_c = nullptr, *tm_mod = nullptr;                          // [cap][Ha], [cap][(6L + 2) Ha]
+  float *tm_bqkv = nullptr, *tm_bgu = nullptr;                       // [L][cap][QR], [L][cap][2 Ia]
   bool fp8_mlp = false;
   std::vector<F8Layer> f8;
   uint8_t *xq_v = nullptr, *aq_v = nullptr;   // [Mp][hidden_v], [Mp][inter_v] codes
@@ -544,9 +552,16 @@ GemmArgs base_args(dm0_ctx* c) {
   return g;
 }
 
+// Per-step pointers of the time-modulated action expert for one layer (all into the tables built by
+// tmod_precompute): the QKV and gate/up feature biases (each norm's shift through the weights), the
+// attention and MLP gates, the MLP norm's 1 + scale, and the next layer's attention 1 + scale.
+struct ModPtrs {
+  const float *qkv_bias, *gate_o, *scale_m, *gu_bias, *gate_d, *next_scale;
+};
+
 // QKV projection of one branch with QK-norm + RoPE; K/V to [B][n_kv][kv_seq][D]
 dm0_status layer_qkv(dm0_ctx* c, cudaStream_t s, int br, int l, const bf16* xn, const float* ssq_in, int tokens,
-                     int seq, int pos_offset, bf16* q_out, bf16* k_out, bf16* v_out) {
+                     int seq, int pos_offset, bf16* q_out, bf16* k_out, bf16* v_out, const ModPtrs* mod = nullptr) {
   const LayerW& w = c->lw[br][l];
   const int H = hidden_of(c->cfg, br);
   GemmArgs g = base_args(c);
@@ -562,6 +577,7 @@ dm0_status layer_qkv(dm0_ctx* c, cudaStream_t s, int br, int l, const bf16* xn, 
   g.seq_len = seq;
   g.pos_offset = pos_offset;
   g.kv_seq = seq;
+  if (mod) g.col_bias = mod->qkv_bias;
   const int site = br == 0 ? DM0_SITE_VLM_QKV : DM0_SITE_ACT_QKV;
   const int e0 = probe_begin(c, s, site);
   TRY(run_gemm(c, s, xn, tokens, H, w.wqkv, qkv_rows(c->cfg), g));
@@ -571,7 +587,8 @@ dm0_status layer_qkv(dm0_ctx* c, cudaStream_t s, int br, int l, const bf16* xn, 
 
 // O-proj (+residual) -> gate/up (+SwiGLU) -> down (+residual) of one branch
 dm0_status layer_rest(dm0_ctx* c, cudaStream_t s, int br, int l, int tokens, float* h, bf16* xn, const bf16* o,
-                      bf16* act, float* ssq_mlp, const float* next_gain, float* next_ssq) {
+                      bf16* act, float* ssq_mlp, const float* next_gain, float* next_ssq,
+                      const ModPtrs* mod = nullptr) {
   const dm0_config& cf = c->cfg;
   const LayerW& w = c->lw[br][l];
   const int H = hidden_of(cf, br), I = inter_of(cf, br);
@@ -581,7 +598,8 @@ dm0_status layer_rest(dm0_ctx* c, cudaStream_t s, int br, int l, int tokens, flo
   g.h = h;
   g.H = H;
   g.xn = xn;
-  g.gain_next = w.mlp_norm;
+  g.gain_next = mod ? mod->scale_m : w.mlp_norm;
+  g.col_gate = mod ? mod->gate_o : nullptr;
   g.ssq_out = ssq_mlp;
   const int so = br == 0 ? DM0_SITE_VLM_O : DM0_SITE_ACT_O;
   int e0 = probe_begin(c, s, so);
@@ -598,6 +616,7 @@ dm0_status layer_rest(dm0_ctx* c, cudaStream_t s, int br, int l, int tokens, flo
   u.inv_hidden = 1.0f / H;
   u.act = act;
   u.inter = I;
+  u.col_bias = mod ? mod->gu_bias : nullptr;
   const int su = br == 0 ? DM0_SITE_VLM_GATEUP : DM0_SITE_ACT_GATEUP;
   e0 = probe_begin(c, s, su);
   if (f8) {
@@ -618,6 +637,7 @@ dm0_status layer_rest(dm0_ctx* c, cudaStream_t s, int br, int l, int tokens, flo
   d.xn = next_gain ? xn : nullptr;
   d.gain_next = next_gain;
   d.ssq_out = next_gain ? next_ssq : nullptr;
+  d.col_gate = mod ? mod->gate_d : nullptr;
   const int sd = br == 0 ? DM0_SITE_VLM_DOWN : DM0_SITE_ACT_DOWN;
   e0 = probe_begin(c, s, sd);
   if (f8) {
@@ -652,7 +672,14 @@ dm0_status enqueue_prefill(dm0_ctx* c, cudaStream_t s, const void* prefix_emb, i
   return DM0_OK;
 }
 
-dm0_status step(dm0_ctx* c, cudaStream_t s, int B, int k_out, int k_in, int steps, float* vel) {
+// The time-modulated expert's step: the final norm of step k_out takes its 1 + scale and shift, the
+// input of step k_in its first attention norm's 1 + scale, and no time embedding (null tables: DM0)
+struct StepMod {
+  const float *final_scale, *final_shift, *attn_scale0;
+};
+
+dm0_status step(dm0_ctx* c, cudaStream_t s, int B, int k_out, int k_in, int steps, float* vel,
+                const StepMod* mod = nullptr) {
   const dm0_config& cf = c->cfg;
   StepArgs a{};
   a.x = c->x;
@@ -674,9 +701,64 @@ dm0_status step(dm0_ctx* c, cudaStream_t s, int B, int k_out, int k_in, int step
   a.k_in = k_in;
   a.steps = steps;
   a.vel = vel;
+  const float* shift = nullptr;
+  if (mod) {
+    a.final_norm = mod->final_scale;
+    a.attn_norm0 = mod->attn_scale0;
+    shift = mod->final_shift;
+  }
   const int e0 = probe_begin(c, s, DM0_SITE_STEP);
-  TRY(launch(c, s, dm0::step_kernel, dim3(B * cf.chunk), dim3(256), sizeof(float) * cf.hidden_a, a));
+  TRY(launch(c, s, dm0::step_kernel, dim3(B * cf.chunk), dim3(256), sizeof(float) * cf.hidden_a, a, shift));
   probe_end(c, s, DM0_SITE_STEP, e0);
+  return DM0_OK;
+}
+
+// Tables of the time-modulated expert for `steps` Euler steps (t_k = 1 - k/K): c(t_k) through the time
+// MLP, every norm's [1 + scale | shift | gate] (one GEMM over all layers' modulators), and each
+// layer's two shifts projected through its QKV and gate/up weights (the biases of those GEMMs).  Each
+// weight is read once per Euler loop, not once per step.
+dm0_status tmod_tables(dm0_ctx* c, int steps) {
+  if (steps <= c->tm_cap) return DM0_OK;
+  const dm0_config& g = c->cfg;
+  const size_t cap = std::max(steps, 16), Ha = g.hidden_a, L = g.layers, R = (6 * L + 2) * Ha;
+  // a larger loop gets new tables; graphs captured earlier keep using (and own) the old ones
+  TRY(dalloc(c, &c->tm_tau, cap * Ha));
+  TRY(dalloc(c, &c->tm_act, cap * Ha));
+  TRY(dalloc(c, &c->tm_c, cap * Ha));
+  TRY(dalloc(c, &c->tm_mod, cap * R));
+  TRY(dalloc(c, &c->tm_beta, L * 2 * cap * Ha));
+  TRY(dalloc(c, &c->tm_bqkv, L * cap * qkv_rows(g)));
+  TRY(dalloc(c, &c->tm_bgu, L * cap * 2 * g.inter_a));
+  c->tm_cap = static_cast<int>(cap);
+  return DM0_OK;
+}
+
+dm0_status tmod_precompute(dm0_ctx* c, cudaStream_t s, int steps) {
+  const dm0_config& g = c->cfg;
+  const int Ha = g.hidden_a, L = g.layers, R = (6 * L + 2) * Ha, QR = qkv_rows(g), GU = 2 * g.inter_a;
+  TRY(tmod_tables(c, steps));
+  GemmArgs f = base_args(c);
+  f.mode = dm0::kModeStoreF32;
+  f.w_stable = 1;
+  TRY(launch(c, s, dm0::tmod_tau_kernel, dim3(steps), dim3(256), 0, c->tm_tau, steps, Ha));
+  f.out_f32 = c->tm_c;
+  TRY(run_gemm(c, s, c->tm_tau, steps, Ha, c->tm_W_ti, Ha, f, 0));
+  TRY(launch(c, s, dm0::tmod_bias_silu_kernel, dim3(steps), dim3(256), 0, static_cast<const float*>(c->tm_c),
+             static_cast<const float*>(c->tm_b_ti), Ha, c->tm_act));
+  TRY(run_gemm(c, s, c->tm_act, steps, Ha, c->tm_W_to, Ha, f, 0));
+  TRY(launch(c, s, dm0::tmod_bias_silu_kernel, dim3(steps), dim3(256), 0, static_cast<const float*>(c->tm_c),
+             static_cast<const float*>(c->tm_b_to), Ha, c->tm_act));
+  f.out_f32 = c->tm_mod;
+  TRY(run_gemm(c, s, c->tm_act, steps, Ha, c->tm_Wmod, R, f, 0));
+  TRY(launch(c, s, dm0::tmod_finish_kernel, dim3((R + 255) / 256, steps), dim3(256), 0, c->tm_mod,
+             static_cast<const float*>(c->tm_bmod), steps, L, Ha, c->tm_beta));
+  for (int l = 0; l < L; ++l) {
+    const LayerW& w = c->lw[1][l];
+    f.out_f32 = c->tm_bqkv + static_cast<size_t>(l) * steps * QR;
+    TRY(run_gemm(c, s, c->tm_beta + (static_cast<size_t>(l) * 2 + 0) * steps * Ha, steps, Ha, w.wqkv, QR, f, 0));
+    f.out_f32 = c->tm_bgu + static_cast<size_t>(l) * steps * GU;
+    TRY(run_gemm(c, s, c->tm_beta + (static_cast<size_t>(l) * 2 + 1) * steps * Ha, steps, Ha, w.wgu, GU, f, 0));
+  }
   return DM0_OK;
 }
 
@@ -687,22 +769,49 @@ dm0_status enqueue_denoise(dm0_ctx* c, cudaStream_t s, int steps, float* vel) {
   const int B = c->kv_B, P = c->kv_P, S = cf.chunk, L = cf.layers, D = cf.head_dim;
   const int Ms = B * S;
   const size_t lstride = static_cast<size_t>(B) * cf.n_kv * P * D;
-  TRY(step(c, s, B, -1, 0, steps, vel));
+  const bool tm = cf.time_mod != 0;
+  const size_t Ha = cf.hidden_a, R = (6 * static_cast<size_t>(L) + 2) * Ha;
+  // time-modulated expert: step k's row of the modulation table, layer l's [scale|shift|gate] x 2 at 6 l Ha
+  auto mrow = [&](int k) { return c->tm_mod + static_cast<size_t>(k) * R; };
+  auto step_mod = [&](int k_out, int k_in) {
+    StepMod m{};
+    // a non-null shift selects the modulated step (no time embedding on the input); at the loop's
+    // start no velocity is formed and step 0's final-norm row is only a placeholder
+    m.final_scale = mrow(k_out >= 0 ? k_out : 0) + 6 * L * Ha;
+    m.final_shift = m.final_scale + Ha;
+    m.attn_scale0 = k_in >= 0 ? mrow(k_in) : c->lw[1][0].attn_norm;
+    return m;
+  };
+  if (tm) TRY(tmod_precompute(c, s, steps));
+  StepMod sm = tm ? step_mod(-1, 0) : StepMod{};
+  TRY(step(c, s, B, -1, 0, steps, vel, tm ? &sm : nullptr));
   for (int k = 0; k < steps; ++k) {
     for (int l = 0; l < L; ++l) {
       const bf16* kl = c->kplane + l * lstride;
       const bf16* vl = c->vplane + l * lstride;
       float* ssq_attn = c->ssq_a + static_cast<size_t>(2 * l) * Ms;
       float* ssq_mlp = ssq_attn + Ms;
-      TRY(layer_qkv(c, s, 1, l, c->xn_a, ssq_attn, Ms, S, P, c->q_a, c->k_s, c->v_s));
+      const bool more = l + 1 < L;
+      ModPtrs mp{};
+      if (tm) {
+        const float* ml = mrow(k) + 6 * static_cast<size_t>(l) * Ha;
+        mp.qkv_bias = c->tm_bqkv + (static_cast<size_t>(l) * steps + k) * qkv_rows(cf);
+        mp.gate_o = ml + 2 * Ha;
+        mp.scale_m = ml + 3 * Ha;
+        mp.gu_bias = c->tm_bgu + (static_cast<size_t>(l) * steps + k) * 2 * cf.inter_a;
+        mp.gate_d = ml + 5 * Ha;
+        mp.next_scale = more ? ml + 6 * Ha : nullptr;
+      }
+      TRY(layer_qkv(c, s, 1, l, c->xn_a, ssq_attn, Ms, S, P, c->q_a, c->k_s, c->v_s, tm ? &mp : nullptr));
       const int e0 = probe_begin(c, s, DM0_SITE_ACT_ATTN);
       TRY(run_attn(c, s, c->q_a, S, kl, vl, P, c->k_s, c->v_s, S, c->o_a, B, 0, 1));
       probe_end(c, s, DM0_SITE_ACT_ATTN, e0);
-      const bool more = l + 1 < L;
-      TRY(layer_rest(c, s, 1, l, Ms, c->h_a, c->xn_a, c->o_a, c->act_a, ssq_mlp,
-                     more ? c->lw[1][l + 1].attn_norm : nullptr, more ? ssq_mlp + Ms : nullptr));
+      const float* next_gain = more ? (tm ? mp.next_scale : c->lw[1][l + 1].attn_norm) : nullptr;
+      TRY(layer_rest(c, s, 1, l, Ms, c->h_a, c->xn_a, c->o_a, c->act_a, ssq_mlp, next_gain,
+                     more ? ssq_mlp + Ms : nullptr, tm ? &mp : nullptr));
     }
-    TRY(step(c, s, B, k, k + 1 < steps ? k + 1 : -1, steps, vel));
+    sm = tm ? step_mod(k, k + 1 < steps ? k + 1 : -1) : StepMod{};
+    TRY(step(c, s, B, k, k + 1 < steps ? k + 1 : -1, steps, vel, tm ? &sm : nullptr));
   }
   return DM0_OK;
 }
@@ -718,6 +827,7 @@ bool persist_plan(dm0_ctx* c, int steps, float* vel, dm0::PdArgs* a, std::string
     return false;
   };
   if (!c->use_persist) return no("disabled");
+  if (g.time_mod) return no("time-modulated expert");
   if (c->persist_resident < 0) {   // once per context: can one CTA of the kernel live on every SM?
     int per_sm = 0, coop = 0;
     cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, c->device);
@@ -874,6 +984,8 @@ dm0_status denoise_from_x(dm0_ctx* c, cudaStream_t s, int steps, float* vel) {
       if (!(st == DM0_ESTATE && c->persist_resident == 0)) return st;   // else fall through
     }
   }
+  // the time-modulation tables are allocated outside any capture (an allocation may synchronise)
+  if (c->cfg.time_mod) TRY(tmod_tables(c, steps));
   if (vel || !c->use_graph || c->probe_mask) return enqueue_denoise(c, s, steps, vel);
   const auto key = std::make_tuple(c->kv_B, c->kv_P, steps);
   auto it = c->graphs.find(key);
@@ -918,6 +1030,7 @@ bool cfg_ok(const dm0_config& g, std::string* why) {
   if (g.max_prefix + g.chunk > 65536) return bad("max_prefix + chunk must be <= 65536");
   if (static_cast<long long>(g.max_batch) * g.chunk > 1 << 20) return bad("max_batch * chunk too large");
   if (!(g.rms_eps > 0.f) || !(g.rope_theta > 1.f)) return bad("rms_eps must be > 0 and rope_theta > 1");
+  if (g.time_mod != 0 && g.time_mod != 1) return bad("time_mod must be 0 or 1");
   return true;
 }
 
@@ -929,7 +1042,10 @@ size_t layer_bytes(const dm0_config& g, int br) {
 
 size_t blob_bytes(const dm0_config& g) {
   const size_t Ha = g.hidden_a, A = g.action_dim;
-  return g.layers * (layer_bytes(g, 0) + layer_bytes(g, 1)) + 2 * Ha * A + 4 * Ha + 4 * Ha + 2 * A * Ha + 4 * A;
+  size_t n = g.layers * (layer_bytes(g, 0) + layer_bytes(g, 1)) + 2 * Ha * A + 4 * Ha + 4 * Ha + 2 * A * Ha + 4 * A;
+  // time MLP (2 x [Ha][Ha] + biases), final modulator ([2Ha][Ha] + bias), two [3Ha][Ha] modulators per layer
+  if (g.time_mod) n += 8 * Ha * Ha + 16 * Ha + g.layers * (12 * Ha * Ha + 24 * Ha);
+  return n;
 }
 
 }  // namespace
@@ -1094,6 +1210,14 @@ dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
   c->W_out = reinterpret_cast<bf16*>(wb + offs[k++]);
   c->b_out = reinterpret_cast<float*>(wb + offs[k++]);
 
+  if (g.time_mod) {
+    const size_t Ha = g.hidden_a, R = (6 * Lz + 2) * Ha;
+    if (dalloc(c, &c->tm_W_ti, Ha * Ha) != DM0_OK || dalloc(c, &c->tm_W_to, Ha * Ha) != DM0_OK ||
+        dalloc(c, &c->tm_Wmod, R * Ha) != DM0_OK || dalloc(c, &c->tm_b_ti, Ha) != DM0_OK ||
+        dalloc(c, &c->tm_b_to, Ha) != DM0_OK || dalloc(c, &c->tm_bmod, R) != DM0_OK)
+      return bail(DM0_ENOMEM);
+  }
+
   const size_t D = g.head_dim, qd = g.n_q * D;
   const size_t Mp = static_cast<size_t>(g.max_batch) * g.max_prefix;
   const size_t Ms = static_cast<size_t>(g.max_batch) * g.chunk;
@@ -1227,6 +1351,21 @@ dm0_status dm0_load_weights(dm0_ctx* c, const void* blob, size_t bytes) {
   TRY(put(c->final_norm, 4 * Ha));
   TRY(put(c->W_out, 2 * Ad * Ha));
   TRY(put(c->b_out, 4 * Ad));
+  if (g.time_mod) {   // the modulators' rows go to one stacked matrix: [l][attention 3Ha | MLP 3Ha], final 2Ha
+    const size_t L = g.layers;
+    TRY(put(c->tm_W_ti, 2 * Ha * Ha));
+    TRY(put(c->tm_b_ti, 4 * Ha));
+    TRY(put(c->tm_W_to, 2 * Ha * Ha));
+    TRY(put(c->tm_b_to, 4 * Ha));
+    TRY(put(c->tm_Wmod + 6 * L * Ha * Ha, 2 * 2 * Ha * Ha));
+    TRY(put(c->tm_bmod + 6 * L * Ha, 4 * 2 * Ha));
+    for (size_t l = 0; l < L; ++l) {
+      for (size_t part = 0; part < 2; ++part) {
+        TRY(put(c->tm_Wmod + (6 * l + 3 * part) * Ha * Ha, 2 * 3 * Ha * Ha));
+        TRY(put(c->tm_bmod + (6 * l + 3 * part) * Ha, 4 * 3 * Ha));
+      }
+    }
+  }
   c->weights_loaded = true;
   if (c->fp8_mlp) {   // keep the FP8 copies in step with the new weights
     TRY(pack_fp8_weights(c, nullptr));
@@ -1319,6 +1458,7 @@ dm0_status dm0_merged_layer(dm0_ctx* c, int layer, const float* h_prefix, const 
     return fail(c, DM0_EINVAL, "null argument");
   if (!c->weights_loaded) return fail(c, DM0_ESTATE, "weights not loaded");
   const dm0_config& g = c->cfg;
+  if (g.time_mod) return fail(c, DM0_EINVAL, "the merged layer has no flow time: it covers the DM0 layer only");
   if (layer < 0 || layer >= g.layers || B < 1 || B > g.max_batch || P < 1 || P > g.max_prefix)
     return fail(c, DM0_ESHAPE, "layer, B or P outside the context capacity");
   cudaStream_t s = static_cast<cudaStream_t>(stream);

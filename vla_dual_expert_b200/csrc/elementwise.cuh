@@ -7,6 +7,8 @@
 //                  x <- x + dt v with dt = -1/K, then the next step's input
 //                  e = x W_in^T + b_in + tau(t) with t = 1 - k/K.
 //   rope_table   : (cos, sin) of position * theta^(-2i/D), in double precision.
+//   tmod_*       : the time-modulation tables of the time-modulated action expert.
+//   quant_rows_e4m3 : per-row FP8 E4M3 codes and scales.
 #pragma once
 #include <cuda_fp8.h>
 
@@ -64,9 +66,12 @@ struct StepArgs {
 // of h go through L2: in the persistent Euler loop other CTAs produced them.  xn / ssq are written
 // only when non-null.  Weight rows are read 16 bytes at a time when the shapes allow it, so the
 // loads of a row are in flight together.
-template <class Sync>
+// kMod: the time-modulated expert's step: final_norm holds the final norm's 1 + scale, final_shift
+// ([Ha]) its shift, and the time embedding is not added to the input (time enters through the
+// modulators).  kMod = false compiles the DM0 step (final_shift unused).
+template <bool kMod = false, class Sync>
 __device__ __forceinline__ void step_token(const StepArgs& a, int tok, int tid, int nthr, float* sx, float* sred,
-                                           float* hs, Sync&& sync) {
+                                           float* hs, Sync&& sync, const float* final_shift = nullptr) {
   const int nw = nthr >> 5, warp = tid >> 5, lane = tid & 31;
   float* hrow = a.h + static_cast<size_t>(tok) * a.Ha;
   const bool vec_out = (a.Ha % 256) == 0, vec_in = (a.A % 8) == 0;
@@ -84,9 +89,10 @@ __device__ __forceinline__ void step_token(const StepArgs& a, int tok, int tid, 
     for (int w = 0; w < nw; ++w) tot += sred[w];
     const float inv = rsqrtf(tot / a.Ha + a.eps);
     const float dt = -1.0f / a.steps;
+    const float* sh = kMod ? final_shift : nullptr;
     for (int o = warp; o < a.A; o += nw) {
       const __nv_bfloat16* wr = a.W_out + static_cast<size_t>(o) * a.Ha;
-      float acc = 0.f;
+      float acc = 0.f, accb = 0.f;   // accb: the modulated norm's shift through W_out
       if (vec_out) {   // lane reads 8 consecutive weights per 256-wide slice
         for (int j0 = lane * 8; j0 < a.Ha; j0 += 256) {
           const uint4 w8 = __ldg(reinterpret_cast<const uint4*>(wr + j0));
@@ -95,14 +101,19 @@ __device__ __forceinline__ void step_token(const StepArgs& a, int tok, int tid, 
           for (int e = 0; e < 4; ++e) {
             const float2 f = __bfloat1622float2(w2[e]);
             acc += f.x * hs[j0 + 2 * e] + f.y * hs[j0 + 2 * e + 1];
+            if (sh) accb += f.x * sh[j0 + 2 * e] + f.y * sh[j0 + 2 * e + 1];
           }
         }
       } else {
-        for (int j = lane; j < a.Ha; j += 32) acc += __bfloat162float(wr[j]) * hs[j];
+        for (int j = lane; j < a.Ha; j += 32) {
+          acc += __bfloat162float(wr[j]) * hs[j];
+          if (sh) accb += __bfloat162float(wr[j]) * sh[j];
+        }
       }
       acc = warp_sum(acc);
+      if (sh) accb = warp_sum(accb);
       if (lane == 0) {
-        const float v = acc * inv + a.b_out[o];
+        const float v = kMod ? acc * inv + (accb + a.b_out[o]) : acc * inv + a.b_out[o];
         float* xp = a.x + static_cast<size_t>(tok) * a.A + o;
         *xp = *xp + dt * v;
         if (a.vel) a.vel[(static_cast<size_t>(a.k_out) * a.tokens + tok) * a.A + o] = v;
@@ -133,9 +144,11 @@ __device__ __forceinline__ void step_token(const StepArgs& a, int tok, int tid, 
       } else {
         for (int i = 0; i < a.A; ++i) e += __bfloat162float(w[i]) * sx[i];
       }
-      const int fi = j < half ? j : j - half;
-      const float arg = t * exp2f(-static_cast<float>(fi) / half * kLog2_10000);
-      e += j < half ? sinf(arg) : cosf(arg);
+      if (!kMod) {
+        const int fi = j < half ? j : j - half;
+        const float arg = t * exp2f(-static_cast<float>(fi) / half * kLog2_10000);
+        e += j < half ? sinf(arg) : cosf(arg);
+      }
       hrow[j] = e;
       if (a.xn) a.xn[static_cast<size_t>(tok) * a.Ha + j] = __float2bfloat16_rn(a.attn_norm0[j] * e);
       sq += e * e;
@@ -155,14 +168,73 @@ __device__ __forceinline__ void step_token(const StepArgs& a, int tok, int tid, 
   }
 }
 
-// One CTA (256 threads) per action token; dynamic shared memory: Ha floats.
-__global__ void __launch_bounds__(256) step_kernel(const StepArgs a) {
+// One CTA (256 threads) per action token; dynamic shared memory: Ha floats.  final_shift non-null
+// selects the time-modulated step.
+__global__ void __launch_bounds__(256) step_kernel(const StepArgs a, const float* final_shift) {
   __shared__ float sx[64];
   __shared__ float sred[8];
   extern __shared__ float step_hs[];
   pdl_launch_dependents();
   pdl_wait();
-  step_token(a, blockIdx.x, threadIdx.x, 256, sx, sred, step_hs, [] { __syncthreads(); });
+  if (final_shift)
+    step_token<true>(a, blockIdx.x, threadIdx.x, 256, sx, sred, step_hs, [] { __syncthreads(); }, final_shift);
+  else
+    step_token<false>(a, blockIdx.x, threadIdx.x, 256, sx, sred, step_hs, [] { __syncthreads(); });
+}
+
+// ---------------------------------------------------------------- time modulation (DM0.5 page, section 5.2)
+//
+// The time-modulated action expert turns the flow time into a condition c(t) = W_to silu(W_ti tau(t) +
+// b_ti) + b_to and every pre-norm into an adaptive RMSNorm whose scale, shift and gate are
+// W_m silu(c) + b_m.  They depend only on t_k = 1 - k/K and the weights, so one pass per Euler loop
+// builds them for all K steps (three GEMMs over K rows, below) instead of per step.
+
+// row k of out: bf16 tau(t_k), t_k = 1 - k / steps, [sin(t w_i) | cos(t w_i)], w_i = 10000^(-i / (Ha/2))
+__global__ void __launch_bounds__(256) tmod_tau_kernel(__nv_bfloat16* out, int steps, int Ha) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int k = blockIdx.x, half = Ha >> 1;
+  const float t = 1.0f - static_cast<float>(k) / static_cast<float>(steps);
+  const float kLog2_10000 = 13.287712379549449f;
+  for (int j = threadIdx.x; j < Ha; j += blockDim.x) {
+    const int fi = j < half ? j : j - half;
+    const float arg = t * exp2f(-static_cast<float>(fi) / half * kLog2_10000);
+    out[static_cast<size_t>(k) * Ha + j] = __float2bfloat16_rn(j < half ? sinf(arg) : cosf(arg));
+  }
+}
+
+// out[r][c] = bf16(silu(in[r][c] + bias[c])): the activation between the time MLP's layers, and the
+// modulators' input silu(c)
+__global__ void __launch_bounds__(256) tmod_bias_silu_kernel(const float* in, const float* bias, int cols,
+                                                             __nv_bfloat16* out) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const size_t r = blockIdx.x;
+  for (int j = threadIdx.x; j < cols; j += blockDim.x) {
+    const float v = in[r * cols + j] + bias[j];
+    out[r * cols + j] = __float2bfloat16_rn(silu_f(v));
+  }
+}
+
+// Finish the modulation table mod[k][0 .. L 6 Ha + 2 Ha) in place: add the bias, turn every scale g
+// into 1 + g (the factor that multiplies x / rms(x)), and copy each layer's two shifts in bf16 to
+// beta[l][0 attention | 1 MLP][k][Ha], the operands of the shift projections.  Per layer the rows are
+// [attention: scale | shift | gate][MLP: scale | shift | gate]; the final norm's [scale | shift] close
+// the row.
+__global__ void __launch_bounds__(256) tmod_finish_kernel(float* mod, const float* bmod, int steps, int L, int Ha,
+                                                          __nv_bfloat16* beta) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int k = blockIdx.y;
+  const int R = (6 * L + 2) * Ha;
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= R) return;
+  float v = mod[static_cast<size_t>(k) * R + r] + bmod[r];
+  const int l = r / (6 * Ha), q = r - l * 6 * Ha, part = q / Ha, j = q - part * Ha;
+  if (part == 0 || part == 3) v += 1.f;   // scales (the final norm's scale is part 0 of "layer" L)
+  if (l < L && (part == 1 || part == 4))
+    beta[((static_cast<size_t>(l) * 2 + (part == 4)) * steps + k) * Ha + j] = __float2bfloat16_rn(v);
+  mod[static_cast<size_t>(k) * R + r] = v;
 }
 
 // Failure-path self-test: one thread waits, with the library's bounded wait, on an mbarrier

@@ -72,6 +72,10 @@ struct GemmArgs {
   // is multiplied by row_scale[token] * col_scale[feature] before the mode's epilogue
   const float* row_scale;   // [M] per-token activation scale
   const float* col_scale;   // [N] per-output-channel weight scale
+  // time-modulated action expert (adaptive RMSNorm): null in the plain model
+  const float* col_bias;    // QKV / SwiGLU: feature bias added after the pending 1/rms (the norm's shift
+                            // projected through the weights)
+  const float* col_gate;    // residual: per-feature gate applied to the sublayer output before the add
 };
 
 constexpr int kGemmThreads = 192;
@@ -154,6 +158,10 @@ __device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool va
       if (!kFromScratch) {   // normal orientation: add into the residual stream here
         float hv[32];
         ld_f32x32(hp, hv);
+        if (a.col_gate) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] *= a.col_gate[col0 + 32 * c + j];
+        }
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] += hv[j];
         st_f32x32(hp, v);
@@ -170,15 +178,26 @@ __device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool va
     }
     return;
   }
-  // QKV and SwiGLU consume the pending RMSNorm's 1/rms of this token
-  const float s = (a.ssq_in && valid) ? rsqrtf(__ldcg(a.ssq_in + tok) * a.inv_hidden + a.eps) : 1.f;
+  // QKV and SwiGLU consume the pending RMSNorm's 1/rms of this token; with a feature bias (the
+  // modulated norm's shift projected through the weights) the loader returns acc / rms + bias and the
+  // code below sees a unit scale
+  const float s_rms = (a.ssq_in && valid) ? rsqrtf(__ldcg(a.ssq_in + tok) * a.inv_hidden + a.eps) : 1.f;
+  const float* bias = a.col_bias;
+  const float s = bias ? 1.f : s_rms;
+  auto ld = [&](int c, float (&v)[32]) {
+    load(c, v);
+    if (bias) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = v[j] * s_rms + bias[col0 + 32 * c + j];
+    }
+  };
   if (a.mode == kModeSwiGLU) {
     // group = [64 gate rows | 64 up rows] of outputs [col0/2, col0/2 + 64)
 #pragma unroll 1
     for (int c = 0; c < 2; ++c) {
       float g[32], u[32];
-      load(c, g);
-      load(c + 2, u);
+      ld(c, g);
+      ld(c + 2, u);
 #pragma unroll
       for (int j = 0; j < 32; ++j) g[j] = silu_f(g[j] * s) * (u[j] * s);
       if (valid) {
@@ -214,7 +233,7 @@ __device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool va
 #pragma unroll 1
       for (int c = h0; c < h0 + cph; ++c) {
         float v[32];
-        load(c, v);
+        ld(c, v);
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] *= s;
         if (valid) st_bf16x32(dst_of(col0 + 32 * c), v);
@@ -227,7 +246,7 @@ __device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool va
 #pragma unroll 1
     for (int c = h0; c < h0 + cph; ++c) {
       float v[32];
-      load(c, v);
+      ld(c, v);
 #pragma unroll
       for (int j = 0; j < 32; ++j) ss += v[j] * v[j];
     }
@@ -235,7 +254,7 @@ __device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool va
     if (D == 32) {
       // one chunk, pairs (j, j + 16)
       float v[32];
-      load(h0, v);
+      ld(h0, v);
       float o[32];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
@@ -250,8 +269,8 @@ __device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool va
 #pragma unroll 1
       for (int c = 0; c < cph / 2; ++c) {
         float lo[32], hi[32];
-        load(h0 + c, lo);
-        load(h0 + c + cph / 2, hi);
+        ld(h0 + c, lo);
+        ld(h0 + c + cph / 2, hi);
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const int d = 32 * c + j;
@@ -420,10 +439,12 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
         for (int c = 0; c < BN / 32; ++c) {
           float v[32];
           tmem_ld32(tl + c * 32, v);
+          // residual with a gate: this split's partial of the gated sublayer output (linear in acc)
+          const float gt = (a.mode == kModeResid && a.col_gate) ? a.col_gate[feat] : 1.f;
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int tok = tokbase + c * 32 + j;
-            if (tok < a.tokens) atomicAdd(dst + static_cast<size_t>(tok) * ld + feat, v[j]);
+            if (tok < a.tokens) atomicAdd(dst + static_cast<size_t>(tok) * ld + feat, v[j] * gt);
           }
         }
         __threadfence();
