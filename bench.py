@@ -115,6 +115,12 @@ def layer_params(d, branch):
     return H * (d.n_q + 2 * d.n_kv) * D + d.n_q * D * H + 3 * H * I
 
 
+def pack_time_mod_weights(weights, d):
+    """Blob of the time-modulated expert: the same seeded weights plus the time MLP and modulators."""
+    from vla_dual_expert_b200._abi import pack_weights
+    return pack_weights(weights, d.layers, time_mod=True)
+
+
 def prefill_gateup_flops(d, B, P):
     """One VLM gate/up GEMM launch: [B*P x H] x [H -> 2I]."""
     return 2.0 * B * P * d.hidden_v * 2 * d.inter_v
@@ -177,7 +183,7 @@ def run_native(args, rank, world, local_rank):
     eng.load_from(weights)
     stream = torch.cuda.current_stream()
 
-    def measure(wl, steps, warmup, probe):
+    def measure(wl, steps, warmup, probe, eng=eng):
         B, P = wl.batch, wl.prefix
         emb = torch.from_numpy(I.prefix_embeddings(d, B, P, seed=1000 + 97 * rank)).cuda().to(torch.bfloat16)
         noise = torch.from_numpy(I.noise(d, B, seed=2000 + 97 * rank)).cuda()
@@ -329,6 +335,21 @@ def run_native(args, rank, world, local_rank):
                             "unit": "TFLOP/s", "frac": round(f8_tf / fp8_peak, 4),
                             "peak_src": f"{peaks['src']} bf16_tflops_sustained x 2 (nominal fp8 / bf16 ratio)"},
             "gpu_launches": f8["launches"], "clocks": f8["clocks"]}
+    if args.time_mod:
+        # the same step for the time-modulated action expert (opt-in; its own weights and context)
+        from vla_dual_expert_b200 import Engine as _Engine
+        eng_tm = _Engine(d, max(wl_main.batch, 1), max(wl_main.prefix, 816), time_mod=True)
+        try:
+            eng_tm.load_weights(pack_time_mod_weights(weights, d))
+            tm = {}
+            for wl in (wl_main, I.WORKLOADS["e2e_b1"]):
+                r = measure(wl, args.steps, args.warmup, None, eng=eng_tm)
+                tm[wl.name] = {"value": round(job_chunks_per_s(world, wl.batch, r["ms"]), 3), "unit": "chunks/s",
+                               "ms_per_step": round(r["ms"], 3), "prefill_ms_p50": round(r["prefill_ms_p50"], 3),
+                               "denoise_ms_p50": round(r["denoise_ms_p50"], 3), "gpu_launches": r["launches"]}
+            result["time_mod"] = tm
+        finally:
+            eng_tm.close()
     if not args.skip_breakdown:
         result["breakdown_ms_per_step"] = breakdown(eng, wl_main)
         if "batch1" in result:
@@ -483,6 +504,8 @@ def main():
     ap.add_argument("--one-layer", action="store_true", help="profiling workload: one layer, B=16, P=2048")
     ap.add_argument("--b1-loop", action="store_true", help="profiling workload: persistent Euler loop, 3 layers, B=1")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--time-mod", action="store_true",
+                    help="also time the step of the time-modulated action expert (reported under time_mod)")
     ap.add_argument("--prefix-fp8", action="store_true",
                     help="also time the step with the VLM MLP in FP8 E4M3 (reported under prefix_fp8)")
     args = ap.parse_args()

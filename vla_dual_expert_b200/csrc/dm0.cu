@@ -7,11 +7,16 @@
 //              QKV GEMM (+QK-norm, RoPE, KV-cache write) -> attention
 //              -> O GEMM (+residual, next-norm operand) -> gate/up GEMM (+SwiGLU)
 //              -> down GEMM (+residual, next-norm operand)
-//   denoise  : step_kernel(input of step 0), then per step 28 action layers of
+//   denoise  : one observation of the DM0-base shapes: the whole Euler loop as one
+//              persistent kernel (denoise_persistent.cuh).  Otherwise
+//              step_kernel(input of step 0), then per step 28 action layers of
 //              the same five kernels (attention over [prefix cache; suffix])
-//              and step_kernel(velocity, Euler update, input of the next step).
-//              The whole loop is captured once per (B, P, steps) into a CUDA
-//              graph and replayed.
+//              and step_kernel(velocity, Euler update, input of the next step),
+//              captured once per (B, P, steps) into a CUDA graph and replayed.
+//   options  : the FP8 E4M3 VLM MLP (dm0_set_prefix_fp8: per-token operand
+//              quantisation + the kind::f8f6f4 GEMM), and the time-modulated
+//              action expert (time_mod: per-loop modulation tables, then the
+//              per-layer kernels with feature biases, gates and per-step gains).
 // Every kernel is launched with programmatic stream serialization, so each
 // kernel's prologue (TMEM allocation, barrier set-up, weight-tile requests)
 // overlaps the previous kernel's tail.
