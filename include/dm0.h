@@ -182,6 +182,36 @@ dm0_status dm0_infer_host(dm0_ctx* ctx, const void* prefix_emb, const float* noi
 dm0_status dm0_merged_layer(dm0_ctx* ctx, int layer, const float* h_prefix, const float* h_suffix, int B, int P,
                             float* out_prefix, float* out_suffix, void* k_out, void* v_out, void* stream);
 
+/* Flow-matching training step (DM0.5 page, section 5.3). ------------------ */
+
+/* Floats of the gradient buffer of dm0_train_step for `cfg`: per action layer
+ * attn_norm[Ha] | Wq[n_q*D][Ha] | Wk[n_kv*D][Ha] | Wv[n_kv*D][Ha] | q_norm[D] |
+ * k_norm[D] | Wo[Ha][n_q*D] | mlp_norm[Ha] | Wg[Ia][Ha] | Wu[Ia][Ha] | Wd[Ha][Ia],
+ * then W_in[Ha][A] | b_in[Ha] | final_norm[Ha] | W_out[A][Ha] | b_out[A]: the
+ * action-expert part of the weight blob, in fp32, no padding. */
+size_t dm0_grad_floats(const dm0_config* cfg);
+
+/* One training step of the DM0 action expert over the context's prefix cache
+ * (the last dm0_prefill or dm0_kv_commit; its B samples):
+ *   x_t = t eps + (1 - t) a and u = eps - a per sample; v = the expert's velocity
+ *   at (x_t, t); loss = sum over valid entries of (v - u)^2 / their count (0 if
+ *   none); grads = dloss / d(every action-expert and head parameter).
+ *   a, eps:  device f32 [B][chunk][action_dim]; t: device f32 [B];
+ *   mask:    device u8 [B][chunk][action_dim], nonzero = valid entry;
+ *   loss:    device f32 [1], written;
+ *   grads:   device f32 [dm0_grad_floats(cfg)] (16-byte aligned), written;
+ *   kv_grads: null (knowledge insulation: the prefix K/V is a constant), or
+ *            device f32 [2][layers][B][n_kv][P][head_dim]: dloss/dK then dloss/dV
+ *            of the cache (where the gradient would enter the VLM).
+ * Forward projections and every dX = dY W, dW = dY^T X run on the tensor-core
+ * GEMM with bf16 operands and fp32 accumulation; the first call after
+ * dm0_load_weights builds transposed copies of the action weights (0.9 GB at
+ * DM0-base widths) and the step's buffers.  Asynchronous on `stream`.
+ * Returns DM0_ESTATE without weights or cache, DM0_EINVAL for null pointers,
+ * misaligned grads or a time_mod context, DM0_ESHAPE if chunk * head_dim > 8192. */
+dm0_status dm0_train_step(dm0_ctx* ctx, const float* a, const float* eps, const float* t, const uint8_t* mask,
+                          float* loss, float* grads, float* kv_grads, void* stream);
+
 /* Kernel-level entry points used by the unit tests. -------------------- */
 
 /* Tensor-core GEMM in fp32 accumulation:

@@ -121,3 +121,22 @@ def test_probe_site_names_match_the_header():
     count = sites.pop("COUNT")
     assert count == len(SITES) == len(sites)
     assert [n.lower() for n, _ in sorted(sites.items(), key=lambda kv: kv[1])] == list(SITES)
+
+
+@pytest.mark.parametrize("dims", [I.TINY, I.DM0_BASE.replace(layers=3)])
+def test_gradient_buffer_layout_matches_the_oracle_parameters(dims):
+    """dm0_grad_floats covers exactly the action-expert and head parameters the training oracle
+    differentiates, in the blob order."""
+    abi, lib = _lib()
+    cfg = abi.make_config(dims, 1, 64)
+    n = lib.dm0_grad_floats(ctypes.byref(cfg))
+    w = I.Weights(dims, seed=0)
+    want = sum(np.size(v) for l in range(dims.layers) for v in w.layer(1, l).values())
+    want += sum(np.size(v) for v in w.head().values())
+    assert n == want
+    layout = abi.grad_layout(dims)
+    for (key, shape) in layout:
+        ref = w.head()[key[1]] if key[0] == "head" else w.layer(1, key[0])[key[1]]
+        assert tuple(shape) == np.shape(ref), key
+    g = abi.unpack_grads(np.arange(n, dtype=np.float32), dims)
+    assert g[(0, "attn_norm")][0] == 0 and g[("head", "b_out")][-1] == n - 1

@@ -1,0 +1,120 @@
+"""Parity of the flow-matching training step (dm0_train_step; DM0.5 page, section 5.3, reading R13)
+with the fp64 oracle oracle/dm0_train.py.
+
+Every GEMM operand of the step (the normalised activations, the attention output, the SwiGLU output,
+every upstream gradient and the token-padded transposes) is rounded to bf16, 2^-9 relative, so each
+gradient tensor is held to RMS(gpu - oracle) <= 3e-2 RMS(oracle) and the loss (dominated by the
+fp32 target u) to 1e-3 relative.  These tests await their first GPU run (DM0_RUN_TRAIN=1).
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import dm0_train as T
+from synth import inputs as I
+from tests.gpu_util import host, rms, to_dev_bf16
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(os.environ.get("DM0_RUN_TRAIN") != "1",
+                                 reason="awaits its first GPU run (DM0_RUN_TRAIN=1)")]
+
+TOL_GRAD, TOL_LOSS = 3e-2, 1e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from vla_dual_expert_b200 import build
+    build.build()
+
+
+def _setup(d, B, P, seed=0):
+    """Engine with weights and an injected random bf16 prefix cache; the oracle's copies of it."""
+    from vla_dual_expert_b200 import Engine
+    from tests.gpu_util import device_view_bf16
+    w = I.Weights(d, seed=seed, gain_jitter=0.1)
+    eng = Engine(d, B, P)
+    eng.load_from(w)
+    kp, vp = eng.kv_view()
+    K = device_view_bf16(kp, (d.layers, B, d.n_kv, P, d.head_dim))
+    V = device_view_bf16(vp, (d.layers, B, d.n_kv, P, d.head_dim))
+    caches = [([], []) for _ in range(B)]
+    for l in range(d.layers):
+        k, v = I.random_kv_layer(d, B, P, l)
+        K[l].copy_(to_dev_bf16(k))
+        V[l].copy_(to_dev_bf16(v))
+        for b in range(B):
+            caches[b][0].append(k[b].astype(np.float64))
+            caches[b][1].append(v[b].astype(np.float64))
+    eng.kv_commit(B, P)
+    return w, eng, caches
+
+
+def _run(eng, d, a, eps, t, mask, with_kv, B, P):
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()   # noqa: E731
+    kv = torch.empty((2, d.layers, B, d.n_kv, P, d.head_dim), device="cuda", dtype=torch.float32) if with_kv else None
+    loss, grads = eng.train_step(dev(a.astype(np.float32)), dev(eps.astype(np.float32)), dev(t.astype(np.float32)),
+                                 dev(mask.astype(np.uint8)), kv_grads=kv)
+    eng.sync()
+    assert eng.device_error() == 0
+    from vla_dual_expert_b200._abi import unpack_grads
+    return float(host(loss)[0]), unpack_grads(host(grads), d), (host(kv) if with_kv else None)
+
+
+def _check_grads(got, ref, what):
+    worst = 0.0
+    for key, r in ref.items():
+        g = got[key]
+        assert np.all(np.isfinite(g)), (what, key)
+        e = rms(g - r) / max(rms(r), 1e-30)
+        worst = max(worst, e)
+        assert e <= TOL_GRAD, f"{what} {key}: RMS(d)/RMS {e:.3e}"
+    print(f"  {what}: worst gradient RMS(d)/RMS {worst:.3e}")
+
+
+@pytest.mark.parametrize("d,B,P", [(I.TINY, 2, 16), (I.DM0_BASE.replace(layers=1), 1, 64)])
+def test_train_step_matches_the_oracle(d, B, P):
+    w, eng, caches = _setup(d, B, P)
+    try:
+        a, eps, t, mask = I.train_batch(d, B)
+        loss, grads, kv = _run(eng, d, a, eps, t, mask, True, B, P)
+    finally:
+        eng.close()
+    ref = T.train_step(w, caches, a.astype(np.float64), eps.astype(np.float64), t, mask, ki=False)
+    assert abs(loss - ref["loss"]) <= TOL_LOSS * ref["loss"]
+    _check_grads(grads, ref["grads"], f"{d.hidden_a}-wide, B={B}")
+    for b in range(B):
+        for l in range(d.layers):
+            for which in (0, 1):
+                r = ref["kv_grads"][b][l][which]
+                e = rms(kv[which, l, b] - r) / rms(r)
+                assert e <= TOL_GRAD, f"cache grad b={b} l={l} {'KV'[which]}: {e:.3e}"
+
+
+def test_knowledge_insulation_leaves_the_parameter_gradients():
+    d, B, P = I.TINY, 2, 16
+    w, eng, _ = _setup(d, B, P)
+    try:
+        a, eps, t, mask = I.train_batch(d, B, seed=4400)
+        l1, g1, _ = _run(eng, d, a, eps, t, mask, True, B, P)
+        l2, g2, _ = _run(eng, d, a, eps, t, mask, False, B, P)
+    finally:
+        eng.close()
+    assert abs(l1 - l2) <= 1e-6 * l1
+    for k in g1:   # atomics in the attention adjoint sum in any order
+        assert rms(g1[k] - g2[k]) <= 1e-5 * max(rms(g1[k]), 1e-30), k
+
+
+def test_empty_mask_gives_zero_loss_and_gradients():
+    d, B, P = I.TINY, 1, 16
+    w, eng, _ = _setup(d, B, P)
+    try:
+        a, eps, t, mask = I.train_batch(d, B)
+        loss, grads, kv = _run(eng, d, a, eps, t, np.zeros_like(mask), True, B, P)
+    finally:
+        eng.close()
+    assert loss == 0.0
+    assert all(not np.any(g) for g in grads.values())
+    assert not np.any(kv)

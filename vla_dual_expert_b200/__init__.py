@@ -154,6 +154,31 @@ class Engine:
         _check_cuda(C, torch.float32, (N, M) if swap else (M, N), "C")
         self._chk(self.lib.dm0_op_gemm(self.h, _ptr(A), _ptr(B), _ptr(C), M, N, K, swap, splits, _stream(stream)))
 
+    def grad_floats(self) -> int:
+        return int(self.lib.dm0_grad_floats(ctypes.byref(self.cfg)))
+
+    def train_step(self, a, eps, t, mask, grads=None, kv_grads=None, stream=None):
+        """One flow-matching training step (dm0_train_step) over the context's prefix cache.
+
+        a, eps: CUDA f32 [B][chunk][A]; t: CUDA f32 [B]; mask: CUDA uint8 [B][chunk][A].  Returns (loss
+        [1], grads [grad_floats]) as CUDA f32 tensors; kv_grads, when given, is CUDA f32
+        [2][layers][B][n_kv][P][head_dim] and receives the cache gradients."""
+        import torch
+        B = a.shape[0]
+        d = self.dims
+        shape = (B, d.chunk, d.action_dim)
+        _check_cuda(a, torch.float32, shape, "a")
+        _check_cuda(eps, torch.float32, shape, "eps")
+        _check_cuda(t, torch.float32, (B,), "t")
+        _check_cuda(mask, torch.uint8, shape, "mask")
+        if grads is None:
+            grads = torch.empty(self.grad_floats(), device=a.device, dtype=torch.float32)
+        _check_cuda(grads, torch.float32, (self.grad_floats(),), "grads")
+        loss = torch.empty(1, device=a.device, dtype=torch.float32)
+        self._chk(self.lib.dm0_train_step(self.h, _ptr(a), _ptr(eps), _ptr(t), _ptr(mask), _ptr(loss), _ptr(grads),
+                                          _ptr(kv_grads), _stream(stream)))
+        return loss, grads
+
     def set_prefix_fp8(self, enable: bool = True, stream=None):
         """Run the VLM MLP's gate/up and down GEMMs in FP8 E4M3 (dm0_set_prefix_fp8)."""
         self._chk(self.lib.dm0_set_prefix_fp8(self.h, 1 if enable else 0, _stream(stream)))

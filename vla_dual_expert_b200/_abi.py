@@ -26,7 +26,7 @@ EXPORTS = ("dm0_create", "dm0_weights_bytes", "dm0_load_weights", "dm0_prefill",
            "dm0_op_attention", "dm0_attention_noalloc", "dm0_debug_view", "dm0_launch_count", "dm0_probe",
            "dm0_probe_read", "dm0_selftest_timeout", "dm0_sync", "dm0_device_error", "dm0_clear_error", "dm0_last_error",
            "dm0_destroy", "dm0_pack_e4m3_rows", "dm0_set_prefix_fp8", "dm0_op_quant_e4m3",
-           "dm0_op_gemm_e4m3")
+           "dm0_op_gemm_e4m3", "dm0_grad_floats", "dm0_train_step")
 
 
 class Dm0Config(ctypes.Structure):
@@ -82,6 +82,8 @@ def load_library() -> ctypes.CDLL:
         "dm0_set_prefix_fp8": (c_int, [P, c_int, P]),
         "dm0_op_quant_e4m3": (c_int, [P, P, c_int, c_int, c_int, P, P, P, P, P]),
         "dm0_op_gemm_e4m3": (c_int, [P, P, P, P, P, P, c_int, c_int, c_int, P]),
+        "dm0_grad_floats": (c_size_t, [P]),
+        "dm0_train_step": (c_int, [P, P, P, P, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -151,4 +153,28 @@ def pack_weights(provider, layers: int, time_mod: bool = False) -> np.ndarray:
         src = _bf16_bits(a) if k == "bf16" else np.ascontiguousarray(a, dtype=np.float32)
         out[off:off + n] = src.reshape(-1).view(np.uint8)
         off += n
+    return out
+
+
+def grad_layout(dims):
+    """(key, shape) of every tensor of the dm0_train_step gradient buffer, in order: (l, name) for the
+    action layers, ("head", name) for the head (the action-expert part of the blob order)."""
+    H, I, D, A = dims.hidden_a, dims.inter_a, dims.head_dim, dims.action_dim
+    shapes = {"attn_norm": (H,), "Wq": (dims.n_q * D, H), "Wk": (dims.n_kv * D, H), "Wv": (dims.n_kv * D, H),
+              "q_norm": (D,), "k_norm": (D,), "Wo": (H, dims.n_q * D), "mlp_norm": (H,), "Wg": (I, H),
+              "Wu": (I, H), "Wd": (H, I)}
+    out = [((l, name), shapes[name]) for l in range(dims.layers) for name, _ in LAYER_ORDER]
+    head = {"W_in": (H, A), "b_in": (H,), "final_norm": (H,), "W_out": (A, H), "b_out": (A,)}
+    out += [(("head", name), head[name]) for name, _ in HEAD_ORDER]
+    return out
+
+
+def unpack_grads(flat: np.ndarray, dims) -> dict:
+    """Split a host copy of the gradient buffer into arrays keyed as in grad_layout."""
+    out, off = {}, 0
+    for key, shape in grad_layout(dims):
+        n = int(np.prod(shape))
+        out[key] = flat[off:off + n].reshape(shape)
+        off += n
+    assert off == flat.size, (off, flat.size)
     return out
