@@ -335,6 +335,32 @@ def run_native(args, rank, world, local_rank):
                             "unit": "TFLOP/s", "frac": round(f8_tf / fp8_peak, 4),
                             "peak_src": f"{peaks['src']} bf16_tflops_sustained x 2 (nominal fp8 / bf16 ratio)"},
             "gpu_launches": f8["launches"], "clocks": f8["clocks"]}
+    if args.train:
+        # one flow-matching training step over the prefix cache the timed step left (opt-in)
+        a_np, e_np, t_np, m_np = I.train_batch(d, B, seed=4000 + 97 * rank)
+        ta, te = torch.from_numpy(a_np).cuda(), torch.from_numpy(e_np).cuda()
+        tt = torch.from_numpy(t_np.astype(np.float32)).cuda()
+        tm_ = torch.from_numpy(m_np.astype(np.uint8)).cuda()
+        grads = torch.empty(eng.grad_floats(), device="cuda", dtype=torch.float32)
+        for _ in range(max(1, args.warmup)):
+            eng.train_step(ta, te, tt, tm_, grads=grads)
+        eng.sync()
+        barrier()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        n0 = eng.launch_count()
+        t0.record(stream)
+        for _ in range(args.steps):
+            loss, _ = eng.train_step(ta, te, tt, tm_, grads=grads)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        tms = rank_max(t0.elapsed_time(t1) / args.steps)
+        result["train"] = {"workload": f"flow-matching training step of the 28-layer action expert, B={B} samples of "
+                                       f"50x32 over a P={P} prefix cache (knowledge insulation)",
+                           "value": round(world * B * 1000.0 / tms, 3), "unit": "samples/s",
+                           "ms_per_step": round(tms, 3), "loss": float(loss.item()),
+                           "gpu_launches": (eng.launch_count() - n0) // max(args.steps, 1)}
     if args.time_mod:
         # the same step for the time-modulated action expert (opt-in; its own weights and context)
         from vla_dual_expert_b200 import Engine as _Engine
@@ -504,6 +530,8 @@ def main():
     ap.add_argument("--one-layer", action="store_true", help="profiling workload: one layer, B=16, P=2048")
     ap.add_argument("--b1-loop", action="store_true", help="profiling workload: persistent Euler loop, 3 layers, B=1")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--train", action="store_true",
+                    help="also time one flow-matching training step (reported under train)")
     ap.add_argument("--time-mod", action="store_true",
                     help="also time the step of the time-modulated action expert (reported under time_mod)")
     ap.add_argument("--prefix-fp8", action="store_true",
