@@ -117,3 +117,44 @@ def test_zero_velocity_head_keeps_noise():
     finally:
         eng.close()
     assert np.array_equal(x, noise.astype(np.float64))
+
+
+def test_single_observation_runs_as_one_persistent_launch():
+    """DM0-base widths, B = 1: the time-modulated Euler loop is the persistent kernel's modulated
+    instantiation (one launch after the table pass), against the oracle and against the per-layer
+    kernels of the same inputs."""
+    d = I.DM0_BASE.replace(layers=2)
+    w = I.Weights(d, seed=0, gain_jitter=0.1)
+    P, steps = 100, 3
+    noise = I.noise(d, 1)
+    k_np, v_np = zip(*[I.random_kv_layer(d, 1, P, l) for l in range(d.layers)])
+    results = {}
+    for mode in ("persistent", "per_layer"):
+        if mode == "per_layer":
+            os.environ["DM0_NO_PERSIST"] = "1"
+        try:
+            eng = _engine(d, 1, P, w)
+        finally:
+            os.environ.pop("DM0_NO_PERSIST", None)
+        try:
+            from tests.gpu_util import device_view_bf16
+            kp, vp = eng.kv_view()
+            K = device_view_bf16(kp, (d.layers, 1, d.n_kv, P, d.head_dim))
+            V = device_view_bf16(vp, (d.layers, 1, d.n_kv, P, d.head_dim))
+            for l in range(d.layers):
+                K[l].copy_(to_dev_bf16(k_np[l]))
+                V[l].copy_(to_dev_bf16(v_np[l]))
+            eng.kv_commit(1, P)
+            n0 = eng.launch_count()
+            x = host(eng.denoise(torch.from_numpy(noise).cuda(), steps))
+            eng.sync()
+            assert eng.device_error() == 0
+            results[mode] = (x, eng.launch_count() - n0)
+        finally:
+            eng.close()
+    ks = [k[0].astype(np.float64) for k in k_np]
+    vs = [v[0].astype(np.float64) for v in v_np]
+    rx, _ = M.denoise(w, ks, vs, noise[0], steps)
+    check_fp(results["persistent"][0][0], rx, TOL_CHUNK, "persistent chunk")
+    check_fp(results["persistent"][0][0], results["per_layer"][0][0], 1e-2, "persistent vs per-layer")
+    assert results["persistent"][1] < results["per_layer"][1]

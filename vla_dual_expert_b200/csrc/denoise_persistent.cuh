@@ -108,6 +108,13 @@ struct PdArgs {
   int* err;
   unsigned long long* trace;  // optional [phase][CTA][kPdTraceSlots] %globaltimer marks; null: off
   StepArgs step;            // x, h, W_in, b_in, final_norm, W_out, b_out, Ha, A, eps, steps, tokens, vel
+  // time-modulated expert (the kernel's kMod instantiation): the per-loop tables of every step's
+  // [1 + scale | shift | gate] x 2 per layer + the final [1 + scale | shift] (rows of tm_R floats), and
+  // the shifts through the QKV and gate/up weights ([L][steps][QR], [L][steps][2 Ia])
+  const float* tm_mod;
+  const float* tm_bqkv;
+  const float* tm_bgu;
+  int tm_R;
 };
 
 __device__ __forceinline__ void pd_geom(const PdArgs& a, int ph, int& tiles, int& nkb, int& rows_pl) {
@@ -312,11 +319,13 @@ __device__ __noinline__ uint32_t pd_stage_attn_out(const PdArgs& a, uint8_t* sme
   return par ^ 1u;
 }
 
-// (E) SwiGLU of the gate/up sums with 1/rms of the MLP norm
-template <int kT>
+// (E) SwiGLU of the gate/up sums with 1/rms of the MLP norm (kMod: plus the feature bias `bias`, the
+// modulated norm's shift through the gate/up weights, in the interleaved column order)
+template <int kT, bool kMod = false>
 __device__ __noinline__ uint32_t pd_stage_swiglu(const PdArgs& a, uint8_t* smem, int ct, int p0, int np, int nkb,
                                                  unsigned long long* mk, uint64_t* btf, uint64_t* sbar, uint32_t par,
-                                                 const CUtensorMap* map_gu, volatile int* abort_flag) {
+                                                 const CUtensorMap* map_gu, volatile int* abort_flag,
+                                                 const float* bias = nullptr) {
   using SM = PdSmem;
   const int T = kT > 0 ? kT : a.T;   // tokens; a compile-time constant for the common shape
   const int c8 = ct & 7;
@@ -345,8 +354,14 @@ __device__ __noinline__ uint32_t pd_stage_swiglu(const PdArgs& a, uint8_t* smem,
       const float gg[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
       const float uu[8] = {ua.x, ua.y, ua.z, ua.w, ub.x, ub.y, ub.z, ub.w};
       float y[8];
+      if constexpr (kMod) {
+        const float* bg = bias + 128 * ((p0 + i) % nkb) + c8 * 8;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) y[e] = silu_f(gg[e] * s) * (uu[e] * s);
+        for (int e = 0; e < 8; ++e) y[e] = silu_f(gg[e] * s + __ldg(bg + e)) * (uu[e] * s + __ldg(bg + 64 + e));
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) y[e] = silu_f(gg[e] * s) * (uu[e] * s);
+      }
       *reinterpret_cast<uint4*>(smem + SM::kOffWork + i * SM::kBTile + sw_chunk(t, c8)) = pack8(y);
     }
     pd_pair_ready(btf, i, ct);
@@ -359,10 +374,13 @@ __device__ __noinline__ uint32_t pd_stage_swiglu(const PdArgs& a, uint8_t* smem,
 // [64 + 8 c8, ...) sit in one thread; a row's 8 units are adjacent lanes, so the head's sum of
 // squares is a 3-step shuffle.  kv = false: Q rows into the Q tile; kv = true: K rows 0..63 and V
 // rows 64..127, written in the SW128 tile layout to `kv_out` (global) instead of shared memory.
-template <int kT>
+// kMod: the sums first become acc / rms + bias (`bias` = this step's and layer's shift through the QKV
+// weights), and the head RMSNorm is taken over that.
+template <int kT, bool kMod = false>
 __device__ __noinline__ uint32_t pd_stage_qkv(const PdArgs& a, uint8_t* smem, int ct, int l, int kvg, bool kv,
                                               __nv_bfloat16* kv_out, unsigned long long* mk, uint64_t* sbar,
-                                              uint32_t par, const CUtensorMap* map_qkv, volatile int* abort_flag) {
+                                              uint32_t par, const CUtensorMap* map_qkv, volatile int* abort_flag,
+                                              const float* bias = nullptr) {
   using SM = PdSmem;
   const int T = kT > 0 ? kT : a.T;   // tokens; a compile-time constant for the common shape
   const int c8 = ct & 7;
@@ -411,13 +429,39 @@ __device__ __noinline__ uint32_t pd_stage_qkv(const PdArgs& a, uint8_t* smem, in
 #pragma unroll
       for (int e = 0; e < 16; ++e) x[e] = 0.f;
     }
+    if constexpr (kMod) {   // x <- x / rms + bias before the head norm
+      if (valid) {
+        const float s = rsqrtf(sq[t] * inv_Ha + a.eps);
+        const int col = kv ? qd + which * kvd + kvg * 128 : (kvg * G + r / T) * 128;
+        const float* bb = bias + col + c8 * 8;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          x[e] = x[e] * s + __ldg(bb + e);
+          x[8 + e] = x[8 + e] * s + __ldg(bb + 64 + e);
+        }
+      }
+    }
     float ss = 0.f;
 #pragma unroll
     for (int e = 0; e < 16; ++e) ss += x[e] * x[e];
     ss += __shfl_xor_sync(0xffffffffu, ss, 1);
     ss += __shfl_xor_sync(0xffffffffu, ss, 2);
     ss += __shfl_xor_sync(0xffffffffu, ss, 4);
-    if (valid) {
+    if (kMod && valid) {
+      if (!(kv && which == 1)) {   // Q / K: RMSNorm over the head of the biased values, RoPE at P + t
+        const float* gain = kv ? sgk : sgq;
+        const float rn = rsqrtf(ss / 128.f + a.eps);
+        const float2* cs = srope + t * 64 + c8 * 8;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int d = c8 * 8 + e;
+          const float2 c2 = cs[e];
+          const float x0 = x[e] * rn * gain[d], x1 = x[8 + e] * rn * gain[d + 64];
+          x[e] = x0 * c2.x - x1 * c2.y;
+          x[8 + e] = x1 * c2.x + x0 * c2.y;
+        }
+      }
+    } else if (valid) {
       const float s = rsqrtf(sq[t] * inv_Ha + a.eps);
       if (kv && which == 1) {   // V: 1/rms only
 #pragma unroll
@@ -449,18 +493,32 @@ __device__ __noinline__ uint32_t pd_stage_qkv(const PdArgs& a, uint8_t* smem, in
   return par ^ 1u;
 }
 
-// step boundary of token blockIdx.x (velocity, Euler update, next input), out of line
+// step boundary of token blockIdx.x (velocity, Euler update, next input), out of line; kMod: the
+// final norm's 1 + scale and shift of step k_out, the first attention norm's 1 + scale of step k_in,
+// no time embedding
+template <bool kMod = false>
 __device__ __noinline__ void pd_step(const PdArgs& a, int k_out, int k_in, int ct, float* sx, float* sred, float* hs) {
   StepArgs s = a.step;
   s.k_out = k_out;
   s.k_in = k_in;
-  step_token(s, blockIdx.x, ct, kPdCompute, sx, sred, hs, [] { named_bar_sync(1, kPdCompute); });
+  if constexpr (kMod) {
+    const float* fin = a.tm_mod + static_cast<size_t>(k_out >= 0 ? k_out : 0) * a.tm_R + 6 * a.L * a.Ha;
+    s.final_norm = fin;
+    if (k_in >= 0) s.attn_norm0 = a.tm_mod + static_cast<size_t>(k_in) * a.tm_R;
+    step_token<true>(s, blockIdx.x, ct, kPdCompute, sx, sred, hs, [] { named_bar_sync(1, kPdCompute); }, fin + a.Ha);
+  } else {
+    step_token(s, blockIdx.x, ct, kPdCompute, sx, sred, hs, [] { named_bar_sync(1, kPdCompute); });
+  }
 }
 
 // the 50-token chunk of one observation gets staging code with the token count folded in; the value
 // is the stage barrier's next parity
 #define PD_STAGE(fn, ...) (a.T == 50 ? fn<50>(__VA_ARGS__) : fn<0>(__VA_ARGS__))
+#define PD_STAGE_M(fn, ...) (a.T == 50 ? fn<50, kMod>(__VA_ARGS__) : fn<0, kMod>(__VA_ARGS__))
 
+// kMod: the time-modulated action expert (per-step gains, feature biases, gates and final norm from the
+// tables in PdArgs); false compiles the DM0 expert.
+template <bool kMod = false>
 __global__ void __launch_bounds__(kPdThreads, 1)
     denoise_persistent_kernel(const __grid_constant__ CUtensorMap tmQKV, const __grid_constant__ CUtensorMap tmO,
                               const __grid_constant__ CUtensorMap tmGU, const __grid_constant__ CUtensorMap tmD,
@@ -846,7 +904,8 @@ __global__ void __launch_bounds__(kPdThreads, 1)
     // accumulator segments -> fp32 tile [64 tokens][128 features] per segment in shared memory, then
     // one TMA bulk reduce-add per segment into dst[t][feature]; this thread: feature row r, tokens
     // [32 half, 32 half + 32)
-    auto reduce_out = [&](int p0, int p1, int nkb, const CUtensorMap* map) -> bool {
+    // gate (kMod, residual phases only): per output feature, applied to the partial tile before the add
+    auto reduce_out = [&](int p0, int p1, int nkb, const CUtensorMap* map, const float* gate) -> bool {
       const int tt0 = p0 / nkb, nseg = (p1 - 1) / nkb - tt0 + 1;
       bool good = true;
       // the reduce tiles reuse the landing area of the operand copies: every warp must be done
@@ -866,6 +925,13 @@ __global__ void __launch_bounds__(kPdThreads, 1)
         for (int hc = half; hc < 2; hc += kPdHalves) {
           float v[32];
           tmem_ld32(tl + seg * 64 + hc * 32, v);
+          if constexpr (kMod) {
+            if (gate) {
+              const float gv = __ldg(gate + (tt0 + seg) * 128 + r);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] *= gv;
+            }
+          }
 #pragma unroll
           for (int j = 0; j < 32; ++j) rt[(hc * 32 + j) * 128 + r] = v[j];
         }
@@ -885,14 +951,20 @@ __global__ void __launch_bounds__(kPdThreads, 1)
       return good;
     };
     auto step_phase = [&](int k_out, int k_in) {
-      if (static_cast<int>(blockIdx.x) < a.T) pd_step(a, k_out, k_in, ct, sx, sred, reinterpret_cast<float*>(smem + SM::kOffLandG));
+      if (static_cast<int>(blockIdx.x) < a.T)
+        pd_step<kMod>(a, k_out, k_in, ct, sx, sred, reinterpret_cast<float*>(smem + SM::kOffLandG));
+    };
+    // kMod tables of step k, layer l
+    auto mod_row = [&](int k, int l) { return a.tm_mod + static_cast<size_t>(k) * a.tm_R + 6 * l * a.Ha; };
+    auto qkv_bias = [&](int k, int l) {
+      return kMod ? a.tm_bqkv + (static_cast<size_t>(l) * a.steps + k) * a.QR : nullptr;
     };
     // ---- attention of one (KV head, key split) item
-    auto attention = [&](int l) -> bool {
+    auto attention = [&](int l, int k) -> bool {
       const PdLayer& ly = a.layers[l];
       const int GT = G * a.T;
-      stage_par = PD_STAGE(pd_stage_qkv, a, smem, ct, l, kvg, false, nullptr, mk_row(), stage_bar, stage_par,
-                           &tmQKVLd, abort_flag);
+      stage_par = PD_STAGE_M(pd_stage_qkv, a, smem, ct, l, kvg, false, nullptr, mk_row(), stage_bar, stage_par,
+                             &tmQKVLd, abort_flag, qkv_bias(k, l));
       fence_async_smem();
       tc_fence_before();
       __syncwarp();
@@ -1020,11 +1092,11 @@ __global__ void __launch_bounds__(kPdThreads, 1)
         for (int ph = 0; ok && ph < 5; ++ph) {
           mark(0);
           if (ph == 1) {
-            if (has_item && !attention(l)) *abort_flag = 1;
+            if (has_item && !attention(l, k)) *abort_flag = 1;
             if (kv_helper) {
               const int g = blockIdx.x - n_items;
-              stage_par = PD_STAGE(pd_stage_qkv, a, smem, ct, l, g, true, a.kv_sfx + static_cast<size_t>(g) * 16384,
-                                   mk_row(), stage_bar, stage_par, &tmQKVLd, abort_flag);
+              stage_par = PD_STAGE_M(pd_stage_qkv, a, smem, ct, l, g, true, a.kv_sfx + static_cast<size_t>(g) * 16384,
+                                     mk_row(), stage_bar, stage_par, &tmQKVLd, abort_flag, qkv_bias(k, l));
               csync();
               if (ct == 0) {
                 __threadfence();
@@ -1040,10 +1112,14 @@ __global__ void __launch_bounds__(kPdThreads, 1)
           pd_range(tiles * nkb, blockIdx.x, gridDim.x, p0, p1);
           const int np = p1 - p0;
           if (np > 0) {
-            if (ph == 0) stage_par = PD_STAGE(pd_stage_norm, a, smem, ct, p0, np, nkb, ly.attn_norm, ssq_attn, mk_row(), btile_full, stage_bar, stage_par, &tmHLd, abort_flag);
+            // kMod: the norms' gains are this step's 1 + scale rows
+            const float* g_attn = kMod ? mod_row(k, l) : ly.attn_norm;
+            const float* g_mlp = kMod ? mod_row(k, l) + 3 * a.Ha : ly.mlp_norm;
+            if (ph == 0) stage_par = PD_STAGE(pd_stage_norm, a, smem, ct, p0, np, nkb, g_attn, ssq_attn, mk_row(), btile_full, stage_bar, stage_par, &tmHLd, abort_flag);
             else if (ph == 2) stage_par = PD_STAGE(pd_stage_attn_out, a, smem, ct, p0, np, nkb, mk_row(), btile_full, stage_bar, stage_par, &tmPO, &tmML, abort_flag);
-            else if (ph == 3) stage_par = PD_STAGE(pd_stage_norm, a, smem, ct, p0, np, nkb, ly.mlp_norm, ssq_mlp, mk_row(), btile_full, stage_bar, stage_par, &tmHLd, abort_flag);
-            else stage_par = PD_STAGE(pd_stage_swiglu, a, smem, ct, p0, np, nkb, mk_row(), btile_full, stage_bar, stage_par, &tmGULd, abort_flag);
+            else if (ph == 3) stage_par = PD_STAGE(pd_stage_norm, a, smem, ct, p0, np, nkb, g_mlp, ssq_mlp, mk_row(), btile_full, stage_bar, stage_par, &tmHLd, abort_flag);
+            else stage_par = PD_STAGE_M(pd_stage_swiglu, a, smem, ct, p0, np, nkb, mk_row(), btile_full, stage_bar, stage_par, &tmGULd, abort_flag,
+                                        kMod ? a.tm_bgu + (static_cast<size_t>(l) * a.steps + k) * 2 * a.Ia : nullptr);
             mark(1);
           }
           // scratch of the other half of the layer, idle in this phase
@@ -1056,7 +1132,8 @@ __global__ void __launch_bounds__(kPdThreads, 1)
           }
           if (np > 0) {
             const CUtensorMap* map = ph == 0 ? &tmAccQKV : (ph == 3 ? &tmAccGU : &tmH);
-            if (!reduce_out(p0, p1, nkb, map)) *abort_flag = 1;
+            const float* gate = kMod && (ph == 2 || ph == 4) ? mod_row(k, l) + (ph == 2 ? 2 : 5) * a.Ha : nullptr;
+            if (!reduce_out(p0, p1, nkb, map, gate)) *abort_flag = 1;
           }
           mark(3);
           ok = grid_sync();

@@ -848,13 +848,15 @@ bool persist_plan(dm0_ctx* c, int steps, float* vel, dm0::PdArgs* a, std::string
     return false;
   };
   if (!c->use_persist) return no("disabled");
-  if (g.time_mod) return no("time-modulated expert");
   if (c->persist_resident < 0) {   // once per context: can one CTA of the kernel live on every SM?
     int per_sm = 0, coop = 0;
     cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, c->device);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dm0::denoise_persistent_kernel, dm0::kPdThreads,
-                                                      dm0::PdSmem::kBytes) != cudaSuccess)
-      per_sm = 0;
+    const cudaError_t oe =
+        g.time_mod ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dm0::denoise_persistent_kernel<true>,
+                                                                   dm0::kPdThreads, dm0::PdSmem::kBytes)
+                   : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dm0::denoise_persistent_kernel<false>,
+                                                                   dm0::kPdThreads, dm0::PdSmem::kBytes);
+    if (oe != cudaSuccess) per_sm = 0;
     cudaGetLastError();
     c->persist_resident = (coop && per_sm >= 1) ? 1 : 0;
   }
@@ -927,6 +929,12 @@ bool persist_plan(dm0_ctx* c, int steps, float* vel, dm0::PdArgs* a, std::string
   st.eps = g.rms_eps;
   st.steps = steps;
   st.vel = vel;
+  if (g.time_mod) {   // the tables tmod_precompute fills before the launch
+    a->tm_mod = c->tm_mod;
+    a->tm_bqkv = c->tm_bqkv;
+    a->tm_bgu = c->tm_bgu;
+    a->tm_R = (6 * g.layers + 2) * g.hidden_a;
+  }
   return true;
 }
 
@@ -970,6 +978,7 @@ dm0_status enqueue_denoise_persistent(dm0_ctx* c, cudaStream_t s, const dm0::PdA
             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(c, DM0_ECUDA, "cuTensorMapEncodeTiled (partial max/sum) failed (" + std::to_string(r) + ")");
   }
+  if (g.time_mod) TRY(tmod_precompute(c, s, a.steps));
   CK(cudaMemsetAsync(c->psync, 0, (2 + g.n_kv) * sizeof(unsigned), s));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(c->num_sms);
@@ -982,8 +991,11 @@ dm0_status enqueue_denoise_persistent(dm0_ctx* c, cudaStream_t s, const dm0::PdA
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const int e0 = probe_begin(c, s, DM0_SITE_LOOP);
-  const cudaError_t le = cudaLaunchKernelEx(&cfg, dm0::denoise_persistent_kernel, tq, to, tgu, td, tk, tv, tacc_qkv, th,
-                                            tacc_gu, th_ld, tgu_ld, tqkv_ld, tpo, tml, a);
+  const cudaError_t le =
+      g.time_mod ? cudaLaunchKernelEx(&cfg, dm0::denoise_persistent_kernel<true>, tq, to, tgu, td, tk, tv, tacc_qkv, th,
+                                      tacc_gu, th_ld, tgu_ld, tqkv_ld, tpo, tml, a)
+                 : cudaLaunchKernelEx(&cfg, dm0::denoise_persistent_kernel<false>, tq, to, tgu, td, tk, tv, tacc_qkv,
+                                      th, tacc_gu, th_ld, tgu_ld, tqkv_ld, tpo, tml, a);
   if (le == cudaErrorCooperativeLaunchTooLarge) {   // fewer SMs available than the device has: use the
     cudaGetLastError();                             // per-layer kernels from now on
     c->persist_resident = 0;
@@ -997,6 +1009,8 @@ dm0_status enqueue_denoise_persistent(dm0_ctx* c, cudaStream_t s, const dm0::PdA
 }
 
 dm0_status denoise_from_x(dm0_ctx* c, cudaStream_t s, int steps, float* vel) {
+  // the time-modulation tables are allocated outside any capture (an allocation may synchronise)
+  if (c->cfg.time_mod) TRY(tmod_tables(c, steps));
   {
     dm0::PdArgs pa;
     std::string why;
@@ -1005,8 +1019,6 @@ dm0_status denoise_from_x(dm0_ctx* c, cudaStream_t s, int steps, float* vel) {
       if (!(st == DM0_ESTATE && c->persist_resident == 0)) return st;   // else fall through
     }
   }
-  // the time-modulation tables are allocated outside any capture (an allocation may synchronise)
-  if (c->cfg.time_mod) TRY(tmod_tables(c, steps));
   if (vel || !c->use_graph || c->probe_mask) return enqueue_denoise(c, s, steps, vel);
   const auto key = std::make_tuple(c->kv_B, c->kv_P, steps);
   auto it = c->graphs.find(key);
@@ -1623,7 +1635,8 @@ dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
             smem_attr(dm0::attn_kernel<32>, dm0::AttnSmem<32>::kBytes) &&
             smem_attr(dm0::fa_tc_kernel<2, 1>, dm0::FaSmemT<2, 1>::kBytes) &&
             smem_attr(dm0::fa_tc_kernel<dm0::kFaDeepStages, 2>, dm0::FaSmemT<dm0::kFaDeepStages, 2>::kBytes) &&
-            smem_attr(dm0::denoise_persistent_kernel, dm0::PdSmem::kBytes) &&
+            smem_attr(dm0::denoise_persistent_kernel<false>, dm0::PdSmem::kBytes) &&
+            smem_attr(dm0::denoise_persistent_kernel<true>, dm0::PdSmem::kBytes) &&
             smem_attr(dm0::train_attn_fwd_kernel, 100 * 1024) && smem_attr(dm0::train_attn_bwd_kernel, 200 * 1024);
   if (!ok) return bail(DM0_ECUDA);
   *out = c;
