@@ -135,3 +135,18 @@ def test_fp8_prefill_reduces_to_the_bf16_prefill_with_an_exact_quantiser():
     _, _, hq = O.prefill_fp8(w, emb)
     rel = np.sqrt(np.mean((hq - h) ** 2)) / np.sqrt(np.mean(h ** 2))
     assert 1e-5 < rel < 0.05     # E4M3 noise on the MLP branch only, not a wiring error
+
+
+def test_merged_layer_fp8_switch_touches_only_the_vlm_mlp():
+    from synth import inputs as I
+    d = I.TINY
+    w = I.Weights(d, seed=0, gain_jitter=0.1)
+    hp, hs = I.hidden_states(24, d.hidden_v, seed=1), I.hidden_states(d.chunk, d.hidden_a, seed=2)
+    ref = O.merged_layer(w.layer(0, 0), w.layer(1, 0), hp, hs, d)
+    ident = lambda m: (np.asarray(m, np.float64), np.ones((np.shape(m)[0], 1)))   # noqa: E731
+    same = O.merged_layer(w.layer(0, 0), w.layer(1, 0), hp, hs, d, vlm_fp8=ident)
+    for a, b in zip(same, ref):
+        assert np.max(np.abs(a - b)) <= 1e-12 * np.max(np.abs(b))
+    q = O.merged_layer(w.layer(0, 0), w.layer(1, 0), hp, hs, d, vlm_fp8=True)
+    assert np.array_equal(q[1], ref[1]) and np.array_equal(q[2], ref[2]) and np.array_equal(q[3], ref[3])
+    assert not np.allclose(q[0], ref[0], rtol=0, atol=1e-6)
