@@ -115,6 +115,9 @@ struct PdArgs {
   const float* tm_bqkv;
   const float* tm_bgu;
   int tm_R;
+  // grid barrier arrival as one release reduction (red.release.gpu) and no fence after the acquire
+  // spin, instead of a full fence, an atomic add, the spin and a second full fence
+  int fast_bar;
 };
 
 __device__ __forceinline__ void pd_geom(const PdArgs& a, int ph, int& tiles, int& nkb, int& rows_pl) {
@@ -872,9 +875,13 @@ __global__ void __launch_bounds__(kPdThreads, 1)
       named_bar_sync(1, kPdCompute);
       ++gen;
       if (ct == 0 && *abort_flag == 0) {
-        __threadfence();
+        // the CTA barrier above orders every thread's writes before this thread's release (cumulativity)
+        if (!a.fast_bar) __threadfence();
         if (a.trace) a.trace[(static_cast<size_t>(gen - 1) * gridDim.x + blockIdx.x) * kPdTraceSlots + 4] = globaltimer();
-        atomicAdd(a.sync, 1u);
+        if (a.fast_bar)
+          asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(a.sync), "r"(1u) : "memory");
+        else
+          atomicAdd(a.sync, 1u);
         if (a.trace) a.trace[(static_cast<size_t>(gen - 1) * gridDim.x + blockIdx.x) * kPdTraceSlots + 5] = globaltimer();
         const unsigned target = gen * gridDim.x;
         const uint64_t t0 = globaltimer();
@@ -887,7 +894,7 @@ __global__ void __launch_bounds__(kPdThreads, 1)
             }
           }
         }
-        __threadfence();
+        if (!a.fast_bar) __threadfence();   // else: the acquire load orders what follows, the CTA barrier below the rest
       }
       if (ct == 0 && *abort_flag) atomicExch(a.sync + 1, 1u);   // release the other CTAs at once
       named_bar_sync(1, kPdCompute);

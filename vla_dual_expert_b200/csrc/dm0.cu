@@ -94,6 +94,7 @@ struct dm0_ctx {
   // per-layer kernels instead); DM0_PERSIST_SPLITS overrides its attention key splits per KV head
   bool use_persist = true;
   int persist_splits = 7;
+  bool persist_fast_bar = false;   // DM0_PERSIST_FASTBAR=1: release-reduction grid barrier arrival
   int persist_resident = -1;   // -1: not checked yet
   // true when the previous operation this context queued on the stream was one of its own
   // kernels: only then may the next kernel overlap it (programmatic dependent launch).  The first
@@ -929,6 +930,7 @@ bool persist_plan(dm0_ctx* c, int steps, float* vel, dm0::PdArgs* a, std::string
   st.eps = g.rms_eps;
   st.steps = steps;
   st.vel = vel;
+  a->fast_bar = c->persist_fast_bar ? 1 : 0;
   if (g.time_mod) {   // the tables tmod_precompute fills before the launch
     a->tm_mod = c->tm_mod;
     a->tm_bqkv = c->tm_bqkv;
@@ -1481,6 +1483,7 @@ dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
   if (const char* e = std::getenv("DM0_NO_GRAPH")) c->use_graph = e[0] == '0';
   if (const char* e = std::getenv("DM0_NO_PERSIST")) c->use_persist = e[0] == '0';
   if (const char* e = std::getenv("DM0_PERSIST_SPLITS")) c->persist_splits = std::max(1, std::atoi(e));
+  if (const char* e = std::getenv("DM0_PERSIST_FASTBAR")) c->persist_fast_bar = e[0] == '1';
 
   // weights: one allocation, 256-byte aligned sub-buffers
   size_t total = 0;
