@@ -1291,7 +1291,7 @@ dm0_status train_layer_fwd(dm0_ctx* c, cudaStream_t s, int l, const float* hin, 
   at.prob = b.prob;
   at.of = b.of;
   at.of_bf = b.of_bf;
-  const size_t fsm = sizeof(float) * (static_cast<size_t>(S) * D + 32 * D + S * 32);
+  const size_t fsm = sizeof(float) * (static_cast<size_t>(S) * D + 32 * (D + 1) + S * 32);
   TRY(launch(c, s, dm0::train_attn_fwd_kernel, dim3(B * g.n_q), dim3(256), fsm, at));
   TRY(gemm_f32(c, s, b.of_bf, T, HqD, w.wo, H, b.tmp));
   const size_t nh = static_cast<size_t>(T) * H;
@@ -1428,7 +1428,7 @@ dm0_status enqueue_train(dm0_ctx* c, cudaStream_t s, const float* a, const float
     at.dqr = b.dqr;
     at.dK = b.dK;
     at.dV = b.dV;
-    const size_t bsm = sizeof(float) * (2 * static_cast<size_t>(S) * D + 2 * 32 * D + 2 * S * 32 + S);
+    const size_t bsm = sizeof(float) * (2 * static_cast<size_t>(S) * D + 2 * 32 * (D + 1) + 2 * S * 32 + S);
     TRY(launch(c, s, dm0::train_attn_bwd_kernel, dim3(B * g.n_q), dim3(256), bsm, at));
     const int qk_warps = T * (g.n_q + 2 * g.n_kv);
     TRY(launch(c, s, dm0::train_qk_bwd_kernel, dim3((qk_warps + 7) / 8), dim3(256), 0, static_cast<const float*>(b.raw),

@@ -306,7 +306,7 @@ __global__ void __launch_bounds__(256) train_deinterleave_kernel(const float* dg
 // Merged attention of the training step, one CTA per (sample, query head), all S query rows: scores
 // against the sample's [prefix cache (bf16); suffix keys (fp32)] keys, softmax (fp32), probabilities
 // kept in prob [B][Hq][S][P + S], o = prob V in fp32 and bf16.  Shared memory: q [S][D], a 32-key
-// tile [32][D], a probability tile [S][32].
+// tile [32][D + 1], a probability tile [S][32].
 struct TrainAttn {
   const float *qr, *kr, *vs;          // [T][Hq D], [T][Hkv D], [T][Hkv D]
   const __nv_bfloat16 *kc, *vc;       // [B][Hkv][P][D] prefix cache
@@ -321,8 +321,10 @@ struct TrainAttn {
   float *dK, *dV;                     // [B][Hkv][P + S][D], accumulated (zeroed by the caller)
 };
 
+// key / value tiles are [32][D + 1]: the padding puts the 32 keys a warp reads at one dimension in 32
+// different banks
 __device__ __forceinline__ void train_load_keys(const TrainAttn& a, bool values, int b, int g, int k0, float* tile) {
-  const int N = a.P + a.S;
+  const int N = a.P + a.S, KP = a.D + 1;
   for (int idx = threadIdx.x; idx < 32 * a.D; idx += blockDim.x) {
     const int kk = idx / a.D, d = idx - (idx / a.D) * a.D, k = k0 + kk;
     float v = 0.f;
@@ -330,7 +332,7 @@ __device__ __forceinline__ void train_load_keys(const TrainAttn& a, bool values,
       v = __bfloat162float((values ? a.vc : a.kc)[((static_cast<size_t>(b) * a.Hkv + g) * a.P + k) * a.D + d]);
     else if (k < N)
       v = (values ? a.vs : a.kr)[(static_cast<size_t>(b * a.S + k - a.P) * a.Hkv + g) * a.D + d];
-    tile[kk * a.D + d] = v;
+    tile[kk * KP + d] = v;
   }
 }
 
@@ -339,10 +341,10 @@ __global__ void __launch_bounds__(256) train_attn_fwd_kernel(const TrainAttn a) 
   pdl_wait();
   extern __shared__ float sm[];
   const int b = blockIdx.x / a.Hq, h = blockIdx.x - (blockIdx.x / a.Hq) * a.Hq, g = h / (a.Hq / a.Hkv);
-  const int S = a.S, D = a.D, N = a.P + a.S;
+  const int S = a.S, D = a.D, N = a.P + a.S, KP = D + 1;
   float* sq = sm;                // [S][D]
-  float* st = sq + S * D;        // [32][D]
-  float* sp = st + 32 * D;       // [S][32]
+  float* st = sq + S * D;        // [32][D + 1]
+  float* sp = st + 32 * KP;      // [S][32]
   float* prob = a.prob + (static_cast<size_t>(b) * a.Hq + h) * S * N;
   for (int idx = threadIdx.x; idx < S * D; idx += blockDim.x) {
     const int s = idx / D, d = idx - (idx / D) * D;
@@ -357,7 +359,7 @@ __global__ void __launch_bounds__(256) train_attn_fwd_kernel(const TrainAttn a) 
       const int s = idx >> 5, kk = idx & 31;
       if (k0 + kk >= N) continue;
       float acc = 0.f;
-      for (int d = 0; d < D; ++d) acc += sq[s * D + d] * st[kk * D + d];
+      for (int d = 0; d < D; ++d) acc += sq[s * D + d] * st[kk * KP + d];
       prob[static_cast<size_t>(s) * N + k0 + kk] = acc * a.scale;
     }
   }
@@ -400,7 +402,7 @@ __global__ void __launch_bounds__(256) train_attn_fwd_kernel(const TrainAttn a) 
       if (idx >= S * D) break;
       const int s = idx / D, d = idx - (idx / D) * D;
       float v = 0.f;
-      for (int kk = 0; kk < 32; ++kk) v += sp[s * 32 + kk] * st[kk * D + d];
+      for (int kk = 0; kk < 32; ++kk) v += sp[s * 32 + kk] * st[kk * KP + d];
       acc[i] += v;
     }
   }
@@ -417,19 +419,19 @@ __global__ void __launch_bounds__(256) train_attn_fwd_kernel(const TrainAttn a) 
 
 // Backward of train_attn_fwd, one CTA per (sample, query head): delta_s = sum_d dO O;
 // dS = prob (dO V^T - delta) scale; dq = dS K; dK += dS^T q; dV += prob^T dO (atomically: the query
-// heads of a group share their KV head).  Shared memory: q, dO [S][D], K and V tiles [32][D], the dS
-// and probability tiles [S][32], delta [S].
+// heads of a group share their KV head).  Shared memory: q, dO [S][D], K and V tiles [32][D + 1], the
+// dS and probability tiles [S][32], delta [S].
 __global__ void __launch_bounds__(256) train_attn_bwd_kernel(const TrainAttn a) {
   pdl_launch_dependents();
   pdl_wait();
   extern __shared__ float sm[];
   const int b = blockIdx.x / a.Hq, h = blockIdx.x - (blockIdx.x / a.Hq) * a.Hq, g = h / (a.Hq / a.Hkv);
-  const int S = a.S, D = a.D, N = a.P + a.S;
+  const int S = a.S, D = a.D, N = a.P + a.S, KP = D + 1;
   float* sq = sm;                 // [S][D]
   float* sdo = sq + S * D;        // [S][D]
-  float* sk = sdo + S * D;        // [32][D]
-  float* sv = sk + 32 * D;        // [32][D]
-  float* sds = sv + 32 * D;       // [S][32]
+  float* sk = sdo + S * D;        // [32][D + 1]
+  float* sv = sk + 32 * KP;       // [32][D + 1]
+  float* sds = sv + 32 * KP;      // [S][32]
   float* sp = sds + S * 32;       // [S][32]
   float* sdelta = sp + S * 32;    // [S]
   const float* prob = a.prob + (static_cast<size_t>(b) * a.Hq + h) * S * N;
@@ -464,7 +466,7 @@ __global__ void __launch_bounds__(256) train_attn_bwd_kernel(const TrainAttn a) 
       if (k0 + kk < N) {
         p = prob[static_cast<size_t>(s) * N + k0 + kk];
         float dp = 0.f;
-        for (int d = 0; d < D; ++d) dp += sdo[s * D + d] * sv[kk * D + d];
+        for (int d = 0; d < D; ++d) dp += sdo[s * D + d] * sv[kk * KP + d];
         ds = p * (dp - sdelta[s]) * a.scale;
       }
       sp[idx] = p;
@@ -477,7 +479,7 @@ __global__ void __launch_bounds__(256) train_attn_bwd_kernel(const TrainAttn a) 
       if (idx >= S * D) break;
       const int s = idx / D, d = idx - (idx / D) * D;
       float v = 0.f;
-      for (int kk = 0; kk < 32; ++kk) v += sds[s * 32 + kk] * sk[kk * D + d];
+      for (int kk = 0; kk < 32; ++kk) v += sds[s * 32 + kk] * sk[kk * KP + d];
       dq[i] += v;
     }
     for (int idx = threadIdx.x; idx < 32 * D; idx += blockDim.x) {
