@@ -562,7 +562,6 @@ __global__ void __launch_bounds__(kPdThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = a.n_q / a.n_kv;
-  const int qd = a.n_q * 128, kvd = a.n_kv * 128;
   const int nA = (a.P + 63) >> 6;                 // prefix blocks; block nA is the suffix
   const int n_items = a.n_kv * a.splits;
   const bool has_item = static_cast<int>(blockIdx.x) < n_items;
@@ -846,7 +845,6 @@ __global__ void __launch_bounds__(kPdThreads, 1)
     const int half = (warp - 2) >> 2;                // 0: warps 2-5, 1: warps 6-9 (when present)
     const int r = lane_base + lane;                  // TMEM lane owned by this thread
     const uint32_t tl = tmem + (static_cast<uint32_t>(lane_base) << 16);
-    const float inv_Ha = 1.0f / a.Ha;
     float* ssq_attn = a.ssq;
     float* ssq_mlp = a.ssq + a.T;
     uint32_t gen = 0, acc_use[2] = {0u, 0u}, blk = 0, stage_par = 0;
@@ -968,7 +966,6 @@ __global__ void __launch_bounds__(kPdThreads, 1)
     };
     // ---- attention of one (KV head, key split) item
     auto attention = [&](int l, int k) -> bool {
-      const PdLayer& ly = a.layers[l];
       const int GT = G * a.T;
       stage_par = PD_STAGE_M(pd_stage_qkv, a, smem, ct, l, kvg, false, nullptr, mk_row(), stage_bar, stage_par,
                              &tmQKVLd, abort_flag, qkv_bias(k, l));
