@@ -125,6 +125,17 @@ dm0_status dm0_load_weights(dm0_ctx* ctx, const void* blob, size_t bytes);
  * Returns DM0_ESHAPE unless 1 <= B <= max_batch and 1 <= P <= max_prefix. */
 dm0_status dm0_prefill(dm0_ctx* ctx, const void* prefix_emb, int B, int P, void* stream);
 
+/* Shape buckets: make dm0_denoise for (B, P, steps) ready ahead of time, so a
+ * later call of that shape does no capture.  Where the Euler loop runs as
+ * per-layer kernels (B >= 2, or the persistent kernel unavailable) this
+ * captures and caches its CUDA graph without launching anything; the
+ * single-observation persistent loop takes B, P and steps as launch arguments
+ * and needs nothing.  The KV cache and its committed shape are untouched.
+ * Call it outside any stream capture (it captures on the context's own
+ * stream).  Returns DM0_ESTATE without weights, DM0_ESHAPE outside the
+ * context's capacity or unless 1 <= steps <= 1000. */
+dm0_status dm0_prepare(dm0_ctx* ctx, int B, int P, int steps);
+
 /* Device pointers of the KV-cache planes (context-owned, valid until
  * dm0_destroy).  With the (B, P) of the last prefill or dm0_kv_commit, plane
  * element [l][b][h][p][d] sits at index (((l*B + b)*n_kv + h)*P + p)*head_dim + d.

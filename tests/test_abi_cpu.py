@@ -140,3 +140,8 @@ def test_gradient_buffer_layout_matches_the_oracle_parameters(dims):
         assert tuple(shape) == np.shape(ref), key
     g = abi.unpack_grads(np.arange(n, dtype=np.float32), dims)
     assert g[(0, "attn_norm")][0] == 0 and g[("head", "b_out")][-1] == n - 1
+
+
+def test_prepare_rejects_a_null_context():
+    _, lib = _lib()
+    assert lib.dm0_prepare(None, 1, 64, 10) == -1

@@ -1,0 +1,47 @@
+"""dm0_prepare: shape buckets made ready ahead of time (the pages' fixed shapes per captured graph,
+several prefix lengths and step counts without a capture at request time).  A prepared bucket's
+denoise matches an unprepared engine's, preparing launches nothing, and preparing another shape
+leaves the committed cache shape alone.  Awaits its first GPU run (DM0_RUN_PREPARE=1)."""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from synth import inputs as I
+from tests.gpu_util import host, rel_err, to_dev_bf16
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(os.environ.get("DM0_RUN_PREPARE") != "1",
+                                 reason="awaits its first GPU run (DM0_RUN_PREPARE=1)")]
+
+
+def _run(prepare):
+    from vla_dual_expert_b200 import Engine
+    d = I.TINY
+    w = I.Weights(d, seed=0, gain_jitter=0.1)
+    B, P, steps = 2, 37, 3
+    eng = Engine(d, B, 64)
+    try:
+        eng.load_from(w)
+        if prepare:
+            n0 = eng.launch_count()
+            eng.prepare(B, P, steps)
+            eng.prepare(B, 20, steps)          # another bucket: captured, the cache shape untouched
+            eng.prepare(1, 64, 5)
+            assert eng.launch_count() == n0    # nothing ran
+        eng.prefill(to_dev_bf16(I.prefix_embeddings(d, B, P)))
+        n1 = eng.launch_count()
+        out = eng.denoise(torch.from_numpy(I.noise(d, B)).cuda(), steps)
+        eng.sync()
+        assert eng.device_error() == 0
+        return host(out), eng.launch_count() - n1
+    finally:
+        eng.close()
+
+
+def test_prepared_bucket_matches_and_launches_the_same_graph():
+    x0, n0 = _run(False)
+    x1, n1 = _run(True)
+    assert n0 == n1
+    assert rel_err(x1, x0) <= 1e-5   # split-K sums may arrive in another order

@@ -101,6 +101,10 @@ class Engine:
         _check_cuda(prefix_emb, torch.bfloat16, (B, P, self.dims.hidden_v), "prefix_emb")
         self._chk(self.lib.dm0_prefill(self.h, _ptr(prefix_emb), B, P, _stream(stream)))
 
+    def prepare(self, B: int, P: int, steps: int):
+        """Capture ahead of time what dm0_denoise needs for (B, P, steps) (dm0_prepare)."""
+        self._chk(self.lib.dm0_prepare(self.h, B, P, steps))
+
     def kv_view(self):
         k, v = ctypes.c_void_p(), ctypes.c_void_p()
         self._chk(self.lib.dm0_kv_view(self.h, ctypes.byref(k), ctypes.byref(v)))

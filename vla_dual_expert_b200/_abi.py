@@ -26,7 +26,7 @@ EXPORTS = ("dm0_create", "dm0_weights_bytes", "dm0_load_weights", "dm0_prefill",
            "dm0_op_attention", "dm0_attention_noalloc", "dm0_debug_view", "dm0_launch_count", "dm0_probe",
            "dm0_probe_read", "dm0_selftest_timeout", "dm0_sync", "dm0_device_error", "dm0_clear_error", "dm0_last_error",
            "dm0_destroy", "dm0_pack_e4m3_rows", "dm0_set_prefix_fp8", "dm0_op_quant_e4m3",
-           "dm0_op_gemm_e4m3", "dm0_grad_floats", "dm0_train_step")
+           "dm0_op_gemm_e4m3", "dm0_grad_floats", "dm0_train_step", "dm0_prepare")
 
 
 class Dm0Config(ctypes.Structure):
@@ -83,6 +83,7 @@ def load_library() -> ctypes.CDLL:
         "dm0_op_quant_e4m3": (c_int, [P, P, c_int, c_int, c_int, P, P, P, P, P]),
         "dm0_op_gemm_e4m3": (c_int, [P, P, P, P, P, P, c_int, c_int, c_int, P]),
         "dm0_grad_floats": (c_size_t, [P]),
+        "dm0_prepare": (c_int, [P, c_int, c_int, c_int]),
         "dm0_train_step": (c_int, [P, P, P, P, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():

@@ -1010,18 +1010,9 @@ dm0_status enqueue_denoise_persistent(dm0_ctx* c, cudaStream_t s, const dm0::PdA
   return DM0_OK;
 }
 
-dm0_status denoise_from_x(dm0_ctx* c, cudaStream_t s, int steps, float* vel) {
-  // the time-modulation tables are allocated outside any capture (an allocation may synchronise)
-  if (c->cfg.time_mod) TRY(tmod_tables(c, steps));
-  {
-    dm0::PdArgs pa;
-    std::string why;
-    if (persist_plan(c, steps, vel, &pa, &why)) {
-      const dm0_status st = enqueue_denoise_persistent(c, s, pa);
-      if (!(st == DM0_ESTATE && c->persist_resident == 0)) return st;   // else fall through
-    }
-  }
-  if (vel || !c->use_graph || c->probe_mask) return enqueue_denoise(c, s, steps, vel);
+// The CUDA graph of the per-layer Euler loop for the context's current (kv_B, kv_P) and `steps`,
+// captured (not launched) on first use and cached
+dm0_status denoise_graph(dm0_ctx* c, int steps, const dm0_ctx::Graph** out) {
   const auto key = std::make_tuple(c->kv_B, c->kv_P, steps);
   auto it = c->graphs.find(key);
   if (it == c->graphs.end()) {
@@ -1043,8 +1034,26 @@ dm0_status denoise_from_x(dm0_ctx* c, cudaStream_t s, int steps, float* vel) {
     if (e != cudaSuccess) return fail(c, DM0_ECUDA, std::string("graph instantiate: ") + cudaGetErrorString(e));
     it = c->graphs.emplace(key, dm0_ctx::Graph{exec, nk}).first;
   }
-  CK(cudaGraphLaunch(it->second.exec, s));
-  c->launches += it->second.kernels;
+  *out = &it->second;
+  return DM0_OK;
+}
+
+dm0_status denoise_from_x(dm0_ctx* c, cudaStream_t s, int steps, float* vel) {
+  // the time-modulation tables are allocated outside any capture (an allocation may synchronise)
+  if (c->cfg.time_mod) TRY(tmod_tables(c, steps));
+  {
+    dm0::PdArgs pa;
+    std::string why;
+    if (persist_plan(c, steps, vel, &pa, &why)) {
+      const dm0_status st = enqueue_denoise_persistent(c, s, pa);
+      if (!(st == DM0_ESTATE && c->persist_resident == 0)) return st;   // else fall through
+    }
+  }
+  if (vel || !c->use_graph || c->probe_mask) return enqueue_denoise(c, s, steps, vel);
+  const dm0_ctx::Graph* gr = nullptr;
+  TRY(denoise_graph(c, steps, &gr));
+  CK(cudaGraphLaunch(gr->exec, s));
+  c->launches += gr->kernels;
   return DM0_OK;
 }
 
@@ -1441,6 +1450,28 @@ dm0_status dm0_prefill(dm0_ctx* c, const void* prefix_emb, int B, int P, void* s
   c->kv_B = B;
   c->kv_P = P;
   return DM0_OK;
+}
+
+dm0_status dm0_prepare(dm0_ctx* c, int B, int P, int steps) {
+  if (!c) return DM0_EINVAL;
+  if (!c->weights_loaded) return fail(c, DM0_ESTATE, "weights not loaded");
+  const dm0_config& g = c->cfg;
+  if (B < 1 || B > g.max_batch || P < 1 || P > g.max_prefix || steps < 1 || steps > 1000)
+    return fail(c, DM0_ESHAPE, "B, P or steps outside the context capacity");
+  if (g.time_mod) TRY(tmod_tables(c, steps));
+  const int kb = c->kv_B, kp = c->kv_P;
+  c->kv_B = B;
+  c->kv_P = P;
+  dm0_status st = DM0_OK;
+  dm0::PdArgs pa;
+  std::string why;
+  if (!persist_plan(c, steps, nullptr, &pa, &why) && c->use_graph) {   // the persistent loop needs no capture
+    const dm0_ctx::Graph* gr = nullptr;
+    st = denoise_graph(c, steps, &gr);
+  }
+  c->kv_B = kb;
+  c->kv_P = kp;
+  return st;
 }
 
 dm0_status dm0_kv_view(dm0_ctx* c, void** k, void** v) {
