@@ -323,6 +323,7 @@ def run_native(args, rank, world, local_rank):
         # probed gate/up site covers the operand quantisation and the FP8 GEMM
         eng.set_prefix_fp8(True)
         f8 = measure(wl_main, args.steps, args.warmup, probe=3)
+        f8_b1 = measure(I.WORKLOADS["e2e_b1"], max(args.steps, 5), args.warmup, probe=None)
         eng.set_prefix_fp8(False)
         f8_ms = f8["probe_ms"] / max(f8["probe_n"], 1)
         f8_tf = prefill_gateup_flops(d, B, P) / (f8_ms * 1e-3) / 1e12
@@ -334,7 +335,10 @@ def run_native(args, rank, world, local_rank):
                             "avg_ms": round(f8_ms, 4), "achieved": round(f8_tf, 1), "peak": round(fp8_peak, 1),
                             "unit": "TFLOP/s", "frac": round(f8_tf / fp8_peak, 4),
                             "peak_src": f"{peaks['src']} bf16_tflops_sustained x 2 (nominal fp8 / bf16 ratio)"},
-            "gpu_launches": f8["launches"], "clocks": f8["clocks"]}
+            "gpu_launches": f8["launches"], "clocks": f8["clocks"],
+            "batch1": {"value": round(job_chunks_per_s(world, 1, f8_b1["ms"]), 3), "unit": "chunks/s",
+                       "prefill_ms_p50": round(f8_b1["prefill_ms_p50"], 3),
+                       "denoise_ms_p50": round(f8_b1["denoise_ms_p50"], 3)}}
     if args.train:
         # one flow-matching training step over the prefix cache the timed step left (opt-in)
         a_np, e_np, t_np, m_np = I.train_batch(d, B, seed=4000 + 97 * rank)
