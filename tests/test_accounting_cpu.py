@@ -29,3 +29,11 @@ def test_denoise_bytes_per_euler_step():
 def test_gate_up_flops_of_the_batched_prefix_pass():
     assert bench.prefill_gateup_flops(D, 16, 2048) == 2 * 16 * 2048 * 2048 * 2 * 6144
     assert abs(bench.prefill_gateup_flops(D, 16, 2048) / 1e12 - 1.649) < 1e-3
+
+
+def test_merged_layer_flops():
+    # one DM0-base layer over 816 prefix + 50 suffix tokens: 83.7 GFLOP of GEMM (82.1 VLM + 1.6 action)
+    # and 5.8 GFLOP of attention (prefix rows over 816 keys, suffix rows over 866, QK^T and PV)
+    gemm, attn = bench.merged_layer_flops(D, 816, 50)
+    assert gemm == 2 * 816 * 50_331_648 + 2 * 50 * 15_728_640
+    assert round(gemm / 1e9, 1) == 83.7 and round(attn / 1e9, 1) == 5.8
