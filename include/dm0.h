@@ -287,7 +287,14 @@ dm0_status dm0_op_attention(dm0_ctx* ctx, const void* q, const void* ka, const v
  * ready, results issued, release fence done, barrier arrival, MMA warp saw the
  * operand, MMA warp issued its last MMA;
  * phase 0 is the input of step 0, then per step 5 phases per layer (QKV,
- * attention, O, gate/up, down) and the step boundary. */
+ * attention, O, gate/up, down) and the step boundary.
+ * "tm_mod", "tm_bqkv", "tm_bgu" (time_mod contexts, NULL before the first
+ * dm0_denoise or dm0_prepare): the modulation tables of the last Euler loop of
+ * K steps, f32 [K][(6*layers + 2)*hidden_a] (per layer [attention: 1 + scale |
+ * shift | gate][MLP: 1 + scale | shift | gate], then the final norm's
+ * [1 + scale | shift]), [layers][K][(n_q + 2 n_kv) head_dim] and
+ * [layers][K][2 inter_a] (the shifts through the QKV and interleaved gate/up
+ * weights). */
 dm0_status dm0_debug_view(dm0_ctx* ctx, const char* name, void** ptr);
 
 /* Merged GQA attention that allocates nothing, for callers that cannot call

@@ -158,3 +158,41 @@ def test_single_observation_runs_as_one_persistent_launch():
     check_fp(results["persistent"][0][0], rx, TOL_CHUNK, "persistent chunk")
     check_fp(results["persistent"][0][0], results["per_layer"][0][0], 1e-2, "persistent vs per-layer")
     assert results["persistent"][1] < results["per_layer"][1]
+
+
+def test_modulation_tables_match_the_oracle():
+    """The per-loop tables (what every layer of every step reads) against the oracle's time condition
+    and modulators: rows within bf16-operand accuracy of modulation(W, b, c(t_k)), scales stored as
+    1 + scale, and the QKV shift bias equal to W_qkv bf16(shift)."""
+    from tests.gpu_util import _Cai
+    d = I.TINY
+    w = I.Weights(d, seed=0, gain_jitter=0.1)
+    steps, P = 4, 16
+    eng = _engine(d, 1, P, w)
+    try:
+        eng.prefill(to_dev_bf16(I.prefix_embeddings(d, 1, P)))
+        eng.denoise(torch.from_numpy(I.noise(d, 1)).cuda(), steps)
+        eng.sync()
+        H, L = d.hidden_a, d.layers
+        R = (6 * L + 2) * H
+        QR = (d.n_q + 2 * d.n_kv) * d.head_dim
+        mod = torch.as_tensor(_Cai(eng.debug_view("tm_mod"), (steps, R), "<f4"), device="cuda").cpu().numpy()
+        bqkv = torch.as_tensor(_Cai(eng.debug_view("tm_bqkv"), (L, steps, QR), "<f4"), device="cuda").cpu().numpy()
+    finally:
+        eng.close()
+    for k, t in enumerate(O.euler_times(steps)):
+        c = M.time_condition(w.time(), t, d)
+        for l in range(L):
+            m = w.mod(l)
+            ga, sa, aa = M.modulation(m["W_ma"], m["b_ma"], c, 3)
+            gm, sm, am = M.modulation(m["W_mm"], m["b_mm"], c, 3)
+            row = mod[k, 6 * l * H:6 * (l + 1) * H]
+            ref = np.concatenate([1 + ga, sa, aa, 1 + gm, sm, am])
+            assert np.max(np.abs(row - ref)) <= 2e-2 * np.max(np.abs(ref)), (k, l)
+            lw = w.layer(1, l)
+            wqkv = np.concatenate([lw["Wq"], lw["Wk"], lw["Wv"]]).astype(np.float64)
+            shift = I.round_bf16(row[H:2 * H].astype(np.float32)).astype(np.float64)
+            np.testing.assert_allclose(bqkv[l, k], wqkv @ shift, rtol=0, atol=1e-4 * np.max(np.abs(wqkv @ shift)))
+        gf, sf = M.modulation(w.time()["W_mf"], w.time()["b_mf"], c, 2)
+        fin = mod[k, 6 * L * H:]
+        assert np.max(np.abs(fin - np.concatenate([1 + gf, sf]))) <= 2e-2 * np.max(np.abs(np.concatenate([1 + gf, sf])))

@@ -1633,7 +1633,7 @@ dm0_status dm0_debug_view(dm0_ctx* c, const char* name, void** ptr) {
       {"h_v", c->h_v},     {"xn_v", c->xn_v},   {"q_v", c->q_v},     {"o_v", c->o_v},     {"act_v", c->act_v},
       {"ssq_v", c->ssq_v}, {"h_a", c->h_a},     {"xn_a", c->xn_a},   {"q_a", c->q_a},     {"o_a", c->o_a},
       {"act_a", c->act_a}, {"ssq_a", c->ssq_a}, {"x", c->x},         {"k_s", c->k_s},     {"v_s", c->v_s},
-      {"loop_trace", c->ptrace}};
+      {"loop_trace", c->ptrace}, {"tm_mod", c->tm_mod}, {"tm_bqkv", c->tm_bqkv}, {"tm_bgu", c->tm_bgu}};
   auto it = bufs.find(name);
   if (it == bufs.end()) return fail(c, DM0_EINVAL, std::string("unknown buffer ") + name);
   *ptr = it->second;
