@@ -1,6 +1,8 @@
 /*
- * dm0.h - C ABI of the DM0 dual-expert merged-attention inference path on
- * NVIDIA B200 (sm_100a).
+ * dm0.h - C ABI of the DM0 dual-expert merged-attention path on NVIDIA B200
+ * (sm_100a): inference (prefix pass, Euler loop), with an FP8 E4M3 VLM MLP
+ * option, the DM0.5 time-modulated action expert as a configuration, and one
+ * flow-matching training step of the action expert.
  *
  * What it computes (page title and section of the sources):
  *   - DM0 architecture notes (dregs-remover.com/news/27019), section 1: in each
@@ -15,8 +17,11 @@
  *     Introduction", section 5.1 (the prefix runs once and its per-layer KV
  *     cache is kept), 5.2 (action_in_proj -> action expert -> action_out_proj
  *     gives the velocity v(x_t, t | c)), 5.3 (Euler integration from noise
- *     x_1 with diffusion_steps = 10 returns the whole chunk), 6.5 (fixed
- *     shapes and a graph captured once and replayed).
+ *     x_1 with diffusion_steps = 10 returns the whole chunk; training regresses
+ *     v onto u_t = eps - a at x_t = t eps + (1 - t) a under an action mask),
+ *     6.3 (FP8 E4M3 for the prefix MLP's GEMMs), 6.5 (fixed shapes and a
+ *     graph captured once and replayed); section 5.2 also names the time MLP
+ *     and per-layer time modulators of the DM0.5 action expert.
  *
  * Conventions shared by every entry point:
  *   - Every call returns a dm0_status; no call throws or aborts.  After a
