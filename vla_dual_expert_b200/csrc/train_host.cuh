@@ -98,23 +98,12 @@ dm0_status gemm_f32(dm0_ctx* c, cudaStream_t s, const bf16* A, int M, int K, con
   return run_gemm(c, s, A, M, K, B, N, g, 0);
 }
 
-// Forward of action layer l from hin over the cached prefix K/V, keeping every intermediate the
-// backward needs; hout (if not null) receives the layer's output.
-dm0_status train_layer_fwd(dm0_ctx* c, cudaStream_t s, int l, const float* hin, float* hout) {
+// Arguments of the training attention kernels of action layer l (forward and adjoint share them)
+dm0::TrainAttn train_attn_args(dm0_ctx* c, int l) {
   const dm0_config& g = c->cfg;
   auto& b = c->tb;
-  const LayerW& w = c->lw[1][l];
-  const int B = c->kv_B, P = c->kv_P, S = g.chunk, T = B * S;
-  const int H = g.hidden_a, I = g.inter_a, D = g.head_dim, QR = qkv_rows(g), HqD = g.n_q * D;
+  const int B = c->kv_B, P = c->kv_P, D = g.head_dim;
   const size_t lstride = static_cast<size_t>(B) * g.n_kv * P * D;
-  TRY(launch(c, s, dm0::train_rms_kernel, dim3((T + 7) / 8), dim3(256), 0, hin, static_cast<const float*>(w.attn_norm),
-             T, H, g.rms_eps, b.r1, b.rho1));
-  TRY(gemm_f32(c, s, b.r1, T, H, w.wqkv, QR, b.raw));
-  const int qk_warps = T * (g.n_q + 2 * g.n_kv);
-  TRY(launch(c, s, dm0::train_qk_fwd_kernel, dim3((qk_warps + 7) / 8), dim3(256), 0, static_cast<const float*>(b.raw),
-             static_cast<const float*>(w.q_norm), static_cast<const float*>(w.k_norm),
-             static_cast<const float2*>(c->rope), T, S, P, g.n_q, g.n_kv, D, g.rms_eps, b.qr, b.kr, b.vs, b.rho_q,
-             b.rho_k));
   dm0::TrainAttn at{};
   at.qr = b.qr;
   at.kr = b.kr;
@@ -122,7 +111,7 @@ dm0_status train_layer_fwd(dm0_ctx* c, cudaStream_t s, int l, const float* hin, 
   at.kc = c->kplane + l * lstride;
   at.vc = c->vplane + l * lstride;
   at.B = B;
-  at.S = S;
+  at.S = g.chunk;
   at.P = P;
   at.Hq = g.n_q;
   at.Hkv = g.n_kv;
@@ -131,6 +120,30 @@ dm0_status train_layer_fwd(dm0_ctx* c, cudaStream_t s, int l, const float* hin, 
   at.prob = b.prob;
   at.of = b.of;
   at.of_bf = b.of_bf;
+  at.dof = b.dof;
+  at.dqr = b.dqr;
+  at.dK = b.dK;
+  at.dV = b.dV;
+  return at;
+}
+
+// Forward of action layer l from hin over the cached prefix K/V, keeping every intermediate the
+// backward needs; hout (if not null) receives the layer's output.
+dm0_status train_layer_fwd(dm0_ctx* c, cudaStream_t s, int l, const float* hin, float* hout) {
+  const dm0_config& g = c->cfg;
+  auto& b = c->tb;
+  const LayerW& w = c->lw[1][l];
+  const int B = c->kv_B, P = c->kv_P, S = g.chunk, T = B * S;
+  const int H = g.hidden_a, I = g.inter_a, D = g.head_dim, QR = qkv_rows(g), HqD = g.n_q * D;
+  TRY(launch(c, s, dm0::train_rms_kernel, dim3((T + 7) / 8), dim3(256), 0, hin, static_cast<const float*>(w.attn_norm),
+             T, H, g.rms_eps, b.r1, b.rho1));
+  TRY(gemm_f32(c, s, b.r1, T, H, w.wqkv, QR, b.raw));
+  const int qk_warps = T * (g.n_q + 2 * g.n_kv);
+  TRY(launch(c, s, dm0::train_qk_fwd_kernel, dim3((qk_warps + 7) / 8), dim3(256), 0, static_cast<const float*>(b.raw),
+             static_cast<const float*>(w.q_norm), static_cast<const float*>(w.k_norm),
+             static_cast<const float2*>(c->rope), T, S, P, g.n_q, g.n_kv, D, g.rms_eps, b.qr, b.kr, b.vs, b.rho_q,
+             b.rho_k));
+  dm0::TrainAttn at = train_attn_args(c, l);
   const size_t fsm = sizeof(float) * (static_cast<size_t>(S) * D + 32 * (D + 1) + S * 32);
   TRY(launch(c, s, dm0::train_attn_fwd_kernel, dim3(B * g.n_q), dim3(256), fsm, at));
   TRY(gemm_f32(c, s, b.of_bf, T, HqD, w.wo, H, b.tmp));
@@ -248,26 +261,7 @@ dm0_status enqueue_train(dm0_ctx* c, cudaStream_t s, const float* a, const float
     CK(cudaMemsetAsync(b.dV, 0, sizeof(float) * B * g.n_kv * N * D, s));
     CK(cudaMemsetAsync(g_qn, 0, sizeof(float) * 2 * D, s));   // q_norm, k_norm (adjacent), accumulated
     c->pdl_ok = false;
-    dm0::TrainAttn at{};
-    const size_t lstride = static_cast<size_t>(B) * g.n_kv * P * D;
-    at.qr = b.qr;
-    at.kr = b.kr;
-    at.vs = b.vs;
-    at.kc = c->kplane + l * lstride;
-    at.vc = c->vplane + l * lstride;
-    at.B = B;
-    at.S = S;
-    at.P = P;
-    at.Hq = g.n_q;
-    at.Hkv = g.n_kv;
-    at.D = D;
-    at.scale = 1.0f / std::sqrt(static_cast<float>(D));
-    at.prob = b.prob;
-    at.of = b.of;
-    at.dof = b.dof;
-    at.dqr = b.dqr;
-    at.dK = b.dK;
-    at.dV = b.dV;
+    dm0::TrainAttn at = train_attn_args(c, l);
     const size_t bsm = sizeof(float) * (2 * static_cast<size_t>(S) * D + 2 * 32 * (D + 1) + 2 * S * 32 + S);
     TRY(launch(c, s, dm0::train_attn_bwd_kernel, dim3(B * g.n_q), dim3(256), bsm, at));
     const int qk_warps = T * (g.n_q + 2 * g.n_kv);
