@@ -284,8 +284,9 @@ dm0_status dm0_op_attention(dm0_ctx* ctx, const void* q, const void* ka, const v
  * (VLM side, rows = B*P tokens) and h_a, xn_a, q_a, o_a, act_a, ssq_a, x,
  * k_s, v_s (action side, rows = B*chunk tokens).  Layouts: h_* f32 [rows][H];
  * xn_* bf16 [rows][H] (gain * h of the pending RMSNorm); q_*, o_* bf16
- * [rows][n_q*head_dim]; act_* bf16 [rows][inter]; ssq_* f32 [2*layers][rows]
- * (sum of squares of h for each pending norm); x f32 [rows][action_dim];
+ * [rows][n_q*head_dim]; act_* bf16 [rows][inter]; ssq_* f32 [2][H/64][rows]
+ * (the attention norm's, then the MLP norm's sums of squares of h, one partial
+ * sum per 64-column group, which the consumer adds in group order); x f32 [rows][action_dim];
  * k_s/v_s bf16 [B][n_kv][chunk][head_dim].  Context-owned; contents are only
  * meaningful after the call that fills them has completed.
  * "loop_trace" (NULL unless DM0_PERSIST_TRACE=1 was set at dm0_create): u64

@@ -2,11 +2,11 @@
 step's velocity against the fp64 oracle, and against the per-layer kernel path of the same context.
 
 DM0-base widths with 3 layers keep the oracle fast; the 28-layer stack goes through the same kernel
-in test_gpu_parity (denoise over a random cache, and end to end).  Prefix lengths cover a whole
+in test_a_gpu_parity (denoise over a random cache, and end to end).  Prefix lengths cover a whole
 number of 64-key blocks (64), a ragged last block (100, 816) and a single key (1); the key-split
 count per KV head is varied from 1 (one CTA per head walks every block) to 8.
 
-Tolerances as in test_gpu_parity: chunk 2e-2 of RMS(chunk), velocities 2e-2 of RMS(v) for this
+Tolerances as in test_a_gpu_parity: chunk 2e-2 of RMS(chunk), velocities 2e-2 of RMS(v) for this
 shallow stack.  The two GPU paths differ only in fp32 summation order (split-K partial sums reach
 the accumulators in a different order), so they agree to 1e-2 of RMS."""
 import os

@@ -8,29 +8,31 @@ quantiser's precision (quantize_rows_f32: fp32 scale and fp32 quotient).  Tolera
                                          on the GPU and in fp64 in the oracle)
   FP8 GEMM                               max |d| <= 2e-5 RMS: the products of E4M3 codes are exact in
                                          fp32, only the order of the fp32 summation differs
-  one merged layer, FP8 VLM MLP          K / V and the action branch as in the bf16 layer test; the VLM
-                                         output RMS(d) <= 5e-3 RMS, max <= 0.1 RMS and at most 2 % of the
-                                         elements beyond 1e-2 RMS: a code whose fp32 quotient lies within
-                                         a few fp32 ulps of an E4M3 midpoint can round either way, and
-                                         one such flip moves a whole output column by a step of 2^-3
-                                         relative (emulated on the CPU with 3-ulp noise on the operands:
-                                         max 0.024, RMS 8e-4, 0.2 % of the elements beyond 1e-2 RMS)
-The quantiser and GEMM tests have run on a B200; the layer-level tests (marked `pending`) run only
-with DM0_RUN_FP8=1 until their first GPU run.
+  FP8 MLP on exact inputs               (a layer whose VLM O-projection is zero, so the MLP's input is the
+                                         fp32 input itself) K / V and the action branch as in the bf16
+                                         layer test; the VLM output RMS(d) <= 5e-3 RMS, max <= 0.1 RMS and
+                                         at most 2 % of the elements beyond 1e-2 RMS: a code whose fp32
+                                         quotient lies within a few fp32 ulps of an E4M3 midpoint can round
+                                         either way, and one such flip moves a whole output column by a
+                                         step of 2^-3 relative (emulated on the CPU with 3-ulp noise on the
+                                         operands: max 0.024, RMS 8e-4, 0.2 % of the elements beyond 1e-2)
+  FP8 MLP inside the whole layer,        twice the error of the CPU emulation of the GPU's bf16 rounding
+  and a whole tiny prefix pass           points followed by the FP8 MLP (tests/tolerances.py): the bf16
+                                         rounding of the attention half moves the MLP's input by ~1e-3
+                                         relative, and the codes near E4M3 midpoints follow it (measured on
+                                         a B200: 1.09e-2 and 1.22e-2 of RMS on the two layers, 2.5e-3 on the
+                                         tiny model's layer 1; emulated 1.11e-2, 1.21e-2, 2.4e-3)
 """
-import os
-
 import numpy as np
 import pytest
 import torch
 
 from oracle import dm0_oracle as O
 from synth import inputs as I
+from tests import tolerances as TOL
 from tests.gpu_util import check_bf16, check_fp, host, rel_err, rms, to_dev_bf16, to_dev_f32
 
 pytestmark = pytest.mark.gpu
-pending = pytest.mark.skipif(os.environ.get("DM0_RUN_FP8") != "1",
-                             reason="awaits its first GPU run (DM0_RUN_FP8=1)")
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -143,37 +145,79 @@ def _fp8_stats(got, ref, what):
     return out
 
 
-@pending
-@pytest.mark.parametrize("B,P", [(1, 816), (2, 333)])
-def test_merged_layer_fp8(eng1, B, P):
-    d, w, eng = eng1
+def _run_merged(eng, d, B, P, seed, fp8):
     S = d.chunk
-    hp = np.stack([I.hidden_states(P, d.hidden_v, seed=40 + b) for b in range(B)])
-    hs = np.stack([I.hidden_states(S, d.hidden_a, seed=140 + b) for b in range(B)])
+    hp = np.stack([I.hidden_states(P, d.hidden_v, seed=seed + b) for b in range(B)])
+    hs = np.stack([I.hidden_states(S, d.hidden_a, seed=seed + 100 + b) for b in range(B)])
     outp = torch.empty((B, P, d.hidden_v), device="cuda", dtype=torch.float32)
     outs = torch.empty((B, S, d.hidden_a), device="cuda", dtype=torch.float32)
     k = torch.empty((B, d.n_kv, P, d.head_dim), device="cuda", dtype=torch.bfloat16)
     v = torch.empty_like(k)
-    eng.set_prefix_fp8(True)
+    eng.set_prefix_fp8(fp8)
     try:
         eng.merged_layer(0, to_dev_f32(hp), to_dev_f32(hs), outp, outs, k, v)
         eng.sync()
     finally:
         eng.set_prefix_fp8(False)
     assert eng.device_error() == 0
+    return hp, hs, host(outp), host(outs), host(k), host(v)
+
+
+@pytest.fixture(scope="module")
+def eng_mlp_only():
+    """One DM0-base layer whose VLM O-projection is zero: the VLM output is h + MLP(rms(h)), so the FP8
+    MLP sees the fp32 input itself and no upstream bf16 rounding."""
+    d = I.DM0_BASE.replace(layers=1)
+    w = I.Weights(d, seed=0, gain_jitter=0.1)
+    w.overrides[(0, 0, "Wo")] = np.zeros((d.hidden_v, d.n_q * d.head_dim), np.float32)
+    eng = _engine(d, 2, 816, w)
+    yield d, w, eng
+    eng.close()
+
+
+@pytest.mark.parametrize("B,P", [(1, 816), (2, 333)])
+def test_merged_layer_fp8_mlp(eng_mlp_only, B, P):
+    """The FP8 MLP on exact inputs: only fp32 rounding separates the GPU's operands from the oracle's,
+    so codes flip only at E4M3 midpoints within a few fp32 ulps (bars of the module docstring)."""
+    d, w, eng = eng_mlp_only
+    hp, hs, outp, outs, k, v = _run_merged(eng, d, B, P, 40, True)
     for b in range(B):
         rp, rs_, rk, rv = O.merged_layer(w.layer(0, 0), w.layer(1, 0), hp[b], hs[b], d, vlm_fp8=O.quantize_rows_f32)
-        check_bf16(host(k[b]), rk, 1e-2, "prefix K")
-        check_bf16(host(v[b]), rv, 1e-2, "prefix V")
-        check_fp(host(outs[b]), rs_, 1e-2, "suffix out (bf16 action branch)")
-        r_rms, r_max, r_frac = _fp8_stats(host(outp[b]), rp, "prefix out, FP8 MLP")
+        check_bf16(k[b], rk, TOL.KV_ONE_LAYER[0], "prefix K", TOL.KV_ONE_LAYER[1])
+        check_bf16(v[b], rv, TOL.KV_ONE_LAYER[0], "prefix V", TOL.KV_ONE_LAYER[1])
+        check_fp(outs[b], rs_, TOL.LAYER, "suffix out (bf16 action branch)")
+        r_rms, r_max, r_frac = _fp8_stats(outp[b], rp, "prefix out, FP8 MLP")
         assert r_rms <= 5e-3 and r_max <= 0.1 and r_frac <= 0.02
         # and it is the FP8 MLP that was run: far closer to the FP8 oracle than to the plain one
         plain = O.merged_layer(w.layer(0, 0), w.layer(1, 0), hp[b], hs[b], d)[0]
-        assert rms(host(outp[b]) - rp) < 0.25 * rms(plain - rp)
+        assert rms(outp[b] - rp) < 0.25 * rms(plain - rp)
+
+
+@pytest.mark.parametrize("B,P", [(1, 816), (2, 333)])
+def test_merged_layer_fp8(eng1, B, P):
+    """The whole layer: the MLP's input now carries the bf16 rounding of the attention half (about 1e-3
+    relative), and every code within that distance of an E4M3 midpoint may round the other way (a few
+    % of them, each by a 2^-3-relative step): the VLM output is held to twice the error the CPU
+    emulation of the GPU's rounding points shows on these inputs (tests/tolerances.py FP8_LAYER_RMS),
+    and the FP8 path must move the output away from the GPU's own bf16 layer by at least half as much
+    as the FP8 oracle moves away from the plain one (the emulation: the same amount)."""
+    d, w, eng = eng1
+    hp, hs, outp, outs, k, v = _run_merged(eng, d, B, P, 40, True)
+    bf = _run_merged(eng, d, B, P, 40, False)[2]
+    for b in range(B):
+        rp, rs_, rk, rv = O.merged_layer(w.layer(0, 0), w.layer(1, 0), hp[b], hs[b], d, vlm_fp8=O.quantize_rows_f32)
+        check_bf16(k[b], rk, TOL.KV_ONE_LAYER[0], "prefix K", TOL.KV_ONE_LAYER[1])
+        check_fp(outs[b], rs_, TOL.LAYER, "suffix out (bf16 action branch)")
+        r_rms, _, _ = _fp8_stats(outp[b], rp, "prefix out, FP8 MLP")
+        assert r_rms <= TOL.FP8_LAYER_RMS
+        plain = O.merged_layer(w.layer(0, 0), w.layer(1, 0), hp[b], hs[b], d)[0]
+        assert rms(outp[b] - bf[b]) >= 0.5 * rms(rp - plain)
 
 
 def test_fp8_toggle_leaves_the_bf16_path_unchanged(eng1):
+    """Switching the FP8 MLP on and off again leaves the bf16 layer bit for bit as it was: the VLM path
+    has no order-dependent sums (the residual epilogue writes per-group sums of squares that the
+    consumer adds in a fixed order)."""
     d, _, eng = eng1
     P, S = 200, d.chunk
     hp, hs = I.hidden_states(P, d.hidden_v, seed=60)[None], I.hidden_states(S, d.hidden_a, seed=61)[None]
@@ -191,9 +235,7 @@ def test_fp8_toggle_leaves_the_bf16_path_unchanged(eng1):
     fp8 = run()
     eng.set_prefix_fp8(False)
     after = run()
-    # the bf16 layer is not bitwise repeatable (the residual epilogue's sums of squares are atomic
-    # fp32 adds in any order), so "unchanged" means equal to fp32 rounding of those sums
-    assert rel_err(after, before) <= 1e-5
+    assert np.array_equal(after, before)
     assert rel_err(fp8, before) > 1e-3
 
 
@@ -209,31 +251,42 @@ def test_enable_before_weights_is_a_state_error():
 
 # ------------------------------------------------------------------ a whole prefix pass (tiny model)
 
-@pending
-def test_tiny_prefill_fp8(eng1):
+def _tiny_prefill(d, w, emb, fp8):
+    from tests.gpu_util import device_view_bf16
     from vla_dual_expert_b200 import Engine
-    d = I.TINY
-    w = I.Weights(d, seed=0, gain_jitter=0.1)
-    P = 64
-    emb = I.prefix_embeddings(d, 1, P)
+    P = emb.shape[1]
     eng = Engine(d, 1, P)
     try:
         eng.load_from(w)
-        eng.set_prefix_fp8(True)
+        eng.set_prefix_fp8(fp8)
         eng.prefill(to_dev_bf16(emb))
         eng.sync()
         assert eng.device_error() == 0
         kp, vp = eng.kv_view()
-        from tests.gpu_util import device_view_bf16
         K = host(device_view_bf16(kp, (d.layers, d.n_kv, P, d.head_dim)))
         V = host(device_view_bf16(vp, (d.layers, d.n_kv, P, d.head_dim)))
     finally:
         eng.close()
+    return K, V
+
+
+def test_tiny_prefill_fp8():
+    """Every layer's K/V after a 2-layer prefix pass with the FP8 MLP: RMS(d) within twice the emulated
+    error (tests/tolerances.py FP8_TINY_KV_RMS; layer 0 precedes any MLP), and the FP8 MLP moves layer
+    1's K/V away from the GPU's own bf16 prefill by at least half as much as the emulation moves them."""
+    from tests import bf16_emulation as E
+    d = I.TINY
+    w = I.Weights(d, seed=0, gain_jitter=0.1)
+    emb = I.prefix_embeddings(d, 1, 64)
+    K, V = _tiny_prefill(d, w, emb, True)
+    K0, V0 = _tiny_prefill(d, w, emb, False)
     ks, vs, _ = O.prefill_fp8(w, emb[0], qrows=O.quantize_rows_f32)
-    ks0, vs0, _ = O.prefill(w, emb[0])
+    eks, evs, _ = E.prefill(w, emb[0], fp8=True)
+    eks0, evs0, _ = E.prefill(w, emb[0])
     for l in range(d.layers):
-        for got, ref, plain, nm in ((K[l], ks[l], ks0[l], "K"), (V[l], vs[l], vs0[l], "V")):
+        for got, got0, ref, emu, emu0, nm in ((K[l], K0[l], ks[l], eks[l], eks0[l], "K"),
+                                              (V[l], V0[l], vs[l], evs[l], evs0[l], "V")):
             r_rms, _, _ = _fp8_stats(got, ref, f"layer {l} {nm}")
-            assert r_rms <= 1e-2 * np.sqrt(l + 1)
-            if l > 0:   # layer 0's K/V precede any MLP
-                assert rms(got - ref) < 0.5 * rms(plain - ref)
+            assert r_rms <= TOL.FP8_TINY_KV_RMS
+            if l > 0:
+                assert rms(got - got0) >= 0.5 * rms(emu - emu0)

@@ -1,9 +1,7 @@
 """dm0_prepare: shape buckets made ready ahead of time (the pages' fixed shapes per captured graph,
 several prefix lengths and step counts without a capture at request time).  A prepared bucket's
 denoise matches an unprepared engine's, preparing launches nothing, and preparing another shape
-leaves the committed cache shape alone.  Awaits its first GPU run (DM0_RUN_PREPARE=1)."""
-import os
-
+leaves the committed cache shape alone."""
 import numpy as np
 import pytest
 import torch
@@ -11,9 +9,7 @@ import torch
 from synth import inputs as I
 from tests.gpu_util import host, rel_err, to_dev_bf16
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skipif(os.environ.get("DM0_RUN_PREPARE") != "1",
-                                 reason="awaits its first GPU run (DM0_RUN_PREPARE=1)")]
+pytestmark = pytest.mark.gpu
 
 
 def _run(prepare):
@@ -44,4 +40,7 @@ def test_prepared_bucket_matches_and_launches_the_same_graph():
     x0, n0 = _run(False)
     x1, n1 = _run(True)
     assert n0 == n1
-    assert rel_err(x1, x0) <= 1e-5   # split-K sums may arrive in another order
+    # the batch-2 loop's swapped GEMMs add their split-K partial sums with fp32 atomics, whose order
+    # varies from run to run: two runs of the same graph differ at the 1e-5 level (measured on a B200:
+    # 1.9e-5 of RMS), so the bar is 1e-4, as between two replays of one graph
+    assert rel_err(x1, x0) <= 1e-4

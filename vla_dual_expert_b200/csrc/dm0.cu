@@ -457,13 +457,14 @@ dm0_status run_gemm_e4m3(dm0_ctx* c, cudaStream_t s, const uint8_t* act, const f
 
 // per-row E4M3 codes and scales of a matrix [rows][cols] (bf16 or fp32), each row optionally scaled by
 // gain[c] and its pending RMSNorm factor from ssq[row] first
+// (ssq: `ssq_slots` partial sums per row, slot-major with stride `ssq_stride`, added in slot order)
 template <typename T>
 dm0_status quant_rows(dm0_ctx* c, cudaStream_t s, const T* x, int rows, int cols, uint8_t* q, float* scale,
-                      const float* gain = nullptr, const float* ssq = nullptr) {
+                      const float* gain = nullptr, const float* ssq = nullptr, int ssq_slots = 1, int ssq_stride = 0) {
   if (rows <= 0) return DM0_OK;
   if (cols <= 0 || cols % 8 != 0) return fail(c, DM0_ESHAPE, "E4M3 row quantisation needs cols % 8 == 0");
-  return launch(c, s, dm0::quant_rows_e4m3_kernel<T>, dim3(rows), dim3(256), 0, x, rows, cols, gain, ssq,
-                1.0f / cols, c->cfg.rms_eps, q, scale);
+  return launch(c, s, dm0::quant_rows_e4m3_kernel<T>, dim3(rows), dim3(256), 0, x, rows, cols, gain, ssq, ssq_slots,
+                ssq_stride > 0 ? ssq_stride : rows, 1.0f / cols, c->cfg.rms_eps, q, scale);
 }
 
 // ---------------------------------------------------------------- attention dispatch
@@ -591,6 +592,8 @@ dm0_status layer_qkv(dm0_ctx* c, cudaStream_t s, int br, int l, const bf16* xn, 
   g.w_stable = 1;
   g.mode = dm0::kModeQKV;
   g.ssq_in = ssq_in;
+  g.ssq_slots = H / 64;
+  g.ssq_stride = tokens;
   g.inv_hidden = 1.0f / H;
   g.q_out = q_out;
   g.k_out = k_out;
@@ -624,6 +627,7 @@ dm0_status layer_rest(dm0_ctx* c, cudaStream_t s, int br, int l, int tokens, flo
   g.gain_next = mod ? mod->scale_m : w.mlp_norm;
   g.col_gate = mod ? mod->gate_o : nullptr;
   g.ssq_out = ssq_mlp;
+  g.ssq_stride = tokens;
   const int so = br == 0 ? DM0_SITE_VLM_O : DM0_SITE_ACT_O;
   int e0 = probe_begin(c, s, so);
   TRY(run_gemm(c, s, o, tokens, cf.n_q * cf.head_dim, w.wo, H, g));
@@ -636,6 +640,8 @@ dm0_status layer_rest(dm0_ctx* c, cudaStream_t s, int br, int l, int tokens, flo
   u.w_stable = 1;
   u.mode = dm0::kModeSwiGLU;
   u.ssq_in = ssq_mlp;
+  u.ssq_slots = H / 64;
+  u.ssq_stride = tokens;
   u.inv_hidden = 1.0f / H;
   u.act = act;
   u.inter = I;
@@ -643,7 +649,8 @@ dm0_status layer_rest(dm0_ctx* c, cudaStream_t s, int br, int l, int tokens, flo
   const int su = br == 0 ? DM0_SITE_VLM_GATEUP : DM0_SITE_ACT_GATEUP;
   e0 = probe_begin(c, s, su);
   if (f8) {
-    TRY(quant_rows(c, s, static_cast<const float*>(h), tokens, H, c->xq_v, c->sxq_v, w.mlp_norm, ssq_mlp));
+    TRY(quant_rows(c, s, static_cast<const float*>(h), tokens, H, c->xq_v, c->sxq_v, w.mlp_norm, ssq_mlp, H / 64,
+                   tokens));
     u.ssq_in = nullptr;
     u.act = nullptr;
     u.act_f32 = c->act32_v;
@@ -660,6 +667,7 @@ dm0_status layer_rest(dm0_ctx* c, cudaStream_t s, int br, int l, int tokens, flo
   d.xn = next_gain ? xn : nullptr;
   d.gain_next = next_gain;
   d.ssq_out = next_gain ? next_ssq : nullptr;
+  d.ssq_stride = tokens;
   d.col_gate = mod ? mod->gate_d : nullptr;
   const int sd = br == 0 ? DM0_SITE_VLM_DOWN : DM0_SITE_ACT_DOWN;
   e0 = probe_begin(c, s, sd);
@@ -678,19 +686,21 @@ dm0_status enqueue_prefill(dm0_ctx* c, cudaStream_t s, const void* prefix_emb, i
   c->pdl_ok = false;
   const int M = B * P, L = cf.layers, D = cf.head_dim;
   const size_t lstride = static_cast<size_t>(B) * cf.n_kv * P * D;
-  TRY(rows_prep(c, s, prefix_emb, 1, c->h_v, c->xn_v, c->lw[0][0].attn_norm, c->ssq_v, 2 * L, M, cf.hidden_v));
+  // sums of squares of the pending norms: [H / 64 groups][M] for the attention norm, then the MLP norm
+  float* ssq_attn = c->ssq_v;
+  float* ssq_mlp = ssq_attn + static_cast<size_t>(cf.hidden_v / 64) * M;
+  TRY(rows_prep(c, s, prefix_emb, 1, c->h_v, c->xn_v, c->lw[0][0].attn_norm, ssq_attn, cf.hidden_v / 64, M,
+                cf.hidden_v));
   for (int l = 0; l < L; ++l) {
     bf16* kl = c->kplane + l * lstride;
     bf16* vl = c->vplane + l * lstride;
-    float* ssq_attn = c->ssq_v + static_cast<size_t>(2 * l) * M;
-    float* ssq_mlp = ssq_attn + M;
     TRY(layer_qkv(c, s, 0, l, c->xn_v, ssq_attn, M, P, 0, c->q_v, kl, vl));
     const int e0 = probe_begin(c, s, DM0_SITE_VLM_ATTN);
     TRY(run_attn(c, s, c->q_v, P, kl, vl, P, nullptr, nullptr, 0, c->o_v, B, 1, 0));
     probe_end(c, s, DM0_SITE_VLM_ATTN, e0);
     const bool more = l + 1 < L;
     TRY(layer_rest(c, s, 0, l, M, c->h_v, c->xn_v, c->o_v, c->act_v, ssq_mlp,
-                   more ? c->lw[0][l + 1].attn_norm : nullptr, more ? ssq_mlp + M : nullptr));
+                   more ? c->lw[0][l + 1].attn_norm : nullptr, more ? ssq_attn : nullptr));
   }
   return DM0_OK;
 }
@@ -708,8 +718,8 @@ dm0_status step(dm0_ctx* c, cudaStream_t s, int B, int k_out, int k_in, int step
   a.x = c->x;
   a.h = c->h_a;
   a.xn = c->xn_a;
-  a.ssq = c->ssq_a;
-  a.n_slots = 2 * cf.layers;
+  a.ssq = c->ssq_a;   // the attention norm's [Ha / 64][tokens] block
+  a.n_slots = cf.hidden_a / 64;
   a.tokens = B * cf.chunk;
   a.W_in = c->W_in;
   a.b_in = c->b_in;
@@ -812,8 +822,8 @@ dm0_status enqueue_denoise(dm0_ctx* c, cudaStream_t s, int steps, float* vel) {
     for (int l = 0; l < L; ++l) {
       const bf16* kl = c->kplane + l * lstride;
       const bf16* vl = c->vplane + l * lstride;
-      float* ssq_attn = c->ssq_a + static_cast<size_t>(2 * l) * Ms;
-      float* ssq_mlp = ssq_attn + Ms;
+      float* ssq_attn = c->ssq_a;
+      float* ssq_mlp = ssq_attn + static_cast<size_t>(cf.hidden_a / 64) * Ms;
       const bool more = l + 1 < L;
       ModPtrs mp{};
       if (tm) {
@@ -831,7 +841,7 @@ dm0_status enqueue_denoise(dm0_ctx* c, cudaStream_t s, int steps, float* vel) {
       probe_end(c, s, DM0_SITE_ACT_ATTN, e0);
       const float* next_gain = more ? (tm ? mp.next_scale : c->lw[1][l + 1].attn_norm) : nullptr;
       TRY(layer_rest(c, s, 1, l, Ms, c->h_a, c->xn_a, c->o_a, c->act_a, ssq_mlp, next_gain,
-                     more ? ssq_mlp + Ms : nullptr, tm ? &mp : nullptr));
+                     more ? ssq_attn : nullptr, tm ? &mp : nullptr));
     }
     sm = tm ? step_mod(k, k + 1 < steps ? k + 1 : -1) : StepMod{};
     TRY(step(c, s, B, k, k + 1 < steps ? k + 1 : -1, steps, vel, tm ? &sm : nullptr));
@@ -1107,6 +1117,9 @@ constexpr int kNoAllocOFloats = kNoAllocSlots * 128 * 128;      // partial O, he
 constexpr int kNoAllocMlFloats = kNoAllocSlots * 128 * 2;       // (m, l) per partial row
 constexpr int kNoAllocCounters = kNoAllocSlots;                 // one arrival counter per (group, row tile)
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocOFloats + kNoAllocMlFloats + kNoAllocCounters];
+// the split combine keeps (m, l) of every split of a row tile (128 rows x 8 bytes each) in the kernel's
+// shared memory: the most splits the slots allow must fit the smallest instance
+static_assert(kNoAllocSlots * 128 * 8 <= dm0::AttnSmem<32>::kBytes, "no-alloc splits exceed the combine's smem");
 
 namespace {
 constexpr int kNoAllocMaxDevices = 64;
@@ -1282,13 +1295,13 @@ dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
   A(dalloc(c, &c->q_v, Mp * qd));
   A(dalloc(c, &c->o_v, Mp * qd));
   A(dalloc(c, &c->act_v, Mp * g.inter_v));
-  A(dalloc(c, &c->ssq_v, Mp * 2 * g.layers));
+  A(dalloc(c, &c->ssq_v, Mp * 2 * (g.hidden_v / 64)));   // [attention, MLP norm][H / 64 groups][rows]
   A(dalloc(c, &c->h_a, Ms * g.hidden_a));
   A(dalloc(c, &c->xn_a, Ms * g.hidden_a));
   A(dalloc(c, &c->q_a, Ms * qd));
   A(dalloc(c, &c->o_a, Ms * qd));
   A(dalloc(c, &c->act_a, Ms * g.inter_a));
-  A(dalloc(c, &c->ssq_a, Ms * 2 * g.layers));
+  A(dalloc(c, &c->ssq_a, Ms * 2 * (g.hidden_a / 64)));
   A(dalloc(c, &c->x, Ms * g.action_dim));
   A(dalloc(c, &c->k_s, Ms * g.n_kv * D));
   A(dalloc(c, &c->v_s, Ms * g.n_kv * D));
@@ -1540,15 +1553,18 @@ dm0_status dm0_merged_layer(dm0_ctx* c, int layer, const float* h_prefix, const 
   bf16* kp = static_cast<bf16*>(k_out);
   bf16* vp = static_cast<bf16*>(v_out);
   c->pdl_ok = false;
-  TRY(rows_prep(c, s, h_prefix, 0, c->h_v, c->xn_v, c->lw[0][layer].attn_norm, c->ssq_v, 2, Mp, g.hidden_v));
-  TRY(rows_prep(c, s, h_suffix, 0, c->h_a, c->xn_a, c->lw[1][layer].attn_norm, c->ssq_a, 2, Ms, g.hidden_a));
+  const int nsv = g.hidden_v / 64, nsa = g.hidden_a / 64;   // sum-of-squares groups per row
+  TRY(rows_prep(c, s, h_prefix, 0, c->h_v, c->xn_v, c->lw[0][layer].attn_norm, c->ssq_v, nsv, Mp, g.hidden_v));
+  TRY(rows_prep(c, s, h_suffix, 0, c->h_a, c->xn_a, c->lw[1][layer].attn_norm, c->ssq_a, nsa, Ms, g.hidden_a));
   TRY(layer_qkv(c, s, 0, layer, c->xn_v, c->ssq_v, Mp, P, 0, c->q_v, kp, vp));
   TRY(layer_qkv(c, s, 1, layer, c->xn_a, c->ssq_a, Ms, S, P, c->q_a, c->k_s, c->v_s));
   // the block mask: prefix rows see the prefix; suffix rows see prefix and suffix
   TRY(run_attn(c, s, c->q_v, P, kp, vp, P, nullptr, nullptr, 0, c->o_v, B, 1, 0));
   TRY(run_attn(c, s, c->q_a, S, kp, vp, P, c->k_s, c->v_s, S, c->o_a, B, 0, 0));
-  TRY(layer_rest(c, s, 0, layer, Mp, c->h_v, c->xn_v, c->o_v, c->act_v, c->ssq_v + Mp, nullptr, nullptr));
-  TRY(layer_rest(c, s, 1, layer, Ms, c->h_a, c->xn_a, c->o_a, c->act_a, c->ssq_a + Ms, nullptr, nullptr));
+  TRY(layer_rest(c, s, 0, layer, Mp, c->h_v, c->xn_v, c->o_v, c->act_v, c->ssq_v + static_cast<size_t>(nsv) * Mp,
+                 nullptr, nullptr));
+  TRY(layer_rest(c, s, 1, layer, Ms, c->h_a, c->xn_a, c->o_a, c->act_a, c->ssq_a + static_cast<size_t>(nsa) * Ms,
+                 nullptr, nullptr));
   CK(cudaMemcpyAsync(out_prefix, c->h_v, static_cast<size_t>(Mp) * g.hidden_v * 4, cudaMemcpyDeviceToDevice, s));
   CK(cudaMemcpyAsync(out_suffix, c->h_a, static_cast<size_t>(Ms) * g.hidden_a * 4, cudaMemcpyDeviceToDevice, s));
   return DM0_OK;
@@ -1691,6 +1707,9 @@ dm0_status dm0_attention_noalloc(const void* q, const void* ka, const void* va, 
   const int bps = (nblk + splits - 1) / splits;
   splits = (nblk + bps - 1) / bps;
   if (splits > 1 && groups * tiles * splits > kNoAllocSlots) return DM0_ESHAPE;   // beyond the static scratch
+  const int smem_bytes = head_dim == 128 ? dm0::AttnSmem<128>::kBytes
+                                         : (head_dim == 64 ? dm0::AttnSmem<64>::kBytes : dm0::AttnSmem<32>::kBytes);
+  if (splits > 1 && splits * 128 * 8 > smem_bytes) return DM0_ESHAPE;   // the combine's (m, l) in shared memory
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* counters = reinterpret_cast<int*>(base + kNoAllocOFloats + kNoAllocMlFloats);
   if (splits > 1 && cudaMemsetAsync(counters, 0, kNoAllocCounters * sizeof(int), s) != cudaSuccess)

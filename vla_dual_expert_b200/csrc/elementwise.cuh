@@ -16,8 +16,8 @@
 
 namespace dm0 {
 
-// h[row] = in[row]; xn[row] = bf16(gain * h); ssq[0][row] = sum h^2; ssq[s][row] = 0 for s >= 1.
-// One warp per row.
+// h[row] = in[row]; xn[row] = bf16(gain * h); ssq[0][row] = sum h^2; ssq[s][row] = 0 for s >= 1
+// (the n_slots partial-sum slots a consumer adds up).  One warp per row.
 __global__ void __launch_bounds__(256) rows_prep_kernel(const void* in, int in_bf16, float* h, __nv_bfloat16* xn,
                                                         const float* gain, float* ssq, int n_slots, int slot_stride,
                                                         int M, int H) {
@@ -251,7 +251,7 @@ __global__ void wait_timeout_selftest_kernel(int* err, unsigned long long limit_
 
 // FP8 E4M3 row quantisation (the operands of the FP8 prefix-MLP GEMMs; DM0.5 page, section 6.3, with
 // per-row scales).  Row r of x (bf16 or fp32), optionally times gain[c] and the row's pending RMSNorm
-// factor 1/sqrt(ssq[r] / cols + eps), is y[c]; scale[r] = amax(|y|) / 448 in fp32 (1 for an all-zero
+// factor 1/sqrt(sum of its ssq slots / cols + eps), is y[c]; scale[r] = amax(|y|) / 448 in fp32 (1 for an all-zero
 // row) and q[r][c] = E4M3(y[c] / scale[r]), the quotient an IEEE fp32 division and the conversion
 // round to nearest even, saturating.  One CTA of 256 threads per row, 16-byte loads (8 bf16 or 4
 // fp32), cols a multiple of 8; the row is read twice, the second time from L1 / L2.  Used for the
@@ -285,8 +285,8 @@ __device__ __forceinline__ void quant_load(const T* row, const float* gain, floa
 
 template <typename T>
 __global__ void __launch_bounds__(256) quant_rows_e4m3_kernel(const T* x, int rows, int cols, const float* gain,
-                                                              const float* ssq, float inv_cols, float eps,
-                                                              uint8_t* q, float* scale) {
+                                                              const float* ssq, int ssq_slots, int ssq_stride,
+                                                              float inv_cols, float eps, uint8_t* q, float* scale) {
   constexpr int kV = 16 / sizeof(T);
   __shared__ float red[8];
   pdl_launch_dependents();
@@ -294,7 +294,12 @@ __global__ void __launch_bounds__(256) quant_rows_e4m3_kernel(const T* x, int ro
   const int row = blockIdx.x;
   if (row >= rows) return;
   const T* src = x + static_cast<size_t>(row) * cols;
-  const float rn = ssq ? rsqrtf(__ldcg(ssq + row) * inv_cols + eps) : 1.f;
+  float rn = 1.f;
+  if (ssq) {   // partial sums of squares of the row, added in slot order
+    float ss = 0.f;
+    for (int q2 = 0; q2 < ssq_slots; ++q2) ss += __ldcg(ssq + static_cast<size_t>(q2) * ssq_stride + row);
+    rn = rsqrtf(ss * inv_cols + eps);
+  }
   const int nvec = cols / kV;
   float amax = 0.f;
   for (int v = threadIdx.x; v < nvec; v += 256) {

@@ -26,7 +26,7 @@ namespace dm0 {
 enum GemmMode : int {
   kModeStoreF32 = 0,  // C = acc (normal) / C += acc (swap)   -- unit tests
   kModeQKV = 1,       // scale by inv_rms, QK-RMSNorm + RoPE on q/k heads, write q / K / V (bf16)
-  kModeResid = 2,     // h += acc; xn = bf16(gain_next * h); ssq_out += sum(h^2)
+  kModeResid = 2,     // h += acc; xn = bf16(gain_next * h); ssq_out = sum(h^2) per 64-column group
   kModeSwiGLU = 3,    // scale by inv_rms; act = silu(gate) * up (bf16); gate/up interleaved by 64 rows
 };
 
@@ -38,9 +38,12 @@ struct GemmArgs {
   int tokens;         // valid activation rows
   int w_stable;       // weight operand was written before the previous kernel: fetch it before the PDL wait
   int* err;           // device error word
-  // input row scale: inv_rms(token) = rsqrt(ssq_in[token] * inv_hidden + eps); null -> 1
+  // input row scale: inv_rms(token) = rsqrt(sum_s ssq_in[s * ssq_stride + token] * inv_hidden + eps)
+  // over the ssq_slots partial sums of squares (one per 64-column group of the residual, added in
+  // slot order so the result does not depend on which CTA finished first); null -> 1
   const float* ssq_in;
   float inv_hidden, eps;
+  int ssq_slots, ssq_stride;   // also the layout of ssq_out
   // split-K accumulation target (swap, QKV / SwiGLU / StoreF32): acc[token * ld_acc + feature]
   float* acc;
   int ld_acc;
@@ -50,7 +53,8 @@ struct GemmArgs {
   int H;
   __nv_bfloat16* xn;  // [tokens][H] bf16(gain_next * h) for the next norm (null: skip)
   const float* gain_next;
-  float* ssq_out;     // [tokens] sum of squares of h (null: skip)
+  float* ssq_out;     // [H / 64][ssq_stride]: per 64-column group, the sum of squares of h over the
+                      // group's columns (plain stores, no atomics; null: skip)
   // kModeQKV
   __nv_bfloat16* q_out;   // [tokens][n_q * head_dim]
   __nv_bfloat16* k_out;   // [B][n_kv][kv_seq][head_dim]
@@ -136,7 +140,7 @@ __device__ __forceinline__ void st_bf16x32(__nv_bfloat16* dst, const float (&v)[
 // `nchunks` (4, or 2 for a 64-column tile) applies to the column-independent modes (residual, store);
 // QKV and SwiGLU always take a full 128-column group.
 template <bool kFromScratch, class Load>
-__device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool valid, int col0, float& ssq_acc,
+__device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool valid, int col0,
                                              Load&& load, int nchunks = 4) {
   const int D = a.head_dim;
   if (a.mode == kModeStoreF32) {
@@ -149,6 +153,7 @@ __device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool va
     return;
   }
   if (a.mode == kModeResid) {
+    float grp = 0.f;   // sum of squares over the current 64-column group
 #pragma unroll 1
     for (int c = 0; c < nchunks; ++c) {
       float v[32];
@@ -171,9 +176,13 @@ __device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool va
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           g[j] = a.gain_next[col0 + 32 * c + j] * v[j];
-          ssq_acc += v[j] * v[j];
+          grp += v[j] * v[j];
         }
         st_bf16x32(a.xn + static_cast<size_t>(tok) * a.H + col0 + 32 * c, g);
+      }
+      if ((c & 1) && a.ssq_out) {   // the group's partial goes to its own slot
+        a.ssq_out[static_cast<size_t>((col0 + 32 * c) >> 6) * a.ssq_stride + tok] = grp;
+        grp = 0.f;
       }
     }
     return;
@@ -181,7 +190,12 @@ __device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool va
   // QKV and SwiGLU consume the pending RMSNorm's 1/rms of this token; with a feature bias (the
   // modulated norm's shift projected through the weights) the loader returns acc / rms + bias and the
   // code below sees a unit scale
-  const float s_rms = (a.ssq_in && valid) ? rsqrtf(__ldcg(a.ssq_in + tok) * a.inv_hidden + a.eps) : 1.f;
+  float s_rms = 1.f;
+  if (a.ssq_in && valid) {
+    float ss = 0.f;
+    for (int q = 0; q < a.ssq_slots; ++q) ss += __ldcg(a.ssq_in + static_cast<size_t>(q) * a.ssq_stride + tok);
+    s_rms = rsqrtf(ss * a.inv_hidden + a.eps);
+  }
   const float* bias = a.col_bias;
   const float s = bias ? 1.f : s_rms;
   auto ld = [&](int c, float (&v)[32]) {
@@ -417,18 +431,16 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
         // TMEM lane = token row of this tile
         const int tok = m_tile * 128 + lane_base + lane;
         const bool valid = tok < a.M;
-        float ssq_acc = 0.f;
         if (BN >= 128) {
           for (int g = 0; g < BN / 128; ++g) {
             const uint32_t tg = tl + g * 128;
-            row_epilogue<false>(a, tok, valid, n_tile * BN + g * 128, ssq_acc,
+            row_epilogue<false>(a, tok, valid, n_tile * BN + g * 128,
                                 [&](int c, float (&v)[32]) { tmem_ld32(tg + c * 32, v); });
           }
         } else {   // 64-column tile: residual / store modes only
-          row_epilogue<false>(a, tok, valid, n_tile * BN, ssq_acc,
+          row_epilogue<false>(a, tok, valid, n_tile * BN,
                               [&](int c, float (&v)[32]) { tmem_ld32(tl + c * 32, v); }, BN / 32);
         }
-        if (a.mode == kModeResid && a.ssq_out && valid) atomicAdd(a.ssq_out + tok, ssq_acc);
       } else {
         // lanes = output features, columns = tokens: add this split's partial sums
         const int feat = m_tile * 128 + lane_base + lane;
@@ -463,8 +475,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
           const bool valid = tok < a.tokens;
           float* row = dst + static_cast<size_t>(valid ? tok : 0) * ld + m_tile * 128;
           const bool zero_after = a.mode != kModeResid;
-          float ssq_acc = 0.f;
-          row_epilogue<true>(a, tok, valid, m_tile * 128, ssq_acc, [&](int c, float (&v)[32]) {
+            row_epilogue<true>(a, tok, valid, m_tile * 128, [&](int c, float (&v)[32]) {
             if (valid) {
               ld_f32x32(row + 32 * c, v);
             } else {
@@ -472,8 +483,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
               for (int j = 0; j < 32; ++j) v[j] = 0.f;
             }
           });
-          if (a.mode == kModeResid && a.ssq_out && valid) atomicAdd(a.ssq_out + tok, ssq_acc);
-          if (zero_after && valid) {   // leave the split-K scratch zeroed for the next launch
+            if (zero_after && valid) {   // leave the split-K scratch zeroed for the next launch
             float4* r4 = reinterpret_cast<float4*>(row);
 #pragma unroll
             for (int i = 0; i < 32; ++i) r4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -680,7 +690,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t tl = tmem + (static_cast<uint32_t>(lane_base) << 16) + buf * BN;
       const int tok = m_tile * 128 + lane_base + lane;
       const bool valid = tok < a.M;
-      float ssq_acc = 0.f;
       // FP8: the token's activation scale (0 for rows past M, whose stores are predicated off anyway)
       const float rs = kF8 && valid ? __ldg(a.row_scale + tok) : 0.f;
       auto scaled = [&](uint32_t taddr, int col, float (&v)[32]) {
@@ -701,15 +710,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int g = 0; g < BN / 128; ++g) {
           const uint32_t tg = tl + g * 128;
           const int col0 = n_tile * BN + g * 128;
-          row_epilogue<false>(a, tok, valid, col0, ssq_acc,
+          row_epilogue<false>(a, tok, valid, col0,
                               [&](int c, float (&v)[32]) { scaled(tg + c * 32, col0 + 32 * c, v); });
         }
       } else {
         const int col0 = n_tile * BN;
-        row_epilogue<false>(a, tok, valid, col0, ssq_acc,
+        row_epilogue<false>(a, tok, valid, col0,
                             [&](int c, float (&v)[32]) { scaled(tl + c * 32, col0 + 32 * c, v); }, BN / 32);
       }
-      if (a.mode == kModeResid && a.ssq_out && valid) atomicAdd(a.ssq_out + tok, ssq_acc);
       // the accumulator buffer is free for tile local + 2
       tc_fence_before();
       __syncwarp();
