@@ -396,6 +396,8 @@ def run_native(args, rank, world, local_rank):
             result["batch1"]["breakdown_ms_per_step"] = breakdown(eng, I.WORKLOADS["e2e_b1"])
     if rank == 0 and world == 1 and not args.skip_cpu:
         result["cpu_baseline"] = cpu_baseline(wl_main, budget_s=args.cpu_budget)
+        if args.cpu_configs:
+            result["cpu_baseline"]["configs_full"] = cpu_configs()
     if rank == 0:
         print(json.dumps(result), flush=True)
     eng.close()
@@ -488,12 +490,60 @@ def cpu_baseline(wl, budget_s=20.0):
     t_a = (time.perf_counter() - t1) / na
     t_chunk = d.layers * t_v + d.layers * EULER_STEPS * t_a
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    return {"value": round(1.0 / t_chunk, 6), "unit": "chunks/s", "cores": threads, "kind": "oracle",
+    return {"value": round(1.0 / t_chunk, 6), "unit": "chunks/s", "cores": host_cores(), "blas_threads": threads,
+            "kind": "oracle", "wall_s": round(time.perf_counter() - t0, 2),
             "sample": f"{nv} VLM layers (P={P}) + {na} action layer evaluations of sample 0, fp64 numpy; "
-                      f"per-chunk time = 28*{t_v:.3f}s + 280*{t_a:.4f}s"}
+                      f"per-chunk time extrapolated = 28*{t_v:.3f}s + 280*{t_a:.4f}s"}
+
+
+def host_cores():
+    """Cores this process may run on (the affinity mask, as nproc reports them)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        return os.cpu_count() or 1
+
+
+def cpu_configs():
+    """The oracle as it stands, timed in full on the host cores on the single-observation configurations:
+    one DM0-base merged layer (P = 816, S = 50), the 28-layer 10-step Euler loop over a random 816-token
+    cache, and prefill (P = 816) + 10-step denoise.  Wall seconds per configuration."""
+    import numpy as np
+
+    from oracle import dm0_oracle as O
+    from synth import inputs as I
+    d = I.DM0_BASE
+    w = I.Weights(d, seed=0)
+    out = {"cores": host_cores()}
+    hp = I.hidden_states(816, d.hidden_v, seed=10)
+    hs = I.hidden_states(d.chunk, d.hidden_a, seed=110)
+    w.layer(0, 0), w.layer(1, 0)
+    t0 = time.perf_counter()
+    O.merged_layer(w.layer(0, 0), w.layer(1, 0), hp, hs, d)
+    out["merged_layer_s"] = round(time.perf_counter() - t0, 3)
+    ks, vs = [], []
+    for l in range(d.layers):
+        k, v = I.random_kv_layer(d, 1, 816, l)
+        ks.append(k[0].astype(np.float64))
+        vs.append(v[0].astype(np.float64))
+        w.layer(1, l)
+    noise = I.noise(d, 1)[0]
+    t0 = time.perf_counter()
+    O.denoise(w, ks, vs, noise, EULER_STEPS)
+    out["denoise_b1_s"] = round(time.perf_counter() - t0, 3)
+    emb = I.prefix_embeddings(d, 1, 816)
+    for l in range(d.layers):
+        w.layer(0, l)
+    t0 = time.perf_counter()
+    O.infer(w, emb, I.noise(d, 1), EULER_STEPS)
+    out["e2e_b1_s"] = round(time.perf_counter() - t0, 3)
+    return out
 
 
 def run_reference(args, rank, world):
+    """The reference arm: the oracle as it stands on the host cores.  Each step is one bounded sample
+    (cpu_baseline) of the workload; ms_per_step is the wall time of a sample step as run, and value is
+    the chunks/s the samples extrapolate to (the per-layer times scaled to a whole chunk)."""
     if rank != 0:
         return
     from synth import inputs as I
@@ -502,15 +552,19 @@ def run_reference(args, rank, world):
     budget = max(5.0, min(30.0, 150.0 / (steps + warmup)))
     for _ in range(warmup):
         cpu_baseline(wl, budget_s=budget / 3)
+    t0 = time.perf_counter()
     vals = [cpu_baseline(wl, budget_s=budget) for _ in range(steps)]
+    wall_ms = 1000.0 * (time.perf_counter() - t0) / steps
     v = sum(x["value"] for x in vals) / len(vals)
     cb = dict(vals[-1])
     cb["value"] = round(v, 6)
     res = {"impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": "chunks/s", "n_gpus": world,
-           "steps": steps, "warmup": warmup, "ms_per_step": round(1000.0 / v, 1), "higher_is_better": True,
+           "steps": steps, "warmup": warmup, "ms_per_step": round(wall_ms, 1), "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "value_basis": "extrapolated: each step times whole VLM layers and action-layer evaluations of one "
+                          "sample and scales them to a chunk (28 VLM layers + 280 action layers per sample)",
            "config": {"workload": f"{wl.name}: prefill B={wl.batch} x P={wl.prefix} + {EULER_STEPS}-step denoise "
-                                  "(bounded per-layer sample, scaled per chunk)"},
+                                  "(bounded per-layer sample per step, scaled per chunk)"},
            "cpu_baseline": cb, "e2e": {"value": round(v, 6), "unit": "chunks/s", "h2d_bytes_per_step": 0,
                                        "d2h_bytes_per_step": 0}}
     print(json.dumps(res), flush=True)
@@ -569,6 +623,90 @@ def run_b1_loop(args):
     eng.close()
 
 
+# ------------------------------------------------------------------ phase timeline of the single-launch loop
+
+# per (phase, CTA) %globaltimer marks of the persistent Euler loop: 0 phase start, 1 operand staged, 2 first
+# accumulator (or S tile) ready, 3 results issued, 4 release fence done, 5 barrier arrival, 6 MMA warp saw
+# the operand, 7 MMA warp issued its last MMA, 8 operand copies issued, 9 copies landed, 10..15 attention
+TRACE_SLOTS = 16
+TRACE_PHASES = ("qkv", "attention", "o_proj", "gate_up", "down")
+
+
+def summarize_loop_trace(arr, layers, items):
+    """Per phase type, medians over the CTAs (the attention phase: its first `items` CTAs) and the layer
+    passes, in microseconds from the phase's start: staged (operand in shared memory), copies (the operand
+    copies in flight), acc_ready (first accumulator or S tile), issued (results out), arrived (this CTA's
+    barrier arrival); and the phase's wall time (the latest start of the next phase minus its own latest
+    start) and last_arrival (the latest arrival minus the latest start).  arr: [rows][CTAs][TRACE_SLOTS]
+    ns; row 0 is the first input, then per Euler step 5 rows per layer and one step boundary."""
+    import numpy as np
+    arr = np.asarray(arr, np.float64) / 1000.0
+    per_step = 5 * layers + 1
+    acc = {}
+    for q in range(1, arr.shape[0] - 1):
+        rr = (q - 1) % per_step
+        name = "step" if rr == 5 * layers else TRACE_PHASES[rr % 5]
+        a = arr[q, :items] if name == "attention" else arr[q]
+        st = a[:, 0]
+        rec = {"staged": np.median(a[:, 1] - st), "copies": np.median(a[:, 9] - a[:, 8]),
+               "acc_ready": np.median(a[:, 2] - st), "issued": np.median(a[:, 3] - st),
+               "arrived": np.median(a[:, 5] - st),
+               "phase": float(arr[q + 1, :, 0].max() - arr[q, :, 0].max()),
+               "last_arrival": float(arr[q, :, 5].max() - arr[q, :, 0].max())}
+        if name == "step":
+            rec = {"phase": rec["phase"]}
+        acc.setdefault(name, []).append(rec)
+    return {k: {kk: round(float(np.mean([x[kk] for x in v])), 2) for kk in v[0]} for k, v in acc.items()}
+
+
+def run_b1_trace(args):
+    """Profiling workload: the single-launch Euler loop of one observation at DM0-base widths over a
+    random 816-token cache, traced (DM0_PERSIST_TRACE=1 set here before the context is created): every
+    CTA stamps %globaltimer at fixed points of each phase.  Prints the loop's CUDA-event time and the
+    per-phase medians of summarize_loop_trace."""
+    os.environ["DM0_PERSIST_TRACE"] = "1"
+    import numpy as np
+    import torch
+
+    from synth import inputs as I
+    from vla_dual_expert_b200 import Engine
+    d = I.DM0_BASE.replace(layers=args.trace_layers)
+    P, steps = 816, 2
+    eng = Engine(d, 1, P)
+    eng.load_from(I.Weights(d, seed=0))
+    n = d.layers * d.n_kv * P * d.head_dim
+    g = torch.Generator(device="cuda").manual_seed(3000)
+    for ptr in eng.kv_view():   # the context-owned cache planes, filled in place with N(0, 1)
+        view = type("Plane", (), {"__cuda_array_interface__": {"shape": (n,), "typestr": "<u2",
+                                                                "data": (ptr, False), "version": 3}})()
+        torch.as_tensor(view, device="cuda").view(torch.bfloat16).normal_(generator=g)
+    eng.kv_commit(1, P)
+    noise = torch.from_numpy(I.noise(d, 1)).cuda()
+    for _ in range(3):
+        eng.denoise(noise, steps)
+    eng.sync()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    eng.denoise(noise, steps)
+    e1.record()
+    eng.sync()
+    torch.cuda.synchronize()
+    nsm = torch.cuda.get_device_properties(0).multi_processor_count
+    rows = 1 + steps * (5 * d.layers + 1)
+    ptr = eng.debug_view("loop_trace")
+    view = type("Trace", (), {"__cuda_array_interface__": {"shape": (rows * nsm * TRACE_SLOTS,), "typestr": "<u8",
+                                                            "data": (ptr, False), "version": 3}})()
+    arr = torch.as_tensor(view, device="cuda").cpu().numpy().reshape(rows, nsm, TRACE_SLOTS)
+    arr = arr.astype(np.float64) - float(arr[0, :, 0].min())
+    splits = min(int(os.environ.get("DM0_PERSIST_SPLITS", "7")), 8)
+    nblk = (P + 63) // 64 + 1
+    bps = -(-nblk // min(splits, nblk))
+    items = d.n_kv * (-(-nblk // bps))
+    print(json.dumps({"b1_trace": "ok", "denoise_ms": round(e0.elapsed_time(e1), 3), "steps": steps,
+                      "layers": d.layers, "phases_us": summarize_loop_trace(arr, d.layers, items)}))
+    eng.close()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -582,7 +720,12 @@ def main():
     ap.add_argument("--skip-breakdown", action="store_true")
     ap.add_argument("--one-layer", action="store_true", help="profiling workload: one layer, B=16, P=2048")
     ap.add_argument("--b1-loop", action="store_true", help="profiling workload: persistent Euler loop, 3 layers, B=1")
+    ap.add_argument("--b1-trace", action="store_true",
+                    help="profiling workload: per-phase timeline of the single-launch Euler loop")
+    ap.add_argument("--trace-layers", type=int, default=28)
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--cpu-configs", action="store_true",
+                    help="also time the oracle in full on the single-observation configurations (~1-2 min)")
     ap.add_argument("--train", action="store_true",
                     help="also time one flow-matching training step (reported under train)")
     ap.add_argument("--time-mod", action="store_true",
@@ -603,6 +746,9 @@ def main():
         return
     if args.b1_loop:
         run_b1_loop(args)
+        return
+    if args.b1_trace:
+        run_b1_trace(args)
         return
     run_native(args, rank, world, local_rank)
 

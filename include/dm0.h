@@ -127,8 +127,6 @@ dm0_status dm0_load_weights(dm0_ctx* ctx, const void* blob, size_t bytes);
  *   prefix_emb: device bf16 [B][P][hidden_v] prefix embeddings.
  * The cache holds, per layer, K after QK-norm and RoPE (positions 0..P-1) and
  * V, as two planes of bf16 [layers][B][n_kv][P][head_dim] (see dm0_kv_view).
- * DM0_FA_PREFIX_DEEP=1 at dm0_create runs its attention on the deeper
- * attention instance (more K/V prefetch, two P buffers; equal up to rounding).
  * Returns DM0_ESHAPE unless 1 <= B <= max_batch and 1 <= P <= max_prefix. */
 dm0_status dm0_prefill(dm0_ctx* ctx, const void* prefix_emb, int B, int P, void* stream);
 

@@ -55,10 +55,10 @@ def qkv(w, h, positions, d):
 
 def attention(q, k, v, key_splits=1, prefix=None):
     """Every query row over all keys (the mask is expressed by which keys are passed), bf16 softmax
-    weights in the PV product.  With key_splits > 1 the keys are cut into 64-key blocks (the first
-    `prefix` keys, then the rest as one more block, as the Euler loop walks [prefix cache; suffix]),
-    the blocks into key_splits contiguous ranges, and each range's normalised output is rounded to
-    bf16 before the exact combine."""
+    weights in the PV product.  With key_splits > 1 (the single-launch Euler loop) the keys are cut into
+    64-key blocks (the first `prefix` keys, then the rest as one more block, as the loop walks [prefix
+    cache; suffix]), the blocks into key_splits contiguous ranges, and each range's normalised output is
+    rounded to bf16 before the exact combine."""
     Hq, Tq, D = q.shape
     G = Hq // k.shape[0]
     Tk = k.shape[1]

@@ -95,7 +95,6 @@ struct dm0_ctx {
   bool use_persist = true;
   int persist_splits = 7;
   bool persist_fast_bar = false;   // DM0_PERSIST_FASTBAR=1: release-reduction grid barrier arrival
-  bool fa_prefix_deep = false;     // DM0_FA_PREFIX_DEEP=1: the prefix pass uses the deep attention instance
   int persist_resident = -1;   // -1: not checked yet
   // true when the previous operation this context queued on the stream was one of its own
   // kernels: only then may the next kernel overlap it (programmatic dependent launch).  The first
@@ -540,7 +539,7 @@ dm0_status run_attn(dm0_ctx* c, cudaStream_t s, const bf16* q, int seq_q, const 
     // prefix pass (K/V blocks shared by many CTAs through L2), and the suffix attention of small
     // batches: two CTAs per SM, small enough (113 KB, 24.5K registers) to share an SM with a
     // swapped GEMM CTA, so neighbouring kernels overlap under programmatic dependent launch
-    if ((len_b == 0 && !c->fa_prefix_deep) || groups * tiles * fs <= c->num_sms / 2)
+    if (len_b == 0 || groups * tiles * fs <= c->num_sms / 2)
       return launch(c, s, dm0::fa_tc_kernel<2, 1>, grid, dim3(dm0::kFaThreads), dm0::FaSmemT<2, 1>::kBytes, tk, tv,
                     tkb, tvb, a);
     // merged suffix attention: the cached prefix is read from DRAM once; deeper K/V prefetch and
@@ -717,6 +716,8 @@ dm0_status step(dm0_ctx* c, cudaStream_t s, int B, int k_out, int k_in, int step
   StepArgs a{};
   a.x = c->x;
   a.h = c->h_a;
+  a.h_ts = cf.hidden_a;
+  a.h_fs = 1;
   a.xn = c->xn_a;
   a.ssq = c->ssq_a;   // the attention norm's [Ha / 64][tokens] block
   a.n_slots = cf.hidden_a / 64;
@@ -926,6 +927,8 @@ bool persist_plan(dm0_ctx* c, int steps, float* vel, dm0::PdArgs* a, std::string
   StepArgs& st = a->step;
   st.x = c->x;
   st.h = c->h_a;
+  st.h_ts = g.hidden_a;
+  st.h_fs = 1;
   st.xn = nullptr;
   st.ssq = nullptr;
   st.n_slots = 0;
@@ -1212,7 +1215,6 @@ dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
   if (const char* e = std::getenv("DM0_NO_PERSIST")) c->use_persist = e[0] == '0';
   if (const char* e = std::getenv("DM0_PERSIST_SPLITS")) c->persist_splits = std::max(1, std::atoi(e));
   if (const char* e = std::getenv("DM0_PERSIST_FASTBAR")) c->persist_fast_bar = e[0] == '1';
-  if (const char* e = std::getenv("DM0_FA_PREFIX_DEEP")) c->fa_prefix_deep = e[0] == '1';
 
   // weights: one allocation, 256-byte aligned sub-buffers
   size_t total = 0;

@@ -43,7 +43,8 @@ __global__ void __launch_bounds__(256) rows_prep_kernel(const void* in, int in_b
 
 struct StepArgs {
   float* x;                    // [tokens][A] flow state
-  float* h;                    // [tokens][Ha] action residual stream
+  float* h;                    // action residual stream: element (token, j) at h[token * h_ts + j * h_fs]
+  int h_ts, h_fs;              // [tokens][Ha] row-major: (Ha, 1); feature-major [Ha][64]: (1, 64)
   __nv_bfloat16* xn;           // [tokens][Ha] bf16(attn_norm_0 * h)
   float* ssq;                  // [n_slots][tokens]
   int n_slots, tokens;
@@ -73,12 +74,12 @@ template <bool kMod = false, class Sync>
 __device__ __forceinline__ void step_token(const StepArgs& a, int tok, int tid, int nthr, float* sx, float* sred,
                                            float* hs, Sync&& sync, const float* final_shift = nullptr) {
   const int nw = nthr >> 5, warp = tid >> 5, lane = tid & 31;
-  float* hrow = a.h + static_cast<size_t>(tok) * a.Ha;
+  float* hrow = a.h + static_cast<size_t>(tok) * a.h_ts;
   const bool vec_out = (a.Ha % 256) == 0, vec_in = (a.A % 8) == 0;
   if (a.k_out >= 0) {
     float sq = 0.f;
     for (int j = tid; j < a.Ha; j += nthr) {
-      const float hv = __ldcg(hrow + j);
+      const float hv = __ldcg(hrow + static_cast<size_t>(j) * a.h_fs);
       hs[j] = hv * a.final_norm[j];
       sq += hv * hv;
     }
@@ -149,7 +150,7 @@ __device__ __forceinline__ void step_token(const StepArgs& a, int tok, int tid, 
         const float arg = t * exp2f(-static_cast<float>(fi) / half * kLog2_10000);
         e += j < half ? sinf(arg) : cosf(arg);
       }
-      hrow[j] = e;
+      hrow[static_cast<size_t>(j) * a.h_fs] = e;
       if (a.xn) a.xn[static_cast<size_t>(tok) * a.Ha + j] = __float2bfloat16_rn(a.attn_norm0[j] * e);
       sq += e * e;
     }
