@@ -571,25 +571,41 @@ def run_reference(args, rank, world):
 
 
 def run_one_layer(args):
-    """Profiling workload: one DM0-base layer (both experts) at B=16, P=2048 — two iterations of
-    dm0_prefill + a 1-step dm0_denoise with per-step velocities (direct launches).  Holds about 2 GB
-    on the device, small enough for full ncu captures of every kernel of the step."""
+    """Profiling workload: one DM0-base layer (both experts), by default at B=16, P=2048 — two
+    iterations of dm0_prefill + a 1-step dm0_denoise with per-step velocities (direct launches).
+    Holds about 2 GB on the device, small enough for full ncu captures of every kernel of the step.
+    --batch / --prefix change the shape, --prefix-fp8 runs the VLM MLP in FP8 E4M3, and --train adds
+    two flow-matching training steps of the layer after the inference iterations."""
+    import numpy as np
     import torch
 
     from synth import inputs as I
     from vla_dual_expert_b200 import Engine
     d = I.DM0_BASE.replace(layers=1)
-    B, P = 16, 2048
+    B, P = args.batch or 16, args.prefix or 2048
     eng = Engine(d, B, P)
     eng.load_from(I.Weights(d, seed=0))
+    if args.prefix_fp8:
+        eng.set_prefix_fp8(True)
     emb = torch.from_numpy(I.prefix_embeddings(d, B, P)).cuda().to(torch.bfloat16)
     noise = torch.from_numpy(I.noise(d, B)).cuda()
     vel = torch.empty((1, B, d.chunk, d.action_dim), device="cuda", dtype=torch.float32)
     for _ in range(2):
         eng.prefill(emb)
         eng.denoise(noise, 1, velocities=vel)
+    out = {"one_layer": "ok", "batch": B, "prefix": P, "prefix_fp8": bool(args.prefix_fp8),
+           "mean_abs_velocity": float(vel.abs().mean())}
+    if args.train:
+        a_np, e_np, t_np, m_np = I.train_batch(d, B, seed=4000)
+        ta, te = torch.from_numpy(a_np).cuda(), torch.from_numpy(e_np).cuda()
+        tt = torch.from_numpy(t_np.astype(np.float32)).cuda()
+        tm_ = torch.from_numpy(m_np.astype(np.uint8)).cuda()
+        grads = torch.empty(eng.grad_floats(), device="cuda", dtype=torch.float32)
+        for _ in range(2):
+            loss, _ = eng.train_step(ta, te, tt, tm_, grads=grads)
+        out["train_loss"] = float(loss.item())
     eng.sync()
-    print(json.dumps({"one_layer": "ok", "mean_abs_velocity": float(vel.abs().mean())}))
+    print(json.dumps(out))
     eng.close()
 
 
@@ -719,6 +735,8 @@ def main():
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-breakdown", action="store_true")
     ap.add_argument("--one-layer", action="store_true", help="profiling workload: one layer, B=16, P=2048")
+    ap.add_argument("--batch", type=int, default=0, help="--one-layer: batch (default 16)")
+    ap.add_argument("--prefix", type=int, default=0, help="--one-layer: prefix length (default 2048)")
     ap.add_argument("--b1-loop", action="store_true", help="profiling workload: persistent Euler loop, 3 layers, B=1")
     ap.add_argument("--b1-trace", action="store_true",
                     help="profiling workload: per-phase timeline of the single-launch Euler loop")

@@ -54,6 +54,8 @@ struct FaSmemT {
   static constexpr uint32_t kOffBar = kOffX + kX;
   static constexpr uint32_t kSlack = 256;                   // the dynamic base is 1024-aligned (no static smem)
   static constexpr uint32_t kBytes = kOffBar + 256 + kSlack;
+  // barriers (K and V rings, S double buffer, P buffers, Q, drain), the TMEM slot and the abort flag
+  static_assert((4 * ST + 4 + 2 * NP + 2) * 8 + 8 <= 256, "barrier area");
 };
 // Prefix pass: 2 K/V stages, one P buffer (112 KB): two CTAs per SM, K/V blocks shared by many CTAs
 // through L2.  Suffix attention: 4 K/V stages and two P buffers (192 KB, one CTA per SM): deeper
@@ -113,9 +115,13 @@ __global__ void __launch_bounds__(FaWarps<NP>::kThreads, NP == 1 ? 2 : 1)
     return;
   }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + FS::kOffBar);
-  uint64_t* kv_full = bars;             // [ST] TMA landed K_j, V_j
-  uint64_t* kv_empty = bars + ST;       // [ST] PV_j done: K/V slot free
-  uint64_t* s_full = bars + 2 * ST;     // [2] S_j in TMEM
+  // K and V have their own rings: K_j's slot is free once S_j completed, V_j's only after PV_j, so
+  // the next K blocks are requested a whole PV earlier than a shared K/V slot would allow
+  uint64_t* k_full = bars;              // [ST] TMA landed K_j
+  uint64_t* v_full = bars + ST;         // [ST] TMA landed V_j
+  uint64_t* k_empty = bars + 2 * ST;    // [ST] S_j done: K slot free
+  uint64_t* v_empty = bars + 3 * ST;    // [ST] PV_j done: V slot free
+  uint64_t* s_full = bars + 4 * ST;     // [2] S_j in TMEM
   uint64_t* s_free = s_full + 2;        // [2] softmax finished reading S_j
   uint64_t* p_full = s_free + 2;        // [NP] P_j in buffer j % NP and O corrected
   uint64_t* pv_done = p_full + NP;      // [NP] PV_j (which read buffer j % NP) finished
@@ -138,8 +144,10 @@ __global__ void __launch_bounds__(FaWarps<NP>::kThreads, NP == 1 ? 2 : 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < ST; ++i) {
-      mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&k_full[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
@@ -174,41 +182,48 @@ __global__ void __launch_bounds__(FaWarps<NP>::kThreads, NP == 1 ? 2 : 1)
         tma_prefetch_desc(&tmVb);
       }
       const uint64_t pol = policy_evict_last();
-      auto issue = [&](int j) {
+      // block j of K (v = 0) or V (v = 1) into slot j % ST
+      auto issue = [&](int j, int v) {
         const int s = j % ST;
         const int jj = jb0 + j;   // global block index
         const bool segA = jj < nA;
-        const CUtensorMap* mk = segA ? &tmK : &tmKb;
-        const CUtensorMap* mv = segA ? &tmV : &tmVb;
+        const CUtensorMap* m = v ? (segA ? &tmV : &tmVb) : (segA ? &tmK : &tmKb);
         const int row = segA ? grp * a.len_a + jj * 64 : grp * a.len_b + (jj - nA) * 64;
-        mbar_arrive_expect_tx(&kv_full[s], 2 * FS::kKV);
-        uint8_t* kd = smem + FS::kOffK + s * FS::kKV;
-        uint8_t* vd = smem + FS::kOffV + s * FS::kKV;
-        tma_load_2d(kd, mk, &kv_full[s], 0, row, pol);
-        tma_load_2d(kd + FS::kHalfKV, mk, &kv_full[s], 64, row, pol);
-        tma_load_2d(vd, mv, &kv_full[s], 0, row, pol);
-        tma_load_2d(vd + FS::kHalfKV, mv, &kv_full[s], 64, row, pol);
+        uint64_t* bar = v ? &v_full[s] : &k_full[s];
+        uint8_t* dst = smem + (v ? FS::kOffV : FS::kOffK) + s * FS::kKV;
+        mbar_arrive_expect_tx(bar, FS::kKV);
+        tma_load_2d(dst, m, bar, 0, row, pol);
+        tma_load_2d(dst + FS::kHalfKV, m, bar, 64, row, pol);
       };
       // segment A written before the previous kernel (the prefix cache during the Euler loop) may be
       // requested before the dependency wait
-      int issued = 0;
+      int nk = 0, nv = 0;   // K and V blocks issued
       if (a.a_stable)
-        for (; issued < ST && issued < nblk && jb0 + issued < nA; ++issued) issue(issued);
-      pdl_wait();
-      for (int j = issued; j < nblk; ++j) {
-        const int s = j % ST;
-        if (j >= ST && !mbar_wait(&kv_empty[s], ((j / ST) - 1) & 1, abort_flag)) {
-          *abort_flag = 1;
-          raise_error(a.err, kErrTimeoutProducer);
-          break;
+        for (; nk < ST && nk < nblk && jb0 + nk < nA; ++nk) {
+          issue(nk, 0);
+          issue(nk, 1);
         }
-        issue(j);
-        issued = j + 1;
+      nv = nk;
+      pdl_wait();
+      for (int j = nk; j < nblk; ++j) {
+        const int s = j % ST;
+        const uint32_t par = ((j / ST) - 1) & 1;
+        if (j >= ST && !mbar_wait(&k_empty[s], par, abort_flag)) break;
+        issue(j, 0);
+        nk = j + 1;
+        if (j >= ST && !mbar_wait(&v_empty[s], par, abort_flag)) break;
+        issue(j, 1);
+        nv = j + 1;
       }
-      for (int j = issued - ST; j < issued; ++j) {   // copies in flight land before the CTA exits
-        if (j < 0) continue;
-        if (!mbar_wait(&kv_full[j % ST], (j / ST) & 1, nullptr, kDrainTimeoutNs)) raise_error(a.err, kErrDrain);
+      if (nv < nblk) {
+        *abort_flag = 1;
+        raise_error(a.err, kErrTimeoutProducer);
       }
+      // copies in flight land before the CTA exits
+      for (int j = nk - ST; j < nk; ++j)
+        if (j >= 0 && !mbar_wait(&k_full[j % ST], (j / ST) & 1, nullptr, kDrainTimeoutNs)) raise_error(a.err, kErrDrain);
+      for (int j = nv - ST; j < nv; ++j)
+        if (j >= 0 && !mbar_wait(&v_full[j % ST], (j / ST) & 1, nullptr, kDrainTimeoutNs)) raise_error(a.err, kErrDrain);
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
@@ -219,6 +234,7 @@ __global__ void __launch_bounds__(FaWarps<NP>::kThreads, NP == 1 ? 2 : 1)
       bool ok = mbar_wait(q_ready, 0, abort_flag);
       auto pv = [&](int i) -> bool {
         if (!mbar_wait(&p_full[i % NP], (i / NP) & 1, abort_flag)) return false;
+        if (!mbar_wait(&v_full[i % ST], (i / ST) & 1, abort_flag)) return false;
         tc_fence_after();
         const uint32_t pa = smem_u32(smem + FS::kOffP + (i % NP) * FS::kP);
         const uint32_t vb = smem_u32(smem + FS::kOffV + (i % ST) * FS::kKV);
@@ -227,13 +243,13 @@ __global__ void __launch_bounds__(FaWarps<NP>::kThreads, NP == 1 ? 2 : 1)
           umma_bf16(tmem + 128, sw128_kmajor_desc(pa + ks * 32), sw128_mnmajor_desc(vb + ks * 2048, FS::kHalfKV),
                     idesc_pv, (i > 0 || ks > 0) ? 1u : 0u);
         umma_commit(&pv_done[i % NP]);
-        umma_commit(&kv_empty[i % ST]);
+        umma_commit(&v_empty[i % ST]);
         return true;
       };
       for (int j = 0; ok && j < nblk; ++j) {
         const int s = j & 1;          // S buffer
         const int kvs = j % ST;       // K/V slot
-        if (!mbar_wait(&kv_full[kvs], (j / ST) & 1, abort_flag)) {
+        if (!mbar_wait(&k_full[kvs], (j / ST) & 1, abort_flag)) {
           ok = false;
           break;
         }
@@ -248,6 +264,7 @@ __global__ void __launch_bounds__(FaWarps<NP>::kThreads, NP == 1 ? 2 : 1)
           umma_bf16(tmem + s * 64, sw128_kmajor_desc(qa + (ks >> 2) * 16384 + (ks & 3) * 32),
                     sw128_kmajor_desc(kb + (ks >> 2) * FS::kHalfKV + (ks & 3) * 32), idesc_s, ks > 0 ? 1u : 0u);
         umma_commit(&s_full[s]);
+        umma_commit(&k_empty[kvs]);
         if (j >= 1 && !pv(j - 1)) {
           ok = false;
           break;

@@ -137,6 +137,102 @@ __device__ __forceinline__ void st_bf16x32(__nv_bfloat16* dst, const float (&v)[
                        bf2(v[8 * i + 6], v[8 * i + 7]));
 }
 
+// Residual epilogue of the persistent (normal-orientation) GEMM with coalesced global traffic.  A
+// warp's 32 tokens are TMEM lanes 32w..32w+31; for each 32-column chunk the warp passes h through a
+// per-warp shared scratch, so h is read and written as whole 128-byte row pieces (4 rows per warp
+// instruction) and the bf16 norm operand as 64-byte pieces (8 rows), where a thread-per-row access
+// touches 32 rows per instruction.  The next chunk of h is requested before the current one is
+// used.  Same results as row_epilogue's residual mode.
+struct ResidScratch {
+  static constexpr int kLd = 36;    // fp32 words per scratch row: 16-byte aligned, rows 4 banks apart
+  static constexpr int kLdX = 20;   // 32-bit words per bf16 row (32 values + pad)
+  static constexpr uint32_t kBytes = 32 * kLd * 4 + 32 * kLdX * 4;
+};
+
+template <class Load>
+__device__ __forceinline__ void resid_epilogue_warp(const GemmArgs& a, int row0, int col0, int nchunks,
+                                                    float* scr, Load&& load) {
+  constexpr int kLd = ResidScratch::kLd, kLdX = ResidScratch::kLdX;
+  const int lane = threadIdx.x & 31;
+  const int tok = row0 + lane;
+  const bool valid = tok < a.M;
+  uint32_t* xs = reinterpret_cast<uint32_t*>(scr + 32 * kLd);
+  const int qr = lane >> 3, qc = lane & 7;   // h piece of this lane: row 4 i + qr, float4 qc
+  float4 hn[8];
+  auto fetch = [&](int c) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = row0 + 4 * i + qr;
+      hn[i] = r < a.M ? __ldcg(reinterpret_cast<const float4*>(a.h + static_cast<size_t>(r) * a.H + col0 + 32 * c) + qc)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  fetch(0);
+  float grp = 0.f;   // sum of squares over the current 64-column group
+#pragma unroll 1
+  for (int c = 0; c < nchunks; ++c) {
+    const int cc = col0 + 32 * c;
+    float v[32];
+    load(c, v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) *reinterpret_cast<float4*>(scr + (4 * i + qr) * kLd + 4 * qc) = hn[i];
+    if (c + 1 < nchunks) fetch(c + 1);
+    __syncwarp();
+    float* mine = scr + lane * kLd;
+#pragma unroll
+    for (int j4 = 0; j4 < 8; ++j4) {
+      const float4 hv = *reinterpret_cast<const float4*>(mine + 4 * j4);
+      if (a.col_gate) {
+        const float4 gt = __ldg(reinterpret_cast<const float4*>(a.col_gate + cc) + j4);
+        v[4 * j4] *= gt.x;
+        v[4 * j4 + 1] *= gt.y;
+        v[4 * j4 + 2] *= gt.z;
+        v[4 * j4 + 3] *= gt.w;
+      }
+      v[4 * j4] += hv.x;
+      v[4 * j4 + 1] += hv.y;
+      v[4 * j4 + 2] += hv.z;
+      v[4 * j4 + 3] += hv.w;
+      *reinterpret_cast<float4*>(mine + 4 * j4) = make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
+    }
+    if (a.xn) {
+#pragma unroll
+      for (int j8 = 0; j8 < 4; ++j8) {
+        const float4 g0 = __ldg(reinterpret_cast<const float4*>(a.gain_next + cc) + 2 * j8);
+        const float4 g1 = __ldg(reinterpret_cast<const float4*>(a.gain_next + cc) + 2 * j8 + 1);
+        const float* w = v + 8 * j8;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) grp += w[j] * w[j];
+        *reinterpret_cast<uint4*>(xs + lane * kLdX + 4 * j8) =
+            make_uint4(bf2(g0.x * w[0], g0.y * w[1]), bf2(g0.z * w[2], g0.w * w[3]), bf2(g1.x * w[4], g1.y * w[5]),
+                       bf2(g1.z * w[6], g1.w * w[7]));
+      }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = 4 * i + qr;
+      if (row0 + r < a.M)
+        reinterpret_cast<float4*>(a.h + static_cast<size_t>(row0 + r) * a.H + cc)[qc] =
+            *reinterpret_cast<const float4*>(scr + r * kLd + 4 * qc);
+    }
+    if (a.xn) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = 8 * i + (lane >> 2), q = lane & 3;
+        if (row0 + r < a.M)
+          reinterpret_cast<uint4*>(a.xn + static_cast<size_t>(row0 + r) * a.H + cc)[q] =
+              *reinterpret_cast<const uint4*>(xs + r * kLdX + 4 * q);
+      }
+    }
+    if ((c & 1) && a.ssq_out) {   // the group's partial goes to its own slot
+      if (valid) a.ssq_out[static_cast<size_t>(cc >> 6) * a.ssq_stride + tok] = grp;
+      grp = 0.f;
+    }
+    __syncwarp();   // the scratch is rewritten by the next chunk
+  }
+}
+
 // `nchunks` (4, or 2 for a 64-column tile) applies to the column-independent modes (residual, store);
 // QKV and SwiGLU always take a full 128-column group.
 template <bool kFromScratch, class Load>
@@ -533,8 +629,11 @@ struct PGemmSmem {
   static constexpr uint32_t kB = BN * 128;
   static constexpr uint32_t kStage = kA + kB;
   static constexpr uint32_t kPipe = STAGES * kStage;
-  static constexpr uint32_t kBytes = kPipe + 256 + 1024;
+  static constexpr uint32_t kOffScr = kPipe + 256;            // after the barriers
+  static constexpr uint32_t kScrWarp = ResidScratch::kBytes;  // per epilogue warp
+  static constexpr uint32_t kBytes = kOffScr + 4 * kScrWarp + 1024;
   static constexpr uint32_t kTmemCols = 2 * BN;
+  static_assert(kBytes <= 232448, "shared memory per CTA");
 };
 
 // kF8: both operands FP8 E4M3 (tensor maps of bytes), a k-block is 128 values instead of 64 (the
@@ -676,6 +775,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else {
     const int lane_base = (warp & 3) * 32;
     pdl_wait();
+    // residual epilogue: each thread reads its token's BN fp32 values of h, one DRAM round trip per
+    // 32-column chunk; the rows of the CTA's next tile are requested into L2 one tile ahead, so
+    // those loads hit L2 while the accumulator of the current tile drains
+    auto prefetch_rows = [&](int t) {
+      if (a.mode != kModeResid || t >= ntiles) return;
+      int m_tile, n_tile;
+      band_tile(t, mt, a.N / BN, m_tile, n_tile);
+      const int tok = m_tile * 128 + lane_base + lane;
+      if (tok < a.M) prefetch_l2_bulk(a.h + static_cast<size_t>(tok) * a.H + n_tile * BN, BN * 4);
+    };
+    prefetch_rows(blockIdx.x);
     int local = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++local) {
       const int buf = local & 1;
@@ -685,6 +795,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after();
+      prefetch_rows(t + gridDim.x);
       int m_tile, n_tile;
       band_tile(t, mt, a.N / BN, m_tile, n_tile);
       const uint32_t tl = tmem + (static_cast<uint32_t>(lane_base) << 16) + buf * BN;
@@ -706,7 +817,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       };
-      if (BN >= 128) {
+      if (a.mode == kModeResid) {
+        float* scr = reinterpret_cast<float*>(smem + L::kOffScr + (warp - 2) * L::kScrWarp);
+        const int row0 = m_tile * 128 + lane_base;
+        for (int g = 0; g < (BN >= 128 ? BN / 128 : 1); ++g) {
+          const uint32_t tg = tl + g * 128;
+          const int col0 = n_tile * BN + g * 128;
+          resid_epilogue_warp(a, row0, col0, BN >= 128 ? 4 : BN / 32, scr,
+                              [&](int c, float (&v)[32]) { scaled(tg + c * 32, col0 + 32 * c, v); });
+        }
+      } else if (BN >= 128) {
         for (int g = 0; g < BN / 128; ++g) {
           const uint32_t tg = tl + g * 128;
           const int col0 = n_tile * BN + g * 128;
