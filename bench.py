@@ -34,15 +34,14 @@ METRIC = "action chunks/sec (prefill+10-step denoise) at batch 1 and 16; HBM GB/
 EULER_STEPS = 10
 # DRAM bytes (read + write) of one prefix-pass gate/up GEMM launch at B=16, P=2048 (M=32768,
 # N=12288, K=2048), from an ncu capture of the same kernel and launch shape in `bench.py --one-layer`
-# (3.079 GB read + 0.353 GB written)
-# Both kernels gained hooks since (null in this configuration, same tiling and raster), so the
-# figures are reported as null until the counters are taken again on the current build.
-COUNTERS_CURRENT = False
-GATEUP_TRAFFIC_BYTES = 3.432e9
+# on the current build (n-fastest raster): 0.417 GB read + 0.381 GB written, against 0.587 GB
+# algorithmic (activations 134 MB + weights 50 MB read, SwiGLU output 403 MB written)
+COUNTERS_CURRENT = True
+GATEUP_TRAFFIC_BYTES = 0.7987e9
 # DRAM bytes (read + write) of the persistent Euler loop per step of 28 action layers at B=1, P=816:
-# the ncu capture of `bench.py --b1-loop` (3 layers, 1 step: 104.79 MB read + 4.15 MB written)
+# the ncu capture of `bench.py --b1-loop` (3 layers, 1 step: 104.80 MB read + 4.71 MB written)
 # scaled by 28/3
-LOOP_TRAFFIC_BYTES_PER_STEP = 1.0168e9
+LOOP_TRAFFIC_BYTES_PER_STEP = 1.0221e9
 
 
 def _peaks():
@@ -134,6 +133,52 @@ def denoise_bytes_per_step(d, B, P):
     w = d.layers * layer_params(d, 1) * 2
     kv = d.layers * B * d.n_kv * P * d.head_dim * 2 * 2
     return w + kv
+
+
+def site_work(d, B, P, name):
+    """Algorithmic work of one launch of a probed kernel site: (amount, kind) with kind "flop" (a
+    tensor-core contraction) or "byte" (the merged suffix attention, which reads the prefix cache
+    once); None for sites without a roofline (the Euler step, the single-launch loop)."""
+    D, nq, nkv, S = d.head_dim, d.n_q, d.n_kv, d.chunk
+    if "_" not in name:
+        return None
+    if name.startswith("vlm_"):
+        T, H, I = B * P, d.hidden_v, d.inter_v
+    else:
+        T, H, I = B * S, d.hidden_a, d.inter_a
+    site = name.split("_", 1)[1]
+    if site == "qkv":
+        return 2.0 * T * H * (nq + 2 * nkv) * D, "flop"
+    if site == "o":
+        return 2.0 * T * nq * D * H, "flop"
+    if site == "gateup":
+        return 2.0 * T * H * 2 * I, "flop"
+    if site == "down":
+        return 2.0 * T * I * H, "flop"
+    if name == "vlm_attn":
+        return 4.0 * B * nq * P * P * D, "flop"
+    if name == "act_attn":
+        return float(B * nkv * (P + S) * D * 2 * 2), "byte"
+    return None
+
+
+def site_rooflines(d, B, P, bd, peaks):
+    """Per-site fraction of its roofline from the probed breakdown (tensor sites against the measured
+    sustained bf16 peak, the suffix attention against the measured copy bandwidth)."""
+    for name, rec in bd.items():
+        w = site_work(d, B, P, name)
+        if w is None or not rec["launches"] or rec["avg_us"] <= 0:
+            continue
+        amount, kind = w
+        sec = rec["avg_us"] * 1e-6
+        if kind == "flop":
+            ach = amount / sec / 1e12
+            rec.update({"achieved": round(ach, 1), "unit": "TFLOP/s",
+                        "frac": round(ach / peaks["bf16_tflops_sustained"], 4)})
+        else:
+            ach = amount / sec / 1e9
+            rec.update({"achieved": round(ach, 1), "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4)})
+    return bd
 
 
 # ------------------------------------------------------------------ rank plumbing
@@ -391,9 +436,10 @@ def run_native(args, rank, world, local_rank):
         finally:
             eng_tm.close()
     if not args.skip_breakdown:
-        result["breakdown_ms_per_step"] = breakdown(eng, wl_main)
+        result["breakdown_ms_per_step"] = site_rooflines(d, B, P, breakdown(eng, wl_main), peaks)
         if "batch1" in result:
-            result["batch1"]["breakdown_ms_per_step"] = breakdown(eng, I.WORKLOADS["e2e_b1"])
+            wl1 = I.WORKLOADS["e2e_b1"]
+            result["batch1"]["breakdown_ms_per_step"] = site_rooflines(d, 1, wl1.prefix, breakdown(eng, wl1), peaks)
     if rank == 0 and world == 1 and not args.skip_cpu:
         result["cpu_baseline"] = cpu_baseline(wl_main, budget_s=args.cpu_budget)
         if args.cpu_configs:

@@ -324,9 +324,13 @@ __global__ void __launch_bounds__(FaWarps<NP>::kThreads, NP == 1 ? 2 : 1)
       float mx = -__int_as_float(0x7f800000);
       if (good) {
         tmem_ld32(tl + s * 64 + half * 32, sv);
+        if (nvalid < 64) {   // keys past a ragged end score -inf: weight 0, no per-key predicate below
 #pragma unroll
-        for (int q = 0; q < 32; ++q)
-          if (half * 32 + q < nvalid) mx = fmaxf(mx, sv[q]);
+          for (int q = 0; q < 32; ++q)
+            if (half * 32 + q >= nvalid) sv[q] = -__int_as_float(0x7f800000);
+        }
+#pragma unroll
+        for (int q = 0; q < 32; ++q) mx = fmaxf(mx, sv[q]);
       }
       xm[((j & 1) * 2 + half) * 128 + r] = mx;
       named_bar_sync(1, kSM);
@@ -343,9 +347,8 @@ __global__ void __launch_bounds__(FaWarps<NP>::kThreads, NP == 1 ? 2 : 1)
         uint32_t pk[16];
 #pragma unroll
         for (int q = 0; q < 32; q += 2) {
-          const int kq = half * 32 + q;
-          const float p0 = kq < nvalid ? ex2_fast(fmaf(sv[q], a.scale_log2, -m_new)) : 0.f;
-          const float p1 = kq + 1 < nvalid ? ex2_fast(fmaf(sv[q + 1], a.scale_log2, -m_new)) : 0.f;
+          const float p0 = ex2_fast(fmaf(sv[q], a.scale_log2, -m_new));
+          const float p1 = ex2_fast(fmaf(sv[q + 1], a.scale_log2, -m_new));
           sum += p0 + p1;
           pk[q >> 1] = pack_bf16(p0, p1);
         }
@@ -485,14 +488,20 @@ __global__ void __launch_bounds__(FaWarps<NP>::kThreads, NP == 1 ? 2 : 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[s]);
-      // block max over the valid keys, eight independent chains
+      // keys past the end of a ragged last block score -inf (their weight 2^-inf is 0), so the max and
+      // exponent loops below carry no per-key predicate
       const float ninf = -__int_as_float(0x7f800000);
+      if (nvalid < 64) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          if (i >= nvalid) sv[i] = ninf;
+      }
+      // block max, eight independent chains
       float mx8[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) mx8[k] = ninf;
 #pragma unroll
-      for (int i = 0; i < 64; ++i)
-        if (i < nvalid) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
+      for (int i = 0; i < 64; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
       const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_blk = mx * a.scale_log2;
@@ -506,8 +515,8 @@ __global__ void __launch_bounds__(FaWarps<NP>::kThreads, NP == 1 ? 2 : 1)
       for (int k = 0; k < 8; ++k) sum8[k] = 0.f;
 #pragma unroll
       for (int i = 0; i < 64; i += 2) {
-        const float p0 = (i < nvalid) ? ex2_fast(fmaf(sv[i], a.scale_log2, -m_new)) : 0.f;
-        const float p1 = (i + 1 < nvalid) ? ex2_fast(fmaf(sv[i + 1], a.scale_log2, -m_new)) : 0.f;
+        const float p0 = ex2_fast(fmaf(sv[i], a.scale_log2, -m_new));
+        const float p1 = ex2_fast(fmaf(sv[i + 1], a.scale_log2, -m_new));
         sum8[(i >> 1) & 7] += p0 + p1;
         pk[i >> 1] = pack_bf16(p0, p1);
       }

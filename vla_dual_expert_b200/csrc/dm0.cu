@@ -95,6 +95,7 @@ struct dm0_ctx {
   bool use_persist = true;
   int persist_splits = 7;
   bool persist_fast_bar = false;   // DM0_PERSIST_FASTBAR=1: release-reduction grid barrier arrival
+  int raster_band_override = 0;     // DM0_RASTER_BAND=n: persistent-GEMM bands of n m-tiles
   int persist_resident = -1;   // -1: not checked yet
   // true when the previous operation this context queued on the stream was one of its own
   // kernels: only then may the next kernel overlap it (programmatic dependent launch).  The first
@@ -349,6 +350,15 @@ void probe_end(dm0_ctx* c, cudaStream_t s, int site, int e0) {
 }
 
 // ---------------------------------------------------------------- GEMM dispatch
+// Raster of the persistent GEMM: weights of up to 64 MB (every DM0-base projection, bf16 or E4M3)
+// stay in the 126 MB L2 for the whole launch under their evict-last policy, so the tiles run
+// n-fastest and each activation tile is read from DRAM once, by the CTAs of one wave; larger
+// weight matrices keep the default 64-m-tile bands.  DM0_RASTER_BAND=n forces bands of n m-tiles.
+int raster_band(const dm0_ctx* c, size_t weight_bytes) {
+  if (c->raster_band_override > 0) return c->raster_band_override;
+  return weight_bytes <= (size_t(64) << 20) ? 1 : 0;
+}
+
 dm0_status run_gemm(dm0_ctx* c, cudaStream_t s, const bf16* act, int tokens, int K, const bf16* W, int wrows,
                     GemmArgs g, int force_swap = -1, int force_splits = 0) {
   if (tokens <= 0) return DM0_OK;
@@ -401,6 +411,7 @@ dm0_status run_gemm(dm0_ctx* c, cudaStream_t s, const bf16* act, int tokens, int
   g.N = wrows;
   g.swap = 0;
   g.kb_per_split = KB;
+  g.band_m = raster_band(c, static_cast<size_t>(wrows) * K * 2);
   TRY(get_tmap(c, &ta, act, tokens, K, 128));
   TRY(get_tmap(c, &tb, W, wrows, K, BN));
   // persistent: at most one CTA per SM walking the tiles
@@ -439,6 +450,7 @@ dm0_status run_gemm_e4m3(dm0_ctx* c, cudaStream_t s, const uint8_t* act, const f
   g.N = wrows;
   g.swap = 0;
   g.kb_per_split = K / 128;
+  g.band_m = raster_band(c, static_cast<size_t>(wrows) * K);
   CUtensorMap ta, tb;
   TRY(get_tmap_u8(c, &ta, act, tokens, K, 128));
   TRY(get_tmap_u8(c, &tb, W, wrows, K, BN));
@@ -1215,6 +1227,7 @@ dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
   if (const char* e = std::getenv("DM0_NO_PERSIST")) c->use_persist = e[0] == '0';
   if (const char* e = std::getenv("DM0_PERSIST_SPLITS")) c->persist_splits = std::max(1, std::atoi(e));
   if (const char* e = std::getenv("DM0_PERSIST_FASTBAR")) c->persist_fast_bar = e[0] == '1';
+  if (const char* e = std::getenv("DM0_RASTER_BAND")) c->raster_band_override = std::max(0, std::atoi(e));
 
   // weights: one allocation, 256-byte aligned sub-buffers
   size_t total = 0;

@@ -48,6 +48,7 @@ struct GemmArgs {
   float* acc;
   int ld_acc;
   int* counters;      // one per 128-feature tile, zero between launches
+  int band_m;         // persistent GEMM: m-tiles per raster band (1: n fastest; <= 0: the default)
   // kModeResid
   float* h;           // [tokens][H] fp32 residual stream
   int H;
@@ -603,22 +604,27 @@ namespace dm0 {
 // ---------------------------------------------------------------- persistent normal-orientation GEMM
 //
 // One CTA per SM walks output tiles t = blockIdx.x, blockIdx.x + gridDim.x, ...
-// in a banded raster: bands of kBandM m-tiles, m fastest inside a band, so the
-// CTAs running together cover a few weight tiles and at most kBandM activation
-// tiles; both stay in L2 while the band is worked (activation tiles are read
-// from DRAM once, weights once per band).  The producer streams
+// in a banded raster: bands of band_m m-tiles, m fastest inside a band, so the
+// CTAs running together cover a few weight tiles and at most band_m activation
+// tiles (activation tiles are read from DRAM once if the band stays in L2,
+// weights once per band).  band_m = 1 is the n-fastest raster: the CTAs of a
+// wave share a few activation tiles and the whole weight matrix, which then
+// has to stay in L2 for the whole launch (the host picks it when the weights
+// are small next to L2; with tall bands the residual and output streams of the
+// epilogues evict the band's activations).  The producer streams
 // k-blocks of consecutive tiles through one ring without pausing between tiles,
 // and the accumulator is double-buffered in TMEM (2 x BN columns): while the
 // epilogue warps finish tile i from one buffer, the MMA warp already
 // accumulates tile i+1 into the other.
-constexpr int kBandM = 64;   // m-tiles per raster band (64 x 128 rows x K bf16 stays L2-resident)
+constexpr int kBandM = 64;   // default m-tiles per raster band (band_m <= 0)
 
 // output tile index t -> (m_tile, n_tile) in the banded raster
-__device__ __forceinline__ void band_tile(int t, int mt, int nt, int& m_tile, int& n_tile) {
-  const int band = t / (kBandM * nt);
-  const int m0 = band * kBandM;
-  const int bm = min(kBandM, mt - m0);   // m-tiles in this band
-  const int r = t - band * kBandM * nt;
+__device__ __forceinline__ void band_tile(int t, int mt, int nt, int band_m, int& m_tile, int& n_tile) {
+  const int bh = band_m > 0 ? band_m : kBandM;
+  const int band = t / (bh * nt);
+  const int m0 = band * bh;
+  const int bm = min(bh, mt - m0);   // m-tiles in this band
+  const int r = t - band * bh * nt;
   m_tile = m0 + r % bm;
   n_tile = r / bm;
 }
@@ -697,7 +703,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (a.w_stable && first < ntiles) {
         pre = KB < STAGES ? KB : STAGES;
         int m_first, n0;
-        band_tile(first, mt, a.N / BN, m_first, n0);
+        band_tile(first, mt, a.N / BN, a.band_m, m_first, n0);
         for (int k = 0; k < pre; ++k) {
           mbar_arrive_expect_tx(&full[k], L::kStage);
           tma_load_2d(smem + k * L::kStage + L::kA, &tmB, &full[k], k * kKB, n0 * BN, pol_w);
@@ -708,7 +714,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       (void)waited;
       for (int t = first; t < ntiles && !*abort_flag; t += gridDim.x) {
         int mtile, ntile;
-        band_tile(t, mt, a.N / BN, mtile, ntile);
+        band_tile(t, mt, a.N / BN, a.band_m, mtile, ntile);
         const int m0 = mtile * 128, n0 = ntile * BN;
         for (int k = 0; k < KB; ++k, ++it) {
           const int s = it % STAGES;
@@ -781,7 +787,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     auto prefetch_rows = [&](int t) {
       if (a.mode != kModeResid || t >= ntiles) return;
       int m_tile, n_tile;
-      band_tile(t, mt, a.N / BN, m_tile, n_tile);
+      band_tile(t, mt, a.N / BN, a.band_m, m_tile, n_tile);
       const int tok = m_tile * 128 + lane_base + lane;
       if (tok < a.M) prefetch_l2_bulk(a.h + static_cast<size_t>(tok) * a.H + n_tile * BN, BN * 4);
     };
@@ -797,7 +803,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       prefetch_rows(t + gridDim.x);
       int m_tile, n_tile;
-      band_tile(t, mt, a.N / BN, m_tile, n_tile);
+      band_tile(t, mt, a.N / BN, a.band_m, m_tile, n_tile);
       const uint32_t tl = tmem + (static_cast<uint32_t>(lane_base) << 16) + buf * BN;
       const int tok = m_tile * 128 + lane_base + lane;
       const bool valid = tok < a.M;
