@@ -769,6 +769,71 @@ def run_b1_trace(args):
     eng.close()
 
 
+GEMM_TRACE_SLOTS = 16
+GEMM_TRACE_MARKS = ("entry", "setup", "dep_wait", "first_stage", "first_issued", "first_acc", "first_done",
+                    "last_done", "last_load", "exit")
+
+
+def summarize_gemm_trace(arr):
+    """Per launch (rows of `arr`: [launch][CTA][16] %globaltimer marks of the persistent GEMM, CTA 0
+    holding the shape in slots 14-15): the shape, the CTAs that ran, the launch span (first entry to
+    last exit) and the median over CTAs of each mark after the launch's first entry, in us."""
+    import numpy as np
+    out = []
+    for row in arr:
+        m_n, k_bn = int(row[0, 14]), int(row[0, 15])
+        if m_n == 0:
+            continue
+        ran = row[:, 0] > 0
+        # CTAs of this launch: their entry is within 1 s of CTA 0's (other rows may be stale)
+        ran &= np.abs(row[:, 0].astype(np.float64) - float(row[0, 0])) < 1e9
+        r = row[ran].astype(np.float64)
+        t0 = r[:, 0].min()
+        last = np.maximum(r[:, 6], r[:, 7])   # one-tile CTAs leave "last_done" at 0
+        rec = {"M": m_n >> 32, "N": m_n & 0xFFFFFFFF, "K": k_bn >> 32, "BN": k_bn & 0xFFFFFFFF,
+               "ctas": int(ran.sum()), "span_us": round((r[:, 9].max() - t0) / 1e3, 2)}
+        for i, name in enumerate(GEMM_TRACE_MARKS):
+            v = last if name == "last_done" else r[:, i]
+            ok = v > 0
+            rec[name] = round(float(np.median(v[ok] - t0)) / 1e3, 2) if ok.any() else None
+        out.append(rec)
+    return out
+
+
+def run_gemm_trace(args):
+    """Profiling workload: the one-layer context of --one-layer (--batch / --prefix), with every
+    persistent GEMM launch stamping a per-CTA timeline (DM0_GEMM_TRACE=1 set here before the context
+    is created).  Two iterations of prefill + a 1-step denoise; prints summarize_gemm_trace of the
+    second iteration's launches."""
+    os.environ["DM0_GEMM_TRACE"] = "1"
+    import numpy as np
+    import torch
+
+    from synth import inputs as I
+    from vla_dual_expert_b200 import Engine
+    d = I.DM0_BASE.replace(layers=1)
+    B, P = args.batch or 16, args.prefix or 2048
+    os.environ["DM0_NO_GRAPH"] = "1"   # direct launches: one trace row per launch
+    eng = Engine(d, B, P)
+    eng.load_from(I.Weights(d, seed=0))
+    emb = torch.from_numpy(I.prefix_embeddings(d, B, P)).cuda().to(torch.bfloat16)
+    noise = torch.from_numpy(I.noise(d, B)).cuda()
+    for _ in range(2):
+        eng.prefill(emb)
+        eng.denoise(noise, 1)
+    eng.sync()
+    torch.cuda.synchronize()
+    nsm = torch.cuda.get_device_properties(0).multi_processor_count
+    rows = 64
+    ptr = eng.debug_view("gemm_trace")
+    view = type("Trace", (), {"__cuda_array_interface__": {"shape": (rows * nsm * GEMM_TRACE_SLOTS,),
+                                                            "typestr": "<u8", "data": (ptr, False), "version": 3}})()
+    arr = torch.as_tensor(view, device="cuda").cpu().numpy().reshape(rows, nsm, GEMM_TRACE_SLOTS)
+    recs = summarize_gemm_trace(arr)   # launch order
+    print(json.dumps({"gemm_trace": "ok", "batch": B, "prefix": P, "launches": recs}))
+    eng.close()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -787,6 +852,8 @@ def main():
     ap.add_argument("--b1-trace", action="store_true",
                     help="profiling workload: per-phase timeline of the single-launch Euler loop")
     ap.add_argument("--trace-layers", type=int, default=28)
+    ap.add_argument("--gemm-trace", action="store_true",
+                    help="profiling workload: per-CTA timeline of every persistent GEMM of one layer")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--cpu-configs", action="store_true",
                     help="also time the oracle in full on the single-observation configurations (~1-2 min)")
@@ -813,6 +880,9 @@ def main():
         return
     if args.b1_trace:
         run_b1_trace(args)
+        return
+    if args.gemm_trace:
+        run_gemm_trace(args)
         return
     run_native(args, rank, world, local_rank)
 

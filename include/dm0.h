@@ -294,6 +294,14 @@ dm0_status dm0_op_attention(dm0_ctx* ctx, const void* q, const void* ka, const v
  * operand, MMA warp issued its last MMA;
  * phase 0 is the input of step 0, then per step 5 phases per layer (QKV,
  * attention, O, gate/up, down) and the step boundary.
+ * "gemm_trace" (NULL unless DM0_GEMM_TRACE=1 was set at dm0_create): u64
+ * %globaltimer marks of the last 64 persistent-GEMM launches (round robin, in
+ * launch order), [launch][CTA (num_sms rows)][16] = entry, setup done, past the
+ * dependency wait, first k-block landed, first tile's MMAs issued, first
+ * accumulator complete, first tile's epilogue done, last tile's epilogue done
+ * (0 for one-tile CTAs), last TMA copy issued, exit; CTA 0's slots 14 and 15
+ * hold (M << 32 | N) and (K << 32 | tile width); rows of CTAs that did not
+ * run in a launch keep stale values.
  * "tm_mod", "tm_bqkv", "tm_bgu" (time_mod contexts, NULL before the first
  * dm0_denoise or dm0_prepare): the modulation tables of the last Euler loop of
  * K steps, f32 [K][(6*layers + 2)*hidden_a] (per layer [attention: 1 + scale |

@@ -163,6 +163,38 @@ def test_prefix_outputs_ignore_the_suffix(layer_engine):
     assert rel_err(got[0][3], got[1][3]) > 1e-2
 
 
+@pytest.mark.parametrize("knob,value", [("DM0_RASTER_BAND", "64"), ("DM0_NO_PDL", "1")])
+def test_gemm_schedule_knobs_do_not_change_results(layer_engine, monkeypatch, knob, value):
+    """The persistent GEMM's tile order (n-fastest raster or 64-m-tile bands) and programmatic
+    dependent launch change only when work runs, never its arithmetic: one merged layer's prefix
+    output and K/V (no order-dependent sums on that path) are bit for bit those of the default
+    schedule."""
+    d, w, eng = layer_engine
+    P, S = 816, d.chunk
+    hp = to_dev_f32(I.hidden_states(P, d.hidden_v, seed=60)[None])
+    hs = to_dev_f32(I.hidden_states(S, d.hidden_a, seed=61)[None])
+
+    def run(e):
+        outp = torch.empty((1, P, d.hidden_v), device="cuda", dtype=torch.float32)
+        outs = torch.empty((1, S, d.hidden_a), device="cuda", dtype=torch.float32)
+        k = torch.empty((1, d.n_kv, P, d.head_dim), device="cuda", dtype=torch.bfloat16)
+        v = torch.empty_like(k)
+        e.merged_layer(0, hp, hs, outp, outs, k, v)
+        e.sync()
+        assert e.device_error() == 0
+        return host(outp), host(k), host(v)
+
+    ref = run(eng)
+    monkeypatch.setenv(knob, value)   # read when a context is created
+    other = _engine(d, 2, 816, w)
+    try:
+        got = run(other)
+    finally:
+        other.close()
+    for g, r, what in zip(got, ref, ("prefix out", "prefix K", "prefix V")):
+        assert np.array_equal(g, r), what
+
+
 # ------------------------------------------------------------------ tiny model (2 layers, head_dim 32)
 
 @pytest.fixture(scope="module")

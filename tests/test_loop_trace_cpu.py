@@ -37,3 +37,32 @@ def test_summary_medians_and_phase_time():
     a = out["attention"]                           # only the two item CTAs, which run 2x slower
     assert (a["staged"], a["issued"], a["arrived"]) == (2.0, 6.0, 8.0)
     assert set(out["step"]) == {"phase"}
+
+
+def test_gemm_trace_summary():
+    """bench.summarize_gemm_trace on a synthetic two-launch trace: the shape words of CTA 0, the
+    CTAs that ran (stale rows and unused slots ignored), the span from the first entry to the last
+    exit, per-mark medians from the first entry, and the last tile's epilogue of one-tile CTAs taken
+    from their first tile."""
+    ctas, slots = 6, bench.GEMM_TRACE_SLOTS
+    arr = np.zeros((3, ctas, slots), dtype=np.uint64)
+    base = 5_000_000_000
+    for c in range(4):   # launch 0: 4 CTAs ran, each 1 us later than the previous
+        t = base + 1000 * c
+        arr[0, c, :10] = [t + 1000 * m for m in range(10)]
+        if c < 2:        # CTAs 0 and 1 had one tile: no "last_done" mark
+            arr[0, c, 7] = 0
+    arr[0, 4, :10] = 7   # a stale row from long before: not part of the launch
+    arr[0, 0, 14] = (816 << 32) | 4096
+    arr[0, 0, 15] = (2048 << 32) | 256
+    arr[1, 0, :10] = [base + 50_000_000 + 2000 * m for m in range(10)]   # launch 1: one CTA
+    arr[1, 0, 14] = (50 << 32) | 128
+    arr[1, 0, 15] = (64 << 32) | 64
+    out = bench.summarize_gemm_trace(arr)
+    assert len(out) == 2
+    a, b = out
+    assert (a["M"], a["N"], a["K"], a["BN"], a["ctas"]) == (816, 4096, 2048, 256, 4)
+    assert a["span_us"] == 12.0            # last exit (CTA 3: +3 + 9 us) after the first entry
+    assert a["setup"] == 2.5               # median over CTAs of (1 us + their 0..3 us delay)
+    assert a["last_done"] == 8.0           # one-tile CTAs count their first tile: 6, 7, 9, 10
+    assert (b["ctas"], b["span_us"], b["exit"]) == (1, 18.0, 18.0)

@@ -82,6 +82,7 @@ struct TmapKey {
 
 constexpr int kGemmStages = 4;
 constexpr int kPartSlots = 1024;   // split-KV partial-state slots (x 128 rows)
+constexpr int kGemmTraceLaunches = 64;   // DM0_GEMM_TRACE rows (persistent GEMM launches, round robin)
 
 }  // namespace
 
@@ -131,6 +132,8 @@ struct dm0_ctx {
   float* part_o = nullptr;
   float2* part_ml = nullptr;
   float2* rope = nullptr;
+  float2* rope_t = nullptr;   // the same table dimension-major: [head_dim / 2][max_pos]
+  int rope_max_pos = 0;
   int* d_err = nullptr;
   // dm0_infer_host staging
   bf16* stage_prefix = nullptr;
@@ -140,6 +143,8 @@ struct dm0_ctx {
   bf16* pkv_sfx = nullptr;      // [n_kv][2][64][128] suffix K/V tiles built by the helper CTAs
   dm0::PdLayer* players = nullptr;
   unsigned long long* ptrace = nullptr;   // DM0_PERSIST_TRACE=1: phase timestamps of the persistent loop
+  unsigned long long* gtrace = nullptr;   // DM0_GEMM_TRACE=1: [kGemmTraceLaunches][num_sms][16] GEMM marks
+  int gtrace_next = 0;                     // next launch slot (round robin)
   int ptrace_steps = 0;
   // FP8 E4M3 prefix MLP (dm0_set_prefix_fp8): per VLM layer the gate/up (interleaved as the bf16
   // copy) and down weights as codes with per-output-channel scales, and the per-token operands
@@ -354,6 +359,13 @@ void probe_end(dm0_ctx* c, cudaStream_t s, int site, int e0) {
 // stay in the 126 MB L2 for the whole launch under their evict-last policy, so the tiles run
 // n-fastest and each activation tile is read from DRAM once, by the CTAs of one wave; larger
 // weight matrices keep the default 64-m-tile bands.  DM0_RASTER_BAND=n forces bands of n m-tiles.
+// DM0_GEMM_TRACE=1: each persistent GEMM launch gets the next of kGemmTraceLaunches rows of marks
+unsigned long long* next_gemm_trace(dm0_ctx* c) {
+  if (!c->gtrace) return nullptr;
+  const int slot = c->gtrace_next++ % kGemmTraceLaunches;
+  return c->gtrace + static_cast<size_t>(slot) * c->num_sms * dm0::kGemmTraceSlots;
+}
+
 int raster_band(const dm0_ctx* c, size_t weight_bytes) {
   if (c->raster_band_override > 0) return c->raster_band_override;
   return weight_bytes <= (size_t(64) << 20) ? 1 : 0;
@@ -412,6 +424,7 @@ dm0_status run_gemm(dm0_ctx* c, cudaStream_t s, const bf16* act, int tokens, int
   g.swap = 0;
   g.kb_per_split = KB;
   g.band_m = raster_band(c, static_cast<size_t>(wrows) * K * 2);
+  g.trace = next_gemm_trace(c);
   TRY(get_tmap(c, &ta, act, tokens, K, 128));
   TRY(get_tmap(c, &tb, W, wrows, K, BN));
   // persistent: at most one CTA per SM walking the tiles
@@ -451,6 +464,7 @@ dm0_status run_gemm_e4m3(dm0_ctx* c, cudaStream_t s, const uint8_t* act, const f
   g.swap = 0;
   g.kb_per_split = K / 128;
   g.band_m = raster_band(c, static_cast<size_t>(wrows) * K);
+  g.trace = next_gemm_trace(c);
   CUtensorMap ta, tb;
   TRY(get_tmap_u8(c, &ta, act, tokens, K, 128));
   TRY(get_tmap_u8(c, &tb, W, wrows, K, BN));
@@ -584,6 +598,8 @@ GemmArgs base_args(dm0_ctx* c) {
   g.n_kv = cf.n_kv;
   g.head_dim = cf.head_dim;
   g.rope = c->rope;
+  g.rope_t = c->rope_t;
+  g.rope_ld = c->rope_max_pos;
   return g;
 }
 
@@ -1332,6 +1348,8 @@ dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
   A(dalloc(c, &c->part_ml, static_cast<size_t>(kPartSlots) * 128));
   const int max_pos = g.max_prefix + g.chunk;
   A(dalloc(c, &c->rope, static_cast<size_t>(max_pos) * D / 2));
+  A(dalloc(c, &c->rope_t, static_cast<size_t>(max_pos) * D / 2));
+  c->rope_max_pos = max_pos;
   A(dalloc(c, &c->d_err, 1));
   A(dalloc(c, &c->stage_prefix, Mp * g.hidden_v));
   A(dalloc(c, &c->pacc_qkv, static_cast<size_t>(64) * qkv_rows(g)));
@@ -1340,6 +1358,10 @@ dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
   A(dalloc(c, &c->psync, 2 + g.n_kv));
   A(dalloc(c, &c->pkv_sfx, static_cast<size_t>(g.n_kv) * 2 * 64 * 128));
   A(dalloc(c, &c->players, g.layers));
+  if (const char* e = std::getenv("DM0_GEMM_TRACE")) {
+    if (e[0] == '1')
+      A(dalloc(c, &c->gtrace, static_cast<size_t>(kGemmTraceLaunches) * c->num_sms * dm0::kGemmTraceSlots));
+  }
   if (const char* e = std::getenv("DM0_PERSIST_TRACE")) {
     if (e[0] == '1') {
       c->ptrace_steps = 16;
@@ -1360,7 +1382,7 @@ dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
       cudaMemset(c->acount, 0, c->acount_n * 4) != cudaSuccess || cudaMemset(c->d_err, 0, 4) != cudaSuccess)
     return bail(DM0_ECUDA);
   const int nrope = max_pos * static_cast<int>(D / 2);
-  dm0::rope_table_kernel<<<(nrope + 255) / 256, 256>>>(c->rope, max_pos, static_cast<int>(D / 2),
+  dm0::rope_table_kernel<<<(nrope + 255) / 256, 256>>>(c->rope, c->rope_t, max_pos, static_cast<int>(D / 2),
                                                        std::log(static_cast<double>(g.rope_theta)));
   if (cudaGetLastError() != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) return bail(DM0_ECUDA);
   if (cudaStreamCreateWithFlags(&c->cap_stream, cudaStreamNonBlocking) != cudaSuccess) return bail(DM0_ECUDA);
@@ -1666,7 +1688,7 @@ dm0_status dm0_debug_view(dm0_ctx* c, const char* name, void** ptr) {
       {"h_v", c->h_v},     {"xn_v", c->xn_v},   {"q_v", c->q_v},     {"o_v", c->o_v},     {"act_v", c->act_v},
       {"ssq_v", c->ssq_v}, {"h_a", c->h_a},     {"xn_a", c->xn_a},   {"q_a", c->q_a},     {"o_a", c->o_a},
       {"act_a", c->act_a}, {"ssq_a", c->ssq_a}, {"x", c->x},         {"k_s", c->k_s},     {"v_s", c->v_s},
-      {"loop_trace", c->ptrace}, {"tm_mod", c->tm_mod}, {"tm_bqkv", c->tm_bqkv}, {"tm_bgu", c->tm_bgu}};
+      {"loop_trace", c->ptrace}, {"gemm_trace", c->gtrace}, {"tm_mod", c->tm_mod}, {"tm_bqkv", c->tm_bqkv}, {"tm_bgu", c->tm_bgu}};
   auto it = bufs.find(name);
   if (it == bufs.end()) return fail(c, DM0_EINVAL, std::string("unknown buffer ") + name);
   *ptr = it->second;

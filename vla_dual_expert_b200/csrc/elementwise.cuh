@@ -337,13 +337,18 @@ __global__ void __launch_bounds__(256) quant_rows_e4m3_kernel(const T* x, int ro
   }
 }
 
-__global__ void rope_table_kernel(float2* tab, int max_pos, int half, double log_theta) {
+// (cos, sin) of every (position, frequency): position-major in `tab` [max_pos][half] and the same
+// values dimension-major in `tab_t` [half][max_pos], where the 32 consecutive tokens of a warp read
+// one frequency as two 128-byte lines
+__global__ void rope_table_kernel(float2* tab, float2* tab_t, int max_pos, int half, double log_theta) {
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= max_pos * half) return;
   const int pos = idx / half, i = idx - (idx / half) * half;
   const double inv_freq = exp(-(2.0 * i / (2.0 * half)) * log_theta);
   const double ang = static_cast<double>(pos) * inv_freq;
-  tab[idx] = make_float2(static_cast<float>(cos(ang)), static_cast<float>(sin(ang)));
+  const float2 cs = make_float2(static_cast<float>(cos(ang)), static_cast<float>(sin(ang)));
+  tab[idx] = cs;
+  tab_t[static_cast<size_t>(i) * max_pos + pos] = cs;
 }
 
 }  // namespace dm0

@@ -49,6 +49,8 @@ struct GemmArgs {
   int ld_acc;
   int* counters;      // one per 128-feature tile, zero between launches
   int band_m;         // persistent GEMM: m-tiles per raster band (1: n fastest; <= 0: the default)
+  // persistent GEMM timeline (null: off): [CTA][kGemmTraceSlots] %globaltimer marks, see kGemmTrace*
+  unsigned long long* trace;
   // kModeResid
   float* h;           // [tokens][H] fp32 residual stream
   int H;
@@ -67,6 +69,8 @@ struct GemmArgs {
   int pos_offset;     // RoPE position of each sample's first token
   int kv_seq;         // per-(sample, kv head) length of the K/V destination
   const float2* rope; // [position][head_dim/2] (cos, sin)
+  const float2* rope_t;   // the same values [head_dim/2][rope_ld]: a warp's consecutive tokens read
+  int rope_ld;            // one frequency as contiguous memory
   // kModeSwiGLU
   __nv_bfloat16* act; // [tokens][inter]
   int inter;
@@ -84,6 +88,25 @@ struct GemmArgs {
 };
 
 constexpr int kGemmThreads = 192;
+
+// Timeline marks of the persistent GEMM, one row of kGemmTraceSlots u64 per CTA; CTA 0 also stores
+// the launch shape in the last two slots ((M << 32) | N and (K << 32) | BN).
+enum GemmTraceMark : int {
+  kGtEntry = 0,        // thread 0 at kernel entry
+  kGtSetup = 1,        // after barrier init, TMEM allocation and the setup barrier
+  kGtDepWait = 2,      // producer past the dependency wait (griddepcontrol.wait)
+  kGtFirstStage = 3,   // MMA warp: first k-block of the first tile landed
+  kGtFirstIssued = 4,  // MMA warp: last MMA of the first tile issued
+  kGtFirstAcc = 5,     // epilogue warp 2: accumulator of the first tile complete
+  kGtFirstDone = 6,    // epilogue warp 2: epilogue of the first tile done
+  kGtLastDone = 7,     // epilogue warp 2: epilogue of the CTA's last tile done
+  kGtLastLoad = 8,     // producer: last TMA copy issued
+  kGtExit = 9,         // thread 0 after the final barrier
+};
+constexpr int kGemmTraceSlots = 16;
+__device__ __forceinline__ void gemm_mark(const unsigned long long* tr, int mark) {
+  if (tr) const_cast<unsigned long long*>(tr)[blockIdx.x * kGemmTraceSlots + mark] = globaltimer();
+}
 
 template <int BN, int STAGES>
 struct GemmSmem {
@@ -326,7 +349,9 @@ __device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool va
   const int b = tok / a.seq_len, p = tok - b * a.seq_len;
   const int pos = a.pos_offset + p;
   const int half = D >> 1;
-  const float2* cs_row = a.rope + static_cast<size_t>(pos) * half;
+  // (cos, sin) of frequency d at this token's position: column `pos` of the dimension-major table,
+  // so the warp's 32 consecutive tokens read one frequency as contiguous memory
+  const float2* cs_col = a.rope_t + pos;
   auto dst_of = [&](int col) -> __nv_bfloat16* {
     if (col < qdim) return a.q_out + static_cast<size_t>(tok) * qdim + col;
     const int sec = col < qdim + kvdim ? 1 : 2;
@@ -370,7 +395,7 @@ __device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool va
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const float x0 = v[j] * rn * gain[j], x1 = v[j + 16] * rn * gain[j + 16];
-        const float2 cs = cs_row[j];
+        const float2 cs = cs_col[static_cast<size_t>(j) * a.rope_ld];
         o[j] = x0 * cs.x - x1 * cs.y;
         o[j + 16] = x1 * cs.x + x0 * cs.y;
       }
@@ -386,7 +411,7 @@ __device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool va
         for (int j = 0; j < 32; ++j) {
           const int d = 32 * c + j;
           const float x0 = lo[j] * rn * gain[d], x1 = hi[j] * rn * gain[d + half];
-          const float2 cs = cs_row[d];
+          const float2 cs = cs_col[static_cast<size_t>(d) * a.rope_ld];
           lo[j] = x0 * cs.x - x1 * cs.y;
           hi[j] = x1 * cs.x + x0 * cs.y;
         }
@@ -667,6 +692,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int ntiles = mt * (a.N / BN);
 
   if (threadIdx.x == 0) {
+    if (a.trace)   // this CTA's row: clear the marks a previous launch may have left
+      for (int i = 0; i < kGemmTraceSlots - 2; ++i) a.trace[blockIdx.x * kGemmTraceSlots + i] = 0ull;
+    gemm_mark(a.trace, kGtEntry);
+    if (a.trace && blockIdx.x == 0) {
+      a.trace[kGemmTraceSlots - 2] = (static_cast<unsigned long long>(a.M) << 32) | static_cast<unsigned>(a.N);
+      a.trace[kGemmTraceSlots - 1] = (static_cast<unsigned long long>(a.K) << 32) | static_cast<unsigned>(BN);
+    }
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -688,6 +720,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   pdl_launch_dependents();
+  if (threadIdx.x == 0) gemm_mark(a.trace, kGtSetup);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -712,6 +745,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       pdl_wait();
       waited = true;
       (void)waited;
+      gemm_mark(a.trace, kGtDepWait);
       for (int t = first; t < ntiles && !*abort_flag; t += gridDim.x) {
         int mtile, ntile;
         band_tile(t, mt, a.N / BN, a.band_m, mtile, ntile);
@@ -732,6 +766,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tma_load_2d(smem + s * L::kStage + L::kA, &tmB, &full[s], k * kKB, n0, pol_w);
         }
       }
+      gemm_mark(a.trace, kGtLastLoad);
       for (int i = it - STAGES; i < it; ++i) {   // copies in flight land before the CTA exits
         if (i < 0) continue;
         if (!mbar_wait(&full[i % STAGES], (i / STAGES) & 1, nullptr, kDrainTimeoutNs)) raise_error(a.err, kErrDrain);
@@ -755,6 +790,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             ok = false;
             break;
           }
+          if (it == 0) gemm_mark(a.trace, kGtFirstStage);
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + s * L::kStage);
           const uint32_t b_addr = a_addr + L::kA;
@@ -769,6 +805,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           umma_commit(&empty[s]);
         }
+        if (local == 0) gemm_mark(a.trace, kGtFirstIssued);
         if (ok) umma_commit(&tfull[buf]);
       }
       if (!ok) {
@@ -800,6 +837,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         raise_error(a.err, kErrTimeoutEpilogue);
         break;
       }
+      if (local == 0 && threadIdx.x == 64) gemm_mark(a.trace, kGtFirstAcc);
       tc_fence_after();
       prefetch_rows(t + gridDim.x);
       int m_tile, n_tile;
@@ -848,10 +886,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);
+      if (threadIdx.x == 64) gemm_mark(a.trace, local == 0 ? kGtFirstDone : kGtLastDone);
     }
   }
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) gemm_mark(a.trace, kGtExit);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
