@@ -84,8 +84,12 @@ def test_gemm_swap_split_k(layer_engine, M, N, K, splits):
 
 # ------------------------------------------------------------------ merged GQA attention
 
+# the last three launch more than half an SM count of CTAs with suffix keys, which runs the one-CTA-per-SM
+# suffix instance (4 K/V stages, two softmax threads per row): an even and an odd number of 64-key
+# blocks, and a key split
 @pytest.mark.parametrize("B,Tq,Ta,Tb,splits", [(1, 50, 130, 50, 1), (2, 50, 816, 50, 5), (1, 200, 200, 0, 1),
-                                               (1, 17, 1, 0, 1), (2, 50, 64, 50, 3), (1, 816, 816, 0, 1)])
+                                               (1, 17, 1, 0, 1), (2, 50, 64, 50, 3), (1, 816, 816, 0, 1),
+                                               (2, 800, 816, 50, 1), (2, 400, 640, 37, 1), (2, 800, 816, 50, 2)])
 def test_attention(layer_engine, B, Tq, Ta, Tb, splits):
     d, _, eng = layer_engine
     rng = np.random.default_rng(B * 1000 + Tq + Ta + Tb + splits)

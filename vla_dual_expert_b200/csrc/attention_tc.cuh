@@ -329,8 +329,10 @@ __global__ void __launch_bounds__(FaWarps<NP>::kThreads, NP == 1 ? 2 : 1)
           for (int q = 0; q < 32; ++q)
             if (half * 32 + q >= nvalid) sv[q] = -__int_as_float(0x7f800000);
         }
+        float mx4[4] = {mx, mx, mx, mx};
 #pragma unroll
-        for (int q = 0; q < 32; ++q) mx = fmaxf(mx, sv[q]);
+        for (int q = 0; q < 32; q += 2) mx4[(q >> 1) & 3] = max3f(mx4[(q >> 1) & 3], sv[q], sv[q + 1]);
+        mx = max3f(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
       }
       xm[((j & 1) * 2 + half) * 128 + r] = mx;
       named_bar_sync(1, kSM);
@@ -345,13 +347,17 @@ __global__ void __launch_bounds__(FaWarps<NP>::kThreads, NP == 1 ? 2 : 1)
       float sum = 0.f;
       if (good) {
         uint32_t pk[16];
+        float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nm2 = make_float2(-m_new, -m_new);
 #pragma unroll
         for (int q = 0; q < 32; q += 2) {
-          const float p0 = ex2_fast(fmaf(sv[q], a.scale_log2, -m_new));
-          const float p1 = ex2_fast(fmaf(sv[q + 1], a.scale_log2, -m_new));
-          sum += p0 + p1;
+          const float2 x = ffma2(make_float2(sv[q], sv[q + 1]), sc2, nm2);
+          const float p0 = ex2_fast(x.x);
+          const float p1 = ex2_fast(x.y);
+          sum2[(q >> 1) & 1] = fadd2(sum2[(q >> 1) & 1], make_float2(p0, p1));
           pk[q >> 1] = pack_bf16(p0, p1);
         }
+        sum = (sum2[0].x + sum2[0].y) + (sum2[1].x + sum2[1].y);
         uint8_t* ps = smem + FS::kOffP + (j % NP) * FS::kP;
 #pragma unroll
         for (int c = 0; c < 4; ++c)
@@ -496,31 +502,35 @@ __global__ void __launch_bounds__(FaWarps<NP>::kThreads, NP == 1 ? 2 : 1)
         for (int i = 0; i < 64; ++i)
           if (i >= nvalid) sv[i] = ninf;
       }
-      // block max, eight independent chains
+      // block max, eight independent chains of three-operand maxima
       float mx8[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) mx8[k] = ninf;
 #pragma unroll
-      for (int i = 0; i < 64; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
+      for (int i = 0; i < 64; i += 2) mx8[(i >> 1) & 7] = max3f(mx8[(i >> 1) & 7], sv[i], sv[i + 1]);
       const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_blk = mx * a.scale_log2;
       const bool move = m_blk > m_ref + 8.f;        // also true on the first block
       const float m_new = move ? m_blk : m_ref;
       const float alpha = move ? exp2f(m_ref - m_new) : 1.f;   // 0 on the first block
-      // P = 2^(s*scale - m), row sum in eight partial sums, packed to bf16
+      // P = 2^(s*scale - m), packed to bf16; the exponent arguments and the row sum (four paired
+      // partial sums) in paired fp32 arithmetic
       uint32_t pk[32];
-      float sum8[8];
+      float2 sum2[4];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) sum8[k] = 0.f;
+      for (int k = 0; k < 4; ++k) sum2[k] = make_float2(0.f, 0.f);
+      const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nm2 = make_float2(-m_new, -m_new);
 #pragma unroll
       for (int i = 0; i < 64; i += 2) {
-        const float p0 = ex2_fast(fmaf(sv[i], a.scale_log2, -m_new));
-        const float p1 = ex2_fast(fmaf(sv[i + 1], a.scale_log2, -m_new));
-        sum8[(i >> 1) & 7] += p0 + p1;
+        const float2 x = ffma2(make_float2(sv[i], sv[i + 1]), sc2, nm2);
+        const float p0 = ex2_fast(x.x);
+        const float p1 = ex2_fast(x.y);
+        sum2[(i >> 1) & 3] = fadd2(sum2[(i >> 1) & 3], make_float2(p0, p1));
         pk[i >> 1] = pack_bf16(p0, p1);
       }
-      const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+      const float sum = ((sum2[0].x + sum2[0].y) + (sum2[1].x + sum2[1].y)) +
+                        ((sum2[2].x + sum2[2].y) + (sum2[3].x + sum2[3].y));
       l_run = l_run * alpha + sum;
       m_ref = m_new;
       // P buffer j % NP is free once PV_{j-NP} completed; O may only be rescaled after PV_{j-1}
