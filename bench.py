@@ -128,6 +128,15 @@ def prefill_gateup_flops(d, B, P):
     return 2.0 * B * P * d.hidden_v * 2 * d.inter_v
 
 
+def train_flops(d, B, P):
+    """Algorithmic FLOPs of one training step of the action expert: 6 T per parameter (forward, dX,
+    dW) for every projection, and 12 S (P + S) D per query head for the merged attention (forward
+    Q K^T and P V, adjoint dP, dQ, dK, dV)."""
+    T, S = B * d.chunk, d.chunk
+    attn = 12.0 * B * d.n_q * S * (P + S) * d.head_dim
+    return d.layers * (6.0 * T * layer_params(d, 1) + attn)
+
+
 def denoise_bytes_per_step(d, B, P):
     """Algorithmic HBM bytes of one Euler step: action-expert bf16 weights + prefix KV cache read once."""
     w = d.layers * layer_params(d, 1) * 2
@@ -415,11 +424,16 @@ def run_native(args, rank, world, local_rank):
         torch.cuda.synchronize()
         barrier()
         tms = rank_max(t0.elapsed_time(t1) / args.steps)
+        tflop = train_flops(d, B, P) / 1e12
         result["train"] = {"workload": f"flow-matching training step of the 28-layer action expert, B={B} samples of "
                                        f"50x32 over a P={P} prefix cache (knowledge insulation)",
                            "value": round(world * B * 1000.0 / tms, 3), "unit": "samples/s",
                            "ms_per_step": round(tms, 3), "loss": float(loss.item()),
-                           "gpu_launches": (eng.launch_count() - n0) // max(args.steps, 1)}
+                           "gpu_launches": (eng.launch_count() - n0) // max(args.steps, 1),
+                           "roofline": {"bound": "tensor", "algorithmic_tflop_per_step": round(tflop, 3),
+                                        "achieved": round(tflop / (tms * 1e-3), 1), "peak": tc_peak,
+                                        "unit": "TFLOP/s", "frac": round(tflop / (tms * 1e-3) / tc_peak, 4),
+                                        "peak_src": f"{peaks['src']} bf16_tflops_sustained"}}
     if args.time_mod:
         # the same step for the time-modulated action expert (opt-in; its own weights and context)
         from vla_dual_expert_b200 import Engine as _Engine

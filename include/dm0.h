@@ -160,8 +160,9 @@ dm0_status dm0_kv_commit(dm0_ctx* ctx, int B, int P);
  * One observation (B = 1) with head_dim 128 runs the whole loop as ONE
  * persistent kernel (one CTA per SM, grid barriers between the phases of a
  * layer; DM0_PERSIST_SPLITS at dm0_create sets its attention key splits per
- * KV head, default 7; DM0_PERSIST_FASTBAR=1 makes each barrier arrival one
- * release reduction with no full fences around it); otherwise, when the kernel cannot be resident on every
+ * KV head, default 7; each barrier arrival is one release reduction and the
+ * wait an acquire spin, with no full fences around them, unless
+ * DM0_PERSIST_FASTBAR=0 was set, which adds them); otherwise, when the kernel cannot be resident on every
  * SM, and when the environment variable DM0_NO_PERSIST=1 was set at
  * dm0_create, the loop is a chain of per-layer kernels captured once per
  * (B, P, steps) as a CUDA graph and replayed (launched directly when

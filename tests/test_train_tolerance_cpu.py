@@ -1,7 +1,8 @@
 """Where the GPU training step's tolerances come from: the step's decomposition (dm0_train_step: bf16
 GEMM operands for the normalised activations, the attention output, the SwiGLU output, every upstream
-gradient dY, dgate / dup and the dq / dk / dv operands
-fp32 elsewhere) emulated in numpy, against
+gradient dY, dgate / dup and the dq / dk / dv operands; for head_dim 128 also the tensor-core
+attention's operands: q and the suffix K / V, the softmax weights before P V, dO, and the
+probabilities and dS of the adjoint; fp32 elsewhere) emulated in numpy, against
 the fp64 oracle (oracle/dm0_train.py).  Its worst per-tensor gradient error must sit at least a
 factor 4 under the GPU tests' bar of 3e-2 RMS, and the loss under 1e-4 relative (bar 1e-3), so the
 bars leave room for fp32 summation order and the GPU's transcendental functions.
@@ -35,17 +36,19 @@ def layer_fwd(w, h, kc, vc, d):
     kn, sk = T._rms_fwd(k3, w["k_norm"], d.rms_eps)
     cos, sin = T._rope_tables(np.arange(P, P + S), D, d.rope_theta)
     qr, kr = T._rope_fwd(qn, cos, sin), T._rope_fwd(kn, cos, sin)
-    K = np.concatenate([kc, kr], axis=1)
-    V = np.concatenate([vc, v3], axis=1)
+    tc = D == 128   # the tcgen05 flash attention: bf16 q, suffix K / V and softmax weights
+    qa = bf(qr) if tc else qr
+    K = np.concatenate([kc, bf(kr) if tc else kr], axis=1)
+    V = np.concatenate([vc, bf(v3) if tc else v3], axis=1)
     group, scale = Hq // Hkv, 1 / np.sqrt(D)
     p = np.empty((Hq, S, P + S))
     o = np.empty((Hq, S, D))
     for hh in range(Hq):
         j = hh // group
-        sc = qr[hh] @ K[j].T * scale
+        sc = qa[hh] @ K[j].T * scale
         e = np.exp(sc - sc.max(-1, keepdims=True))
         p[hh] = e / e.sum(-1, keepdims=True)
-        o[hh] = p[hh] @ V[j]
+        o[hh] = ((bf(e) @ V[j]) / e.sum(-1, keepdims=True)) if tc else p[hh] @ V[j]
     of = o.transpose(1, 0, 2).reshape(S, Hq * D)
     ofb = bf(of)
     h1 = h + ofb @ W["Wo"].T
@@ -55,7 +58,7 @@ def layer_fwd(w, h, kc, vc, d):
     sg = gate / (1 + np.exp(-gate))
     act = bf(sg * up)
     h2 = h1 + act @ W["Wd"].T
-    return h2, dict(W=W, r1=r1, s1=s1, sq=sq, sk=sk, cos=cos, sin=sin, qr=qr, K=K, V=V, p=p, of=of, ofb=ofb,
+    return h2, dict(W=W, r1=r1, s1=s1, sq=sq, sk=sk, cos=cos, sin=sin, qr=qa, K=K, V=V, p=p, of=of, ofb=ofb, tc=tc,
                     r2=r2, s2=s2, gate=gate, up=up, act=act, P=P, S=S, h=h, h1=h1)
 
 
@@ -81,12 +84,20 @@ def layer_bwd(w, c, dh2, d):
     group, scale = Hq // Hkv, 1 / np.sqrt(D)
     dK, dV = np.zeros_like(c["K"]), np.zeros_like(c["V"])
     dqr = np.empty_like(c["qr"])
+    ofb3 = c["ofb"].reshape(S, Hq, D).transpose(1, 0, 2)
     for hh in range(Hq):
         j = hh // group
         p = c["p"][hh]
-        dp = do[hh] @ c["V"][j].T
-        dV[j] += p.T @ do[hh]
-        ds = p * (dp - np.sum(dp * p, -1, keepdims=True)) * scale
+        if c["tc"]:   # the tcgen05 adjoint: bf16 dO, P and dS; delta from fp32 dO and the bf16 output
+            dob = bf(do[hh])
+            dp = dob @ c["V"][j].T
+            delta = np.sum(do[hh] * ofb3[hh], -1, keepdims=True)
+            ds = bf(p * (dp - delta) * scale)
+            dV[j] += bf(p).T @ dob
+        else:
+            dp = do[hh] @ c["V"][j].T
+            dV[j] += p.T @ do[hh]
+            ds = p * (dp - np.sum(dp * p, -1, keepdims=True)) * scale
         dqr[hh] = ds @ c["K"][j]
         dK[j] += ds.T @ c["qr"][hh]
     dq3, g["q_norm"] = T._rms_bwd(T._rope_bwd(dqr, c["cos"], c["sin"]), w["q_norm"], c["sq"])

@@ -38,6 +38,9 @@ struct AttnArgs {
   float2* part_ml;          // [slots][128]
   int* counters;            // [groups * row tiles]
   int* err;
+  // tcgen05 kernel, unsplit launches only (null: off): per query row, at the row's place in o
+  // ([B][seq_q][n_q]), the base-2 log-sum-exp m + log2(l) of its scaled scores (p = 2^(s * scale_log2 - lse))
+  float* lse;
 };
 
 constexpr int kAttnThreads = 256;

@@ -402,6 +402,7 @@ __global__ void __launch_bounds__(FaWarps<NP>::kThreads, NP == 1 ? 2 : 1)
         if (gridDim.z == 1) {
           const float inv = 1.f / l_tot;
           __nv_bfloat16* dst = a.o + ((static_cast<size_t>(b) * a.seq_q + pos) * a.n_q + head) * D;
+          if (a.lse && half == 0 && valid) a.lse[(static_cast<size_t>(b) * a.seq_q + pos) * a.n_q + head] = m_ref + log2f(l_tot);
 #pragma unroll 1
           for (int c = half * 2; c < half * 2 + 2; ++c) {
             float o[32];
@@ -581,6 +582,7 @@ __global__ void __launch_bounds__(FaWarps<NP>::kThreads, NP == 1 ? 2 : 1)
         if (gridDim.z == 1) {
           const float inv = 1.f / l_run;
           __nv_bfloat16* dst = a.o + ((static_cast<size_t>(b) * a.seq_q + pos) * a.n_q + head) * D;
+          if (a.lse && valid) a.lse[(static_cast<size_t>(b) * a.seq_q + pos) * a.n_q + head] = m_ref + log2f(l_run);
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {
             float o[32];

@@ -37,6 +37,7 @@
 #include "dm0.h"
 #include "attention.cuh"
 #include "attention_tc.cuh"
+#include "attention_bwd.cuh"
 #include "denoise_persistent.cuh"
 #include "elementwise.cuh"
 #include "gemm.cuh"
@@ -95,7 +96,7 @@ struct dm0_ctx {
   // per-layer kernels instead); DM0_PERSIST_SPLITS overrides its attention key splits per KV head
   bool use_persist = true;
   int persist_splits = 7;
-  bool persist_fast_bar = false;   // DM0_PERSIST_FASTBAR=1: release-reduction grid barrier arrival
+  bool persist_fast_bar = true;    // release-reduction grid barrier arrival (DM0_PERSIST_FASTBAR=0: full fences)
   int raster_band_override = 0;     // DM0_RASTER_BAND=n: persistent-GEMM bands of n m-tiles
   int persist_resident = -1;   // -1: not checked yet
   // true when the previous operation this context queued on the stream was one of its own
@@ -169,9 +170,10 @@ struct dm0_ctx {
   bool train_wt_ok = false;
   struct TrainBuf {
     float *hs, *xt, *u, *rho1, *rho2, *rhof, *rho_q, *rho_k;
-    float *raw, *qr, *kr, *vs, *prob, *of, *tmp, *h1, *gu, *rf, *dv, *drf;
+    float *raw, *qr, *kr, *vs, *prob, *of, *lse, *tmp, *h1, *gu, *rf, *dv, *drf;
     float *dh, *dh_alt, *dact, *dr, *dof, *dqr, *dK, *dV, *dgu_w;
     bf16 *r1, *r2, *of_bf, *act, *dgu, *dqkv, *dy_bf, *tA, *tB;
+    bf16 *q_bf, *k_bf, *v_bf;   // tensor-core attention operands: q [T][Hq D], suffix K / V [B][Hkv][S][D]
     int* count;
   } tb{};
   bool train_alloc = false;
@@ -494,7 +496,8 @@ dm0_status quant_rows(dm0_ctx* c, cudaStream_t s, const T* x, int rows, int cols
 
 // ---------------------------------------------------------------- attention dispatch
 dm0_status run_attn(dm0_ctx* c, cudaStream_t s, const bf16* q, int seq_q, const bf16* ka, const bf16* va, int len_a,
-                    const bf16* kb, const bf16* vb, int len_b, bf16* o, int B, int splits_req, int a_stable) {
+                    const bf16* kb, const bf16* vb, int len_b, bf16* o, int B, int splits_req, int a_stable,
+                    float* lse = nullptr) {
   const dm0_config& g = c->cfg;
   const int G = g.n_q / g.n_kv;
   const int tiles = (G * seq_q + 127) / 128;
@@ -534,6 +537,7 @@ dm0_status run_attn(dm0_ctx* c, cudaStream_t s, const bf16* q, int seq_q, const 
   a.part_ml = c->part_ml;
   a.counters = c->acount;
   a.err = c->d_err;
+  a.lse = lse;
   if (g.head_dim == 128) {
     // tcgen05 flash attention, K/V tiles of both segments by TMA; keys split in 64-key blocks
     const int fblk = (len_a + 63) / 64 + (len_b + 63) / 64;
@@ -1242,7 +1246,7 @@ dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
   if (const char* e = std::getenv("DM0_NO_GRAPH")) c->use_graph = e[0] == '0';
   if (const char* e = std::getenv("DM0_NO_PERSIST")) c->use_persist = e[0] == '0';
   if (const char* e = std::getenv("DM0_PERSIST_SPLITS")) c->persist_splits = std::max(1, std::atoi(e));
-  if (const char* e = std::getenv("DM0_PERSIST_FASTBAR")) c->persist_fast_bar = e[0] == '1';
+  if (const char* e = std::getenv("DM0_PERSIST_FASTBAR")) c->persist_fast_bar = e[0] != '0';
   if (const char* e = std::getenv("DM0_RASTER_BAND")) c->raster_band_override = std::max(0, std::atoi(e));
 
   // weights: one allocation, 256-byte aligned sub-buffers
@@ -1406,7 +1410,8 @@ dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
             smem_attr(dm0::fa_tc_kernel<dm0::kFaDeepStages, 2>, dm0::FaSmemT<dm0::kFaDeepStages, 2>::kBytes) &&
             smem_attr(dm0::denoise_persistent_kernel<false>, dm0::PdSmem::kBytes) &&
             smem_attr(dm0::denoise_persistent_kernel<true>, dm0::PdSmem::kBytes) &&
-            smem_attr(dm0::train_attn_fwd_kernel, 100 * 1024) && smem_attr(dm0::train_attn_bwd_kernel, 200 * 1024);
+            smem_attr(dm0::train_attn_fwd_kernel, 100 * 1024) && smem_attr(dm0::train_attn_bwd_kernel, 200 * 1024) &&
+            smem_attr(dm0::fa_bwd_kernel, dm0::FaBwdSmem::kBytes);
   if (!ok) return bail(DM0_ECUDA);
   *out = c;
   return DM0_OK;

@@ -303,7 +303,8 @@ __global__ void __launch_bounds__(256) train_deinterleave_kernel(const float* dg
   }
 }
 
-// Merged attention of the training step, one CTA per (sample, query head), all S query rows: scores
+// Merged attention of the training step on CUDA cores, for head_dim 32 and 64 (head_dim 128 runs the
+// tcgen05 flash attention and its adjoint kernel): one CTA per (sample, query head), all S query rows: scores
 // against the sample's [prefix cache (bf16); suffix keys (fp32)] keys, softmax (fp32), probabilities
 // kept in prob [B][Hq][S][P + S], o = prob V in fp32 and bf16.  Shared memory: q [S][D], a 32-key
 // tile [32][D + 1], a probability tile [S][32].
@@ -500,6 +501,32 @@ __global__ void __launch_bounds__(256) train_attn_bwd_kernel(const TrainAttn a) 
     if (idx >= S * D) break;
     const int s = idx / D, d = idx - (idx / D) * D;
     a.dqr[(static_cast<size_t>(b * S + s) * a.Hq + h) * D + d] = dq[i];
+  }
+}
+
+// Operands of the training step's tensor-core attention from the fp32 layer intermediates: q (after
+// QK-norm and RoPE) in bf16 in its own layout [T][Hq D], and the suffix keys and values in bf16 as the
+// second key segment [B][Hkv][S][D] (the prefix cache is the first).  One thread per element.
+__global__ void __launch_bounds__(256) train_attn_prep_kernel(const float* qr, const float* kr, const float* vs, int B,
+                                                              int S, int Hq, int Hkv, int D, __nv_bfloat16* q_bf,
+                                                              __nv_bfloat16* k_bf, __nv_bfloat16* v_bf) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const size_t nq = static_cast<size_t>(B) * S * Hq * D, nk = static_cast<size_t>(B) * S * Hkv * D;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < nq + nk; i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    if (i < nq) {
+      q_bf[i] = __float2bfloat16_rn(qr[i]);
+      continue;
+    }
+    const size_t k = i - nq;   // source [b S + s][g D + d] -> [b][g][s][d]
+    const int d = static_cast<int>(k % D);
+    const size_t rest = k / D;
+    const int g = static_cast<int>(rest % Hkv);
+    const size_t t = rest / Hkv;
+    const int b = static_cast<int>(t / S), s = static_cast<int>(t % S);
+    const size_t dst = ((static_cast<size_t>(b) * Hkv + g) * S + s) * D + d;
+    k_bf[dst] = __float2bfloat16_rn(kr[k]);
+    v_bf[dst] = __float2bfloat16_rn(vs[k]);
   }
 }
 

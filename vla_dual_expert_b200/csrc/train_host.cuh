@@ -41,8 +41,15 @@ dm0_status train_buffers(dm0_ctx* c) {
   TRY(dalloc(c, &b.qr, T * HqD));
   TRY(dalloc(c, &b.kr, T * HkvD));
   TRY(dalloc(c, &b.vs, T * HkvD));
-  TRY(dalloc(c, &b.prob, static_cast<size_t>(g.max_batch) * g.n_q * g.chunk * N));
-  TRY(dalloc(c, &b.of, T * HqD));
+  if (D == 128) {   // tcgen05 attention: bf16 operands and the forward's row log-sum-exp
+    TRY(dalloc(c, &b.q_bf, T * HqD));
+    TRY(dalloc(c, &b.k_bf, T * HkvD));
+    TRY(dalloc(c, &b.v_bf, T * HkvD));
+    TRY(dalloc(c, &b.lse, T * g.n_q));
+  } else {          // CUDA-core attention: the probabilities are kept for the adjoint
+    TRY(dalloc(c, &b.prob, static_cast<size_t>(g.max_batch) * g.n_q * g.chunk * N));
+    TRY(dalloc(c, &b.of, T * HqD));
+  }
   TRY(dalloc(c, &b.tmp, T * H));
   TRY(dalloc(c, &b.h1, T * H));
   TRY(dalloc(c, &b.gu, T * 2 * I));
@@ -127,6 +134,40 @@ dm0::TrainAttn train_attn_args(dm0_ctx* c, int l) {
   return at;
 }
 
+// Adjoint of the tensor-core attention of action layer l (head_dim 128): dq into b.dqr, dK / dV of every
+// key of [prefix cache; suffix] added into b.dK / b.dV, from the recomputed forward's bf16 q, suffix
+// K / V, output and row log-sum-exp, and the fp32 gradient of the output in b.dof.
+dm0_status run_attn_bwd(dm0_ctx* c, cudaStream_t s, int l) {
+  const dm0_config& g = c->cfg;
+  auto& b = c->tb;
+  const int B = c->kv_B, P = c->kv_P, S = g.chunk, D = g.head_dim;
+  const int G = g.n_q / g.n_kv, groups = B * g.n_kv, tiles = (G * S + 127) / 128;
+  const size_t lstride = static_cast<size_t>(B) * g.n_kv * P * D;
+  dm0::AttnBwdArgs a{};
+  a.q = b.q_bf;
+  a.o = b.of_bf;
+  a.dout = b.dof;
+  a.lse = b.lse;
+  a.seq_q = S;
+  a.len_a = P;
+  a.len_b = S;
+  a.n_q = g.n_q;
+  a.n_kv = g.n_kv;
+  a.scale = 1.0f / std::sqrt(static_cast<float>(D));
+  a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+  a.dq = b.dqr;
+  a.dk = b.dK;
+  a.dv = b.dV;
+  a.err = c->d_err;
+  CUtensorMap tk, tv, tkb, tvb;
+  TRY(get_tmap(c, &tk, c->kplane + l * lstride, static_cast<uint64_t>(groups) * P, 128, dm0::FaSmem::kKeys));
+  TRY(get_tmap(c, &tv, c->vplane + l * lstride, static_cast<uint64_t>(groups) * P, 128, dm0::FaSmem::kKeys));
+  TRY(get_tmap(c, &tkb, b.k_bf, static_cast<uint64_t>(groups) * S, 128, dm0::FaSmem::kKeys));
+  TRY(get_tmap(c, &tvb, b.v_bf, static_cast<uint64_t>(groups) * S, 128, dm0::FaSmem::kKeys));
+  return launch(c, s, dm0::fa_bwd_kernel, dim3(tiles, groups), dim3(dm0::kFaBwdThreads), dm0::FaBwdSmem::kBytes, tk,
+                tv, tkb, tvb, a);
+}
+
 // Forward of action layer l from hin over the cached prefix K/V, keeping every intermediate the
 // backward needs; hout (if not null) receives the layer's output.
 dm0_status train_layer_fwd(dm0_ctx* c, cudaStream_t s, int l, const float* hin, float* hout) {
@@ -143,9 +184,19 @@ dm0_status train_layer_fwd(dm0_ctx* c, cudaStream_t s, int l, const float* hin, 
              static_cast<const float*>(w.q_norm), static_cast<const float*>(w.k_norm),
              static_cast<const float2*>(c->rope), T, S, P, g.n_q, g.n_kv, D, g.rms_eps, b.qr, b.kr, b.vs, b.rho_q,
              b.rho_k));
-  dm0::TrainAttn at = train_attn_args(c, l);
-  const size_t fsm = sizeof(float) * (static_cast<size_t>(S) * D + 32 * (D + 1) + S * 32);
-  TRY(launch(c, s, dm0::train_attn_fwd_kernel, dim3(B * g.n_q), dim3(256), fsm, at));
+  if (D == 128) {   // bf16 operands, then the tcgen05 flash attention over [prefix cache; suffix], lse kept
+    const size_t n = static_cast<size_t>(T) * (HqD + g.n_kv * D);
+    TRY(launch(c, s, dm0::train_attn_prep_kernel, dim3(grid_for(n)), dim3(256), 0, static_cast<const float*>(b.qr),
+               static_cast<const float*>(b.kr), static_cast<const float*>(b.vs), B, S, g.n_q, g.n_kv, D, b.q_bf,
+               b.k_bf, b.v_bf));
+    const size_t lstride = static_cast<size_t>(B) * g.n_kv * P * D;
+    TRY(run_attn(c, s, b.q_bf, S, c->kplane + l * lstride, c->vplane + l * lstride, P, b.k_bf, b.v_bf, S, b.of_bf, B,
+                 1, 0, b.lse));
+  } else {
+    dm0::TrainAttn at = train_attn_args(c, l);
+    const size_t fsm = sizeof(float) * (static_cast<size_t>(S) * D + 32 * (D + 1) + S * 32);
+    TRY(launch(c, s, dm0::train_attn_fwd_kernel, dim3(B * g.n_q), dim3(256), fsm, at));
+  }
   TRY(gemm_f32(c, s, b.of_bf, T, HqD, w.wo, H, b.tmp));
   const size_t nh = static_cast<size_t>(T) * H;
   TRY(launch(c, s, dm0::train_add_kernel, dim3(grid_for(nh)), dim3(256), 0, hin, static_cast<const float*>(b.tmp), nh,
@@ -261,9 +312,13 @@ dm0_status enqueue_train(dm0_ctx* c, cudaStream_t s, const float* a, const float
     CK(cudaMemsetAsync(b.dV, 0, sizeof(float) * B * g.n_kv * N * D, s));
     CK(cudaMemsetAsync(g_qn, 0, sizeof(float) * 2 * D, s));   // q_norm, k_norm (adjacent), accumulated
     c->pdl_ok = false;
-    dm0::TrainAttn at = train_attn_args(c, l);
-    const size_t bsm = sizeof(float) * (2 * static_cast<size_t>(S) * D + 2 * 32 * (D + 1) + 2 * S * 32 + S);
-    TRY(launch(c, s, dm0::train_attn_bwd_kernel, dim3(B * g.n_q), dim3(256), bsm, at));
+    if (D == 128) {
+      TRY(run_attn_bwd(c, s, l));
+    } else {
+      dm0::TrainAttn at = train_attn_args(c, l);
+      const size_t bsm = sizeof(float) * (2 * static_cast<size_t>(S) * D + 2 * 32 * (D + 1) + 2 * S * 32 + S);
+      TRY(launch(c, s, dm0::train_attn_bwd_kernel, dim3(B * g.n_q), dim3(256), bsm, at));
+    }
     const int qk_warps = T * (g.n_q + 2 * g.n_kv);
     TRY(launch(c, s, dm0::train_qk_bwd_kernel, dim3((qk_warps + 7) / 8), dim3(256), 0, static_cast<const float*>(b.raw),
                static_cast<const float*>(w.q_norm), static_cast<const float*>(w.k_norm),
