@@ -434,12 +434,18 @@ dm0_status run_gemm(dm0_ctx* c, cudaStream_t s, const bf16* act, int tokens, int
   const dim3 grid(std::min(ntiles, c->num_sms));
   // as many stages as fit in ~192 KB: more bytes in flight per SM for the narrower tiles
   if (BN == 256)
-    return launch(c, s, dm0::gemm_tc_persistent<256, 4>, grid, dim3(dm0::kGemmThreads),
-                  dm0::PGemmSmem<256, 4>::kBytes, ta, tb, g);
+    return g.mode == dm0::kModeQKV
+               ? launch(c, s, dm0::gemm_tc_persistent<256, 4, false, 4>, grid, dim3(dm0::PGemmWarps<4>::kThreads),
+                        dm0::PGemmSmem<256, 4, 4>::kBytes, ta, tb, g)
+               : launch(c, s, dm0::gemm_tc_persistent<256, 4>, grid, dim3(dm0::PGemmWarps<8>::kThreads),
+                        dm0::PGemmSmem<256, 4>::kBytes, ta, tb, g);
   if (BN == 128)
-    return launch(c, s, dm0::gemm_tc_persistent<128, 6>, grid, dim3(dm0::kGemmThreads),
-                  dm0::PGemmSmem<128, 6>::kBytes, ta, tb, g);
-  return launch(c, s, dm0::gemm_tc_persistent<64, 8>, grid, dim3(dm0::kGemmThreads), dm0::PGemmSmem<64, 8>::kBytes,
+    return g.mode == dm0::kModeQKV
+               ? launch(c, s, dm0::gemm_tc_persistent<128, 6, false, 4>, grid, dim3(dm0::PGemmWarps<4>::kThreads),
+                        dm0::PGemmSmem<128, 6, 4>::kBytes, ta, tb, g)
+               : launch(c, s, dm0::gemm_tc_persistent<128, 6>, grid, dim3(dm0::PGemmWarps<8>::kThreads),
+                        dm0::PGemmSmem<128, 6>::kBytes, ta, tb, g);
+  return launch(c, s, dm0::gemm_tc_persistent<64, 8>, grid, dim3(dm0::PGemmWarps<8>::kThreads), dm0::PGemmSmem<64, 8>::kBytes,
                 ta, tb, g);
 }
 
@@ -473,12 +479,12 @@ dm0_status run_gemm_e4m3(dm0_ctx* c, cudaStream_t s, const uint8_t* act, const f
   const int ntiles = mt * (wrows / BN);
   const dim3 grid(std::min(ntiles, c->num_sms));
   if (BN == 256)
-    return launch(c, s, dm0::gemm_tc_persistent<256, 4, true>, grid, dim3(dm0::kGemmThreads),
+    return launch(c, s, dm0::gemm_tc_persistent<256, 4, true>, grid, dim3(dm0::PGemmWarps<8>::kThreads),
                   dm0::PGemmSmem<256, 4>::kBytes, ta, tb, g);
   if (BN == 128)
-    return launch(c, s, dm0::gemm_tc_persistent<128, 6, true>, grid, dim3(dm0::kGemmThreads),
+    return launch(c, s, dm0::gemm_tc_persistent<128, 6, true>, grid, dim3(dm0::PGemmWarps<8>::kThreads),
                   dm0::PGemmSmem<128, 6>::kBytes, ta, tb, g);
-  return launch(c, s, dm0::gemm_tc_persistent<64, 8, true>, grid, dim3(dm0::kGemmThreads),
+  return launch(c, s, dm0::gemm_tc_persistent<64, 8, true>, grid, dim3(dm0::PGemmWarps<8>::kThreads),
                 dm0::PGemmSmem<64, 8>::kBytes, ta, tb, g);
 }
 
@@ -1400,6 +1406,8 @@ dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
             smem_attr(dm0::gemm_tc_persistent<64, 8>, dm0::PGemmSmem<64, 8>::kBytes) &&
             smem_attr(dm0::gemm_tc_persistent<128, 6>, dm0::PGemmSmem<128, 6>::kBytes) &&
             smem_attr(dm0::gemm_tc_persistent<256, 4>, dm0::PGemmSmem<256, 4>::kBytes) &&
+            smem_attr(dm0::gemm_tc_persistent<256, 4, false, 4>, dm0::PGemmSmem<256, 4, 4>::kBytes) &&
+            smem_attr(dm0::gemm_tc_persistent<128, 6, false, 4>, dm0::PGemmSmem<128, 6, 4>::kBytes) &&
             smem_attr(dm0::gemm_tc_persistent<64, 8, true>, dm0::PGemmSmem<64, 8>::kBytes) &&
             smem_attr(dm0::gemm_tc_persistent<128, 6, true>, dm0::PGemmSmem<128, 6>::kBytes) &&
             smem_attr(dm0::gemm_tc_persistent<256, 4, true>, dm0::PGemmSmem<256, 4>::kBytes) &&

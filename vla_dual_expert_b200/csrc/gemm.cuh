@@ -88,6 +88,12 @@ struct GemmArgs {
 };
 
 constexpr int kGemmThreads = 192;
+// persistent GEMM: producer warp, MMA warp and EPI epilogue warps (4: one per TMEM lane quarter, up to
+// 255 registers a thread, for the register-hungry QKV epilogue; 8: two per quarter, 168 registers)
+template <int EPI>
+struct PGemmWarps {
+  static constexpr int kThreads = 64 + 32 * EPI;
+};
 
 // Timeline marks of the persistent GEMM, one row of kGemmTraceSlots u64 per CTA; CTA 0 also stores
 // the launch shape in the last two slots ((M << 32) | N and (K << 32) | BN).
@@ -168,19 +174,21 @@ __device__ __forceinline__ void st_bf16x32(__nv_bfloat16* dst, const float (&v)[
 // touches 32 rows per instruction.  The next chunk of h is requested before the current one is
 // used.  Same results as row_epilogue's residual mode.
 struct ResidScratch {
-  static constexpr int kLd = 36;    // fp32 words per scratch row: 16-byte aligned, rows 4 banks apart
-  static constexpr int kLdX = 20;   // 32-bit words per bf16 row (32 values + pad)
-  static constexpr uint32_t kBytes = 32 * kLd * 4 + 32 * kLdX * 4;
+  // 32 rows x 32 fp32, 128 bytes a row, the 16-byte pieces of row r swizzled by r mod 8 so that both a
+  // row-per-lane pass and a 4-rows-per-instruction pass hit every bank once per 128 bytes; the bf16
+  // norm operand reuses it once h has left
+  static constexpr uint32_t kBytes = 4096;
 };
+__device__ __forceinline__ uint32_t resid_swz(int row, int piece) {   // byte offset of 16-byte piece `piece`
+  return static_cast<uint32_t>(row * 128 + ((piece ^ (row & 7)) << 4));
+}
 
 template <class Load>
 __device__ __forceinline__ void resid_epilogue_warp(const GemmArgs& a, int row0, int col0, int nchunks,
-                                                    float* scr, Load&& load) {
-  constexpr int kLd = ResidScratch::kLd, kLdX = ResidScratch::kLdX;
+                                                    uint8_t* scr, Load&& load) {
   const int lane = threadIdx.x & 31;
   const int tok = row0 + lane;
   const bool valid = tok < a.M;
-  uint32_t* xs = reinterpret_cast<uint32_t*>(scr + 32 * kLd);
   const int qr = lane >> 3, qc = lane & 7;   // h piece of this lane: row 4 i + qr, float4 qc
   float4 hn[8];
   auto fetch = [&](int c) {
@@ -199,13 +207,13 @@ __device__ __forceinline__ void resid_epilogue_warp(const GemmArgs& a, int row0,
     float v[32];
     load(c, v);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) *reinterpret_cast<float4*>(scr + (4 * i + qr) * kLd + 4 * qc) = hn[i];
+    for (int i = 0; i < 8; ++i) *reinterpret_cast<float4*>(scr + resid_swz(4 * i + qr, qc)) = hn[i];
     if (c + 1 < nchunks) fetch(c + 1);
     __syncwarp();
-    float* mine = scr + lane * kLd;
 #pragma unroll
     for (int j4 = 0; j4 < 8; ++j4) {
-      const float4 hv = *reinterpret_cast<const float4*>(mine + 4 * j4);
+      float4* slot = reinterpret_cast<float4*>(scr + resid_swz(lane, j4));
+      const float4 hv = *slot;
       if (a.col_gate) {
         const float4 gt = __ldg(reinterpret_cast<const float4*>(a.col_gate + cc) + j4);
         v[4 * j4] *= gt.x;
@@ -217,20 +225,7 @@ __device__ __forceinline__ void resid_epilogue_warp(const GemmArgs& a, int row0,
       v[4 * j4 + 1] += hv.y;
       v[4 * j4 + 2] += hv.z;
       v[4 * j4 + 3] += hv.w;
-      *reinterpret_cast<float4*>(mine + 4 * j4) = make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
-    }
-    if (a.xn) {
-#pragma unroll
-      for (int j8 = 0; j8 < 4; ++j8) {
-        const float4 g0 = __ldg(reinterpret_cast<const float4*>(a.gain_next + cc) + 2 * j8);
-        const float4 g1 = __ldg(reinterpret_cast<const float4*>(a.gain_next + cc) + 2 * j8 + 1);
-        const float* w = v + 8 * j8;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) grp += w[j] * w[j];
-        *reinterpret_cast<uint4*>(xs + lane * kLdX + 4 * j8) =
-            make_uint4(bf2(g0.x * w[0], g0.y * w[1]), bf2(g0.z * w[2], g0.w * w[3]), bf2(g1.x * w[4], g1.y * w[5]),
-                       bf2(g1.z * w[6], g1.w * w[7]));
-      }
+      *slot = make_float4(v[4 * j4], v[4 * j4 + 1], v[4 * j4 + 2], v[4 * j4 + 3]);
     }
     __syncwarp();
 #pragma unroll
@@ -238,15 +233,28 @@ __device__ __forceinline__ void resid_epilogue_warp(const GemmArgs& a, int row0,
       const int r = 4 * i + qr;
       if (row0 + r < a.M)
         reinterpret_cast<float4*>(a.h + static_cast<size_t>(row0 + r) * a.H + cc)[qc] =
-            *reinterpret_cast<const float4*>(scr + r * kLd + 4 * qc);
+            *reinterpret_cast<const float4*>(scr + resid_swz(r, qc));
     }
     if (a.xn) {
+      __syncwarp();   // h has been read out of the scratch
+#pragma unroll
+      for (int j8 = 0; j8 < 4; ++j8) {
+        const float4 g0 = __ldg(reinterpret_cast<const float4*>(a.gain_next + cc) + 2 * j8);
+        const float4 g1 = __ldg(reinterpret_cast<const float4*>(a.gain_next + cc) + 2 * j8 + 1);
+        const float* w = v + 8 * j8;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) grp += w[j] * w[j];
+        *reinterpret_cast<uint4*>(scr + resid_swz(lane, j8)) =
+            make_uint4(bf2(g0.x * w[0], g0.y * w[1]), bf2(g0.z * w[2], g0.w * w[3]), bf2(g1.x * w[4], g1.y * w[5]),
+                       bf2(g1.z * w[6], g1.w * w[7]));
+      }
+      __syncwarp();
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int r = 8 * i + (lane >> 2), q = lane & 3;
         if (row0 + r < a.M)
           reinterpret_cast<uint4*>(a.xn + static_cast<size_t>(row0 + r) * a.H + cc)[q] =
-              *reinterpret_cast<const uint4*>(xs + r * kLdX + 4 * q);
+              *reinterpret_cast<const uint4*>(scr + resid_swz(r, q));
       }
     }
     if ((c & 1) && a.ssq_out) {   // the group's partial goes to its own slot
@@ -654,7 +662,7 @@ __device__ __forceinline__ void band_tile(int t, int mt, int nt, int band_m, int
   n_tile = r / bm;
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int EPI = 8>
 struct PGemmSmem {
   static constexpr uint32_t kA = 128 * 128;
   static constexpr uint32_t kB = BN * 128;
@@ -662,7 +670,7 @@ struct PGemmSmem {
   static constexpr uint32_t kPipe = STAGES * kStage;
   static constexpr uint32_t kOffScr = kPipe + 256;            // after the barriers
   static constexpr uint32_t kScrWarp = ResidScratch::kBytes;  // per epilogue warp
-  static constexpr uint32_t kBytes = kOffScr + 4 * kScrWarp + 1024;
+  static constexpr uint32_t kBytes = kOffScr + EPI * kScrWarp + 1024;
   static constexpr uint32_t kTmemCols = 2 * BN;
   static_assert(kBytes <= 232448, "shared memory per CTA");
 };
@@ -670,11 +678,11 @@ struct PGemmSmem {
 // kF8: both operands FP8 E4M3 (tensor maps of bytes), a k-block is 128 values instead of 64 (the
 // same 128-byte rows, so the ring, the swizzle and the descriptors are unchanged), and the epilogue
 // applies the per-token and per-output-channel scales.
-template <int BN, int STAGES, bool kF8 = false>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+template <int BN, int STAGES, bool kF8 = false, int EPI = 8>
+__global__ void __launch_bounds__(PGemmWarps<EPI>::kThreads, 1)
     gemm_tc_persistent(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const GemmArgs a) {
-  using L = PGemmSmem<BN, STAGES>;
+  using L = PGemmSmem<BN, STAGES, EPI>;
   constexpr int kKB = kF8 ? 128 : 64;   // operand values per 128-byte k-block row
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -705,7 +713,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 4);
+      mbar_init(&tempty[i], EPI);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -816,19 +824,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!mbar_wait(drain, 0, nullptr, kWaitTimeoutNs + kDrainTimeoutNs)) raise_error(a.err, kErrDrain);
     }
   } else {
+    // epilogue warps 2..9: lane quarter (warp mod 4) and column half hf.  A 256-wide tile's two
+    // 128-column groups go one to each half; a 128-wide tile of the column-independent modes
+    // (residual, store) splits into two 64-column halves, the QKV and SwiGLU groups stay whole (half 0);
+    // a 64-wide tile is half 0's
     const int lane_base = (warp & 3) * 32;
+    const int hf = (warp - 2) >> 2;
     pdl_wait();
-    // residual epilogue: each thread reads its token's BN fp32 values of h, one DRAM round trip per
-    // 32-column chunk; the rows of the CTA's next tile are requested into L2 one tile ahead, so
-    // those loads hit L2 while the accumulator of the current tile drains
+    // residual epilogue: the rows of the CTA's next tile are requested into L2 one tile ahead, so the
+    // h loads of that tile hit L2 while the accumulator of the current tile drains
     auto prefetch_rows = [&](int t) {
-      if (a.mode != kModeResid || t >= ntiles) return;
+      if (a.mode != kModeResid || t >= ntiles || hf != 0) return;
       int m_tile, n_tile;
       band_tile(t, mt, a.N / BN, a.band_m, m_tile, n_tile);
       const int tok = m_tile * 128 + lane_base + lane;
       if (tok < a.M) prefetch_l2_bulk(a.h + static_cast<size_t>(tok) * a.H + n_tile * BN, BN * 4);
     };
     prefetch_rows(blockIdx.x);
+    const bool col_indep = a.mode == kModeResid || a.mode == kModeStoreF32;
     int local = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++local) {
       const int buf = local & 1;
@@ -861,26 +874,42 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       };
-      if (a.mode == kModeResid) {
-        float* scr = reinterpret_cast<float*>(smem + L::kOffScr + (warp - 2) * L::kScrWarp);
-        const int row0 = m_tile * 128 + lane_base;
+      // this warp's columns of the tile: [c0, c0 + 32 nch) relative to the tile
+      int c0 = 0, nch = 0;
+      if (EPI == 4) {   // one warp per lane quarter walks the whole tile, 128-column group by group
         for (int g = 0; g < (BN >= 128 ? BN / 128 : 1); ++g) {
           const uint32_t tg = tl + g * 128;
           const int col0 = n_tile * BN + g * 128;
-          resid_epilogue_warp(a, row0, col0, BN >= 128 ? 4 : BN / 32, scr,
-                              [&](int c, float (&v)[32]) { scaled(tg + c * 32, col0 + 32 * c, v); });
+          const int ng = BN >= 128 ? 4 : BN / 32;
+          if (a.mode == kModeResid) {
+            uint8_t* scr = smem + L::kOffScr + (warp - 2) * L::kScrWarp;
+            resid_epilogue_warp(a, m_tile * 128 + lane_base, col0, ng, scr,
+                                [&](int c, float (&v)[32]) { scaled(tg + c * 32, col0 + 32 * c, v); });
+          } else {
+            row_epilogue<false>(a, tok, valid, col0,
+                                [&](int c, float (&v)[32]) { scaled(tg + c * 32, col0 + 32 * c, v); }, ng);
+          }
         }
-      } else if (BN >= 128) {
-        for (int g = 0; g < BN / 128; ++g) {
-          const uint32_t tg = tl + g * 128;
-          const int col0 = n_tile * BN + g * 128;
-          row_epilogue<false>(a, tok, valid, col0,
-                              [&](int c, float (&v)[32]) { scaled(tg + c * 32, col0 + 32 * c, v); });
-        }
+      } else if (BN == 256) {
+        c0 = 128 * hf;
+        nch = 4;
+      } else if (BN == 128) {
+        c0 = col_indep ? 64 * hf : 0;
+        nch = col_indep ? 2 : (hf == 0 ? 4 : 0);
       } else {
-        const int col0 = n_tile * BN;
-        row_epilogue<false>(a, tok, valid, col0,
-                            [&](int c, float (&v)[32]) { scaled(tl + c * 32, col0 + 32 * c, v); }, BN / 32);
+        nch = hf == 0 ? BN / 32 : 0;
+      }
+      if (nch > 0) {
+        const uint32_t tg = tl + c0;
+        const int col0 = n_tile * BN + c0;
+        if (a.mode == kModeResid) {
+          uint8_t* scr = smem + L::kOffScr + (warp - 2) * L::kScrWarp;
+          resid_epilogue_warp(a, m_tile * 128 + lane_base, col0, nch, scr,
+                              [&](int c, float (&v)[32]) { scaled(tg + c * 32, col0 + 32 * c, v); });
+        } else {
+          row_epilogue<false>(a, tok, valid, col0,
+                              [&](int c, float (&v)[32]) { scaled(tg + c * 32, col0 + 32 * c, v); }, nch);
+        }
       }
       // the accumulator buffer is free for tile local + 2
       tc_fence_before();
