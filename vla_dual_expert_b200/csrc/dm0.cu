@@ -96,6 +96,7 @@ struct dm0_ctx {
   // per-layer kernels instead); DM0_PERSIST_SPLITS overrides its attention key splits per KV head
   bool use_persist = true;
   int persist_splits = 7;
+  bool qkv_epi4 = true;              // DM0_QKV_EPI=8: the QKV epilogue on eight warps (measured equal)
   bool persist_fast_bar = true;    // release-reduction grid barrier arrival (DM0_PERSIST_FASTBAR=0: full fences)
   int raster_band_override = 0;     // DM0_RASTER_BAND=n: persistent-GEMM bands of n m-tiles
   int persist_resident = -1;   // -1: not checked yet
@@ -434,13 +435,13 @@ dm0_status run_gemm(dm0_ctx* c, cudaStream_t s, const bf16* act, int tokens, int
   const dim3 grid(std::min(ntiles, c->num_sms));
   // as many stages as fit in ~192 KB: more bytes in flight per SM for the narrower tiles
   if (BN == 256)
-    return g.mode == dm0::kModeQKV
+    return g.mode == dm0::kModeQKV && c->qkv_epi4
                ? launch(c, s, dm0::gemm_tc_persistent<256, 4, false, 4>, grid, dim3(dm0::PGemmWarps<4>::kThreads),
                         dm0::PGemmSmem<256, 4, 4>::kBytes, ta, tb, g)
                : launch(c, s, dm0::gemm_tc_persistent<256, 4>, grid, dim3(dm0::PGemmWarps<8>::kThreads),
                         dm0::PGemmSmem<256, 4>::kBytes, ta, tb, g);
   if (BN == 128)
-    return g.mode == dm0::kModeQKV
+    return g.mode == dm0::kModeQKV && c->qkv_epi4
                ? launch(c, s, dm0::gemm_tc_persistent<128, 6, false, 4>, grid, dim3(dm0::PGemmWarps<4>::kThreads),
                         dm0::PGemmSmem<128, 6, 4>::kBytes, ta, tb, g)
                : launch(c, s, dm0::gemm_tc_persistent<128, 6>, grid, dim3(dm0::PGemmWarps<8>::kThreads),
@@ -1253,6 +1254,7 @@ dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
   if (const char* e = std::getenv("DM0_NO_PERSIST")) c->use_persist = e[0] == '0';
   if (const char* e = std::getenv("DM0_PERSIST_SPLITS")) c->persist_splits = std::max(1, std::atoi(e));
   if (const char* e = std::getenv("DM0_PERSIST_FASTBAR")) c->persist_fast_bar = e[0] != '0';
+  if (const char* e = std::getenv("DM0_QKV_EPI")) c->qkv_epi4 = std::atoi(e) != 8;
   if (const char* e = std::getenv("DM0_RASTER_BAND")) c->raster_band_override = std::max(0, std::atoi(e));
 
   // weights: one allocation, 256-byte aligned sub-buffers

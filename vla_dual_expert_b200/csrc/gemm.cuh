@@ -416,12 +416,17 @@ __device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool va
         ld(h0 + c, lo);
         ld(h0 + c + cph / 2, hi);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int d = 32 * c + j;
-          const float x0 = lo[j] * rn * gain[d], x1 = hi[j] * rn * gain[d + half];
-          const float2 cs = cs_col[static_cast<size_t>(d) * a.rope_ld];
-          lo[j] = x0 * cs.x - x1 * cs.y;
-          hi[j] = x1 * cs.x + x0 * cs.y;
+        for (int jh = 0; jh < 2; ++jh) {   // (cos, sin) of 16 dimensions requested together, then used
+          float2 cs[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) cs[j] = cs_col[static_cast<size_t>(32 * c + 16 * jh + j) * a.rope_ld];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int jj = 16 * jh + j, d = 32 * c + jj;
+            const float x0 = lo[jj] * rn * gain[d], x1 = hi[jj] * rn * gain[d + half];
+            lo[jj] = x0 * cs[j].x - x1 * cs[j].y;
+            hi[jj] = x1 * cs[j].x + x0 * cs[j].y;
+          }
         }
         if (valid) {
           st_bf16x32(dst_of(colh + 32 * c), lo);
