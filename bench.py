@@ -359,13 +359,19 @@ def run_native(args, rank, world, local_rank):
     }
     if args.workload == "e2e_b16" and not args.skip_batch1:
         wl1 = I.WORKLOADS["e2e_b1"]
-        b1 = measure(wl1, max(args.steps, 5), args.warmup, probe=None)
+        # at ~18 ms per chunk, 50 chunks give the 200 ms clock sampler a few samples in the timed region
+        b1 = measure(wl1, max(args.steps, 50), args.warmup, probe=None)
         den_gbs = denoise_bytes_per_step(d, 1, wl1.prefix) * EULER_STEPS / (b1["denoise_ms_p50"] * 1e-3) / 1e9
+        b1_mhz = (b1["clocks"] or {}).get("sm_mhz")
         result["batch1"] = {
             "workload": "e2e_b1: prefill B=1 x P=816 + 10-step denoise",
             "value": round(job_chunks_per_s(world, 1, b1["ms"]), 3),
             "unit": "chunks/s", "ms_per_step": round(b1["ms"], 3), "prefill_ms_p50": round(b1["prefill_ms_p50"], 3),
             "denoise_ms_p50": round(b1["denoise_ms_p50"], 3), "denoise_ms_p90": round(b1["denoise_ms_p90"], 3),
+            # the latency-bound loop scales with the SM clock: its time in millions of SM cycles at the
+            # median clock sampled during this measurement, comparable across boxes and power states
+            "denoise_mcycles_p50": round(b1["denoise_ms_p50"] * b1_mhz / 1000.0, 2) if b1_mhz else None,
+            "clocks": b1["clocks"],
             "gpu_launches": b1["launches"],
             "denoise_roofline": {"bound": "hbm",
                                  "kernel": "denoise_persistent_kernel (the 10-step Euler loop, one launch)",

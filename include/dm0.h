@@ -98,7 +98,18 @@ typedef enum {
  * per-layer KV cache for max_batch x max_prefix, activation buffers and the
  * RoPE table (built on the device).  *out receives the context.  Nothing is
  * allocated afterwards except CUDA-graph instantiations (one per distinct
- * (B, P, steps) of dm0_denoise). */
+ * (B, P, steps) of dm0_denoise).
+ * Environment switches read here (scheduling only: none changes what is
+ * computed, and every one keeps its default when unset):
+ *   DM0_NO_PDL=1         no programmatic dependent launch between kernels
+ *   DM0_NO_GRAPH=1       batched Euler loops as direct launches, no CUDA graph
+ *   DM0_NO_PERSIST=1     one observation's Euler loop as per-layer kernels
+ *   DM0_PERSIST_SPLITS=n attention key splits per KV head of that loop (7)
+ *   DM0_PERSIST_FASTBAR=0  its grid barriers with full fences (see dm0_denoise)
+ *   DM0_RASTER_BAND=n    persistent-GEMM tile bands of n m-tiles (default: n-fastest
+ *                        for weights up to 64 MB, 64-m-tile bands above)
+ *   DM0_QKV_EPI=8        the QKV GEMM epilogue on eight warps instead of four
+ *   DM0_PERSIST_TRACE=1, DM0_GEMM_TRACE=1  timestamp buffers (dm0_debug_view) */
 dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out);
 
 /* Weight blob size in bytes for `cfg`. */
