@@ -34,14 +34,14 @@ METRIC = "action chunks/sec (prefill+10-step denoise) at batch 1 and 16; HBM GB/
 EULER_STEPS = 10
 # DRAM bytes (read + write) of one prefix-pass gate/up GEMM launch at B=16, P=2048 (M=32768,
 # N=12288, K=2048), from an ncu capture of the same kernel and launch shape in `bench.py --one-layer`
-# on the current build (n-fastest raster): 0.417 GB read + 0.381 GB written, against 0.587 GB
-# algorithmic (activations 134 MB + weights 50 MB read, SwiGLU output 403 MB written)
+# on the current build (n-fastest raster, eight epilogue warps): 0.439 GB read + 0.379 GB written,
+# against 0.587 GB algorithmic (activations 134 MB + weights 50 MB read, SwiGLU output 403 MB written)
 COUNTERS_CURRENT = True
-GATEUP_TRAFFIC_BYTES = 0.7987e9
+GATEUP_TRAFFIC_BYTES = 0.8182e9
 # DRAM bytes (read + write) of the persistent Euler loop per step of 28 action layers at B=1, P=816:
-# the ncu capture of `bench.py --b1-loop` (3 layers, 1 step: 104.80 MB read + 4.71 MB written)
+# the ncu capture of `bench.py --b1-loop` (3 layers, 1 step: 104.80 MB read + 3.57 MB written)
 # scaled by 28/3
-LOOP_TRAFFIC_BYTES_PER_STEP = 1.0221e9
+LOOP_TRAFFIC_BYTES_PER_STEP = 1.0114e9
 
 
 def _peaks():
