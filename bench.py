@@ -854,6 +854,62 @@ def run_gemm_trace(args):
     eng.close()
 
 
+def summarize_attn_trace(arr, nblk):
+    """Per-block medians over the CTAs of the suffix attention's trace ([CTA][block][4] %globaltimer:
+    S seen, max exchanged, P announced, S issued by the MMA warp), in us: the softmax's wait for S
+    after announcing the previous P, its S -> max-exchange and max-exchange -> P times, the period
+    between consecutive P announcements, and how long before the softmax sees S the MMA warp issued it."""
+    import numpy as np
+    a = arr[:, :nblk, :].astype(np.float64)
+    ok = np.all(a[:, :, :4] > 0, axis=(1, 2))
+    a = a[ok]
+    if not len(a):   # no CTA of the traced instance ran (small batches use the two-CTAs-per-SM instance)
+        return {"ctas": 0, "blocks": nblk}
+    med = lambda x: round(float(np.median(x)) / 1e3, 3)   # noqa: E731
+    return {"ctas": int(ok.sum()), "blocks": nblk,
+            "wait_for_s": med(a[:, 1:, 0] - a[:, :-1, 2]),
+            "s_to_max": med(a[:, :, 1] - a[:, :, 0]),
+            "max_to_p": med(a[:, :, 2] - a[:, :, 1]),
+            "period": med(a[:, 1:, 2] - a[:, :-1, 2]),
+            "s_issue_lead": med(a[:, :, 0] - a[:, :, 3]),
+            "first_s_seen": med(a[:, 0, 0] - a[:, 0, 3].min()),
+            "walk_us": med(a[:, -1, 2] - a[:, 0, 0])}
+
+
+def run_attn_trace(args):
+    """Profiling workload: the one-layer context of --one-layer (B=16, P=2048 by default) with the
+    suffix attention stamping %globaltimer per CTA and 64-key block (DM0_ATTN_TRACE=1 set here);
+    prints summarize_attn_trace of the last Euler step's launch."""
+    os.environ["DM0_ATTN_TRACE"] = "1"
+    os.environ["DM0_NO_GRAPH"] = "1"
+    import numpy as np
+    import torch
+
+    from synth import inputs as I
+    from vla_dual_expert_b200 import Engine
+    d = I.DM0_BASE.replace(layers=1)
+    B, P = args.batch or 16, args.prefix or 2048
+    eng = Engine(d, B, P)
+    eng.load_from(I.Weights(d, seed=0))
+    emb = torch.from_numpy(I.prefix_embeddings(d, B, P)).cuda().to(torch.bfloat16)
+    noise = torch.from_numpy(I.noise(d, B)).cuda()
+    for _ in range(2):
+        eng.prefill(emb)
+        eng.denoise(noise, 1)
+    eng.sync()
+    torch.cuda.synchronize()
+    ctas = B * d.n_kv
+    nblk = (P + 63) // 64 + (d.chunk + 63) // 64
+    slots = 1024 * 64 * 4
+    ptr = eng.debug_view("attn_trace")
+    view = type("Trace", (), {"__cuda_array_interface__": {"shape": (slots,), "typestr": "<u8",
+                                                            "data": (ptr, False), "version": 3}})()
+    arr = torch.as_tensor(view, device="cuda").cpu().numpy().reshape(1024, 64, 4)[:ctas]
+    print(json.dumps({"attn_trace": "ok", "batch": B, "prefix": P,
+                      "blocks_us": summarize_attn_trace(arr, min(nblk, 64))}))
+    eng.close()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -872,6 +928,8 @@ def main():
     ap.add_argument("--b1-trace", action="store_true",
                     help="profiling workload: per-phase timeline of the single-launch Euler loop")
     ap.add_argument("--trace-layers", type=int, default=28)
+    ap.add_argument("--attn-trace", action="store_true",
+                    help="profiling workload: per-block timeline of the merged suffix attention of one layer")
     ap.add_argument("--gemm-trace", action="store_true",
                     help="profiling workload: per-CTA timeline of every persistent GEMM of one layer")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
@@ -903,6 +961,9 @@ def main():
         return
     if args.gemm_trace:
         run_gemm_trace(args)
+        return
+    if args.attn_trace:
+        run_attn_trace(args)
         return
     run_native(args, rank, world, local_rank)
 

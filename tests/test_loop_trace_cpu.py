@@ -66,3 +66,21 @@ def test_gemm_trace_summary():
     assert a["setup"] == 2.5               # median over CTAs of (1 us + their 0..3 us delay)
     assert a["last_done"] == 8.0           # one-tile CTAs count their first tile: 6, 7, 9, 10
     assert (b["ctas"], b["span_us"], b["exit"]) == (1, 18.0, 18.0)
+
+
+def test_attn_trace_summary():
+    """bench.summarize_attn_trace on a synthetic trace: every CTA announces P of block j at 2 us j +
+    1.6 us, sees S 0.5 us after the MMA warp issued it, and exchanges the max 0.4 us later; a CTA with a
+    missing stamp is left out."""
+    arr = np.zeros((5, 64, 4), dtype=np.uint64)
+    for c in range(4):
+        for j in range(10):
+            base = 1_000_000 + 100 * c + 2000 * j
+            arr[c, j] = [base + 500, base + 900, base + 1600, base]
+    arr[4, :10] = 7
+    arr[4, 3, 2] = 0
+    out = bench.summarize_attn_trace(arr, 10)
+    assert out["ctas"] == 4
+    assert (out["period"], out["wait_for_s"], out["s_to_max"], out["max_to_p"], out["s_issue_lead"]) == \
+        (2.0, 0.9, 0.4, 0.7, 0.5)
+    assert out["walk_us"] == 19.1

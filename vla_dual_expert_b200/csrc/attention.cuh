@@ -41,7 +41,12 @@ struct AttnArgs {
   // tcgen05 kernel, unsplit launches only (null: off): per query row, at the row's place in o
   // ([B][seq_q][n_q]), the base-2 log-sum-exp m + log2(l) of its scaled scores (p = 2^(s * scale_log2 - lse))
   float* lse;
+  // tcgen05 kernel, two-threads-per-row instance (null: off): per CTA (blockIdx linear, x fastest) and
+  // 64-key block j < kAttnTraceBlocks, %globaltimer at [0] S_j seen by the softmax, [1] the row max
+  // exchanged, [2] P_j written and announced, [3] the MMA warp's S_j issued
+  unsigned long long* trace;
 };
+constexpr int kAttnTraceBlocks = 64;
 
 constexpr int kAttnThreads = 256;
 

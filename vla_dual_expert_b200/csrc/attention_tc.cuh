@@ -132,6 +132,10 @@ __global__ void __launch_bounds__(FaWarps<NP>::kThreads, NP == 1 ? 2 : 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tile = blockIdx.x, grp = blockIdx.y;
+  const size_t cta_lin = (static_cast<size_t>(blockIdx.z) * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+  auto amark = [&](int j, int k) {
+    if (a.trace && j < kAttnTraceBlocks) a.trace[(cta_lin * kAttnTraceBlocks + j) * 4 + k] = globaltimer();
+  };
   const int b = grp / a.n_kv, kvh = grp - b * a.n_kv;
   const int G = a.n_q / a.n_kv;
   const int rows_total = G * a.seq_q;
@@ -264,6 +268,7 @@ __global__ void __launch_bounds__(FaWarps<NP>::kThreads, NP == 1 ? 2 : 1)
           umma_bf16(tmem + s * 64, sw128_kmajor_desc(qa + (ks >> 2) * 16384 + (ks & 3) * 32),
                     sw128_kmajor_desc(kb + (ks >> 2) * FS::kHalfKV + (ks & 3) * 32), idesc_s, ks > 0 ? 1u : 0u);
         umma_commit(&s_full[s]);
+        amark(j, 3);
         umma_commit(&k_empty[kvs]);
         if (j >= 1 && !pv(j - 1)) {
           ok = false;
@@ -317,6 +322,7 @@ __global__ void __launch_bounds__(FaWarps<NP>::kThreads, NP == 1 ? 2 : 1)
     for (int j = 0; j < nblk; ++j) {
       const int s = j & 1;
       bool good = *abort_flag == 0 && warp_wait(&s_full[s], (j >> 1) & 1);
+      if (threadIdx.x == 64) amark(j, 0);
       tc_fence_after();
       const int jj = jb0 + j;
       const int nvalid = jj < nA ? min(64, a.len_a - jj * 64) : min(64, a.len_b - (jj - nA) * 64);
@@ -336,6 +342,7 @@ __global__ void __launch_bounds__(FaWarps<NP>::kThreads, NP == 1 ? 2 : 1)
       }
       xm[((j & 1) * 2 + half) * 128 + r] = mx;
       named_bar_sync(1, kSM);
+      if (threadIdx.x == 64) amark(j, 1);
       mx = fmaxf(mx, xm[((j & 1) * 2 + (half ^ 1)) * 128 + r]);
       const float m_blk = mx * a.scale_log2;
       const bool move = m_blk > m_ref + 8.f;        // also true on the first block
@@ -391,6 +398,7 @@ __global__ void __launch_bounds__(FaWarps<NP>::kThreads, NP == 1 ? 2 : 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[j % NP]);
+      if (threadIdx.x == 64) amark(j, 2);
     }
     if (nblk > 0) {
       xl[half * 128 + r] = l_run;

@@ -146,6 +146,7 @@ struct dm0_ctx {
   dm0::PdLayer* players = nullptr;
   unsigned long long* ptrace = nullptr;   // DM0_PERSIST_TRACE=1: phase timestamps of the persistent loop
   unsigned long long* gtrace = nullptr;   // DM0_GEMM_TRACE=1: [kGemmTraceLaunches][num_sms][16] GEMM marks
+  unsigned long long* atrace = nullptr;   // DM0_ATTN_TRACE=1: suffix-attention block marks (last launch)
   int gtrace_next = 0;                     // next launch slot (round robin)
   int ptrace_steps = 0;
   // FP8 E4M3 prefix MLP (dm0_set_prefix_fp8): per VLM layer the gate/up (interleaved as the bf16
@@ -581,6 +582,7 @@ dm0_status run_attn(dm0_ctx* c, cudaStream_t s, const bf16* q, int seq_q, const 
                     tkb, tvb, a);
     // merged suffix attention: the cached prefix is read from DRAM once; deeper K/V prefetch and
     // two P buffers so the softmax runs ahead of the PV MMAs
+    if (static_cast<size_t>(groups) * tiles * fs <= kPartSlots) a.trace = c->atrace;
     return launch(c, s, dm0::fa_tc_kernel<dm0::kFaDeepStages, 2>, grid, dim3(dm0::FaWarps<2>::kThreads),
                   dm0::FaSmemT<dm0::kFaDeepStages, 2>::kBytes, tk, tv, tkb, tvb, a);
   }
@@ -1370,6 +1372,9 @@ dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
   A(dalloc(c, &c->psync, 2 + g.n_kv));
   A(dalloc(c, &c->pkv_sfx, static_cast<size_t>(g.n_kv) * 2 * 64 * 128));
   A(dalloc(c, &c->players, g.layers));
+  if (const char* e = std::getenv("DM0_ATTN_TRACE")) {
+    if (e[0] == '1') A(dalloc(c, &c->atrace, static_cast<size_t>(kPartSlots) * dm0::kAttnTraceBlocks * 4));
+  }
   if (const char* e = std::getenv("DM0_GEMM_TRACE")) {
     if (e[0] == '1')
       A(dalloc(c, &c->gtrace, static_cast<size_t>(kGemmTraceLaunches) * c->num_sms * dm0::kGemmTraceSlots));
@@ -1703,7 +1708,7 @@ dm0_status dm0_debug_view(dm0_ctx* c, const char* name, void** ptr) {
       {"h_v", c->h_v},     {"xn_v", c->xn_v},   {"q_v", c->q_v},     {"o_v", c->o_v},     {"act_v", c->act_v},
       {"ssq_v", c->ssq_v}, {"h_a", c->h_a},     {"xn_a", c->xn_a},   {"q_a", c->q_a},     {"o_a", c->o_a},
       {"act_a", c->act_a}, {"ssq_a", c->ssq_a}, {"x", c->x},         {"k_s", c->k_s},     {"v_s", c->v_s},
-      {"loop_trace", c->ptrace}, {"gemm_trace", c->gtrace}, {"tm_mod", c->tm_mod}, {"tm_bqkv", c->tm_bqkv}, {"tm_bgu", c->tm_bgu}};
+      {"loop_trace", c->ptrace}, {"gemm_trace", c->gtrace}, {"attn_trace", c->atrace}, {"tm_mod", c->tm_mod}, {"tm_bqkv", c->tm_bqkv}, {"tm_bgu", c->tm_bgu}};
   auto it = bufs.find(name);
   if (it == bufs.end()) return fail(c, DM0_EINVAL, std::string("unknown buffer ") + name);
   *ptr = it->second;
