@@ -717,7 +717,8 @@ TRACE_PHASES = ("qkv", "attention", "o_proj", "gate_up", "down")
 def summarize_loop_trace(arr, layers, items):
     """Per phase type, medians over the CTAs (the attention phase: its first `items` CTAs) and the layer
     passes, in microseconds from the phase's start: staged (operand in shared memory), copies (the operand
-    copies in flight), acc_ready (first accumulator or S tile), issued (results out), arrived (this CTA's
+    copies in flight), to_copies (from the start until the copies are issued), build (from the copies'
+    landing until the operand is staged), acc_ready (first accumulator or S tile), issued (results out), arrived (this CTA's
     barrier arrival); and the phase's wall time (the latest start of the next phase minus its own latest
     start) and last_arrival (the latest arrival minus the latest start).  arr: [rows][CTAs][TRACE_SLOTS]
     ns; row 0 is the first input, then per Euler step 5 rows per layer and one step boundary."""
@@ -731,6 +732,7 @@ def summarize_loop_trace(arr, layers, items):
         a = arr[q, :items] if name == "attention" else arr[q]
         st = a[:, 0]
         rec = {"staged": np.median(a[:, 1] - st), "copies": np.median(a[:, 9] - a[:, 8]),
+               "to_copies": np.median(a[:, 8] - st), "build": np.median(a[:, 1] - a[:, 9]),
                "acc_ready": np.median(a[:, 2] - st), "issued": np.median(a[:, 3] - st),
                "arrived": np.median(a[:, 5] - st),
                "phase": float(arr[q + 1, :, 0].max() - arr[q, :, 0].max()),
@@ -780,6 +782,8 @@ def run_b1_trace(args):
                                                             "data": (ptr, False), "version": 3}})()
     arr = torch.as_tensor(view, device="cuda").cpu().numpy().reshape(rows, nsm, TRACE_SLOTS)
     arr = arr.astype(np.float64) - float(arr[0, :, 0].min())
+    if args.trace_out:
+        np.save(args.trace_out, arr)
     splits = min(int(os.environ.get("DM0_PERSIST_SPLITS", "7")), 8)
     nblk = (P + 63) // 64 + 1
     bps = -(-nblk // min(splits, nblk))
@@ -928,6 +932,7 @@ def main():
     ap.add_argument("--b1-trace", action="store_true",
                     help="profiling workload: per-phase timeline of the single-launch Euler loop")
     ap.add_argument("--trace-layers", type=int, default=28)
+    ap.add_argument("--trace-out", default="", help="--b1-trace: also save the raw [rows][CTAs][slots] ns array (.npy)")
     ap.add_argument("--attn-trace", action="store_true",
                     help="profiling workload: per-block timeline of the merged suffix attention of one layer")
     ap.add_argument("--gemm-trace", action="store_true",

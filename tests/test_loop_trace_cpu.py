@@ -32,6 +32,8 @@ def test_summary_medians_and_phase_time():
     q = out["qkv"]
     assert (q["staged"], q["acc_ready"], q["issued"], q["arrived"]) == (1.0, 2.0, 3.0, 4.0)
     assert abs(q["copies"] - 0.2) < 1e-9
+    assert abs(q["to_copies"] - 0.5) < 1e-9      # copies issued 0.5 us after the start
+    assert abs(q["build"] - 0.3) < 1e-9          # landed at +0.7, staged at +1.0
     assert abs(q["phase"] - 10.0) < 1e-9          # latest start to the next phase's latest start
     assert abs(q["last_arrival"] - 4.0) < 1e-9    # the latest CTA also starts latest
     a = out["attention"]                           # only the two item CTAs, which run 2x slower

@@ -59,7 +59,9 @@ constexpr int kPdMaxSplits = 8;    // attention key splits per KV head
 // ready, 3 results issued, 4 after the release fence, 5 barrier arrival, 6 MMA warp saw the
 // operand, 7 MMA warp issued its last MMA of the phase
 // 8 operand copies issued, 9 copies landed; attention: 10 / 12 S of block 0 / 1 read, 11 / 13 P of
-// block 0 / 1 written, 14 O readout, 15 MMA warp issued PV of block 0
+// block 0 / 1 written, 14 O readout, 15 MMA warp issued PV of block 0; GEMM phases, in SM cycles
+// (clock64) for finer steps than %globaltimer's: 12 phase start, 13 staging entered, 15 copies issued,
+// 11 copies landed, 14 first pair's operand built, 10 staging done
 constexpr int kPdTraceSlots = 16;
 
 struct PdSmem {
@@ -85,9 +87,6 @@ struct PdSmem {
   static_assert(kOffLandA + 65536 <= kOffWork + kWork, "attention landing area overflows the work area");
 };
 
-struct PdLayer {
-  const float *attn_norm, *q_norm, *k_norm, *mlp_norm;
-};
 
 struct PdArgs {
   int L, T, P, steps;       // layers, tokens (<= 64), prefix length, Euler steps
@@ -95,7 +94,10 @@ struct PdArgs {
   int QR;                   // (n_q + 2 n_kv) * 128
   float eps, scale_log2;
   int splits, bps;          // attention: key splits per KV head, 64-key blocks per split
-  const PdLayer* layers;    // [L]
+  // RMSNorm gains of layer l: attn_norm0 + l norm_stride (and likewise q / k / mlp); computed, not
+  // loaded, so no gain address waits on a load after a grid barrier
+  const float *attn_norm0, *q_norm0, *k_norm0, *mlp_norm0;
+  int norm_stride;          // floats between consecutive layers' gains
   const float2* rope;       // [position][64] (cos, sin)
   float* h;                 // [T][Ha] residual stream
   float* acc_qkv;           // [T][QR]  zero at launch
@@ -131,9 +133,34 @@ __device__ __forceinline__ void pd_geom(const PdArgs& a, int ph, int& tiles, int
     tiles = a.Ha >> 7, nkb = a.Ia >> 6, rows_pl = a.Ha;
   }
 }
-__device__ __forceinline__ void pd_range(int total, int c, int n, int& p0, int& p1) {
+__host__ __device__ __forceinline__ void pd_range(int total, int c, int n, int& p0, int& p1) {
   p0 = static_cast<int>(static_cast<long long>(total) * c / n);
   p1 = static_cast<int>(static_cast<long long>(total) * (c + 1) / n);
+}
+// The (weight tile, k-block) pairs of one GEMM phase for CTA c of n.  With at least as many CTAs as
+// tiles, every tile gets floor(n / tiles) or one more CTAs, which split its k-blocks evenly: no CTA
+// straddles two tiles, so each adds one output segment (a CTA with two segments finished about
+// 1 us after the rest and held every CTA at the grid barrier).  Fewer CTAs than tiles: an even
+// contiguous split of all pairs.
+__host__ __device__ __forceinline__ void pd_pairs(int tiles, int nkb, int c, int n, int& p0, int& p1) {
+  if (n < tiles) {
+    pd_range(tiles * nkb, c, n, p0, p1);
+    return;
+  }
+  const int base = n / tiles, extra = n - base * tiles;   // the first `extra` tiles get base + 1 CTAs
+  int t, j, m;
+  if (c < extra * (base + 1)) {
+    m = base + 1;
+    t = c / m;
+    j = c - t * m;
+  } else {
+    const int c2 = c - extra * (base + 1);
+    m = base;
+    t = extra + c2 / m;
+    j = c2 - (t - extra) * m;
+  }
+  p0 = t * nkb + nkb * j / m;
+  p1 = t * nkb + nkb * (j + 1) / m;
 }
 // byte offset of 16-byte chunk c16 of row `row` in a SW128 K-major tile (128-byte rows, 1024-aligned base)
 __device__ __forceinline__ uint32_t sw_chunk(int row, int c16) {
@@ -168,7 +195,8 @@ __device__ __forceinline__ void pd_pair_ready(uint64_t* btf, int i, int ct) {
   if ((ct & 31) == 0) mbar_arrive(&btf[i]);
 }
 
-// Operand staging, one function per phase type, kept out of line.  Thread 0 of the compute group
+// Operand staging, one function per phase type, inlined (as out-of-line calls, the 10-step loop of
+// one observation took 6 % longer).  Thread 0 of the compute group
 // requests the phase's L2 data with a few TMA tensor / bulk copies into a shared-memory landing
 // area (after a proxy fence: other CTAs wrote that data through the generic proxy) and every
 // compute thread waits on the stage mbarrier; the operand is then built from shared memory.  A
@@ -203,7 +231,7 @@ __device__ __forceinline__ void pd_stage_wait(uint64_t* sbar, uint32_t par, vola
 
 // (A, D) bf16(g * h) for pairs [p0, p0 + np); weight tile 0 also adds sum h^2 into ssq
 template <int kT>
-__device__ __noinline__ uint32_t pd_stage_norm(const PdArgs& a, uint8_t* smem, int ct, int p0, int np, int nkb,
+__device__ __forceinline__ uint32_t pd_stage_norm(const PdArgs& a, uint8_t* smem, int ct, int p0, int np, int nkb,
                                                const float* gain, float* ssq, unsigned long long* mk, uint64_t* btf,
                                                uint64_t* sbar, uint32_t par, const CUtensorMap* map_h,
                                                volatile int* abort_flag) {
@@ -213,6 +241,7 @@ __device__ __noinline__ uint32_t pd_stage_norm(const PdArgs& a, uint8_t* smem, i
   float* land = reinterpret_cast<float*>(smem + SM::kOffLandG);   // [np][T][64]
   float* sg = reinterpret_cast<float*>(smem + SM::kOffAux);       // [np][64]
   if (ct == 0) {
+    if (mk) mk[13] = clock64();
     fence_proxy_async_global();
     mbar_arrive_expect_tx(sbar, np * (T * 256 + 256));
     int kb = p0 % nkb;
@@ -221,10 +250,12 @@ __device__ __noinline__ uint32_t pd_stage_norm(const PdArgs& a, uint8_t* smem, i
       bulk_load(sg + i * 64, gain + kb * 64, 256, sbar);
       if (++kb == nkb) kb = 0;
     }
+    if (mk) mk[15] = clock64();
     if (mk) mk[8] = globaltimer();
   }
   pd_stage_wait(sbar, par, abort_flag);
   if (mk && ct == 0) mk[9] = globaltimer();
+  if (mk && ct == 0) mk[11] = clock64();
   const int tile0_pairs = p0 < nkb ? min(np, nkb - p0) : 0;   // pairs of weight tile 0 add to ssq
   for (int i = 0; i < np; ++i) {
     for (int base = 0; base < T * 8; base += kPdCompute) {   // validity is uniform over each 8-lane group
@@ -248,8 +279,10 @@ __device__ __noinline__ uint32_t pd_stage_norm(const PdArgs& a, uint8_t* smem, i
         if (t < T && c8 == 0) atomicAdd(ssq + t, ss);
       }
     }
+    if (mk && ct == 0 && i == 0) mk[14] = clock64();
     pd_pair_ready(btf, i, ct);
   }
+  if (mk && ct == 0) mk[10] = clock64();
   return par ^ 1u;
 }
 
@@ -258,7 +291,7 @@ __device__ __noinline__ uint32_t pd_stage_norm(const PdArgs& a, uint8_t* smem, i
 // map_po: partial O as [slot][128 rows][128 dims] bf16, box {64 dims, T rows, S slots}; map_ml: (max, sum)
 // as [slot][128 rows] 8-byte elements, box {T rows, S slots}: one copy each per staged pair
 template <int kT>
-__device__ __noinline__ uint32_t pd_stage_attn_out(const PdArgs& a, uint8_t* smem, int ct, int p0, int np, int nkb,
+__device__ __forceinline__ uint32_t pd_stage_attn_out(const PdArgs& a, uint8_t* smem, int ct, int p0, int np, int nkb,
                                                    unsigned long long* mk, uint64_t* btf, uint64_t* sbar,
                                                    uint32_t par, const CUtensorMap* map_po, const CUtensorMap* map_ml,
                                                    volatile int* abort_flag) {
@@ -272,6 +305,7 @@ __device__ __noinline__ uint32_t pd_stage_attn_out(const PdArgs& a, uint8_t* sme
   float2* lml = reinterpret_cast<float2*>(lo + static_cast<size_t>(nrows) * 64);   // [np][mls]: [S][T] used
   float* wts = reinterpret_cast<float*>(lml + np * mls);                          // [np][S][T]
   if (ct == 0) {
+    if (mk) mk[13] = clock64();
     fence_proxy_async_global();
     mbar_arrive_expect_tx(sbar, nrows * (128 + 8));
     int kb = p0 % nkb;
@@ -281,10 +315,12 @@ __device__ __noinline__ uint32_t pd_stage_attn_out(const PdArgs& a, uint8_t* sme
       tma_load_2d_plain(lml + i * mls, map_ml, sbar, hh * T, g2 * S);
       if (++kb == nkb) kb = 0;
     }
+    if (mk) mk[15] = clock64();
     if (mk) mk[8] = globaltimer();
   }
   pd_stage_wait(sbar, par, abort_flag);
   if (mk && ct == 0) mk[9] = globaltimer();
+  if (mk && ct == 0) mk[11] = clock64();
   for (int q = ct; q < np * T; q += kPdCompute) {   // normalised split weights of each (pair, token)
     const int i = q / T, t = q - i * T;
     float mx = -__int_as_float(0x7f800000);
@@ -317,15 +353,17 @@ __device__ __noinline__ uint32_t pd_stage_attn_out(const PdArgs& a, uint8_t* sme
       }
       *reinterpret_cast<uint4*>(smem + SM::kOffWork + i * SM::kBTile + sw_chunk(t, c8)) = pack8(acc);
     }
+    if (mk && ct == 0 && i == 0) mk[14] = clock64();
     pd_pair_ready(btf, i, ct);
   }
+  if (mk && ct == 0) mk[10] = clock64();
   return par ^ 1u;
 }
 
 // (E) SwiGLU of the gate/up sums with 1/rms of the MLP norm (kMod: plus the feature bias `bias`, the
 // modulated norm's shift through the gate/up weights, in the interleaved column order)
 template <int kT, bool kMod = false>
-__device__ __noinline__ uint32_t pd_stage_swiglu(const PdArgs& a, uint8_t* smem, int ct, int p0, int np, int nkb,
+__device__ __forceinline__ uint32_t pd_stage_swiglu(const PdArgs& a, uint8_t* smem, int ct, int p0, int np, int nkb,
                                                  unsigned long long* mk, uint64_t* btf, uint64_t* sbar, uint32_t par,
                                                  const CUtensorMap* map_gu, volatile int* abort_flag,
                                                  const float* bias = nullptr) {
@@ -336,6 +374,7 @@ __device__ __noinline__ uint32_t pd_stage_swiglu(const PdArgs& a, uint8_t* smem,
   float* land = reinterpret_cast<float*>(smem + SM::kOffLandG);   // [np][T][128]: gate 64 | up 64
   float* sq = reinterpret_cast<float*>(smem + SM::kOffAux);       // [2T] both sums of squares
   if (ct == 0) {
+    if (mk) mk[13] = clock64();
     fence_proxy_async_global();
     mbar_arrive_expect_tx(sbar, np * T * 512 + 8 * T);
     int kb = p0 % nkb;
@@ -344,10 +383,12 @@ __device__ __noinline__ uint32_t pd_stage_swiglu(const PdArgs& a, uint8_t* smem,
       if (++kb == nkb) kb = 0;
     }
     bulk_load(sq, a.ssq, 8 * T, sbar);
+    if (mk) mk[15] = clock64();
     if (mk) mk[8] = globaltimer();
   }
   pd_stage_wait(sbar, par, abort_flag);
   if (mk && ct == 0) mk[9] = globaltimer();
+  if (mk && ct == 0) mk[11] = clock64();
   for (int i = 0; i < np; ++i) {
     for (int u = ct; u < T * 8; u += kPdCompute) {
       const int t = u >> 3;
@@ -367,8 +408,10 @@ __device__ __noinline__ uint32_t pd_stage_swiglu(const PdArgs& a, uint8_t* smem,
       }
       *reinterpret_cast<uint4*>(smem + SM::kOffWork + i * SM::kBTile + sw_chunk(t, c8)) = pack8(y);
     }
+    if (mk && ct == 0 && i == 0) mk[14] = clock64();
     pd_pair_ready(btf, i, ct);
   }
+  if (mk && ct == 0) mk[10] = clock64();
   return par ^ 1u;
 }
 
@@ -380,7 +423,7 @@ __device__ __noinline__ uint32_t pd_stage_swiglu(const PdArgs& a, uint8_t* smem,
 // kMod: the sums first become acc / rms + bias (`bias` = this step's and layer's shift through the QKV
 // weights), and the head RMSNorm is taken over that.
 template <int kT, bool kMod = false>
-__device__ __noinline__ uint32_t pd_stage_qkv(const PdArgs& a, uint8_t* smem, int ct, int l, int kvg, bool kv,
+__device__ __forceinline__ uint32_t pd_stage_qkv(const PdArgs& a, uint8_t* smem, int ct, int l, int kvg, bool kv,
                                               __nv_bfloat16* kv_out, unsigned long long* mk, uint64_t* sbar,
                                               uint32_t par, const CUtensorMap* map_qkv, volatile int* abort_flag,
                                               const float* bias = nullptr) {
@@ -397,7 +440,6 @@ __device__ __noinline__ uint32_t pd_stage_qkv(const PdArgs& a, uint8_t* smem, in
   float* sgk = reinterpret_cast<float*>(smem + SM::kOffP + 768);      // [128]
   float2* srope = reinterpret_cast<float2*>(smem + SM::kOffP + 1280); // [T][64] (cos, sin) at P + t
   if (ct == 0) {
-    const PdLayer& ly = a.layers[l];
     const uint32_t sq_bytes = (4 * T + 15) & ~15u;
     fence_proxy_async_global();
     mbar_arrive_expect_tx(sbar, (kv ? 2 : G) * T * 512 + T * 512 + 1024 + sq_bytes);
@@ -409,8 +451,8 @@ __device__ __noinline__ uint32_t pd_stage_qkv(const PdArgs& a, uint8_t* smem, in
         tma_load_2d_plain(land + w * 64 * 128, map_qkv, sbar, qd + w * kvd + kvg * 128, 0);
     }
     bulk_load(srope, a.rope + static_cast<size_t>(a.P) * 64, T * 512, sbar);
-    bulk_load(sgq, ly.q_norm, 512, sbar);
-    bulk_load(sgk, ly.k_norm, 512, sbar);
+    bulk_load(sgq, a.q_norm0 + static_cast<size_t>(l) * a.norm_stride, 512, sbar);
+    bulk_load(sgk, a.k_norm0 + static_cast<size_t>(l) * a.norm_stride, 512, sbar);
     bulk_load(sq, a.ssq, sq_bytes, sbar);
     if (mk) mk[8] = globaltimer();
   }
@@ -669,7 +711,7 @@ __global__ void __launch_bounds__(kPdThreads, 1)
             }
             int tiles, nkb, rpl, p0, p1;
             pd_geom(a, ph, tiles, nkb, rpl);
-            pd_range(tiles * nkb, blockIdx.x, gridDim.x, p0, p1);
+            pd_pairs(tiles, nkb, blockIdx.x, gridDim.x, p0, p1);
             const CUtensorMap* m = ph == 0 ? &tmQKV : (ph == 2 ? &tmO : (ph == 3 ? &tmGU : &tmD));
             for (int p = p0; p < p1; ++p) {
               const int st = acquire(rs);
@@ -793,7 +835,7 @@ __global__ void __launch_bounds__(kPdThreads, 1)
             }
             int tiles, nkb, rpl, p0, p1;
             pd_geom(a, ph, tiles, nkb, rpl);
-            pd_range(tiles * nkb, blockIdx.x, gridDim.x, p0, p1);
+            pd_pairs(tiles, nkb, blockIdx.x, gridDim.x, p0, p1);
             if (p0 >= p1) continue;
             int seg = 0, seg_start = p0, cur_tile = p0 / nkb, kbc = p0 - cur_tile * nkb;
             for (int p = p0; p < p1; ++p) {
@@ -1092,9 +1134,10 @@ __global__ void __launch_bounds__(kPdThreads, 1)
     ok = grid_sync();
     for (int k = 0; ok && k < a.steps; ++k) {
       for (int l = 0; ok && l < a.L; ++l) {
-        const PdLayer& ly = a.layers[l];
         for (int ph = 0; ok && ph < 5; ++ph) {
           mark(0);
+          if (ph != 1 && a.trace && ct == 0)
+            a.trace[(static_cast<size_t>(gen) * gridDim.x + blockIdx.x) * kPdTraceSlots + 12] = clock64();
           if (ph == 1) {
             if (has_item && !attention(l, k)) *abort_flag = 1;
             if (kv_helper) {
@@ -1113,12 +1156,12 @@ __global__ void __launch_bounds__(kPdThreads, 1)
           }
           int tiles, nkb, rpl, p0, p1;
           pd_geom(a, ph, tiles, nkb, rpl);
-          pd_range(tiles * nkb, blockIdx.x, gridDim.x, p0, p1);
+          pd_pairs(tiles, nkb, blockIdx.x, gridDim.x, p0, p1);
           const int np = p1 - p0;
           if (np > 0) {
             // kMod: the norms' gains are this step's 1 + scale rows
-            const float* g_attn = kMod ? mod_row(k, l) : ly.attn_norm;
-            const float* g_mlp = kMod ? mod_row(k, l) + 3 * a.Ha : ly.mlp_norm;
+            const float* g_attn = kMod ? mod_row(k, l) : a.attn_norm0 + static_cast<size_t>(l) * a.norm_stride;
+            const float* g_mlp = kMod ? mod_row(k, l) + 3 * a.Ha : a.mlp_norm0 + static_cast<size_t>(l) * a.norm_stride;
             if (ph == 0) stage_par = PD_STAGE(pd_stage_norm, a, smem, ct, p0, np, nkb, g_attn, ssq_attn, mk_row(), btile_full, stage_bar, stage_par, &tmHLd, abort_flag);
             else if (ph == 2) stage_par = PD_STAGE(pd_stage_attn_out, a, smem, ct, p0, np, nkb, mk_row(), btile_full, stage_bar, stage_par, &tmPO, &tmML, abort_flag);
             else if (ph == 3) stage_par = PD_STAGE(pd_stage_norm, a, smem, ct, p0, np, nkb, g_mlp, ssq_mlp, mk_row(), btile_full, stage_bar, stage_par, &tmHLd, abort_flag);

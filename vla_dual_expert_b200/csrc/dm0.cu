@@ -143,7 +143,6 @@ struct dm0_ctx {
   float *pacc_qkv = nullptr, *pacc_gu = nullptr, *pssq = nullptr;
   unsigned* psync = nullptr;   // [0] barrier, [1] abort, [2 + g] suffix K/V flags
   bf16* pkv_sfx = nullptr;      // [n_kv][2][64][128] suffix K/V tiles built by the helper CTAs
-  dm0::PdLayer* players = nullptr;
   unsigned long long* ptrace = nullptr;   // DM0_PERSIST_TRACE=1: phase timestamps of the persistent loop
   unsigned long long* gtrace = nullptr;   // DM0_GEMM_TRACE=1: [kGemmTraceLaunches][num_sms][16] GEMM marks
   unsigned long long* atrace = nullptr;   // DM0_ATTN_TRACE=1: suffix-attention block marks (last launch)
@@ -933,7 +932,12 @@ bool persist_plan(dm0_ctx* c, int steps, float* vel, dm0::PdArgs* a, std::string
                          {g.inter_a / 64, g.hidden_a / 64},
                          {g.hidden_a / 128, g.inter_a / 64}};
   for (int ph = 0; ph < 4; ++ph) {
-    const int per = (geo[ph][0] * geo[ph][1] + nsm - 1) / nsm;
+    int per = 0;   // the longest pair range of the kernel's split (dm0::pd_pairs)
+    for (int cc = 0; cc < nsm; ++cc) {
+      int q0, q1;
+      dm0::pd_pairs(geo[ph][0], geo[ph][1], cc, nsm, q0, q1);
+      per = std::max(per, q1 - q0);
+    }
     if (per > dm0::kPdBTiles || per > geo[ph][1]) return no("GEMM ranges too long for the staging area");
     if (per * land_per[ph] > static_cast<long>(dm0::PdSmem::kLandG)) return no("operand copies exceed the landing area");
   }
@@ -953,7 +957,20 @@ bool persist_plan(dm0_ctx* c, int steps, float* vel, dm0::PdArgs* a, std::string
   a->scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(g.head_dim)));
   a->splits = splits;
   a->bps = bps;
-  a->layers = c->players;
+  {
+    // the gains sit at one stride per layer in the weight buffer (see the weight layout in dm0_create)
+    const LayerW* w = c->lw[1];
+    const ptrdiff_t stride = g.layers > 1 ? w[1].attn_norm - w[0].attn_norm : 0;
+    for (int l = 0; l < g.layers; ++l)
+      if (w[l].attn_norm != w[0].attn_norm + l * stride || w[l].q_norm != w[0].q_norm + l * stride ||
+          w[l].k_norm != w[0].k_norm + l * stride || w[l].mlp_norm != w[0].mlp_norm + l * stride)
+        return no("layer gains not evenly strided");
+    a->attn_norm0 = w[0].attn_norm;
+    a->q_norm0 = w[0].q_norm;
+    a->k_norm0 = w[0].k_norm;
+    a->mlp_norm0 = w[0].mlp_norm;
+    a->norm_stride = static_cast<int>(stride);
+  }
   a->rope = c->rope;
   a->h = c->h_a;
   a->acc_qkv = c->pacc_qkv;
@@ -1371,7 +1388,6 @@ dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
   A(dalloc(c, &c->pssq, 128));
   A(dalloc(c, &c->psync, 2 + g.n_kv));
   A(dalloc(c, &c->pkv_sfx, static_cast<size_t>(g.n_kv) * 2 * 64 * 128));
-  A(dalloc(c, &c->players, g.layers));
   if (const char* e = std::getenv("DM0_ATTN_TRACE")) {
     if (e[0] == '1') A(dalloc(c, &c->atrace, static_cast<size_t>(kPartSlots) * dm0::kAttnTraceBlocks * 4));
   }
@@ -1386,15 +1402,6 @@ dm0_status dm0_create(const dm0_config* cfg, dm0_ctx** out) {
     }
   }
   if (st != DM0_OK) return bail(st);
-  {
-    std::vector<dm0::PdLayer> pl(g.layers);
-    for (int l = 0; l < g.layers; ++l) {
-      const LayerW& w = c->lw[1][l];
-      pl[l] = dm0::PdLayer{w.attn_norm, w.q_norm, w.k_norm, w.mlp_norm};
-    }
-    if (cudaMemcpy(c->players, pl.data(), pl.size() * sizeof(dm0::PdLayer), cudaMemcpyHostToDevice) != cudaSuccess)
-      return bail(DM0_ECUDA);
-  }
   if (cudaMemset(c->acc, 0, c->acc_elems * 4) != cudaSuccess || cudaMemset(c->gcount, 0, 1024 * 4) != cudaSuccess ||
       cudaMemset(c->acount, 0, c->acount_n * 4) != cudaSuccess || cudaMemset(c->d_err, 0, 4) != cudaSuccess)
     return bail(DM0_ECUDA);
