@@ -232,27 +232,13 @@ __device__ __forceinline__ void pd_stage_wait(uint64_t* sbar, uint32_t par, vola
 // (A, D) bf16(g * h) for pairs [p0, p0 + np); weight tile 0 also adds sum h^2 into ssq
 template <int kT>
 __device__ __forceinline__ uint32_t pd_stage_norm(const PdArgs& a, uint8_t* smem, int ct, int p0, int np, int nkb,
-                                               const float* gain, float* ssq, unsigned long long* mk, uint64_t* btf,
-                                               uint64_t* sbar, uint32_t par, const CUtensorMap* map_h,
-                                               volatile int* abort_flag) {
+                                                  float* ssq, unsigned long long* mk, uint64_t* btf, uint64_t* sbar,
+                                                  uint32_t par, volatile int* abort_flag) {
   using SM = PdSmem;
   const int T = kT > 0 ? kT : a.T;   // tokens; a compile-time constant for the common shape
   const int c8 = ct & 7;
   float* land = reinterpret_cast<float*>(smem + SM::kOffLandG);   // [np][T][64]
   float* sg = reinterpret_cast<float*>(smem + SM::kOffAux);       // [np][64]
-  if (ct == 0) {
-    if (mk) mk[13] = clock64();
-    fence_proxy_async_global();
-    mbar_arrive_expect_tx(sbar, np * (T * 256 + 256));
-    int kb = p0 % nkb;
-    for (int i = 0; i < np; ++i) {
-      tma_load_2d_plain(land + i * T * 64, map_h, sbar, kb * 64, 0);
-      bulk_load(sg + i * 64, gain + kb * 64, 256, sbar);
-      if (++kb == nkb) kb = 0;
-    }
-    if (mk) mk[15] = clock64();
-    if (mk) mk[8] = globaltimer();
-  }
   pd_stage_wait(sbar, par, abort_flag);
   if (mk && ct == 0) mk[9] = globaltimer();
   if (mk && ct == 0) mk[11] = clock64();
@@ -291,33 +277,18 @@ __device__ __forceinline__ uint32_t pd_stage_norm(const PdArgs& a, uint8_t* smem
 // map_po: partial O as [slot][128 rows][128 dims] bf16, box {64 dims, T rows, S slots}; map_ml: (max, sum)
 // as [slot][128 rows] 8-byte elements, box {T rows, S slots}: one copy each per staged pair
 template <int kT>
-__device__ __forceinline__ uint32_t pd_stage_attn_out(const PdArgs& a, uint8_t* smem, int ct, int p0, int np, int nkb,
-                                                   unsigned long long* mk, uint64_t* btf, uint64_t* sbar,
-                                                   uint32_t par, const CUtensorMap* map_po, const CUtensorMap* map_ml,
-                                                   volatile int* abort_flag) {
+__device__ __forceinline__ uint32_t pd_stage_attn_out(const PdArgs& a, uint8_t* smem, int ct, int np,
+                                                      unsigned long long* mk, uint64_t* btf, uint64_t* sbar,
+                                                      uint32_t par, volatile int* abort_flag) {
   using SM = PdSmem;
   const int T = kT > 0 ? kT : a.T;   // tokens; a compile-time constant for the common shape
   const int c8 = ct & 7;
-  const int G = a.n_q / a.n_kv, S = a.splits;
+  const int S = a.splits;
   const int nrows = np * S * T;
   const int mls = (S * T + 15) & ~15;   // (max, sum) entries per pair, padded to 128 bytes
   __nv_bfloat16* lo = reinterpret_cast<__nv_bfloat16*>(smem + SM::kOffLandG);   // [np][S][T][64]
   float2* lml = reinterpret_cast<float2*>(lo + static_cast<size_t>(nrows) * 64);   // [np][mls]: [S][T] used
   float* wts = reinterpret_cast<float*>(lml + np * mls);                          // [np][S][T]
-  if (ct == 0) {
-    if (mk) mk[13] = clock64();
-    fence_proxy_async_global();
-    mbar_arrive_expect_tx(sbar, nrows * (128 + 8));
-    int kb = p0 % nkb;
-    for (int i = 0; i < np; ++i) {
-      const int hq = kb >> 1, g2 = hq / G, hh = hq - g2 * G;   // slots g2 S .. g2 S + S - 1, rows hh T ..
-      tma_load_3d_plain(lo + static_cast<size_t>(i) * S * T * 64, map_po, sbar, (kb & 1) * 64, hh * T, g2 * S);
-      tma_load_2d_plain(lml + i * mls, map_ml, sbar, hh * T, g2 * S);
-      if (++kb == nkb) kb = 0;
-    }
-    if (mk) mk[15] = clock64();
-    if (mk) mk[8] = globaltimer();
-  }
   pd_stage_wait(sbar, par, abort_flag);
   if (mk && ct == 0) mk[9] = globaltimer();
   if (mk && ct == 0) mk[11] = clock64();
@@ -364,28 +335,14 @@ __device__ __forceinline__ uint32_t pd_stage_attn_out(const PdArgs& a, uint8_t* 
 // modulated norm's shift through the gate/up weights, in the interleaved column order)
 template <int kT, bool kMod = false>
 __device__ __forceinline__ uint32_t pd_stage_swiglu(const PdArgs& a, uint8_t* smem, int ct, int p0, int np, int nkb,
-                                                 unsigned long long* mk, uint64_t* btf, uint64_t* sbar, uint32_t par,
-                                                 const CUtensorMap* map_gu, volatile int* abort_flag,
-                                                 const float* bias = nullptr) {
+                                                    unsigned long long* mk, uint64_t* btf, uint64_t* sbar, uint32_t par,
+                                                    volatile int* abort_flag, const float* bias = nullptr) {
   using SM = PdSmem;
   const int T = kT > 0 ? kT : a.T;   // tokens; a compile-time constant for the common shape
   const int c8 = ct & 7;
   const float inv_Ha = 1.0f / a.Ha;
   float* land = reinterpret_cast<float*>(smem + SM::kOffLandG);   // [np][T][128]: gate 64 | up 64
   float* sq = reinterpret_cast<float*>(smem + SM::kOffAux);       // [2T] both sums of squares
-  if (ct == 0) {
-    if (mk) mk[13] = clock64();
-    fence_proxy_async_global();
-    mbar_arrive_expect_tx(sbar, np * T * 512 + 8 * T);
-    int kb = p0 % nkb;
-    for (int i = 0; i < np; ++i) {
-      tma_load_2d_plain(land + i * T * 128, map_gu, sbar, 128 * kb, 0);
-      if (++kb == nkb) kb = 0;
-    }
-    bulk_load(sq, a.ssq, 8 * T, sbar);
-    if (mk) mk[15] = clock64();
-    if (mk) mk[8] = globaltimer();
-  }
   pd_stage_wait(sbar, par, abort_flag);
   if (mk && ct == 0) mk[9] = globaltimer();
   if (mk && ct == 0) mk[11] = clock64();
@@ -423,10 +380,9 @@ __device__ __forceinline__ uint32_t pd_stage_swiglu(const PdArgs& a, uint8_t* sm
 // kMod: the sums first become acc / rms + bias (`bias` = this step's and layer's shift through the QKV
 // weights), and the head RMSNorm is taken over that.
 template <int kT, bool kMod = false>
-__device__ __forceinline__ uint32_t pd_stage_qkv(const PdArgs& a, uint8_t* smem, int ct, int l, int kvg, bool kv,
-                                              __nv_bfloat16* kv_out, unsigned long long* mk, uint64_t* sbar,
-                                              uint32_t par, const CUtensorMap* map_qkv, volatile int* abort_flag,
-                                              const float* bias = nullptr) {
+__device__ __forceinline__ uint32_t pd_stage_qkv(const PdArgs& a, uint8_t* smem, int ct, int kvg, bool kv,
+                                                 __nv_bfloat16* kv_out, unsigned long long* mk, uint64_t* sbar,
+                                                 uint32_t par, volatile int* abort_flag, const float* bias = nullptr) {
   using SM = PdSmem;
   const int T = kT > 0 ? kT : a.T;   // tokens; a compile-time constant for the common shape
   const int c8 = ct & 7;
@@ -439,23 +395,6 @@ __device__ __forceinline__ uint32_t pd_stage_qkv(const PdArgs& a, uint8_t* smem,
   float* sgq = reinterpret_cast<float*>(smem + SM::kOffP + 256);      // [128]
   float* sgk = reinterpret_cast<float*>(smem + SM::kOffP + 768);      // [128]
   float2* srope = reinterpret_cast<float2*>(smem + SM::kOffP + 1280); // [T][64] (cos, sin) at P + t
-  if (ct == 0) {
-    const uint32_t sq_bytes = (4 * T + 15) & ~15u;
-    fence_proxy_async_global();
-    mbar_arrive_expect_tx(sbar, (kv ? 2 : G) * T * 512 + T * 512 + 1024 + sq_bytes);
-    if (!kv) {
-      for (int r = 0; r < G; ++r)   // head r of the group: rows r T .. r T + T - 1
-        tma_load_2d_plain(land + r * T * 128, map_qkv, sbar, (kvg * G + r) * 128, 0);
-    } else {
-      for (int w = 0; w < 2; ++w)   // K rows at 0.., V rows at 64..
-        tma_load_2d_plain(land + w * 64 * 128, map_qkv, sbar, qd + w * kvd + kvg * 128, 0);
-    }
-    bulk_load(srope, a.rope + static_cast<size_t>(a.P) * 64, T * 512, sbar);
-    bulk_load(sgq, a.q_norm0 + static_cast<size_t>(l) * a.norm_stride, 512, sbar);
-    bulk_load(sgk, a.k_norm0 + static_cast<size_t>(l) * a.norm_stride, 512, sbar);
-    bulk_load(sq, a.ssq, sq_bytes, sbar);
-    if (mk) mk[8] = globaltimer();
-  }
   pd_stage_wait(sbar, par, abort_flag);
   if (mk && ct == 0) mk[9] = globaltimer();
 #pragma unroll 1
@@ -558,6 +497,99 @@ __device__ __noinline__ void pd_step(const PdArgs& a, int k_out, int k_in, int c
 
 // the 50-token chunk of one observation gets staging code with the token count folded in; the value
 // is the stage barrier's next parity
+// The operand copies of phase ph of layer l, Euler step k, for this CTA: issued by compute thread 0
+// inside the grid barrier that precedes the phase, as soon as its spin ends and before the other
+// compute threads are released, so the copies fly while they leave the barrier.  Each staging
+// function above waits for exactly these bytes.  pr: this CTA's pair range [p0, p1) per phase; role
+// of the attention phase: 1 an attention item of KV head kvg, 2 the suffix K/V helper of head kvg,
+// 0 nothing to stage.  Returns whether copies were issued.  The landing areas are free: every
+// compute thread passed the barrier's CTA-wide named barrier, and the previous phase's MMAs and
+// bulk reductions completed before it.
+template <bool kMod>
+__device__ __forceinline__ bool pd_issue(const PdArgs& a, uint8_t* smem, int k, int l, int ph, const int* pr, int role,
+                                         int kvg, uint64_t* sbar, const CUtensorMap* map_h, const CUtensorMap* map_po,
+                                         const CUtensorMap* map_ml, const CUtensorMap* map_gu,
+                                         const CUtensorMap* map_qkv, unsigned long long* mk) {
+  using SM = PdSmem;
+  const int T = a.T;
+  if (mk) mk[13] = clock64();
+  if (ph == 1) {
+    if (role == 0) return false;
+    const bool kv = role == 2;
+    const int G = a.n_q / a.n_kv;
+    const int qd = a.n_q * 128, kvd = a.n_kv * 128;
+    float* land = reinterpret_cast<float*>(smem + SM::kOffLandA);
+    float* sq = reinterpret_cast<float*>(smem + SM::kOffP);
+    float* sgq = reinterpret_cast<float*>(smem + SM::kOffP + 256);
+    float* sgk = reinterpret_cast<float*>(smem + SM::kOffP + 768);
+    float2* srope = reinterpret_cast<float2*>(smem + SM::kOffP + 1280);
+    const uint32_t sq_bytes = (4 * T + 15) & ~15u;
+    fence_proxy_async_global();
+    mbar_arrive_expect_tx(sbar, (kv ? 2 : G) * T * 512 + T * 512 + 1024 + sq_bytes);
+    if (!kv) {
+      for (int r = 0; r < G; ++r)   // head r of the group: rows r T .. r T + T - 1
+        tma_load_2d_plain(land + r * T * 128, map_qkv, sbar, (kvg * G + r) * 128, 0);
+    } else {
+      for (int w = 0; w < 2; ++w)   // K rows at 0.., V rows at 64..
+        tma_load_2d_plain(land + w * 64 * 128, map_qkv, sbar, qd + w * kvd + kvg * 128, 0);
+    }
+    bulk_load(srope, a.rope + static_cast<size_t>(a.P) * 64, T * 512, sbar);
+    bulk_load(sgq, a.q_norm0 + static_cast<size_t>(l) * a.norm_stride, 512, sbar);
+    bulk_load(sgk, a.k_norm0 + static_cast<size_t>(l) * a.norm_stride, 512, sbar);
+    bulk_load(sq, a.ssq, sq_bytes, sbar);
+  } else {
+    const int p0 = pr[2 * ph], np = pr[2 * ph + 1] - p0;
+    if (np <= 0) return false;
+    int tiles, nkb, rpl;
+    pd_geom(a, ph, tiles, nkb, rpl);
+    int kb = p0 % nkb;
+    fence_proxy_async_global();
+    if (ph == 0 || ph == 3) {   // h rows and the norm's gains (kMod: this step's 1 + scale rows)
+      const float* gain;
+      if constexpr (kMod) {
+        gain = a.tm_mod + static_cast<size_t>(k) * a.tm_R + 6 * l * a.Ha + (ph == 0 ? 0 : 3 * a.Ha);
+      } else {
+        gain = (ph == 0 ? a.attn_norm0 : a.mlp_norm0) + static_cast<size_t>(l) * a.norm_stride;
+      }
+      float* land = reinterpret_cast<float*>(smem + SM::kOffLandG);   // [np][T][64]
+      float* sg = reinterpret_cast<float*>(smem + SM::kOffAux);       // [np][64]
+      mbar_arrive_expect_tx(sbar, np * (T * 256 + 256));
+      for (int i = 0; i < np; ++i) {
+        tma_load_2d_plain(land + i * T * 64, map_h, sbar, kb * 64, 0);
+        bulk_load(sg + i * 64, gain + kb * 64, 256, sbar);
+        if (++kb == nkb) kb = 0;
+      }
+    } else if (ph == 2) {       // the key splits' partial O and (max, sum) rows
+      const int G = a.n_q / a.n_kv, S = a.splits;
+      const int nrows = np * S * T;
+      const int mls = (S * T + 15) & ~15;
+      __nv_bfloat16* lo = reinterpret_cast<__nv_bfloat16*>(smem + SM::kOffLandG);
+      float2* lml = reinterpret_cast<float2*>(lo + static_cast<size_t>(nrows) * 64);
+      mbar_arrive_expect_tx(sbar, nrows * (128 + 8));
+      for (int i = 0; i < np; ++i) {
+        const int hq = kb >> 1, g2 = hq / G, hh = hq - g2 * G;   // slots g2 S .. g2 S + S - 1, rows hh T ..
+        tma_load_3d_plain(lo + static_cast<size_t>(i) * S * T * 64, map_po, sbar, (kb & 1) * 64, hh * T, g2 * S);
+        tma_load_2d_plain(lml + i * mls, map_ml, sbar, hh * T, g2 * S);
+        if (++kb == nkb) kb = 0;
+      }
+    } else {                    // the gate / up sums and both sums of squares
+      float* land = reinterpret_cast<float*>(smem + SM::kOffLandG);   // [np][T][128]
+      float* sq = reinterpret_cast<float*>(smem + SM::kOffAux);
+      mbar_arrive_expect_tx(sbar, np * T * 512 + 8 * T);
+      for (int i = 0; i < np; ++i) {
+        tma_load_2d_plain(land + i * T * 128, map_gu, sbar, 128 * kb, 0);
+        if (++kb == nkb) kb = 0;
+      }
+      bulk_load(sq, a.ssq, 8 * T, sbar);
+    }
+  }
+  if (mk) {
+    mk[15] = clock64();
+    mk[8] = globaltimer();
+  }
+  return true;
+}
+
 #define PD_STAGE(fn, ...) (a.T == 50 ? fn<50>(__VA_ARGS__) : fn<0>(__VA_ARGS__))
 #define PD_STAGE_M(fn, ...) (a.T == 50 ? fn<50, kMod>(__VA_ARGS__) : fn<0, kMod>(__VA_ARGS__))
 
@@ -601,6 +633,7 @@ __global__ void __launch_bounds__(kPdThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* sx = reinterpret_cast<float*>(smem + SM::kOffMisc);   // [64]
   float* sred = sx + 64;                                        // [8]
+  int* pr = reinterpret_cast<int*>(smem + SM::kOffMisc + 320);  // [5 phases][p0, p1]: this CTA's GEMM pairs
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = a.n_q / a.n_kv;
@@ -639,6 +672,12 @@ __global__ void __launch_bounds__(kPdThreads, 1)
     mbar_init(kvs_ready, 1);
     *abort_flag = 0;
     fence_mbar_init();
+    for (int ph = 0; ph < 5; ++ph) {   // once per launch: the split-K division of every GEMM phase
+      int tiles, nkb, rpl;
+      pd_geom(a, ph, tiles, nkb, rpl);
+      if (ph == 1) pr[2] = pr[3] = 0;
+      else pd_pairs(tiles, nkb, blockIdx.x, gridDim.x, pr[2 * ph], pr[2 * ph + 1]);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 256);
@@ -711,7 +750,7 @@ __global__ void __launch_bounds__(kPdThreads, 1)
             }
             int tiles, nkb, rpl, p0, p1;
             pd_geom(a, ph, tiles, nkb, rpl);
-            pd_pairs(tiles, nkb, blockIdx.x, gridDim.x, p0, p1);
+            p0 = pr[2 * ph], p1 = pr[2 * ph + 1];
             const CUtensorMap* m = ph == 0 ? &tmQKV : (ph == 2 ? &tmO : (ph == 3 ? &tmGU : &tmD));
             for (int p = p0; p < p1; ++p) {
               const int st = acquire(rs);
@@ -835,7 +874,7 @@ __global__ void __launch_bounds__(kPdThreads, 1)
             }
             int tiles, nkb, rpl, p0, p1;
             pd_geom(a, ph, tiles, nkb, rpl);
-            pd_pairs(tiles, nkb, blockIdx.x, gridDim.x, p0, p1);
+            p0 = pr[2 * ph], p1 = pr[2 * ph + 1];
             if (p0 >= p1) continue;
             int seg = 0, seg_start = p0, cur_tile = p0 / nkb, kbc = p0 - cur_tile * nkb;
             for (int p = p0; p < p1; ++p) {
@@ -911,7 +950,13 @@ __global__ void __launch_bounds__(kPdThreads, 1)
     // Every compute thread calls this after every phase, whatever happened in it, so the named
     // barriers always see all 256 threads; the result is the CTA abort flag, read after the last
     // named barrier (the same value in every thread).
-    auto grid_sync = [&]() -> bool {
+    // role of this CTA in the attention phase for the operand copies: 1 item, 2 suffix K/V helper, 0 none
+    const int att_role = has_item ? 1 : (kv_helper ? 2 : 0);
+    const int att_kvg = has_item ? kvg : (kv_helper ? static_cast<int>(blockIdx.x) - n_items : 0);
+    bool stage_pending = false;   // thread 0: copies issued that no staging function has waited for yet
+    // (nk, nl, nph): the phase that follows the barrier, whose operand copies thread 0 issues as soon as
+    // its spin ends; nph < 0: none (the step phase, or the end)
+    auto grid_sync = [&](int nk, int nl, int nph) -> bool {
       named_bar_sync(1, kPdCompute);
       ++gen;
       if (ct == 0 && *abort_flag == 0) {
@@ -935,6 +980,9 @@ __global__ void __launch_bounds__(kPdThreads, 1)
           }
         }
         if (!a.fast_bar) __threadfence();   // else: the acquire load orders what follows, the CTA barrier below the rest
+        if (*abort_flag == 0 && nph >= 0)
+          stage_pending = pd_issue<kMod>(a, smem, nk, nl, nph, pr, att_role, att_kvg, stage_bar, &tmHLd, &tmPO, &tmML,
+                                         &tmGULd, &tmQKVLd, mk_row());
       }
       if (ct == 0 && *abort_flag) atomicExch(a.sync + 1, 1u);   // release the other CTAs at once
       named_bar_sync(1, kPdCompute);
@@ -1009,8 +1057,9 @@ __global__ void __launch_bounds__(kPdThreads, 1)
     // ---- attention of one (KV head, key split) item
     auto attention = [&](int l, int k) -> bool {
       const int GT = G * a.T;
-      stage_par = PD_STAGE_M(pd_stage_qkv, a, smem, ct, l, kvg, false, nullptr, mk_row(), stage_bar, stage_par,
-                             &tmQKVLd, abort_flag, qkv_bias(k, l));
+      stage_par = PD_STAGE_M(pd_stage_qkv, a, smem, ct, kvg, false, nullptr, mk_row(), stage_bar, stage_par, abort_flag,
+                             qkv_bias(k, l));
+      stage_pending = false;
       fence_async_smem();
       tc_fence_before();
       __syncwarp();
@@ -1131,7 +1180,7 @@ __global__ void __launch_bounds__(kPdThreads, 1)
     step_phase(-1, 0);
     zero_share(a.acc_qkv, a.T * a.QR);
     if (blockIdx.x == 0 && ct < 2 * a.T) a.ssq[ct] = 0.f;
-    ok = grid_sync();
+    ok = grid_sync(0, 0, a.steps > 0 && a.L > 0 ? 0 : -1);
     for (int k = 0; ok && k < a.steps; ++k) {
       for (int l = 0; ok && l < a.L; ++l) {
         for (int ph = 0; ok && ph < 5; ++ph) {
@@ -1142,8 +1191,9 @@ __global__ void __launch_bounds__(kPdThreads, 1)
             if (has_item && !attention(l, k)) *abort_flag = 1;
             if (kv_helper) {
               const int g = blockIdx.x - n_items;
-              stage_par = PD_STAGE_M(pd_stage_qkv, a, smem, ct, l, g, true, a.kv_sfx + static_cast<size_t>(g) * 16384,
-                                     mk_row(), stage_bar, stage_par, &tmQKVLd, abort_flag, qkv_bias(k, l));
+              stage_par = PD_STAGE_M(pd_stage_qkv, a, smem, ct, g, true, a.kv_sfx + static_cast<size_t>(g) * 16384,
+                                     mk_row(), stage_bar, stage_par, abort_flag, qkv_bias(k, l));
+              stage_pending = false;
               csync();
               if (ct == 0) {
                 __threadfence();
@@ -1151,22 +1201,20 @@ __global__ void __launch_bounds__(kPdThreads, 1)
               }
             }
             mark(3);
-            ok = grid_sync();
+            ok = grid_sync(k, l, 2);
             continue;
           }
           int tiles, nkb, rpl, p0, p1;
           pd_geom(a, ph, tiles, nkb, rpl);
-          pd_pairs(tiles, nkb, blockIdx.x, gridDim.x, p0, p1);
+          p0 = pr[2 * ph], p1 = pr[2 * ph + 1];
           const int np = p1 - p0;
-          if (np > 0) {
-            // kMod: the norms' gains are this step's 1 + scale rows
-            const float* g_attn = kMod ? mod_row(k, l) : a.attn_norm0 + static_cast<size_t>(l) * a.norm_stride;
-            const float* g_mlp = kMod ? mod_row(k, l) + 3 * a.Ha : a.mlp_norm0 + static_cast<size_t>(l) * a.norm_stride;
-            if (ph == 0) stage_par = PD_STAGE(pd_stage_norm, a, smem, ct, p0, np, nkb, g_attn, ssq_attn, mk_row(), btile_full, stage_bar, stage_par, &tmHLd, abort_flag);
-            else if (ph == 2) stage_par = PD_STAGE(pd_stage_attn_out, a, smem, ct, p0, np, nkb, mk_row(), btile_full, stage_bar, stage_par, &tmPO, &tmML, abort_flag);
-            else if (ph == 3) stage_par = PD_STAGE(pd_stage_norm, a, smem, ct, p0, np, nkb, g_mlp, ssq_mlp, mk_row(), btile_full, stage_bar, stage_par, &tmHLd, abort_flag);
-            else stage_par = PD_STAGE_M(pd_stage_swiglu, a, smem, ct, p0, np, nkb, mk_row(), btile_full, stage_bar, stage_par, &tmGULd, abort_flag,
+          if (np > 0) {   // the operand copies were issued inside the barrier before this phase
+            if (ph == 0) stage_par = PD_STAGE(pd_stage_norm, a, smem, ct, p0, np, nkb, ssq_attn, mk_row(), btile_full, stage_bar, stage_par, abort_flag);
+            else if (ph == 2) stage_par = PD_STAGE(pd_stage_attn_out, a, smem, ct, np, mk_row(), btile_full, stage_bar, stage_par, abort_flag);
+            else if (ph == 3) stage_par = PD_STAGE(pd_stage_norm, a, smem, ct, p0, np, nkb, ssq_mlp, mk_row(), btile_full, stage_bar, stage_par, abort_flag);
+            else stage_par = PD_STAGE_M(pd_stage_swiglu, a, smem, ct, p0, np, nkb, mk_row(), btile_full, stage_bar, stage_par, abort_flag,
                                         kMod ? a.tm_bgu + (static_cast<size_t>(l) * a.steps + k) * 2 * a.Ia : nullptr);
+            stage_pending = false;
             mark(1);
           }
           // scratch of the other half of the layer, idle in this phase
@@ -1183,20 +1231,25 @@ __global__ void __launch_bounds__(kPdThreads, 1)
             if (!reduce_out(p0, p1, nkb, map, gate)) *abort_flag = 1;
           }
           mark(3);
-          ok = grid_sync();
+          // next: the following phase of this layer, the next layer's QKV, or the step phase (no copies)
+          const bool last = ph == 4 && l + 1 == a.L;
+          ok = grid_sync(k, ph == 4 ? l + 1 : l, last ? -1 : (ph + 1) % 5);
         }
       }
       if (!ok) break;
       mark(0);
       step_phase(k, k + 1 < a.steps ? k + 1 : -1);
       mark(3);
-      if (k + 1 < a.steps) ok = grid_sync();
+      if (k + 1 < a.steps) ok = grid_sync(k + 1, 0, 0);
     }
     if (!ok) {
       *abort_flag = 1;
       raise_error(a.err, kErrTimeoutEpilogue);
       atomicExch(a.sync + 1, 1u);
     }
+    // operand copies issued for a phase that an abort skipped land before the CTA exits
+    if (ct == 0 && stage_pending && !mbar_wait(stage_bar, stage_par, nullptr, kDrainTimeoutNs))
+      raise_error(a.err, kErrDrain);
   }
   tc_fence_before();
   __syncthreads();
