@@ -39,9 +39,10 @@ EULER_STEPS = 10
 COUNTERS_CURRENT = True
 GATEUP_TRAFFIC_BYTES = 0.8182e9
 # DRAM bytes (read + write) of the persistent Euler loop per step of 28 action layers at B=1, P=816:
-# the ncu capture of `bench.py --b1-loop` (3 layers, 1 step: 104.80 MB read + 3.57 MB written)
-# scaled by 28/3
-LOOP_TRAFFIC_BYTES_PER_STEP = 1.0114e9
+# the ncu capture of `bench.py --b1-loop` (3 layers, 1 step: 104.81 MB read + 3.06 MB written)
+# scaled by 28/3; LOOP_COUNTERS_CURRENT is false while the kernel differs from the captured build
+LOOP_COUNTERS_CURRENT = True
+LOOP_TRAFFIC_BYTES_PER_STEP = 1.0068e9
 
 
 def _peaks():
@@ -352,7 +353,8 @@ def run_native(args, rank, world, local_rank):
                      "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
                      "peak_src": f"{peaks['src']} bf16_tflops_sustained", "launches": main["probe_n"],
                      "avg_launch_ms": round(gu_ms, 4)},
-        "e2e": {"value": round(job_chunks_per_s(world, B, e2e["ms"]), 3), "unit": "chunks/s",
+        "e2e": {"value": (round(job_chunks_per_s(world, B, e2e["ms"]), 3) if e2e["ms"] == e2e["ms"] else None),
+                "unit": "chunks/s",
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
         "gpu_launches": main["launches"],
         "clocks": main["clocks"],
@@ -378,7 +380,7 @@ def run_native(args, rank, world, local_rank):
                                  "achieved": round(den_gbs, 1), "peak": peaks["hbm_gbs"],
                                  "unit": "GB/s", "frac": round(den_gbs / peaks["hbm_gbs"], 4),
                                  "algorithmic_bytes_per_euler_step": denoise_bytes_per_step(d, 1, wl1.prefix),
-                                 "traffic_per_euler_step": LOOP_TRAFFIC_BYTES_PER_STEP if COUNTERS_CURRENT else None,
+                                 "traffic_per_euler_step": LOOP_TRAFFIC_BYTES_PER_STEP if LOOP_COUNTERS_CURRENT else None,
                                  "peak_src": f"{peaks['src']} hbm_gbs"},
         }
     if not args.skip_batch1:
