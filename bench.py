@@ -822,6 +822,15 @@ def summarize_gemm_trace(arr):
             v = last if name == "last_done" else r[:, i]
             ok = v > 0
             rec[name] = round(float(np.median(v[ok] - t0)) / 1e3, 2) if ok.any() else None
+        # QKV epilogue of the CTA's last tile, SM cycles (slots 10-13: group 0 entered, its first head's
+        # RMS pass done, that head's RoPE pass done, group 1 done)
+        c = r[:, 10:14]
+        okc = (c > 0).all(axis=1)
+        if okc.any():
+            cc = c[okc]
+            rec["qkv_epi_kcycles"] = {"rms_pass": round(float(np.median(cc[:, 1] - cc[:, 0])) / 1e3, 2),
+                                      "rope_pass": round(float(np.median(cc[:, 2] - cc[:, 1])) / 1e3, 2),
+                                      "tile": round(float(np.median(cc[:, 3] - cc[:, 0])) / 1e3, 2)}
         out.append(rec)
     return out
 

@@ -267,9 +267,11 @@ __device__ __forceinline__ void resid_epilogue_warp(const GemmArgs& a, int row0,
 
 // `nchunks` (4, or 2 for a 64-column tile) applies to the column-independent modes (residual, store);
 // QKV and SwiGLU always take a full 128-column group.
+// sgain (optional): the QK-norm gains [q | k], head_dim each, staged in shared memory by the caller;
+// null: read from global memory
 template <bool kFromScratch, class Load>
 __device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool valid, int col0,
-                                             Load&& load, int nchunks = 4) {
+                                             Load&& load, int nchunks = 4, const float* sgain = nullptr) {
   const int D = a.head_dim;
   if (a.mode == kModeStoreF32) {
 #pragma unroll 1
@@ -369,6 +371,14 @@ __device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool va
     return base + ((static_cast<size_t>(b) * a.n_kv + kvh) * a.kv_seq + p) * D + d;
   };
   const int cph = D >> 5;   // 32-column chunks per head
+  // trace (first epilogue thread, SM cycles): 10 first 128-column group entered, 11 its first head's
+  // RMS pass done, 12 that head's RoPE pass done, 13 the tile's second group done
+  const bool cmk = a.trace && threadIdx.x == 64;
+  const int grp = (col0 >> 7) & 1;
+  auto cmark = [&](int slot) {
+    if (cmk) const_cast<unsigned long long*>(a.trace)[blockIdx.x * kGemmTraceSlots + slot] = clock64();
+  };
+  if (grp == 0) cmark(10);
 #pragma unroll 1
   for (int h0 = 0; h0 < 4; h0 += cph) {
     const int colh = col0 + 32 * h0;
@@ -384,7 +394,7 @@ __device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool va
       }
       continue;
     }
-    const float* gain = colh < qdim ? a.q_gain : a.k_gain;
+    const float* gain = sgain ? (colh < qdim ? sgain : sgain + D) : (colh < qdim ? a.q_gain : a.k_gain);
     // pass 1: RMS of the head
     float ss = 0.f;
 #pragma unroll 1
@@ -395,6 +405,7 @@ __device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool va
       for (int j = 0; j < 32; ++j) ss += v[j] * v[j];
     }
     const float rn = s * rsqrtf(ss * s * s / D + a.eps);
+    if (grp == 0 && h0 == 0) cmark(11);
     if (D == 32) {
       // one chunk, pairs (j, j + 16)
       float v[32];
@@ -412,21 +423,20 @@ __device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool va
       // chunk c (head dims 32c'..) pairs with chunk c + cph/2
 #pragma unroll 1
       for (int c = 0; c < cph / 2; ++c) {
+        // the (cos, sin) of the chunk's 32 dimensions are requested before the accumulator loads, so
+        // the global loads' latency overlaps the TMEM loads
+        float2 cs[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) cs[j] = cs_col[static_cast<size_t>(32 * c + j) * a.rope_ld];
         float lo[32], hi[32];
         ld(h0 + c, lo);
         ld(h0 + c + cph / 2, hi);
 #pragma unroll
-        for (int jh = 0; jh < 2; ++jh) {   // (cos, sin) of 16 dimensions requested together, then used
-          float2 cs[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) cs[j] = cs_col[static_cast<size_t>(32 * c + 16 * jh + j) * a.rope_ld];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int jj = 16 * jh + j, d = 32 * c + jj;
-            const float x0 = lo[jj] * rn * gain[d], x1 = hi[jj] * rn * gain[d + half];
-            lo[jj] = x0 * cs[j].x - x1 * cs[j].y;
-            hi[jj] = x1 * cs[j].x + x0 * cs[j].y;
-          }
+        for (int jj = 0; jj < 32; ++jj) {
+          const int d = 32 * c + jj;
+          const float x0 = lo[jj] * rn * gain[d], x1 = hi[jj] * rn * gain[d + half];
+          lo[jj] = x0 * cs[jj].x - x1 * cs[jj].y;
+          hi[jj] = x1 * cs[jj].x + x0 * cs[jj].y;
         }
         if (valid) {
           st_bf16x32(dst_of(colh + 32 * c), lo);
@@ -434,7 +444,9 @@ __device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool va
         }
       }
     }
+    if (grp == 0 && h0 == 0) cmark(12);
   }
+  if (grp == 1) cmark(13);
 }
 
 template <int BN, int STAGES>
@@ -728,6 +740,14 @@ __global__ void __launch_bounds__(PGemmWarps<EPI>::kThreads, 1)
     tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();
   }
+  // QKV: the QK-norm gains (weights, which no kernel writes) staged once per launch in the epilogue
+  // scratch, which only the residual mode uses otherwise
+  float* sgain = a.mode == kModeQKV && a.q_gain && a.k_gain && 8 * a.head_dim <= static_cast<int>(EPI * L::kScrWarp)
+                     ? reinterpret_cast<float*>(smem + L::kOffScr)
+                     : nullptr;
+  if (sgain)
+    for (int i = threadIdx.x; i < 2 * a.head_dim; i += blockDim.x)
+      sgain[i] = i < a.head_dim ? a.q_gain[i] : a.k_gain[i - a.head_dim];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -892,7 +912,7 @@ __global__ void __launch_bounds__(PGemmWarps<EPI>::kThreads, 1)
                                 [&](int c, float (&v)[32]) { scaled(tg + c * 32, col0 + 32 * c, v); });
           } else {
             row_epilogue<false>(a, tok, valid, col0,
-                                [&](int c, float (&v)[32]) { scaled(tg + c * 32, col0 + 32 * c, v); }, ng);
+                                [&](int c, float (&v)[32]) { scaled(tg + c * 32, col0 + 32 * c, v); }, ng, sgain);
           }
         }
       } else if (BN == 256) {
@@ -913,7 +933,7 @@ __global__ void __launch_bounds__(PGemmWarps<EPI>::kThreads, 1)
                               [&](int c, float (&v)[32]) { scaled(tg + c * 32, col0 + 32 * c, v); });
         } else {
           row_epilogue<false>(a, tok, valid, col0,
-                              [&](int c, float (&v)[32]) { scaled(tg + c * 32, col0 + 32 * c, v); }, nch);
+                              [&](int c, float (&v)[32]) { scaled(tg + c * 32, col0 + 32 * c, v); }, nch, sgain);
         }
       }
       // the accumulator buffer is free for tile local + 2
