@@ -395,6 +395,13 @@ __device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool va
       continue;
     }
     const float* gain = sgain ? (colh < qdim ? sgain : sgain + D) : (colh < qdim ? a.q_gain : a.k_gain);
+    // the (cos, sin) of the first RoPE chunk's 32 dimensions, requested before the RMS pass so their
+    // latency overlaps its TMEM loads; each later chunk's are requested while the previous one is stored
+    float2 cs[32];
+    if (D > 32) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) cs[j] = cs_col[static_cast<size_t>(j) * a.rope_ld];
+    }
     // pass 1: RMS of the head
     float ss = 0.f;
 #pragma unroll 1
@@ -423,11 +430,6 @@ __device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool va
       // chunk c (head dims 32c'..) pairs with chunk c + cph/2
 #pragma unroll 1
       for (int c = 0; c < cph / 2; ++c) {
-        // the (cos, sin) of the chunk's 32 dimensions are requested before the accumulator loads, so
-        // the global loads' latency overlaps the TMEM loads
-        float2 cs[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) cs[j] = cs_col[static_cast<size_t>(32 * c + j) * a.rope_ld];
         float lo[32], hi[32];
         ld(h0 + c, lo);
         ld(h0 + c + cph / 2, hi);
@@ -437,6 +439,10 @@ __device__ __forceinline__ void row_epilogue(const GemmArgs& a, int tok, bool va
           const float x0 = lo[jj] * rn * gain[d], x1 = hi[jj] * rn * gain[d + half];
           lo[jj] = x0 * cs[jj].x - x1 * cs[jj].y;
           hi[jj] = x1 * cs[jj].x + x0 * cs[jj].y;
+        }
+        if (c + 1 < cph / 2) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) cs[j] = cs_col[static_cast<size_t>(32 * (c + 1) + j) * a.rope_ld];
         }
         if (valid) {
           st_bf16x32(dst_of(colh + 32 * c), lo);
