@@ -34,10 +34,11 @@ METRIC = "action chunks/sec (prefill+10-step denoise) at batch 1 and 16; HBM GB/
 EULER_STEPS = 10
 # DRAM bytes (read + write) of one prefix-pass gate/up GEMM launch at B=16, P=2048 (M=32768,
 # N=12288, K=2048), from an ncu capture of the same kernel and launch shape in `bench.py --one-layer`
-# on the current build (n-fastest raster, eight epilogue warps): 0.439 GB read + 0.379 GB written,
-# against 0.587 GB algorithmic (activations 134 MB + weights 50 MB read, SwiGLU output 403 MB written)
+# on the current build (n-fastest raster, eight epilogue warps): 0.665 GB read + 0.396 GB written,
+# against 0.587 GB algorithmic (activations 134 MB + weights 50 MB read, SwiGLU output 403 MB written);
+# the same code measured 0.439 + 0.379 GB on another box
 COUNTERS_CURRENT = True
-GATEUP_TRAFFIC_BYTES = 0.8182e9
+GATEUP_TRAFFIC_BYTES = 1.0602e9
 # DRAM bytes (read + write) of the persistent Euler loop per step of 28 action layers at B=1, P=816:
 # the ncu capture of `bench.py --b1-loop` (3 layers, 1 step: 104.81 MB read + 3.06 MB written)
 # scaled by 28/3; LOOP_COUNTERS_CURRENT is false while the kernel differs from the captured build
