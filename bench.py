@@ -720,7 +720,8 @@ TRACE_PHASES = ("qkv", "attention", "o_proj", "gate_up", "down")
 def summarize_loop_trace(arr, layers, items):
     """Per phase type, medians over the CTAs (the attention phase: its first `items` CTAs) and the layer
     passes, in microseconds from the phase's start: staged (operand in shared memory), copies (the operand
-    copies in flight), to_copies (from the start until the copies are issued), build (from the copies'
+    copies in flight), to_copies (from the start until the copies are issued: negative, since the
+    barrier's spinning thread issues them before it releases the phase), build (from the copies'
     landing until the operand is staged), acc_ready (first accumulator or S tile), issued (results out), arrived (this CTA's
     barrier arrival); and the phase's wall time (the latest start of the next phase minus its own latest
     start) and last_arrival (the latest arrival minus the latest start).  arr: [rows][CTAs][TRACE_SLOTS]
