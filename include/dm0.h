@@ -300,10 +300,15 @@ dm0_status dm0_op_attention(dm0_ctx* ctx, const void* q, const void* ka, const v
  * k_s/v_s bf16 [B][n_kv][chunk][head_dim].  Context-owned; contents are only
  * meaningful after the call that fills them has completed.
  * "loop_trace" (NULL unless DM0_PERSIST_TRACE=1 was set at dm0_create): u64
- * %globaltimer marks of the persistent Euler loop (runs of <= 16 steps),
- * [phase][CTA][8] = phase start, operand staged, first accumulator (or S tile)
- * ready, results issued, release fence done, barrier arrival, MMA warp saw the
- * operand, MMA warp issued its last MMA;
+ * marks of the persistent Euler loop (runs of <= 16 steps), [phase][CTA][16]:
+ * %globaltimer at 0 phase start, 1 operand staged, 2 first accumulator (or S
+ * tile) ready, 3 results issued, 4 release fence done, 5 barrier arrival, 6 MMA
+ * warp saw the operand, 7 MMA warp issued its last MMA, 8 operand copies issued
+ * (inside the preceding barrier), 9 copies landed; attention items: 10 / 12 S
+ * of key block 0 / 1 read, 11 / 13 its P written, 14 O read out, 15 first PV
+ * issued; GEMM phases, SM cycles (clock64): 12 phase start, 13 copies' issue
+ * entered, 15 copies issued, 11 copies landed, 14 first pair's operand built,
+ * 10 staging done;
  * phase 0 is the input of step 0, then per step 5 phases per layer (QKV,
  * attention, O, gate/up, down) and the step boundary.
  * "gemm_trace" (NULL unless DM0_GEMM_TRACE=1 was set at dm0_create): u64
@@ -311,9 +316,12 @@ dm0_status dm0_op_attention(dm0_ctx* ctx, const void* q, const void* ka, const v
  * launch order), [launch][CTA (num_sms rows)][16] = entry, setup done, past the
  * dependency wait, first k-block landed, first tile's MMAs issued, first
  * accumulator complete, first tile's epilogue done, last tile's epilogue done
- * (0 for one-tile CTAs), last TMA copy issued, exit; CTA 0's slots 14 and 15
- * hold (M << 32 | N) and (K << 32 | tile width); rows of CTAs that did not
- * run in a launch keep stale values.
+ * (0 for one-tile CTAs), last TMA copy issued, exit; QKV launches: slots 10-13
+ * SM cycles (clock64) of the first epilogue thread's last tile (first 128-column
+ * group entered, its first head's RMS pass done, that head's RoPE pass done,
+ * second group done); CTA 0's slots 14 and 15 hold (M << 32 | N) and
+ * (K << 32 | tile width); rows of CTAs that did not run in a launch keep stale
+ * values.
  * "tm_mod", "tm_bqkv", "tm_bgu" (time_mod contexts, NULL before the first
  * dm0_denoise or dm0_prepare): the modulation tables of the last Euler loop of
  * K steps, f32 [K][(6*layers + 2)*hidden_a] (per layer [attention: 1 + scale |
