@@ -29,9 +29,11 @@
 //   E  h[t][f] += sum_k Wd[f][k] * bf16(silu(gate / rms) * (up / rms))
 // and after layer L-1 the step boundary (velocity, Euler update, next input;
 // one CTA per token).  The GEMM work of a phase, (128-row weight tile, 64-wide
-// k-block) pairs in tile-major order, is cut into contiguous equal ranges, one
-// per CTA; a range covers at most two tiles, each accumulated in its own
-// 64-column TMEM segment.
+// k-block) pairs in tile-major order, is cut into contiguous ranges, one per
+// CTA, aligned to the weight tiles (pd_pairs) when there are at least as many
+// CTAs as tiles; a range covers at most two tiles, each accumulated in its own
+// 64-column TMEM segment.  The thread that spins on a grid barrier issues the
+// next phase's operand copies as soon as the barrier completes (pd_issue).
 //
 // Warp roles (320 threads): warp 0 TMA producer (weights, prefix K/V, the
 // suffix K/V from the helper), warp 1 TMEM owner and tcgen05.mma issuer (it

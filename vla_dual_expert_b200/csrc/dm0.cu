@@ -892,7 +892,8 @@ dm0_status enqueue_denoise(dm0_ctx* c, cudaStream_t s, int steps, float* vel) {
 
 // The persistent Euler loop covers one observation of the DM0-base shapes: head_dim 128, at most
 // 64 suffix tokens and 128 attention rows per KV head, 128-row weight tiles, and per GEMM phase at
-// most kPdBTiles pairs (and two weight tiles) per CTA.  Fills everything of `a` but the stream-time
+// most kPdBTiles pairs (and two weight tiles) per CTA under the kernel's split (dm0::pd_pairs).  Fills
+// everything of `a` but the stream-time
 // fields; false (with the reason) sends the loop to the per-layer kernels.
 bool persist_plan(dm0_ctx* c, int steps, float* vel, dm0::PdArgs* a, std::string* why) {
   const dm0_config& g = c->cfg;
