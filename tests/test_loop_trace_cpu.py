@@ -60,6 +60,11 @@ def test_gemm_trace_summary():
     arr[1, 0, :10] = [base + 50_000_000 + 2000 * m for m in range(10)]   # launch 1: one CTA
     arr[1, 0, 14] = (50 << 32) | 128
     arr[1, 0, 15] = (64 << 32) | 64
+    # QKV epilogue SM-cycle marks (slots 10-13) on launch 0: the RMS pass 1000 + 100 c cycles, the RoPE
+    # pass 5000, the tile 14000; CTA 3 has no marks (a V-only tile) and is left out of them
+    for c in range(3):
+        c0 = 1_000_000 * (c + 1)
+        arr[0, c, 10:14] = [c0, c0 + 1000 + 100 * c, c0 + 6000 + 100 * c, c0 + 14000]
     out = bench.summarize_gemm_trace(arr)
     assert len(out) == 2
     a, b = out
@@ -67,7 +72,9 @@ def test_gemm_trace_summary():
     assert a["span_us"] == 12.0            # last exit (CTA 3: +3 + 9 us) after the first entry
     assert a["setup"] == 2.5               # median over CTAs of (1 us + their 0..3 us delay)
     assert a["last_done"] == 8.0           # one-tile CTAs count their first tile: 6, 7, 9, 10
+    assert a["qkv_epi_kcycles"] == {"rms_pass": 1.1, "rope_pass": 5.0, "tile": 14.0}
     assert (b["ctas"], b["span_us"], b["exit"]) == (1, 18.0, 18.0)
+    assert "qkv_epi_kcycles" not in b
 
 
 def test_attn_trace_summary():
